@@ -1,0 +1,214 @@
+"""Plain fp64 CPU oracle for grouped / latent-KV attention (ctypes wrapper).
+
+TEST INFRASTRUCTURE, NOT PRODUCT CODE.  Only the test-suite, the smoke check
+and the benchmark's CPU-baseline leg may import this package.  The product
+library (``latent_kv_attention_b200``) never imports it and shares no code with
+it; the only thing both sides consume is the seeded inputs of ``synthetic.py``.
+
+The arithmetic lives in ``oracle.c`` (plain C, double precision, one output row
+at a time); this module only builds it with gcc, converts arrays to contiguous
+float64/int32 numpy arrays, calls it and returns numpy outputs.  See the header
+of ``oracle.c`` for the definitions, the pages they follow and the readings
+taken where the pages are silent.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so (gcc, -O2, pthreads). Returns the path."""
+    stale = (not os.path.exists(_LIB_PATH)) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)
+    if force or stale:
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread", "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def load_library(path: str):
+    """Open an oracle shared library and declare its C signatures."""
+    lib = ctypes.CDLL(path)
+    dp = ctypes.POINTER(ctypes.c_double)
+    ip = ctypes.POINTER(ctypes.c_int)
+    I, D = ctypes.c_int, ctypes.c_double
+    lib.oracle_gqa.argtypes = [dp, dp, dp, ip, I, I, I, I, I, I, I, D, dp, dp, ip, I, I]
+    lib.oracle_gqa_probs.argtypes = [dp, dp, ip, I, I, I, I, I, I, I, D, I, I, I, dp]
+    lat = [dp, dp, dp, dp, dp, ip, I, I, I, I, I, I, I, I, I, D, dp, dp, ip, I, I]
+    lib.oracle_latent_expanded.argtypes = lat
+    lib.oracle_latent_absorbed.argtypes = lat
+    lib.oracle_latent_expand_cache.argtypes = [dp, dp, dp, I, I, I, I, I, I, dp, dp, dp, I]
+    lib.oracle_gta.argtypes = [dp, dp, dp, ip, I, I, I, I, I, I, I, I, D, dp, dp, ip, I, I]
+    lib.oracle_merge_partials.argtypes = [dp, dp, I, I, dp, dp]
+    lib.oracle_threads_used.argtypes = [I, ctypes.c_long]
+    for f in ("oracle_gqa", "oracle_gqa_probs", "oracle_latent_expanded", "oracle_latent_absorbed",
+              "oracle_latent_expand_cache", "oracle_gta", "oracle_merge_partials", "oracle_threads_used"):
+        getattr(lib, f).restype = ctypes.c_int
+    return lib
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            _lib = load_library(_LIB_PATH)
+    return _lib
+
+
+def _f64(x) -> np.ndarray:
+    if hasattr(x, "detach"):  # torch tensor (any dtype, any device)
+        x = x.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _i32(x) -> np.ndarray:
+    if hasattr(x, "detach"):
+        x = x.detach().to("cpu").numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.int32))
+
+
+def _dp(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _ip(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int))
+
+
+def _rows(rows_b):
+    if rows_b is None:
+        return None, 0
+    r = _i32(rows_b)
+    return r, int(r.size)
+
+
+def _check(rc: int, name: str):
+    if rc != 0:
+        raise ValueError(f"{name}: invalid argument (oracle returned {rc})")
+
+
+def threads_used(n_threads: int, n_items: int) -> int:
+    """Threads the oracle's pool uses for n_items work items (0 = all online cores)."""
+    return int(_load().oracle_threads_used(int(n_threads), int(n_items)))
+
+
+def gqa(q, k, v, cache_lens, causal: bool, scale: float, rows_b=None, n_threads: int = 0):
+    """Grouped-query attention. q [B,h_q,s_q,d], k/v [B,h_kv,Lmax,d], cache_lens [B].
+
+    Returns (out [B,h_q,s_q,d], lse [B,h_q,s_q]) as float64 numpy arrays; with
+    ``rows_b`` only those batch rows are evaluated (the others stay NaN)."""
+    q, k, v, lens = _f64(q), _f64(k), _f64(v), _i32(cache_lens)
+    B, h_q, s_q, d = q.shape
+    _, h_kv, Lmax, _ = k.shape
+    out = np.full((B, h_q, s_q, d), np.nan)
+    lse = np.full((B, h_q, s_q), np.nan)
+    r, nr = _rows(rows_b)
+    rc = _load().oracle_gqa(_dp(q), _dp(k), _dp(v), _ip(lens), B, h_q, h_kv, s_q, d, Lmax, int(causal),
+                            float(scale), _dp(out), _dp(lse), _ip(r), nr, int(n_threads))
+    _check(rc, "oracle_gqa")
+    return out, lse
+
+
+def gqa_probs(q, k, cache_lens, causal: bool, scale: float, b: int, i: int, t: int, h_kv: int):
+    """Softmax probabilities of one query row of the GQA definition (visible keys only)."""
+    q, k, lens = _f64(q), _f64(k), _i32(cache_lens)
+    B, h_q, s_q, d = q.shape
+    Lmax = k.shape[2]
+    p = np.zeros(Lmax)
+    n = _load().oracle_gqa_probs(_dp(q), _dp(k), _ip(lens), B, h_q, h_kv, s_q, d, Lmax, int(causal),
+                                 float(scale), int(b), int(i), int(t), _dp(p))
+    if n < 0:
+        raise ValueError("oracle_gqa_probs: invalid argument")
+    return p[:n]
+
+
+def _latent(fn_name, q_c, q_r, w_uk, w_uv, latent, cache_lens, causal, scale, rows_b, n_threads):
+    q_c, q_r, w_uk, w_uv, latent, lens = (_f64(q_c), _f64(q_r), _f64(w_uk), _f64(w_uv), _f64(latent),
+                                          _i32(cache_lens))
+    B, h_q, s_q, d_h = q_c.shape
+    d_r = q_r.shape[3]
+    g, _, r_kv = w_uk.shape
+    Lmax = latent.shape[1]
+    if latent.shape[2] != r_kv + d_r:
+        raise ValueError("latent last dim must be r_kv + d_r")
+    out = np.full((B, h_q, s_q, d_h), np.nan)
+    lse = np.full((B, h_q, s_q), np.nan)
+    r, nr = _rows(rows_b)
+    rc = getattr(_load(), fn_name)(_dp(q_c), _dp(q_r), _dp(w_uk), _dp(w_uv), _dp(latent), _ip(lens), B, h_q,
+                                   g, s_q, d_h, r_kv, d_r, Lmax, int(causal), float(scale), _dp(out),
+                                   _dp(lse), _ip(r), nr, int(n_threads))
+    _check(rc, fn_name)
+    return out, lse
+
+
+def latent_expanded(q_c, q_r, w_uk, w_uv, latent, cache_lens, causal: bool, scale: float, rows_b=None,
+                    n_threads: int = 0):
+    """GQLA attention from its definition (eq. (1)): per-group keys/values expanded from the latent.
+
+    q_c [B,h_q,s_q,d_h], q_r [B,h_q,s_q,d_r], w_uk/w_uv [g,d_h,r_kv], latent [B,Lmax,r_kv+d_r]."""
+    return _latent("oracle_latent_expanded", q_c, q_r, w_uk, w_uv, latent, cache_lens, causal, scale,
+                   rows_b, n_threads)
+
+
+def latent_absorbed(q_c, q_r, w_uk, w_uv, latent, cache_lens, causal: bool, scale: float, rows_b=None,
+                    n_threads: int = 0):
+    """GQLA attention in the MQA-absorbed form (W^UK folded into q, W^UV applied after)."""
+    return _latent("oracle_latent_absorbed", q_c, q_r, w_uk, w_uv, latent, cache_lens, causal, scale,
+                   rows_b, n_threads)
+
+
+def latent_expand_cache(latent, w_uk, w_uv, n_threads: int = 0):
+    """One-time conversion latent -> (kc [B,g,Lmax,d_h], vc [B,g,Lmax,d_h], kr [B,Lmax,d_r])."""
+    latent, w_uk, w_uv = _f64(latent), _f64(w_uk), _f64(w_uv)
+    B, Lmax, W = latent.shape
+    g, d_h, r_kv = w_uk.shape
+    d_r = W - r_kv
+    kc = np.zeros((B, g, Lmax, d_h))
+    vc = np.zeros((B, g, Lmax, d_h))
+    kr = np.zeros((B, Lmax, d_r))
+    rc = _load().oracle_latent_expand_cache(_dp(latent), _dp(w_uk), _dp(w_uv), B, Lmax, g, d_h, r_kv, d_r,
+                                            _dp(kc), _dp(vc), _dp(kr), int(n_threads))
+    _check(rc, "oracle_latent_expand_cache")
+    return kc, vc, kr
+
+
+def gta(q_g, k_g, v, cache_lens, causal: bool, scale: float, rows_b=None, n_threads: int = 0):
+    """GTA shared-score attention. q_g [B,G,s_q,d_qk], k_g [B,G,Lmax,d_qk], v [B,H,Lmax,d_v].
+
+    Returns (out [B,H,s_q,d_v], lse [B,G,s_q])."""
+    q_g, k_g, v, lens = _f64(q_g), _f64(k_g), _f64(v), _i32(cache_lens)
+    B, G, s_q, d_qk = q_g.shape
+    _, H, Lmax, d_v = v.shape
+    out = np.full((B, H, s_q, d_v), np.nan)
+    lse = np.full((B, G, s_q), np.nan)
+    r, nr = _rows(rows_b)
+    rc = _load().oracle_gta(_dp(q_g), _dp(k_g), _dp(v), _ip(lens), B, G, H, s_q, d_qk, d_v, Lmax, int(causal),
+                            float(scale), _dp(out), _dp(lse), _ip(r), nr, int(n_threads))
+    _check(rc, "oracle_gta")
+    return out, lse
+
+
+def merge_partials(parts_o, parts_lse):
+    """Merge attention partials over disjoint key sets: parts_o [n,dv], parts_lse [n]."""
+    po, pl = _f64(parts_o), _f64(parts_lse)
+    n, dv = po.shape
+    out = np.zeros(dv)
+    lse = np.zeros(1)
+    rc = _load().oracle_merge_partials(_dp(po), _dp(pl), n, dv, _dp(out), _dp(lse))
+    _check(rc, "oracle_merge_partials")
+    return out, float(lse[0])

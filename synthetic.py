@@ -1,0 +1,156 @@
+"""Seeded synthetic inputs shared by the tests, the smoke check and the benchmark.
+
+This module holds no attention arithmetic: it only draws seeded random tensors
+with the shapes, dtypes and value distributions of the workloads on the pages
+(a Llama-3.1-8B-shaped GQA decode layer, a GQLA/MLA latent decode layer with
+(h_q, d_h, r_kv, d_h^R) = (128, 128, 512, 64), a GTA grouped shared-score
+prefill).  There is no public dataset behind any of them; the values are
+N(0, 1) (or N(0, 1/512) for the latent up-projections), cast to the compute
+dtype with round-to-nearest-even.
+
+Both sides of every parity check consume the tensors returned here: the CUDA
+library receives them on the device, the oracle receives the same values
+widened to float64.
+
+Layouts (row-major, last dimension contiguous):
+  GQA      q [B,h_q,s_q,d]   k,v [B,h_kv,Lmax,d]   cache_lens int32 [B]
+  latent   q_c [B,h_q,s_q,d_h]  q_r [B,h_q,s_q,d_r]  w_uk,w_uv [g,d_h,r_kv]
+           latent [B,Lmax,r_kv+d_r] (c^KV then k^R)
+  expanded kc,vc [B,g,Lmax,d_h]  kr [B,Lmax,d_r]
+  GTA      q_g [B,G,s_q,d_qk]  k_g [B,G,Lmax,d_qk]  v [B,H,Lmax,d_v]
+cache_lens[b] counts the valid tokens of sequence b including the s_q new
+query tokens.
+"""
+from __future__ import annotations
+
+import math
+
+import torch
+
+
+def _gen(seed: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return g
+
+
+def _randn(shape, g, dtype, device, std: float = 1.0, chunk_elems: int = 1 << 28):
+    """N(0, std^2) in `dtype`, drawn in fp32 (in chunks along dim 0 to bound peak memory)."""
+    out = torch.empty(shape, dtype=dtype, device=device)
+    n0 = shape[0]
+    per = max(1, math.prod(shape[1:]))
+    step = max(1, chunk_elems // per)
+    for s in range(0, n0, step):
+        e = min(n0, s + step)
+        x = torch.randn((e - s,) + tuple(shape[1:]), generator=g, device=device, dtype=torch.float32)
+        if std != 1.0:
+            x.mul_(std)
+        out[s:e].copy_(x)
+    return out
+
+
+def _lens(g, B, lo, hi, device):
+    if lo == hi:
+        return torch.full((B,), hi, dtype=torch.int32, device=device)
+    return torch.randint(lo, hi + 1, (B,), generator=g, device=device, dtype=torch.int64).to(torch.int32)
+
+
+def gqa_page_example():
+    """The glossary page's worked example: seed 0, q (1,8,16,64), k,v (1,2,16,64), fp32 on the CPU,
+    drawn in that order; then one decode step continuing the same generator:
+    q17 (1,8,1,64), k17, v17 (1,2,1,64)."""
+    torch.manual_seed(0)
+    q = torch.randn(1, 8, 16, 64)
+    k = torch.randn(1, 2, 16, 64)
+    v = torch.randn(1, 2, 16, 64)
+    q17 = torch.randn(1, 8, 1, 64)
+    k17 = torch.randn(1, 2, 1, 64)
+    v17 = torch.randn(1, 2, 1, 64)
+    return dict(q=q, k=k, v=v, q17=q17, k17=k17, v17=v17)
+
+
+def gqa_inputs(seed, B, h_q, h_kv, d, s_q, L_lo, L_hi, Lmax=None, dtype=torch.bfloat16, device="cpu"):
+    """GQA decode/prefill inputs; cache lengths uniform in [L_lo, L_hi] (inclusive)."""
+    Lmax = L_hi if Lmax is None else Lmax
+    g = _gen(seed, device)
+    lens = _lens(g, B, L_lo, L_hi, device)
+    q = _randn((B, h_q, s_q, d), g, dtype, device)
+    k = _randn((B, h_kv, Lmax, d), g, dtype, device)
+    v = _randn((B, h_kv, Lmax, d), g, dtype, device)
+    return dict(q=q, k=k, v=v, cache_lens=lens, scale=1.0 / math.sqrt(d))
+
+
+def latent_inputs(seed, B, h_q, g_groups, d_h, r_kv, d_r, s_q, L_lo, L_hi, Lmax=None, dtype=torch.bfloat16,
+                  device="cpu"):
+    """GQLA latent decode inputs: c^KV, k^R, q^C, q^R ~ N(0,1); W^UK, W^UV ~ N(0, 1/r_kv)."""
+    Lmax = L_hi if Lmax is None else Lmax
+    g = _gen(seed, device)
+    lens = _lens(g, B, L_lo, L_hi, device)
+    q_c = _randn((B, h_q, s_q, d_h), g, dtype, device)
+    q_r = _randn((B, h_q, s_q, d_r), g, dtype, device)
+    w_std = 1.0 / math.sqrt(r_kv)
+    w_uk = _randn((g_groups, d_h, r_kv), g, dtype, device, std=w_std)
+    w_uv = _randn((g_groups, d_h, r_kv), g, dtype, device, std=w_std)
+    latent = _randn((B, Lmax, r_kv + d_r), g, dtype, device)
+    return dict(q_c=q_c, q_r=q_r, w_uk=w_uk, w_uv=w_uv, latent=latent, cache_lens=lens,
+                scale=1.0 / math.sqrt(d_h + d_r))
+
+
+def expanded_inputs(seed, B, h_q, g_groups, d_h, d_r, s_q, L_lo, L_hi, Lmax=None, dtype=torch.bfloat16,
+                    device="cpu"):
+    """Inputs of the expanded (per-group GQA) latent path drawn directly: kc, vc, kr ~ N(0,1)."""
+    Lmax = L_hi if Lmax is None else Lmax
+    g = _gen(seed, device)
+    lens = _lens(g, B, L_lo, L_hi, device)
+    q_c = _randn((B, h_q, s_q, d_h), g, dtype, device)
+    q_r = _randn((B, h_q, s_q, d_r), g, dtype, device)
+    kc = _randn((B, g_groups, Lmax, d_h), g, dtype, device)
+    vc = _randn((B, g_groups, Lmax, d_h), g, dtype, device)
+    kr = _randn((B, Lmax, d_r), g, dtype, device)
+    return dict(q_c=q_c, q_r=q_r, kc=kc, vc=vc, kr=kr, cache_lens=lens, scale=1.0 / math.sqrt(d_h + d_r))
+
+
+def gta_inputs(seed, B, G, H, d_qk, d_v, s_q, L_lo, L_hi, Lmax=None, dtype=torch.bfloat16, device="cpu"):
+    """GTA shared-score inputs, all N(0,1). For prefill pass s_q == L_lo == L_hi."""
+    Lmax = L_hi if Lmax is None else Lmax
+    g = _gen(seed, device)
+    lens = _lens(g, B, L_lo, L_hi, device)
+    q_g = _randn((B, G, s_q, d_qk), g, dtype, device)
+    k_g = _randn((B, G, Lmax, d_qk), g, dtype, device)
+    v = _randn((B, H, Lmax, d_v), g, dtype, device)
+    return dict(q_g=q_g, k_g=k_g, v=v, cache_lens=lens, scale=1.0 / math.sqrt(d_qk))
+
+
+# The five workloads, by name.  Sizes follow the pages' layer shapes.
+WORKLOADS = {
+    "gqa_decode_llama8b": dict(kind="gqa", seed=2, B=64, h_q=32, h_kv=8, d=128, s_q=1, L_lo=1024, L_hi=8192,
+                               causal=True),
+    "gta_prefill_4k": dict(kind="gta", seed=3, B=8, G=3, H=12, d_qk=64, d_v=64, s_q=4096, L_lo=4096,
+                           L_hi=4096, causal=True),
+    "latent_decode_4k_sq1": dict(kind="latent", seed=4, B=64, h_q=128, g=8, d_h=128, r_kv=512, d_r=64, s_q=1,
+                                 L_lo=4096, L_hi=4096, causal=True),
+    "latent_decode_4k_sq2": dict(kind="latent", seed=4, B=64, h_q=128, g=8, d_h=128, r_kv=512, d_r=64, s_q=2,
+                                 L_lo=4096, L_hi=4096, causal=True),
+}
+
+
+def sweep_workload(kind: str, L: int) -> dict:
+    """Long-context sweep points: batch 64, s_q 1, equal cache length L for every sequence."""
+    if kind == "gqa":
+        return dict(kind="gqa", seed=5, B=64, h_q=32, h_kv=8, d=128, s_q=1, L_lo=L, L_hi=L, causal=True)
+    return dict(kind="latent", seed=5, B=64, h_q=128, g=8, d_h=128, r_kv=512, d_r=64, s_q=1, L_lo=L, L_hi=L,
+                causal=True)
+
+
+def make(w: dict, device="cpu", dtype=torch.bfloat16) -> dict:
+    """Materialise a workload description from WORKLOADS / sweep_workload."""
+    if w["kind"] == "gqa":
+        return gqa_inputs(w["seed"], w["B"], w["h_q"], w["h_kv"], w["d"], w["s_q"], w["L_lo"], w["L_hi"],
+                          dtype=dtype, device=device)
+    if w["kind"] == "latent":
+        return latent_inputs(w["seed"], w["B"], w["h_q"], w["g"], w["d_h"], w["r_kv"], w["d_r"], w["s_q"],
+                             w["L_lo"], w["L_hi"], dtype=dtype, device=device)
+    if w["kind"] == "gta":
+        return gta_inputs(w["seed"], w["B"], w["G"], w["H"], w["d_qk"], w["d_v"], w["s_q"], w["L_lo"], w["L_hi"],
+                          dtype=dtype, device=device)
+    raise ValueError(w["kind"])

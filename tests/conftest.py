@@ -1,0 +1,29 @@
+"""Shared pytest configuration.
+
+Markers:
+  gpu -- needs a CUDA device (B200, sm_100a).  Everything else runs on the CPU.
+"""
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def pytest_configure(config):
+    config.addinivalue_line("markers", "gpu: test needs a CUDA device (B200, sm_100a)")
+
+
+def pytest_collection_modifyitems(config, items):
+    # GPU tests need a GPU; make their absence loud rather than silently green.
+    import torch
+
+    if torch.cuda.is_available():
+        return
+    skip = pytest.mark.skip(reason="no CUDA device in this process")
+    for it in items:
+        if "gpu" in it.keywords:
+            it.add_marker(skip)

@@ -1,0 +1,323 @@
+"""Pins of the fp64 oracle to things other than itself (CPU only).
+
+Each test ties an oracle routine to something the pages or the mathematics fix:
+the glossary page's worked example and its printed facts, a library routine
+(torch's float64 scaled_dot_product_attention with an explicit mask) on the
+special cases it covers, closed forms, invariants the pages state (GQA with
+h_kv = h_q is MHA, h_kv = 1 is MQA, GQA equals MHA over repeat_interleave'd
+K/V, the absorbed latent path equals the expanded per-group path, a GTA group
+of one head is MHA) and brute-force special cases.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+import synthetic
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def golden(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+def bottom_right_mask(s_q, L, causal):
+    t = torch.arange(s_q)[:, None]
+    j = torch.arange(L)[None, :]
+    if not causal:
+        return torch.ones(s_q, L, dtype=torch.bool)
+    return j <= (L - s_q + t)
+
+
+def sdpa64(q, k, v, L, causal, scale):
+    """Library routine: torch float64 SDPA over the first L cache slots, bottom-right causal mask."""
+    s_q = q.shape[-2]
+    m = bottom_right_mask(s_q, L, causal)
+    return F.scaled_dot_product_attention(q.double(), k[..., :L, :].double(), v[..., :L, :].double(),
+                                          attn_mask=m, scale=scale)
+
+
+def rand(*shape, seed=0):
+    g = torch.Generator().manual_seed(seed)
+    return torch.randn(*shape, generator=g, dtype=torch.float64)
+
+
+# --------------------------------------------------------------------------- glossary example
+def test_glossary_worked_example():
+    gd = golden("gqa_glossary_example.json")
+    ex = synthetic.gqa_page_example()
+    q, k, v = ex["q"], ex["k"], ex["v"]
+    assert list(q.shape) == gd["q_shape"] and list(k.shape) == gd["kv_shape"]
+    lens = [16]
+    out, _ = oracle.gqa(q, k, v, lens, causal=True, scale=1 / 8)
+    assert list(out.shape) == gd["printed_output_shape"]
+    # "same as copied heads": GQA equals MHA over repeat_interleave'd K/V
+    rep = q.shape[1] // k.shape[1]
+    out_mha, _ = oracle.gqa(q, k.repeat_interleave(rep, 1), v.repeat_interleave(rep, 1), lens, True, 1 / 8)
+    assert np.allclose(out, out_mha, atol=gd["allclose_atol"]) == gd["printed_same_as_copied_heads"]
+    # the library routine the page calls, in float64
+    ref = F.scaled_dot_product_attention(q.double(), k.double(), v.double(), is_causal=True, enable_gqa=True)
+    assert np.abs(out - ref.numpy()).max() < 1e-12
+    # the page's second printed line
+    assert k[0, :, 0].numel() * 2 == gd["printed_cached_values_per_token_gqa"]
+    assert k.repeat_interleave(rep, 1)[0, :, 0].numel() * 2 == gd["printed_cached_values_per_token_mha"]
+
+
+def test_decode_step_equals_prefill_row():
+    """Appending a 17th token and decoding it equals row 17 of a 17-token causal prefill."""
+    ex = synthetic.gqa_page_example()
+    k = torch.cat([ex["k"], ex["k17"]], 2)
+    v = torch.cat([ex["v"], ex["v17"]], 2)
+    dec, dlse = oracle.gqa(ex["q17"], k, v, [17], True, 1 / 8)
+    pre, plse = oracle.gqa(torch.cat([ex["q"], ex["q17"]], 2), k, v, [17], True, 1 / 8)
+    assert np.abs(dec[:, :, 0] - pre[:, :, 16]).max() < 1e-14
+    assert np.abs(dlse[:, :, 0] - plse[:, :, 16]).max() < 1e-14
+
+
+# --------------------------------------------------------------------------- GQA against SDPA
+@pytest.mark.parametrize("h_q,h_kv", [(8, 8), (8, 1), (8, 2), (6, 3)])
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("s_q", [1, 2, 5])
+def test_gqa_matches_library_sdpa(h_q, h_kv, causal, s_q):
+    B, d, Lmax = 3, 16, 23
+    q, k, v = rand(B, h_q, s_q, d, seed=1), rand(B, h_kv, Lmax, d, seed=2), rand(B, h_kv, Lmax, d, seed=3)
+    lens = [23, 7, s_q]
+    scale = 0.37
+    out, lse = oracle.gqa(q, k, v, lens, causal, scale)
+    rep = h_q // h_kv
+    for b, L in enumerate(lens):
+        ref = sdpa64(q[b:b + 1], k[b:b + 1].repeat_interleave(rep, 1), v[b:b + 1].repeat_interleave(rep, 1), L,
+                     causal, scale)
+        assert np.abs(out[b] - ref[0].numpy()).max() < 1e-12
+        # lse from its definition: log of the softmax normaliser of the scaled scores
+        kk = k[b].repeat_interleave(rep, 0)[:, :L]
+        s = scale * torch.einsum("htd,hjd->htj", q[b], kk)
+        s = s.masked_fill(~bottom_right_mask(s_q, L, causal), -math.inf)
+        assert np.abs(lse[b] - torch.logsumexp(s, -1).numpy()).max() < 1e-12
+
+
+def test_bottom_right_reading_differs_from_top_left():
+    """The decode/MTP reading: query t sees keys <= L - s_q + t (torch's is_causal is top-left)."""
+    q, k, v = rand(1, 2, 2, 8, seed=4), rand(1, 2, 9, 8, seed=5), rand(1, 2, 9, 8, seed=6)
+    out, _ = oracle.gqa(q, k, v, [9], True, 0.5)
+    br = sdpa64(q, k, v, 9, True, 0.5).numpy()
+    tl = F.scaled_dot_product_attention(q, k, v, is_causal=True, scale=0.5).numpy()
+    assert np.abs(out - br).max() < 1e-12
+    assert np.abs(out - tl).max() > 1e-3
+
+
+def test_grouping_is_contiguous():
+    """Head i uses KV head floor(i / (h_q/h_kv)) -- repeat_interleave, not i % h_kv."""
+    q, k, v = rand(1, 4, 1, 8, seed=7), rand(1, 2, 5, 8, seed=8), rand(1, 2, 5, 8, seed=9)
+    out, _ = oracle.gqa(q, k, v, [5], False, 1.0)
+    wrong = sdpa64(q, k.repeat(1, 2, 1, 1), v.repeat(1, 2, 1, 1), 5, False, 1.0).numpy()
+    right = sdpa64(q, k.repeat_interleave(2, 1), v.repeat_interleave(2, 1), 5, False, 1.0).numpy()
+    assert np.abs(out - right).max() < 1e-12 and np.abs(out - wrong).max() > 1e-3
+
+
+# --------------------------------------------------------------------------- brute-force special cases
+def test_single_key_returns_its_value():
+    q, k, v = rand(2, 4, 1, 8, seed=10), rand(2, 2, 4, 8, seed=11), rand(2, 2, 4, 8, seed=12)
+    out, lse = oracle.gqa(q, k, v, [1, 1], True, 0.3)
+    for i in range(4):
+        assert np.abs(out[:, i, 0] - v[:, i // 2, 0].numpy()).max() < 1e-15
+        s0 = 0.3 * (q[:, i, 0] * k[:, i // 2, 0]).sum(-1).numpy()
+        assert np.abs(lse[:, i, 0] - s0).max() < 1e-14
+
+
+def test_zero_scale_is_prefix_mean():
+    q, k, v = rand(1, 2, 3, 8, seed=13), rand(1, 1, 10, 8, seed=14), rand(1, 1, 10, 8, seed=15)
+    out, lse = oracle.gqa(q, k, v, [10], True, 0.0)
+    for t in range(3):
+        n = 10 - 3 + t + 1
+        assert np.abs(out[0, :, t] - v[0, 0, :n].mean(0).numpy()).max() < 1e-14
+        assert abs(lse[0, 0, t] - math.log(n)) < 1e-14
+
+
+def test_equal_keys_give_mean_of_values():
+    q = rand(1, 2, 1, 8, seed=16)
+    k = rand(1, 1, 1, 8, seed=17).expand(1, 1, 12, 8).contiguous()
+    v = rand(1, 1, 12, 8, seed=18)
+    out, _ = oracle.gqa(q, k, v, [12], False, 0.9)
+    assert np.abs(out[0, :, 0] - v[0, 0].mean(0).numpy()).max() < 1e-14
+
+
+def test_key_permutation_invariance():
+    q, k, v = rand(1, 2, 2, 8, seed=19), rand(1, 1, 11, 8, seed=20), rand(1, 1, 11, 8, seed=21)
+    perm = torch.randperm(11, generator=torch.Generator().manual_seed(3))
+    a, la = oracle.gqa(q, k, v, [11], False, 0.7)
+    b, lb = oracle.gqa(q, k[:, :, perm], v[:, :, perm], [11], False, 0.7)
+    assert np.abs(a - b).max() < 1e-13 and np.abs(la - lb).max() < 1e-13
+
+
+def test_dominant_score_selects_value():
+    d = 8
+    q = torch.zeros(1, 1, 1, d, dtype=torch.float64)
+    q[..., 0] = 1.0
+    k = rand(1, 1, 6, d, seed=22) * 0.01
+    k[0, 0, 4, 0] = 50.0
+    v = rand(1, 1, 6, d, seed=23)
+    out, _ = oracle.gqa(q, k, v, [6], False, 1.0)
+    assert np.abs(out[0, 0, 0] - v[0, 0, 4].numpy()).max() < 1e-15
+
+
+def test_probabilities_sum_to_one_and_reproduce_output():
+    q, k, v = rand(2, 4, 2, 16, seed=24), rand(2, 2, 30, 16, seed=25), rand(2, 2, 30, 16, seed=26)
+    lens = [30, 13]
+    out, _ = oracle.gqa(q, k, v, lens, True, 0.25)
+    for b in range(2):
+        for i in range(4):
+            for t in range(2):
+                p = oracle.gqa_probs(q, k, lens, True, 0.25, b, i, t, h_kv=2)
+                assert len(p) == lens[b] - 2 + t + 1
+                assert abs(p.sum() - 1.0) < 1e-12 and (p >= 0).all()
+                assert np.abs(p @ v[b, i // 2, :len(p)].numpy() - out[b, i, t]).max() < 1e-13
+
+
+def test_merge_of_disjoint_partials_equals_full_attention():
+    """The split-KV combine, pinned against attention over the whole key set."""
+    q, k, v = rand(1, 1, 1, 16, seed=27), rand(1, 1, 40, 16, seed=28), rand(1, 1, 40, 16, seed=29)
+    full, flse = oracle.gqa(q, k, v, [40], False, 0.5)
+    cuts = [0, 7, 8, 25, 40]
+    po, pl = [], []
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        o, l = oracle.gqa(q, k[:, :, a:b].contiguous(), v[:, :, a:b].contiguous(), [b - a], False, 0.5)
+        po.append(o[0, 0, 0])
+        pl.append(l[0, 0, 0])
+    m, ml = oracle.merge_partials(np.stack(po), np.array(pl))
+    assert np.abs(m - full[0, 0, 0]).max() < 1e-13 and abs(ml - flse[0, 0, 0]) < 1e-13
+
+
+def test_invalid_arguments_rejected():
+    q, k, v = rand(1, 2, 2, 8), rand(1, 1, 5, 8), rand(1, 1, 5, 8)
+    with pytest.raises(ValueError):
+        oracle.gqa(q, k, v, [6], True, 1.0)  # L > Lmax
+    with pytest.raises(ValueError):
+        oracle.gqa(q, k, v, [1], True, 1.0)  # causal with L < s_q
+    with pytest.raises(ValueError):
+        oracle.gqa(rand(1, 3, 1, 8), rand(1, 2, 5, 8), rand(1, 2, 5, 8), [5], False, 1.0)  # h_q % h_kv
+
+
+# --------------------------------------------------------------------------- GQLA latent
+def latent_case(B=2, h_q=8, g=2, d_h=16, r_kv=32, d_r=8, s_q=2, Lmax=19, seed=40):
+    lat = synthetic.latent_inputs(seed, B, h_q, g, d_h, r_kv, d_r, s_q, 3, Lmax, dtype=torch.float64)
+    return lat
+
+
+def torch_latent_expanded(lat, causal):
+    """Eq. (1) with torch ops: k^C = W^UK_gamma c, v^C = W^UV_gamma c, key [k^C; k^R], query [q^C; q^R]."""
+    q_c, q_r, w_uk, w_uv, c = lat["q_c"], lat["q_r"], lat["w_uk"], lat["w_uv"], lat["latent"]
+    g, d_h, r_kv = w_uk.shape
+    B, h_q, s_q, _ = q_c.shape
+    rep = h_q // g
+    outs = []
+    for b, L in enumerate(lat["cache_lens"].tolist()):
+        cb = c[b, :L, :r_kv]
+        kr = c[b, :L, r_kv:]
+        kc = torch.einsum("gdr,jr->gjd", w_uk, cb)          # [g, L, d_h]
+        vc = torch.einsum("gdr,jr->gjd", w_uv, cb)
+        key = torch.cat([kc, kr.expand(g, L, kr.shape[-1])], -1).repeat_interleave(rep, 0)
+        val = vc.repeat_interleave(rep, 0)
+        qry = torch.cat([q_c[b], q_r[b]], -1)
+        outs.append(sdpa64(qry, key, val, L, causal, lat["scale"]))
+    return torch.stack(outs).numpy()
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_latent_expanded_matches_library(causal):
+    lat = latent_case()
+    out, _ = oracle.latent_expanded(lat["q_c"], lat["q_r"], lat["w_uk"], lat["w_uv"], lat["latent"],
+                                    lat["cache_lens"], causal, lat["scale"])
+    ref = torch_latent_expanded(lat, causal)
+    assert np.abs(out - ref).max() < 1e-12
+
+
+@pytest.mark.parametrize("s_q", [1, 2])
+def test_absorbed_equals_expanded(s_q):
+    """GQLA section 3.1 / Figure 2: the two decode paths give the same output."""
+    lat = latent_case(s_q=s_q, seed=41)
+    args = (lat["q_c"], lat["q_r"], lat["w_uk"], lat["w_uv"], lat["latent"], lat["cache_lens"], True,
+            lat["scale"])
+    a, la = oracle.latent_absorbed(*args)
+    e, le = oracle.latent_expanded(*args)
+    assert np.abs(a - e).max() <= 1e-10 * np.abs(e).max()
+    assert np.abs(la - le).max() < 1e-11
+
+
+def test_latent_identity_weights_reduce_to_mqa():
+    """g = 1, d_h = r_kv, W^UK = W^UV = I: one shared key [c; k^R] and value c for all heads (MQA)."""
+    B, h_q, r, d_r, s_q, Lmax = 2, 4, 16, 8, 2, 9
+    lat = synthetic.latent_inputs(42, B, h_q, 1, r, r, d_r, s_q, 4, Lmax, dtype=torch.float64)
+    eye = torch.eye(r, dtype=torch.float64)[None]
+    args = (lat["q_c"], lat["q_r"], eye, eye, lat["latent"], lat["cache_lens"], True, 0.3)
+    a, _ = oracle.latent_absorbed(*args)
+    e, _ = oracle.latent_expanded(*args)
+    for b, L in enumerate(lat["cache_lens"].tolist()):
+        key = lat["latent"][b:b + 1, None, :L].expand(1, h_q, L, r + d_r)
+        val = lat["latent"][b:b + 1, None, :L, :r].expand(1, h_q, L, r)
+        qry = torch.cat([lat["q_c"][b:b + 1], lat["q_r"][b:b + 1]], -1)
+        ref = sdpa64(qry, key, val, L, True, 0.3)[0].numpy()
+        assert np.abs(a[b] - ref).max() < 1e-12 and np.abs(e[b] - ref).max() < 1e-12
+
+
+def test_expand_cache_then_gqa_equals_latent():
+    """The one-time cache expansion followed by GQA over [kc; kr] equals the latent definition."""
+    lat = latent_case(seed=43)
+    kc, vc, kr = oracle.latent_expand_cache(lat["latent"], lat["w_uk"], lat["w_uv"])
+    g = lat["w_uk"].shape[0]
+    key = np.concatenate([kc, np.broadcast_to(kr[:, None], kc.shape[:3] + (kr.shape[-1],))], -1)
+    # GQA over the concatenated key needs equal K/V widths: pad V with zeros, then drop them.
+    pad = np.zeros(vc.shape[:3] + (kr.shape[-1],))
+    val = np.concatenate([vc, pad], -1)
+    q = torch.cat([lat["q_c"], lat["q_r"]], -1)
+    out, lse = oracle.gqa(q, key, val, lat["cache_lens"], True, lat["scale"])
+    e, le = oracle.latent_expanded(lat["q_c"], lat["q_r"], lat["w_uk"], lat["w_uv"], lat["latent"],
+                                   lat["cache_lens"], True, lat["scale"])
+    assert np.abs(out[..., :kc.shape[-1]] - e).max() < 1e-12
+    assert np.abs(out[..., kc.shape[-1]:]).max() == 0.0
+    assert np.abs(lse - le).max() < 1e-12
+    assert g == kc.shape[1]
+
+
+# --------------------------------------------------------------------------- GTA
+@pytest.mark.parametrize("G,H", [(3, 12), (2, 2), (1, 4)])
+@pytest.mark.parametrize("causal", [True, False])
+def test_gta_matches_library(G, H, causal):
+    B, s_q, d_qk, d_v, Lmax = 2, 5, 16, 8, 13
+    gt = synthetic.gta_inputs(44, B, G, H, d_qk, d_v, s_q, 5, Lmax, dtype=torch.float64)
+    out, lse = oracle.gta(gt["q_g"], gt["k_g"], gt["v"], gt["cache_lens"], causal, 0.4)
+    rep = H // G
+    for b, L in enumerate(gt["cache_lens"].tolist()):
+        ref = sdpa64(gt["q_g"][b].repeat_interleave(rep, 0), gt["k_g"][b].repeat_interleave(rep, 0), gt["v"][b], L,
+                     causal, 0.4)
+        assert np.abs(out[b] - ref.numpy()).max() < 1e-12
+        s = 0.4 * torch.einsum("gtd,gjd->gtj", gt["q_g"][b], gt["k_g"][b, :, :L])
+        s = s.masked_fill(~bottom_right_mask(s_q, L, causal), -math.inf)
+        assert np.abs(lse[b] - torch.logsumexp(s, -1).numpy()).max() < 1e-12
+
+
+def test_gta_equal_values_give_equal_head_outputs():
+    B, G, H, s_q, d, Lmax = 1, 2, 8, 3, 8, 7
+    gt = synthetic.gta_inputs(45, B, G, H, d, d, s_q, 7, Lmax, dtype=torch.float64)
+    v = gt["v"][:, :1].expand(B, H, Lmax, d).contiguous()
+    out, _ = oracle.gta(gt["q_g"], gt["k_g"], v, gt["cache_lens"], True, 0.5)
+    for grp in range(G):
+        hs = range(grp * 4, grp * 4 + 4)
+        for h in hs:
+            assert np.abs(out[0, h] - out[0, grp * 4]).max() == 0.0
+    assert np.abs(out[0, 0] - out[0, 4]).max() > 1e-6
+
+
+def test_gta_single_head_groups_is_mha():
+    B, H, s_q, d, Lmax = 2, 3, 4, 8, 9
+    gt = synthetic.gta_inputs(46, B, H, H, d, d, s_q, 4, Lmax, dtype=torch.float64)
+    out, _ = oracle.gta(gt["q_g"], gt["k_g"], gt["v"], gt["cache_lens"], True, 0.6)
+    ref, _ = oracle.gqa(gt["q_g"], gt["k_g"], gt["v"], gt["cache_lens"], True, 0.6)
+    assert np.abs(out - ref).max() == 0.0
