@@ -1,0 +1,179 @@
+/*
+ * lka.h -- C ABI of latent_kv_attention_b200: grouped / latent-KV scaled-dot-
+ * product attention on NVIDIA B200 (sm_100a).
+ *
+ * Four attention entry points, one per cache layout the pages describe, plus
+ * the one-time cache conversion and a few helpers.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE pointers owned by the caller, row-major
+ *    with the last dimension contiguous, 16-byte aligned.  The library never
+ *    allocates device memory and keeps no per-call state: scratch space is the
+ *    caller's workspace `ws` (size from the matching *_workspace_size call).
+ *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream).  Calls on one workspace must not overlap.
+ *  - cache_lens is a DEVICE int32 array [B]: cache_lens[b] = L_b counts the
+ *    valid cache tokens of sequence b INCLUDING the s_q new query tokens,
+ *    whose keys/values the caller has already written at positions
+ *    L_b - s_q .. L_b - 1.  Requirement: 1 <= L_b <= Lmax, and L_b >= s_q when
+ *    causal.  The device cannot report a bad length synchronously: an entry
+ *    outside the range is clamped into it and LKA_ERR_BAD_LENGTH is raised in
+ *    the workspace status word (read it with lka_device_status).
+ *  - causal != 0 selects bottom-right aligned causal masking: query t
+ *    (0 <= t < s_q) sees keys 0 .. L_b - s_q + t.  causal == 0 lets every query
+ *    see keys 0 .. L_b - 1.  Prefill is s_q == L_b; decode is s_q = 1, or 2 for
+ *    multi-token prediction.
+ *  - scale multiplies the query-key dot products before the softmax.
+ *  - Outputs have the input dtype (bf16 results are rounded to nearest even);
+ *    lse (optional, may be NULL) is fp32, natural log of the softmax
+ *    normaliser of each query row.
+ *  - Errors are return codes; on a validation error nothing is enqueued and
+ *    nothing is written.  Asynchronous CUDA launch failures are reported as
+ *    LKA_ERR_CUDA.
+ *
+ * Sources (web pages on the subject, cited by title and section):
+ *  [GQA]  "Grouped Query Attention (GQA)" glossary page, "How GQA works" and
+ *         "How GQA shrinks the KV cache".
+ *  [GQLA] "GQLA: Group-Query Latent Attention for Hardware-Adaptive Large
+ *         Language Model Decoding", section 1 and section 3.1 with eq. (1) and
+ *         Figure 2.
+ *  [GTA]  "GTA: Grouped-head latenT Attention" press article, section on the
+ *         grouped shared attention matrix.
+ */
+#ifndef LKA_H
+#define LKA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LKA_API __attribute__((visibility("default")))
+#else
+#define LKA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LKA_OK = 0,
+    LKA_ERR_INVALID_ARG = 1,  /* a host-visible argument is out of range or a pointer is NULL/misaligned */
+    LKA_ERR_UNSUPPORTED = 2,  /* valid arguments this build has no kernel for (dtype, head dim, ...) */
+    LKA_ERR_WORKSPACE = 3,    /* ws is NULL or ws_bytes is below the *_workspace_size value */
+    LKA_ERR_CUDA = 4,         /* a CUDA call or kernel launch failed */
+    LKA_ERR_TIMEOUT = 5,      /* device status: a bounded in-kernel wait ran out (the kernel exited early) */
+    LKA_ERR_BAD_LENGTH = 6    /* device status: a cache_lens entry was outside its range and was clamped */
+} lka_status_t;
+
+typedef enum { LKA_BF16 = 0, LKA_FP32 = 1 } lka_dtype_t;
+
+/* ------------------------------------------------------------------------ */
+/* (a) GQA attention  [GQA "How GQA works"]                                 */
+/*  Query head i (0 <= i < h_q) attends with KV head floor(i / (h_q/h_kv)):  */
+/*  each KV head serves a contiguous group of h_q/h_kv query heads.          */
+/*  h_kv == h_q is MHA, h_kv == 1 is MQA.                                    */
+/*   q   [B, h_q,  s_q,  d_h]     k, v [B, h_kv, Lmax, d_h]                  */
+/*   out [B, h_q,  s_q,  d_h]     lse  [B, h_q, s_q] fp32 or NULL            */
+/*  dtype: LKA_BF16 (d_h in {64, 128, 256}) or LKA_FP32 (d_h in {64, 128}).  */
+/*  Split-KV flash decoding: long caches are split over CTAs and merged by   */
+/*  log-sum-exp; the split partials live in ws.                              */
+/* ------------------------------------------------------------------------ */
+LKA_API size_t gqa_attn_workspace_size(int B, int h_q, int h_kv, int s_q, int d_h, int Lmax);
+LKA_API lka_status_t gqa_attn(const void *q, const void *k, const void *v, const int32_t *cache_lens, void *out,
+                      float *lse, int B, int h_q, int h_kv, int s_q, int d_h, int Lmax, int causal, float scale,
+                      lka_dtype_t dtype, void *ws, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* (b) GQLA MQA-absorbed latent attention  [GQLA sec. 1, sec. 3.1 eq. (1),  */
+/*     Figure 2(b)]                                                         */
+/*  The cache holds, per token, the joint latent c^KV (r_kv values) followed */
+/*  by the shared RoPE key k^R (d_r values).  Head i belongs to group        */
+/*  gamma = floor(i / (h_q/g)); W^UK_gamma, W^UV_gamma are d_h x r_kv.       */
+/*  Computes, for every head i and query t:                                  */
+/*     q~  = W^UK_gamma^T q^C                (absorption into the query)     */
+/*     s_j = scale * (<q~, c_j> + <q^R, k^R_j>)                              */
+/*     o~  = sum_j softmax(s)_j c_j          (attention over the latent)     */
+/*     out = W^UV_gamma o~                   (up-projection of the output)   */
+/*  which equals GQA over the per-group expanded keys/values (see (c)).      */
+/*   q_c [B,h_q,s_q,d_h]  q_r [B,h_q,s_q,d_r]  w_uk, w_uv [g,d_h,r_kv]       */
+/*   latent [B,Lmax,r_kv+d_r]  out [B,h_q,s_q,d_h]  lse [B,h_q,s_q] or NULL  */
+/*  Supported: bf16, r_kv = 512, d_r = 64, d_h = 128, h_q = 128, s_q <= 2.   */
+/* ------------------------------------------------------------------------ */
+LKA_API size_t latent_absorbed_attn_workspace_size(int B, int h_q, int g, int s_q, int d_h, int r_kv, int d_r, int Lmax);
+LKA_API lka_status_t latent_absorbed_attn(const void *q_c, const void *q_r, const void *w_uk, const void *w_uv,
+                                  const void *latent, const int32_t *cache_lens, void *out, float *lse, int B,
+                                  int h_q, int g, int s_q, int d_h, int r_kv, int d_r, int Lmax, int causal,
+                                  float scale, lka_dtype_t dtype, void *ws, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* (c) GQLA GQA path over the per-group expanded cache  [GQLA sec. 1,       */
+/*     sec. 3.1, Figure 2(a)]                                               */
+/*  Key of group gamma at token j: [kc[b,gamma,j,:] ; kr[b,j,:]] (the RoPE   */
+/*  key is stored once and shared by all groups); value: vc[b,gamma,j,:];    */
+/*  query of head i: [q_c ; q_r].  h_q/g query heads per group.              */
+/*   kc, vc [B,g,Lmax,d_h]  kr [B,Lmax,d_r]  other arguments as in (b).      */
+/*  Supported: bf16, d_h = 128, d_r = 64, h_q/g = 16, s_q <= 2.              */
+/* ------------------------------------------------------------------------ */
+LKA_API size_t latent_expand_gqa_attn_workspace_size(int B, int h_q, int g, int s_q, int d_h, int d_r, int Lmax);
+LKA_API lka_status_t latent_expand_gqa_attn(const void *q_c, const void *q_r, const void *kc, const void *vc,
+                                    const void *kr, const int32_t *cache_lens, void *out, float *lse, int B,
+                                    int h_q, int g, int s_q, int d_h, int d_r, int Lmax, int causal, float scale,
+                                    lka_dtype_t dtype, void *ws, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* (d) GTA shared-score attention  [GTA, grouped shared attention matrix]   */
+/*  H heads in G groups of H/G; head h uses group gamma = floor(h/(H/G)).    */
+/*  One score matrix softmax(scale q_g k_g^T) per group is computed once and */
+/*  applied to the values of every head of the group.                        */
+/*   q_g [B,G,s_q,d_qk]  k_g [B,G,Lmax,d_qk]  v [B,H,Lmax,d_v]               */
+/*   out [B,H,s_q,d_v]   lse [B,G,s_q] (one per group and query) or NULL     */
+/*  Supported: bf16, d_qk = d_v = 64, H/G <= 4.                              */
+/* ------------------------------------------------------------------------ */
+LKA_API size_t gta_shared_score_attn_workspace_size(int B, int G, int H, int s_q, int d_qk, int d_v, int Lmax);
+LKA_API lka_status_t gta_shared_score_attn(const void *q_g, const void *k_g, const void *v, const int32_t *cache_lens,
+                                   void *out, float *lse, int B, int G, int H, int s_q, int d_qk, int d_v,
+                                   int Lmax, int causal, float scale, lka_dtype_t dtype, void *ws, size_t ws_bytes,
+                                   void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* One-time cache conversion latent -> per-group expanded cache             */
+/* [GQLA sec. 3.1: switching paths needs a one-time compression/expansion   */
+/*  of the KV cache at deployment, never at run time]                       */
+/*   kc[b,gamma,j,:] = W^UK_gamma c_j,  vc[b,gamma,j,:] = W^UV_gamma c_j,     */
+/*   kr[b,j,:] = k^R_j  for every slot j < Lmax.  bf16 in/out, fp32 sums.   */
+/* ------------------------------------------------------------------------ */
+LKA_API lka_status_t latent_expand_cache(const void *latent, const void *w_uk, const void *w_uv, int B, int Lmax, int g,
+                                 int d_h, int r_kv, int d_r, void *kc, void *vc, void *kr, lka_dtype_t dtype,
+                                 void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Helpers                                                                  */
+/* ------------------------------------------------------------------------ */
+/* Synchronises `stream`, then returns the sticky status word of workspace ws:
+ * LKA_OK, LKA_ERR_TIMEOUT (takes precedence) or LKA_ERR_BAD_LENGTH. */
+LKA_API lka_status_t lka_device_status(const void *ws, void *stream);
+/* Enqueues a reset of the workspace status word to LKA_OK on `stream`. */
+LKA_API lka_status_t lka_clear_status(void *ws, void *stream);
+/* Human-readable name of a status code (static string, never NULL). */
+LKA_API const char *lka_status_string(lka_status_t status);
+/* Process-wide split size (KV tokens per CTA) for the split-KV kernels; 0 restores the automatic choice.
+ * A tuning and test knob: results do not depend on it beyond rounding.  Returns the previous value. */
+LKA_API int lka_set_split_tokens(int tokens);
+/* Timing hook for benchmarks: lka_kernel_timing(1) discards earlier records and starts recording a pair of
+ * CUDA events around the main (dominant) kernel of every later entry-point call, on that call's stream;
+ * lka_kernel_timing(0) stops recording.  lka_kernel_timing_read waits for the recorded events and returns the
+ * number of timed launches and their summed duration in milliseconds. */
+LKA_API lka_status_t lka_kernel_timing(int enable);
+LKA_API lka_status_t lka_kernel_timing_read(int *launches, double *total_ms);
+/* Self-test of the bounded in-kernel wait: launches one CTA that waits on a barrier nobody arrives at,
+ * for at most limit_us microseconds, then records LKA_ERR_TIMEOUT in ws's status word and exits.
+ * Used to check the timeout path without hanging the GPU. */
+LKA_API lka_status_t lka_selftest_wait_timeout(void *ws, size_t ws_bytes, int limit_us, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LKA_H */

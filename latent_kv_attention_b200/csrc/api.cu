@@ -1,0 +1,226 @@
+// api.cu -- the C ABI entry points (include/lka.h): argument validation,
+// split planning, workspace carving, TMA descriptors and kernel dispatch.
+// No allocation happens here: all scratch space is the caller's workspace.
+#include <math.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+#include <utility>
+#include <vector>
+
+#include "common.cuh"
+#include "gqa_decode.h"
+#include "host_util.h"
+
+namespace lka {
+
+static std::atomic<int> g_split_tokens{0};
+int split_tokens_knob() { return g_split_tokens.load(std::memory_order_relaxed); }
+
+// ---------------------------------------------------------------- kernel timing hook
+struct TimingRegistry {
+    std::mutex mu;
+    std::atomic<bool> on{false};
+    std::vector<cudaEvent_t> pool;
+    std::vector<std::pair<cudaEvent_t, cudaEvent_t>> pending;
+};
+static TimingRegistry& timing_reg() {
+    static TimingRegistry r;
+    return r;
+}
+bool kernel_timing_on() { return timing_reg().on.load(std::memory_order_relaxed); }
+cudaEvent_t kernel_timing_event() {
+    auto& r = timing_reg();
+    std::lock_guard<std::mutex> g(r.mu);
+    if (!r.pool.empty()) {
+        cudaEvent_t e = r.pool.back();
+        r.pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+void kernel_timing_push(cudaEvent_t a, cudaEvent_t b) {
+    auto& r = timing_reg();
+    std::lock_guard<std::mutex> g(r.mu);
+    r.pending.emplace_back(a, b);
+}
+
+// ---------------------------------------------------------------- GQA plan
+struct GqaPlan {
+    int rb, n_rb, tile, split_tokens, nsplit;
+    size_t off_lse, off_o, ws_bytes;
+};
+
+static int pick_rb(int rows, int d, int dtype_bytes) {
+    int cap = 16;
+    if ((dtype_bytes == 2 && d == 64) || d == 256) cap = 8;
+    int rb = 1;
+    while (rb < rows && rb < cap) rb *= 2;
+    return rb;
+}
+
+static lka_status_t gqa_plan(int B, int h_q, int h_kv, int s_q, int d_h, int Lmax, int dtype_bytes, GqaPlan* pl) {
+    if (B < 0 || h_q < 1 || h_kv < 1 || s_q < 1 || Lmax < 1 || d_h < 1) return LKA_ERR_INVALID_ARG;
+    if (h_q % h_kv) return LKA_ERR_INVALID_ARG;
+    const bool d_ok = dtype_bytes == 2 ? (d_h == 64 || d_h == 128 || d_h == 256) : (d_h == 64 || d_h == 128);
+    if (!d_ok) return LKA_ERR_UNSUPPORTED;
+    if ((long long)B * h_kv * Lmax >= (1ll << 31)) return LKA_ERR_UNSUPPORTED;
+    const int R = (h_q / h_kv) * s_q;
+    pl->rb = pick_rb(R, d_h, dtype_bytes);
+    pl->n_rb = cdiv(R, pl->rb);
+    if ((long long)h_kv * pl->n_rb > 65535 || B > 65535) return LKA_ERR_UNSUPPORTED;
+    pl->tile = gqa_tile_tokens(dtype_bytes, d_h, pl->rb);
+    if (pl->tile <= 0) return LKA_ERR_UNSUPPORTED;
+    int st = split_tokens_knob();
+    if (st <= 0) {
+        // aim at ~12 waves of 2 resident CTAs per SM over the worst-case (Lmax) work
+        const long long units = (long long)(B > 0 ? B : 1) * h_kv * pl->n_rb;
+        const long long target = (long long)sm_count() * 2 * 12;
+        long long nsp = (target + units - 1) / units;
+        if (nsp < 1) nsp = 1;
+        st = (int)((Lmax + nsp - 1) / nsp);
+        if (st < 4 * pl->tile) st = 4 * pl->tile;
+    }
+    st = cdiv(st, pl->tile) * pl->tile;
+    pl->split_tokens = st;
+    pl->nsplit = cdiv(Lmax, st);
+    WsCarve c;
+    const size_t rows = (size_t)B * h_q * s_q;
+    if (pl->nsplit > 1) {
+        pl->off_lse = c.take(rows * pl->nsplit * sizeof(float));
+        pl->off_o = c.take(rows * pl->nsplit * (size_t)d_h * sizeof(float));
+    } else {
+        pl->off_lse = pl->off_o = 0;
+    }
+    pl->ws_bytes = c.off;
+    return LKA_OK;
+}
+
+static lka_status_t launch_status(cudaError_t e) { return e == cudaSuccess ? LKA_OK : LKA_ERR_CUDA; }
+
+}  // namespace lka
+
+using namespace lka;
+
+extern "C" {
+
+const char* lka_status_string(lka_status_t s) {
+    switch (s) {
+        case LKA_OK: return "LKA_OK";
+        case LKA_ERR_INVALID_ARG: return "LKA_ERR_INVALID_ARG";
+        case LKA_ERR_UNSUPPORTED: return "LKA_ERR_UNSUPPORTED";
+        case LKA_ERR_WORKSPACE: return "LKA_ERR_WORKSPACE";
+        case LKA_ERR_CUDA: return "LKA_ERR_CUDA";
+        case LKA_ERR_TIMEOUT: return "LKA_ERR_TIMEOUT";
+        case LKA_ERR_BAD_LENGTH: return "LKA_ERR_BAD_LENGTH";
+    }
+    return "LKA_ERR_UNKNOWN";
+}
+
+int lka_set_split_tokens(int tokens) { return g_split_tokens.exchange(tokens < 0 ? 0 : tokens); }
+
+lka_status_t lka_kernel_timing(int enable) {
+    auto& r = timing_reg();
+    std::lock_guard<std::mutex> g(r.mu);
+    for (auto& pr : r.pending) {
+        r.pool.push_back(pr.first);
+        r.pool.push_back(pr.second);
+    }
+    r.pending.clear();
+    r.on.store(enable != 0);
+    return LKA_OK;
+}
+
+lka_status_t lka_kernel_timing_read(int* launches, double* total_ms) {
+    if (!launches || !total_ms) return LKA_ERR_INVALID_ARG;
+    auto& r = timing_reg();
+    std::lock_guard<std::mutex> g(r.mu);
+    double ms = 0.0;
+    for (auto& pr : r.pending) {
+        if (cudaEventSynchronize(pr.second) != cudaSuccess) return LKA_ERR_CUDA;
+        float t = 0.f;
+        if (cudaEventElapsedTime(&t, pr.first, pr.second) != cudaSuccess) return LKA_ERR_CUDA;
+        ms += t;
+    }
+    *launches = (int)r.pending.size();
+    *total_ms = ms;
+    return LKA_OK;
+}
+
+lka_status_t lka_device_status(const void* ws, void* stream) {
+    if (!ws) return LKA_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return LKA_ERR_CUDA;
+    uint32_t st = 0;
+    if (cudaMemcpy(&st, ws, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess) return LKA_ERR_CUDA;
+    if (st & kDevTimeout) return LKA_ERR_TIMEOUT;
+    if (st & kDevBadLength) return LKA_ERR_BAD_LENGTH;
+    return LKA_OK;
+}
+
+lka_status_t lka_clear_status(void* ws, void* stream) {
+    if (!ws) return LKA_ERR_INVALID_ARG;
+    return launch_status(cudaMemsetAsync(ws, 0, sizeof(uint32_t), (cudaStream_t)stream));
+}
+
+size_t gqa_attn_workspace_size(int B, int h_q, int h_kv, int s_q, int d_h, int Lmax) {
+    GqaPlan pl;
+    // the size does not depend on the dtype beyond the supported head dims: plan with bf16, then fp32
+    if (gqa_plan(B, h_q, h_kv, s_q, d_h, Lmax, 2, &pl) == LKA_OK) {
+        GqaPlan pf;
+        if (gqa_plan(B, h_q, h_kv, s_q, d_h, Lmax, 4, &pf) == LKA_OK && pf.ws_bytes > pl.ws_bytes) return pf.ws_bytes;
+        return pl.ws_bytes;
+    }
+    if (gqa_plan(B, h_q, h_kv, s_q, d_h, Lmax, 4, &pl) == LKA_OK) return pl.ws_bytes;
+    return 0;
+}
+
+lka_status_t gqa_attn(const void* q, const void* k, const void* v, const int32_t* cache_lens, void* out, float* lse,
+                      int B, int h_q, int h_kv, int s_q, int d_h, int Lmax, int causal, float scale,
+                      lka_dtype_t dtype, void* ws, size_t ws_bytes, void* stream) {
+    if (dtype != LKA_BF16 && dtype != LKA_FP32) return LKA_ERR_UNSUPPORTED;
+    const int eb = dtype == LKA_BF16 ? 2 : 4;
+    GqaPlan pl;
+    lka_status_t s = gqa_plan(B, h_q, h_kv, s_q, d_h, Lmax, eb, &pl);
+    if (s != LKA_OK) return s;
+    if (B == 0) return LKA_OK;
+    if (!q || !k || !v || !cache_lens || !out) return LKA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(cache_lens))
+        return LKA_ERR_INVALID_ARG;
+    if (!isfinite(scale)) return LKA_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < pl.ws_bytes) return LKA_ERR_WORKSPACE;
+    if (!aligned16(ws)) return LKA_ERR_INVALID_ARG;
+
+    const CUtensorMapDataType tdt = eb == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    const uint64_t rows = (uint64_t)B * h_kv * Lmax;
+    CUtensorMap tk, tv;
+    if (!make_tmap_2d(&tk, tdt, k, d_h, rows, (uint64_t)d_h * eb, 128 / eb, pl.tile) ||
+        !make_tmap_2d(&tv, tdt, v, d_h, rows, (uint64_t)d_h * eb, 128 / eb, pl.tile))
+        return LKA_ERR_CUDA;
+
+    GqaParams p;
+    p.q = q;
+    p.out = out;
+    p.lse = lse;
+    p.lens = cache_lens;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    p.part_lse = pl.nsplit > 1 ? reinterpret_cast<float*>(w + pl.off_lse) : nullptr;
+    p.part_o = pl.nsplit > 1 ? reinterpret_cast<float*>(w + pl.off_o) : nullptr;
+    p.status = reinterpret_cast<uint32_t*>(w);
+    p.B = B;
+    p.h_q = h_q;
+    p.h_kv = h_kv;
+    p.s_q = s_q;
+    p.Lmax = Lmax;
+    p.causal = causal ? 1 : 0;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.split_tokens = pl.split_tokens;
+    p.nsplit_max = pl.nsplit;
+    p.n_rb = pl.n_rb;
+    p.ratio = h_q / h_kv;
+    return launch_status(gqa_decode_launch(tk, tv, p, eb, d_h, pl.rb, pl.nsplit, (cudaStream_t)stream));
+}
+
+}  // extern "C"

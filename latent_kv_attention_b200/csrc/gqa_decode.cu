@@ -1,0 +1,519 @@
+// gqa_decode.cu -- split-KV flash decoding for grouped-query attention on
+// CUDA cores, and the log-sum-exp merge of its split partials.
+//
+// Operation ("Grouped Query Attention (GQA)" glossary page, "How GQA works"):
+// per query head plain scaled-dot-product attention, with each KV head shared
+// by a contiguous group of h_q/h_kv query heads.  Decode is bound by reading
+// the KV cache ("How GQA shrinks the KV cache": every new token reads the whole
+// cache), at 4 FLOPs per cache byte for 4 heads per group, far below the
+// tensor-core ridge, so the contraction runs on the FP32 pipes and the design
+// goal is streaming the cache at HBM speed.
+//
+// One CTA = (sequence b, KV head, block of RB query rows of that group, split
+// of the key range).  A producer warp streams K and V tiles of T_TILE tokens
+// with TMA (128-byte swizzle) through an NSTAGE ring of mbarrier-guarded
+// stages; each KV tile is read from HBM once and used by all query rows of the
+// group.  Four consumer warps each own a quarter of every tile and run an
+// independent online softmax over it:
+//   scores: LPT lanes per token, each lane holding its slice of the RB query
+//           rows in registers (pre-scaled by scale*log2 e), a shuffle
+//           reduce-scatter over the LPT lanes;
+//   softmax: running max / sum per row with warp shuffles, exp2;
+//   P*V:    each lane owns D/32 output dims of all RB rows, P is broadcast from
+//           shared memory.
+// The four warp states are merged in shared memory at the end.  A split whose
+// sequence needs a single split writes the final output directly; otherwise it
+// writes an fp32 partial (normalised O and log2-domain lse) that
+// gqa_combine_kernel merges.
+#include "common.cuh"
+#include "gqa_decode.h"
+#include "host_util.h"
+
+namespace lka {
+
+template <typename T, int D, int RB>
+struct GqaCfg {
+    static constexpr int E = sizeof(T);
+    static constexpr int EPC = 16 / E;           // elements per 16-byte chunk
+    static constexpr int CPR = D * E / 16;       // chunks per row
+    static constexpr int NSEG = D * E / 128;     // 128-byte swizzle segments per row
+    static constexpr int SEG_ELEMS = 128 / E;    // elements per segment (TMA box width)
+    // lanes per token in the score phase: enough that the query slice held per
+    // lane stays at 64 fp32 registers, never fewer than the rows (so that the
+    // reduce-scatter leaves one row per lane), at most one chunk per lane
+    static constexpr int LPT0 = RB * D / 64 > RB ? RB * D / 64 : RB;
+    static constexpr int LPT1 = LPT0 < CPR ? LPT0 : CPR;
+    static constexpr int LPT = LPT1 < 32 ? LPT1 : 32;
+    static constexpr int CPL = CPR / LPT;        // chunks per lane
+    static constexpr int DUP = LPT / RB;         // lanes holding the same row after the reduction
+    static constexpr int P = 32 / LPT;           // tokens per warp pass
+    static constexpr int TW = P > 16 ? P : 16;   // tokens per warp per tile
+    static constexpr int NPASS = TW / P;
+    static constexpr int T_TILE = 4 * TW;
+    static constexpr int DPLV = D / 32;          // value dims per lane
+    static constexpr int MAT_BYTES = T_TILE * D * E;
+    static constexpr int STAGE_BYTES = 2 * MAT_BYTES;
+    static constexpr int NSTAGE0 = (96 * 1024) / STAGE_BYTES;
+    static constexpr int NSTAGE = NSTAGE0 < 2 ? 2 : (NSTAGE0 > 4 ? 4 : NSTAGE0);
+    static constexpr int P_BYTES = 4 * TW * RB * 4 + 4 * RB * 4;  // probabilities + rescale factors
+    static constexpr int MERGE_BYTES = 4 * RB * D * 4 + 2 * 4 * RB * 4;
+    static constexpr int SMEM = 1024 /*align slack*/ + NSTAGE * STAGE_BYTES + P_BYTES + 256 /*barriers*/;
+    static constexpr int MINB = (RB <= 8 && SMEM <= 110 * 1024) ? 2 : 1;  // resident CTAs per SM
+    static_assert(D * E >= 128 && (D * E) % 128 == 0, "row must be whole 128-byte segments");
+    static_assert(LPT >= RB && LPT <= 32 && LPT <= CPR && CPR % LPT == 0, "lane split must own whole chunks");
+    static_assert(MERGE_BYTES <= NSTAGE * STAGE_BYTES, "merge scratch reuses the stage ring");
+    static_assert(D % 32 == 0 && (DPLV * E) % 4 == 0, "value slice per lane");
+};
+
+// Byte offset of 16-byte chunk `chunk` of segment `seg` of tile row `row`
+// inside one TMA-loaded matrix of the stage (SWIZZLE_128B: chunk ^= row % 8).
+template <int T_TILE>
+__device__ __forceinline__ uint32_t swz_off(int seg, int row, int chunk) {
+    return (uint32_t)(seg * T_TILE * 128 + row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+template <typename T, int DPLV>
+__device__ __forceinline__ void load_v_slice(const uint8_t* p, float* v);
+
+template <>
+__device__ __forceinline__ void load_v_slice<__nv_bfloat16, 2>(const uint8_t* p, float* v) {
+    uint32_t w = *reinterpret_cast<const uint32_t*>(p);
+    bf16x2_to_f32(w, v[0], v[1]);
+}
+template <>
+__device__ __forceinline__ void load_v_slice<__nv_bfloat16, 4>(const uint8_t* p, float* v) {
+    uint2 w = *reinterpret_cast<const uint2*>(p);
+    bf16x2_to_f32(w.x, v[0], v[1]);
+    bf16x2_to_f32(w.y, v[2], v[3]);
+}
+template <>
+__device__ __forceinline__ void load_v_slice<__nv_bfloat16, 8>(const uint8_t* p, float* v) {
+    uint4 w = *reinterpret_cast<const uint4*>(p);
+    bf16x8_to_f32(w, v);
+}
+template <>
+__device__ __forceinline__ void load_v_slice<float, 2>(const uint8_t* p, float* v) {
+    float2 w = *reinterpret_cast<const float2*>(p);
+    v[0] = w.x;
+    v[1] = w.y;
+}
+template <>
+__device__ __forceinline__ void load_v_slice<float, 4>(const uint8_t* p, float* v) {
+    float4 w = *reinterpret_cast<const float4*>(p);
+    v[0] = w.x;
+    v[1] = w.y;
+    v[2] = w.z;
+    v[3] = w.w;
+}
+
+template <typename T>
+__device__ __forceinline__ void load_chunk(const uint8_t* p, float* f);
+template <>
+__device__ __forceinline__ void load_chunk<__nv_bfloat16>(const uint8_t* p, float* f) {
+    bf16x8_to_f32(*reinterpret_cast<const uint4*>(p), f);
+}
+template <>
+__device__ __forceinline__ void load_chunk<float>(const uint8_t* p, float* f) {
+    float4 w = *reinterpret_cast<const float4*>(p);
+    f[0] = w.x;
+    f[1] = w.y;
+    f[2] = w.z;
+    f[3] = w.w;
+}
+
+// (segment, chunk) of the c-th chunk owned by lane li of a token's LPT lanes.
+// Chosen so that every 8-lane shared-memory phase of a 16-byte load touches 8
+// distinct bank groups under the 128-byte swizzle.
+template <int LPT, int NSEG>
+__device__ __forceinline__ void lane_chunk(int li, int c, int& seg, int& chunk) {
+    if constexpr (LPT <= 8) {
+        constexpr int PER_SEG = 8 / LPT;
+        seg = c / PER_SEG;
+        chunk = li * PER_SEG + c % PER_SEG;
+    } else {
+        seg = li / 8 + c * (LPT / 8);
+        chunk = li % 8;
+    }
+}
+
+template <typename T, int D, int RB>
+__global__ void __launch_bounds__(160, GqaCfg<T, D, RB>::MINB)
+    gqa_decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                      const GqaParams p) {
+    using C = GqaCfg<T, D, RB>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
+    uint8_t* stages = smem;
+    float* p_buf = reinterpret_cast<float*>(smem + C::NSTAGE * C::STAGE_BYTES);  // [4][TW][RB]
+    float* a_buf = p_buf + 4 * C::TW * RB;                                          // [4][RB]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::NSTAGE * C::STAGE_BYTES + C::P_BYTES);
+    __shared__ int s_abort;
+
+    const int split = blockIdx.x;
+    const int kvh = blockIdx.y / p.n_rb;
+    const int rb = blockIdx.y % p.n_rb;
+    const int b = blockIdx.z;
+    const int R = p.ratio * p.s_q;  // query rows of this group
+    const int row0 = rb * RB;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+    const int L = clamp_len(p.lens, b, p.Lmax, p.s_q, p.causal, p.status,
+                            threadIdx.x == 0 && split == 0 && kvh == 0 && rb == 0);
+    // keys needed by the rows of this block: causal row t sees L - s_q + t + 1
+    int rows_here = R - row0 < RB ? R - row0 : RB;
+    int need = L;
+    if (p.causal) {
+        int tmax = 0;
+        for (int r = 0; r < rows_here; ++r) {
+            int t = (row0 + r) % p.s_q;
+            tmax = t > tmax ? t : tmax;
+        }
+        need = L - p.s_q + tmax + 1;
+    }
+    const int kbeg = split * p.split_tokens;
+    if (kbeg >= need) return;  // no row of this block has keys in this split
+    const int kend = min(need, kbeg + p.split_tokens);
+    const int n_tiles = cdiv(kend - kbeg, C::T_TILE);
+    const int ybase = (b * p.h_kv + kvh) * p.Lmax;
+
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        for (int s = 0; s < C::NSTAGE; ++s) {
+            mbar_init(smem_u32(&bars[s]), 1);                 // full: producer arrival + tx bytes
+            mbar_init(smem_u32(&bars[C::NSTAGE + s]), 4);     // empty: one arrival per consumer warp
+        }
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    if (warp == 4) {
+        // ------------------------------ producer ------------------------------
+        if (lane == 0) {
+            prefetch_tensormap(&tmK);
+            prefetch_tensormap(&tmV);
+            int issued = 0;
+            for (int it = 0; it < n_tiles; ++it) {
+                const int s = it % C::NSTAGE;
+                if (it >= C::NSTAGE) {
+                    if (!mbar_wait(smem_u32(&bars[C::NSTAGE + s]), ((it / C::NSTAGE) - 1) & 1, p.status)) {
+                        s_abort = 1;
+                        break;
+                    }
+                }
+                if (*(volatile int*)&s_abort) break;
+                const uint32_t full = smem_u32(&bars[s]);
+                mbar_arrive_expect_tx(full, C::STAGE_BYTES);
+                const uint32_t kdst = smem_u32(stages + s * C::STAGE_BYTES);
+                const uint32_t vdst = kdst + C::MAT_BYTES;
+                const int y = ybase + kbeg + it * C::T_TILE;
+#pragma unroll
+                for (int sg = 0; sg < C::NSEG; ++sg) {
+                    tma_load_2d(kdst + sg * C::T_TILE * 128, &tmK, sg * C::SEG_ELEMS, y, full);
+                    tma_load_2d(vdst + sg * C::T_TILE * 128, &tmV, sg * C::SEG_ELEMS, y, full);
+                }
+                ++issued;
+            }
+            // drain: every issued copy must land before the CTA may exit
+            for (int it = issued - 1; it >= 0 && it >= issued - C::NSTAGE; --it)
+                mbar_wait(smem_u32(&bars[it % C::NSTAGE]), (it / C::NSTAGE) & 1, p.status);
+        }
+        return;
+    }
+
+    // -------------------------------- consumers --------------------------------
+    const int li = lane % C::LPT;           // lane within the token's lane group
+    const int tok_in_pass = lane / C::LPT;  // token of this lane within a pass
+    const int my_row = li / C::DUP;         // row this lane holds after the reduction
+    const int g_row = row0 + my_row;        // row index within the group
+    const bool row_ok = g_row < R;
+    const int my_t = row_ok ? g_row % p.s_q : 0;
+    const int my_last = p.causal ? (L - p.s_q + my_t) : (L - 1);  // last visible key of my row
+
+    // query slice of this lane, pre-scaled into the log2 domain
+    float qreg[RB][C::CPL * C::EPC];
+    {
+        const T* qbase = reinterpret_cast<const T*>(p.q) +
+                         ((size_t)(b * p.h_q + kvh * p.ratio) * p.s_q) * D;  // first row of the group
+#pragma unroll
+        for (int r = 0; r < RB; ++r) {
+            const bool ok = row0 + r < R;
+#pragma unroll
+            for (int c = 0; c < C::CPL; ++c) {
+                int seg, chunk;
+                lane_chunk<C::LPT, C::NSEG>(li, c, seg, chunk);
+                const int e0 = seg * C::SEG_ELEMS + chunk * C::EPC;
+#pragma unroll
+                for (int e = 0; e < C::EPC; ++e)
+                    qreg[r][c * C::EPC + e] =
+                        ok ? to_f32<T>(qbase[(size_t)(row0 + r) * D + e0 + e]) * p.scale_log2 : 0.f;
+            }
+        }
+    }
+
+    float m_run = -INFINITY, l_run = 0.f;
+    float o[RB][C::DPLV];
+#pragma unroll
+    for (int r = 0; r < RB; ++r)
+#pragma unroll
+        for (int d = 0; d < C::DPLV; ++d) o[r][d] = 0.f;
+
+    float* pw = p_buf + warp * C::TW * RB;
+    float* aw = a_buf + warp * RB;
+    bool aborted = false;
+
+    for (int it = 0; it < n_tiles; ++it) {
+        const int s = it % C::NSTAGE;
+        if (!mbar_wait(smem_u32(&bars[s]), (it / C::NSTAGE) & 1, p.status)) {
+            aborted = true;
+            s_abort = 1;
+            break;
+        }
+        const uint8_t* kt = stages + s * C::STAGE_BYTES;
+        const uint8_t* vt = kt + C::MAT_BYTES;
+        const int tbase = kbeg + it * C::T_TILE;
+
+        // ---- scores for this warp's TW tokens ----
+        float sc[C::NPASS];
+#pragma unroll
+        for (int ps = 0; ps < C::NPASS; ++ps) {
+            const int jt = warp * C::TW + ps * C::P + tok_in_pass;  // token row in the tile
+            float acc[RB];
+#pragma unroll
+            for (int r = 0; r < RB; ++r) acc[r] = 0.f;
+#pragma unroll
+            for (int c = 0; c < C::CPL; ++c) {
+                int seg, chunk;
+                lane_chunk<C::LPT, C::NSEG>(li, c, seg, chunk);
+                float kf[C::EPC];
+                load_chunk<T>(kt + swz_off<C::T_TILE>(seg, jt, chunk), kf);
+#pragma unroll
+                for (int r = 0; r < RB; ++r)
+#pragma unroll
+                    for (int e = 0; e < C::EPC; ++e) acc[r] = fmaf(qreg[r][c * C::EPC + e], kf[e], acc[r]);
+            }
+            // reduce-scatter over the LPT lanes of the token: lane li ends with row li / DUP
+            int nr = RB;
+#pragma unroll
+            for (int m = C::LPT / 2; m >= 1; m /= 2) {
+                if (nr > 1) {
+                    const bool upper = (li & m) != 0;
+                    const int half = nr / 2;
+#pragma unroll
+                    for (int k2 = 0; k2 < RB / 2; ++k2) {
+                        if (k2 < half) {
+                            float send = upper ? acc[k2] : acc[half + k2];
+                            float keep = upper ? acc[half + k2] : acc[k2];
+                            acc[k2] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+                        }
+                    }
+                    nr = half;
+                } else {
+                    acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], m);
+                }
+            }
+            const int kpos = tbase + jt;
+            const bool ok = row_ok && kpos < kend && kpos <= my_last;
+            sc[ps] = ok ? acc[0] : -INFINITY;
+        }
+
+        // ---- online softmax over this warp's tokens (per row) ----
+        float mx = sc[0];
+#pragma unroll
+        for (int ps = 1; ps < C::NPASS; ++ps) mx = fmaxf(mx, sc[ps]);
+#pragma unroll
+        for (int m = C::LPT; m < 32; m *= 2) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
+        const float m_new = fmaxf(m_run, mx);
+        const float m_ref = m_new == -INFINITY ? 0.f : m_new;
+        const float alpha = exp2f(m_run - m_ref);
+        float sum = 0.f;
+#pragma unroll
+        for (int ps = 0; ps < C::NPASS; ++ps) {
+            const float pv = exp2f(sc[ps] - m_ref);
+            sum += pv;
+            if (li % C::DUP == 0) pw[(ps * C::P + tok_in_pass) * RB + my_row] = pv;
+        }
+#pragma unroll
+        for (int m = C::LPT; m < 32; m *= 2) sum += __shfl_xor_sync(0xffffffffu, sum, m);
+        l_run = l_run * alpha + sum;
+        m_run = m_new;
+        if (tok_in_pass == 0 && li % C::DUP == 0) aw[my_row] = alpha;
+        __syncwarp();
+
+        // ---- O = alpha * O + P V over this warp's tokens ----
+        float al[RB];
+#pragma unroll
+        for (int r = 0; r < RB; ++r) al[r] = aw[r];
+#pragma unroll
+        for (int r = 0; r < RB; ++r)
+#pragma unroll
+            for (int d = 0; d < C::DPLV; ++d) o[r][d] *= al[r];
+        {
+            const int ob = lane * C::DPLV * C::E;  // byte offset of this lane's value slice in a row
+            const int vseg = ob / 128, vchunk = (ob % 128) / 16, vin = ob % 16;
+            int nvalid = kend - (tbase + warp * C::TW);
+            nvalid = nvalid < 0 ? 0 : (nvalid > C::TW ? C::TW : nvalid);
+#pragma unroll 4
+            for (int jj = 0; jj < nvalid; ++jj) {
+                const int jt = warp * C::TW + jj;
+                float vf[C::DPLV];
+                load_v_slice<T, C::DPLV>(vt + swz_off<C::T_TILE>(vseg, jt, vchunk) + vin, vf);
+                const float* pr = pw + jj * RB;
+#pragma unroll
+                for (int r = 0; r < RB; ++r) {
+                    const float pj = pr[r];
+#pragma unroll
+                    for (int d = 0; d < C::DPLV; ++d) o[r][d] = fmaf(pj, vf[d], o[r][d]);
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars[C::NSTAGE + s]));
+    }
+
+    // all consumer warps reach here; aborted CTAs stop without writing results
+    named_barrier(1, 128);
+    if (*(volatile int*)&s_abort || aborted) return;
+
+    // ---- merge the four warp states in shared memory (reusing the stage ring) ----
+    float* om = reinterpret_cast<float*>(stages);  // [4][RB][D]
+    float* mm = om + 4 * RB * D;                    // [4][RB]
+    float* lm = mm + 4 * RB;                        // [4][RB]
+#pragma unroll
+    for (int r = 0; r < RB; ++r)
+#pragma unroll
+        for (int d = 0; d < C::DPLV; ++d) om[(warp * RB + r) * D + lane * C::DPLV + d] = o[r][d];
+    if (tok_in_pass == 0 && li % C::DUP == 0) {
+        mm[warp * RB + my_row] = m_run;
+        lm[warp * RB + my_row] = l_run;
+    }
+    named_barrier(1, 128);
+
+    for (int idx = threadIdx.x; idx < rows_here * D; idx += 128) {
+        const int r = idx / D, d = idx % D;
+        const int gr = row0 + r;
+        const int t = gr % p.s_q;
+        const int hq = kvh * p.ratio + gr / p.s_q;
+        const size_t orow = ((size_t)b * p.h_q + hq) * p.s_q + t;
+        const int n_t = p.causal ? (L - p.s_q + t + 1) : L;
+        const int nsp = cdiv(n_t, p.split_tokens);
+        if (kbeg >= n_t) continue;  // this row has no keys in this split
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) M = fmaxf(M, mm[w * RB + r]);
+        float lsum = 0.f, acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const float f = exp2f(mm[w * RB + r] - M);  // warps without keys: exp2(-inf) = 0
+            lsum += f * lm[w * RB + r];
+            acc += f * om[(w * RB + r) * D + d];
+        }
+        const float ov = acc / lsum;
+        const float lse2 = M + log2f(lsum);
+        if (nsp == 1) {
+            reinterpret_cast<T*>(p.out)[orow * D + d] = from_f32<T>(ov);
+            if (p.lse && d == 0) p.lse[orow] = lse2 * 0.69314718055994530942f;
+        } else {
+            p.part_o[(orow * p.nsplit_max + split) * D + d] = ov;
+            if (d == 0) p.part_lse[orow * p.nsplit_max + split] = lse2;
+        }
+    }
+}
+
+// Merge of split partials: with w_i = 2^(lse_i - max lse),
+// O = sum_i w_i O_i / sum_i w_i and lse = max lse + log2(sum_i w_i).
+// One warp per output row; rows that needed a single split were written
+// directly by the decode kernel and are skipped.
+template <typename T, int D>
+__global__ void __launch_bounds__(128) gqa_combine_kernel(const GqaParams p) {
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const size_t row = (size_t)blockIdx.x * 4 + warp;
+    const size_t nrows = (size_t)p.B * p.h_q * p.s_q;
+    if (row >= nrows) return;
+    const int t = (int)(row % p.s_q);
+    const int b = (int)(row / ((size_t)p.h_q * p.s_q));
+    const int L = clamp_len(p.lens, b, p.Lmax, p.s_q, p.causal, p.status, false);
+    const int n_t = p.causal ? (L - p.s_q + t + 1) : L;
+    const int nsp = cdiv(n_t, p.split_tokens);
+    if (nsp == 1) return;
+    const float* pl = p.part_lse + row * p.nsplit_max;
+    float M = -INFINITY;
+    for (int i = lane; i < nsp; i += 32) M = fmaxf(M, pl[i]);
+#pragma unroll
+    for (int m = 16; m >= 1; m /= 2) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, m));
+    constexpr int DPL = D / 32;
+    float acc[DPL];
+#pragma unroll
+    for (int d = 0; d < DPL; ++d) acc[d] = 0.f;
+    float wsum = 0.f;
+    const float* po = p.part_o + row * p.nsplit_max * D;
+    for (int i = 0; i < nsp; ++i) {
+        const float w = exp2f(pl[i] - M);
+        wsum += w;
+#pragma unroll
+        for (int d = 0; d < DPL; ++d) acc[d] = fmaf(w, po[(size_t)i * D + d * 32 + lane], acc[d]);
+    }
+    T* out = reinterpret_cast<T*>(p.out) + row * D;
+#pragma unroll
+    for (int d = 0; d < DPL; ++d) out[d * 32 + lane] = from_f32<T>(acc[d] / wsum);
+    if (p.lse && lane == 0) p.lse[row] = (M + log2f(wsum)) * 0.69314718055994530942f;
+}
+
+// ---- host-side dispatch -------------------------------------------------------
+template <typename T, int D, int RB>
+static cudaError_t launch_one(const CUtensorMap& tk, const CUtensorMap& tv, const GqaParams& p, int nsplit,
+                              cudaStream_t st) {
+    using C = GqaCfg<T, D, RB>;
+    auto kern = gqa_decode_kernel<T, D, RB>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    dim3 grid(nsplit, p.h_kv * p.n_rb, p.B);
+    TimedLaunch timer(st);
+    kern<<<grid, 160, C::SMEM, st>>>(tk, tv, p);
+    timer.stop();
+    e = cudaPeekAtLastError();
+    if (e != cudaSuccess) return e;
+    const size_t nrows = (size_t)p.B * p.h_q * p.s_q;
+    if (nsplit > 1) {
+        gqa_combine_kernel<T, D><<<(unsigned)((nrows + 3) / 4), 128, 0, st>>>(p);
+        e = cudaPeekAtLastError();
+    }
+    return e;
+}
+
+int gqa_tile_tokens(int dtype_bytes, int d, int rb) {
+#define LKA_TILE_CASE(T, DD, R) \
+    if (dtype_bytes == (int)sizeof(T) && d == DD && rb == R) return GqaCfg<T, DD, R>::T_TILE;
+    LKA_TILE_CASE(__nv_bfloat16, 64, 1) LKA_TILE_CASE(__nv_bfloat16, 64, 2) LKA_TILE_CASE(__nv_bfloat16, 64, 4)
+    LKA_TILE_CASE(__nv_bfloat16, 64, 8)
+    LKA_TILE_CASE(__nv_bfloat16, 128, 1) LKA_TILE_CASE(__nv_bfloat16, 128, 2) LKA_TILE_CASE(__nv_bfloat16, 128, 4)
+    LKA_TILE_CASE(__nv_bfloat16, 128, 8) LKA_TILE_CASE(__nv_bfloat16, 128, 16)
+    LKA_TILE_CASE(__nv_bfloat16, 256, 1) LKA_TILE_CASE(__nv_bfloat16, 256, 2) LKA_TILE_CASE(__nv_bfloat16, 256, 4)
+    LKA_TILE_CASE(__nv_bfloat16, 256, 8)
+    LKA_TILE_CASE(float, 64, 1) LKA_TILE_CASE(float, 64, 2) LKA_TILE_CASE(float, 64, 4) LKA_TILE_CASE(float, 64, 8)
+    LKA_TILE_CASE(float, 64, 16)
+    LKA_TILE_CASE(float, 128, 1) LKA_TILE_CASE(float, 128, 2) LKA_TILE_CASE(float, 128, 4)
+    LKA_TILE_CASE(float, 128, 8) LKA_TILE_CASE(float, 128, 16)
+#undef LKA_TILE_CASE
+    return 0;
+}
+
+cudaError_t gqa_decode_launch(const CUtensorMap& tk, const CUtensorMap& tv, const GqaParams& p, int dtype_bytes,
+                              int d, int rb, int nsplit, cudaStream_t st) {
+#define LKA_LAUNCH_CASE(T, DD, R) \
+    if (dtype_bytes == (int)sizeof(T) && d == DD && rb == R) return launch_one<T, DD, R>(tk, tv, p, nsplit, st);
+    LKA_LAUNCH_CASE(__nv_bfloat16, 64, 1) LKA_LAUNCH_CASE(__nv_bfloat16, 64, 2)
+    LKA_LAUNCH_CASE(__nv_bfloat16, 64, 4) LKA_LAUNCH_CASE(__nv_bfloat16, 64, 8)
+    LKA_LAUNCH_CASE(__nv_bfloat16, 128, 1) LKA_LAUNCH_CASE(__nv_bfloat16, 128, 2)
+    LKA_LAUNCH_CASE(__nv_bfloat16, 128, 4) LKA_LAUNCH_CASE(__nv_bfloat16, 128, 8)
+    LKA_LAUNCH_CASE(__nv_bfloat16, 128, 16)
+    LKA_LAUNCH_CASE(__nv_bfloat16, 256, 1) LKA_LAUNCH_CASE(__nv_bfloat16, 256, 2)
+    LKA_LAUNCH_CASE(__nv_bfloat16, 256, 4) LKA_LAUNCH_CASE(__nv_bfloat16, 256, 8)
+    LKA_LAUNCH_CASE(float, 64, 1) LKA_LAUNCH_CASE(float, 64, 2) LKA_LAUNCH_CASE(float, 64, 4)
+    LKA_LAUNCH_CASE(float, 64, 8) LKA_LAUNCH_CASE(float, 64, 16)
+    LKA_LAUNCH_CASE(float, 128, 1) LKA_LAUNCH_CASE(float, 128, 2) LKA_LAUNCH_CASE(float, 128, 4)
+    LKA_LAUNCH_CASE(float, 128, 8) LKA_LAUNCH_CASE(float, 128, 16)
+#undef LKA_LAUNCH_CASE
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace lka

@@ -1,0 +1,31 @@
+// gqa_decode.h -- launch interface of the split-KV GQA decode kernels.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace lka {
+
+struct GqaParams {
+    const void* q;          // [B, h_q, s_q, D]
+    void* out;              // [B, h_q, s_q, D]
+    float* lse;             // [B, h_q, s_q] natural log, or nullptr
+    const int32_t* lens;    // device [B]
+    float* part_o;          // [B*h_q*s_q][nsplit_max][D] fp32 partials
+    float* part_lse;        // [B*h_q*s_q][nsplit_max] log2-domain partial lse
+    uint32_t* status;       // workspace status word
+    int B, h_q, h_kv, s_q, Lmax, causal;
+    float scale_log2;       // scale * log2(e)
+    int split_tokens;       // keys per split (multiple of the tile)
+    int nsplit_max;         // ceil(Lmax / split_tokens)
+    int n_rb;               // row blocks per KV head
+    int ratio;              // h_q / h_kv
+};
+
+// Tokens per TMA tile of the kernel instance (0 if the instance does not exist).
+int gqa_tile_tokens(int dtype_bytes, int d, int rb);
+// Launches the decode kernel (grid nsplit x h_kv*n_rb x B) and, when nsplit > 1, the merge.
+cudaError_t gqa_decode_launch(const CUtensorMap& tk, const CUtensorMap& tv, const GqaParams& p, int dtype_bytes,
+                              int d, int rb, int nsplit, cudaStream_t st);
+
+}  // namespace lka

@@ -125,6 +125,9 @@ def gta_inputs(seed, B, G, H, d_qk, d_v, s_q, L_lo, L_hi, Lmax=None, dtype=torch
 WORKLOADS = {
     "gqa_decode_llama8b": dict(kind="gqa", seed=2, B=64, h_q=32, h_kv=8, d=128, s_q=1, L_lo=1024, L_hi=8192,
                                causal=True),
+    # the same layer with a quarter of the batch: the small case for full ncu captures (K/V still > L2)
+    "gqa_decode_llama8b_b16": dict(kind="gqa", seed=2, B=16, h_q=32, h_kv=8, d=128, s_q=1, L_lo=1024, L_hi=8192,
+                                   causal=True),
     "gta_prefill_4k": dict(kind="gta", seed=3, B=8, G=3, H=12, d_qk=64, d_v=64, s_q=4096, L_lo=4096,
                            L_hi=4096, causal=True),
     "latent_decode_4k_sq1": dict(kind="latent", seed=4, B=64, h_q=128, g=8, d_h=128, r_kv=512, d_r=64, s_q=1,

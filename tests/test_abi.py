@@ -1,0 +1,83 @@
+"""The C-ABI library: it loads without a GPU, exports every symbol include/lka.h declares, and the
+binding's ctypes signatures match the header's parameter lists (CPU only, no compute calls)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import latent_kv_attention_b200 as lka
+from latent_kv_attention_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lka.h")
+
+
+def declarations():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    decls = {}
+    for m in re.finditer(r"LKA_API\s+([\w\s\*]+?)\b(\w+)\s*\(([^;]*?)\)\s*;", text, flags=re.S):
+        ret, name, params = m.group(1).strip(), m.group(2), m.group(3).strip()
+        n = 0 if params in ("", "void") else params.count(",") + 1
+        decls[name] = (ret, n)
+    return decls
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return lka.library()
+
+
+def test_header_declares_the_four_entry_points():
+    d = declarations()
+    for name in ("gqa_attn", "latent_absorbed_attn", "latent_expand_gqa_attn", "gta_shared_score_attn",
+                 "latent_expand_cache"):
+        assert name in d
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declarations():
+        assert hasattr(lib, name), f"liblka.so does not export {name}"
+
+
+def test_binding_signatures_match_header(lib):
+    d = declarations()
+    assert set(d) == set(lka.SIGNATURES)
+    for name, (ret, n) in d.items():
+        assert len(lka.SIGNATURES[name][1]) == n, f"{name}: header has {n} parameters"
+
+
+def test_status_strings(lib):
+    for code, name in lka.STATUS_NAMES.items():
+        assert lka.status_string(code) == name
+    assert lka.status_string(99) == "LKA_ERR_UNKNOWN"
+
+
+def test_host_validation_without_gpu(lib):
+    # argument errors are caught on the host before anything is enqueued
+    P = ctypes.c_void_p
+    rc = lib.gqa_attn(P(16), P(16), P(16), P(16), P(16), None, 1, 6, 4, 1, 128, 64, 1, 1.0, 0, P(16), 1 << 20, None)
+    assert rc == 1  # h_q % h_kv != 0
+    rc = lib.gqa_attn(P(16), P(16), P(16), P(16), P(16), None, 1, 8, 2, 1, 96, 64, 1, 1.0, 0, P(16), 1 << 20, None)
+    assert rc == 2  # unsupported head dim
+    rc = lib.gqa_attn(P(16), P(16), P(16), P(16), P(16), None, 1, 8, 2, 1, 128, 64, 1, 1.0, 0, None, 0, None)
+    assert rc == 3  # no workspace
+    rc = lib.gqa_attn(P(18), P(16), P(16), P(16), P(16), None, 1, 8, 2, 1, 128, 64, 1, 1.0, 0, P(16), 1 << 20, None)
+    assert rc == 1  # misaligned q
+    rc = lib.gqa_attn(None, None, None, None, None, None, 0, 8, 2, 1, 128, 64, 1, 1.0, 0, None, 0, None)
+    assert rc == 0  # empty batch is a no-op
+
+
+def test_workspace_sizes(lib):
+    small = lib.gqa_attn_workspace_size(1, 8, 2, 1, 64, 17)
+    assert small >= 256
+    big = lib.gqa_attn_workspace_size(64, 32, 8, 1, 128, 8192)
+    assert big > small
+    assert lib.gqa_attn_workspace_size(1, 6, 4, 1, 64, 17) == 0  # invalid grouping
+
+
+def test_split_knob_roundtrip(lib):
+    prev = lka.set_split_tokens(512)
+    assert lka.set_split_tokens(prev) == 512
