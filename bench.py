@@ -106,6 +106,15 @@ class ClockSampler:
         except (OSError, FileNotFoundError):
             self.proc = None
 
+    def wait_first_sample(self, timeout_s=5.0):
+        """Blocks until nvidia-smi has written a sample (so that samples cover what follows)."""
+        t0 = time.time()
+        while self.proc is not None and time.time() - t0 < timeout_s:
+            self.fh.flush()
+            if os.path.getsize(self.path) > 0:
+                return
+            time.sleep(0.05)
+
     def stop(self):
         if self.proc is None:
             return None
@@ -231,10 +240,18 @@ def run_lka(args, rank, world, device):
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     clocks = ClockSampler(device.index if device.index is not None else 0)
+    clocks.start()
+    clocks.wait_first_sample()
+    # keep the GPU under this load for ~1 s before the timed region so that the clock samples
+    # (every 200 ms) describe the state the timed steps run in; the sampler runs through both
+    t_soak = time.time()
+    while time.time() - t_soak < 1.0:
+        for _ in range(20):
+            wl.step()
+        torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    clocks.start()
     lka.kernel_timing(True)
     for s in range(args.steps):
         flush.zero_()  # L2 flush, outside the events
