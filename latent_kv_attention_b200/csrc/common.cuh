@@ -93,7 +93,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (globaltimer() - t0 > limit_ns) {
-            atomicOr(status, kDevTimeout);
+            if (status) atomicOr(status, kDevTimeout);
             return false;
         }
     }

@@ -1,0 +1,216 @@
+// latent_api.cu -- C ABI of the GQLA latent paths: latent_absorbed_attn (MQA-
+// absorbed attention over the latent cache) and latent_expand_cache (the
+// one-time conversion to the per-group cache).  Validation, workspace carving,
+// TMA descriptors and the launch sequence
+//   absorb GEMM (q~ = W^UK^T q^C) -> latent attention (+ split merge) -> up-projection GEMM (W^UV o~).
+#include <math.h>
+
+#include "common.cuh"
+#include "host_util.h"
+#include "latent.h"
+
+namespace lka {
+
+struct LatentPlan {
+    int split_tokens, nsplit;
+    size_t off_qt, off_olat, off_plse, off_po, ws_bytes;
+};
+
+static lka_status_t latent_plan(int B, int h_q, int g, int s_q, int d_h, int r_kv, int d_r, int Lmax,
+                                LatentPlan* pl) {
+    if (B < 0 || h_q < 1 || g < 1 || s_q < 1 || d_h < 1 || r_kv < 1 || d_r < 0 || Lmax < 1) return LKA_ERR_INVALID_ARG;
+    if (h_q % g) return LKA_ERR_INVALID_ARG;
+    // the kernels are specialised to the GQLA/MLA shape (h_q, d_h, r_kv, d_h^R) = (128, 128, 512, 64)
+    if (h_q != 128 || d_h != 128 || r_kv != 512 || d_r != 64) return LKA_ERR_UNSUPPORTED;
+    const int HPG = h_q / g;
+    if (HPG < 16 || 128 % (HPG * s_q) != 0) return LKA_ERR_UNSUPPORTED;
+    if ((long long)B * Lmax >= (1ll << 31) || B > 65535) return LKA_ERR_UNSUPPORTED;
+    const int NT = latent_tile_tokens();
+    int st = split_tokens_knob();
+    if (st <= 0) {
+        // one CTA pair per (sequence, query token) already fills the GPU for the decode batches of
+        // interest; split the keys only when there are fewer pairs than SM pairs
+        const long long units = (long long)(B > 0 ? B : 1) * s_q;
+        const long long pairs = sm_count() / 2;
+        long long nsp = units >= pairs ? 1 : (pairs + units - 1) / units;
+        st = (int)((Lmax + nsp - 1) / nsp);
+        if (st < 8 * NT) st = 8 * NT;
+    }
+    st = cdiv(st, NT) * NT;
+    pl->split_tokens = st;
+    pl->nsplit = cdiv(Lmax, st);
+    WsCarve c;
+    const size_t rows = (size_t)B * s_q * h_q;
+    pl->off_qt = c.take(rows * r_kv * 2);
+    pl->off_olat = c.take(rows * r_kv * 2);
+    if (pl->nsplit > 1) {
+        pl->off_plse = c.take(rows * pl->nsplit * 4);
+        pl->off_po = c.take(rows * pl->nsplit * (size_t)r_kv * 4);
+    } else {
+        pl->off_plse = pl->off_po = 0;
+    }
+    pl->ws_bytes = c.off;
+    return LKA_OK;
+}
+
+static lka_status_t st_of(cudaError_t e) { return e == cudaSuccess ? LKA_OK : LKA_ERR_CUDA; }
+
+}  // namespace lka
+
+using namespace lka;
+
+extern "C" {
+
+size_t latent_absorbed_attn_workspace_size(int B, int h_q, int g, int s_q, int d_h, int r_kv, int d_r, int Lmax) {
+    LatentPlan pl;
+    return latent_plan(B, h_q, g, s_q, d_h, r_kv, d_r, Lmax, &pl) == LKA_OK ? pl.ws_bytes : 0;
+}
+
+lka_status_t latent_absorbed_attn(const void* q_c, const void* q_r, const void* w_uk, const void* w_uv,
+                                  const void* latent, const int32_t* cache_lens, void* out, float* lse, int B, int h_q,
+                                  int g, int s_q, int d_h, int r_kv, int d_r, int Lmax, int causal, float scale,
+                                  lka_dtype_t dtype, void* ws, size_t ws_bytes, void* stream) {
+    if (dtype != LKA_BF16) return LKA_ERR_UNSUPPORTED;
+    LatentPlan pl;
+    lka_status_t s = latent_plan(B, h_q, g, s_q, d_h, r_kv, d_r, Lmax, &pl);
+    if (s != LKA_OK) return s;
+    if (B == 0) return LKA_OK;
+    const void* ptrs[] = {q_c, q_r, w_uk, w_uv, latent, cache_lens, out};
+    for (const void* ptr : ptrs)
+        if (!ptr || !aligned16(ptr)) return LKA_ERR_INVALID_ARG;
+    if (!isfinite(scale)) return LKA_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < pl.ws_bytes) return LKA_ERR_WORKSPACE;
+    if (!aligned16(ws)) return LKA_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    uint32_t* status = reinterpret_cast<uint32_t*>(w);
+    const int HPG = h_q / g;
+    const int slab = HPG * s_q;
+    const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    __nv_bfloat16* qt = reinterpret_cast<__nv_bfloat16*>(w + pl.off_qt);
+    __nv_bfloat16* olat = reinterpret_cast<__nv_bfloat16*>(w + pl.off_olat);
+
+    // 1) absorption q~ = W^UK_gamma^T q^C
+    CUtensorMap tm_qc, tm_wuk;
+    {
+        const uint64_t dims[3] = {(uint64_t)d_h, (uint64_t)h_q * s_q, (uint64_t)B};
+        const uint64_t str[2] = {(uint64_t)d_h * 2, (uint64_t)h_q * s_q * d_h * 2};
+        const uint32_t box[3] = {64, (uint32_t)slab, (uint32_t)(128 / slab)};
+        if (!make_tmap_nd(&tm_qc, BF, q_c, 3, dims, str, box)) return LKA_ERR_CUDA;
+        if (!make_tmap_2d(&tm_wuk, BF, w_uk, r_kv, (uint64_t)g * d_h, (uint64_t)r_kv * 2, 64, 64)) return LKA_ERR_CUDA;
+    }
+    GemmParams ga{};
+    ga.out = qt;
+    ga.status = status;
+    ga.K = d_h;
+    ga.N = r_kv;
+    ga.B = B;
+    ga.HPG = HPG;
+    ga.s_q = s_q;
+    ga.h_q = h_q;
+    ga.g = g;
+    ga.Lmax = Lmax;
+    if ((s = st_of(gemm_absorb(tm_qc, tm_wuk, ga, st))) != LKA_OK) return s;
+
+    // 2) attention of all heads over the latent cache (+ merge of key splits)
+    CUtensorMap tm_qt, tm_qr, tm_lat;
+    {
+        if (!make_tmap_2d(&tm_qt, BF, qt, r_kv, (uint64_t)B * s_q * h_q, (uint64_t)r_kv * 2, 64, 128)) return LKA_ERR_CUDA;
+        const uint64_t dims[3] = {(uint64_t)d_r, (uint64_t)s_q, (uint64_t)B * h_q};
+        const uint64_t str[2] = {(uint64_t)d_r * 2, (uint64_t)s_q * d_r * 2};
+        const uint32_t box[3] = {64, 1, 128};
+        if (!make_tmap_nd(&tm_qr, BF, q_r, 3, dims, str, box)) return LKA_ERR_CUDA;
+        if (!make_tmap_2d(&tm_lat, BF, latent, r_kv + d_r, (uint64_t)B * Lmax, (uint64_t)(r_kv + d_r) * 2, 64,
+                          latent_tile_tokens()))
+            return LKA_ERR_CUDA;
+    }
+    LatentParams lp{};
+    lp.lens = cache_lens;
+    lp.o_lat = olat;
+    lp.lse = lse;
+    lp.part_o = pl.nsplit > 1 ? reinterpret_cast<float*>(w + pl.off_po) : nullptr;
+    lp.part_lse = pl.nsplit > 1 ? reinterpret_cast<float*>(w + pl.off_plse) : nullptr;
+    lp.status = status;
+    lp.B = B;
+    lp.h_q = h_q;
+    lp.g = g;
+    lp.s_q = s_q;
+    lp.Lmax = Lmax;
+    lp.causal = causal ? 1 : 0;
+    lp.scale_log2 = scale * 1.4426950408889634f;
+    lp.split_tokens = pl.split_tokens;
+    lp.nsplit = pl.nsplit;
+    if ((s = st_of(latent_attn_launch(tm_qt, tm_qr, tm_lat, lp, st))) != LKA_OK) return s;
+
+    // 3) up-projection out = W^UV_gamma o~
+    CUtensorMap tm_ol, tm_wuv;
+    const int M_rows = B * slab;
+    if (!make_tmap_2d(&tm_ol, BF, olat, r_kv, (uint64_t)g * M_rows, (uint64_t)r_kv * 2, 64, 128) ||
+        !make_tmap_2d(&tm_wuv, BF, w_uv, r_kv, (uint64_t)g * d_h, (uint64_t)r_kv * 2, 64, 128))
+        return LKA_ERR_CUDA;
+    GemmParams gu = ga;
+    gu.out = out;
+    gu.M_rows = M_rows;
+    gu.K = r_kv;
+    gu.N = d_h;
+    return st_of(gemm_upproj(tm_ol, tm_wuv, gu, st));
+}
+
+}  // extern "C"
+
+namespace lka {
+// kr[b, j, :] = latent[b, j, r_kv : r_kv + d_r]  (16-byte pieces)
+__global__ void copy_rope_key_kernel(const uint8_t* latent, uint8_t* kr, long long n_tokens, int row_bytes,
+                                     int off_bytes, int kr_bytes) {
+    const int per = kr_bytes / 16;
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n_tokens * per) return;
+    const long long tok = i / per;
+    const int c = (int)(i % per);
+    *reinterpret_cast<uint4*>(kr + tok * kr_bytes + c * 16) =
+        *reinterpret_cast<const uint4*>(latent + tok * row_bytes + off_bytes + c * 16);
+}
+}  // namespace lka
+
+extern "C" lka_status_t latent_expand_cache(const void* latent, const void* w_uk, const void* w_uv, int B, int Lmax,
+                                            int g, int d_h, int r_kv, int d_r, void* kc, void* vc, void* kr,
+                                            lka_dtype_t dtype, void* stream) {
+    if (dtype != LKA_BF16) return LKA_ERR_UNSUPPORTED;
+    if (B < 0 || Lmax < 1 || g < 1 || d_h < 1 || r_kv < 1 || d_r < 0) return LKA_ERR_INVALID_ARG;
+    if (d_h % 128 || r_kv % 64 || d_r % 8 || ((r_kv + d_r) * 2) % 16) return LKA_ERR_UNSUPPORTED;
+    if ((long long)B * Lmax >= (1ll << 31)) return LKA_ERR_UNSUPPORTED;
+    if (B == 0) return LKA_OK;
+    const void* ptrs[] = {latent, w_uk, w_uv, kc, vc};
+    for (const void* p : ptrs)
+        if (!p || !aligned16(p)) return LKA_ERR_INVALID_ARG;
+    if (d_r > 0 && (!kr || !aligned16(kr))) return LKA_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    CUtensorMap ta, tk, tv;
+    if (!make_tmap_2d(&ta, BF, latent, r_kv + d_r, (uint64_t)B * Lmax, (uint64_t)(r_kv + d_r) * 2, 64, 128) ||
+        !make_tmap_2d(&tk, BF, w_uk, r_kv, (uint64_t)g * d_h, (uint64_t)r_kv * 2, 64, 128) ||
+        !make_tmap_2d(&tv, BF, w_uv, r_kv, (uint64_t)g * d_h, (uint64_t)r_kv * 2, 64, 128))
+        return LKA_ERR_CUDA;
+    GemmParams p{};
+    p.status = nullptr;
+    p.K = r_kv;
+    p.N = d_h;
+    p.B = B;
+    p.g = g;
+    p.Lmax = Lmax;
+    p.tiles_per_b = cdiv(Lmax, 128);
+    // the helper takes no workspace, so it has no status word: a timed-out wait only ends the kernel
+    p.status = nullptr;
+    p.out = kc;
+    if (gemm_expand(ta, tk, p, st) != cudaSuccess) return LKA_ERR_CUDA;
+    p.out = vc;
+    if (gemm_expand(ta, tv, p, st) != cudaSuccess) return LKA_ERR_CUDA;
+    if (d_r > 0) {
+        const long long n = (long long)B * Lmax * (d_r * 2 / 16);
+        copy_rope_key_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
+            static_cast<const uint8_t*>(latent), static_cast<uint8_t*>(kr), (long long)B * Lmax, (r_kv + d_r) * 2,
+            r_kv * 2, d_r * 2);
+        if (cudaPeekAtLastError() != cudaSuccess) return LKA_ERR_CUDA;
+    }
+    return LKA_OK;
+}

@@ -1,0 +1,460 @@
+// latent_attn.cu -- MQA-absorbed attention over the GQLA/MLA latent cache on
+// the 5th-generation tensor cores, and the merge of its split partials.
+//
+// Operation ("GQLA: Group-Query Latent Attention ..." section 1, section 3.1
+// eq. (1) and Figure 2(b)): after W^UK is folded into the query, all h_q = 128
+// heads attend to the cached latent itself.  The key of token j is the
+// 576-value row [c_j ; k^R_j] (r_kv = 512 latent values and the shared d_h^R =
+// 64 RoPE key); the value is its first 512 values.  For query row (head) h:
+//     s_j = scale * <[q~_h ; q^R_h], [c_j ; k^R_j]>,  o~_h = sum_j softmax(s)_j c_j.
+// The 128 x 576 x tokens score contraction and the 128 x tokens x 512 value
+// contraction are dense, so both run as tcgen05 MMAs with M = 128 heads.
+//
+// Tensor memory holds 512 fp32 columns per SM and the output alone needs
+// 128 x 512, so each work item is processed by a CLUSTER OF TWO CTAs that split
+// the latent dimensions: rank 0 loads latent values [0, 256), rank 1 loads
+// [256, 512) and the RoPE key [512, 576).  Each rank multiplies the query slice
+// it holds with the tile slice it loaded (a split-K partial of the scores),
+// the two partials are exchanged through distributed shared memory (st.async
+// with mbarrier transaction counts) and summed identically on both sides, so
+// both run the same online softmax and each accumulates the 256 output columns
+// of the latent values it loaded.  No tile byte is loaded twice and no score
+// is computed twice.
+//
+// Per CTA: warp 4 streams the query slice once and 32-token tiles of the
+// latent through a 4-stage TMA ring; warp 5 issues the MMAs (S = Q K^T into a
+// double-buffered TMEM score tile; O += P V with P read from TMEM); warps 0-3
+// own one head row each per thread: exchange, mask, online softmax with lazy
+// rescaling (the running maximum is only moved when it grows by more than 2^8,
+// which leaves the final O / l exact), P written back to TMEM as bf16.
+#include "common.cuh"
+#include "host_util.h"
+#include "latent.h"
+#include "tc.cuh"
+
+namespace lka {
+
+namespace lat {
+constexpr int NT = 32;          // tokens per tile
+constexpr int NST = 4;          // TMA ring depth
+constexpr int KB_MAX = 5;       // 64-wide K blocks per rank (rank 1: 4 latent + 1 RoPE)
+constexpr int Q_BYTES = KB_MAX * 128 * 128;
+constexpr int BOX = NT * 128;   // one 64-value box of NT tokens
+constexpr int STAGE = KB_MAX * BOX;
+constexpr int XROW = NT * 4;    // bytes of one exchanged score row
+constexpr int XBUF = 128 * XROW;
+constexpr int OFF_Q = 0;
+constexpr int OFF_KV = OFF_Q + Q_BYTES;
+constexpr int OFF_X = OFF_KV + NST * STAGE;
+constexpr int OFF_BAR = OFF_X + 2 * XBUF;
+constexpr int SMEM = 1024 + OFF_BAR + 256;
+// tensor memory columns
+constexpr uint32_t T_O = 0;          // 256 fp32 columns: this rank's half of the output
+constexpr uint32_t T_S = 256;        // 2 x NT fp32 score partials
+constexpr uint32_t T_P = 256 + 2 * NT;  // 2 x NT/2 columns of bf16 pairs
+constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 domain
+}  // namespace lat
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t mapa_peer(uint32_t saddr, uint32_t peer) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(peer));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void st_async_v4(uint32_t raddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
+                                            uint32_t rbar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                     raddr),
+                 "r"(a), "r"(b), "r"(c), "r"(d), "r"(rbar)
+                 : "memory");
+}
+__device__ __forceinline__ void remote_arrive(uint32_t rbar) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(rbar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// bounded wait with cluster-scope acquire (for data written by the peer CTA)
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, uint32_t* status) {
+    for (int i = 0; i < 32; ++i)
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    while (true) {
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if (globaltimer() - t0 > kWaitLimitNs) {
+            if (status) atomicOr(status, kDevTimeout);
+            return false;
+        }
+    }
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+    latent_attn_kernel(const __grid_constant__ CUtensorMap tm_qt, const __grid_constant__ CUtensorMap tm_qr,
+                       const __grid_constant__ CUtensorMap tm_lat, const LatentParams p) {
+    using namespace lat;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+    uint64_t* q_full = bars + 0;
+    uint64_t* kv_full = bars + 1;
+    uint64_t* kv_empty = bars + 1 + NST;
+    uint64_t* s_ready = bars + 1 + 2 * NST;
+    uint64_t* p_ready = s_ready + 2;
+    uint64_t* o_ready = p_ready + 2;
+    uint64_t* xfull = o_ready + 1;
+    uint64_t* xempty = xfull + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xempty + 2);
+    __shared__ int s_abort;
+
+    const uint32_t rank = cluster_rank();
+    const uint32_t peer = rank ^ 1u;
+    const int nkb = rank == 0 ? 4 : 5;
+    const int pair = blockIdx.x >> 1;
+    const int t = pair % p.s_q;
+    const int split = pair / p.s_q;
+    const int b = blockIdx.y;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+    const int L = clamp_len(p.lens, b, p.Lmax, p.s_q, p.causal, p.status,
+                            threadIdx.x == 0 && rank == 0 && pair == 0);
+    const int last_key = p.causal ? L - p.s_q + t : L - 1;  // last key query t may see
+    const int kbeg = split * p.split_tokens;
+    const int kend = min(last_key + 1, kbeg + p.split_tokens);
+    const int n_tiles = kend > kbeg ? cdiv(kend - kbeg, NT) : 0;
+
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        mbar_init(smem_u32(q_full), 1);
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(smem_u32(&kv_full[s]), 1);
+            mbar_init(smem_u32(&kv_empty[s]), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_u32(&s_ready[i]), 1);
+            mbar_init(smem_u32(&p_ready[i]), 4);
+            mbar_init(smem_u32(&xfull[i]), 1);
+            mbar_init(smem_u32(&xempty[i]), 1);
+        }
+        mbar_init(smem_u32(o_ready), 1);
+        fence_barrier_init();
+        // the first two exchange buffers are open for the peer's partial scores
+        mbar_arrive_expect_tx(smem_u32(&xfull[0]), XBUF);
+        mbar_arrive_expect_tx(smem_u32(&xfull[1]), XBUF);
+    }
+    if (warp == 5) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    cluster_sync();  // barriers of both CTAs initialised before any remote traffic
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (n_tiles > 0 && warp == 4) {
+        // ------------------------------- TMA producer -------------------------------
+        if (lane == 0) {
+            prefetch_tensormap(&tm_qt);
+            prefetch_tensormap(&tm_lat);
+            const uint32_t qb = smem_u32(q_full);
+            mbar_arrive_expect_tx(qb, nkb * 128 * 128);
+            const int qrow = (b * p.s_q + t) * 128;
+            for (int kb = 0; kb < 4; ++kb)
+                tma_load_2d(smem_u32(smem + OFF_Q + kb * 16384), &tm_qt, (int)(rank * 4 + kb) * 64, qrow, qb);
+            if (rank == 1) tma_load_3d(smem_u32(smem + OFF_Q + 4 * 16384), &tm_qr, 0, t, b * 128, qb);
+            int issued = 0;
+            for (int i = 0; i < n_tiles; ++i) {
+                const int s = i % NST;
+                if (i >= NST && !mbar_wait(smem_u32(&kv_empty[s]), ((i / NST) - 1) & 1, p.status)) {
+                    s_abort = 1;
+                    break;
+                }
+                if (*(volatile int*)&s_abort) break;
+                const uint32_t fb = smem_u32(&kv_full[s]);
+                mbar_arrive_expect_tx(fb, nkb * BOX);
+                const uint32_t dst = smem_u32(smem + OFF_KV + s * STAGE);
+                const int y = b * p.Lmax + kbeg + i * NT;
+                for (int kb = 0; kb < nkb; ++kb) tma_load_2d(dst + kb * BOX, &tm_lat, (int)rank * 256 + kb * 64, y, fb);
+                ++issued;
+            }
+            for (int i = issued - 1; i >= 0 && i >= issued - NST; --i)
+                mbar_wait(smem_u32(&kv_full[i % NST]), (i / NST) & 1, p.status);
+            mbar_wait(qb, 0, p.status);
+        }
+    } else if (n_tiles > 0 && warp == 5) {
+        // ------------------------------- MMA issuer -------------------------------
+        constexpr uint32_t idesc_qk = idesc_bf16_f32(128, NT, false, false);
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
+        bool ok = mbar_wait(smem_u32(q_full), 0, p.status);
+        auto issue_qk = [&](int j) -> bool {
+            const int s = j % NST;
+            if (!mbar_wait(smem_u32(&kv_full[s]), (j / NST) & 1, p.status)) return false;
+            uint8_t* st = smem + OFF_KV + s * STAGE;
+            const int nvalid = min(NT, kend - (kbeg + j * NT));
+            if (nvalid < NT) {
+                // rows past the last visible key may hold anything (even NaN): zero them so
+                // that P = 0 times V contributes exactly 0
+                const int rows = NT - nvalid;
+                for (int idx = lane; idx < nkb * rows * 8; idx += 32) {
+                    const int kb = idx / (rows * 8), rr = (idx / 8) % rows, c = idx % 8;
+                    *reinterpret_cast<uint4*>(st + kb * BOX + (nvalid + rr) * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+            }
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t qa = smem_u32(smem + OFF_Q);
+                const uint32_t kva = smem_u32(st);
+                for (int kb = 0; kb < nkb; ++kb)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        umma_ss(tmem + T_S + (j & 1) * NT, smem_desc_sw128(qa + kb * 16384 + k * 32, 16, 1024),
+                                smem_desc_sw128(kva + kb * BOX + k * 32, 16, 1024), idesc_qk, (kb | k) != 0);
+                umma_commit(smem_u32(&s_ready[j & 1]));
+            }
+            __syncwarp();
+            return true;
+        };
+        if (ok) ok = issue_qk(0);
+        for (int i = 0; ok && i < n_tiles; ++i) {
+            if (i + 1 < n_tiles && !issue_qk(i + 1)) break;
+            if (!mbar_wait(smem_u32(&p_ready[i & 1]), (i >> 1) & 1, p.status)) break;
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t va = smem_u32(smem + OFF_KV + (i % NST) * STAGE);
+#pragma unroll
+                for (int kk = 0; kk < NT / 16; ++kk)
+                    umma_ts(tmem + T_O, tmem + T_P + (i & 1) * (NT / 2) + kk * 8,
+                            smem_desc_sw128(va + kk * 2048, BOX, 1024), idesc_pv, (i | kk) != 0);
+                umma_commit(smem_u32(&kv_empty[i % NST]));
+                umma_commit(smem_u32(o_ready));
+            }
+            __syncwarp();
+        }
+    } else if (warp < 4) {
+        // ------------------------- softmax / exchange warps -------------------------
+        const int h = warp * 32 + lane;  // head row == TMEM lane
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const uint32_t xloc[2] = {smem_u32(smem + OFF_X), smem_u32(smem + OFF_X + XBUF)};
+        const uint32_t xrem[2] = {mapa_peer(xloc[0] + h * XROW, peer), mapa_peer(xloc[1] + h * XROW, peer)};
+        const uint32_t xfull_rem[2] = {mapa_peer(smem_u32(&xfull[0]), peer), mapa_peer(smem_u32(&xfull[1]), peer)};
+        const uint32_t xempty_rem[2] = {mapa_peer(smem_u32(&xempty[0]), peer),
+                                        mapa_peer(smem_u32(&xempty[1]), peer)};
+        const int sw = h & 7;
+        float m_ref = -INFINITY, l = 0.f;
+        bool ok = true;
+        // A failed (timed-out) wait clears `ok`; the loop then keeps its shape without waiting, so that
+        // every warp still reaches the named barrier below and the CTA pair can exit.
+        for (int i = 0; i < n_tiles; ++i) {
+            const int x = i & 1;
+            if (ok) ok = mbar_wait(smem_u32(&s_ready[x]), (i >> 1) & 1, p.status);
+            tc_fence_after();
+            uint32_t sr[NT];
+            tmem_ld16(tmem + lane_base + T_S + x * NT, sr);
+            tmem_ld16(tmem + lane_base + T_S + x * NT + 16, sr + 16);
+            tmem_ld_wait();
+            // ---- exchange the partial scores with the peer CTA ----
+            if (ok && i >= 2) ok = mbar_wait_cluster(smem_u32(&xempty[x]), ((i >> 1) - 1) & 1, p.status);
+#pragma unroll
+            for (int c = 0; c < NT / 4; ++c)
+                st_async_v4(xrem[x] + ((c ^ sw) << 4), sr[4 * c], sr[4 * c + 1], sr[4 * c + 2], sr[4 * c + 3],
+                            xfull_rem[x]);
+            if (ok) ok = mbar_wait_cluster(smem_u32(&xfull[x]), (i >> 1) & 1, p.status);
+            float s[NT];
+            const uint8_t* xr = smem + OFF_X + x * XBUF + h * XROW;
+#pragma unroll
+            for (int c = 0; c < NT / 4; ++c) {
+                const float4 v = *reinterpret_cast<const float4*>(xr + ((c ^ sw) << 4));
+                s[4 * c] = __uint_as_float(sr[4 * c]) + v.x;
+                s[4 * c + 1] = __uint_as_float(sr[4 * c + 1]) + v.y;
+                s[4 * c + 2] = __uint_as_float(sr[4 * c + 2]) + v.z;
+                s[4 * c + 3] = __uint_as_float(sr[4 * c + 3]) + v.w;
+            }
+            named_barrier(1, 128);  // every row has read exchange buffer x
+            if (threadIdx.x == 0 && i + 2 < n_tiles) {
+                mbar_arrive_expect_tx(smem_u32(&xfull[x]), XBUF);  // reopen it for tile i + 2 ...
+                remote_arrive(xempty_rem[x]);                      // ... and tell the peer
+            }
+            // ---- mask, online softmax ----
+            const int k0 = kbeg + i * NT;
+            float mx = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < NT; ++j) {
+                const int kp = k0 + j;
+                s[j] = (kp < kend) ? s[j] * p.scale_log2 : -INFINITY;
+                mx = fmaxf(mx, s[j]);
+            }
+            const float m_new = fmaxf(m_ref, mx);
+            bool resc = false;
+            float alpha = 1.f;
+            float m_use = m_ref;
+            if (m_ref == -INFINITY) {
+                m_use = m_new;
+            } else if (m_new > m_ref + RESCALE_THRESHOLD) {
+                resc = true;
+                alpha = exp2f(m_ref - m_new);
+                m_use = m_new;
+            }
+            float rs = 0.f;
+            uint32_t pk[NT / 2];
+#pragma unroll
+            for (int j = 0; j < NT; j += 2) {
+                const float p0 = m_use == -INFINITY ? 0.f : exp2f(s[j] - m_use);
+                const float p1 = m_use == -INFINITY ? 0.f : exp2f(s[j + 1] - m_use);
+                rs += p0 + p1;
+                pk[j / 2] = pack_bf16x2(p0, p1);
+            }
+            l = (resc ? l * alpha : l) + rs;
+            m_ref = m_use;
+            tmem_st16(tmem + lane_base + T_P + x * (NT / 2), pk);
+            tmem_st_wait();
+            // ---- PV(i-1) must be complete before O is rescaled / P(i) consumed ----
+            if (ok && i >= 1) ok = mbar_wait(smem_u32(o_ready), (i - 1) & 1, p.status);
+            if (__any_sync(0xffffffffu, resc)) {
+                tc_fence_after();
+                for (int c0 = 0; c0 < 256; c0 += 16) {
+                    uint32_t o[16];
+                    tmem_ld16(tmem + lane_base + T_O + c0, o);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
+                    tmem_st16(tmem + lane_base + T_O + c0, o);
+                }
+                tmem_st_wait();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&p_ready[x]));
+        }
+        if (!ok) s_abort = 1;
+        // ---- epilogue: normalise this rank's 256 output columns ----
+        if (ok && n_tiles > 0 && mbar_wait(smem_u32(o_ready), (n_tiles - 1) & 1, p.status)) {
+            tc_fence_after();
+            const float inv_l = l > 0.f ? 1.f / l : 0.f;
+            const int HPG = p.h_q / p.g;
+            const int grp = h / HPG, hh = h % HPG;
+            const size_t prow = ((size_t)(b * p.s_q + t) * p.h_q + h);
+            __nv_bfloat16* orow =
+                p.o_lat + ((size_t)grp * p.B * HPG * p.s_q + (size_t)(b * HPG + hh) * p.s_q + t) * 512 + rank * 256;
+            float* prt = p.nsplit > 1 ? p.part_o + (prow * p.nsplit + split) * 512 + rank * 256 : nullptr;
+            for (int c0 = 0; c0 < 256; c0 += 16) {
+                uint32_t o[16];
+                tmem_ld16(tmem + lane_base + T_O + c0, o);
+                tmem_ld_wait();
+                if (prt) {
+                    float4* d = reinterpret_cast<float4*>(prt + c0);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        d[q] = make_float4(__uint_as_float(o[4 * q]) * inv_l, __uint_as_float(o[4 * q + 1]) * inv_l,
+                                           __uint_as_float(o[4 * q + 2]) * inv_l, __uint_as_float(o[4 * q + 3]) * inv_l);
+                } else {
+                    uint32_t pkk[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        pkk[q] = pack_bf16x2(__uint_as_float(o[2 * q]) * inv_l, __uint_as_float(o[2 * q + 1]) * inv_l);
+                    uint4* d = reinterpret_cast<uint4*>(orow + c0);
+                    d[0] = make_uint4(pkk[0], pkk[1], pkk[2], pkk[3]);
+                    d[1] = make_uint4(pkk[4], pkk[5], pkk[6], pkk[7]);
+                }
+            }
+            if (rank == 0) {
+                const float lse2 = l > 0.f ? m_ref + log2f(l) : -INFINITY;
+                if (p.nsplit > 1)
+                    p.part_lse[prow * p.nsplit + split] = lse2;
+                else if (p.lse)
+                    p.lse[((size_t)b * p.h_q + h) * p.s_q + t] = lse2 * 0.69314718055994530942f;
+            }
+        }
+    }
+    // both CTAs stay resident until the peer is done writing into their shared memory
+    tc_fence_before();
+    __syncwarp();
+    cluster_sync();
+    if (warp == 5) tmem_dealloc(tmem, 512);
+}
+
+// Merge of the split partials of the latent attention (same rule as the GQA
+// merge: weights 2^(lse_i - max lse)); writes o~ in the layout the
+// up-projection reads and the natural-log lse.  One warp per (b, t, head) row.
+__global__ void __launch_bounds__(128) latent_combine_kernel(const LatentParams p) {
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const size_t row = (size_t)blockIdx.x * 4 + warp;  // ((b*s_q + t)*h_q + h)
+    const size_t nrows = (size_t)p.B * p.s_q * p.h_q;
+    if (row >= nrows) return;
+    const int h = (int)(row % p.h_q);
+    const int t = (int)((row / p.h_q) % p.s_q);
+    const int b = (int)(row / ((size_t)p.h_q * p.s_q));
+    const int L = clamp_len(p.lens, b, p.Lmax, p.s_q, p.causal, p.status, false);
+    const int n_t = p.causal ? L - p.s_q + t + 1 : L;
+    const int nsp = cdiv(n_t, p.split_tokens);
+    const float* pl = p.part_lse + row * p.nsplit;
+    float M = -INFINITY;
+    for (int i = lane; i < nsp; i += 32) M = fmaxf(M, pl[i]);
+#pragma unroll
+    for (int m = 16; m >= 1; m /= 2) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, m));
+    float acc[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) acc[q] = 0.f;
+    float wsum = 0.f;
+    for (int i = 0; i < nsp; ++i) {
+        const float w = exp2f(pl[i] - M);
+        wsum += w;
+        const float4* src = reinterpret_cast<const float4*>(p.part_o + (row * p.nsplit + i) * 512);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float4 v = src[q * 32 + lane];
+            acc[4 * q] = fmaf(w, v.x, acc[4 * q]);
+            acc[4 * q + 1] = fmaf(w, v.y, acc[4 * q + 1]);
+            acc[4 * q + 2] = fmaf(w, v.z, acc[4 * q + 2]);
+            acc[4 * q + 3] = fmaf(w, v.w, acc[4 * q + 3]);
+        }
+    }
+    const float inv = 1.f / wsum;
+    const int HPG = p.h_q / p.g;
+    const int grp = h / HPG, hh = h % HPG;
+    __nv_bfloat16* orow = p.o_lat + ((size_t)grp * p.B * HPG * p.s_q + (size_t)(b * HPG + hh) * p.s_q + t) * 512;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint2 v;
+        v.x = pack_bf16x2(acc[4 * q] * inv, acc[4 * q + 1] * inv);
+        v.y = pack_bf16x2(acc[4 * q + 2] * inv, acc[4 * q + 3] * inv);
+        *reinterpret_cast<uint2*>(orow + (q * 32 + lane) * 4) = v;
+    }
+    if (p.lse && lane == 0) p.lse[((size_t)b * p.h_q + h) * p.s_q + t] = (M + log2f(wsum)) * 0.69314718055994530942f;
+}
+
+int latent_tile_tokens() { return lat::NT; }
+
+cudaError_t latent_attn_launch(const CUtensorMap& tm_qt, const CUtensorMap& tm_qr, const CUtensorMap& tm_lat,
+                               const LatentParams& p, cudaStream_t st) {
+    cudaError_t e = cudaFuncSetAttribute(latent_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, lat::SMEM);
+    if (e != cudaSuccess) return e;
+    dim3 grid(2 * p.s_q * p.nsplit, p.B);
+    {
+        TimedLaunch timer(st);
+        latent_attn_kernel<<<grid, 192, lat::SMEM, st>>>(tm_qt, tm_qr, tm_lat, p);
+        timer.stop();
+    }
+    e = cudaPeekAtLastError();
+    if (e != cudaSuccess || p.nsplit == 1) return e;
+    const size_t nrows = (size_t)p.B * p.s_q * p.h_q;
+    latent_combine_kernel<<<(unsigned)((nrows + 3) / 4), 128, 0, st>>>(p);
+    return cudaPeekAtLastError();
+}
+
+}  // namespace lka

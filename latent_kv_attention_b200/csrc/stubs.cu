@@ -4,12 +4,6 @@
 
 extern "C" {
 
-size_t latent_absorbed_attn_workspace_size(int, int, int, int, int, int, int, int) { return 0; }
-lka_status_t latent_absorbed_attn(const void*, const void*, const void*, const void*, const void*, const int32_t*,
-                                  void*, float*, int, int, int, int, int, int, int, int, int, float, lka_dtype_t,
-                                  void*, size_t, void*) {
-    return LKA_ERR_UNSUPPORTED;
-}
 size_t latent_expand_gqa_attn_workspace_size(int, int, int, int, int, int, int) { return 0; }
 lka_status_t latent_expand_gqa_attn(const void*, const void*, const void*, const void*, const void*,
                                     const int32_t*, void*, float*, int, int, int, int, int, int, int, int, float,
@@ -19,10 +13,6 @@ lka_status_t latent_expand_gqa_attn(const void*, const void*, const void*, const
 size_t gta_shared_score_attn_workspace_size(int, int, int, int, int, int, int) { return 0; }
 lka_status_t gta_shared_score_attn(const void*, const void*, const void*, const int32_t*, void*, float*, int, int,
                                    int, int, int, int, int, int, float, lka_dtype_t, void*, size_t, void*) {
-    return LKA_ERR_UNSUPPORTED;
-}
-lka_status_t latent_expand_cache(const void*, const void*, const void*, int, int, int, int, int, int, void*, void*,
-                                 void*, lka_dtype_t, void*) {
     return LKA_ERR_UNSUPPORTED;
 }
 
