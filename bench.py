@@ -11,6 +11,12 @@ decode kernel plus log-sum-exp merge.  Inputs are seeded synthetic tensors
 (synthetic.py) resident in HBM; their 2.1 GB exceed the 126 MB L2, and L2 is
 flushed between timed steps anyway.
 
+Unless --no-extras is given, the line also carries `other_paths`: the same
+measurement (step time, GB/s, TFLOP/s, tokens/s, roofline of the main kernel,
+end-to-end time) for the GQLA latent decode layer on the MQA-absorbed path
+(s_q = 1 and 2), on the per-group GQA path (s_q = 2), and for the GTA causal
+prefill.
+
 Prints ONE JSON line (rank 0).  `value` is the algorithmic HBM traffic of the
 step (every cache byte once, q read once, out written once) divided by the
 device time of a step, summed over ranks (weak scaling: every rank runs its own
@@ -146,114 +152,302 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- workloads
-class GqaDecode:
-    """One gqa_attn call over the Llama-3.1-8B-shaped decode batch."""
+def _pinned(t):
+    return t.cpu().pin_memory()
+
+
+def _nbytes(*ts):
+    return sum(t.numel() * t.element_size() for t in ts)
+
+
+class Workload:
+    """One attention-layer call over a synthetic batch (a bench `step`), with its algorithmic costs."""
+
+    kernel = ""
+    src = ()
+    bound = "hbm"
+    oracle_n = 8  # sequences in the oracle's bounded sample
+
+    def __init__(self, name, device, reference=False):
+        self.name = name
+        self.w = synthetic.WORKLOADS[name]
+        self.device = device
+        self.inp = synthetic.make(self.w, device=device)
+        self.lens = self.inp["cache_lens"].cpu().tolist()
+        self.setup_costs()
+        if reference:
+            return
+        import latent_kv_attention_b200 as lka
+
+        self.lka = lka
+        self.setup_device()
+
+    # e2e: per-step inputs come from pinned host buffers, the result goes back to one
+    def step_e2e(self):
+        for dst, src in self.h2d_pairs:
+            dst.copy_(src, non_blocking=True)
+        self.step()
+        self.out_host.copy_(self.out, non_blocking=True)
+
+    @property
+    def h2d(self):
+        return sum(_nbytes(src) for _, src in self.h2d_pairs)
+
+    @property
+    def d2h(self):
+        return _nbytes(self.out_host)
+
+
+class GqaDecode(Workload):
+    """gqa_attn over the Llama-3.1-8B-shaped decode batch: split-KV decode kernel + log-sum-exp merge."""
 
     kernel = "gqa_decode_kernel"
     src = ("latent_kv_attention_b200/csrc/gqa_decode.cu", "latent_kv_attention_b200/csrc/common.cuh")
 
-    def __init__(self, name, device, reference=False):
-        self.w = synthetic.WORKLOADS[name]
+    def setup_costs(self):
         w = self.w
-        self.name = name
-        self.inp = synthetic.make(w, device=device)
-        self.lens = self.inp["cache_lens"].cpu().tolist()
         self.bytes = costs.gqa_bytes(self.lens, w["h_q"], w["h_kv"], w["d"], w["s_q"])
         self.flops = costs.gqa_flops(self.lens, w["h_q"], w["d"], w["s_q"], w["causal"])
         self.tokens = w["B"] * w["s_q"]
-        if reference:
-            return  # the reference arm only runs the oracle
-        import latent_kv_attention_b200 as lka
 
-        self.lka = lka
-        self.out = torch.empty_like(self.inp["q"])
-        ws = lka.library().gqa_attn_workspace_size(w["B"], w["h_q"], w["h_kv"], w["s_q"], w["d"], w["L_hi"])
+    def setup_device(self):
+        w, i = self.w, self.inp
+        self.out = torch.empty_like(i["q"])
+        ws = self.lka.library().gqa_attn_workspace_size(w["B"], w["h_q"], w["h_kv"], w["s_q"], w["d"], w["L_hi"])
         self.launches = 2 if ws > 256 else 1  # decode kernel (+ merge kernel when the cache is split)
-        # end-to-end: the step's inputs (q, cache_lens) come from pinned host memory, out goes back to it
-        self.q_host = self.inp["q"].cpu().pin_memory()
-        self.lens_host = self.inp["cache_lens"].cpu().pin_memory()
-        self.out_host = torch.empty_like(self.q_host).pin_memory()
-        self.h2d = self.q_host.numel() * self.q_host.element_size() + self.lens_host.numel() * 4
-        self.d2h = self.out_host.numel() * self.out_host.element_size()
+        self.h2d_pairs = [(i["q"], _pinned(i["q"])), (i["cache_lens"], _pinned(i["cache_lens"]))]
+        self.out_host = torch.empty_like(self.out, device="cpu").pin_memory()
 
     def step(self):
         i = self.inp
         self.lka.gqa_attn(i["q"], i["k"], i["v"], i["cache_lens"], causal=self.w["causal"], scale=i["scale"],
                           out=self.out)
 
-    def step_e2e(self):
-        i = self.inp
-        i["q"].copy_(self.q_host, non_blocking=True)
-        i["cache_lens"].copy_(self.lens_host, non_blocking=True)
-        self.lka.gqa_attn(i["q"], i["k"], i["v"], i["cache_lens"], causal=self.w["causal"], scale=i["scale"],
-                          out=self.out)
-        self.out_host.copy_(self.out, non_blocking=True)
-
     def config(self):
         w = self.w
         return {"workload": self.name, "B": w["B"], "h_q": w["h_q"], "h_kv": w["h_kv"], "d_h": w["d"],
                 "s_q": w["s_q"], "cache_lens": f"uniform [{w['L_lo']}, {w['L_hi']}]", "causal": w["causal"],
-                "l2": "K/V cache larger than L2; L2 flushed between timed steps",
+                "l2": "K/V cache larger than L2; L2 flushed between timed steps", "parallelism": "replicas"}
+
+    def oracle_run(self, n):
+        import oracle
+
+        sub = {k: (v[:n].cpu().double() if isinstance(v, torch.Tensor) and k != "cache_lens" else v)
+               for k, v in self.inp.items()}
+        lens = self.inp["cache_lens"][:n].cpu()
+        w = self.w
+        fn = lambda: oracle.gqa(sub["q"], sub["k"], sub["v"], lens, w["causal"], self.inp["scale"])  # noqa: E731
+        nbytes = costs.gqa_bytes(lens.tolist(), w["h_q"], w["h_kv"], w["d"], w["s_q"])
+        return fn, nbytes, oracle.threads_used(0, n * w["h_q"]), f"first {n} of {w['B']} sequences"
+
+
+class LatentAbsorbed(Workload):
+    """latent_absorbed_attn over the GQLA/MLA decode batch: absorb GEMM, latent attention, up-projection."""
+
+    kernel = "latent_attn_kernel"
+    src = ("latent_kv_attention_b200/csrc/latent_attn.cu", "latent_kv_attention_b200/csrc/tc.cuh",
+           "latent_kv_attention_b200/csrc/common.cuh")
+
+    def setup_costs(self):
+        w = self.w
+        self.bytes = costs.latent_bytes(self.lens, w["h_q"], w["g"], w["d_h"], w["r_kv"], w["d_r"], w["s_q"])
+        self.core_flops = costs.latent_core_flops(self.lens, w["h_q"], w["r_kv"], w["d_r"], w["s_q"], w["causal"])
+        self.flops = self.core_flops + costs.latent_proj_flops(w["B"], w["h_q"], w["d_h"], w["r_kv"], w["s_q"])
+        self.tokens = w["B"] * w["s_q"]
+
+    def kernel_work(self, pk):
+        """(bound, achieved-unit work per launch, peak) of the attention kernel: roofline = slower of the two."""
+        cache = sum(self.lens) * (self.w["r_kv"] + self.w["d_r"]) * 2
+        t_mem = cache / (pk["hbm_gbs"] * 1e9)
+        t_tc = self.core_flops / (pk["bf16_tflops"] * 1e12)
+        return ("tensor", self.core_flops) if t_tc > t_mem else ("hbm", cache)
+
+    def setup_device(self):
+        w, i = self.w, self.inp
+        self.out = torch.empty_like(i["q_c"])
+        ws = self.lka.library().latent_absorbed_attn_workspace_size(w["B"], w["h_q"], w["g"], w["s_q"], w["d_h"],
+                                                                    w["r_kv"], w["d_r"], w["L_hi"])
+        rows = w["B"] * w["s_q"] * w["h_q"]
+        split = ws > 256 + 2 * (rows * w["r_kv"] * 2 + 256)
+        self.launches = 3 + (1 if split else 0)  # absorb GEMM, attention, (+ merge), up-projection GEMM
+        self.h2d_pairs = [(i["q_c"], _pinned(i["q_c"])), (i["q_r"], _pinned(i["q_r"])),
+                          (i["cache_lens"], _pinned(i["cache_lens"]))]
+        self.out_host = torch.empty_like(self.out, device="cpu").pin_memory()
+
+    def step(self):
+        i = self.inp
+        self.lka.latent_absorbed_attn(i["q_c"], i["q_r"], i["w_uk"], i["w_uv"], i["latent"], i["cache_lens"],
+                                      causal=self.w["causal"], scale=i["scale"], out=self.out)
+
+    def config(self):
+        w = self.w
+        return {"workload": self.name, "B": w["B"], "h_q": w["h_q"], "g": w["g"], "d_h": w["d_h"], "r_kv": w["r_kv"],
+                "d_r": w["d_r"], "s_q": w["s_q"], "cache_lens": w["L_hi"], "causal": w["causal"],
+                "path": "MQA-absorbed", "l2": "latent cache larger than L2; L2 flushed between timed steps",
                 "parallelism": "replicas"}
 
-    # oracle on the host cores, on a bounded sample of the same workload
-    def oracle_sample(self, target_s: float):
+    def oracle_run(self, n):
         import oracle
 
         i = self.inp
-        n = 8
-        rows = list(range(n))
-        sub = {k: (v[:n].cpu() if isinstance(v, torch.Tensor) else v) for k, v in i.items()}
-        q64, k64, v64 = sub["q"].double(), sub["k"].double(), sub["v"].double()
-        t0 = time.perf_counter()
-        oracle.gqa(q64, k64, v64, sub["cache_lens"], self.w["causal"], i["scale"])
-        t1 = time.perf_counter() - t0
-        reps = max(1, int(math.ceil(target_s / max(t1, 1e-3))) - 1)
-        t0 = time.perf_counter()
-        for _ in range(reps):
-            oracle.gqa(q64, k64, v64, sub["cache_lens"], self.w["causal"], i["scale"])
-        dt = time.perf_counter() - t0
-        lens = [self.lens[r] for r in rows]
+        sub = {k: (v[:n].cpu().double() if k in ("q_c", "q_r", "latent") else v) for k, v in i.items()}
+        lens = i["cache_lens"][:n].cpu()
+        w_uk, w_uv = i["w_uk"].cpu().double(), i["w_uv"].cpu().double()
         w = self.w
-        nbytes = costs.gqa_bytes(lens, w["h_q"], w["h_kv"], w["d"], w["s_q"]) * reps
-        cores = oracle.threads_used(0, n * w["h_q"])
-        return dict(value=nbytes / dt / 1e9, unit="GB/s", cores=cores, kind="oracle",
-                    sample=f"first {n} of {w['B']} sequences ({sum(lens)} cache tokens), {reps} repetitions, "
-                           f"{dt:.1f} s", seconds=dt, reps=reps, n=n)
+        fn = lambda: oracle.latent_absorbed(sub["q_c"], sub["q_r"], w_uk, w_uv, sub["latent"], lens,  # noqa: E731
+                                            w["causal"], i["scale"])
+        nbytes = costs.latent_bytes(lens.tolist(), w["h_q"], w["g"], w["d_h"], w["r_kv"], w["d_r"], w["s_q"])
+        return fn, nbytes, oracle.threads_used(0, n * w["h_q"]), f"first {n} of {w['B']} sequences"
 
 
-WORKLOAD_CLASSES = {"gqa_decode_llama8b": GqaDecode, "gqa_decode_llama8b_b16": GqaDecode}
+class LatentExpanded(LatentAbsorbed):
+    """latent_expand_gqa_attn over the per-group expanded cache (made once, outside the timed steps)."""
+
+    kernel = "expanded_attn_kernel"
+    src = ("latent_kv_attention_b200/csrc/expanded_attn.cu", "latent_kv_attention_b200/csrc/tc.cuh",
+           "latent_kv_attention_b200/csrc/common.cuh")
+
+    def setup_costs(self):
+        w = self.w
+        self.bytes = costs.expanded_bytes(self.lens, w["h_q"], w["g"], w["d_h"], w["d_r"], w["s_q"])
+        self.core_flops = costs.expanded_flops(self.lens, w["h_q"], w["d_h"], w["d_r"], w["s_q"], w["causal"])
+        self.flops = self.core_flops
+        self.tokens = w["B"] * w["s_q"]
+
+    def kernel_work(self, pk):
+        cache = sum(self.lens) * (2 * self.w["g"] * self.w["d_h"] + self.w["d_r"]) * 2
+        return "hbm", cache
+
+    def setup_device(self):
+        w, i = self.w, self.inp
+        self.kc, self.vc, self.kr = self.lka.latent_expand_cache(i["latent"], i["w_uk"], i["w_uv"])
+        del i["latent"]
+        self.out = torch.empty_like(i["q_c"])
+        ws = self.lka.library().latent_expand_gqa_attn_workspace_size(w["B"], w["h_q"], w["g"], w["s_q"], w["d_h"],
+                                                                      w["d_r"], w["L_hi"])
+        self.launches = 2 if ws > 256 else 1
+        self.h2d_pairs = [(i["q_c"], _pinned(i["q_c"])), (i["q_r"], _pinned(i["q_r"])),
+                          (i["cache_lens"], _pinned(i["cache_lens"]))]
+        self.out_host = torch.empty_like(self.out, device="cpu").pin_memory()
+
+    def step(self):
+        i = self.inp
+        self.lka.latent_expand_gqa_attn(i["q_c"], i["q_r"], self.kc, self.vc, self.kr, i["cache_lens"],
+                                        causal=self.w["causal"], scale=i["scale"], out=self.out)
+
+    def config(self):
+        c = super().config()
+        c["path"] = "per-group GQA over the expanded cache"
+        return c
+
+
+class GtaPrefill(Workload):
+    """gta_shared_score_attn causal prefill: one score matrix per group of 4 heads."""
+
+    kernel = "gta_attn_kernel"
+    src = ("latent_kv_attention_b200/csrc/gta_attn.cu", "latent_kv_attention_b200/csrc/tc.cuh",
+           "latent_kv_attention_b200/csrc/common.cuh")
+    bound = "tensor"
+    oracle_n = 1
+
+    def setup_costs(self):
+        w = self.w
+        self.bytes = costs.gta_bytes(self.lens, w["G"], w["H"], w["d_qk"], w["d_v"], w["s_q"])
+        self.flops = costs.gta_flops(self.lens, w["G"], w["H"], w["d_qk"], w["d_v"], w["s_q"], w["causal"])
+        self.core_flops = self.flops
+        self.tokens = w["B"] * w["s_q"]
+
+    def kernel_work(self, pk):
+        return "tensor", self.flops
+
+    def setup_device(self):
+        i = self.inp
+        w = self.w
+        self.out = torch.empty((w["B"], w["H"], w["s_q"], w["d_v"]), dtype=torch.bfloat16, device=self.device)
+        self.launches = 1
+        self.h2d_pairs = [(i[k], _pinned(i[k])) for k in ("q_g", "k_g", "v", "cache_lens")]
+        self.out_host = torch.empty_like(self.out, device="cpu").pin_memory()
+
+    def step(self):
+        i = self.inp
+        self.lka.gta_shared_score_attn(i["q_g"], i["k_g"], i["v"], i["cache_lens"], causal=self.w["causal"],
+                                       scale=i["scale"], out=self.out)
+
+    def config(self):
+        w = self.w
+        return {"workload": self.name, "B": w["B"], "G": w["G"], "H": w["H"], "d_qk": w["d_qk"], "d_v": w["d_v"],
+                "s_q": w["s_q"], "cache_lens": w["L_hi"], "causal": w["causal"],
+                "l2": "inputs 126 MB; L2 flushed between timed steps", "parallelism": "replicas"}
+
+    def oracle_run(self, n):
+        import oracle
+
+        i = self.inp
+        sub = {k: (v[:n].cpu().double() if k in ("q_g", "k_g", "v") else v) for k, v in i.items()}
+        lens = i["cache_lens"][:n].cpu()
+        w = self.w
+        fn = lambda: oracle.gta(sub["q_g"], sub["k_g"], sub["v"], lens, w["causal"], i["scale"])  # noqa: E731
+        nbytes = costs.gta_bytes(lens.tolist(), w["G"], w["H"], w["d_qk"], w["d_v"], w["s_q"])
+        self.oracle_flops = costs.gta_flops(lens.tolist(), w["G"], w["H"], w["d_qk"], w["d_v"], w["s_q"], w["causal"])
+        return fn, nbytes, oracle.threads_used(0, n * w["H"]), f"first {n} of {w['B']} sequences"
+
+
+GqaDecode.kernel_work = lambda self, pk: ("hbm", self.bytes)
+
+WORKLOAD_CLASSES = {
+    "gqa_decode_llama8b": GqaDecode,
+    "gqa_decode_llama8b_b16": GqaDecode,
+    "latent_decode_4k_sq1": LatentAbsorbed,
+    "latent_decode_4k_sq2": LatentAbsorbed,
+    "latent_expanded_4k_sq1": LatentExpanded,
+    "latent_expanded_4k_sq2": LatentExpanded,
+    "gta_prefill_4k": GtaPrefill,
+}
+EXTRAS = ["latent_decode_4k_sq1", "latent_decode_4k_sq2", "latent_expanded_4k_sq2", "gta_prefill_4k"]
+
+
+def oracle_sample(wl, target_s: float):
+    """Times the oracle, as it stands, on the first few sequences, repeated to about target_s seconds."""
+    fn, nbytes, cores, what = wl.oracle_run(wl.oracle_n)
+    t0 = time.perf_counter()
+    fn()
+    t1 = time.perf_counter() - t0
+    reps = max(1, int(math.ceil(target_s / max(t1, 1e-3))) - 1) if target_s > 0 else 1
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        fn()
+    dt = time.perf_counter() - t0
+    return dict(value=nbytes * reps / dt / 1e9, unit="GB/s", cores=cores, kind="oracle",
+                sample=f"{what}, {reps} repetition(s), {dt:.1f} s", seconds=dt)
 
 
 # ----------------------------------------------------------------------------- arms
-def run_lka(args, rank, world, device):
-    import latent_kv_attention_b200 as lka
-
-    wl = WORKLOAD_CLASSES[args.workload](args.workload, device)
-    pk = peaks()
+def measure(wl, steps, warmup, pk, device, world, soak_s=1.0, clocks=None):
+    """Device time of `steps` steps (CUDA events per step, L2 flushed between steps), the main kernel's
+    average launch time from the library's event hook, and the end-to-end time through host buffers."""
+    lka = wl.lka
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
-    for _ in range(max(3, args.warmup)):
+    for _ in range(max(3, warmup)):
         wl.step()
     torch.cuda.synchronize()
     lka.clear_status()
-
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    clocks = ClockSampler(device.index if device.index is not None else 0)
-    clocks.start()
-    clocks.wait_first_sample()
-    # keep the GPU under this load for ~1 s before the timed region so that the clock samples
-    # (every 200 ms) describe the state the timed steps run in; the sampler runs through both
+    if clocks is not None:
+        clocks.start()
+        clocks.wait_first_sample()
+    # keep the GPU under this load for ~soak_s before the timed steps, so the clock samples (every 200 ms)
+    # describe the state the timed steps run in
     t_soak = time.time()
-    while time.time() - t_soak < 1.0:
-        for _ in range(20):
+    while time.time() - t_soak < soak_s:
+        for _ in range(10):
             wl.step()
         torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     lka.kernel_timing(True)
-    for s in range(args.steps):
+    for s in range(steps):
         flush.zero_()  # L2 flush, outside the events
         starts[s].record()
         wl.step()
@@ -264,58 +458,88 @@ def run_lka(args, rank, world, device):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    clk = clocks.stop()
-    step_ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / args.steps
+    clk = clocks.stop() if clocks is not None else None
+    step_ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / steps
     status = lka.device_status()
     if status != 0:
-        raise RuntimeError(f"device status after the timed region: {lka.status_string(status)}")
-
-    # end to end through the public API with pinned host buffers
+        raise RuntimeError(f"{wl.name}: device status after the timed steps: {lka.status_string(status)}")
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     for _ in range(2):
         wl.step_e2e()
     torch.cuda.synchronize()
     e2e_total = 0.0
-    for s in range(args.steps):
+    for s in range(steps):
         flush.zero_()
         e_start.record()
         wl.step_e2e()
         e_end.record()
         e_end.synchronize()
         e2e_total += e_start.elapsed_time(e_end)
-    e2e_ms = e2e_total / args.steps
-
-    t = torch.tensor([step_ms, e2e_ms, kern_ms / max(1, n_timed)], dtype=torch.float64, device=device)
+    t = torch.tensor([step_ms, e2e_total / steps, kern_ms / max(1, n_timed)], dtype=torch.float64, device=device)
     if world > 1:
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    step_ms, e2e_ms, kern_avg_ms = t.tolist()
+    step_ms, e2e_ms, kern_ms = t.tolist()
+    bound, work = wl.kernel_work(pk)
+    if bound == "hbm":
+        peak, unit, achieved = pk["hbm_gbs"], "GB/s", work / (kern_ms * 1e-3) / 1e9
+        peak_src = "hbm_gbs"
+    else:
+        peak, unit, achieved = pk["bf16_tflops"], "TFLOP/s", work / (kern_ms * 1e-3) / 1e12
+        peak_src = "bf16_tflops (burst)"
+    traffic = recorded_traffic(wl.kernel, wl.name, wl.src)
+    roof = {"bound": bound, "kernel": wl.kernel, "achieved": round(achieved, 1), "peak": peak, "unit": unit,
+            "frac": round(achieved / peak, 4), "traffic": traffic, "algorithmic_work_per_launch": work,
+            "launch_ms": round(kern_ms, 4),
+            "peak_source": f"{pk['source']} (MEASURED_PEAKS.json {peak_src})" if pk["source"] == "measured"
+            else "fallback"}
+    return dict(step_ms=step_ms, e2e_ms=e2e_ms, roofline=roof, clocks=clk)
+
+
+def summary(wl, m, world):
+    t = m["step_ms"] * 1e-3
+    return {"ms_per_step": round(m["step_ms"], 4), "gbs": round(wl.bytes * world / t / 1e9, 1),
+            "tflops": round(wl.flops * world / t / 1e12, 2), "tokens_per_s": round(wl.tokens * world / t, 1),
+            "roofline": m["roofline"],
+            "e2e_ms_per_step": round(m["e2e_ms"], 4), "config": wl.config()}
+
+
+def run_lka(args, rank, world, device):
+    pk = peaks()
+    wl = WORKLOAD_CLASSES[args.workload](args.workload, device)
+    clocks = ClockSampler(device.index if device.index is not None else 0)
+    m = measure(wl, args.steps, args.warmup, pk, device, world, clocks=clocks)
+    extras = {}
+    if not args.no_extras:
+        for name in EXTRAS:
+            if name == args.workload:
+                continue
+            x = WORKLOAD_CLASSES[name](name, device)
+            extras[name] = summary(x, measure(x, min(args.steps, 20), args.warmup, pk, device, world, soak_s=0.3),
+                                   world)
+            del x
+            torch.cuda.empty_cache()
     if rank != 0:
         return None
-
-    gbs = wl.bytes * world / (step_ms * 1e-3) / 1e9
-    tflops = wl.flops * world / (step_ms * 1e-3) / 1e12
-    achieved = wl.bytes / (kern_avg_ms * 1e-3) / 1e9
-    traffic = recorded_traffic(wl.kernel, wl.name, wl.src)
+    t = m["step_ms"] * 1e-3
+    gbs = wl.bytes * world / t / 1e9
     line = {
         "metric": METRIC, "value": round(gbs, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(step_ms, 4), "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": round(m["step_ms"], 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) inputs, see synthetic.py)",
         "config": wl.config(),
-        "tokens_per_s": round(wl.tokens * world / (step_ms * 1e-3), 1),
-        "tflops": round(tflops, 3),
+        "tokens_per_s": round(wl.tokens * world / t, 1),
+        "tflops": round(wl.flops * world / t / 1e12, 3),
         "hbm_frac_of_peak": round(gbs / world / pk["hbm_gbs"], 4),
-        "roofline": {"bound": "hbm", "kernel": wl.kernel, "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
-                     "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": traffic,
-                     "algorithmic_bytes_per_launch": wl.bytes, "launch_ms": round(kern_avg_ms, 4),
-                     "peak_source": pk["source"] + " (MEASURED_PEAKS.json hbm_gbs)" if pk["source"] == "measured"
-                     else "fallback"},
-        "e2e": {"value": round(wl.bytes * world / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
-                "h2d_bytes_per_step": wl.h2d, "d2h_bytes_per_step": wl.d2h, "ms_per_step": round(e2e_ms, 4)},
+        "roofline": m["roofline"],
+        "e2e": {"value": round(wl.bytes * world / (m["e2e_ms"] * 1e-3) / 1e9, 1), "unit": "GB/s",
+                "h2d_bytes_per_step": wl.h2d, "d2h_bytes_per_step": wl.d2h, "ms_per_step": round(m["e2e_ms"], 4)},
         "gpu_launches": wl.launches * args.steps,
-        "clocks": clk,
+        "clocks": m["clocks"],
     }
+    if extras:
+        line["other_paths"] = extras
     if world == 1 and not args.no_cpu_baseline:
-        cb = wl.oracle_sample(args.cpu_seconds)
+        cb = oracle_sample(wl, args.cpu_seconds)
         line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
         line["cpu_baseline"]["value"] = round(cb["value"], 4)
     return line
@@ -326,12 +550,12 @@ def run_reference(args, rank, world, device):
     if rank != 0:
         return None
     wl = WORKLOAD_CLASSES[args.workload](args.workload, device, reference=True)
-    per_step = max(1.0, 60.0 / max(1, args.steps + args.warmup))
+    per_step = max(0.5, min(5.0, 60.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
-        wl.oracle_sample(0.0)
+        oracle_sample(wl, 0.0)
     vals, secs, last = [], 0.0, None
     for _ in range(args.steps):
-        last = wl.oracle_sample(min(per_step, 5.0))
+        last = oracle_sample(wl, per_step)
         vals.append(last["value"])
         secs += last["seconds"]
     v = statistics.median(vals)
@@ -356,6 +580,7 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOAD_CLASSES), default="gqa_decode_llama8b")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="measure only --workload, not the other paths")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 

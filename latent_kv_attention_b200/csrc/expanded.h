@@ -1,0 +1,25 @@
+// expanded.h -- launch interface of the GQLA per-group (expanded-cache) GQA path.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace lka {
+
+struct ExpParams {
+    const int32_t* lens;   // device [B]
+    __nv_bfloat16* out;    // [B, h_q, s_q, 128]
+    float* lse;            // [B, h_q, s_q] natural log, or nullptr
+    float* part_o;         // [B*h_q*s_q][nsplit][128] (nsplit > 1)
+    float* part_lse;       // [B*h_q*s_q][nsplit] log2 domain
+    uint32_t* status;
+    int B, h_q, g, s_q, Lmax, causal;
+    float scale_log2;
+    int split_tokens, nsplit;
+};
+
+cudaError_t expanded_attn_launch(const CUtensorMap& qc, const CUtensorMap& qr, const CUtensorMap& kc,
+                                 const CUtensorMap& kr, const CUtensorMap& vc, const ExpParams& p, cudaStream_t st);
+
+}  // namespace lka

@@ -480,6 +480,18 @@ static cudaError_t launch_one(const CUtensorMap& tk, const CUtensorMap& tv, cons
     return e;
 }
 
+cudaError_t gqa_combine_launch(const GqaParams& p, int dtype_bytes, int d, cudaStream_t st) {
+    const size_t nrows = (size_t)p.B * p.h_q * p.s_q;
+    const unsigned grid = (unsigned)((nrows + 3) / 4);
+    if (dtype_bytes == 2 && d == 128) gqa_combine_kernel<__nv_bfloat16, 128><<<grid, 128, 0, st>>>(p);
+    else if (dtype_bytes == 2 && d == 64) gqa_combine_kernel<__nv_bfloat16, 64><<<grid, 128, 0, st>>>(p);
+    else if (dtype_bytes == 2 && d == 256) gqa_combine_kernel<__nv_bfloat16, 256><<<grid, 128, 0, st>>>(p);
+    else if (dtype_bytes == 4 && d == 128) gqa_combine_kernel<float, 128><<<grid, 128, 0, st>>>(p);
+    else if (dtype_bytes == 4 && d == 64) gqa_combine_kernel<float, 64><<<grid, 128, 0, st>>>(p);
+    else return cudaErrorInvalidValue;
+    return cudaPeekAtLastError();
+}
+
 int gqa_tile_tokens(int dtype_bytes, int d, int rb) {
 #define LKA_TILE_CASE(T, DD, R) \
     if (dtype_bytes == (int)sizeof(T) && d == DD && rb == R) return GqaCfg<T, DD, R>::T_TILE;

@@ -22,6 +22,8 @@ struct GqaParams {
     int ratio;              // h_q / h_kv
 };
 
+// Merge of split partials for rows [B*h_q*s_q] of D values (rows needing one split are skipped).
+cudaError_t gqa_combine_launch(const GqaParams& p, int dtype_bytes, int d, cudaStream_t st);
 // Tokens per TMA tile of the kernel instance (0 if the instance does not exist).
 int gqa_tile_tokens(int dtype_bytes, int d, int rb);
 // Launches the decode kernel (grid nsplit x h_kv*n_rb x B) and, when nsplit > 1, the merge.

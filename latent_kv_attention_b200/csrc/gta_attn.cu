@@ -1,0 +1,335 @@
+// gta_attn.cu -- GTA-style grouped shared-score attention on the 5th-generation
+// tensor cores.
+//
+// Operation ("GTA: Grouped-head latenT Attention" press article, section on
+// the grouped shared attention matrix): the heads are split into groups (for
+// example 4 heads per group) and the members of a group share one attention
+// matrix: the scores are computed once per group and then used by every head
+// of the group with that head's own values:
+//     P_gamma = softmax(scale * Q_gamma K_gamma^T)  (causal: bottom-right mask)
+//     O_h     = P_gamma V_h        for every head h of group gamma.
+// Prefill is dense in both contractions, so both run as tcgen05 MMAs.
+//
+// One CTA = (128-query tile, group, sequence); q-tiles are scheduled longest
+// first.  Warp 4 streams 128-key tiles of K_gamma and the V tiles of the
+// group's heads with TMA (2 stages of 80 KB); warp 5 issues S = Q K^T
+// (M = N = 128, K = 64) into tensor memory and, once the softmax has written P
+// back to tensor memory as bf16, one P*V MMA chain per head (M = 128, N = 64,
+// K = 128; A = P from tensor memory) -- the score tile is computed and
+// normalised once and reused by all heads of the group.  Warps 0-3 hold one
+// query row per thread: mask, online softmax with lazy rescaling (the running
+// maximum only moves when it grows by more than 2^8), P to tensor memory.
+#include "common.cuh"
+#include "host_util.h"
+#include "tc.cuh"
+
+namespace lka {
+
+struct GtaParams {
+    const int32_t* lens;
+    __nv_bfloat16* out;  // [B, H, s_q, 64]
+    float* lse;          // [B, G, s_q] or nullptr
+    uint32_t* status;
+    int B, G, H, s_q, Lmax, causal;
+    float scale_log2;
+};
+
+namespace gta {
+constexpr int TQ = 128, TK = 128, NST = 2;
+constexpr int BOX = TK * 128;       // 128 rows x 64 bf16
+constexpr int STAGE = 5 * BOX;      // K_gamma + up to 4 value tiles
+constexpr int OFF_Q = 0;
+constexpr int OFF_KV = BOX;
+constexpr int OFF_BAR = OFF_KV + NST * STAGE;
+constexpr int SMEM = 1024 + OFF_BAR + 256;
+constexpr uint32_t T_O = 0;         // 4 heads x 64 fp32 columns
+constexpr uint32_t T_S = 256;       // 128 fp32 columns
+constexpr uint32_t T_P = 384;       // 64 columns of bf16 pairs
+}  // namespace gta
+
+__global__ void __launch_bounds__(192, 1)
+    gta_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const GtaParams p) {
+    using namespace gta;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+    uint64_t* q_full = bars;
+    uint64_t* kv_full = bars + 1;
+    uint64_t* kv_empty = kv_full + NST;
+    uint64_t* s_ready = kv_empty + NST;
+    uint64_t* s_free = s_ready + 1;
+    uint64_t* p_ready = s_free + 1;
+    uint64_t* o_ready = p_ready + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_ready + 1);
+    __shared__ int s_abort;
+
+    const int n_qt = cdiv(p.s_q, TQ);
+    const int qt = n_qt - 1 - (int)blockIdx.x;  // longest tiles first
+    const int grp = blockIdx.y, b = blockIdx.z;
+    const int HPG = p.H / p.G;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int L = clamp_len(p.lens, b, p.Lmax, p.s_q, p.causal, p.status,
+                            threadIdx.x == 0 && blockIdx.x == 0 && grp == 0);
+    const int q0 = qt * TQ;
+    const int q_last = min(q0 + TQ, p.s_q) - 1;
+    const int key_end = p.causal ? (L - p.s_q + q_last + 1) : L;  // keys any row of the tile may see
+    const int n_tiles = cdiv(key_end, TK);
+
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        mbar_init(smem_u32(q_full), 1);
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(smem_u32(&kv_full[s]), 1);
+            mbar_init(smem_u32(&kv_empty[s]), 1);
+        }
+        mbar_init(smem_u32(s_ready), 1);
+        mbar_init(smem_u32(s_free), 4);
+        mbar_init(smem_u32(p_ready), 4);
+        mbar_init(smem_u32(o_ready), 1);
+        fence_barrier_init();
+    }
+    if (warp == 5) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 4) {
+        // ------------------------------ producer ------------------------------
+        if (lane == 0) {
+            const uint32_t qb = smem_u32(q_full);
+            mbar_arrive_expect_tx(qb, BOX);
+            tma_load_2d(smem_u32(smem + OFF_Q), &tm_q, 0, (b * p.G + grp) * p.s_q + q0, qb);
+            int issued = 0;
+            for (int i = 0; i < n_tiles; ++i) {
+                const int s = i % NST;
+                if (i >= NST && !mbar_wait(smem_u32(&kv_empty[s]), ((i / NST) - 1) & 1, p.status)) {
+                    s_abort = 1;
+                    break;
+                }
+                if (*(volatile int*)&s_abort) break;
+                const uint32_t fb = smem_u32(&kv_full[s]);
+                mbar_arrive_expect_tx(fb, (1 + HPG) * BOX);
+                const uint32_t d = smem_u32(smem + OFF_KV + s * STAGE);
+                const int k0 = i * TK;
+                tma_load_2d(d, &tm_k, 0, (b * p.G + grp) * p.Lmax + k0, fb);
+                for (int hh = 0; hh < HPG; ++hh)
+                    tma_load_2d(d + (1 + hh) * BOX, &tm_v, 0, (b * p.H + grp * HPG + hh) * p.Lmax + k0, fb);
+                ++issued;
+            }
+            for (int i = issued - 1; i >= 0 && i >= issued - NST; --i)
+                mbar_wait(smem_u32(&kv_full[i % NST]), (i / NST) & 1, p.status);
+            mbar_wait(qb, 0, p.status);
+        }
+    } else if (warp == 5) {
+        // ------------------------------ MMA issuer ------------------------------
+        constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 64, false, true);
+        bool ok = mbar_wait(smem_u32(q_full), 0, p.status);
+        auto issue_qk = [&](int j) -> bool {
+            const int s = j % NST;
+            if (!mbar_wait(smem_u32(&kv_full[s]), (j / NST) & 1, p.status)) return false;
+            uint8_t* st = smem + OFF_KV + s * STAGE;
+            const int nvalid = min(TK, L - j * TK);
+            if (nvalid < TK) {
+                // keys past the cache length may hold anything (even NaN): zero K and V rows there
+                const int rows = TK - nvalid;
+                for (int idx = lane; idx < (1 + HPG) * rows * 8; idx += 32) {
+                    const int bx = idx / (rows * 8), rr = (idx / 8) % rows, c = idx % 8;
+                    *reinterpret_cast<uint4*>(st + bx * BOX + (nvalid + rr) * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+            }
+            if (j >= 1 && !mbar_wait(smem_u32(s_free), (j - 1) & 1, p.status)) return false;
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t qa = smem_u32(smem + OFF_Q), ka = smem_u32(st);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    umma_ss(tmem + T_S, smem_desc_sw128(qa + k * 32, 16, 1024), smem_desc_sw128(ka + k * 32, 16, 1024),
+                            idesc_qk, k != 0);
+                umma_commit(smem_u32(s_ready));
+            }
+            __syncwarp();
+            return true;
+        };
+        if (ok) ok = issue_qk(0);
+        for (int j = 0; ok && j < n_tiles; ++j) {
+            if (j + 1 < n_tiles && !issue_qk(j + 1)) break;
+            if (!mbar_wait(smem_u32(p_ready), j & 1, p.status)) break;
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t va = smem_u32(smem + OFF_KV + (j % NST) * STAGE + BOX);
+                for (int hh = 0; hh < HPG; ++hh)
+#pragma unroll
+                    for (int kk = 0; kk < TK / 16; ++kk)
+                        umma_ts(tmem + T_O + hh * 64, tmem + T_P + kk * 8,
+                                smem_desc_sw128(va + hh * BOX + kk * 2048, BOX, 1024), idesc_pv, (j | kk) != 0);
+                umma_commit(smem_u32(&kv_empty[j % NST]));
+                umma_commit(smem_u32(o_ready));
+            }
+            __syncwarp();
+        }
+    } else {
+        // --------------------------- softmax warps 0-3 ---------------------------
+        const int row = warp * 32 + lane;  // query row in the tile == TMEM lane
+        const int q = q0 + row;
+        const bool row_ok = q < p.s_q;
+        const int vis_end = row_ok ? (p.causal ? L - p.s_q + q + 1 : L) : 0;  // keys < vis_end are visible
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        float m_ref = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < n_tiles; ++j) {
+            if (ok) ok = mbar_wait(smem_u32(s_ready), j & 1, p.status);
+            tc_fence_after();
+            uint32_t sr[TK];
+#pragma unroll
+            for (int c0 = 0; c0 < TK; c0 += 16) tmem_ld16(tmem + lane_base + T_S + c0, sr + c0);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(s_free));  // the next score tile may be written
+            const int k0 = j * TK;
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < TK; ++c) {
+                const float v = (k0 + c < vis_end) ? __uint_as_float(sr[c]) * p.scale_log2 : -INFINITY;
+                sr[c] = __float_as_uint(v);
+                mx = fmaxf(mx, v);
+            }
+            const float m_new = fmaxf(m_ref, mx);
+            bool resc = false;
+            float alpha = 1.f, m_use = m_ref;
+            if (m_ref == -INFINITY) {
+                m_use = m_new;
+            } else if (m_new > m_ref + 8.0f) {
+                resc = true;
+                alpha = exp2f(m_ref - m_new);
+                m_use = m_new;
+            }
+            float rs = 0.f;
+            uint32_t pk[TK / 2];
+#pragma unroll
+            for (int c = 0; c < TK; c += 2) {
+                const float p0 = m_use == -INFINITY ? 0.f : exp2f(__uint_as_float(sr[c]) - m_use);
+                const float p1 = m_use == -INFINITY ? 0.f : exp2f(__uint_as_float(sr[c + 1]) - m_use);
+                rs += p0 + p1;
+                pk[c / 2] = pack_bf16x2(p0, p1);
+            }
+            l = (resc ? l * alpha : l) + rs;
+            m_ref = m_use;
+            // P(j-1) and O must be released by PV(j-1) before P(j) is written and O rescaled
+            if (ok && j >= 1) ok = mbar_wait(smem_u32(o_ready), (j - 1) & 1, p.status);
+            tc_fence_after();
+#pragma unroll
+            for (int c0 = 0; c0 < TK / 2; c0 += 16) tmem_st16(tmem + lane_base + T_P + c0, pk + c0);
+            if (__any_sync(0xffffffffu, resc)) {
+                for (int c0 = 0; c0 < 64 * HPG; c0 += 16) {
+                    uint32_t o[16];
+                    tmem_ld16(tmem + lane_base + T_O + c0, o);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    tmem_st16(tmem + lane_base + T_O + c0, o);
+                }
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(p_ready));
+        }
+        if (ok) ok = mbar_wait(smem_u32(o_ready), (n_tiles - 1) & 1, p.status);
+        if (!ok) {
+            s_abort = 1;
+        } else {
+            tc_fence_after();
+            const float inv_l = l > 0.f ? 1.f / l : 0.f;
+            for (int hh = 0; hh < HPG; ++hh) {
+                for (int c0 = 0; c0 < 64; c0 += 16) {
+                    uint32_t o[16];
+                    tmem_ld16(tmem + lane_base + T_O + hh * 64 + c0, o);
+                    tmem_ld_wait();
+                    if (row_ok) {
+                        uint32_t pkk[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            pkk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+                        uint4* d = reinterpret_cast<uint4*>(
+                            p.out + (((size_t)b * p.H + grp * HPG + hh) * p.s_q + q) * 64 + c0);
+                        d[0] = make_uint4(pkk[0], pkk[1], pkk[2], pkk[3]);
+                        d[1] = make_uint4(pkk[4], pkk[5], pkk[6], pkk[7]);
+                    }
+                }
+            }
+            if (row_ok && p.lse)
+                p.lse[((size_t)b * p.G + grp) * p.s_q + q] =
+                    (l > 0.f ? m_ref + log2f(l) : -INFINITY) * 0.69314718055994530942f;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace lka
+
+using namespace lka;
+
+extern "C" {
+
+size_t gta_shared_score_attn_workspace_size(int B, int G, int H, int s_q, int d_qk, int d_v, int Lmax) {
+    if (B < 0 || G < 1 || H < 1 || s_q < 1 || Lmax < 1 || H % G) return 0;
+    (void)d_qk;
+    (void)d_v;
+    return kWsHeaderBytes;  // status word only: one CTA covers the whole key range of its query tile
+}
+
+lka_status_t gta_shared_score_attn(const void* q_g, const void* k_g, const void* v, const int32_t* cache_lens,
+                                   void* out, float* lse, int B, int G, int H, int s_q, int d_qk, int d_v, int Lmax,
+                                   int causal, float scale, lka_dtype_t dtype, void* ws, size_t ws_bytes,
+                                   void* stream) {
+    if (B < 0 || G < 1 || H < 1 || s_q < 1 || Lmax < 1 || d_qk < 1 || d_v < 1) return LKA_ERR_INVALID_ARG;
+    if (H % G) return LKA_ERR_INVALID_ARG;
+    if (dtype != LKA_BF16 || d_qk != 64 || d_v != 64 || H / G > 4) return LKA_ERR_UNSUPPORTED;
+    if ((long long)B * H * Lmax >= (1ll << 31) || (long long)B * G * s_q >= (1ll << 31) || B > 65535 || G > 65535)
+        return LKA_ERR_UNSUPPORTED;
+    if (B == 0) return LKA_OK;
+    const void* ptrs[] = {q_g, k_g, v, cache_lens, out};
+    for (const void* ptr : ptrs)
+        if (!ptr || !aligned16(ptr)) return LKA_ERR_INVALID_ARG;
+    if (!isfinite(scale)) return LKA_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < kWsHeaderBytes) return LKA_ERR_WORKSPACE;
+    const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    CUtensorMap tq, tk, tv;
+    if (!make_tmap_2d(&tq, BF, q_g, 64, (uint64_t)B * G * s_q, 128, 64, 128) ||
+        !make_tmap_2d(&tk, BF, k_g, 64, (uint64_t)B * G * Lmax, 128, 64, 128) ||
+        !make_tmap_2d(&tv, BF, v, 64, (uint64_t)B * H * Lmax, 128, 64, 128))
+        return LKA_ERR_CUDA;
+    GtaParams p{};
+    p.lens = cache_lens;
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.lse = lse;
+    p.status = static_cast<uint32_t*>(ws);
+    p.B = B;
+    p.G = G;
+    p.H = H;
+    p.s_q = s_q;
+    p.Lmax = Lmax;
+    p.causal = causal ? 1 : 0;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (cudaFuncSetAttribute(gta_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gta::SMEM) != cudaSuccess)
+        return LKA_ERR_CUDA;
+    dim3 grid(cdiv(s_q, gta::TQ), G, B);
+    TimedLaunch timer(st);
+    gta_attn_kernel<<<grid, 192, gta::SMEM, st>>>(tq, tk, tv, p);
+    timer.stop();
+    return cudaPeekAtLastError() == cudaSuccess ? LKA_OK : LKA_ERR_CUDA;
+}
+
+}  // extern "C"

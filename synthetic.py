@@ -134,6 +134,11 @@ WORKLOADS = {
                                  L_lo=4096, L_hi=4096, causal=True),
     "latent_decode_4k_sq2": dict(kind="latent", seed=4, B=64, h_q=128, g=8, d_h=128, r_kv=512, d_r=64, s_q=2,
                                  L_lo=4096, L_hi=4096, causal=True),
+    # the same latent inputs, run through the per-group GQA path after the one-time cache expansion
+    "latent_expanded_4k_sq1": dict(kind="latent", seed=4, B=64, h_q=128, g=8, d_h=128, r_kv=512, d_r=64, s_q=1,
+                                   L_lo=4096, L_hi=4096, causal=True),
+    "latent_expanded_4k_sq2": dict(kind="latent", seed=4, B=64, h_q=128, g=8, d_h=128, r_kv=512, d_r=64, s_q=2,
+                                   L_lo=4096, L_hi=4096, causal=True),
 }
 
 
