@@ -55,7 +55,7 @@ struct GqaCfg {
     static constexpr int STAGE_BYTES = 2 * MAT_BYTES;
     static constexpr int NSTAGE0 = (96 * 1024) / STAGE_BYTES;
     static constexpr int NSTAGE = NSTAGE0 < 2 ? 2 : (NSTAGE0 > 4 ? 4 : NSTAGE0);
-    static constexpr int P_BYTES = 4 * TW * RB * 4 + 4 * RB * 4;  // probabilities + rescale factors
+    static constexpr int P_BYTES = 4 * TW * RB * 8 + 4 * RB * 4;  // probabilities (stored as pairs) + rescale
     static constexpr int MERGE_BYTES = 4 * RB * D * 4 + 2 * 4 * RB * 4;
     static constexpr int SMEM = 1024 /*align slack*/ + NSTAGE * STAGE_BYTES + P_BYTES + 256 /*barriers*/;
     static constexpr int MINB = (RB <= 8 && SMEM <= 110 * 1024) ? 2 : 1;  // resident CTAs per SM
@@ -144,8 +144,8 @@ __global__ void __launch_bounds__(160, GqaCfg<T, D, RB>::MINB)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
     uint8_t* stages = smem;
-    float* p_buf = reinterpret_cast<float*>(smem + C::NSTAGE * C::STAGE_BYTES);  // [4][TW][RB]
-    float* a_buf = p_buf + 4 * C::TW * RB;                                          // [4][RB]
+    float2* p_buf = reinterpret_cast<float2*>(smem + C::NSTAGE * C::STAGE_BYTES);  // [4][TW][RB] (p, p) pairs
+    float* a_buf = reinterpret_cast<float*>(p_buf + 4 * C::TW * RB);                 // [4][RB]
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::NSTAGE * C::STAGE_BYTES + C::P_BYTES);
     __shared__ int s_abort;
 
@@ -230,6 +230,7 @@ __global__ void __launch_bounds__(160, GqaCfg<T, D, RB>::MINB)
     const int my_last = p.causal ? (L - p.s_q + my_t) : (L - 1);  // last visible key of my row
 
     // query slice of this lane, pre-scaled into the log2 domain
+    // the two halves of each pair multiply consecutive key elements (packed fp32x2 FMAs)
     float qreg[RB][C::CPL * C::EPC];
     {
         const T* qbase = reinterpret_cast<const T*>(p.q) +
@@ -251,13 +252,13 @@ __global__ void __launch_bounds__(160, GqaCfg<T, D, RB>::MINB)
     }
 
     float m_run = -INFINITY, l_run = 0.f;
-    float o[RB][C::DPLV];
+    float2 o[RB][C::DPLV / 2];
 #pragma unroll
     for (int r = 0; r < RB; ++r)
 #pragma unroll
-        for (int d = 0; d < C::DPLV; ++d) o[r][d] = 0.f;
+        for (int d = 0; d < C::DPLV / 2; ++d) o[r][d] = make_float2(0.f, 0.f);
 
-    float* pw = p_buf + warp * C::TW * RB;
+    float2* pw = p_buf + warp * C::TW * RB;
     float* aw = a_buf + warp * RB;
     bool aborted = false;
 
@@ -277,9 +278,9 @@ __global__ void __launch_bounds__(160, GqaCfg<T, D, RB>::MINB)
 #pragma unroll
         for (int ps = 0; ps < C::NPASS; ++ps) {
             const int jt = warp * C::TW + ps * C::P + tok_in_pass;  // token row in the tile
-            float acc[RB];
+            float2 acc2[RB];
 #pragma unroll
-            for (int r = 0; r < RB; ++r) acc[r] = 0.f;
+            for (int r = 0; r < RB; ++r) acc2[r] = make_float2(0.f, 0.f);
 #pragma unroll
             for (int c = 0; c < C::CPL; ++c) {
                 int seg, chunk;
@@ -289,8 +290,13 @@ __global__ void __launch_bounds__(160, GqaCfg<T, D, RB>::MINB)
 #pragma unroll
                 for (int r = 0; r < RB; ++r)
 #pragma unroll
-                    for (int e = 0; e < C::EPC; ++e) acc[r] = fmaf(qreg[r][c * C::EPC + e], kf[e], acc[r]);
+                    for (int e = 0; e < C::EPC; e += 2)
+                        acc2[r] = __ffma2_rn(make_float2(qreg[r][c * C::EPC + e], qreg[r][c * C::EPC + e + 1]),
+                                             make_float2(kf[e], kf[e + 1]), acc2[r]);
             }
+            float acc[RB];
+#pragma unroll
+            for (int r = 0; r < RB; ++r) acc[r] = acc2[r].x + acc2[r].y;
             // reduce-scatter over the LPT lanes of the token: lane li ends with row li / DUP
             int nr = RB;
 #pragma unroll
@@ -330,7 +336,7 @@ __global__ void __launch_bounds__(160, GqaCfg<T, D, RB>::MINB)
         for (int ps = 0; ps < C::NPASS; ++ps) {
             const float pv = exp2f(sc[ps] - m_ref);
             sum += pv;
-            if (li % C::DUP == 0) pw[(ps * C::P + tok_in_pass) * RB + my_row] = pv;
+            if (li % C::DUP == 0) pw[(ps * C::P + tok_in_pass) * RB + my_row] = make_float2(pv, pv);
         }
 #pragma unroll
         for (int m = C::LPT; m < 32; m *= 2) sum += __shfl_xor_sync(0xffffffffu, sum, m);
@@ -346,7 +352,7 @@ __global__ void __launch_bounds__(160, GqaCfg<T, D, RB>::MINB)
 #pragma unroll
         for (int r = 0; r < RB; ++r)
 #pragma unroll
-            for (int d = 0; d < C::DPLV; ++d) o[r][d] *= al[r];
+            for (int d = 0; d < C::DPLV / 2; ++d) o[r][d] = __fmul2_rn(o[r][d], make_float2(al[r], al[r]));
         {
             const int ob = lane * C::DPLV * C::E;  // byte offset of this lane's value slice in a row
             const int vseg = ob / 128, vchunk = (ob % 128) / 16, vin = ob % 16;
@@ -357,12 +363,13 @@ __global__ void __launch_bounds__(160, GqaCfg<T, D, RB>::MINB)
                 const int jt = warp * C::TW + jj;
                 float vf[C::DPLV];
                 load_v_slice<T, C::DPLV>(vt + swz_off<C::T_TILE>(vseg, jt, vchunk) + vin, vf);
-                const float* pr = pw + jj * RB;
+                const float2* pr = pw + jj * RB;
 #pragma unroll
                 for (int r = 0; r < RB; ++r) {
-                    const float pj = pr[r];
+                    const float2 pj = pr[r];
 #pragma unroll
-                    for (int d = 0; d < C::DPLV; ++d) o[r][d] = fmaf(pj, vf[d], o[r][d]);
+                    for (int d = 0; d < C::DPLV / 2; ++d)
+                        o[r][d] = __ffma2_rn(pj, make_float2(vf[2 * d], vf[2 * d + 1]), o[r][d]);
                 }
             }
         }
@@ -381,7 +388,8 @@ __global__ void __launch_bounds__(160, GqaCfg<T, D, RB>::MINB)
 #pragma unroll
     for (int r = 0; r < RB; ++r)
 #pragma unroll
-        for (int d = 0; d < C::DPLV; ++d) om[(warp * RB + r) * D + lane * C::DPLV + d] = o[r][d];
+        for (int d = 0; d < C::DPLV / 2; ++d)
+            *reinterpret_cast<float2*>(&om[(warp * RB + r) * D + lane * C::DPLV + 2 * d]) = o[r][d];
     if (tok_in_pass == 0 && li % C::DUP == 0) {
         mm[warp * RB + my_row] = m_run;
         lm[warp * RB + my_row] = l_run;
