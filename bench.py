@@ -402,6 +402,10 @@ WORKLOAD_CLASSES = {
     "latent_expanded_4k_sq1": LatentExpanded,
     "latent_expanded_4k_sq2": LatentExpanded,
     "gta_prefill_4k": GtaPrefill,
+    # smaller cases for full ncu captures
+    "latent_decode_4k_sq1_b32": LatentAbsorbed,
+    "latent_expanded_4k_sq2_b16": LatentExpanded,
+    "gta_prefill_4k_b2": GtaPrefill,
 }
 EXTRAS = ["latent_decode_4k_sq1", "latent_decode_4k_sq2", "latent_expanded_4k_sq2", "gta_prefill_4k"]
 

@@ -117,6 +117,13 @@ __device__ __forceinline__ void named_barrier(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// 2^x with the hardware approximation (MUFU; ftz; 2^-inf = +0).
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // ---- element conversion -------------------------------------------------------
 // Unpack 8 bf16 values held in 16 bytes into fp32 (exact).
 __device__ __forceinline__ void bf16x8_to_f32(const uint4 u, float* f) {

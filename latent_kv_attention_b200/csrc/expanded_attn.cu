@@ -63,10 +63,11 @@ __global__ void __launch_bounds__(192, 1)
     uint64_t* q_full = bars;
     uint64_t* kv_full = bars + 1;
     uint64_t* kv_empty = kv_full + NST;
-    uint64_t* s_ready = kv_empty + NST;
-    uint64_t* p_ready = s_ready + 2;
-    uint64_t* o_ready = p_ready + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_ready + 1);
+    uint64_t* s_ready = kv_empty + NST;  // [2] QK(j) done
+    uint64_t* s_free = s_ready + 2;      // [2] S(j) loaded by the softmax warps
+    uint64_t* p_ready = s_free + 2;      // [2] P^T(j) written
+    uint64_t* o_ready = p_ready + 2;     // [2] PV(j) done
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_ready + 2);
     float* alpha_buf = reinterpret_cast<float*>(smem + C::OFF_AUX);
     float* l_buf = alpha_buf + NR;
     float* m_buf = l_buf + NR;
@@ -91,9 +92,10 @@ __global__ void __launch_bounds__(192, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(smem_u32(&s_ready[i]), 1);
+            mbar_init(smem_u32(&s_free[i]), 4);
             mbar_init(smem_u32(&p_ready[i]), 4);
+            mbar_init(smem_u32(&o_ready[i]), 1);
         }
-        mbar_init(smem_u32(o_ready), 1);
         fence_barrier_init();
     }
     if (warp == 5) {
@@ -141,55 +143,59 @@ __global__ void __launch_bounds__(192, 1)
         }
     } else if (warp == 5) {
         // -------------------------------- MMA issuer --------------------------------
+        // per step j: QK(j) (needs S(j-2) loaded by the softmax warps) and PV(j-1); with two
+        // KV stages, QK(j) also needs PV(j-2) to have released its stage
         constexpr uint32_t idesc_qk = idesc_bf16_f32(128, NR, false, false);
         constexpr uint32_t idesc_pv = idesc_bf16_f32(128, NR, true, false);
         bool ok = mbar_wait(smem_u32(q_full), 0, p.status);
-        auto issue_qk = [&](int j) -> bool {
-            const int s = j % NST;
-            if (!mbar_wait(smem_u32(&kv_full[s]), (j / NST) & 1, p.status)) return false;
-            uint8_t* st = smem + C::OFF_KV + s * C::STAGE;
-            const int nvalid = min(TK, kend - (kbeg + j * TK));
-            if (nvalid < TK) {
-                // tokens past the key range may hold anything (even NaN): zero them so P = 0 adds nothing
-                const int rows = TK - nvalid;
-                for (int idx = lane; idx < 5 * rows * 8; idx += 32) {
-                    const int bx = idx / (rows * 8), rr = (idx / 8) % rows, c = idx % 8;
-                    *reinterpret_cast<uint4*>(st + bx * C::BOX + (nvalid + rr) * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+        for (int j = 0; ok && j < n_tiles + 1; ++j) {
+            if (j < n_tiles) {
+                const int s = j % NST;
+                if (!mbar_wait(smem_u32(&kv_full[s]), (j / NST) & 1, p.status)) break;
+                uint8_t* st = smem + C::OFF_KV + s * C::STAGE;
+                const int nvalid = min(TK, kend - (kbeg + j * TK));
+                if (nvalid < TK) {
+                    // tokens past the key range may hold anything (even NaN): zero them so P = 0 adds nothing
+                    const int rows = TK - nvalid;
+                    for (int idx = lane; idx < 5 * rows * 8; idx += 32) {
+                        const int bx = idx / (rows * 8), rr = (idx / 8) % rows, c = idx % 8;
+                        *reinterpret_cast<uint4*>(st + bx * C::BOX + (nvalid + rr) * 128 + c * 16) =
+                            make_uint4(0, 0, 0, 0);
+                    }
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
                 }
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                if (j >= 2 && !mbar_wait(smem_u32(&s_free[j & 1]), ((j >> 1) - 1) & 1, p.status)) break;
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t ka = smem_u32(st);
+                    const uint32_t qa = smem_u32(smem + C::OFF_Q);
+                    for (int kb = 0; kb < 3; ++kb)
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            umma_ss(tmem + C::T_S + (j & 1) * NR, smem_desc_sw128(ka + kb * C::BOX + k * 32, 16, 1024),
+                                    smem_desc_sw128(qa + kb * NR * 128 + k * 32, 16, 1024), idesc_qk, (kb | k) != 0);
+                    umma_commit(smem_u32(&s_ready[j & 1]));
+                }
                 __syncwarp();
             }
-            tc_fence_after();
-            if (lane == 0) {
-                const uint32_t ka = smem_u32(st);
-                const uint32_t qa = smem_u32(smem + C::OFF_Q);
-                for (int kb = 0; kb < 3; ++kb)
+            if (j >= 1) {
+                const int i = j - 1;
+                if (!mbar_wait(smem_u32(&p_ready[i & 1]), (i >> 1) & 1, p.status)) break;
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t va = smem_u32(smem + C::OFF_KV + (i % NST) * C::STAGE + 3 * C::BOX);
+                    const uint32_t pa = smem_u32(smem + C::OFF_PT + (i & 1) * C::PT_BYTES);
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        umma_ss(tmem + C::T_S + (j & 1) * NR, smem_desc_sw128(ka + kb * C::BOX + k * 32, 16, 1024),
-                                smem_desc_sw128(qa + kb * NR * 128 + k * 32, 16, 1024), idesc_qk, (kb | k) != 0);
-                umma_commit(smem_u32(&s_ready[j & 1]));
+                    for (int kk = 0; kk < TK / 16; ++kk)
+                        umma_ss(tmem + C::T_O, smem_desc_sw128(va + kk * 2048, C::BOX, 1024),
+                                smem_desc_sw128(pa + (kk / 4) * NR * 128 + (kk % 4) * 32, 16, 1024), idesc_pv,
+                                (i | kk) != 0);
+                    umma_commit(smem_u32(&kv_empty[i % NST]));
+                    umma_commit(smem_u32(&o_ready[i & 1]));
+                }
+                __syncwarp();
             }
-            __syncwarp();
-            return true;
-        };
-        if (ok) ok = issue_qk(0);
-        for (int i = 0; ok && i < n_tiles; ++i) {
-            if (i + 1 < n_tiles && !issue_qk(i + 1)) break;
-            if (!mbar_wait(smem_u32(&p_ready[i & 1]), (i >> 1) & 1, p.status)) break;
-            tc_fence_after();
-            if (lane == 0) {
-                const uint32_t va = smem_u32(smem + C::OFF_KV + (i % NST) * C::STAGE + 3 * C::BOX);
-                const uint32_t pa = smem_u32(smem + C::OFF_PT + (i & 1) * C::PT_BYTES);
-#pragma unroll
-                for (int kk = 0; kk < TK / 16; ++kk)
-                    umma_ss(tmem + C::T_O, smem_desc_sw128(va + kk * 2048, C::BOX, 1024),
-                            smem_desc_sw128(pa + (kk / 4) * NR * 128 + (kk % 4) * 32, 16, 1024), idesc_pv,
-                            (i | kk) != 0);
-                umma_commit(smem_u32(&kv_empty[i % NST]));
-                umma_commit(smem_u32(o_ready));
-            }
-            __syncwarp();
         }
     } else {
         // ----------------------------- softmax warps (0-3) -----------------------------
@@ -213,9 +219,14 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
                 for (int c0 = 0; c0 < NR; c0 += 16) tmem_ld16(tmem + lane_base + C::T_S + x * NR + c0, v + c0);
                 tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&s_free[x]));  // the score buffer may be rewritten
 #pragma unroll
                 for (int r = 0; r < NR; ++r) sc[r * TK + tid] = __uint_as_float(v[r]);
             }
+            // P^T buffer x was last read by PV(i-2)
+            if (ok && i >= 2) ok = mbar_wait(smem_u32(&o_ready[x]), ((i >> 1) - 1) & 1, p.status);
             named_barrier(1, 128);
             uint8_t* pt = smem + C::OFF_PT + x * C::PT_BYTES;
             const int k0 = kbeg + i * TK;
@@ -240,13 +251,13 @@ __global__ void __launch_bounds__(192, 1)
                 if (m_ref[k] == -INFINITY) {
                     m_use = m_new;
                 } else if (m_new > m_ref[k] + 8.0f) {
-                    alpha = exp2f(m_ref[k] - m_new);
+                    alpha = fast_exp2(m_ref[k] - m_new);
                     m_use = m_new;
                 }
                 float pv[8], rs = 0.f;
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    pv[e] = m_use == -INFINITY ? 0.f : exp2f(s[e] - m_use);
+                    pv[e] = m_use == -INFINITY ? 0.f : fast_exp2(s[e] - m_use);
                     rs += pv[e];
                 }
 #pragma unroll
@@ -260,12 +271,13 @@ __global__ void __launch_bounds__(192, 1)
                 if (c8 == 0) alpha_buf[r] = alpha;
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            if (ok && i >= 1) ok = mbar_wait(smem_u32(o_ready), (i - 1) & 1, p.status);
             named_barrier(1, 128);  // alpha_buf complete
             bool any = false;
 #pragma unroll
             for (int r = 0; r < NR; ++r) any |= alpha_buf[r] != 1.f;
             if (any) {
+                // O^T may only be rescaled once PV(i-1) has been accumulated into it
+                if (ok && i >= 1) ok = mbar_wait(smem_u32(&o_ready[(i - 1) & 1]), ((i - 1) >> 1) & 1, p.status);
                 tc_fence_after();
                 uint32_t o[NR];
 #pragma unroll
@@ -282,7 +294,7 @@ __global__ void __launch_bounds__(192, 1)
             if (lane == 0) mbar_arrive(smem_u32(&p_ready[x]));
         }
         // ---- epilogue ----
-        if (ok) ok = mbar_wait(smem_u32(o_ready), (n_tiles - 1) & 1, p.status);
+        if (ok) ok = mbar_wait(smem_u32(&o_ready[(n_tiles - 1) & 1]), ((n_tiles - 1) >> 1) & 1, p.status);
 #pragma unroll
         for (int k = 0; k < C::K_ITEMS; ++k) {
             const int r = 8 * k + 2 * warp + lane / 16;

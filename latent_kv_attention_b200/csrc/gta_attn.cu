@@ -44,7 +44,7 @@ constexpr int OFF_BAR = OFF_KV + NST * STAGE;
 constexpr int SMEM = 1024 + OFF_BAR + 256;
 constexpr uint32_t T_O = 0;         // 4 heads x 64 fp32 columns
 constexpr uint32_t T_S = 256;       // 128 fp32 columns
-constexpr uint32_t T_P = 384;       // 64 columns of bf16 pairs
+constexpr uint32_t T_P = 384;       // 2 x 64 columns of bf16 pairs (double-buffered P)
 }  // namespace gta
 
 __global__ void __launch_bounds__(192, 1)
@@ -59,9 +59,9 @@ __global__ void __launch_bounds__(192, 1)
     uint64_t* kv_empty = kv_full + NST;
     uint64_t* s_ready = kv_empty + NST;
     uint64_t* s_free = s_ready + 1;
-    uint64_t* p_ready = s_free + 1;
-    uint64_t* o_ready = p_ready + 1;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_ready + 1);
+    uint64_t* p_ready = s_free + 1;   // [2] P(j) in buffer j&1 written
+    uint64_t* o_ready = p_ready + 2;  // [2] PV(j) done
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_ready + 2);
     __shared__ int s_abort;
 
     const int n_qt = cdiv(p.s_q, TQ);
@@ -85,8 +85,10 @@ __global__ void __launch_bounds__(192, 1)
         }
         mbar_init(smem_u32(s_ready), 1);
         mbar_init(smem_u32(s_free), 4);
-        mbar_init(smem_u32(p_ready), 4);
-        mbar_init(smem_u32(o_ready), 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_u32(&p_ready[i]), 4);
+            mbar_init(smem_u32(&o_ready[i]), 1);
+        }
         fence_barrier_init();
     }
     if (warp == 5) {
@@ -161,17 +163,17 @@ __global__ void __launch_bounds__(192, 1)
         if (ok) ok = issue_qk(0);
         for (int j = 0; ok && j < n_tiles; ++j) {
             if (j + 1 < n_tiles && !issue_qk(j + 1)) break;
-            if (!mbar_wait(smem_u32(p_ready), j & 1, p.status)) break;
+            if (!mbar_wait(smem_u32(&p_ready[j & 1]), (j >> 1) & 1, p.status)) break;
             tc_fence_after();
             if (lane == 0) {
                 const uint32_t va = smem_u32(smem + OFF_KV + (j % NST) * STAGE + BOX);
                 for (int hh = 0; hh < HPG; ++hh)
 #pragma unroll
                     for (int kk = 0; kk < TK / 16; ++kk)
-                        umma_ts(tmem + T_O + hh * 64, tmem + T_P + kk * 8,
+                        umma_ts(tmem + T_O + hh * 64, tmem + T_P + (j & 1) * 64 + kk * 8,
                                 smem_desc_sw128(va + hh * BOX + kk * 2048, BOX, 1024), idesc_pv, (j | kk) != 0);
                 umma_commit(smem_u32(&kv_empty[j % NST]));
-                umma_commit(smem_u32(o_ready));
+                umma_commit(smem_u32(&o_ready[j & 1]));
             }
             __syncwarp();
         }
@@ -209,26 +211,29 @@ __global__ void __launch_bounds__(192, 1)
                 m_use = m_new;
             } else if (m_new > m_ref + 8.0f) {
                 resc = true;
-                alpha = exp2f(m_ref - m_new);
+                alpha = fast_exp2(m_ref - m_new);
                 m_use = m_new;
             }
             float rs = 0.f;
             uint32_t pk[TK / 2];
 #pragma unroll
             for (int c = 0; c < TK; c += 2) {
-                const float p0 = m_use == -INFINITY ? 0.f : exp2f(__uint_as_float(sr[c]) - m_use);
-                const float p1 = m_use == -INFINITY ? 0.f : exp2f(__uint_as_float(sr[c + 1]) - m_use);
+                const float p0 = m_use == -INFINITY ? 0.f : fast_exp2(__uint_as_float(sr[c]) - m_use);
+                const float p1 = m_use == -INFINITY ? 0.f : fast_exp2(__uint_as_float(sr[c + 1]) - m_use);
                 rs += p0 + p1;
                 pk[c / 2] = pack_bf16x2(p0, p1);
             }
             l = (resc ? l * alpha : l) + rs;
             m_ref = m_use;
-            // P(j-1) and O must be released by PV(j-1) before P(j) is written and O rescaled
-            if (ok && j >= 1) ok = mbar_wait(smem_u32(o_ready), (j - 1) & 1, p.status);
+            // P buffer j&1 was last read by PV(j-2); O may only be rescaled after PV(j-1)
+            if (ok && j >= 2) ok = mbar_wait(smem_u32(&o_ready[j & 1]), ((j >> 1) - 1) & 1, p.status);
+            const bool any_resc = __any_sync(0xffffffffu, resc);
+            if (any_resc && ok && j >= 1)
+                ok = mbar_wait(smem_u32(&o_ready[(j - 1) & 1]), ((j - 1) >> 1) & 1, p.status);
             tc_fence_after();
 #pragma unroll
-            for (int c0 = 0; c0 < TK / 2; c0 += 16) tmem_st16(tmem + lane_base + T_P + c0, pk + c0);
-            if (__any_sync(0xffffffffu, resc)) {
+            for (int c0 = 0; c0 < TK / 2; c0 += 16) tmem_st16(tmem + lane_base + T_P + (j & 1) * 64 + c0, pk + c0);
+            if (any_resc) {
                 for (int c0 = 0; c0 < 64 * HPG; c0 += 16) {
                     uint32_t o[16];
                     tmem_ld16(tmem + lane_base + T_O + c0, o);
@@ -241,9 +246,9 @@ __global__ void __launch_bounds__(192, 1)
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(p_ready));
+            if (lane == 0) mbar_arrive(smem_u32(&p_ready[j & 1]));
         }
-        if (ok) ok = mbar_wait(smem_u32(o_ready), (n_tiles - 1) & 1, p.status);
+        if (ok) ok = mbar_wait(smem_u32(&o_ready[(n_tiles - 1) & 1]), ((n_tiles - 1) >> 1) & 1, p.status);
         if (!ok) {
             s_abort = 1;
         } else {

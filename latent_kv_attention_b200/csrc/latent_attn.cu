@@ -47,7 +47,7 @@ constexpr int OFF_Q = 0;
 constexpr int OFF_KV = OFF_Q + Q_BYTES;
 constexpr int OFF_X = OFF_KV + NST * STAGE;
 constexpr int OFF_BAR = OFF_X + 2 * XBUF;
-constexpr int SMEM = 1024 + OFF_BAR + 256;
+constexpr int SMEM = 1024 + OFF_BAR + 512;
 // tensor memory columns
 constexpr uint32_t T_O = 0;          // 256 fp32 columns: this rank's half of the output
 constexpr uint32_t T_S = 256;        // 2 x NT fp32 score partials
@@ -112,13 +112,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
     uint64_t* q_full = bars + 0;
     uint64_t* kv_full = bars + 1;
-    uint64_t* kv_empty = bars + 1 + NST;
-    uint64_t* s_ready = bars + 1 + 2 * NST;
-    uint64_t* p_ready = s_ready + 2;
-    uint64_t* o_ready = p_ready + 2;
-    uint64_t* xfull = o_ready + 1;
-    uint64_t* xempty = xfull + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xempty + 2);
+    uint64_t* kv_empty = kv_full + NST;
+    uint64_t* s_ready = kv_empty + NST;   // [2] QK(j) done (buffer j&1)
+    uint64_t* s_free = s_ready + 2;       // [2] S(j) loaded by all four softmax warps
+    uint64_t* p_ready = s_free + 2;       // [2] P(j) written by all four softmax warps
+    uint64_t* o_ready = p_ready + 2;      // [2] PV(j) done
+    uint64_t* xfull = o_ready + 2;        // [2][4] the peer's partial scores of warp w's rows arrived
+    uint64_t* xempty = xfull + 8;         // [2][4] the peer has consumed this CTA's partial for warp w's rows
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xempty + 8);
     __shared__ int s_abort;
 
     const uint32_t rank = cluster_rank();
@@ -146,15 +147,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(smem_u32(&s_ready[i]), 1);
+            mbar_init(smem_u32(&s_free[i]), 4);
             mbar_init(smem_u32(&p_ready[i]), 4);
+            mbar_init(smem_u32(&o_ready[i]), 1);
+        }
+        for (int i = 0; i < 8; ++i) {
             mbar_init(smem_u32(&xfull[i]), 1);
             mbar_init(smem_u32(&xempty[i]), 1);
         }
-        mbar_init(smem_u32(o_ready), 1);
         fence_barrier_init();
         // the first two exchange buffers are open for the peer's partial scores
-        mbar_arrive_expect_tx(smem_u32(&xfull[0]), XBUF);
-        mbar_arrive_expect_tx(smem_u32(&xfull[1]), XBUF);
+        for (int i = 0; i < 8; ++i) mbar_arrive_expect_tx(smem_u32(&xfull[i]), XBUF / 4);
     }
     if (warp == 5) {
         tmem_alloc(tmem_slot, 512);
@@ -197,106 +200,120 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         }
     } else if (n_tiles > 0 && warp == 5) {
         // ------------------------------- MMA issuer -------------------------------
+        // Order: QK(0), QK(1), then per step j: QK(j) and PV(j-2).  QK(j) only needs the softmax
+        // warps to have loaded S(j-2) (s_free), so score tiles run two ahead of P*V.
         constexpr uint32_t idesc_qk = idesc_bf16_f32(128, NT, false, false);
         constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
         bool ok = mbar_wait(smem_u32(q_full), 0, p.status);
-        auto issue_qk = [&](int j) -> bool {
-            const int s = j % NST;
-            if (!mbar_wait(smem_u32(&kv_full[s]), (j / NST) & 1, p.status)) return false;
-            uint8_t* st = smem + OFF_KV + s * STAGE;
-            const int nvalid = min(NT, kend - (kbeg + j * NT));
-            if (nvalid < NT) {
-                // rows past the last visible key may hold anything (even NaN): zero them so
-                // that P = 0 times V contributes exactly 0
-                const int rows = NT - nvalid;
-                for (int idx = lane; idx < nkb * rows * 8; idx += 32) {
-                    const int kb = idx / (rows * 8), rr = (idx / 8) % rows, c = idx % 8;
-                    *reinterpret_cast<uint4*>(st + kb * BOX + (nvalid + rr) * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+        for (int j = 0; ok && j < n_tiles + 2; ++j) {
+            if (j < n_tiles) {
+                const int s = j % NST;
+                if (!mbar_wait(smem_u32(&kv_full[s]), (j / NST) & 1, p.status)) break;
+                uint8_t* st = smem + OFF_KV + s * STAGE;
+                const int nvalid = min(NT, kend - (kbeg + j * NT));
+                if (nvalid < NT) {
+                    // rows past the last visible key may hold anything (even NaN): zero them so
+                    // that P = 0 times V contributes exactly 0
+                    const int rows = NT - nvalid;
+                    for (int idx = lane; idx < nkb * rows * 8; idx += 32) {
+                        const int kb = idx / (rows * 8), rr = (idx / 8) % rows, c = idx % 8;
+                        *reinterpret_cast<uint4*>(st + kb * BOX + (nvalid + rr) * 128 + c * 16) =
+                            make_uint4(0, 0, 0, 0);
+                    }
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
                 }
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                if (j >= 2 && !mbar_wait(smem_u32(&s_free[j & 1]), ((j >> 1) - 1) & 1, p.status)) break;
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t qa = smem_u32(smem + OFF_Q);
+                    const uint32_t kva = smem_u32(st);
+                    for (int kb = 0; kb < nkb; ++kb)
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            umma_ss(tmem + T_S + (j & 1) * NT, smem_desc_sw128(qa + kb * 16384 + k * 32, 16, 1024),
+                                    smem_desc_sw128(kva + kb * BOX + k * 32, 16, 1024), idesc_qk, (kb | k) != 0);
+                    umma_commit(smem_u32(&s_ready[j & 1]));
+                }
                 __syncwarp();
             }
-            tc_fence_after();
-            if (lane == 0) {
-                const uint32_t qa = smem_u32(smem + OFF_Q);
-                const uint32_t kva = smem_u32(st);
-                for (int kb = 0; kb < nkb; ++kb)
+            if (j >= 2) {
+                const int i = j - 2;
+                if (!mbar_wait(smem_u32(&p_ready[i & 1]), (i >> 1) & 1, p.status)) break;
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t va = smem_u32(smem + OFF_KV + (i % NST) * STAGE);
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        umma_ss(tmem + T_S + (j & 1) * NT, smem_desc_sw128(qa + kb * 16384 + k * 32, 16, 1024),
-                                smem_desc_sw128(kva + kb * BOX + k * 32, 16, 1024), idesc_qk, (kb | k) != 0);
-                umma_commit(smem_u32(&s_ready[j & 1]));
+                    for (int kk = 0; kk < NT / 16; ++kk)
+                        umma_ts(tmem + T_O, tmem + T_P + (i & 1) * (NT / 2) + kk * 8,
+                                smem_desc_sw128(va + kk * 2048, BOX, 1024), idesc_pv, (i | kk) != 0);
+                    umma_commit(smem_u32(&kv_empty[i % NST]));
+                    umma_commit(smem_u32(&o_ready[i & 1]));
+                }
+                __syncwarp();
             }
-            __syncwarp();
-            return true;
-        };
-        if (ok) ok = issue_qk(0);
-        for (int i = 0; ok && i < n_tiles; ++i) {
-            if (i + 1 < n_tiles && !issue_qk(i + 1)) break;
-            if (!mbar_wait(smem_u32(&p_ready[i & 1]), (i >> 1) & 1, p.status)) break;
-            tc_fence_after();
-            if (lane == 0) {
-                const uint32_t va = smem_u32(smem + OFF_KV + (i % NST) * STAGE);
-#pragma unroll
-                for (int kk = 0; kk < NT / 16; ++kk)
-                    umma_ts(tmem + T_O, tmem + T_P + (i & 1) * (NT / 2) + kk * 8,
-                            smem_desc_sw128(va + kk * 2048, BOX, 1024), idesc_pv, (i | kk) != 0);
-                umma_commit(smem_u32(&kv_empty[i % NST]));
-                umma_commit(smem_u32(o_ready));
-            }
-            __syncwarp();
         }
     } else if (warp < 4) {
         // ------------------------- softmax / exchange warps -------------------------
+        // Each warp owns 32 head rows and its own exchange barriers, so the four warps never wait
+        // for one another.  The partial scores of tile i+1 are sent to the peer before tile i is
+        // consumed, so the peer's copy is usually in place when it is needed.
         const int h = warp * 32 + lane;  // head row == TMEM lane
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        const uint32_t xloc[2] = {smem_u32(smem + OFF_X), smem_u32(smem + OFF_X + XBUF)};
-        const uint32_t xrem[2] = {mapa_peer(xloc[0] + h * XROW, peer), mapa_peer(xloc[1] + h * XROW, peer)};
-        const uint32_t xfull_rem[2] = {mapa_peer(smem_u32(&xfull[0]), peer), mapa_peer(smem_u32(&xfull[1]), peer)};
-        const uint32_t xempty_rem[2] = {mapa_peer(smem_u32(&xempty[0]), peer),
-                                        mapa_peer(smem_u32(&xempty[1]), peer)};
+        const uint32_t xrem[2] = {mapa_peer(smem_u32(smem + OFF_X) + h * XROW, peer),
+                                  mapa_peer(smem_u32(smem + OFF_X + XBUF) + h * XROW, peer)};
+        const uint32_t xfull_rem[2] = {mapa_peer(smem_u32(&xfull[0 * 4 + warp]), peer),
+                                       mapa_peer(smem_u32(&xfull[1 * 4 + warp]), peer)};
+        const uint32_t xempty_rem[2] = {mapa_peer(smem_u32(&xempty[0 * 4 + warp]), peer),
+                                        mapa_peer(smem_u32(&xempty[1 * 4 + warp]), peer)};
         const int sw = h & 7;
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
-        // A failed (timed-out) wait clears `ok`; the loop then keeps its shape without waiting, so that
-        // every warp still reaches the named barrier below and the CTA pair can exit.
-        for (int i = 0; i < n_tiles; ++i) {
-            const int x = i & 1;
-            if (ok) ok = mbar_wait(smem_u32(&s_ready[x]), (i >> 1) & 1, p.status);
+        uint32_t cur[NT], nxt[NT];
+        // load S(j) into regs, release the TMEM buffer, send the partial to the peer
+        auto fetch_and_send = [&](int j, uint32_t* dst) {
+            const int x = j & 1;
+            if (ok) ok = mbar_wait(smem_u32(&s_ready[x]), (j >> 1) & 1, p.status);
             tc_fence_after();
-            uint32_t sr[NT];
-            tmem_ld16(tmem + lane_base + T_S + x * NT, sr);
-            tmem_ld16(tmem + lane_base + T_S + x * NT + 16, sr + 16);
+            tmem_ld16(tmem + lane_base + T_S + x * NT, dst);
+            tmem_ld16(tmem + lane_base + T_S + x * NT + 16, dst + 16);
             tmem_ld_wait();
-            // ---- exchange the partial scores with the peer CTA ----
-            if (ok && i >= 2) ok = mbar_wait_cluster(smem_u32(&xempty[x]), ((i >> 1) - 1) & 1, p.status);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&s_free[x]));
+            if (ok && j >= 2) ok = mbar_wait_cluster(smem_u32(&xempty[x * 4 + warp]), ((j >> 1) - 1) & 1, p.status);
 #pragma unroll
             for (int c = 0; c < NT / 4; ++c)
-                st_async_v4(xrem[x] + ((c ^ sw) << 4), sr[4 * c], sr[4 * c + 1], sr[4 * c + 2], sr[4 * c + 3],
+                st_async_v4(xrem[x] + ((c ^ sw) << 4), dst[4 * c], dst[4 * c + 1], dst[4 * c + 2], dst[4 * c + 3],
                             xfull_rem[x]);
-            if (ok) ok = mbar_wait_cluster(smem_u32(&xfull[x]), (i >> 1) & 1, p.status);
+        };
+        if (n_tiles > 0) fetch_and_send(0, cur);
+        for (int i = 0; i < n_tiles; ++i) {
+            const int x = i & 1;
+            if (i + 1 < n_tiles) fetch_and_send(i + 1, nxt);
+            // ---- the peer's partial of tile i ----
+            if (ok) ok = mbar_wait_cluster(smem_u32(&xfull[x * 4 + warp]), (i >> 1) & 1, p.status);
             float s[NT];
             const uint8_t* xr = smem + OFF_X + x * XBUF + h * XROW;
 #pragma unroll
             for (int c = 0; c < NT / 4; ++c) {
                 const float4 v = *reinterpret_cast<const float4*>(xr + ((c ^ sw) << 4));
-                s[4 * c] = __uint_as_float(sr[4 * c]) + v.x;
-                s[4 * c + 1] = __uint_as_float(sr[4 * c + 1]) + v.y;
-                s[4 * c + 2] = __uint_as_float(sr[4 * c + 2]) + v.z;
-                s[4 * c + 3] = __uint_as_float(sr[4 * c + 3]) + v.w;
+                s[4 * c] = __uint_as_float(cur[4 * c]) + v.x;
+                s[4 * c + 1] = __uint_as_float(cur[4 * c + 1]) + v.y;
+                s[4 * c + 2] = __uint_as_float(cur[4 * c + 2]) + v.z;
+                s[4 * c + 3] = __uint_as_float(cur[4 * c + 3]) + v.w;
             }
-            named_barrier(1, 128);  // every row has read exchange buffer x
-            if (threadIdx.x == 0 && i + 2 < n_tiles) {
-                mbar_arrive_expect_tx(smem_u32(&xfull[x]), XBUF);  // reopen it for tile i + 2 ...
-                remote_arrive(xempty_rem[x]);                      // ... and tell the peer
+            __syncwarp();
+            if (lane == 0 && i + 2 < n_tiles) {
+                mbar_arrive_expect_tx(smem_u32(&xfull[x * 4 + warp]), XBUF / 4);  // reopen for tile i + 2 ...
+                remote_arrive(xempty_rem[x]);                                     // ... and tell the peer
             }
             // ---- mask, online softmax ----
             const int k0 = kbeg + i * NT;
             float mx = -INFINITY;
 #pragma unroll
             for (int j = 0; j < NT; ++j) {
-                const int kp = k0 + j;
-                s[j] = (kp < kend) ? s[j] * p.scale_log2 : -INFINITY;
+                s[j] = (k0 + j < kend) ? s[j] * p.scale_log2 : -INFINITY;
                 mx = fmaxf(mx, s[j]);
             }
             const float m_new = fmaxf(m_ref, mx);
@@ -307,25 +324,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                 m_use = m_new;
             } else if (m_new > m_ref + RESCALE_THRESHOLD) {
                 resc = true;
-                alpha = exp2f(m_ref - m_new);
+                alpha = fast_exp2(m_ref - m_new);
                 m_use = m_new;
             }
             float rs = 0.f;
             uint32_t pk[NT / 2];
 #pragma unroll
             for (int j = 0; j < NT; j += 2) {
-                const float p0 = m_use == -INFINITY ? 0.f : exp2f(s[j] - m_use);
-                const float p1 = m_use == -INFINITY ? 0.f : exp2f(s[j + 1] - m_use);
+                const float p0 = m_use == -INFINITY ? 0.f : fast_exp2(s[j] - m_use);
+                const float p1 = m_use == -INFINITY ? 0.f : fast_exp2(s[j + 1] - m_use);
                 rs += p0 + p1;
                 pk[j / 2] = pack_bf16x2(p0, p1);
             }
             l = (resc ? l * alpha : l) + rs;
             m_ref = m_use;
-            tmem_st16(tmem + lane_base + T_P + x * (NT / 2), pk);
-            tmem_st_wait();
-            // ---- PV(i-1) must be complete before O is rescaled / P(i) consumed ----
-            if (ok && i >= 1) ok = mbar_wait(smem_u32(o_ready), (i - 1) & 1, p.status);
+            // P buffer x was last read by PV(i-2)
+            if (ok && i >= 2) ok = mbar_wait(smem_u32(&o_ready[x]), ((i >> 1) - 1) & 1, p.status);
             if (__any_sync(0xffffffffu, resc)) {
+                // O may only be rescaled once PV(i-1) has been accumulated into it
+                if (ok && i >= 1) ok = mbar_wait(smem_u32(&o_ready[(i - 1) & 1]), ((i - 1) >> 1) & 1, p.status);
                 tc_fence_after();
                 for (int c0 = 0; c0 < 256; c0 += 16) {
                     uint32_t o[16];
@@ -335,15 +352,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                     for (int q = 0; q < 16; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
                     tmem_st16(tmem + lane_base + T_O + c0, o);
                 }
-                tmem_st_wait();
             }
+            tc_fence_after();
+            tmem_st16(tmem + lane_base + T_P + x * (NT / 2), pk);
+            tmem_st_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&p_ready[x]));
+#pragma unroll
+            for (int j = 0; j < NT; ++j) cur[j] = nxt[j];
         }
         if (!ok) s_abort = 1;
         // ---- epilogue: normalise this rank's 256 output columns ----
-        if (ok && n_tiles > 0 && mbar_wait(smem_u32(o_ready), (n_tiles - 1) & 1, p.status)) {
+        const int last = n_tiles - 1;
+        if (ok && n_tiles > 0 && mbar_wait(smem_u32(&o_ready[last & 1]), (last >> 1) & 1, p.status)) {
             tc_fence_after();
             const float inv_l = l > 0.f ? 1.f / l : 0.f;
             const int HPG = p.h_q / p.g;

@@ -134,6 +134,13 @@ WORKLOADS = {
                                  L_lo=4096, L_hi=4096, causal=True),
     "latent_decode_4k_sq2": dict(kind="latent", seed=4, B=64, h_q=128, g=8, d_h=128, r_kv=512, d_r=64, s_q=2,
                                  L_lo=4096, L_hi=4096, causal=True),
+    # half the batch: the small case for full ncu captures of the latent kernels (latent cache 151 MB > L2)
+    "latent_decode_4k_sq1_b32": dict(kind="latent", seed=4, B=32, h_q=128, g=8, d_h=128, r_kv=512, d_r=64, s_q=1,
+                                     L_lo=4096, L_hi=4096, causal=True),
+    "latent_expanded_4k_sq2_b16": dict(kind="latent", seed=4, B=16, h_q=128, g=8, d_h=128, r_kv=512, d_r=64, s_q=2,
+                                       L_lo=4096, L_hi=4096, causal=True),
+    "gta_prefill_4k_b2": dict(kind="gta", seed=3, B=2, G=3, H=12, d_qk=64, d_v=64, s_q=4096, L_lo=4096, L_hi=4096,
+                              causal=True),
     # the same latent inputs, run through the per-group GQA path after the one-time cache expansion
     "latent_expanded_4k_sq1": dict(kind="latent", seed=4, B=64, h_q=128, g=8, d_h=128, r_kv=512, d_r=64, s_q=1,
                                    L_lo=4096, L_hi=4096, causal=True),
