@@ -85,6 +85,25 @@ LKA_API lka_status_t gqa_attn(const void *q, const void *k, const void *v, const
                       float *lse, int B, int h_q, int h_kv, int s_q, int d_h, int Lmax, int causal, float scale,
                       lka_dtype_t dtype, void *ws, size_t ws_bytes, void *stream);
 
+/* gqa_attn for callers that cannot allocate device memory.  No counterpart in
+ * the papers: it exists for callers that are handed only their input and
+ * output buffers (a plugin or custom operator inside another runtime) or run
+ * where the host framework forbids device allocations, and so cannot provide
+ * the workspace gqa_attn takes.  Same arguments, result and dtypes as
+ * gqa_attn minus the workspace: the split-KV scratch lives in a 16 MiB device
+ * array inside the library (held by every GPU that loads the library until
+ * the process exits).  This call allocates nothing.  Its first call on a
+ * device looks up that array's device address (cudaGetSymbolAddress), so make
+ * the first call on each device before any stream capture.  Returns
+ * LKA_ERR_WORKSPACE when the workspace gqa_attn_workspace_size reports for the
+ * sizes exceeds 16 MiB.  All calls share the one array: calls that overlap on
+ * the GPU (other streams, other host threads) race and must be serialised by
+ * the caller.  Device-side status flags (LKA_ERR_TIMEOUT, LKA_ERR_BAD_LENGTH)
+ * are not reported by this variant. */
+LKA_API lka_status_t gqa_attn_noalloc(const void *q, const void *k, const void *v, const int32_t *cache_lens,
+                              void *out, float *lse, int B, int h_q, int h_kv, int s_q, int d_h, int Lmax,
+                              int causal, float scale, lka_dtype_t dtype, void *stream);
+
 /* ------------------------------------------------------------------------ */
 /* (b) GQLA MQA-absorbed latent attention  [GQLA sec. 1, sec. 3.1 eq. (1),  */
 /*     Figure 2(b)]                                                         */

@@ -40,6 +40,7 @@ _FP = ctypes.POINTER(ctypes.c_float)
 SIGNATURES = {
     "gqa_attn_workspace_size": (_Z, [_I] * 6),
     "gqa_attn": (_I, [_P] * 6 + [_I] * 7 + [_F, _I, _P, _Z, _P]),
+    "gqa_attn_noalloc": (_I, [_P] * 6 + [_I] * 7 + [_F, _I, _P]),
     "latent_absorbed_attn_workspace_size": (_Z, [_I] * 8),
     "latent_absorbed_attn": (_I, [_P] * 8 + [_I] * 9 + [_F, _I, _P, _Z, _P]),
     "latent_expand_gqa_attn_workspace_size": (_Z, [_I] * 7),
