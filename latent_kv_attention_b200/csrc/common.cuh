@@ -124,6 +124,25 @@ __device__ __forceinline__ float fast_exp2(float x) {
     return y;
 }
 
+// Pairwise (tree) max and sum of N register values: log2(N) dependent steps instead of N,
+// so a single warp per scheduler is not bound by the add/max latency chain.
+template <int N>
+__device__ __forceinline__ float tree_max(const float* v) {
+    if constexpr (N == 1) {
+        return v[0];
+    } else {
+        return fmaxf(tree_max<N / 2>(v), tree_max<N - N / 2>(v + N / 2));
+    }
+}
+template <int N>
+__device__ __forceinline__ float tree_sum(const float* v) {
+    if constexpr (N == 1) {
+        return v[0];
+    } else {
+        return tree_sum<N / 2>(v) + tree_sum<N - N / 2>(v + N / 2);
+    }
+}
+
 // ---- element conversion -------------------------------------------------------
 // Unpack 8 bf16 values held in 16 bytes into fp32 (exact).
 __device__ __forceinline__ void bf16x8_to_f32(const uint4 u, float* f) {

@@ -31,10 +31,12 @@ namespace lka {
 template <int NR>
 struct ExpCfg {
     static constexpr int TK = 128;                 // tokens per tile (MMA M)
-    static constexpr int NST = 2;
+    static constexpr int NST = 2;                  // depth of the key ring and of the value ring
     static constexpr int BOX = TK * 128;           // 128 tokens x 64 bf16
     static constexpr int Q_BYTES = 3 * NR * 128;   // Q^T: 3 K-blocks (q_c 0..63, 64..127, q_r)
-    static constexpr int STAGE = 5 * BOX;          // kc x2, kr, vc x2
+    static constexpr int KSTAGE = 3 * BOX;         // kc x2, kr (released after S^T = K Q^T)
+    static constexpr int VSTAGE = 2 * BOX;         // vc x2 (released after O^T += V^T P^T)
+    static constexpr int STAGE = KSTAGE + VSTAGE;
     static constexpr int SC_BYTES = NR * TK * 4;   // transposed scores
     static constexpr int PT_BYTES = 2 * NR * 128;  // P^T: 2 K-blocks of 64 tokens
     static constexpr int OFF_Q = 0;
@@ -61,9 +63,11 @@ __global__ void __launch_bounds__(192, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* q_full = bars;
-    uint64_t* kv_full = bars + 1;
-    uint64_t* kv_empty = kv_full + NST;
-    uint64_t* s_ready = kv_empty + NST;  // [2] QK(j) done
+    uint64_t* k_full = bars + 1;
+    uint64_t* k_empty = k_full + NST;
+    uint64_t* v_full = k_empty + NST;
+    uint64_t* v_empty = v_full + NST;
+    uint64_t* s_ready = v_empty + NST;   // [2] QK(j) done
     uint64_t* s_free = s_ready + 2;      // [2] S(j) loaded by the softmax warps
     uint64_t* p_ready = s_free + 2;      // [2] P^T(j) written
     uint64_t* o_ready = p_ready + 2;     // [2] PV(j) done
@@ -87,8 +91,10 @@ __global__ void __launch_bounds__(192, 1)
         s_abort = 0;
         mbar_init(smem_u32(q_full), 1);
         for (int s = 0; s < NST; ++s) {
-            mbar_init(smem_u32(&kv_full[s]), 1);
-            mbar_init(smem_u32(&kv_empty[s]), 1);
+            mbar_init(smem_u32(&k_full[s]), 1);
+            mbar_init(smem_u32(&k_empty[s]), 1);
+            mbar_init(smem_u32(&v_full[s]), 1);
+            mbar_init(smem_u32(&v_empty[s]), 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(smem_u32(&s_ready[i]), 1);
@@ -117,47 +123,65 @@ __global__ void __launch_bounds__(192, 1)
             tma_load_2d(qd, &tm_qc, 0, qrow, qb);
             tma_load_2d(qd + NR * 128, &tm_qc, 64, qrow, qb);
             tma_load_2d(qd + 2 * NR * 128, &tm_qr, 0, qrow, qb);
-            int issued = 0;
-            for (int i = 0; i < n_tiles; ++i) {
+            // issue order K(0), then per tile i: K(i+1), V(i); key tiles are released as soon as
+            // their score MMAs complete, value tiles after their P*V MMAs
+            int k_issued = 0, v_issued = 0;
+            bool ok = true;
+            auto issue_k = [&](int i) {
                 const int s = i % NST;
-                if (i >= NST && !mbar_wait(smem_u32(&kv_empty[s]), ((i / NST) - 1) & 1, p.status)) {
-                    s_abort = 1;
-                    break;
-                }
-                if (*(volatile int*)&s_abort) break;
-                const uint32_t fb = smem_u32(&kv_full[s]);
-                mbar_arrive_expect_tx(fb, C::STAGE);
+                if (i >= NST && !mbar_wait(smem_u32(&k_empty[s]), ((i / NST) - 1) & 1, p.status)) return false;
+                const uint32_t fb = smem_u32(&k_full[s]);
+                mbar_arrive_expect_tx(fb, C::KSTAGE);
                 const uint32_t d = smem_u32(smem + C::OFF_KV + s * C::STAGE);
                 const int k0 = kbeg + i * TK;
                 const int yg = (b * p.g + grp) * p.Lmax + k0;
                 tma_load_2d(d, &tm_kc, 0, yg, fb);
                 tma_load_2d(d + C::BOX, &tm_kc, 64, yg, fb);
                 tma_load_2d(d + 2 * C::BOX, &tm_kr, 0, b * p.Lmax + k0, fb);
-                tma_load_2d(d + 3 * C::BOX, &tm_vc, 0, yg, fb);
-                tma_load_2d(d + 4 * C::BOX, &tm_vc, 64, yg, fb);
-                ++issued;
+                ++k_issued;
+                return true;
+            };
+            auto issue_v = [&](int i) {
+                const int s = i % NST;
+                if (i >= NST && !mbar_wait(smem_u32(&v_empty[s]), ((i / NST) - 1) & 1, p.status)) return false;
+                const uint32_t fb = smem_u32(&v_full[s]);
+                mbar_arrive_expect_tx(fb, C::VSTAGE);
+                const uint32_t d = smem_u32(smem + C::OFF_KV + s * C::STAGE + C::KSTAGE);
+                const int yg = (b * p.g + grp) * p.Lmax + kbeg + i * TK;
+                tma_load_2d(d, &tm_vc, 0, yg, fb);
+                tma_load_2d(d + C::BOX, &tm_vc, 64, yg, fb);
+                ++v_issued;
+                return true;
+            };
+            ok = issue_k(0);
+            for (int i = 0; ok && i < n_tiles; ++i) {
+                if (*(volatile int*)&s_abort) break;
+                if (i + 1 < n_tiles) ok = issue_k(i + 1);
+                if (ok) ok = issue_v(i);
             }
-            for (int i = issued - 1; i >= 0 && i >= issued - NST; --i)
-                mbar_wait(smem_u32(&kv_full[i % NST]), (i / NST) & 1, p.status);
+            if (!ok) s_abort = 1;
+            for (int i = k_issued - 1; i >= 0 && i >= k_issued - NST; --i)
+                mbar_wait(smem_u32(&k_full[i % NST]), (i / NST) & 1, p.status);
+            for (int i = v_issued - 1; i >= 0 && i >= v_issued - NST; --i)
+                mbar_wait(smem_u32(&v_full[i % NST]), (i / NST) & 1, p.status);
             mbar_wait(qb, 0, p.status);
         }
     } else if (warp == 5) {
         // -------------------------------- MMA issuer --------------------------------
-        // per step j: QK(j) (needs S(j-2) loaded by the softmax warps) and PV(j-1); with two
-        // KV stages, QK(j) also needs PV(j-2) to have released its stage
+        // per step j: QK(j) (needs S(j-2) loaded by the softmax warps) and PV(j-1)
         constexpr uint32_t idesc_qk = idesc_bf16_f32(128, NR, false, false);
         constexpr uint32_t idesc_pv = idesc_bf16_f32(128, NR, true, false);
         bool ok = mbar_wait(smem_u32(q_full), 0, p.status);
         for (int j = 0; ok && j < n_tiles + 1; ++j) {
             if (j < n_tiles) {
                 const int s = j % NST;
-                if (!mbar_wait(smem_u32(&kv_full[s]), (j / NST) & 1, p.status)) break;
+                if (!mbar_wait(smem_u32(&k_full[s]), (j / NST) & 1, p.status)) break;
                 uint8_t* st = smem + C::OFF_KV + s * C::STAGE;
                 const int nvalid = min(TK, kend - (kbeg + j * TK));
                 if (nvalid < TK) {
-                    // tokens past the key range may hold anything (even NaN): zero them so P = 0 adds nothing
+                    // keys past the key range may hold anything (even NaN): zero them
                     const int rows = TK - nvalid;
-                    for (int idx = lane; idx < 5 * rows * 8; idx += 32) {
+                    for (int idx = lane; idx < 3 * rows * 8; idx += 32) {
                         const int bx = idx / (rows * 8), rr = (idx / 8) % rows, c = idx % 8;
                         *reinterpret_cast<uint4*>(st + bx * C::BOX + (nvalid + rr) * 128 + c * 16) =
                             make_uint4(0, 0, 0, 0);
@@ -176,22 +200,38 @@ __global__ void __launch_bounds__(192, 1)
                             umma_ss(tmem + C::T_S + (j & 1) * NR, smem_desc_sw128(ka + kb * C::BOX + k * 32, 16, 1024),
                                     smem_desc_sw128(qa + kb * NR * 128 + k * 32, 16, 1024), idesc_qk, (kb | k) != 0);
                     umma_commit(smem_u32(&s_ready[j & 1]));
+                    umma_commit(smem_u32(&k_empty[s]));
                 }
                 __syncwarp();
             }
             if (j >= 1) {
                 const int i = j - 1;
+                const int sv = i % NST;
+                if (!mbar_wait(smem_u32(&v_full[sv]), (i / NST) & 1, p.status)) break;
+                uint8_t* vt = smem + C::OFF_KV + sv * C::STAGE + C::KSTAGE;
+                const int nvalid = min(TK, kend - (kbeg + i * TK));
+                if (nvalid < TK) {
+                    // values past the key range may hold anything (even NaN): zero them so P = 0 adds nothing
+                    const int rows = TK - nvalid;
+                    for (int idx = lane; idx < 2 * rows * 8; idx += 32) {
+                        const int bx = idx / (rows * 8), rr = (idx / 8) % rows, c = idx % 8;
+                        *reinterpret_cast<uint4*>(vt + bx * C::BOX + (nvalid + rr) * 128 + c * 16) =
+                            make_uint4(0, 0, 0, 0);
+                    }
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                }
                 if (!mbar_wait(smem_u32(&p_ready[i & 1]), (i >> 1) & 1, p.status)) break;
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t va = smem_u32(smem + C::OFF_KV + (i % NST) * C::STAGE + 3 * C::BOX);
+                    const uint32_t va = smem_u32(vt);
                     const uint32_t pa = smem_u32(smem + C::OFF_PT + (i & 1) * C::PT_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < TK / 16; ++kk)
                         umma_ss(tmem + C::T_O, smem_desc_sw128(va + kk * 2048, C::BOX, 1024),
                                 smem_desc_sw128(pa + (kk / 4) * NR * 128 + (kk % 4) * 32, 16, 1024), idesc_pv,
                                 (i | kk) != 0);
-                    umma_commit(smem_u32(&kv_empty[i % NST]));
+                    umma_commit(smem_u32(&v_empty[sv]));
                     umma_commit(smem_u32(&o_ready[i & 1]));
                 }
                 __syncwarp();
@@ -238,12 +278,9 @@ __global__ void __launch_bounds__(192, 1)
                 const float4 a = *reinterpret_cast<const float4*>(sc + r * TK + 8 * c8);
                 const float4 bq = *reinterpret_cast<const float4*>(sc + r * TK + 8 * c8 + 4);
                 float s[8] = {a.x, a.y, a.z, a.w, bq.x, bq.y, bq.z, bq.w};
-                float mx = -INFINITY;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    s[e] = (k0 + 8 * c8 + e < rend) ? s[e] * p.scale_log2 : -INFINITY;
-                    mx = fmaxf(mx, s[e]);
-                }
+                for (int e = 0; e < 8; ++e) s[e] = (k0 + 8 * c8 + e < rend) ? s[e] * p.scale_log2 : -INFINITY;
+                float mx = tree_max<8>(s);
 #pragma unroll
                 for (int m = 8; m >= 1; m /= 2) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
                 const float m_new = fmaxf(m_ref[k], mx);
@@ -254,12 +291,11 @@ __global__ void __launch_bounds__(192, 1)
                     alpha = fast_exp2(m_ref[k] - m_new);
                     m_use = m_new;
                 }
-                float pv[8], rs = 0.f;
+                float pv[8];
+                const float m_sub = m_use == -INFINITY ? 0.f : m_use;  // all scores -inf: p = 0
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    pv[e] = m_use == -INFINITY ? 0.f : fast_exp2(s[e] - m_use);
-                    rs += pv[e];
-                }
+                for (int e = 0; e < 8; ++e) pv[e] = fast_exp2(s[e] - m_sub);
+                float rs = tree_sum<8>(pv);
 #pragma unroll
                 for (int m = 8; m >= 1; m /= 2) rs += __shfl_xor_sync(0xffffffffu, rs, m);
                 lsum[k] = lsum[k] * alpha + rs;

@@ -29,6 +29,19 @@
 #include "gqa_decode.h"
 #include "host_util.h"
 
+// Tuning knobs of the build: shared-memory budget of the TMA ring per CTA (KiB) and
+// the number of CTAs per SM the small-row instances are compiled for.
+#ifndef LKA_GQA_STAGE_KB
+#define LKA_GQA_STAGE_KB 96
+#endif
+#ifndef LKA_GQA_MINB
+#define LKA_GQA_MINB 2
+#endif
+// fp32 query values each lane keeps in registers in the score phase
+#ifndef LKA_GQA_QREGS
+#define LKA_GQA_QREGS 64
+#endif
+
 namespace lka {
 
 template <typename T, int D, int RB>
@@ -39,9 +52,9 @@ struct GqaCfg {
     static constexpr int NSEG = D * E / 128;     // 128-byte swizzle segments per row
     static constexpr int SEG_ELEMS = 128 / E;    // elements per segment (TMA box width)
     // lanes per token in the score phase: enough that the query slice held per
-    // lane stays at 64 fp32 registers, never fewer than the rows (so that the
+    // lane stays at LKA_GQA_QREGS fp32 registers, never fewer than the rows (so that the
     // reduce-scatter leaves one row per lane), at most one chunk per lane
-    static constexpr int LPT0 = RB * D / 64 > RB ? RB * D / 64 : RB;
+    static constexpr int LPT0 = RB * D / LKA_GQA_QREGS > RB ? RB * D / LKA_GQA_QREGS : RB;
     static constexpr int LPT1 = LPT0 < CPR ? LPT0 : CPR;
     static constexpr int LPT = LPT1 < 32 ? LPT1 : 32;
     static constexpr int CPL = CPR / LPT;        // chunks per lane
@@ -53,12 +66,14 @@ struct GqaCfg {
     static constexpr int DPLV = D / 32;          // value dims per lane
     static constexpr int MAT_BYTES = T_TILE * D * E;
     static constexpr int STAGE_BYTES = 2 * MAT_BYTES;
-    static constexpr int NSTAGE0 = (96 * 1024) / STAGE_BYTES;
+    static constexpr int NSTAGE0 = (LKA_GQA_STAGE_KB * 1024) / STAGE_BYTES;
     static constexpr int NSTAGE = NSTAGE0 < 2 ? 2 : (NSTAGE0 > 4 ? 4 : NSTAGE0);
     static constexpr int P_BYTES = 4 * TW * RB * 8 + 4 * RB * 4;  // probabilities (stored as pairs) + rescale
     static constexpr int MERGE_BYTES = 4 * RB * D * 4 + 2 * 4 * RB * 4;
     static constexpr int SMEM = 1024 /*align slack*/ + NSTAGE * STAGE_BYTES + P_BYTES + 256 /*barriers*/;
-    static constexpr int MINB = (RB <= 8 && SMEM <= 110 * 1024) ? 2 : 1;  // resident CTAs per SM
+    static constexpr int MINB0 = (RB <= 8 && SMEM <= 110 * 1024) ? 2 : 1;  // resident CTAs per SM
+    static constexpr int MINB = (RB <= 4 && LKA_GQA_MINB > MINB0 && SMEM * LKA_GQA_MINB <= 225 * 1024) ? LKA_GQA_MINB
+                                                                                                    : MINB0;
     static_assert(D * E >= 128 && (D * E) % 128 == 0, "row must be whole 128-byte segments");
     static_assert(LPT >= RB && LPT <= 32 && LPT <= CPR && CPR % LPT == 0, "lane split must own whole chunks");
     static_assert(MERGE_BYTES <= NSTAGE * STAGE_BYTES, "merge scratch reuses the stage ring");

@@ -35,13 +35,17 @@ struct GtaParams {
 };
 
 namespace gta {
-constexpr int TQ = 128, TK = 128, NST = 2;
+constexpr int TQ = 128, TK = 128;
+constexpr int NSK = 4;              // K ring depth: key tiles are released right after S = Q K^T
+constexpr int NSV = 2;              // V ring depth: value tiles live until their P*V MMAs complete
 constexpr int BOX = TK * 128;       // 128 rows x 64 bf16
-constexpr int STAGE = 5 * BOX;      // K_gamma + up to 4 value tiles
+constexpr int VSTAGE = 4 * BOX;     // up to 4 heads' value tiles
 constexpr int OFF_Q = 0;
-constexpr int OFF_KV = BOX;
-constexpr int OFF_BAR = OFF_KV + NST * STAGE;
+constexpr int OFF_K = BOX;
+constexpr int OFF_V = OFF_K + NSK * BOX;
+constexpr int OFF_BAR = OFF_V + NSV * VSTAGE;
 constexpr int SMEM = 1024 + OFF_BAR + 256;
+constexpr int K_LEAD = 2;           // key tiles the producer keeps ahead of the value tiles
 constexpr uint32_t T_O = 0;         // 4 heads x 64 fp32 columns
 constexpr uint32_t T_S = 256;       // 128 fp32 columns
 constexpr uint32_t T_P = 384;       // 2 x 64 columns of bf16 pairs (double-buffered P)
@@ -55,9 +59,11 @@ __global__ void __launch_bounds__(192, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
     uint64_t* q_full = bars;
-    uint64_t* kv_full = bars + 1;
-    uint64_t* kv_empty = kv_full + NST;
-    uint64_t* s_ready = kv_empty + NST;
+    uint64_t* k_full = bars + 1;
+    uint64_t* k_empty = k_full + NSK;
+    uint64_t* v_full = k_empty + NSK;
+    uint64_t* v_empty = v_full + NSV;
+    uint64_t* s_ready = v_empty + NSV;
     uint64_t* s_free = s_ready + 1;
     uint64_t* p_ready = s_free + 1;   // [2] P(j) in buffer j&1 written
     uint64_t* o_ready = p_ready + 2;  // [2] PV(j) done
@@ -79,9 +85,13 @@ __global__ void __launch_bounds__(192, 1)
     if (threadIdx.x == 0) {
         s_abort = 0;
         mbar_init(smem_u32(q_full), 1);
-        for (int s = 0; s < NST; ++s) {
-            mbar_init(smem_u32(&kv_full[s]), 1);
-            mbar_init(smem_u32(&kv_empty[s]), 1);
+        for (int s = 0; s < NSK; ++s) {
+            mbar_init(smem_u32(&k_full[s]), 1);
+            mbar_init(smem_u32(&k_empty[s]), 1);
+        }
+        for (int s = 0; s < NSV; ++s) {
+            mbar_init(smem_u32(&v_full[s]), 1);
+            mbar_init(smem_u32(&v_empty[s]), 1);
         }
         mbar_init(smem_u32(s_ready), 1);
         mbar_init(smem_u32(s_free), 4);
@@ -102,29 +112,45 @@ __global__ void __launch_bounds__(192, 1)
 
     if (warp == 4) {
         // ------------------------------ producer ------------------------------
+        // issue order K(0..K_LEAD-1), then per tile i: K(i + K_LEAD), V(i)
         if (lane == 0) {
             const uint32_t qb = smem_u32(q_full);
             mbar_arrive_expect_tx(qb, BOX);
             tma_load_2d(smem_u32(smem + OFF_Q), &tm_q, 0, (b * p.G + grp) * p.s_q + q0, qb);
-            int issued = 0;
-            for (int i = 0; i < n_tiles; ++i) {
-                const int s = i % NST;
-                if (i >= NST && !mbar_wait(smem_u32(&kv_empty[s]), ((i / NST) - 1) & 1, p.status)) {
-                    s_abort = 1;
-                    break;
-                }
-                if (*(volatile int*)&s_abort) break;
-                const uint32_t fb = smem_u32(&kv_full[s]);
-                mbar_arrive_expect_tx(fb, (1 + HPG) * BOX);
-                const uint32_t d = smem_u32(smem + OFF_KV + s * STAGE);
-                const int k0 = i * TK;
-                tma_load_2d(d, &tm_k, 0, (b * p.G + grp) * p.Lmax + k0, fb);
+            int k_issued = 0, v_issued = 0;
+            bool ok = true;
+            auto issue_k = [&](int i) {
+                const int s = i % NSK;
+                if (i >= NSK && !mbar_wait(smem_u32(&k_empty[s]), ((i / NSK) - 1) & 1, p.status)) return false;
+                const uint32_t fb = smem_u32(&k_full[s]);
+                mbar_arrive_expect_tx(fb, BOX);
+                tma_load_2d(smem_u32(smem + OFF_K + s * BOX), &tm_k, 0, (b * p.G + grp) * p.Lmax + i * TK, fb);
+                ++k_issued;
+                return true;
+            };
+            auto issue_v = [&](int i) {
+                const int s = i % NSV;
+                if (i >= NSV && !mbar_wait(smem_u32(&v_empty[s]), ((i / NSV) - 1) & 1, p.status)) return false;
+                const uint32_t fb = smem_u32(&v_full[s]);
+                mbar_arrive_expect_tx(fb, HPG * BOX);
+                const uint32_t d = smem_u32(smem + OFF_V + s * VSTAGE);
                 for (int hh = 0; hh < HPG; ++hh)
-                    tma_load_2d(d + (1 + hh) * BOX, &tm_v, 0, (b * p.H + grp * HPG + hh) * p.Lmax + k0, fb);
-                ++issued;
+                    tma_load_2d(d + hh * BOX, &tm_v, 0, (b * p.H + grp * HPG + hh) * p.Lmax + i * TK, fb);
+                ++v_issued;
+                return true;
+            };
+            for (int i = 0; ok && i < K_LEAD && i < n_tiles; ++i) ok = issue_k(i);
+            for (int i = 0; ok && i < n_tiles; ++i) {
+                if (*(volatile int*)&s_abort) break;
+                if (i + K_LEAD < n_tiles) ok = issue_k(i + K_LEAD);
+                if (ok) ok = issue_v(i);
             }
-            for (int i = issued - 1; i >= 0 && i >= issued - NST; --i)
-                mbar_wait(smem_u32(&kv_full[i % NST]), (i / NST) & 1, p.status);
+            if (!ok) s_abort = 1;
+            // drain: every issued copy must land before the CTA may exit
+            for (int i = k_issued - 1; i >= 0 && i >= k_issued - NSK; --i)
+                mbar_wait(smem_u32(&k_full[i % NSK]), (i / NSK) & 1, p.status);
+            for (int i = v_issued - 1; i >= 0 && i >= v_issued - NSV; --i)
+                mbar_wait(smem_u32(&v_full[i % NSV]), (i / NSV) & 1, p.status);
             mbar_wait(qb, 0, p.status);
         }
     } else if (warp == 5) {
@@ -132,30 +158,33 @@ __global__ void __launch_bounds__(192, 1)
         constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
         constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 64, false, true);
         bool ok = mbar_wait(smem_u32(q_full), 0, p.status);
-        auto issue_qk = [&](int j) -> bool {
-            const int s = j % NST;
-            if (!mbar_wait(smem_u32(&kv_full[s]), (j / NST) & 1, p.status)) return false;
-            uint8_t* st = smem + OFF_KV + s * STAGE;
+        // zero the rows of a tile past the cache length (they may hold anything, even NaN)
+        auto zero_tail = [&](uint8_t* base, int nbox, int j) {
             const int nvalid = min(TK, L - j * TK);
-            if (nvalid < TK) {
-                // keys past the cache length may hold anything (even NaN): zero K and V rows there
-                const int rows = TK - nvalid;
-                for (int idx = lane; idx < (1 + HPG) * rows * 8; idx += 32) {
-                    const int bx = idx / (rows * 8), rr = (idx / 8) % rows, c = idx % 8;
-                    *reinterpret_cast<uint4*>(st + bx * BOX + (nvalid + rr) * 128 + c * 16) = make_uint4(0, 0, 0, 0);
-                }
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                __syncwarp();
+            if (nvalid >= TK) return;
+            const int rows = TK - nvalid;
+            for (int idx = lane; idx < nbox * rows * 8; idx += 32) {
+                const int bx = idx / (rows * 8), rr = (idx / 8) % rows, c = idx % 8;
+                *reinterpret_cast<uint4*>(base + bx * BOX + (nvalid + rr) * 128 + c * 16) = make_uint4(0, 0, 0, 0);
             }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+        };
+        auto issue_qk = [&](int j) -> bool {
+            const int s = j % NSK;
+            if (!mbar_wait(smem_u32(&k_full[s]), (j / NSK) & 1, p.status)) return false;
+            uint8_t* kt = smem + OFF_K + s * BOX;
+            zero_tail(kt, 1, j);
             if (j >= 1 && !mbar_wait(smem_u32(s_free), (j - 1) & 1, p.status)) return false;
             tc_fence_after();
             if (lane == 0) {
-                const uint32_t qa = smem_u32(smem + OFF_Q), ka = smem_u32(st);
+                const uint32_t qa = smem_u32(smem + OFF_Q), ka = smem_u32(kt);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
                     umma_ss(tmem + T_S, smem_desc_sw128(qa + k * 32, 16, 1024), smem_desc_sw128(ka + k * 32, 16, 1024),
                             idesc_qk, k != 0);
                 umma_commit(smem_u32(s_ready));
+                umma_commit(smem_u32(&k_empty[s]));  // the key tile is free once the scores are computed
             }
             __syncwarp();
             return true;
@@ -163,16 +192,20 @@ __global__ void __launch_bounds__(192, 1)
         if (ok) ok = issue_qk(0);
         for (int j = 0; ok && j < n_tiles; ++j) {
             if (j + 1 < n_tiles && !issue_qk(j + 1)) break;
+            const int sv = j % NSV;
+            if (!mbar_wait(smem_u32(&v_full[sv]), (j / NSV) & 1, p.status)) break;
+            uint8_t* vt = smem + OFF_V + sv * VSTAGE;
+            zero_tail(vt, HPG, j);
             if (!mbar_wait(smem_u32(&p_ready[j & 1]), (j >> 1) & 1, p.status)) break;
             tc_fence_after();
             if (lane == 0) {
-                const uint32_t va = smem_u32(smem + OFF_KV + (j % NST) * STAGE + BOX);
+                const uint32_t va = smem_u32(vt);
                 for (int hh = 0; hh < HPG; ++hh)
 #pragma unroll
                     for (int kk = 0; kk < TK / 16; ++kk)
                         umma_ts(tmem + T_O + hh * 64, tmem + T_P + (j & 1) * 64 + kk * 8,
                                 smem_desc_sw128(va + hh * BOX + kk * 2048, BOX, 1024), idesc_pv, (j | kk) != 0);
-                umma_commit(smem_u32(&kv_empty[j % NST]));
+                umma_commit(smem_u32(&v_empty[sv]));
                 umma_commit(smem_u32(&o_ready[j & 1]));
             }
             __syncwarp();
@@ -197,14 +230,16 @@ __global__ void __launch_bounds__(192, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(s_free));  // the next score tile may be written
             const int k0 = j * TK;
-            float mx = -INFINITY;
+            float* sf = reinterpret_cast<float*>(sr);
+            if (k0 + TK <= vis_end) {
 #pragma unroll
-            for (int c = 0; c < TK; ++c) {
-                const float v = (k0 + c < vis_end) ? __uint_as_float(sr[c]) * p.scale_log2 : -INFINITY;
-                sr[c] = __float_as_uint(v);
-                mx = fmaxf(mx, v);
+                for (int c = 0; c < TK; ++c) sf[c] = __uint_as_float(sr[c]) * p.scale_log2;
+            } else {
+#pragma unroll
+                for (int c = 0; c < TK; ++c)
+                    sf[c] = (k0 + c < vis_end) ? __uint_as_float(sr[c]) * p.scale_log2 : -INFINITY;
             }
-            const float m_new = fmaxf(m_ref, mx);
+            const float m_new = fmaxf(m_ref, tree_max<TK>(sf));
             bool resc = false;
             float alpha = 1.f, m_use = m_ref;
             if (m_ref == -INFINITY) {
@@ -214,15 +249,13 @@ __global__ void __launch_bounds__(192, 1)
                 alpha = fast_exp2(m_ref - m_new);
                 m_use = m_new;
             }
-            float rs = 0.f;
             uint32_t pk[TK / 2];
+            const float m_sub = m_use == -INFINITY ? 0.f : m_use;  // all scores -inf: p = 2^-inf = 0
 #pragma unroll
-            for (int c = 0; c < TK; c += 2) {
-                const float p0 = m_use == -INFINITY ? 0.f : fast_exp2(__uint_as_float(sr[c]) - m_use);
-                const float p1 = m_use == -INFINITY ? 0.f : fast_exp2(__uint_as_float(sr[c + 1]) - m_use);
-                rs += p0 + p1;
-                pk[c / 2] = pack_bf16x2(p0, p1);
-            }
+            for (int c = 0; c < TK; ++c) sf[c] = fast_exp2(sf[c] - m_sub);
+#pragma unroll
+            for (int c = 0; c < TK; c += 2) pk[c / 2] = pack_bf16x2(sf[c], sf[c + 1]);
+            const float rs = tree_sum<TK>(sf);
             l = (resc ? l * alpha : l) + rs;
             m_ref = m_use;
             // P buffer j&1 was last read by PV(j-2); O may only be rescaled after PV(j-1)

@@ -5,6 +5,8 @@
 //   absorb GEMM (q~ = W^UK^T q^C) -> latent attention (+ split merge) -> up-projection GEMM (W^UV o~).
 #include <math.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "host_util.h"
 #include "latent.h"
@@ -28,12 +30,25 @@ static lka_status_t latent_plan(int B, int h_q, int g, int s_q, int d_h, int r_k
     const int NT = latent_tile_tokens();
     int st = split_tokens_knob();
     if (st <= 0) {
-        // one CTA pair per (sequence, query token) already fills the GPU for the decode batches of
-        // interest; split the keys only when there are fewer pairs than SM pairs
+        // One CTA pair per (sequence, query token, key split).  Pick the split count n that
+        // minimises waves x (work per split + writing its partial result), in units of the work of
+        // a whole sequence: ceil(units * n / pairs) * (1/n + part), where part = the partial's
+        // bytes per CTA (128 x 256 fp32) over the cache bytes a CTA reads for a whole sequence
+        // (Lmax x 576); no partial when n = 1.  Ties go to fewer splits.
         const long long units = (long long)(B > 0 ? B : 1) * s_q;
         const long long pairs = sm_count() / 2;
-        long long nsp = units >= pairs ? 1 : (pairs + units - 1) / units;
-        st = (int)((Lmax + nsp - 1) / nsp);
+        const double part = (128.0 * 256.0 * 4.0) / ((double)Lmax * 576.0);
+        int best = 1;
+        double best_cost = 1e30;
+        const int max_n = std::max(1, std::min(256, Lmax / (8 * NT)));
+        for (int n = 1; n <= max_n; ++n) {
+            const double cost = (double)((units * n + pairs - 1) / pairs) * (1.0 / n + (n > 1 ? part : 0.0));
+            if (cost < best_cost - 1e-9) {
+                best_cost = cost;
+                best = n;
+            }
+        }
+        st = (Lmax + best - 1) / best;
         if (st < 8 * NT) st = 8 * NT;
     }
     st = cdiv(st, NT) * NT;

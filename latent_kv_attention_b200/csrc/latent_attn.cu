@@ -46,7 +46,8 @@ constexpr int XBUF = 128 * XROW;
 constexpr int OFF_Q = 0;
 constexpr int OFF_KV = OFF_Q + Q_BYTES;
 constexpr int OFF_X = OFF_KV + NST * STAGE;
-constexpr int OFF_BAR = OFF_X + 2 * XBUF;
+constexpr int NXB = 3;          // exchange buffers: a partial is sent up to two tiles before it is used
+constexpr int OFF_BAR = OFF_X + NXB * XBUF;
 constexpr int SMEM = 1024 + OFF_BAR + 512;
 // tensor memory columns
 constexpr uint32_t T_O = 0;          // 256 fp32 columns: this rank's half of the output
@@ -75,33 +76,16 @@ __device__ __forceinline__ void st_async_v4(uint32_t raddr, uint32_t a, uint32_t
                  "r"(a), "r"(b), "r"(c), "r"(d), "r"(rbar)
                  : "memory");
 }
+// Arrival on the peer's "buffer free" barrier.  Relaxed: it only follows local shared-memory
+// loads whose values have already been consumed, and a release fence here would also wait for
+// this thread's outstanding remote stores.
 __device__ __forceinline__ void remote_arrive(uint32_t rbar) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(rbar) : "memory");
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(rbar) : "memory");
 }
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-// bounded wait with cluster-scope acquire (for data written by the peer CTA)
-__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, uint32_t* status) {
-    for (int i = 0; i < 32; ++i)
-        if (mbar_try_wait_cluster(bar, parity)) return true;
-    const uint64_t t0 = globaltimer();
-    while (true) {
-        if (mbar_try_wait_cluster(bar, parity)) return true;
-        if (globaltimer() - t0 > kWaitLimitNs) {
-            if (status) atomicOr(status, kDevTimeout);
-            return false;
-        }
-    }
-}
+// Waits on the exchange barriers use the default (CTA-scope) acquire: the peer's partial scores
+// arrive through st.async, whose bytes complete the local barrier's transaction count, and the
+// peer's "buffer free" arrival (release at cluster scope) is only ever followed by new remote
+// stores, never by reads of data the peer produced.
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     latent_attn_kernel(const __grid_constant__ CUtensorMap tm_qt, const __grid_constant__ CUtensorMap tm_qr,
@@ -117,9 +101,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     uint64_t* s_free = s_ready + 2;       // [2] S(j) loaded by all four softmax warps
     uint64_t* p_ready = s_free + 2;       // [2] P(j) written by all four softmax warps
     uint64_t* o_ready = p_ready + 2;      // [2] PV(j) done
-    uint64_t* xfull = o_ready + 2;        // [2][4] the peer's partial scores of warp w's rows arrived
-    uint64_t* xempty = xfull + 8;         // [2][4] the peer has consumed this CTA's partial for warp w's rows
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xempty + 8);
+    uint64_t* xfull = o_ready + 2;        // [NXB][4] the peer's partial scores of warp w's rows arrived
+    uint64_t* xempty = xfull + 4 * NXB;   // [NXB][4] the peer has consumed this CTA's partial for warp w's rows
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xempty + 4 * NXB);
     __shared__ int s_abort;
 
     const uint32_t rank = cluster_rank();
@@ -151,13 +135,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
             mbar_init(smem_u32(&p_ready[i]), 4);
             mbar_init(smem_u32(&o_ready[i]), 1);
         }
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < 4 * NXB; ++i) {
             mbar_init(smem_u32(&xfull[i]), 1);
             mbar_init(smem_u32(&xempty[i]), 1);
         }
         fence_barrier_init();
-        // the first two exchange buffers are open for the peer's partial scores
-        for (int i = 0; i < 8; ++i) mbar_arrive_expect_tx(smem_u32(&xfull[i]), XBUF / 4);
+        // every exchange buffer starts open for the peer's partial scores
+        for (int i = 0; i < 4 * NXB; ++i) mbar_arrive_expect_tx(smem_u32(&xfull[i]), XBUF / 4);
     }
     if (warp == 5) {
         tmem_alloc(tmem_slot, 512);
@@ -260,12 +244,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         // consumed, so the peer's copy is usually in place when it is needed.
         const int h = warp * 32 + lane;  // head row == TMEM lane
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        const uint32_t xrem[2] = {mapa_peer(smem_u32(smem + OFF_X) + h * XROW, peer),
-                                  mapa_peer(smem_u32(smem + OFF_X + XBUF) + h * XROW, peer)};
-        const uint32_t xfull_rem[2] = {mapa_peer(smem_u32(&xfull[0 * 4 + warp]), peer),
-                                       mapa_peer(smem_u32(&xfull[1 * 4 + warp]), peer)};
-        const uint32_t xempty_rem[2] = {mapa_peer(smem_u32(&xempty[0 * 4 + warp]), peer),
-                                        mapa_peer(smem_u32(&xempty[1 * 4 + warp]), peer)};
+        uint32_t xrem[NXB], xfull_rem[NXB], xempty_rem[NXB];
+#pragma unroll
+        for (int e = 0; e < NXB; ++e) {
+            xrem[e] = mapa_peer(smem_u32(smem + OFF_X + e * XBUF) + h * XROW, peer);
+            xfull_rem[e] = mapa_peer(smem_u32(&xfull[e * 4 + warp]), peer);
+            xempty_rem[e] = mapa_peer(smem_u32(&xempty[e * 4 + warp]), peer);
+        }
         const int sw = h & 7;
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
@@ -281,20 +266,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&s_free[x]));
-            if (ok && j >= 2) ok = mbar_wait_cluster(smem_u32(&xempty[x * 4 + warp]), ((j >> 1) - 1) & 1, p.status);
+            const int e = j % NXB;
+            if (ok && j >= NXB) ok = mbar_wait(smem_u32(&xempty[e * 4 + warp]), ((j / NXB) - 1) & 1, p.status);
 #pragma unroll
             for (int c = 0; c < NT / 4; ++c)
-                st_async_v4(xrem[x] + ((c ^ sw) << 4), dst[4 * c], dst[4 * c + 1], dst[4 * c + 2], dst[4 * c + 3],
-                            xfull_rem[x]);
+                st_async_v4(xrem[e] + ((c ^ sw) << 4), dst[4 * c], dst[4 * c + 1], dst[4 * c + 2], dst[4 * c + 3],
+                            xfull_rem[e]);
         };
         if (n_tiles > 0) fetch_and_send(0, cur);
         for (int i = 0; i < n_tiles; ++i) {
             const int x = i & 1;
             if (i + 1 < n_tiles) fetch_and_send(i + 1, nxt);
             // ---- the peer's partial of tile i ----
-            if (ok) ok = mbar_wait_cluster(smem_u32(&xfull[x * 4 + warp]), (i >> 1) & 1, p.status);
+            const int e = i % NXB;
+            if (ok) ok = mbar_wait(smem_u32(&xfull[e * 4 + warp]), (i / NXB) & 1, p.status);
             float s[NT];
-            const uint8_t* xr = smem + OFF_X + x * XBUF + h * XROW;
+            const uint8_t* xr = smem + OFF_X + e * XBUF + h * XROW;
 #pragma unroll
             for (int c = 0; c < NT / 4; ++c) {
                 const float4 v = *reinterpret_cast<const float4*>(xr + ((c ^ sw) << 4));
@@ -304,19 +291,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                 s[4 * c + 3] = __uint_as_float(cur[4 * c + 3]) + v.w;
             }
             __syncwarp();
-            if (lane == 0 && i + 2 < n_tiles) {
-                mbar_arrive_expect_tx(smem_u32(&xfull[x * 4 + warp]), XBUF / 4);  // reopen for tile i + 2 ...
-                remote_arrive(xempty_rem[x]);                                     // ... and tell the peer
+            if (lane == 0 && i + NXB < n_tiles) {
+                mbar_arrive_expect_tx(smem_u32(&xfull[e * 4 + warp]), XBUF / 4);  // reopen for tile i + NXB ...
+                remote_arrive(xempty_rem[e]);                                     // ... and tell the peer
             }
             // ---- mask, online softmax ----
             const int k0 = kbeg + i * NT;
-            float mx = -INFINITY;
+            if (k0 + NT <= kend) {
 #pragma unroll
-            for (int j = 0; j < NT; ++j) {
-                s[j] = (k0 + j < kend) ? s[j] * p.scale_log2 : -INFINITY;
-                mx = fmaxf(mx, s[j]);
+                for (int j = 0; j < NT; ++j) s[j] *= p.scale_log2;
+            } else {
+#pragma unroll
+                for (int j = 0; j < NT; ++j) s[j] = (k0 + j < kend) ? s[j] * p.scale_log2 : -INFINITY;
             }
-            const float m_new = fmaxf(m_ref, mx);
+            const float m_new = fmaxf(m_ref, tree_max<NT>(s));
             bool resc = false;
             float alpha = 1.f;
             float m_use = m_ref;
@@ -327,15 +315,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                 alpha = fast_exp2(m_ref - m_new);
                 m_use = m_new;
             }
-            float rs = 0.f;
             uint32_t pk[NT / 2];
+            const float m_sub = m_use == -INFINITY ? 0.f : m_use;  // all scores -inf: p = 2^-inf = 0
 #pragma unroll
-            for (int j = 0; j < NT; j += 2) {
-                const float p0 = m_use == -INFINITY ? 0.f : fast_exp2(s[j] - m_use);
-                const float p1 = m_use == -INFINITY ? 0.f : fast_exp2(s[j + 1] - m_use);
-                rs += p0 + p1;
-                pk[j / 2] = pack_bf16x2(p0, p1);
-            }
+            for (int j = 0; j < NT; ++j) s[j] = fast_exp2(s[j] - m_sub);
+#pragma unroll
+            for (int j = 0; j < NT; j += 2) pk[j / 2] = pack_bf16x2(s[j], s[j + 1]);
+            const float rs = tree_sum<NT>(s);
             l = (resc ? l * alpha : l) + rs;
             m_ref = m_use;
             // P buffer x was last read by PV(i-2)
