@@ -24,6 +24,8 @@ cudaError_t gemm_expand(const CUtensorMap& a, const CUtensorMap& b, const GemmPa
 
 struct LatentParams {
     const int32_t* lens;   // device [B]
+    const __nv_bfloat16* q_t;  // [B*s_q*h_q][r_kv] absorbed query q~ (rows (b, t, h))
+    const __nv_bfloat16* q_r;  // [B, h_q, s_q, d_r] RoPE query
     __nv_bfloat16* o_lat;  // [g][B*HPG*s_q][r_kv] bf16 latent-space output (rows (b, hh, t) per group)
     float* lse;            // [B, h_q, s_q] natural log, or nullptr
     float* part_o;         // [B*s_q*h_q][nsplit][r_kv] fp32 partials (nsplit > 1)
@@ -34,8 +36,7 @@ struct LatentParams {
     int split_tokens, nsplit;
 };
 
-cudaError_t latent_attn_launch(const CUtensorMap& tm_qt, const CUtensorMap& tm_qr, const CUtensorMap& tm_lat,
-                               const LatentParams& p, cudaStream_t st);
+cudaError_t latent_attn_launch(const CUtensorMap& tm_lat, const LatentParams& p, cudaStream_t st);
 int latent_tile_tokens();
 
 }  // namespace lka

@@ -128,19 +128,14 @@ lka_status_t latent_absorbed_attn(const void* q_c, const void* q_r, const void* 
     if ((s = st_of(gemm_absorb(tm_qc, tm_wuk, ga, st))) != LKA_OK) return s;
 
     // 2) attention of all heads over the latent cache (+ merge of key splits)
-    CUtensorMap tm_qt, tm_qr, tm_lat;
-    {
-        if (!make_tmap_2d(&tm_qt, BF, qt, r_kv, (uint64_t)B * s_q * h_q, (uint64_t)r_kv * 2, 64, 128)) return LKA_ERR_CUDA;
-        const uint64_t dims[3] = {(uint64_t)d_r, (uint64_t)s_q, (uint64_t)B * h_q};
-        const uint64_t str[2] = {(uint64_t)d_r * 2, (uint64_t)s_q * d_r * 2};
-        const uint32_t box[3] = {64, 1, 128};
-        if (!make_tmap_nd(&tm_qr, BF, q_r, 3, dims, str, box)) return LKA_ERR_CUDA;
-        if (!make_tmap_2d(&tm_lat, BF, latent, r_kv + d_r, (uint64_t)B * Lmax, (uint64_t)(r_kv + d_r) * 2, 64,
-                          latent_tile_tokens()))
-            return LKA_ERR_CUDA;
-    }
+    CUtensorMap tm_lat;
+    if (!make_tmap_2d(&tm_lat, BF, latent, r_kv + d_r, (uint64_t)B * Lmax, (uint64_t)(r_kv + d_r) * 2, 64,
+                      latent_tile_tokens()))
+        return LKA_ERR_CUDA;
     LatentParams lp{};
     lp.lens = cache_lens;
+    lp.q_t = qt;
+    lp.q_r = static_cast<const __nv_bfloat16*>(q_r);
     lp.o_lat = olat;
     lp.lse = lse;
     lp.part_o = pl.nsplit > 1 ? reinterpret_cast<float*>(w + pl.off_po) : nullptr;
@@ -155,7 +150,7 @@ lka_status_t latent_absorbed_attn(const void* q_c, const void* q_r, const void* 
     lp.scale_log2 = scale * 1.4426950408889634f;
     lp.split_tokens = pl.split_tokens;
     lp.nsplit = pl.nsplit;
-    if ((s = st_of(latent_attn_launch(tm_qt, tm_qr, tm_lat, lp, st))) != LKA_OK) return s;
+    if ((s = st_of(latent_attn_launch(tm_lat, lp, st))) != LKA_OK) return s;
 
     // 3) up-projection out = W^UV_gamma o~
     CUtensorMap tm_ol, tm_wuv;

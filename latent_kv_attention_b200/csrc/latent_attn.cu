@@ -11,22 +11,29 @@
 // contraction are dense, so both run as tcgen05 MMAs with M = 128 heads.
 //
 // Tensor memory holds 512 fp32 columns per SM and the output alone needs
-// 128 x 512, so each work item is processed by a CLUSTER OF TWO CTAs that split
-// the latent dimensions: rank 0 loads latent values [0, 256), rank 1 loads
-// [256, 512) and the RoPE key [512, 576).  Each rank multiplies the query slice
-// it holds with the tile slice it loaded (a split-K partial of the scores),
-// the two partials are exchanged through distributed shared memory (st.async
-// with mbarrier transaction counts) and summed identically on both sides, so
-// both run the same online softmax and each accumulates the 256 output columns
-// of the latent values it loaded.  No tile byte is loaded twice and no score
-// is computed twice.
+// 128 x 512, so each work item is processed by a CLUSTER OF TWO CTAs: rank r
+// accumulates output columns [256 r, 256 r + 256) and computes the split-K
+// partial of the scores over key values [288 r, 288 r + 288).  For that it
+// loads latent values [256 r, 256 r + 320) of every token (rank 0: [0, 320),
+// rank 1: [256, 576), i.e. its 256 value columns plus the rest of its score
+// range; the 64 values [256, 320) are read by both ranks, the second read
+// coming from L2).  The two score partials are exchanged through distributed
+// shared memory (st.async with mbarrier transaction counts) and summed
+// identically on both sides, so both run the same online softmax.
 //
-// Per CTA: warp 4 streams the query slice once and 32-token tiles of the
-// latent through a 4-stage TMA ring; warp 5 issues the MMAs (S = Q K^T into a
-// double-buffered TMEM score tile; O += P V with P read from TMEM); warps 0-3
-// own one head row each per thread: exchange, mask, online softmax with lazy
-// rescaling (the running maximum is only moved when it grows by more than 2^8,
-// which leaves the final O / l exact), P written back to TMEM as bf16.
+// Each tcgen05.mma with M = 128 and K = 16 takes about the same time whatever
+// its N (up to 256), so the tiles are as wide as memory allows: 64 tokens.  The
+// query slice lives in tensor memory (the A operand of the score MMA), which
+// leaves shared memory to a 3-stage TMA ring, two exchange buffers and an
+// outbox: a partial is written to the outbox and sent with one bulk copy per
+// warp (the copy engine moves it; the warp does not wait for the transfer).
+//
+// Per CTA: warp 4 streams 64-token tiles of the latent through the ring; warp 5
+// issues the MMAs (S = Q K^T into the TMEM score tile, O += P V with P read
+// from TMEM); warps 0-3 own one head row each per thread: they write the query
+// slice to TMEM once, then per tile exchange, mask and run the online softmax
+// with lazy rescaling (the running maximum is only moved when it grows by more
+// than 2^8, which leaves the final O / l exact), P written back to TMEM as bf16.
 #include "common.cuh"
 #include "host_util.h"
 #include "latent.h"
@@ -35,24 +42,27 @@
 namespace lka {
 
 namespace lat {
-constexpr int NT = 32;          // tokens per tile
-constexpr int NST = 4;          // TMA ring depth
-constexpr int KB_MAX = 5;       // 64-wide K blocks per rank (rank 1: 4 latent + 1 RoPE)
-constexpr int Q_BYTES = KB_MAX * 128 * 128;
+constexpr int NT = 64;          // tokens per tile (the N of the score MMA)
+constexpr int NST = 3;          // TMA ring depth
+constexpr int NKB = 5;          // 64-value boxes per rank and tile
+constexpr int KSTEPS = 18;      // K = 16 steps of this rank's 288 score values
 constexpr int BOX = NT * 128;   // one 64-value box of NT tokens
-constexpr int STAGE = KB_MAX * BOX;
+constexpr int STAGE = NKB * BOX;
 constexpr int XROW = NT * 4;    // bytes of one exchanged score row
 constexpr int XBUF = 128 * XROW;
-constexpr int OFF_Q = 0;
-constexpr int OFF_KV = OFF_Q + Q_BYTES;
+constexpr int OFF_KV = 0;
 constexpr int OFF_X = OFF_KV + NST * STAGE;
-constexpr int NXB = 3;          // exchange buffers: a partial is sent up to two tiles before it is used
-constexpr int OFF_BAR = OFF_X + NXB * XBUF;
+constexpr int NXB = 2;          // exchange buffers
+constexpr int OFF_OUT = OFF_X + NXB * XBUF;  // this CTA's partial on its way to the peer
+constexpr int OFF_BAR = OFF_OUT + XBUF;
 constexpr int SMEM = 1024 + OFF_BAR + 512;
+static_assert(SMEM <= 232448, "shared memory budget");
 // tensor memory columns
 constexpr uint32_t T_O = 0;          // 256 fp32 columns: this rank's half of the output
-constexpr uint32_t T_S = 256;        // 2 x NT fp32 score partials
-constexpr uint32_t T_P = 256 + 2 * NT;  // 2 x NT/2 columns of bf16 pairs
+constexpr uint32_t T_Q = 256;        // 144 columns: this rank's 288 query values as bf16 pairs
+constexpr uint32_t T_P = 400;        // NT/2 columns of bf16 pairs
+constexpr uint32_t T_S = 448;        // NT fp32 score partials
+static_assert(T_Q + KSTEPS * 8 <= T_P && T_P + NT / 2 <= T_S && T_S + NT <= 512, "tensor memory budget");
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 domain
 }  // namespace lat
 
@@ -76,6 +86,19 @@ __device__ __forceinline__ void st_async_v4(uint32_t raddr, uint32_t a, uint32_t
                  "r"(a), "r"(b), "r"(c), "r"(d), "r"(rbar)
                  : "memory");
 }
+// Bulk copy of `bytes` from this CTA's shared memory to the peer's (cluster address `dst`),
+// completing `bytes` of the transaction count of the peer's barrier `rbar`.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t rbar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "r"(src), "r"(bytes), "r"(rbar)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until the bulk copies this thread committed have finished reading their sources.
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Wait until they have completed entirely.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 // Arrival on the peer's "buffer free" barrier.  Relaxed: it only follows local shared-memory
 // loads whose values have already been consumed, and a release fence here would also wait for
 // this thread's outstanding remote stores.
@@ -88,27 +111,25 @@ __device__ __forceinline__ void remote_arrive(uint32_t rbar) {
 // stores, never by reads of data the peer produced.
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
-    latent_attn_kernel(const __grid_constant__ CUtensorMap tm_qt, const __grid_constant__ CUtensorMap tm_qr,
-                       const __grid_constant__ CUtensorMap tm_lat, const LatentParams p) {
+    latent_attn_kernel(const __grid_constant__ CUtensorMap tm_lat, const LatentParams p) {
     using namespace lat;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-    uint64_t* q_full = bars + 0;
+    uint64_t* q_full = bars + 0;          // the query slice is in tensor memory (4 softmax-warp arrivals)
     uint64_t* kv_full = bars + 1;
     uint64_t* kv_empty = kv_full + NST;
-    uint64_t* s_ready = kv_empty + NST;   // [2] QK(j) done (buffer j&1)
-    uint64_t* s_free = s_ready + 2;       // [2] S(j) loaded by all four softmax warps
-    uint64_t* p_ready = s_free + 2;       // [2] P(j) written by all four softmax warps
-    uint64_t* o_ready = p_ready + 2;      // [2] PV(j) done
-    uint64_t* xfull = o_ready + 2;        // [NXB][4] the peer's partial scores of warp w's rows arrived
+    uint64_t* s_ready = kv_empty + NST;   // QK(j) done
+    uint64_t* s_free = s_ready + 1;       // S(j) loaded by all four softmax warps
+    uint64_t* p_ready = s_free + 1;       // P(j) written by all four softmax warps
+    uint64_t* o_ready = p_ready + 1;      // PV(j) done
+    uint64_t* xfull = o_ready + 1;        // [NXB][4] the peer's partial scores of warp w's rows arrived
     uint64_t* xempty = xfull + 4 * NXB;   // [NXB][4] the peer has consumed this CTA's partial for warp w's rows
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xempty + 4 * NXB);
     __shared__ int s_abort;
 
     const uint32_t rank = cluster_rank();
     const uint32_t peer = rank ^ 1u;
-    const int nkb = rank == 0 ? 4 : 5;
     const int pair = blockIdx.x >> 1;
     const int t = pair % p.s_q;
     const int split = pair / p.s_q;
@@ -124,17 +145,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
 
     if (threadIdx.x == 0) {
         s_abort = 0;
-        mbar_init(smem_u32(q_full), 1);
+        mbar_init(smem_u32(q_full), 4);
         for (int s = 0; s < NST; ++s) {
             mbar_init(smem_u32(&kv_full[s]), 1);
             mbar_init(smem_u32(&kv_empty[s]), 1);
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(smem_u32(&s_ready[i]), 1);
-            mbar_init(smem_u32(&s_free[i]), 4);
-            mbar_init(smem_u32(&p_ready[i]), 4);
-            mbar_init(smem_u32(&o_ready[i]), 1);
-        }
+        mbar_init(smem_u32(s_ready), 1);
+        mbar_init(smem_u32(s_free), 4);
+        mbar_init(smem_u32(p_ready), 4);
+        mbar_init(smem_u32(o_ready), 1);
         for (int i = 0; i < 4 * NXB; ++i) {
             mbar_init(smem_u32(&xfull[i]), 1);
             mbar_init(smem_u32(&xempty[i]), 1);
@@ -155,14 +174,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     if (n_tiles > 0 && warp == 4) {
         // ------------------------------- TMA producer -------------------------------
         if (lane == 0) {
-            prefetch_tensormap(&tm_qt);
             prefetch_tensormap(&tm_lat);
-            const uint32_t qb = smem_u32(q_full);
-            mbar_arrive_expect_tx(qb, nkb * 128 * 128);
-            const int qrow = (b * p.s_q + t) * 128;
-            for (int kb = 0; kb < 4; ++kb)
-                tma_load_2d(smem_u32(smem + OFF_Q + kb * 16384), &tm_qt, (int)(rank * 4 + kb) * 64, qrow, qb);
-            if (rank == 1) tma_load_3d(smem_u32(smem + OFF_Q + 4 * 16384), &tm_qr, 0, t, b * 128, qb);
             int issued = 0;
             for (int i = 0; i < n_tiles; ++i) {
                 const int s = i % NST;
@@ -172,24 +184,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                 }
                 if (*(volatile int*)&s_abort) break;
                 const uint32_t fb = smem_u32(&kv_full[s]);
-                mbar_arrive_expect_tx(fb, nkb * BOX);
+                mbar_arrive_expect_tx(fb, NKB * BOX);
                 const uint32_t dst = smem_u32(smem + OFF_KV + s * STAGE);
                 const int y = b * p.Lmax + kbeg + i * NT;
-                for (int kb = 0; kb < nkb; ++kb) tma_load_2d(dst + kb * BOX, &tm_lat, (int)rank * 256 + kb * 64, y, fb);
+                for (int kb = 0; kb < NKB; ++kb) tma_load_2d(dst + kb * BOX, &tm_lat, (int)rank * 256 + kb * 64, y, fb);
                 ++issued;
             }
             for (int i = issued - 1; i >= 0 && i >= issued - NST; --i)
                 mbar_wait(smem_u32(&kv_full[i % NST]), (i / NST) & 1, p.status);
-            mbar_wait(qb, 0, p.status);
         }
     } else if (n_tiles > 0 && warp == 5) {
         // ------------------------------- MMA issuer -------------------------------
-        // Order: QK(0), QK(1), then per step j: QK(j) and PV(j-2).  QK(j) only needs the softmax
-        // warps to have loaded S(j-2) (s_free), so score tiles run two ahead of P*V.
+        // Per step j: QK(j) once the softmax warps have loaded S(j-1), then PV(j-1) once P(j-1)
+        // is in tensor memory; QK(j) runs while the softmax of tile j-1 is computed.
         constexpr uint32_t idesc_qk = idesc_bf16_f32(128, NT, false, false);
         constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
         bool ok = mbar_wait(smem_u32(q_full), 0, p.status);
-        for (int j = 0; ok && j < n_tiles + 2; ++j) {
+        for (int j = 0; ok && j <= n_tiles; ++j) {
             if (j < n_tiles) {
                 const int s = j % NST;
                 if (!mbar_wait(smem_u32(&kv_full[s]), (j / NST) & 1, p.status)) break;
@@ -199,7 +210,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                     // rows past the last visible key may hold anything (even NaN): zero them so
                     // that P = 0 times V contributes exactly 0
                     const int rows = NT - nvalid;
-                    for (int idx = lane; idx < nkb * rows * 8; idx += 32) {
+                    for (int idx = lane; idx < NKB * rows * 8; idx += 32) {
                         const int kb = idx / (rows * 8), rr = (idx / 8) % rows, c = idx % 8;
                         *reinterpret_cast<uint4*>(st + kb * BOX + (nvalid + rr) * 128 + c * 16) =
                             make_uint4(0, 0, 0, 0);
@@ -207,32 +218,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     __syncwarp();
                 }
-                if (j >= 2 && !mbar_wait(smem_u32(&s_free[j & 1]), ((j >> 1) - 1) & 1, p.status)) break;
+                if (j >= 1 && !mbar_wait(smem_u32(s_free), (j - 1) & 1, p.status)) break;
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t qa = smem_u32(smem + OFF_Q);
                     const uint32_t kva = smem_u32(st);
-                    for (int kb = 0; kb < nkb; ++kb)
 #pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            umma_ss(tmem + T_S + (j & 1) * NT, smem_desc_sw128(qa + kb * 16384 + k * 32, 16, 1024),
-                                    smem_desc_sw128(kva + kb * BOX + k * 32, 16, 1024), idesc_qk, (kb | k) != 0);
-                    umma_commit(smem_u32(&s_ready[j & 1]));
+                    for (int ks = 0; ks < KSTEPS; ++ks) {
+                        // score value 288 rank + 16 ks sits at offset 32 rank + 16 ks of this rank's tile
+                        const int off = (int)rank * 32 + ks * 16;
+                        umma_ts(tmem + T_S, tmem + T_Q + ks * 8,
+                                smem_desc_sw128(kva + (off / 64) * BOX + (off % 64) * 2, 16, 1024), idesc_qk, ks != 0);
+                    }
+                    umma_commit(smem_u32(s_ready));
                 }
                 __syncwarp();
             }
-            if (j >= 2) {
-                const int i = j - 2;
-                if (!mbar_wait(smem_u32(&p_ready[i & 1]), (i >> 1) & 1, p.status)) break;
+            if (j >= 1) {
+                const int i = j - 1;
+                if (!mbar_wait(smem_u32(p_ready), i & 1, p.status)) break;
                 tc_fence_after();
                 if (lane == 0) {
                     const uint32_t va = smem_u32(smem + OFF_KV + (i % NST) * STAGE);
 #pragma unroll
                     for (int kk = 0; kk < NT / 16; ++kk)
-                        umma_ts(tmem + T_O, tmem + T_P + (i & 1) * (NT / 2) + kk * 8,
-                                smem_desc_sw128(va + kk * 2048, BOX, 1024), idesc_pv, (i | kk) != 0);
+                        umma_ts(tmem + T_O, tmem + T_P + kk * 8, smem_desc_sw128(va + kk * 2048, BOX, 1024), idesc_pv,
+                                (i | kk) != 0);
                     umma_commit(smem_u32(&kv_empty[i % NST]));
-                    umma_commit(smem_u32(&o_ready[i & 1]));
+                    umma_commit(smem_u32(o_ready));
                 }
                 __syncwarp();
             }
@@ -240,45 +252,73 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     } else if (warp < 4) {
         // ------------------------- softmax / exchange warps -------------------------
         // Each warp owns 32 head rows and its own exchange barriers, so the four warps never wait
-        // for one another.  The partial scores of tile i+1 are sent to the peer before tile i is
-        // consumed, so the peer's copy is usually in place when it is needed.
+        // for one another.
         const int h = warp * 32 + lane;  // head row == TMEM lane
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        uint32_t xrem[NXB], xfull_rem[NXB], xempty_rem[NXB];
-#pragma unroll
-        for (int e = 0; e < NXB; ++e) {
-            xrem[e] = mapa_peer(smem_u32(smem + OFF_X + e * XBUF) + h * XROW, peer);
-            xfull_rem[e] = mapa_peer(smem_u32(&xfull[e * 4 + warp]), peer);
-            xempty_rem[e] = mapa_peer(smem_u32(&xempty[e * 4 + warp]), peer);
-        }
+        // the peer's buffer and barriers for exchange slot 0; slot e is a fixed offset further on
+        // (mapa maps a whole shared-memory window, so offsets carry over)
+        const uint32_t xrem0 = mapa_peer(smem_u32(smem + OFF_X) + warp * 32 * XROW, peer);  // this warp's rows
+        uint8_t* outrow = smem + OFF_OUT + h * XROW;
+        const uint32_t xfull_rem0 = mapa_peer(smem_u32(&xfull[warp]), peer);
+        const uint32_t xempty_rem0 = mapa_peer(smem_u32(&xempty[warp]), peer);
         const int sw = h & 7;
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
-        uint32_t cur[NT], nxt[NT];
-        // load S(j) into regs, release the TMEM buffer, send the partial to the peer
-        auto fetch_and_send = [&](int j, uint32_t* dst) {
-            const int x = j & 1;
-            if (ok) ok = mbar_wait(smem_u32(&s_ready[x]), (j >> 1) & 1, p.status);
+        if (n_tiles > 0) {
+            // this rank's 288 values of the query row [q~_h ; q^R_h] -> tensor memory (A operand of the
+            // score MMA, K-major: column c holds values 2c and 2c+1): rank 0 q~[0:288), rank 1
+            // q~[288:512) followed by q^R
+            const uint4* qt = reinterpret_cast<const uint4*>(p.q_t + ((size_t)(b * p.s_q + t) * p.h_q + h) * 512);
+            const uint4* qr = reinterpret_cast<const uint4*>(p.q_r + (((size_t)b * p.h_q + h) * p.s_q + t) * 64);
+#pragma unroll
+            for (int c0 = 0; c0 < KSTEPS / 2; ++c0) {  // 9 x 16 columns = 288 values
+                uint32_t w[16];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int d = (int)rank * 288 + (c0 * 4 + q) * 8;  // first of these 8 values
+                    const uint4 v = d < 512 ? qt[d / 8] : qr[(d - 512) / 8];
+                    w[4 * q] = v.x;
+                    w[4 * q + 1] = v.y;
+                    w[4 * q + 2] = v.z;
+                    w[4 * q + 3] = v.w;
+                }
+                tmem_st16(tmem + lane_base + T_Q + c0 * 16, w);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(q_full));
+        }
+        for (int i = 0; i < n_tiles; ++i) {
+            // ---- this rank's partial of tile i: registers, release the TMEM tile, send to the peer ----
+            uint32_t cur[NT];
+            if (ok) ok = mbar_wait(smem_u32(s_ready), i & 1, p.status);
             tc_fence_after();
-            tmem_ld16(tmem + lane_base + T_S + x * NT, dst);
-            tmem_ld16(tmem + lane_base + T_S + x * NT + 16, dst + 16);
+#pragma unroll
+            for (int c0 = 0; c0 < NT; c0 += 16) tmem_ld16(tmem + lane_base + T_S + c0, cur + c0);
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&s_free[x]));
-            const int e = j % NXB;
-            if (ok && j >= NXB) ok = mbar_wait(smem_u32(&xempty[e * 4 + warp]), ((j / NXB) - 1) & 1, p.status);
+            if (lane == 0) mbar_arrive(smem_u32(s_free));
+            const int e = i % NXB;
+            // the outbox rows of this warp are free once the previous bulk copy has read them
+            if (lane == 0) bulk_wait_read();
+            __syncwarp();
 #pragma unroll
             for (int c = 0; c < NT / 4; ++c)
-                st_async_v4(xrem[e] + ((c ^ sw) << 4), dst[4 * c], dst[4 * c + 1], dst[4 * c + 2], dst[4 * c + 3],
-                            xfull_rem[e]);
-        };
-        if (n_tiles > 0) fetch_and_send(0, cur);
-        for (int i = 0; i < n_tiles; ++i) {
-            const int x = i & 1;
-            if (i + 1 < n_tiles) fetch_and_send(i + 1, nxt);
+                *reinterpret_cast<uint4*>(outrow + ((c ^ sw) << 4)) =
+                    make_uint4(cur[4 * c], cur[4 * c + 1], cur[4 * c + 2], cur[4 * c + 3]);
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the copy engine
+            __syncwarp();
+            if (lane == 0) {
+                if (ok && i >= NXB) ok = mbar_wait(smem_u32(&xempty[e * 4 + warp]), ((i / NXB) - 1) & 1, p.status);
+                if (ok)
+                    bulk_copy_to_peer(xrem0 + e * XBUF, smem_u32(smem + OFF_OUT + warp * 32 * XROW), 32 * XROW,
+                                      xfull_rem0 + e * 4 * 8);
+                bulk_commit();
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
             // ---- the peer's partial of tile i ----
-            const int e = i % NXB;
             if (ok) ok = mbar_wait(smem_u32(&xfull[e * 4 + warp]), (i / NXB) & 1, p.status);
             float s[NT];
             const uint8_t* xr = smem + OFF_X + e * XBUF + h * XROW;
@@ -293,7 +333,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
             __syncwarp();
             if (lane == 0 && i + NXB < n_tiles) {
                 mbar_arrive_expect_tx(smem_u32(&xfull[e * 4 + warp]), XBUF / 4);  // reopen for tile i + NXB ...
-                remote_arrive(xempty_rem[e]);                                     // ... and tell the peer
+                remote_arrive(xempty_rem0 + e * 4 * 8);                           // ... and tell the peer
             }
             // ---- mask, online softmax ----
             const int k0 = kbeg + i * NT;
@@ -324,12 +364,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
             const float rs = tree_sum<NT>(s);
             l = (resc ? l * alpha : l) + rs;
             m_ref = m_use;
-            // P buffer x was last read by PV(i-2)
-            if (ok && i >= 2) ok = mbar_wait(smem_u32(&o_ready[x]), ((i >> 1) - 1) & 1, p.status);
+            // PV(i-1) must be done: it reads the P buffer, and a rescale of O must follow its update
+            if (ok && i >= 1) ok = mbar_wait(smem_u32(o_ready), (i - 1) & 1, p.status);
+            tc_fence_after();
             if (__any_sync(0xffffffffu, resc)) {
-                // O may only be rescaled once PV(i-1) has been accumulated into it
-                if (ok && i >= 1) ok = mbar_wait(smem_u32(&o_ready[(i - 1) & 1]), ((i - 1) >> 1) & 1, p.status);
-                tc_fence_after();
                 for (int c0 = 0; c0 < 256; c0 += 16) {
                     uint32_t o[16];
                     tmem_ld16(tmem + lane_base + T_O + c0, o);
@@ -339,19 +377,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                     tmem_st16(tmem + lane_base + T_O + c0, o);
                 }
             }
-            tc_fence_after();
-            tmem_st16(tmem + lane_base + T_P + x * (NT / 2), pk);
+            tmem_st16(tmem + lane_base + T_P, pk);
+            tmem_st16(tmem + lane_base + T_P + 16, pk + 16);
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&p_ready[x]));
-#pragma unroll
-            for (int j = 0; j < NT; ++j) cur[j] = nxt[j];
+            if (lane == 0) mbar_arrive(smem_u32(p_ready));
         }
+        if (lane == 0) bulk_wait_all();
         if (!ok) s_abort = 1;
         // ---- epilogue: normalise this rank's 256 output columns ----
         const int last = n_tiles - 1;
-        if (ok && n_tiles > 0 && mbar_wait(smem_u32(&o_ready[last & 1]), (last >> 1) & 1, p.status)) {
+        if (ok && n_tiles > 0 && mbar_wait(smem_u32(o_ready), last & 1, p.status)) {
             tc_fence_after();
             const float inv_l = l > 0.f ? 1.f / l : 0.f;
             const int HPG = p.h_q / p.g;
@@ -448,14 +485,13 @@ __global__ void __launch_bounds__(128) latent_combine_kernel(const LatentParams 
 
 int latent_tile_tokens() { return lat::NT; }
 
-cudaError_t latent_attn_launch(const CUtensorMap& tm_qt, const CUtensorMap& tm_qr, const CUtensorMap& tm_lat,
-                               const LatentParams& p, cudaStream_t st) {
+cudaError_t latent_attn_launch(const CUtensorMap& tm_lat, const LatentParams& p, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(latent_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, lat::SMEM);
     if (e != cudaSuccess) return e;
     dim3 grid(2 * p.s_q * p.nsplit, p.B);
     {
         TimedLaunch timer(st);
-        latent_attn_kernel<<<grid, 192, lat::SMEM, st>>>(tm_qt, tm_qr, tm_lat, p);
+        latent_attn_kernel<<<grid, 192, lat::SMEM, st>>>(tm_lat, p);
         timer.stop();
     }
     e = cudaPeekAtLastError();
