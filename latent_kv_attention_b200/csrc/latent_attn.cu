@@ -24,9 +24,12 @@
 // Each tcgen05.mma with M = 128 and K = 16 takes about the same time whatever
 // its N (up to 256), so the tiles are as wide as memory allows: 64 tokens.  The
 // query slice lives in tensor memory (the A operand of the score MMA), which
-// leaves shared memory to a 3-stage TMA ring, two exchange buffers and an
+// leaves shared memory to a 4-stage TMA ring, one exchange buffer and an
 // outbox: a partial is written to the outbox and sent with one bulk copy per
 // warp (the copy engine moves it; the warp does not wait for the transfer).
+// The softmax warps fetch and send the partial of tile i+1 before they work on
+// tile i, and the score MMA runs two tiles ahead of P*V, so the exchange is
+// off the per-tile critical path.
 //
 // Per CTA: warp 4 streams 64-token tiles of the latent through the ring; warp 5
 // issues the MMAs (S = Q K^T into the TMEM score tile, O += P V with P read
@@ -43,7 +46,7 @@ namespace lka {
 
 namespace lat {
 constexpr int NT = 64;          // tokens per tile (the N of the score MMA)
-constexpr int NST = 3;          // TMA ring depth
+constexpr int NST = 4;          // TMA ring depth
 constexpr int NKB = 5;          // 64-value boxes per rank and tile
 constexpr int KSTEPS = 18;      // K = 16 steps of this rank's 288 score values
 constexpr int BOX = NT * 128;   // one 64-value box of NT tokens
@@ -52,7 +55,7 @@ constexpr int XROW = NT * 4;    // bytes of one exchanged score row
 constexpr int XBUF = 128 * XROW;
 constexpr int OFF_KV = 0;
 constexpr int OFF_X = OFF_KV + NST * STAGE;
-constexpr int NXB = 2;          // exchange buffers
+constexpr int NXB = 1;          // exchange buffers
 constexpr int OFF_OUT = OFF_X + NXB * XBUF;  // this CTA's partial on its way to the peer
 constexpr int OFF_BAR = OFF_OUT + XBUF;
 constexpr int SMEM = 1024 + OFF_BAR + 512;
@@ -195,12 +198,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         }
     } else if (n_tiles > 0 && warp == 5) {
         // ------------------------------- MMA issuer -------------------------------
-        // Per step j: QK(j) once the softmax warps have loaded S(j-1), then PV(j-1) once P(j-1)
-        // is in tensor memory; QK(j) runs while the softmax of tile j-1 is computed.
+        // Per step j: QK(j) once the softmax warps have loaded S(j-1), then PV(j-2) once P(j-2)
+        // is in tensor memory.  The softmax warps load S(j-1) before they compute P(j-2), so
+        // QK(j) runs while tile j-2 is being finished.
         constexpr uint32_t idesc_qk = idesc_bf16_f32(128, NT, false, false);
         constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
         bool ok = mbar_wait(smem_u32(q_full), 0, p.status);
-        for (int j = 0; ok && j <= n_tiles; ++j) {
+        for (int j = 0; ok && j < n_tiles + 2; ++j) {
             if (j < n_tiles) {
                 const int s = j % NST;
                 if (!mbar_wait(smem_u32(&kv_full[s]), (j / NST) & 1, p.status)) break;
@@ -233,8 +237,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                 }
                 __syncwarp();
             }
-            if (j >= 1) {
-                const int i = j - 1;
+            if (j >= 2) {
+                const int i = j - 2;
                 if (!mbar_wait(smem_u32(p_ready), i & 1, p.status)) break;
                 tc_fence_after();
                 if (lane == 0) {
@@ -255,8 +259,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         // for one another.
         const int h = warp * 32 + lane;  // head row == TMEM lane
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        // the peer's buffer and barriers for exchange slot 0; slot e is a fixed offset further on
-        // (mapa maps a whole shared-memory window, so offsets carry over)
+        // the peer's exchange buffer rows and barriers of this warp
         const uint32_t xrem0 = mapa_peer(smem_u32(smem + OFF_X) + warp * 32 * XROW, peer);  // this warp's rows
         uint8_t* outrow = smem + OFF_OUT + h * XROW;
         const uint32_t xfull_rem0 = mapa_peer(smem_u32(&xfull[warp]), peer);
@@ -289,10 +292,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(q_full));
         }
-        for (int i = 0; i < n_tiles; ++i) {
-            // ---- this rank's partial of tile i: registers, release the TMEM tile, send to the peer ----
-            uint32_t cur[NT];
-            if (ok) ok = mbar_wait(smem_u32(s_ready), i & 1, p.status);
+        uint32_t cur[NT];
+        // this rank's partial of tile j: registers, release the TMEM tile, send it to the peer
+        auto fetch_and_send = [&](int j) {
+            if (ok) ok = mbar_wait(smem_u32(s_ready), j & 1, p.status);
             tc_fence_after();
 #pragma unroll
             for (int c0 = 0; c0 < NT; c0 += 16) tmem_ld16(tmem + lane_base + T_S + c0, cur + c0);
@@ -300,7 +303,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(s_free));
-            const int e = i % NXB;
             // the outbox rows of this warp are free once the previous bulk copy has read them
             if (lane == 0) bulk_wait_read();
             __syncwarp();
@@ -311,17 +313,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the copy engine
             __syncwarp();
             if (lane == 0) {
-                if (ok && i >= NXB) ok = mbar_wait(smem_u32(&xempty[e * 4 + warp]), ((i / NXB) - 1) & 1, p.status);
+                // the peer's buffer is free once it has consumed partial j-1
+                if (ok && j >= 1) ok = mbar_wait(smem_u32(&xempty[warp]), (j - 1) & 1, p.status);
                 if (ok)
-                    bulk_copy_to_peer(xrem0 + e * XBUF, smem_u32(smem + OFF_OUT + warp * 32 * XROW), 32 * XROW,
-                                      xfull_rem0 + e * 4 * 8);
+                    bulk_copy_to_peer(xrem0, smem_u32(smem + OFF_OUT + warp * 32 * XROW), 32 * XROW, xfull_rem0);
                 bulk_commit();
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
-            // ---- the peer's partial of tile i ----
-            if (ok) ok = mbar_wait(smem_u32(&xfull[e * 4 + warp]), (i / NXB) & 1, p.status);
+        };
+        if (n_tiles > 0) fetch_and_send(0);
+        for (int i = 0; i < n_tiles; ++i) {
+            // ---- the peer's partial of tile i, added to this rank's ----
+            if (ok) ok = mbar_wait(smem_u32(&xfull[warp]), i & 1, p.status);
             float s[NT];
-            const uint8_t* xr = smem + OFF_X + e * XBUF + h * XROW;
+            const uint8_t* xr = smem + OFF_X + h * XROW;
 #pragma unroll
             for (int c = 0; c < NT / 4; ++c) {
                 const float4 v = *reinterpret_cast<const float4*>(xr + ((c ^ sw) << 4));
@@ -331,10 +336,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                 s[4 * c + 3] = __uint_as_float(cur[4 * c + 3]) + v.w;
             }
             __syncwarp();
-            if (lane == 0 && i + NXB < n_tiles) {
-                mbar_arrive_expect_tx(smem_u32(&xfull[e * 4 + warp]), XBUF / 4);  // reopen for tile i + NXB ...
-                remote_arrive(xempty_rem0 + e * 4 * 8);                           // ... and tell the peer
+            if (lane == 0 && i + 1 < n_tiles) {
+                mbar_arrive_expect_tx(smem_u32(&xfull[warp]), XBUF / 4);  // reopen for tile i + 1 ...
+                remote_arrive(xempty_rem0);                                // ... and tell the peer
             }
+            // ---- tile i+1 goes out before tile i is finished ----
+            if (i + 1 < n_tiles) fetch_and_send(i + 1);
             // ---- mask, online softmax ----
             const int k0 = kbeg + i * NT;
             if (k0 + NT <= kend) {
