@@ -31,12 +31,14 @@
 // tile i, and the score MMA runs two tiles ahead of P*V, so the exchange is
 // off the per-tile critical path.
 //
-// Per CTA: warp 4 streams 64-token tiles of the latent through the ring; warp 5
+// Per CTA: warp 8 streams 64-token tiles of the latent through the ring; warp 9
 // issues the MMAs (S = Q K^T into the TMEM score tile, O += P V with P read
-// from TMEM); warps 0-3 own one head row each per thread: they write the query
-// slice to TMEM once, then per tile exchange, mask and run the online softmax
-// with lazy rescaling (the running maximum is only moved when it grows by more
-// than 2^8, which leaves the final O / l exact), P written back to TMEM as bf16.
+// from TMEM); warps 0-7 write the query slice to TMEM once, then per tile
+// exchange, mask and run the online softmax, two warps per group of 32 head
+// rows (warps w and w + 4 take the two 32-token halves of the tile and swap
+// their row maxima through two spare TMEM columns), with lazy rescaling (the
+// running maximum is only moved when it grows by more than 2^8, which leaves
+// the final O / l exact); P is written back to TMEM as bf16.
 #include "common.cuh"
 #include "host_util.h"
 #include "latent.h"
@@ -51,12 +53,14 @@ constexpr int NKB = 5;          // 64-value boxes per rank and tile
 constexpr int KSTEPS = 18;      // K = 16 steps of this rank's 288 score values
 constexpr int BOX = NT * 128;   // one 64-value box of NT tokens
 constexpr int STAGE = NKB * BOX;
-constexpr int XROW = NT * 4;    // bytes of one exchanged score row
-constexpr int XBUF = 128 * XROW;
+constexpr int NSW = 8;          // softmax warps: 4 lane quarters x 2 column halves
+constexpr int CW = NT / 2;      // score columns per softmax warp
+constexpr int NTHREADS = 32 * (NSW + 2);
+constexpr int XROW = CW * 4;    // bytes of one row of one half of an exchanged partial
+constexpr int XBUF = 2 * 128 * XROW;  // [half][head row][CW] fp32; each warp's block is contiguous
 constexpr int OFF_KV = 0;
 constexpr int OFF_X = OFF_KV + NST * STAGE;
-constexpr int NXB = 1;          // exchange buffers
-constexpr int OFF_OUT = OFF_X + NXB * XBUF;  // this CTA's partial on its way to the peer
+constexpr int OFF_OUT = OFF_X + XBUF;  // this CTA's partial on its way to the peer
 constexpr int OFF_BAR = OFF_OUT + XBUF;
 constexpr int SMEM = 1024 + OFF_BAR + 512;
 static_assert(SMEM <= 232448, "shared memory budget");
@@ -64,8 +68,10 @@ static_assert(SMEM <= 232448, "shared memory budget");
 constexpr uint32_t T_O = 0;          // 256 fp32 columns: this rank's half of the output
 constexpr uint32_t T_Q = 256;        // 144 columns: this rank's 288 query values as bf16 pairs
 constexpr uint32_t T_P = 400;        // NT/2 columns of bf16 pairs
+constexpr uint32_t T_R = 432;        // 6 columns: row maxima (2 tiles x 2 halves) and row sums of the warp pairs
 constexpr uint32_t T_S = 448;        // NT fp32 score partials
-static_assert(T_Q + KSTEPS * 8 <= T_P && T_P + NT / 2 <= T_S && T_S + NT <= 512, "tensor memory budget");
+static_assert(T_Q + KSTEPS * 8 <= T_P && T_P + NT / 2 <= T_R && T_R + 6 <= T_S && T_S + NT <= 512,
+              "tensor memory budget");
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 domain
 }  // namespace lat
 
@@ -113,22 +119,22 @@ __device__ __forceinline__ void remote_arrive(uint32_t rbar) {
 // peer's "buffer free" arrival (release at cluster scope) is only ever followed by new remote
 // stores, never by reads of data the peer produced.
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(lat::NTHREADS, 1)
     latent_attn_kernel(const __grid_constant__ CUtensorMap tm_lat, const LatentParams p) {
     using namespace lat;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-    uint64_t* q_full = bars + 0;          // the query slice is in tensor memory (4 softmax-warp arrivals)
+    uint64_t* q_full = bars + 0;          // the query slice is in tensor memory (all softmax warps arrived)
     uint64_t* kv_full = bars + 1;
     uint64_t* kv_empty = kv_full + NST;
     uint64_t* s_ready = kv_empty + NST;   // QK(j) done
-    uint64_t* s_free = s_ready + 1;       // S(j) loaded by all four softmax warps
-    uint64_t* p_ready = s_free + 1;       // P(j) written by all four softmax warps
+    uint64_t* s_free = s_ready + 1;       // S(j) loaded by all softmax warps
+    uint64_t* p_ready = s_free + 1;       // P(j) written by all softmax warps
     uint64_t* o_ready = p_ready + 1;      // PV(j) done
-    uint64_t* xfull = o_ready + 1;        // [NXB][4] the peer's partial scores of warp w's rows arrived
-    uint64_t* xempty = xfull + 4 * NXB;   // [NXB][4] the peer has consumed this CTA's partial for warp w's rows
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xempty + 4 * NXB);
+    uint64_t* xfull = o_ready + 1;        // [NSW] the peer's partial of warp w's block arrived
+    uint64_t* xempty = xfull + NSW;       // [NSW] the peer has consumed this CTA's partial of warp w's block
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xempty + NSW);
     __shared__ int s_abort;
 
     const uint32_t rank = cluster_rank();
@@ -148,24 +154,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
 
     if (threadIdx.x == 0) {
         s_abort = 0;
-        mbar_init(smem_u32(q_full), 4);
+        mbar_init(smem_u32(q_full), NSW);
         for (int s = 0; s < NST; ++s) {
             mbar_init(smem_u32(&kv_full[s]), 1);
             mbar_init(smem_u32(&kv_empty[s]), 1);
         }
         mbar_init(smem_u32(s_ready), 1);
-        mbar_init(smem_u32(s_free), 4);
-        mbar_init(smem_u32(p_ready), 4);
+        mbar_init(smem_u32(s_free), NSW);
+        mbar_init(smem_u32(p_ready), NSW);
         mbar_init(smem_u32(o_ready), 1);
-        for (int i = 0; i < 4 * NXB; ++i) {
+        for (int i = 0; i < NSW; ++i) {
             mbar_init(smem_u32(&xfull[i]), 1);
             mbar_init(smem_u32(&xempty[i]), 1);
         }
         fence_barrier_init();
-        // every exchange buffer starts open for the peer's partial scores
-        for (int i = 0; i < 4 * NXB; ++i) mbar_arrive_expect_tx(smem_u32(&xfull[i]), XBUF / 4);
+        // the exchange buffer starts open for the peer's partial scores
+        for (int i = 0; i < NSW; ++i) mbar_arrive_expect_tx(smem_u32(&xfull[i]), XBUF / NSW);
     }
-    if (warp == 5) {
+    if (warp == NSW + 1) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
@@ -174,7 +180,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (n_tiles > 0 && warp == 4) {
+    if (n_tiles > 0 && warp == NSW) {
         // ------------------------------- TMA producer -------------------------------
         if (lane == 0) {
             prefetch_tensormap(&tm_lat);
@@ -196,7 +202,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
             for (int i = issued - 1; i >= 0 && i >= issued - NST; --i)
                 mbar_wait(smem_u32(&kv_full[i % NST]), (i / NST) & 1, p.status);
         }
-    } else if (n_tiles > 0 && warp == 5) {
+    } else if (n_tiles > 0 && warp == NSW + 1) {
         // ------------------------------- MMA issuer -------------------------------
         // Per step j: QK(j) once the softmax warps have loaded S(j-1), then PV(j-2) once P(j-2)
         // is in tensor memory.  The softmax warps load S(j-1) before they compute P(j-2), so
@@ -253,28 +259,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                 __syncwarp();
             }
         }
-    } else if (warp < 4) {
+    } else if (warp < NSW) {
         // ------------------------- softmax / exchange warps -------------------------
-        // Each warp owns 32 head rows and its own exchange barriers, so the four warps never wait
-        // for one another.
-        const int h = warp * 32 + lane;  // head row == TMEM lane
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        // the peer's exchange buffer rows and barriers of this warp
-        const uint32_t xrem0 = mapa_peer(smem_u32(smem + OFF_X) + warp * 32 * XROW, peer);  // this warp's rows
-        uint8_t* outrow = smem + OFF_OUT + h * XROW;
-        const uint32_t xfull_rem0 = mapa_peer(smem_u32(&xfull[warp]), peer);
-        const uint32_t xempty_rem0 = mapa_peer(smem_u32(&xempty[warp]), peer);
-        const int sw = h & 7;
+        // Warp w owns head rows 32(w%4) .. +31 (its TMEM lane quarter) and score columns
+        // [32(w/4), +32) of every tile, with its own exchange barriers; the two warps of a lane
+        // quarter meet once per tile to combine their row maxima.
+        const int qw = warp & 3, half = warp >> 2;
+        const int h = qw * 32 + lane;  // head row == TMEM lane
+        const uint32_t lane_base = (uint32_t)(qw * 32) << 16;
+        const int col0 = half * CW;
+        const int blk = half * 128 * XROW + qw * 32 * XROW;  // this warp's block in the exchange buffer
+        // the peer's exchange block and barriers of this warp
+        const uint32_t xrem = mapa_peer(smem_u32(smem + OFF_X + blk), peer);
+        const uint32_t xfull_rem = mapa_peer(smem_u32(&xfull[warp]), peer);
+        const uint32_t xempty_rem = mapa_peer(smem_u32(&xempty[warp]), peer);
+        uint8_t* outrow = smem + OFF_OUT + blk + lane * XROW;
+        const int sw = lane & 7;
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
         if (n_tiles > 0) {
             // this rank's 288 values of the query row [q~_h ; q^R_h] -> tensor memory (A operand of the
             // score MMA, K-major: column c holds values 2c and 2c+1): rank 0 q~[0:288), rank 1
-            // q~[288:512) followed by q^R
+            // q~[288:512) followed by q^R.  Nine 16-column chunks: the first warp of the lane
+            // quarter writes chunks 0-4, the second 5-8.
             const uint4* qt = reinterpret_cast<const uint4*>(p.q_t + ((size_t)(b * p.s_q + t) * p.h_q + h) * 512);
             const uint4* qr = reinterpret_cast<const uint4*>(p.q_r + (((size_t)b * p.h_q + h) * p.s_q + t) * 64);
-#pragma unroll
-            for (int c0 = 0; c0 < KSTEPS / 2; ++c0) {  // 9 x 16 columns = 288 values
+            for (int c0 = half * 5; c0 < (half ? KSTEPS / 2 : 5); ++c0) {
                 uint32_t w[16];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
@@ -292,22 +302,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(q_full));
         }
-        uint32_t cur[NT];
-        // this rank's partial of tile j: registers, release the TMEM tile, send it to the peer
+        uint32_t cur[CW];
+        // this warp's block of the partial of tile j: registers, release the TMEM tile, send it
         auto fetch_and_send = [&](int j) {
             if (ok) ok = mbar_wait(smem_u32(s_ready), j & 1, p.status);
             tc_fence_after();
-#pragma unroll
-            for (int c0 = 0; c0 < NT; c0 += 16) tmem_ld16(tmem + lane_base + T_S + c0, cur + c0);
+            tmem_ld16(tmem + lane_base + T_S + col0, cur);
+            tmem_ld16(tmem + lane_base + T_S + col0 + 16, cur + 16);
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(s_free));
-            // the outbox rows of this warp are free once the previous bulk copy has read them
+            // the outbox block of this warp is free once the previous bulk copy has read it
             if (lane == 0) bulk_wait_read();
             __syncwarp();
 #pragma unroll
-            for (int c = 0; c < NT / 4; ++c)
+            for (int c = 0; c < CW / 4; ++c)
                 *reinterpret_cast<uint4*>(outrow + ((c ^ sw) << 4)) =
                     make_uint4(cur[4 * c], cur[4 * c + 1], cur[4 * c + 2], cur[4 * c + 3]);
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the copy engine
@@ -315,43 +325,66 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
             if (lane == 0) {
                 // the peer's buffer is free once it has consumed partial j-1
                 if (ok && j >= 1) ok = mbar_wait(smem_u32(&xempty[warp]), (j - 1) & 1, p.status);
-                if (ok)
-                    bulk_copy_to_peer(xrem0, smem_u32(smem + OFF_OUT + warp * 32 * XROW), 32 * XROW, xfull_rem0);
+                if (ok) bulk_copy_to_peer(xrem, smem_u32(smem + OFF_OUT + blk), 32 * XROW, xfull_rem);
                 bulk_commit();
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
         };
+        // combine a per-row value with the partner warp's through TMEM column T_R + col (+ 1 for
+        // the partner's); both warps of the lane quarter call it with the same col
+        auto swap_with_partner = [&](float v, uint32_t col) -> float {
+            tmem_st1(tmem + lane_base + T_R + col + half, __float_as_uint(v));
+            tmem_st_wait();
+            tc_fence_before();
+            named_barrier(1 + qw, 64);
+            tc_fence_after();
+            const uint32_t o = tmem_ld1(tmem + lane_base + T_R + col + (half ^ 1));
+            tmem_ld_wait();
+            return __uint_as_float(o);
+        };
         if (n_tiles > 0) fetch_and_send(0);
         for (int i = 0; i < n_tiles; ++i) {
-            // ---- the peer's partial of tile i, added to this rank's ----
+            // ---- the peer's partial of this block, added to this rank's ----
             if (ok) ok = mbar_wait(smem_u32(&xfull[warp]), i & 1, p.status);
-            float s[NT];
-            const uint8_t* xr = smem + OFF_X + h * XROW;
+            float s[CW];
+            const uint8_t* xr = smem + OFF_X + blk + lane * XROW;
 #pragma unroll
-            for (int c = 0; c < NT / 4; ++c) {
+            for (int c = 0; c < CW / 4; ++c) {
                 const float4 v = *reinterpret_cast<const float4*>(xr + ((c ^ sw) << 4));
-                s[4 * c] = __uint_as_float(cur[4 * c]) + v.x;
-                s[4 * c + 1] = __uint_as_float(cur[4 * c + 1]) + v.y;
-                s[4 * c + 2] = __uint_as_float(cur[4 * c + 2]) + v.z;
-                s[4 * c + 3] = __uint_as_float(cur[4 * c + 3]) + v.w;
+                const float2 a = __fadd2_rn(make_float2(__uint_as_float(cur[4 * c]), __uint_as_float(cur[4 * c + 1])),
+                                            make_float2(v.x, v.y));
+                const float2 bb = __fadd2_rn(
+                    make_float2(__uint_as_float(cur[4 * c + 2]), __uint_as_float(cur[4 * c + 3])), make_float2(v.z, v.w));
+                s[4 * c] = a.x;
+                s[4 * c + 1] = a.y;
+                s[4 * c + 2] = bb.x;
+                s[4 * c + 3] = bb.y;
             }
             __syncwarp();
             if (lane == 0 && i + 1 < n_tiles) {
-                mbar_arrive_expect_tx(smem_u32(&xfull[warp]), XBUF / 4);  // reopen for tile i + 1 ...
-                remote_arrive(xempty_rem0);                                // ... and tell the peer
+                mbar_arrive_expect_tx(smem_u32(&xfull[warp]), XBUF / NSW);  // reopen for tile i + 1 ...
+                remote_arrive(xempty_rem);                                   // ... and tell the peer
             }
             // ---- tile i+1 goes out before tile i is finished ----
             if (i + 1 < n_tiles) fetch_and_send(i + 1);
             // ---- mask, online softmax ----
-            const int k0 = kbeg + i * NT;
-            if (k0 + NT <= kend) {
+            const int k0 = kbeg + i * NT + col0;
+            const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+            if (kbeg + (i + 1) * NT <= kend) {
 #pragma unroll
-                for (int j = 0; j < NT; ++j) s[j] *= p.scale_log2;
+                for (int j = 0; j < CW; j += 2) {
+                    const float2 v = __fmul2_rn(make_float2(s[j], s[j + 1]), sc2);
+                    s[j] = v.x;
+                    s[j + 1] = v.y;
+                }
             } else {
 #pragma unroll
-                for (int j = 0; j < NT; ++j) s[j] = (k0 + j < kend) ? s[j] * p.scale_log2 : -INFINITY;
+                for (int j = 0; j < CW; ++j) s[j] = (k0 + j < kend) ? s[j] * p.scale_log2 : -INFINITY;
             }
-            const float m_new = fmaxf(m_ref, tree_max<NT>(s));
+            // row maximum of the whole tile: this warp's half and the partner warp's half
+            float mx = tree_max<CW>(s);
+            mx = fmaxf(mx, swap_with_partner(mx, 2u * (i & 1)));
+            const float m_new = fmaxf(m_ref, mx);
             bool resc = false;
             float alpha = 1.f;
             float m_use = m_ref;
@@ -362,20 +395,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                 alpha = fast_exp2(m_ref - m_new);
                 m_use = m_new;
             }
-            uint32_t pk[NT / 2];
+            uint32_t pk[CW / 2];
             const float m_sub = m_use == -INFINITY ? 0.f : m_use;  // all scores -inf: p = 2^-inf = 0
+            const float2 nm2 = make_float2(-m_sub, -m_sub);
 #pragma unroll
-            for (int j = 0; j < NT; ++j) s[j] = fast_exp2(s[j] - m_sub);
-#pragma unroll
-            for (int j = 0; j < NT; j += 2) pk[j / 2] = pack_bf16x2(s[j], s[j + 1]);
-            const float rs = tree_sum<NT>(s);
-            l = (resc ? l * alpha : l) + rs;
+            for (int j = 0; j < CW; j += 2) {
+                const float2 v = __fadd2_rn(make_float2(s[j], s[j + 1]), nm2);
+                s[j] = fast_exp2(v.x);
+                s[j + 1] = fast_exp2(v.y);
+                pk[j / 2] = pack_bf16x2(s[j], s[j + 1]);
+            }
+            const float rs = tree_sum<CW>(s);
+            l = (resc ? l * alpha : l) + rs;  // this warp's share of the row sum
             m_ref = m_use;
             // PV(i-1) must be done: it reads the P buffer, and a rescale of O must follow its update
             if (ok && i >= 1) ok = mbar_wait(smem_u32(o_ready), (i - 1) & 1, p.status);
             tc_fence_after();
             if (__any_sync(0xffffffffu, resc)) {
-                for (int c0 = 0; c0 < 256; c0 += 16) {
+                // each warp of the pair rescales half of this rank's 256 output columns
+                for (int c0 = half * 128; c0 < half * 128 + 128; c0 += 16) {
                     uint32_t o[16];
                     tmem_ld16(tmem + lane_base + T_O + c0, o);
                     tmem_ld_wait();
@@ -384,8 +422,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                     tmem_st16(tmem + lane_base + T_O + c0, o);
                 }
             }
-            tmem_st16(tmem + lane_base + T_P, pk);
-            tmem_st16(tmem + lane_base + T_P + 16, pk + 16);
+            tmem_st16(tmem + lane_base + T_P + half * (CW / 2), pk);
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
@@ -393,7 +430,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         }
         if (lane == 0) bulk_wait_all();
         if (!ok) s_abort = 1;
-        // ---- epilogue: normalise this rank's 256 output columns ----
+        // ---- epilogue: the full row sum, then normalise this warp's 128 output columns ----
+        l += swap_with_partner(l, 4u);
         const int last = n_tiles - 1;
         if (ok && n_tiles > 0 && mbar_wait(smem_u32(o_ready), last & 1, p.status)) {
             tc_fence_after();
@@ -404,7 +442,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
             __nv_bfloat16* orow =
                 p.o_lat + ((size_t)grp * p.B * HPG * p.s_q + (size_t)(b * HPG + hh) * p.s_q + t) * 512 + rank * 256;
             float* prt = p.nsplit > 1 ? p.part_o + (prow * p.nsplit + split) * 512 + rank * 256 : nullptr;
-            for (int c0 = 0; c0 < 256; c0 += 16) {
+            for (int c0 = half * 128; c0 < half * 128 + 128; c0 += 16) {
                 uint32_t o[16];
                 tmem_ld16(tmem + lane_base + T_O + c0, o);
                 tmem_ld_wait();
@@ -424,7 +462,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                     d[1] = make_uint4(pkk[4], pkk[5], pkk[6], pkk[7]);
                 }
             }
-            if (rank == 0) {
+            if (rank == 0 && half == 0) {
                 const float lse2 = l > 0.f ? m_ref + log2f(l) : -INFINITY;
                 if (p.nsplit > 1)
                     p.part_lse[prow * p.nsplit + split] = lse2;
@@ -437,7 +475,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     tc_fence_before();
     __syncwarp();
     cluster_sync();
-    if (warp == 5) tmem_dealloc(tmem, 512);
+    if (warp == NSW + 1) tmem_dealloc(tmem, 512);
 }
 
 // Merge of the split partials of the latent attention (same rule as the GQA
@@ -498,7 +536,7 @@ cudaError_t latent_attn_launch(const CUtensorMap& tm_lat, const LatentParams& p,
     dim3 grid(2 * p.s_q * p.nsplit, p.B);
     {
         TimedLaunch timer(st);
-        latent_attn_kernel<<<grid, 192, lat::SMEM, st>>>(tm_lat, p);
+        latent_attn_kernel<<<grid, lat::NTHREADS, lat::SMEM, st>>>(tm_lat, p);
         timer.stop();
     }
     e = cudaPeekAtLastError();
