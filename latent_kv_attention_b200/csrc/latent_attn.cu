@@ -49,6 +49,7 @@ namespace lka {
 namespace lat {
 constexpr int NT = 64;          // tokens per tile (the N of the score MMA)
 constexpr int NST = 4;          // TMA ring depth
+constexpr int PF = 6;           // L2 prefetch distance in tiles
 constexpr int NKB = 5;          // 64-value boxes per rank and tile
 constexpr int KSTEPS = 18;      // K = 16 steps of this rank's 288 score values
 constexpr int BOX = NT * 128;   // one 64-value box of NT tokens
@@ -184,6 +185,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(lat::NTHREADS, 1)
         // ------------------------------- TMA producer -------------------------------
         if (lane == 0) {
             prefetch_tensormap(&tm_lat);
+            // tiles PF ahead of the one being loaded are prefetched into L2, so that the ring (whose
+            // stages stay busy until P*V) is refilled from L2 rather than from DRAM
+            auto prefetch = [&](int i) {
+                const int y = b * p.Lmax + kbeg + i * NT;
+                for (int kb = 0; kb < NKB; ++kb) tma_prefetch_2d(&tm_lat, (int)rank * 256 + kb * 64, y);
+            };
+            for (int i = NST; i < min(n_tiles, PF); ++i) prefetch(i);
             int issued = 0;
             for (int i = 0; i < n_tiles; ++i) {
                 const int s = i % NST;
@@ -197,6 +205,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(lat::NTHREADS, 1)
                 const uint32_t dst = smem_u32(smem + OFF_KV + s * STAGE);
                 const int y = b * p.Lmax + kbeg + i * NT;
                 for (int kb = 0; kb < NKB; ++kb) tma_load_2d(dst + kb * BOX, &tm_lat, (int)rank * 256 + kb * 64, y, fb);
+                if (i + PF < n_tiles) prefetch(i + PF);
                 ++issued;
             }
             for (int i = issued - 1; i >= 0 && i >= issued - NST; --i)
