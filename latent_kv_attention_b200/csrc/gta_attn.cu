@@ -14,9 +14,12 @@
 // first.  Warp 4 streams 128-key tiles of K_gamma and the V tiles of the
 // group's heads with TMA (2 stages of 80 KB); warp 5 issues S = Q K^T
 // (M = N = 128, K = 64) into tensor memory and, once the softmax has written P
-// back to tensor memory as bf16, one P*V MMA chain per head (M = 128, N = 64,
-// K = 128; A = P from tensor memory) -- the score tile is computed and
-// normalised once and reused by all heads of the group.  Warps 0-3 hold one
+// back to tensor memory as bf16, P*V for all heads of the group at once
+// (M = 128, N = 64 x heads, K = 128; A = P from tensor memory; the heads' value
+// tiles sit one box apart, which is the stride between the 64-column blocks of
+// the B operand) -- the score tile is computed and normalised once and reused
+// by all heads of the group.  A tcgen05.mma costs about the same for any N up
+// to 256, so one wide MMA replaces one per head.  Warps 0-3 hold one
 // query row per thread: mask, online softmax with lazy rescaling (the running
 // maximum only moves when it grows by more than 2^8), P to tensor memory.
 #include "common.cuh"
@@ -156,7 +159,7 @@ __global__ void __launch_bounds__(192, 1)
     } else if (warp == 5) {
         // ------------------------------ MMA issuer ------------------------------
         constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
-        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 64, false, true);
+        const uint32_t idesc_pv = idesc_bf16_f32(128, 64 * HPG, false, true);
         bool ok = mbar_wait(smem_u32(q_full), 0, p.status);
         // zero the rows of a tile past the cache length (they may hold anything, even NaN)
         auto zero_tail = [&](uint8_t* base, int nbox, int j) {
@@ -200,11 +203,10 @@ __global__ void __launch_bounds__(192, 1)
             tc_fence_after();
             if (lane == 0) {
                 const uint32_t va = smem_u32(vt);
-                for (int hh = 0; hh < HPG; ++hh)
 #pragma unroll
-                    for (int kk = 0; kk < TK / 16; ++kk)
-                        umma_ts(tmem + T_O + hh * 64, tmem + T_P + (j & 1) * 64 + kk * 8,
-                                smem_desc_sw128(va + hh * BOX + kk * 2048, BOX, 1024), idesc_pv, (j | kk) != 0);
+                for (int kk = 0; kk < TK / 16; ++kk)
+                    umma_ts(tmem + T_O, tmem + T_P + (j & 1) * 64 + kk * 8, smem_desc_sw128(va + kk * 2048, BOX, 1024),
+                            idesc_pv, (j | kk) != 0);
                 umma_commit(smem_u32(&v_empty[sv]));
                 umma_commit(smem_u32(&o_ready[j & 1]));
             }
