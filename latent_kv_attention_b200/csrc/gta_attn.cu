@@ -11,17 +11,19 @@
 // Prefill is dense in both contractions, so both run as tcgen05 MMAs.
 //
 // One CTA = (128-query tile, group, sequence); q-tiles are scheduled longest
-// first.  Warp 4 streams 128-key tiles of K_gamma and the V tiles of the
-// group's heads with TMA (2 stages of 80 KB); warp 5 issues S = Q K^T
+// first.  Warp 8 streams 128-key tiles of K_gamma and the V tiles of the
+// group's heads with TMA (2 stages of 80 KB); warp 9 issues S = Q K^T
 // (M = N = 128, K = 64) into tensor memory and, once the softmax has written P
 // back to tensor memory as bf16, P*V for all heads of the group at once
 // (M = 128, N = 64 x heads, K = 128; A = P from tensor memory; the heads' value
 // tiles sit one box apart, which is the stride between the 64-column blocks of
 // the B operand) -- the score tile is computed and normalised once and reused
 // by all heads of the group.  A tcgen05.mma costs about the same for any N up
-// to 256, so one wide MMA replaces one per head.  Warps 0-3 hold one
-// query row per thread: mask, online softmax with lazy rescaling (the running
-// maximum only moves when it grows by more than 2^8), P to tensor memory.
+// to 256, so one wide MMA replaces one per head.  Warps 0-7 run the mask and
+// the online softmax, two warps per group of 32 query rows (warps w and w + 4
+// take the two 64-key halves of the tile and combine their row maxima through
+// shared memory), with lazy rescaling (the running maximum only moves when it
+// grows by more than 2^8); P goes to tensor memory.
 #include "common.cuh"
 #include "host_util.h"
 #include "tc.cuh"
@@ -46,7 +48,11 @@ constexpr int VSTAGE = 4 * BOX;     // up to 4 heads' value tiles
 constexpr int OFF_Q = 0;
 constexpr int OFF_K = BOX;
 constexpr int OFF_V = OFF_K + NSK * BOX;
-constexpr int OFF_BAR = OFF_V + NSV * VSTAGE;
+constexpr int NSW = 8;              // softmax warps: 4 lane quarters x 2 key halves
+constexpr int CW = TK / 2;          // score columns per softmax warp
+constexpr int NTHREADS = 32 * (NSW + 2);
+constexpr int OFF_RED = OFF_V + NSV * VSTAGE;  // float [2][NSW][32] row maxima + [NSW][32] row sums
+constexpr int OFF_BAR = OFF_RED + 3 * NSW * 32 * 4;
 constexpr int SMEM = 1024 + OFF_BAR + 256;
 constexpr int K_LEAD = 2;           // key tiles the producer keeps ahead of the value tiles
 constexpr uint32_t T_O = 0;         // 4 heads x 64 fp32 columns
@@ -54,7 +60,7 @@ constexpr uint32_t T_S = 256;       // 128 fp32 columns
 constexpr uint32_t T_P = 384;       // 2 x 64 columns of bf16 pairs (double-buffered P)
 }  // namespace gta
 
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(gta::NTHREADS, 1)
     gta_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const GtaParams p) {
     using namespace gta;
@@ -97,14 +103,14 @@ __global__ void __launch_bounds__(192, 1)
             mbar_init(smem_u32(&v_empty[s]), 1);
         }
         mbar_init(smem_u32(s_ready), 1);
-        mbar_init(smem_u32(s_free), 4);
+        mbar_init(smem_u32(s_free), NSW);
         for (int i = 0; i < 2; ++i) {
-            mbar_init(smem_u32(&p_ready[i]), 4);
+            mbar_init(smem_u32(&p_ready[i]), NSW);
             mbar_init(smem_u32(&o_ready[i]), 1);
         }
         fence_barrier_init();
     }
-    if (warp == 5) {
+    if (warp == NSW + 1) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
@@ -113,7 +119,7 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 4) {
+    if (warp == NSW) {
         // ------------------------------ producer ------------------------------
         // issue order K(0..K_LEAD-1), then per tile i: K(i + K_LEAD), V(i)
         if (lane == 0) {
@@ -156,7 +162,7 @@ __global__ void __launch_bounds__(192, 1)
                 mbar_wait(smem_u32(&v_full[i % NSV]), (i / NSV) & 1, p.status);
             mbar_wait(qb, 0, p.status);
         }
-    } else if (warp == 5) {
+    } else if (warp == NSW + 1) {
         // ------------------------------ MMA issuer ------------------------------
         constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
         const uint32_t idesc_pv = idesc_bf16_f32(128, 64 * HPG, false, true);
@@ -213,35 +219,52 @@ __global__ void __launch_bounds__(192, 1)
             __syncwarp();
         }
     } else {
-        // --------------------------- softmax warps 0-3 ---------------------------
-        const int row = warp * 32 + lane;  // query row in the tile == TMEM lane
+        // --------------------------- softmax warps 0-7 ---------------------------
+        // Warp w: query rows 32(w%4) .. +31 (its TMEM lane quarter), key columns [64(w/4), +64)
+        // of every tile; output columns are split between the two warps in alternate 16-column
+        // chunks.
+        const int qw = warp & 3, half = warp >> 2;
+        const int row = qw * 32 + lane;  // query row in the tile == TMEM lane
         const int q = q0 + row;
         const bool row_ok = q < p.s_q;
         const int vis_end = row_ok ? (p.causal ? L - p.s_q + q + 1 : L) : 0;  // keys < vis_end are visible
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const uint32_t lane_base = (uint32_t)(qw * 32) << 16;
+        const int col0 = half * CW;
+        float* red_max = reinterpret_cast<float*>(smem + OFF_RED);  // [2][NSW][32]
+        float* red_sum = red_max + 2 * NSW * 32;                    // [NSW][32]
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
         for (int j = 0; j < n_tiles; ++j) {
             if (ok) ok = mbar_wait(smem_u32(s_ready), j & 1, p.status);
             tc_fence_after();
-            uint32_t sr[TK];
+            uint32_t sr[CW];
 #pragma unroll
-            for (int c0 = 0; c0 < TK; c0 += 16) tmem_ld16(tmem + lane_base + T_S + c0, sr + c0);
+            for (int c0 = 0; c0 < CW; c0 += 16) tmem_ld16(tmem + lane_base + T_S + col0 + c0, sr + c0);
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(s_free));  // the next score tile may be written
-            const int k0 = j * TK;
+            const int k0 = j * TK + col0;
             float* sf = reinterpret_cast<float*>(sr);
-            if (k0 + TK <= vis_end) {
+            if (j * TK + TK <= vis_end) {
+                const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
 #pragma unroll
-                for (int c = 0; c < TK; ++c) sf[c] = __uint_as_float(sr[c]) * p.scale_log2;
+                for (int c = 0; c < CW; c += 2) {
+                    const float2 v = __fmul2_rn(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sc2);
+                    sf[c] = v.x;
+                    sf[c + 1] = v.y;
+                }
             } else {
 #pragma unroll
-                for (int c = 0; c < TK; ++c)
+                for (int c = 0; c < CW; ++c)
                     sf[c] = (k0 + c < vis_end) ? __uint_as_float(sr[c]) * p.scale_log2 : -INFINITY;
             }
-            const float m_new = fmaxf(m_ref, tree_max<TK>(sf));
+            // row maximum of the whole tile: this warp's half and the partner warp's half
+            float mx = tree_max<CW>(sf);
+            red_max[((j & 1) * NSW + warp) * 32 + lane] = mx;
+            named_barrier(1 + qw, 64);
+            mx = fmaxf(mx, red_max[((j & 1) * NSW + (warp ^ 4)) * 32 + lane]);
+            const float m_new = fmaxf(m_ref, mx);
             bool resc = false;
             float alpha = 1.f, m_use = m_ref;
             if (m_ref == -INFINITY) {
@@ -251,14 +274,18 @@ __global__ void __launch_bounds__(192, 1)
                 alpha = fast_exp2(m_ref - m_new);
                 m_use = m_new;
             }
-            uint32_t pk[TK / 2];
+            uint32_t pk[CW / 2];
             const float m_sub = m_use == -INFINITY ? 0.f : m_use;  // all scores -inf: p = 2^-inf = 0
+            const float2 nm2 = make_float2(-m_sub, -m_sub);
 #pragma unroll
-            for (int c = 0; c < TK; ++c) sf[c] = fast_exp2(sf[c] - m_sub);
-#pragma unroll
-            for (int c = 0; c < TK; c += 2) pk[c / 2] = pack_bf16x2(sf[c], sf[c + 1]);
-            const float rs = tree_sum<TK>(sf);
-            l = (resc ? l * alpha : l) + rs;
+            for (int c = 0; c < CW; c += 2) {
+                const float2 v = __fadd2_rn(make_float2(sf[c], sf[c + 1]), nm2);
+                sf[c] = fast_exp2(v.x);
+                sf[c + 1] = fast_exp2(v.y);
+                pk[c / 2] = pack_bf16x2(sf[c], sf[c + 1]);
+            }
+            const float rs = tree_sum<CW>(sf);
+            l = (resc ? l * alpha : l) + rs;  // this warp's share of the row sum
             m_ref = m_use;
             // P buffer j&1 was last read by PV(j-2); O may only be rescaled after PV(j-1)
             if (ok && j >= 2) ok = mbar_wait(smem_u32(&o_ready[j & 1]), ((j >> 1) - 1) & 1, p.status);
@@ -267,9 +294,10 @@ __global__ void __launch_bounds__(192, 1)
                 ok = mbar_wait(smem_u32(&o_ready[(j - 1) & 1]), ((j - 1) >> 1) & 1, p.status);
             tc_fence_after();
 #pragma unroll
-            for (int c0 = 0; c0 < TK / 2; c0 += 16) tmem_st16(tmem + lane_base + T_P + (j & 1) * 64 + c0, pk + c0);
+            for (int c0 = 0; c0 < CW / 2; c0 += 16)
+                tmem_st16(tmem + lane_base + T_P + (j & 1) * 64 + half * (CW / 2) + c0, pk + c0);
             if (any_resc) {
-                for (int c0 = 0; c0 < 64 * HPG; c0 += 16) {
+                for (int c0 = half * 16; c0 < 64 * HPG; c0 += 32) {
                     uint32_t o[16];
                     tmem_ld16(tmem + lane_base + T_O + c0, o);
                     tmem_ld_wait();
@@ -283,37 +311,40 @@ __global__ void __launch_bounds__(192, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&p_ready[j & 1]));
         }
+        // the full row sum
+        red_sum[warp * 32 + lane] = l;
+        named_barrier(1 + qw, 64);
+        l += red_sum[(warp ^ 4) * 32 + lane];
         if (ok) ok = mbar_wait(smem_u32(&o_ready[(n_tiles - 1) & 1]), ((n_tiles - 1) >> 1) & 1, p.status);
         if (!ok) {
             s_abort = 1;
         } else {
             tc_fence_after();
             const float inv_l = l > 0.f ? 1.f / l : 0.f;
-            for (int hh = 0; hh < HPG; ++hh) {
-                for (int c0 = 0; c0 < 64; c0 += 16) {
-                    uint32_t o[16];
-                    tmem_ld16(tmem + lane_base + T_O + hh * 64 + c0, o);
-                    tmem_ld_wait();
-                    if (row_ok) {
-                        uint32_t pkk[8];
+            for (int c0 = half * 16; c0 < 64 * HPG; c0 += 32) {
+                const int hh = c0 / 64;
+                uint32_t o[16];
+                tmem_ld16(tmem + lane_base + T_O + c0, o);
+                tmem_ld_wait();
+                if (row_ok) {
+                    uint32_t pkk[8];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            pkk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
-                        uint4* d = reinterpret_cast<uint4*>(
-                            p.out + (((size_t)b * p.H + grp * HPG + hh) * p.s_q + q) * 64 + c0);
-                        d[0] = make_uint4(pkk[0], pkk[1], pkk[2], pkk[3]);
-                        d[1] = make_uint4(pkk[4], pkk[5], pkk[6], pkk[7]);
-                    }
+                    for (int e = 0; e < 8; ++e)
+                        pkk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+                    uint4* d = reinterpret_cast<uint4*>(p.out + (((size_t)b * p.H + grp * HPG + hh) * p.s_q + q) * 64 +
+                                                        (c0 % 64));
+                    d[0] = make_uint4(pkk[0], pkk[1], pkk[2], pkk[3]);
+                    d[1] = make_uint4(pkk[4], pkk[5], pkk[6], pkk[7]);
                 }
             }
-            if (row_ok && p.lse)
+            if (row_ok && p.lse && half == 0)
                 p.lse[((size_t)b * p.G + grp) * p.s_q + q] =
                     (l > 0.f ? m_ref + log2f(l) : -INFINITY) * 0.69314718055994530942f;
         }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) tmem_dealloc(tmem, 512);
+    if (warp == NSW + 1) tmem_dealloc(tmem, 512);
 }
 
 }  // namespace lka
@@ -367,7 +398,7 @@ lka_status_t gta_shared_score_attn(const void* q_g, const void* k_g, const void*
         return LKA_ERR_CUDA;
     dim3 grid(cdiv(s_q, gta::TQ), G, B);
     TimedLaunch timer(st);
-    gta_attn_kernel<<<grid, 192, gta::SMEM, st>>>(tq, tk, tv, p);
+    gta_attn_kernel<<<grid, gta::NTHREADS, gta::SMEM, st>>>(tq, tk, tv, p);
     timer.stop();
     return cudaPeekAtLastError() == cudaSuccess ? LKA_OK : LKA_ERR_CUDA;
 }
