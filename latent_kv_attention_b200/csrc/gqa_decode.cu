@@ -277,6 +277,25 @@ __global__ void __launch_bounds__(160, GqaCfg<T, D, RB>::MINB)
     float* aw = a_buf + warp * RB;
     bool aborted = false;
 
+    // Byte offsets, inside a stage, of the chunks this lane reads.  Score phase: token row jt = warp * TW +
+    // ps * P + tok_in_pass; TW is a multiple of 8, so the swizzle phase jt & 7 only depends on ps through
+    // (ps * P) & 7, which takes NCLS values.  Value phase: row warp * TW + jj has swizzle phase jj & 7.
+    constexpr int NCLS = C::P >= 8 ? 1 : 8 / C::P;
+    uint32_t koff[NCLS][C::CPL];
+#pragma unroll
+    for (int cls = 0; cls < NCLS; ++cls)
+#pragma unroll
+        for (int c = 0; c < C::CPL; ++c) {
+            int seg, chunk;
+            lane_chunk<C::LPT, C::NSEG>(li, c, seg, chunk);
+            koff[cls][c] = swz_off<C::T_TILE>(seg, warp * C::TW + cls * C::P + tok_in_pass, chunk);
+        }
+    const int v_ob = lane * C::DPLV * C::E;  // byte offset of this lane's value slice in a row
+    const int v_seg = v_ob / 128, v_chunk = (v_ob % 128) / 16, v_in = v_ob % 16;
+    uint32_t voff[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) voff[k] = swz_off<C::T_TILE>(v_seg, warp * C::TW + k, v_chunk) + v_in;
+
     for (int it = 0; it < n_tiles; ++it) {
         const int s = it % C::NSTAGE;
         if (!mbar_wait(smem_u32(&bars[s]), (it / C::NSTAGE) & 1, p.status)) {
@@ -298,10 +317,8 @@ __global__ void __launch_bounds__(160, GqaCfg<T, D, RB>::MINB)
             for (int r = 0; r < RB; ++r) acc2[r] = make_float2(0.f, 0.f);
 #pragma unroll
             for (int c = 0; c < C::CPL; ++c) {
-                int seg, chunk;
-                lane_chunk<C::LPT, C::NSEG>(li, c, seg, chunk);
                 float kf[C::EPC];
-                load_chunk<T>(kt + swz_off<C::T_TILE>(seg, jt, chunk), kf);
+                load_chunk<T>(kt + koff[ps % NCLS][c] + (ps / NCLS) * NCLS * C::P * 128, kf);
 #pragma unroll
                 for (int r = 0; r < RB; ++r)
 #pragma unroll
@@ -369,22 +386,47 @@ __global__ void __launch_bounds__(160, GqaCfg<T, D, RB>::MINB)
 #pragma unroll
             for (int d = 0; d < C::DPLV / 2; ++d) o[r][d] = __fmul2_rn(o[r][d], make_float2(al[r], al[r]));
         {
-            const int ob = lane * C::DPLV * C::E;  // byte offset of this lane's value slice in a row
-            const int vseg = ob / 128, vchunk = (ob % 128) / 16, vin = ob % 16;
             int nvalid = kend - (tbase + warp * C::TW);
             nvalid = nvalid < 0 ? 0 : (nvalid > C::TW ? C::TW : nvalid);
+            if (nvalid == C::TW) {
+                // every token of this warp's quarter is a key: fully unrolled, constant offsets
+#pragma unroll
+                for (int jj = 0; jj < C::TW; ++jj) {
+                    float vf[C::DPLV];
+                    load_v_slice<T, C::DPLV>(vt + voff[jj & 7] + (jj & ~7) * 128, vf);
+                    float2 pj[RB];
+                    if constexpr (RB % 2 == 0) {
+                        const float4* pr4 = reinterpret_cast<const float4*>(pw + jj * RB);
+#pragma unroll
+                        for (int rp = 0; rp < RB / 2; ++rp) {
+                            const float4 v4 = pr4[rp];
+                            pj[2 * rp] = make_float2(v4.x, v4.y);
+                            pj[2 * rp + 1] = make_float2(v4.z, v4.w);
+                        }
+                    } else {
+#pragma unroll
+                        for (int r = 0; r < RB; ++r) pj[r] = pw[jj * RB + r];
+                    }
+#pragma unroll
+                    for (int r = 0; r < RB; ++r)
+#pragma unroll
+                        for (int d = 0; d < C::DPLV / 2; ++d)
+                            o[r][d] = __ffma2_rn(pj[r], make_float2(vf[2 * d], vf[2 * d + 1]), o[r][d]);
+                }
+            } else {
 #pragma unroll 4
-            for (int jj = 0; jj < nvalid; ++jj) {
-                const int jt = warp * C::TW + jj;
-                float vf[C::DPLV];
-                load_v_slice<T, C::DPLV>(vt + swz_off<C::T_TILE>(vseg, jt, vchunk) + vin, vf);
-                const float2* pr = pw + jj * RB;
+                for (int jj = 0; jj < nvalid; ++jj) {
+                    const int jt = warp * C::TW + jj;
+                    float vf[C::DPLV];
+                    load_v_slice<T, C::DPLV>(vt + swz_off<C::T_TILE>(v_seg, jt, v_chunk) + v_in, vf);
+                    const float2* pr = pw + jj * RB;
 #pragma unroll
-                for (int r = 0; r < RB; ++r) {
-                    const float2 pj = pr[r];
+                    for (int r = 0; r < RB; ++r) {
+                        const float2 pj = pr[r];
 #pragma unroll
-                    for (int d = 0; d < C::DPLV / 2; ++d)
-                        o[r][d] = __ffma2_rn(pj, make_float2(vf[2 * d], vf[2 * d + 1]), o[r][d]);
+                        for (int d = 0; d < C::DPLV / 2; ++d)
+                            o[r][d] = __ffma2_rn(pj, make_float2(vf[2 * d], vf[2 * d + 1]), o[r][d]);
+                    }
                 }
             }
         }
