@@ -276,6 +276,12 @@ __global__ void __launch_bounds__(160, GqaCfg<T, D, RB>::MINB)
     float2* pw = p_buf + warp * C::TW * RB;
     float* aw = a_buf + warp * RB;
     bool aborted = false;
+    // keys below mask_from are visible to every row of the block: tiles below it need no mask
+    int mask_from = kend;
+    for (int r = 0; r < rows_here; ++r) {
+        const int last = p.causal ? L - p.s_q + (row0 + r) % p.s_q : L - 1;
+        mask_from = min(mask_from, last + 1);
+    }
 
     // Byte offsets, inside a stage, of the chunks this lane reads.  Score phase: token row jt = warp * TW +
     // ps * P + tok_in_pass; TW is a multiple of 8, so the swizzle phase jt & 7 only depends on ps through
@@ -349,42 +355,59 @@ __global__ void __launch_bounds__(160, GqaCfg<T, D, RB>::MINB)
                     acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], m);
                 }
             }
-            const int kpos = tbase + jt;
-            const bool ok = row_ok && kpos < kend && kpos <= my_last;
-            sc[ps] = ok ? acc[0] : -INFINITY;
+            if (tbase + C::T_TILE > mask_from) {
+                const int kpos = tbase + jt;
+                const bool ok = row_ok && kpos < kend && kpos <= my_last;
+                sc[ps] = ok ? acc[0] : -INFINITY;
+            } else {
+                sc[ps] = acc[0];
+            }
         }
 
-        // ---- online softmax over this warp's tokens (per row) ----
+        // ---- online softmax over this warp's tokens (per row), lazily rescaled: p is taken against a
+        // reference maximum m_run that only moves when a score exceeds it by more than 2^8 (the final
+        // O / l is exact); the row maximum is only reduced across the lanes when that happens ----
         float mx = sc[0];
 #pragma unroll
         for (int ps = 1; ps < C::NPASS; ++ps) mx = fmaxf(mx, sc[ps]);
+        if (__any_sync(0xffffffffu, mx > m_run + 8.0f)) {  // (an unset reference is exceeded by any key)
 #pragma unroll
-        for (int m = C::LPT; m < 32; m *= 2) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
-        const float m_new = fmaxf(m_run, mx);
-        const float m_ref = m_new == -INFINITY ? 0.f : m_new;
-        const float alpha = exp2f(m_run - m_ref);
-        float sum = 0.f;
+            for (int m = C::LPT; m < 32; m *= 2) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
+            const float m_new = fmaxf(m_run, mx);
+            float alpha = 1.f;
+            if (m_run == -INFINITY) {
+                m_run = m_new;  // O and l of the row are still zero
+            } else if (m_new > m_run + 8.0f) {
+                alpha = fast_exp2(m_run - m_new);
+                m_run = m_new;
+            }
+            if (__any_sync(0xffffffffu, alpha != 1.f)) {
+                l_run *= alpha;
+                if (tok_in_pass == 0 && li % C::DUP == 0) aw[my_row] = alpha;
+                __syncwarp();
+                float al[RB];
 #pragma unroll
-        for (int ps = 0; ps < C::NPASS; ++ps) {
-            const float pv = exp2f(sc[ps] - m_ref);
-            sum += pv;
-            if (li % C::DUP == 0) pw[(ps * C::P + tok_in_pass) * RB + my_row] = make_float2(pv, pv);
+                for (int r = 0; r < RB; ++r) al[r] = aw[r];
+#pragma unroll
+                for (int r = 0; r < RB; ++r)
+#pragma unroll
+                    for (int d = 0; d < C::DPLV / 2; ++d)
+                        o[r][d] = __fmul2_rn(o[r][d], make_float2(al[r], al[r]));
+                __syncwarp();
+            }
         }
+        {
+            const float m_sub = m_run == -INFINITY ? 0.f : m_run;  // no visible key yet: p = 2^-inf = 0
 #pragma unroll
-        for (int m = C::LPT; m < 32; m *= 2) sum += __shfl_xor_sync(0xffffffffu, sum, m);
-        l_run = l_run * alpha + sum;
-        m_run = m_new;
-        if (tok_in_pass == 0 && li % C::DUP == 0) aw[my_row] = alpha;
+            for (int ps = 0; ps < C::NPASS; ++ps) {
+                const float pv = fast_exp2(sc[ps] - m_sub);
+                l_run += pv;  // this lane's share; summed over the lanes of the row at the end
+                if (li % C::DUP == 0) pw[(ps * C::P + tok_in_pass) * RB + my_row] = make_float2(pv, pv);
+            }
+        }
         __syncwarp();
 
-        // ---- O = alpha * O + P V over this warp's tokens ----
-        float al[RB];
-#pragma unroll
-        for (int r = 0; r < RB; ++r) al[r] = aw[r];
-#pragma unroll
-        for (int r = 0; r < RB; ++r)
-#pragma unroll
-            for (int d = 0; d < C::DPLV / 2; ++d) o[r][d] = __fmul2_rn(o[r][d], make_float2(al[r], al[r]));
+        // ---- O += P V over this warp's tokens ----
         {
             int nvalid = kend - (tbase + warp * C::TW);
             nvalid = nvalid < 0 ? 0 : (nvalid > C::TW ? C::TW : nvalid);
@@ -433,6 +456,10 @@ __global__ void __launch_bounds__(160, GqaCfg<T, D, RB>::MINB)
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&bars[C::NSTAGE + s]));
     }
+
+    // the row sums: this lane's share summed over the token groups of the warp
+#pragma unroll
+    for (int m = C::LPT; m < 32; m *= 2) l_run += __shfl_xor_sync(0xffffffffu, l_run, m);
 
     // all consumer warps reach here; aborted CTAs stop without writing results
     named_barrier(1, 128);
