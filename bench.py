@@ -13,9 +13,9 @@ flushed between timed steps anyway.
 
 Unless --no-extras is given, the line also carries `other_paths`: the same
 measurement (step time, GB/s, TFLOP/s, tokens/s, roofline of the main kernel,
-end-to-end time) for the GQLA latent decode layer on the MQA-absorbed path
-(s_q = 1 and 2), on the per-group GQA path (s_q = 2), and for the GTA causal
-prefill.
+end-to-end time) for the GQA layer over a paged cache (64-token pages), the
+GQLA latent decode layer on the MQA-absorbed path (s_q = 1 and 2), on the
+per-group GQA path (s_q = 2), and for the GTA causal prefill.
 
 Prints ONE JSON line (rank 0).  `value` is the algorithmic HBM traffic of the
 step (every cache byte once, q read once, out written once) divided by the
@@ -241,6 +241,27 @@ class GqaDecode(Workload):
         return fn, nbytes, oracle.threads_used(0, n * w["h_q"]), f"first {n} of {w['B']} sequences"
 
 
+class GqaDecodePaged(GqaDecode):
+    """gqa_attn_paged over the same decode batch with the K/V cache in 64-token pages of a shuffled pool."""
+
+    def setup_device(self):
+        super().setup_device()
+        for k in ("k", "v"):  # the contiguous copies are not used by the paged step
+            self.inp.pop(k, None)
+        torch.cuda.empty_cache()
+
+    def step(self):
+        i = self.inp
+        self.lka.gqa_attn_paged(i["q"], i["k_pages"], i["v_pages"], i["block_table"], i["cache_lens"],
+                                causal=self.w["causal"], scale=i["scale"], out=self.out)
+
+    def config(self):
+        c = super().config()
+        c["page_size"] = self.w["page_size"]
+        c["cache_layout"] = "paged (shuffled page pool + block table)"
+        return c
+
+
 class LatentAbsorbed(Workload):
     """latent_absorbed_attn over the GQLA/MLA decode batch: absorb GEMM, latent attention, up-projection."""
 
@@ -397,6 +418,7 @@ GqaDecode.kernel_work = lambda self, pk: ("hbm", self.bytes)
 WORKLOAD_CLASSES = {
     "gqa_decode_llama8b": GqaDecode,
     "gqa_decode_llama8b_b16": GqaDecode,
+    "gqa_decode_llama8b_paged": GqaDecodePaged,
     "latent_decode_4k_sq1": LatentAbsorbed,
     "latent_decode_4k_sq2": LatentAbsorbed,
     "latent_expanded_4k_sq1": LatentExpanded,
@@ -407,7 +429,8 @@ WORKLOAD_CLASSES = {
     "latent_expanded_4k_sq2_b16": LatentExpanded,
     "gta_prefill_4k_b2": GtaPrefill,
 }
-EXTRAS = ["latent_decode_4k_sq1", "latent_decode_4k_sq2", "latent_expanded_4k_sq2", "gta_prefill_4k"]
+EXTRAS = ["gqa_decode_llama8b_paged", "latent_decode_4k_sq1", "latent_decode_4k_sq2", "latent_expanded_4k_sq2",
+          "gta_prefill_4k"]
 
 
 def oracle_sample(wl, target_s: float):

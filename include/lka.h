@@ -64,7 +64,8 @@ typedef enum {
     LKA_ERR_WORKSPACE = 3,    /* ws is NULL or ws_bytes is below the *_workspace_size value */
     LKA_ERR_CUDA = 4,         /* a CUDA call or kernel launch failed */
     LKA_ERR_TIMEOUT = 5,      /* device status: a bounded in-kernel wait ran out (the kernel exited early) */
-    LKA_ERR_BAD_LENGTH = 6    /* device status: a cache_lens entry was outside its range and was clamped */
+    LKA_ERR_BAD_LENGTH = 6,   /* device status: a cache_lens entry was outside its range and was clamped */
+    LKA_ERR_BAD_PAGE = 7      /* device status: a block-table entry a call needed was outside the page pool */
 } lka_status_t;
 
 typedef enum { LKA_BF16 = 0, LKA_FP32 = 1 } lka_dtype_t;
@@ -84,6 +85,26 @@ LKA_API size_t gqa_attn_workspace_size(int B, int h_q, int h_kv, int s_q, int d_
 LKA_API lka_status_t gqa_attn(const void *q, const void *k, const void *v, const int32_t *cache_lens, void *out,
                       float *lse, int B, int h_q, int h_kv, int s_q, int d_h, int Lmax, int causal, float scale,
                       lka_dtype_t dtype, void *ws, size_t ws_bytes, void *stream);
+
+/* (a') GQA attention over a paged KV cache  [GQA "GQA compared with related
+ *  techniques": PagedAttention allocates the cache in fixed-size blocks;
+ *  GQLA sec. 2: paged KV caches are complementary system techniques].
+ *  Same computation, arguments and dtypes as gqa_attn, with the cache held
+ *  in a pool of fixed-size pages instead of one [Lmax] slab per sequence:
+ *   k_pages, v_pages [num_pages, h_kv, page_size, d_h]   (device)
+ *   block_table      [B, max_pages] int32 (device): token t of sequence b
+ *                    is row t % page_size of page block_table[b][t / page_size]
+ *  page_size is a power of two >= 8; the logical capacity of a sequence is
+ *  max_pages * page_size (cache_lens entries above it are clamped, raising
+ *  LKA_ERR_BAD_LENGTH).  Table entries of pages a sequence does not use may
+ *  hold anything; an entry the call needs that is outside [0, num_pages) is
+ *  replaced by page 0 and LKA_ERR_BAD_PAGE is raised in the workspace status.
+ *  The workspace is sized by gqa_attn_paged_workspace_size. */
+LKA_API size_t gqa_attn_paged_workspace_size(int B, int h_q, int h_kv, int s_q, int d_h, int page_size, int max_pages);
+LKA_API lka_status_t gqa_attn_paged(const void *q, const void *k_pages, const void *v_pages,
+                            const int32_t *block_table, const int32_t *cache_lens, void *out, float *lse, int B,
+                            int h_q, int h_kv, int s_q, int d_h, int page_size, int max_pages, int num_pages,
+                            int causal, float scale, lka_dtype_t dtype, void *ws, size_t ws_bytes, void *stream);
 
 /* gqa_attn for callers that cannot allocate device memory.  No counterpart in
  * the papers: it exists for callers that are handed only their input and
@@ -171,7 +192,7 @@ LKA_API lka_status_t latent_expand_cache(const void *latent, const void *w_uk, c
 /* Helpers                                                                  */
 /* ------------------------------------------------------------------------ */
 /* Synchronises `stream`, then returns the sticky status word of workspace ws:
- * LKA_OK, LKA_ERR_TIMEOUT (takes precedence) or LKA_ERR_BAD_LENGTH. */
+ * LKA_OK, LKA_ERR_TIMEOUT (takes precedence), LKA_ERR_BAD_LENGTH or LKA_ERR_BAD_PAGE. */
 LKA_API lka_status_t lka_device_status(const void *ws, void *stream);
 /* Enqueues a reset of the workspace status word to LKA_OK on `stream`. */
 LKA_API lka_status_t lka_clear_status(void *ws, void *stream);

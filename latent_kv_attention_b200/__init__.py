@@ -10,6 +10,7 @@ raised.
 
 Entry points (same names as the C ABI):
   gqa_attn                 GQA decode / prefill          ("Grouped Query Attention (GQA)" glossary page)
+  gqa_attn_paged           the same over a paged KV cache (glossary page: PagedAttention comparison)
   latent_absorbed_attn     GQLA MQA-absorbed latent path (GQLA paper, sec. 3.1, Figure 2(b))
   latent_expand_gqa_attn   GQLA per-group GQA path       (GQLA paper, sec. 3.1, Figure 2(a))
   gta_shared_score_attn    GTA shared score per group    (GTA article, grouped shared attention matrix)
@@ -31,7 +32,7 @@ LIB_PATH = os.path.join(_HERE, "liblka.so")
 
 LKA_OK = 0
 STATUS_NAMES = {0: "LKA_OK", 1: "LKA_ERR_INVALID_ARG", 2: "LKA_ERR_UNSUPPORTED", 3: "LKA_ERR_WORKSPACE",
-                4: "LKA_ERR_CUDA", 5: "LKA_ERR_TIMEOUT", 6: "LKA_ERR_BAD_LENGTH"}
+                4: "LKA_ERR_CUDA", 5: "LKA_ERR_TIMEOUT", 6: "LKA_ERR_BAD_LENGTH", 7: "LKA_ERR_BAD_PAGE"}
 _DT = {torch.bfloat16: 0, torch.float32: 1}
 
 # Every symbol include/lka.h declares, with its ctypes signature (restype, argtypes).
@@ -41,6 +42,8 @@ SIGNATURES = {
     "gqa_attn_workspace_size": (_Z, [_I] * 6),
     "gqa_attn": (_I, [_P] * 6 + [_I] * 7 + [_F, _I, _P, _Z, _P]),
     "gqa_attn_noalloc": (_I, [_P] * 6 + [_I] * 7 + [_F, _I, _P]),
+    "gqa_attn_paged_workspace_size": (_Z, [_I] * 7),
+    "gqa_attn_paged": (_I, [_P] * 7 + [_I] * 9 + [_F, _I, _P, _Z, _P]),
     "latent_absorbed_attn_workspace_size": (_Z, [_I] * 8),
     "latent_absorbed_attn": (_I, [_P] * 8 + [_I] * 9 + [_F, _I, _P, _Z, _P]),
     "latent_expand_gqa_attn_workspace_size": (_Z, [_I] * 7),
@@ -166,6 +169,37 @@ def gqa_attn(q, k, v, cache_lens, causal: bool = True, scale: float | None = Non
     rc = lib.gqa_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(cache_lens), _ptr(out), _ptr(lse), B, h_q, h_kv, s_q, d, Lmax,
                       int(bool(causal)), scale, _dtype_code(q), _ptr(ws), ws.numel(), _stream_ptr())
     _check("gqa_attn", rc)
+    return (out, lse) if return_lse else out
+
+
+def gqa_attn_paged(q, k_pages, v_pages, block_table, cache_lens, causal: bool = True, scale: float | None = None,
+                   out=None, return_lse: bool = False):
+    """GQA attention over a paged KV cache. q [B,h_q,s_q,d]; k_pages/v_pages [num_pages,h_kv,page_size,d];
+    block_table int32 [B,max_pages] (token t of sequence b: row t % page_size of page block_table[b, t // page_size]);
+    cache_lens int32 [B]. Returns out [B,h_q,s_q,d] (and lse [B,h_q,s_q] fp32 if return_lse)."""
+    for n, t in (("q", q), ("k_pages", k_pages), ("v_pages", v_pages)):
+        _device_tensor(t, n, q.dtype)
+    _require(q.dim() == 4 and k_pages.dim() == 4 and v_pages.shape == k_pages.shape,
+             "q [B,h_q,s_q,d], k_pages/v_pages [num_pages,h_kv,page_size,d]")
+    B, h_q, s_q, d = q.shape
+    num_pages, h_kv, page_size, dk = k_pages.shape
+    _require(dk == d, "q and the pages disagree on d")
+    _device_tensor(block_table, "block_table", torch.int32)
+    _require(block_table.dim() == 2 and block_table.shape[0] == B and block_table.device == q.device,
+             "block_table must be int32 [B, max_pages] on q's device")
+    max_pages = block_table.shape[1]
+    _lens_tensor(cache_lens, B, q.device)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    out = torch.empty_like(q) if out is None else out
+    _device_tensor(out, "out", q.dtype)
+    lse = torch.empty((B, h_q, s_q), dtype=torch.float32, device=q.device) if return_lse else None
+    lib = library()
+    nbytes = lib.gqa_attn_paged_workspace_size(B, h_q, h_kv, s_q, d, page_size, max_pages)
+    ws = workspaces.get(nbytes, q.device)
+    rc = lib.gqa_attn_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(cache_lens), _ptr(out),
+                            _ptr(lse), B, h_q, h_kv, s_q, d, page_size, max_pages, num_pages, int(bool(causal)), scale,
+                            _dtype_code(q), _ptr(ws), ws.numel(), _stream_ptr())
+    _check("gqa_attn_paged", rc)
     return (out, lse) if return_lse else out
 
 

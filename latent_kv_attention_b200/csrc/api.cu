@@ -62,12 +62,13 @@ static int pick_rb(int rows, int d, int dtype_bytes) {
     return rb;
 }
 
-static lka_status_t gqa_plan(int B, int h_q, int h_kv, int s_q, int d_h, int Lmax, int dtype_bytes, GqaPlan* pl) {
+static lka_status_t gqa_plan(int B, int h_q, int h_kv, int s_q, int d_h, int Lmax, int dtype_bytes, GqaPlan* pl,
+                             bool paged = false) {
     if (B < 0 || h_q < 1 || h_kv < 1 || s_q < 1 || Lmax < 1 || d_h < 1) return LKA_ERR_INVALID_ARG;
     if (h_q % h_kv) return LKA_ERR_INVALID_ARG;
     const bool d_ok = dtype_bytes == 2 ? (d_h == 64 || d_h == 128 || d_h == 256) : (d_h == 64 || d_h == 128);
     if (!d_ok) return LKA_ERR_UNSUPPORTED;
-    if ((long long)B * h_kv * Lmax >= (1ll << 31)) return LKA_ERR_UNSUPPORTED;
+    if (!paged && (long long)B * h_kv * Lmax >= (1ll << 31)) return LKA_ERR_UNSUPPORTED;
     const int R = (h_q / h_kv) * s_q;
     pl->rb = pick_rb(R, d_h, dtype_bytes);
     pl->n_rb = cdiv(R, pl->rb);
@@ -101,6 +102,20 @@ static lka_status_t gqa_plan(int B, int h_q, int h_kv, int s_q, int d_h, int Lma
 
 static lka_status_t launch_status(cudaError_t e) { return e == cudaSuccess ? LKA_OK : LKA_ERR_CUDA; }
 
+// Workspace bytes of a GQA call; the size does not depend on the dtype beyond the supported head dims: plan
+// with bf16, then fp32, and take the larger.
+static size_t gqa_ws_size(int B, int h_q, int h_kv, int s_q, int d_h, int Lmax, bool paged) {
+    GqaPlan pl;
+    if (gqa_plan(B, h_q, h_kv, s_q, d_h, Lmax, 2, &pl, paged) == LKA_OK) {
+        GqaPlan pf;
+        if (gqa_plan(B, h_q, h_kv, s_q, d_h, Lmax, 4, &pf, paged) == LKA_OK && pf.ws_bytes > pl.ws_bytes)
+            return pf.ws_bytes;
+        return pl.ws_bytes;
+    }
+    if (gqa_plan(B, h_q, h_kv, s_q, d_h, Lmax, 4, &pl, paged) == LKA_OK) return pl.ws_bytes;
+    return 0;
+}
+
 }  // namespace lka
 
 using namespace lka;
@@ -116,6 +131,7 @@ const char* lka_status_string(lka_status_t s) {
         case LKA_ERR_CUDA: return "LKA_ERR_CUDA";
         case LKA_ERR_TIMEOUT: return "LKA_ERR_TIMEOUT";
         case LKA_ERR_BAD_LENGTH: return "LKA_ERR_BAD_LENGTH";
+        case LKA_ERR_BAD_PAGE: return "LKA_ERR_BAD_PAGE";
     }
     return "LKA_ERR_UNKNOWN";
 }
@@ -157,6 +173,7 @@ lka_status_t lka_device_status(const void* ws, void* stream) {
     if (cudaMemcpy(&st, ws, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess) return LKA_ERR_CUDA;
     if (st & kDevTimeout) return LKA_ERR_TIMEOUT;
     if (st & kDevBadLength) return LKA_ERR_BAD_LENGTH;
+    if (st & kDevBadPage) return LKA_ERR_BAD_PAGE;
     return LKA_OK;
 }
 
@@ -166,24 +183,25 @@ lka_status_t lka_clear_status(void* ws, void* stream) {
 }
 
 size_t gqa_attn_workspace_size(int B, int h_q, int h_kv, int s_q, int d_h, int Lmax) {
-    GqaPlan pl;
-    // the size does not depend on the dtype beyond the supported head dims: plan with bf16, then fp32
-    if (gqa_plan(B, h_q, h_kv, s_q, d_h, Lmax, 2, &pl) == LKA_OK) {
-        GqaPlan pf;
-        if (gqa_plan(B, h_q, h_kv, s_q, d_h, Lmax, 4, &pf) == LKA_OK && pf.ws_bytes > pl.ws_bytes) return pf.ws_bytes;
-        return pl.ws_bytes;
-    }
-    if (gqa_plan(B, h_q, h_kv, s_q, d_h, Lmax, 4, &pl) == LKA_OK) return pl.ws_bytes;
-    return 0;
+    return gqa_ws_size(B, h_q, h_kv, s_q, d_h, Lmax, false);
 }
 
-lka_status_t gqa_attn(const void* q, const void* k, const void* v, const int32_t* cache_lens, void* out, float* lse,
-                      int B, int h_q, int h_kv, int s_q, int d_h, int Lmax, int causal, float scale,
-                      lka_dtype_t dtype, void* ws, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace lka {
+struct PagedDesc {
+    const int32_t* block_table;
+    int page_size, max_pages, num_pages;
+};
+
+// Shared by gqa_attn (pg == nullptr: contiguous cache [B, h_kv, Lmax, d]) and gqa_attn_paged.
+static lka_status_t gqa_run(const void* q, const void* k, const void* v, const int32_t* cache_lens, void* out,
+                            float* lse, int B, int h_q, int h_kv, int s_q, int d_h, int Lmax, int causal, float scale,
+                            lka_dtype_t dtype, void* ws, size_t ws_bytes, void* stream, const PagedDesc* pg) {
     if (dtype != LKA_BF16 && dtype != LKA_FP32) return LKA_ERR_UNSUPPORTED;
     const int eb = dtype == LKA_BF16 ? 2 : 4;
     GqaPlan pl;
-    lka_status_t s = gqa_plan(B, h_q, h_kv, s_q, d_h, Lmax, eb, &pl);
+    lka_status_t s = gqa_plan(B, h_q, h_kv, s_q, d_h, Lmax, eb, &pl, pg != nullptr);
     if (s != LKA_OK) return s;
     if (B == 0) return LKA_OK;
     if (!q || !k || !v || !cache_lens || !out) return LKA_ERR_INVALID_ARG;
@@ -194,10 +212,15 @@ lka_status_t gqa_attn(const void* q, const void* k, const void* v, const int32_t
     if (!aligned16(ws)) return LKA_ERR_INVALID_ARG;
 
     const CUtensorMapDataType tdt = eb == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-    const uint64_t rows = (uint64_t)B * h_kv * Lmax;
+    uint64_t rows = (uint64_t)B * h_kv * Lmax;
+    uint32_t box_rows = (uint32_t)pl.tile;
+    if (pg) {
+        rows = (uint64_t)pg->num_pages * h_kv * pg->page_size;
+        box_rows = (uint32_t)(pg->page_size < pl.tile ? pg->page_size : pl.tile);
+    }
     CUtensorMap tk, tv;
-    if (!make_tmap_2d(&tk, tdt, k, d_h, rows, (uint64_t)d_h * eb, 128 / eb, pl.tile) ||
-        !make_tmap_2d(&tv, tdt, v, d_h, rows, (uint64_t)d_h * eb, 128 / eb, pl.tile))
+    if (!make_tmap_2d(&tk, tdt, k, d_h, rows, (uint64_t)d_h * eb, 128 / eb, box_rows) ||
+        !make_tmap_2d(&tv, tdt, v, d_h, rows, (uint64_t)d_h * eb, 128 / eb, box_rows))
         return LKA_ERR_CUDA;
 
     GqaParams p;
@@ -220,7 +243,50 @@ lka_status_t gqa_attn(const void* q, const void* k, const void* v, const int32_t
     p.nsplit_max = pl.nsplit;
     p.n_rb = pl.n_rb;
     p.ratio = h_q / h_kv;
+    p.block_table = pg ? pg->block_table : nullptr;
+    p.page_size = pg ? pg->page_size : 0;
+    p.max_pages = pg ? pg->max_pages : 0;
+    p.num_pages = pg ? pg->num_pages : 0;
+    p.box_rows = (int)box_rows;
     return launch_status(gqa_decode_launch(tk, tv, p, eb, d_h, pl.rb, pl.nsplit, (cudaStream_t)stream));
+}
+
+// Paged-cache arguments: page_size a power of two >= 8, a table of max_pages entries per sequence, a pool
+// of num_pages pages that TMA coordinates can address.
+static lka_status_t paged_args_ok(int h_kv, int page_size, int max_pages, int num_pages) {
+    if (page_size < 8 || (page_size & (page_size - 1)) || max_pages < 1 || num_pages < 1 || h_kv < 1)
+        return LKA_ERR_INVALID_ARG;
+    if ((long long)max_pages * page_size >= (1ll << 31) ||
+        (long long)num_pages * h_kv * page_size >= (1ll << 31))
+        return LKA_ERR_UNSUPPORTED;
+    return LKA_OK;
+}
+}  // namespace lka
+
+extern "C" {
+
+lka_status_t gqa_attn(const void* q, const void* k, const void* v, const int32_t* cache_lens, void* out, float* lse,
+                      int B, int h_q, int h_kv, int s_q, int d_h, int Lmax, int causal, float scale,
+                      lka_dtype_t dtype, void* ws, size_t ws_bytes, void* stream) {
+    return gqa_run(q, k, v, cache_lens, out, lse, B, h_q, h_kv, s_q, d_h, Lmax, causal, scale, dtype, ws, ws_bytes,
+                   stream, nullptr);
+}
+
+size_t gqa_attn_paged_workspace_size(int B, int h_q, int h_kv, int s_q, int d_h, int page_size, int max_pages) {
+    if (paged_args_ok(h_kv, page_size, max_pages, 1) != LKA_OK) return 0;
+    return gqa_ws_size(B, h_q, h_kv, s_q, d_h, page_size * max_pages, true);
+}
+
+lka_status_t gqa_attn_paged(const void* q, const void* k_pages, const void* v_pages, const int32_t* block_table,
+                            const int32_t* cache_lens, void* out, float* lse, int B, int h_q, int h_kv, int s_q,
+                            int d_h, int page_size, int max_pages, int num_pages, int causal, float scale,
+                            lka_dtype_t dtype, void* ws, size_t ws_bytes, void* stream) {
+    lka_status_t s = paged_args_ok(h_kv, page_size, max_pages, num_pages);
+    if (s != LKA_OK) return s;
+    if (B > 0 && (!block_table || (reinterpret_cast<uintptr_t>(block_table) & 3u))) return LKA_ERR_INVALID_ARG;
+    const PagedDesc pg{block_table, page_size, max_pages, num_pages};
+    return gqa_run(q, k_pages, v_pages, cache_lens, out, lse, B, h_q, h_kv, s_q, d_h, page_size * max_pages, causal,
+                   scale, dtype, ws, ws_bytes, stream, &pg);
 }
 
 }  // extern "C"

@@ -151,6 +151,24 @@ __device__ __forceinline__ void lane_chunk(int li, int c, int& seg, int& chunk) 
     }
 }
 
+// Row of token `tok` of sequence b, KV head kvh, in the paged cache [num_pages][h_kv][page_size][D]
+// ("Grouped Query Attention (GQA)" glossary page, comparison with related techniques: PagedAttention
+// allocates the cache in fixed-size blocks): page block_table[b][tok / page_size], offset tok % page_size.
+// Table entries outside [0, num_pages) are replaced by page 0; for a token the attention needs (`live`)
+// that raises kDevBadPage.  Tokens past the table's capacity (the tail of a last tile) read page 0.
+__device__ __forceinline__ int paged_row(const GqaParams& p, int b, int kvh, int tok, bool live) {
+    int page = 0;
+    const int j = tok / p.page_size;
+    if (j < p.max_pages) {
+        page = p.block_table[(size_t)b * p.max_pages + j];
+        if (page < 0 || page >= p.num_pages) {
+            if (live) atomicOr(p.status, kDevBadPage);
+            page = 0;
+        }
+    }
+    return (page * p.h_kv + kvh) * p.page_size + tok % p.page_size;
+}
+
 template <typename T, int D, int RB>
 __global__ void __launch_bounds__(160, GqaCfg<T, D, RB>::MINB)
     gqa_decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -220,11 +238,25 @@ __global__ void __launch_bounds__(160, GqaCfg<T, D, RB>::MINB)
                 mbar_arrive_expect_tx(full, C::STAGE_BYTES);
                 const uint32_t kdst = smem_u32(stages + s * C::STAGE_BYTES);
                 const uint32_t vdst = kdst + C::MAT_BYTES;
-                const int y = ybase + kbeg + it * C::T_TILE;
+                const int tok0 = kbeg + it * C::T_TILE;
+                if (!p.block_table) {
+                    const int y = ybase + tok0;
 #pragma unroll
-                for (int sg = 0; sg < C::NSEG; ++sg) {
-                    tma_load_2d(kdst + sg * C::T_TILE * 128, &tmK, sg * C::SEG_ELEMS, y, full);
-                    tma_load_2d(vdst + sg * C::T_TILE * 128, &tmV, sg * C::SEG_ELEMS, y, full);
+                    for (int sg = 0; sg < C::NSEG; ++sg) {
+                        tma_load_2d(kdst + sg * C::T_TILE * 128, &tmK, sg * C::SEG_ELEMS, y, full);
+                        tma_load_2d(vdst + sg * C::T_TILE * 128, &tmV, sg * C::SEG_ELEMS, y, full);
+                    }
+                } else {
+                    // paged cache: the tile is box_rows-row pieces, each inside one page of the block table
+                    for (int r0 = 0; r0 < C::T_TILE; r0 += p.box_rows) {
+                        const int tok = tok0 + r0;
+                        const int y = paged_row(p, b, kvh, tok, tok < L);
+#pragma unroll
+                        for (int sg = 0; sg < C::NSEG; ++sg) {
+                            tma_load_2d(kdst + sg * C::T_TILE * 128 + r0 * 128, &tmK, sg * C::SEG_ELEMS, y, full);
+                            tma_load_2d(vdst + sg * C::T_TILE * 128 + r0 * 128, &tmV, sg * C::SEG_ELEMS, y, full);
+                        }
+                    }
                 }
                 ++issued;
             }

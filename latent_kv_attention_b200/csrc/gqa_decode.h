@@ -20,6 +20,10 @@ struct GqaParams {
     int nsplit_max;         // ceil(Lmax / split_tokens)
     int n_rb;               // row blocks per KV head
     int ratio;              // h_q / h_kv
+    // paged cache (block_table == nullptr: contiguous [B, h_kv, Lmax, D])
+    const int32_t* block_table;  // device [B][max_pages] page indices, or nullptr
+    int page_size, max_pages, num_pages;
+    int box_rows;           // rows per TMA box: min(page_size, tile)
 };
 
 // Merge of split partials for rows [B*h_q*s_q] of D values (rows needing one split are skipped).

@@ -124,6 +124,38 @@ def gqa(q, k, v, cache_lens, causal: bool, scale: float, rows_b=None, n_threads:
     return out, lse
 
 
+def paged_to_contiguous(pages, block_table, Lmax: int):
+    """The cache a block table describes, as one slab per sequence: cache[b, h, t] = pages[block_table[b,
+    t // page_size], h, t % page_size] for t < Lmax ("Grouped Query Attention (GQA)" glossary page, comparison
+    with related techniques: PagedAttention keeps the cache in fixed-size blocks).  pages [num_pages, h_kv,
+    page_size, d]; entries of the table past a sequence's pages may hold anything: rows they address are filled
+    with NaN, which the attention definition never reads for t >= cache_lens[b]."""
+    pages = _f64(pages)
+    bt = _i32(block_table)
+    num_pages, h_kv, ps, d = pages.shape
+    B = bt.shape[0]
+    out = np.full((B, h_kv, Lmax, d), np.nan)
+    for b in range(B):
+        for t0 in range(0, Lmax, ps):
+            j = t0 // ps
+            if j >= bt.shape[1] or not (0 <= bt[b, j] < num_pages):
+                continue
+            n = min(ps, Lmax - t0)
+            out[b, :, t0:t0 + n, :] = pages[bt[b, j], :, :n, :]
+    return out
+
+
+def gqa_paged(q, k_pages, v_pages, block_table, cache_lens, causal: bool, scale: float, rows_b=None,
+              n_threads: int = 0):
+    """GQA attention over a paged cache: the contiguous cache the block table describes, then gqa()."""
+    bt = _i32(block_table)
+    ps = int(np.asarray(k_pages.shape)[2])
+    Lmax = bt.shape[1] * ps
+    k = paged_to_contiguous(k_pages, bt, Lmax)
+    v = paged_to_contiguous(v_pages, bt, Lmax)
+    return gqa(q, k, v, cache_lens, causal, scale, rows_b=rows_b, n_threads=n_threads)
+
+
 def gqa_probs(q, k, cache_lens, causal: bool, scale: float, b: int, i: int, t: int, h_kv: int):
     """Softmax probabilities of one query row of the GQA definition (visible keys only)."""
     q, k, lens = _f64(q), _f64(k), _i32(cache_lens)

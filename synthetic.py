@@ -80,6 +80,44 @@ def gqa_inputs(seed, B, h_q, h_kv, d, s_q, L_lo, L_hi, Lmax=None, dtype=torch.bf
     return dict(q=q, k=k, v=v, cache_lens=lens, scale=1.0 / math.sqrt(d))
 
 
+def to_pages(caches, lens, page_size, gen, spare_pages=0):
+    """Scatters contiguous caches [B, h_kv, Lmax, d] (e.g. K and V) into shuffled page pools [num_pages, h_kv,
+    page_size, d] sharing one block table [B, Lmax / page_size] (int32): the pages a sequence uses
+    (ceil(len / page_size)) go to slots of a random permutation of the pool; its unused table entries are -1 and
+    unused pool slots hold random values.  Layout only: no attention arithmetic."""
+    B, h_kv, Lmax, d = caches[0].shape
+    assert Lmax % page_size == 0
+    max_pages = Lmax // page_size
+    num_pages = B * max_pages + spare_pages
+    dev = caches[0].device
+    perm = torch.randperm(num_pages, generator=gen, device=dev).tolist()
+    pools = [torch.randn((num_pages, h_kv, page_size, d), generator=gen, device=dev, dtype=torch.float32).to(c.dtype)
+             for c in caches]
+    table = torch.full((B, max_pages), -1, dtype=torch.int32)
+    lens_l = lens.tolist()
+    for b in range(B):
+        used = -(-int(lens_l[b]) // page_size)
+        for j in range(used):
+            slot = perm[b * max_pages + j]
+            table[b, j] = slot
+            for pool, c in zip(pools, caches):
+                pool[slot] = c[b, :, j * page_size:(j + 1) * page_size, :]
+    return pools, table.to(dev)
+
+
+def gqa_paged_inputs(seed, B, h_q, h_kv, d, s_q, L_lo, L_hi, page_size, Lmax=None, dtype=torch.bfloat16,
+                     device="cpu", spare_pages=3):
+    """GQA inputs (as gqa_inputs) with the K/V cache moved into shuffled page pools and a block table; the
+    capacity Lmax (default L_hi) is rounded up to whole pages."""
+    Lmax = L_hi if Lmax is None else Lmax
+    Lmax = -(-Lmax // page_size) * page_size
+    inp = gqa_inputs(seed, B, h_q, h_kv, d, s_q, L_lo, L_hi, Lmax=Lmax, dtype=dtype, device=device)
+    g = _gen(seed + 7919, device)
+    (k_pages, v_pages), table = to_pages([inp["k"], inp["v"]], inp["cache_lens"], page_size, g, spare_pages)
+    inp.update(k_pages=k_pages, v_pages=v_pages, block_table=table, page_size=page_size)
+    return inp
+
+
 def latent_inputs(seed, B, h_q, g_groups, d_h, r_kv, d_r, s_q, L_lo, L_hi, Lmax=None, dtype=torch.bfloat16,
                   device="cpu"):
     """GQLA latent decode inputs: c^KV, k^R, q^C, q^R ~ N(0,1); W^UK, W^UV ~ N(0, 1/r_kv)."""
@@ -128,6 +166,9 @@ WORKLOADS = {
     # the same layer with a quarter of the batch: the small case for full ncu captures (K/V still > L2)
     "gqa_decode_llama8b_b16": dict(kind="gqa", seed=2, B=16, h_q=32, h_kv=8, d=128, s_q=1, L_lo=1024, L_hi=8192,
                                    causal=True),
+    # the same layer over a paged cache: 64-token pages in a shuffled pool, addressed through a block table
+    "gqa_decode_llama8b_paged": dict(kind="gqa_paged", seed=2, B=64, h_q=32, h_kv=8, d=128, s_q=1, L_lo=1024,
+                                     L_hi=8192, causal=True, page_size=64),
     "gta_prefill_4k": dict(kind="gta", seed=3, B=8, G=3, H=12, d_qk=64, d_v=64, s_q=4096, L_lo=4096,
                            L_hi=4096, causal=True),
     "latent_decode_4k_sq1": dict(kind="latent", seed=4, B=64, h_q=128, g=8, d_h=128, r_kv=512, d_r=64, s_q=1,
@@ -162,6 +203,9 @@ def make(w: dict, device="cpu", dtype=torch.bfloat16) -> dict:
     if w["kind"] == "gqa":
         return gqa_inputs(w["seed"], w["B"], w["h_q"], w["h_kv"], w["d"], w["s_q"], w["L_lo"], w["L_hi"],
                           dtype=dtype, device=device)
+    if w["kind"] == "gqa_paged":
+        return gqa_paged_inputs(w["seed"], w["B"], w["h_q"], w["h_kv"], w["d"], w["s_q"], w["L_lo"], w["L_hi"],
+                                w["page_size"], dtype=dtype, device=device)
     if w["kind"] == "latent":
         return latent_inputs(w["seed"], w["B"], w["h_q"], w["g"], w["d_h"], w["r_kv"], w["d_r"], w["s_q"],
                              w["L_lo"], w["L_hi"], dtype=dtype, device=device)

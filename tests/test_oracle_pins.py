@@ -321,3 +321,40 @@ def test_gta_single_head_groups_is_mha():
     out, _ = oracle.gta(gt["q_g"], gt["k_g"], gt["v"], gt["cache_lens"], True, 0.6)
     ref, _ = oracle.gqa(gt["q_g"], gt["k_g"], gt["v"], gt["cache_lens"], True, 0.6)
     assert np.abs(out - ref).max() == 0.0
+
+
+# ------------------------------------------------------------------ paged KV cache (gather) -----------------
+def test_paged_oracle_identity_layout_equals_contiguous():
+    """Pages cut from the contiguous cache in order (block_table[b, j] = b * max_pages + j): the paged
+    definition is the contiguous one ("Grouped Query Attention (GQA)" glossary page, PagedAttention keeps the
+    cache in fixed-size blocks)."""
+    inp = synthetic.gqa_inputs(61, 3, 8, 2, 32, 2, 2, 48, Lmax=48, dtype=torch.float32)
+    ps = 16
+    B, h_kv, Lmax, d = inp["k"].shape
+    mp = Lmax // ps
+    pages = lambda c: c.reshape(B, h_kv, mp, ps, d).permute(0, 2, 1, 3, 4).reshape(B * mp, h_kv, ps, d)  # noqa: E731
+    table = torch.arange(B * mp, dtype=torch.int32).reshape(B, mp)
+    ref, ref_lse = oracle.gqa(inp["q"], inp["k"], inp["v"], inp["cache_lens"], True, 0.2)
+    out, lse = oracle.gqa_paged(inp["q"], pages(inp["k"]), pages(inp["v"]), table, inp["cache_lens"], True, 0.2)
+    assert np.array_equal(out, ref) and np.array_equal(lse, ref_lse)
+
+
+def test_paged_oracle_shuffled_pool_and_shared_prefix():
+    # a shuffled pool with unused entries -1 gives the contiguous result
+    inp = synthetic.gqa_paged_inputs(62, 4, 8, 4, 32, 1, 1, 60, 8, Lmax=64, dtype=torch.float32)
+    ref, _ = oracle.gqa(inp["q"], inp["k"], inp["v"], inp["cache_lens"], False, 0.3)
+    out, _ = oracle.gqa_paged(inp["q"], inp["k_pages"], inp["v_pages"], inp["block_table"], inp["cache_lens"],
+                              False, 0.3)
+    assert np.allclose(out, ref, atol=0, rtol=0)
+    # two sequences sharing their first page (a common prompt prefix): equal to duplicating that page
+    g = torch.Generator().manual_seed(63)
+    pool_k = torch.randn(5, 2, 8, 16, generator=g)
+    pool_v = torch.randn(5, 2, 8, 16, generator=g)
+    table = torch.tensor([[3, 1], [3, 4]], dtype=torch.int32)
+    lens = torch.tensor([13, 16], dtype=torch.int32)
+    q = torch.randn(2, 4, 1, 16, generator=g)
+    k = torch.stack([torch.cat([pool_k[3], pool_k[1]], 1), torch.cat([pool_k[3], pool_k[4]], 1)])
+    v = torch.stack([torch.cat([pool_v[3], pool_v[1]], 1), torch.cat([pool_v[3], pool_v[4]], 1)])
+    ref, _ = oracle.gqa(q, k, v, lens, True, 0.25)
+    out, _ = oracle.gqa_paged(q, pool_k, pool_v, table, lens, True, 0.25)
+    assert np.array_equal(out, ref)
