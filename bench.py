@@ -14,8 +14,9 @@ flushed between timed steps anyway.
 Unless --no-extras is given, the line also carries `other_paths`: the same
 measurement (step time, GB/s, TFLOP/s, tokens/s, roofline of the main kernel,
 end-to-end time) for the GQA layer over a paged cache (64-token pages), the
-GQLA latent decode layer on the MQA-absorbed path (s_q = 1 and 2), on the
-per-group GQA path (s_q = 2), and for the GTA causal prefill.
+GQLA latent decode layer on the MQA-absorbed path (s_q = 1 and 2; s_q = 1 also
+over a paged latent cache), on the per-group GQA path (s_q = 2), and for the
+GTA causal prefill.
 
 Prints ONE JSON line (rank 0).  `value` is the algorithmic HBM traffic of the
 step (every cache byte once, q read once, out written once) divided by the
@@ -321,6 +322,27 @@ class LatentAbsorbed(Workload):
         return fn, nbytes, oracle.threads_used(0, n * w["h_q"]), f"first {n} of {w['B']} sequences"
 
 
+class LatentAbsorbedPaged(LatentAbsorbed):
+    """latent_absorbed_attn_paged over the s_q = 1 batch with the latent cache in 64-token pages of a shuffled pool."""
+
+    def setup_device(self):
+        super().setup_device()
+        self.inp.pop("latent", None)  # the contiguous copy is not used by the paged step
+        torch.cuda.empty_cache()
+
+    def step(self):
+        i = self.inp
+        self.lka.latent_absorbed_attn_paged(i["q_c"], i["q_r"], i["w_uk"], i["w_uv"], i["latent_pages"],
+                                            i["block_table"], i["cache_lens"], causal=self.w["causal"],
+                                            scale=i["scale"], out=self.out)
+
+    def config(self):
+        c = super().config()
+        c["page_size"] = self.w["page_size"]
+        c["cache_layout"] = "paged (shuffled page pool + block table)"
+        return c
+
+
 class LatentExpanded(LatentAbsorbed):
     """latent_expand_gqa_attn over the per-group expanded cache (made once, outside the timed steps)."""
 
@@ -421,6 +443,7 @@ WORKLOAD_CLASSES = {
     "gqa_decode_llama8b_paged": GqaDecodePaged,
     "latent_decode_4k_sq1": LatentAbsorbed,
     "latent_decode_4k_sq2": LatentAbsorbed,
+    "latent_decode_4k_sq1_paged": LatentAbsorbedPaged,
     "latent_expanded_4k_sq1": LatentExpanded,
     "latent_expanded_4k_sq2": LatentExpanded,
     "gta_prefill_4k": GtaPrefill,
@@ -429,8 +452,8 @@ WORKLOAD_CLASSES = {
     "latent_expanded_4k_sq2_b16": LatentExpanded,
     "gta_prefill_4k_b2": GtaPrefill,
 }
-EXTRAS = ["gqa_decode_llama8b_paged", "latent_decode_4k_sq1", "latent_decode_4k_sq2", "latent_expanded_4k_sq2",
-          "gta_prefill_4k"]
+EXTRAS = ["gqa_decode_llama8b_paged", "latent_decode_4k_sq1", "latent_decode_4k_sq1_paged", "latent_decode_4k_sq2",
+          "latent_expanded_4k_sq2", "gta_prefill_4k"]
 
 
 def oracle_sample(wl, target_s: float):

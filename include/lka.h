@@ -147,6 +147,23 @@ LKA_API lka_status_t latent_absorbed_attn(const void *q_c, const void *q_r, cons
                                   int h_q, int g, int s_q, int d_h, int r_kv, int d_r, int Lmax, int causal,
                                   float scale, lka_dtype_t dtype, void *ws, size_t ws_bytes, void *stream);
 
+/* (b') The same over a paged latent cache  [GQA "GQA compared with related
+ *  techniques" (PagedAttention); GQLA sec. 2 (paged KV caches)].
+ *   latent_pages [num_pages, page_size, r_kv + d_r]  (device)
+ *   block_table  [B, max_pages] int32 (device): token t of sequence b is
+ *                row t % page_size of page block_table[b][t / page_size]
+ *  page_size a power of two >= 8; capacity max_pages * page_size per
+ *  sequence; out-of-pool entries a call needs are replaced by page 0 and
+ *  raise LKA_ERR_BAD_PAGE.  Other arguments and results as in (b). */
+LKA_API size_t latent_absorbed_attn_paged_workspace_size(int B, int h_q, int g, int s_q, int d_h, int r_kv, int d_r,
+                                                         int page_size, int max_pages);
+LKA_API lka_status_t latent_absorbed_attn_paged(const void *q_c, const void *q_r, const void *w_uk,
+                                        const void *w_uv, const void *latent_pages, const int32_t *block_table,
+                                        const int32_t *cache_lens, void *out, float *lse, int B, int h_q, int g,
+                                        int s_q, int d_h, int r_kv, int d_r, int page_size, int max_pages,
+                                        int num_pages, int causal, float scale, lka_dtype_t dtype, void *ws,
+                                        size_t ws_bytes, void *stream);
+
 /* ------------------------------------------------------------------------ */
 /* (c) GQLA GQA path over the per-group expanded cache  [GQLA sec. 1,       */
 /*     sec. 3.1, Figure 2(a)]                                               */

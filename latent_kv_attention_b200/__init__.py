@@ -46,6 +46,8 @@ SIGNATURES = {
     "gqa_attn_paged": (_I, [_P] * 7 + [_I] * 9 + [_F, _I, _P, _Z, _P]),
     "latent_absorbed_attn_workspace_size": (_Z, [_I] * 8),
     "latent_absorbed_attn": (_I, [_P] * 8 + [_I] * 9 + [_F, _I, _P, _Z, _P]),
+    "latent_absorbed_attn_paged_workspace_size": (_Z, [_I] * 9),
+    "latent_absorbed_attn_paged": (_I, [_P] * 9 + [_I] * 11 + [_F, _I, _P, _Z, _P]),
     "latent_expand_gqa_attn_workspace_size": (_Z, [_I] * 7),
     "latent_expand_gqa_attn": (_I, [_P] * 8 + [_I] * 8 + [_F, _I, _P, _Z, _P]),
     "gta_shared_score_attn_workspace_size": (_Z, [_I] * 7),
@@ -226,6 +228,36 @@ def latent_absorbed_attn(q_c, q_r, w_uk, w_uv, latent, cache_lens, causal: bool 
                                   _ptr(out), _ptr(lse), B, h_q, g, s_q, d_h, r_kv, d_r, Lmax, int(bool(causal)),
                                   scale, _dtype_code(q_c), _ptr(ws), ws.numel(), _stream_ptr())
     _check("latent_absorbed_attn", rc)
+    return (out, lse) if return_lse else out
+
+
+def latent_absorbed_attn_paged(q_c, q_r, w_uk, w_uv, latent_pages, block_table, cache_lens, causal: bool = True,
+                               scale: float | None = None, out=None, return_lse: bool = False):
+    """latent_absorbed_attn over a paged latent cache: latent_pages [num_pages, page_size, r_kv + d_r], block_table
+    int32 [B, max_pages] (token t of sequence b: row t % page_size of page block_table[b, t // page_size])."""
+    for n, t in (("q_c", q_c), ("q_r", q_r), ("w_uk", w_uk), ("w_uv", w_uv), ("latent_pages", latent_pages)):
+        _device_tensor(t, n, torch.bfloat16)
+    B, h_q, s_q, d_h = q_c.shape
+    d_r = q_r.shape[-1]
+    g, _, r_kv = w_uk.shape
+    num_pages, page_size, width = latent_pages.shape
+    _require(width == r_kv + d_r, "latent_pages [num_pages, page_size, r_kv + d_r]")
+    _device_tensor(block_table, "block_table", torch.int32)
+    _require(block_table.dim() == 2 and block_table.shape[0] == B, "block_table must be int32 [B, max_pages]")
+    max_pages = block_table.shape[1]
+    _lens_tensor(cache_lens, B, q_c.device)
+    scale = 1.0 / math.sqrt(d_h + d_r) if scale is None else float(scale)
+    out = torch.empty_like(q_c) if out is None else out
+    lse = torch.empty((B, h_q, s_q), dtype=torch.float32, device=q_c.device) if return_lse else None
+    lib = library()
+    nbytes = lib.latent_absorbed_attn_paged_workspace_size(B, h_q, g, s_q, d_h, r_kv, d_r, page_size, max_pages)
+    _require(nbytes > 0, "unsupported latent shape or page layout")
+    ws = workspaces.get(nbytes, q_c.device)
+    rc = lib.latent_absorbed_attn_paged(_ptr(q_c), _ptr(q_r), _ptr(w_uk), _ptr(w_uv), _ptr(latent_pages),
+                                        _ptr(block_table), _ptr(cache_lens), _ptr(out), _ptr(lse), B, h_q, g, s_q, d_h,
+                                        r_kv, d_r, page_size, max_pages, num_pages, int(bool(causal)), scale, 0,
+                                        _ptr(ws), ws.numel(), _stream_ptr())
+    _check("latent_absorbed_attn_paged", rc)
     return (out, lse) if return_lse else out
 
 

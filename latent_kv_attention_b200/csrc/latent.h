@@ -34,6 +34,10 @@ struct LatentParams {
     int B, h_q, g, s_q, Lmax, causal;
     float scale_log2;
     int split_tokens, nsplit;
+    // paged latent cache (block_table == nullptr: contiguous [B, Lmax, r_kv + d_r])
+    const int32_t* block_table;  // device [B][max_pages] page indices, or nullptr
+    int page_size, max_pages, num_pages;
+    int box_rows;                // rows per TMA box: min(page_size, tile)
 };
 
 cudaError_t latent_attn_launch(const CUtensorMap& tm_lat, const LatentParams& p, cudaStream_t st);

@@ -19,14 +19,14 @@ struct LatentPlan {
 };
 
 static lka_status_t latent_plan(int B, int h_q, int g, int s_q, int d_h, int r_kv, int d_r, int Lmax,
-                                LatentPlan* pl) {
+                                LatentPlan* pl, bool paged = false) {
     if (B < 0 || h_q < 1 || g < 1 || s_q < 1 || d_h < 1 || r_kv < 1 || d_r < 0 || Lmax < 1) return LKA_ERR_INVALID_ARG;
     if (h_q % g) return LKA_ERR_INVALID_ARG;
     // the kernels are specialised to the GQLA/MLA shape (h_q, d_h, r_kv, d_h^R) = (128, 128, 512, 64)
     if (h_q != 128 || d_h != 128 || r_kv != 512 || d_r != 64) return LKA_ERR_UNSUPPORTED;
     const int HPG = h_q / g;
     if (HPG < 16 || 128 % (HPG * s_q) != 0) return LKA_ERR_UNSUPPORTED;
-    if ((long long)B * Lmax >= (1ll << 31) || B > 65535) return LKA_ERR_UNSUPPORTED;
+    if ((!paged && (long long)B * Lmax >= (1ll << 31)) || B > 65535) return LKA_ERR_UNSUPPORTED;
     const int NT = latent_tile_tokens();
     int st = split_tokens_knob();
     if (st <= 0) {
@@ -81,13 +81,21 @@ size_t latent_absorbed_attn_workspace_size(int B, int h_q, int g, int s_q, int d
     return latent_plan(B, h_q, g, s_q, d_h, r_kv, d_r, Lmax, &pl) == LKA_OK ? pl.ws_bytes : 0;
 }
 
-lka_status_t latent_absorbed_attn(const void* q_c, const void* q_r, const void* w_uk, const void* w_uv,
-                                  const void* latent, const int32_t* cache_lens, void* out, float* lse, int B, int h_q,
-                                  int g, int s_q, int d_h, int r_kv, int d_r, int Lmax, int causal, float scale,
-                                  lka_dtype_t dtype, void* ws, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace lka {
+struct LatentPages {
+    const int32_t* block_table;
+    int page_size, max_pages, num_pages;
+};
+
+static lka_status_t latent_run(const void* q_c, const void* q_r, const void* w_uk, const void* w_uv,
+                               const void* latent, const int32_t* cache_lens, void* out, float* lse, int B, int h_q,
+                               int g, int s_q, int d_h, int r_kv, int d_r, int Lmax, int causal, float scale,
+                               lka_dtype_t dtype, void* ws, size_t ws_bytes, void* stream, const LatentPages* pg) {
     if (dtype != LKA_BF16) return LKA_ERR_UNSUPPORTED;
     LatentPlan pl;
-    lka_status_t s = latent_plan(B, h_q, g, s_q, d_h, r_kv, d_r, Lmax, &pl);
+    lka_status_t s = latent_plan(B, h_q, g, s_q, d_h, r_kv, d_r, Lmax, &pl, pg != nullptr);
     if (s != LKA_OK) return s;
     if (B == 0) return LKA_OK;
     const void* ptrs[] = {q_c, q_r, w_uk, w_uv, latent, cache_lens, out};
@@ -129,8 +137,9 @@ lka_status_t latent_absorbed_attn(const void* q_c, const void* q_r, const void* 
 
     // 2) attention of all heads over the latent cache (+ merge of key splits)
     CUtensorMap tm_lat;
-    if (!make_tmap_2d(&tm_lat, BF, latent, r_kv + d_r, (uint64_t)B * Lmax, (uint64_t)(r_kv + d_r) * 2, 64,
-                      latent_tile_tokens()))
+    const uint64_t lat_rows = pg ? (uint64_t)pg->num_pages * pg->page_size : (uint64_t)B * Lmax;
+    const int box_rows = pg && pg->page_size < latent_tile_tokens() ? pg->page_size : latent_tile_tokens();
+    if (!make_tmap_2d(&tm_lat, BF, latent, r_kv + d_r, lat_rows, (uint64_t)(r_kv + d_r) * 2, 64, box_rows))
         return LKA_ERR_CUDA;
     LatentParams lp{};
     lp.lens = cache_lens;
@@ -150,6 +159,11 @@ lka_status_t latent_absorbed_attn(const void* q_c, const void* q_r, const void* 
     lp.scale_log2 = scale * 1.4426950408889634f;
     lp.split_tokens = pl.split_tokens;
     lp.nsplit = pl.nsplit;
+    lp.block_table = pg ? pg->block_table : nullptr;
+    lp.page_size = pg ? pg->page_size : 0;
+    lp.max_pages = pg ? pg->max_pages : 0;
+    lp.num_pages = pg ? pg->num_pages : 0;
+    lp.box_rows = box_rows;
     if ((s = st_of(latent_attn_launch(tm_lat, lp, st))) != LKA_OK) return s;
 
     // 3) up-projection out = W^UV_gamma o~
@@ -164,6 +178,43 @@ lka_status_t latent_absorbed_attn(const void* q_c, const void* q_r, const void* 
     gu.K = r_kv;
     gu.N = d_h;
     return st_of(gemm_upproj(tm_ol, tm_wuv, gu, st));
+}
+
+
+}  // namespace lka
+
+extern "C" {
+
+lka_status_t latent_absorbed_attn(const void* q_c, const void* q_r, const void* w_uk, const void* w_uv,
+                                  const void* latent, const int32_t* cache_lens, void* out, float* lse, int B, int h_q,
+                                  int g, int s_q, int d_h, int r_kv, int d_r, int Lmax, int causal, float scale,
+                                  lka_dtype_t dtype, void* ws, size_t ws_bytes, void* stream) {
+    return latent_run(q_c, q_r, w_uk, w_uv, latent, cache_lens, out, lse, B, h_q, g, s_q, d_h, r_kv, d_r, Lmax, causal,
+                      scale, dtype, ws, ws_bytes, stream, nullptr);
+}
+
+size_t latent_absorbed_attn_paged_workspace_size(int B, int h_q, int g, int s_q, int d_h, int r_kv, int d_r,
+                                                 int page_size, int max_pages) {
+    if (page_size < 8 || (page_size & (page_size - 1)) || max_pages < 1 ||
+        (long long)page_size * max_pages >= (1ll << 31))
+        return 0;
+    LatentPlan pl;
+    return latent_plan(B, h_q, g, s_q, d_h, r_kv, d_r, page_size * max_pages, &pl, true) == LKA_OK ? pl.ws_bytes : 0;
+}
+
+lka_status_t latent_absorbed_attn_paged(const void* q_c, const void* q_r, const void* w_uk, const void* w_uv,
+                                        const void* latent_pages, const int32_t* block_table,
+                                        const int32_t* cache_lens, void* out, float* lse, int B, int h_q, int g,
+                                        int s_q, int d_h, int r_kv, int d_r, int page_size, int max_pages,
+                                        int num_pages, int causal, float scale, lka_dtype_t dtype, void* ws,
+                                        size_t ws_bytes, void* stream) {
+    if (page_size < 8 || (page_size & (page_size - 1)) || max_pages < 1 || num_pages < 1) return LKA_ERR_INVALID_ARG;
+    if ((long long)page_size * max_pages >= (1ll << 31) || (long long)num_pages * page_size >= (1ll << 31))
+        return LKA_ERR_UNSUPPORTED;
+    if (B > 0 && (!block_table || (reinterpret_cast<uintptr_t>(block_table) & 3u))) return LKA_ERR_INVALID_ARG;
+    const LatentPages pg{block_table, page_size, max_pages, num_pages};
+    return latent_run(q_c, q_r, w_uk, w_uv, latent_pages, cache_lens, out, lse, B, h_q, g, s_q, d_h, r_kv, d_r,
+                      page_size * max_pages, causal, scale, dtype, ws, ws_bytes, stream, &pg);
 }
 
 }  // extern "C"

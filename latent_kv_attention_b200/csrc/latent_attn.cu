@@ -187,9 +187,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(lat::NTHREADS, 1)
             prefetch_tensormap(&tm_lat);
             // tiles PF ahead of the one being loaded are prefetched into L2, so that the ring (whose
             // stages stay busy until P*V) is refilled from L2 rather than from DRAM
+            // row of token `tok` of this sequence in the cache: contiguous [B][Lmax] slabs, or a page of the
+            // block table ([num_pages][page_size] rows; entries outside the pool are replaced by page 0, which
+            // is reported when the attention needs the token)
+            auto cache_row = [&](int tok) -> int {
+                if (!p.block_table) return b * p.Lmax + tok;
+                int page = 0;
+                const int j = tok / p.page_size;
+                if (j < p.max_pages) {
+                    page = p.block_table[(size_t)b * p.max_pages + j];
+                    if (page < 0 || page >= p.num_pages) {
+                        if (tok < kend) atomicOr(p.status, kDevBadPage);
+                        page = 0;
+                    }
+                }
+                return page * p.page_size + tok % p.page_size;
+            };
             auto prefetch = [&](int i) {
-                const int y = b * p.Lmax + kbeg + i * NT;
-                for (int kb = 0; kb < NKB; ++kb) tma_prefetch_2d(&tm_lat, (int)rank * 256 + kb * 64, y);
+                for (int r0 = 0; r0 < NT; r0 += p.box_rows) {
+                    const int y = cache_row(kbeg + i * NT + r0);
+                    for (int kb = 0; kb < NKB; ++kb) tma_prefetch_2d(&tm_lat, (int)rank * 256 + kb * 64, y);
+                }
             };
             for (int i = NST; i < min(n_tiles, PF); ++i) prefetch(i);
             int issued = 0;
@@ -203,8 +221,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(lat::NTHREADS, 1)
                 const uint32_t fb = smem_u32(&kv_full[s]);
                 mbar_arrive_expect_tx(fb, NKB * BOX);
                 const uint32_t dst = smem_u32(smem + OFF_KV + s * STAGE);
-                const int y = b * p.Lmax + kbeg + i * NT;
-                for (int kb = 0; kb < NKB; ++kb) tma_load_2d(dst + kb * BOX, &tm_lat, (int)rank * 256 + kb * 64, y, fb);
+                for (int r0 = 0; r0 < NT; r0 += p.box_rows) {  // one box, or one per page piece of the tile
+                    const int y = cache_row(kbeg + i * NT + r0);
+                    for (int kb = 0; kb < NKB; ++kb)
+                        tma_load_2d(dst + kb * BOX + r0 * 128, &tm_lat, (int)rank * 256 + kb * 64, y, fb);
+                }
                 if (i + PF < n_tiles) prefetch(i + PF);
                 ++issued;
             }

@@ -156,6 +156,18 @@ def gqa_paged(q, k_pages, v_pages, block_table, cache_lens, causal: bool, scale:
     return gqa(q, k, v, cache_lens, causal, scale, rows_b=rows_b, n_threads=n_threads)
 
 
+def latent_absorbed_paged(q_c, q_r, w_uk, w_uv, latent_pages, block_table, cache_lens, causal: bool, scale: float,
+                          rows_b=None, n_threads: int = 0):
+    """The MQA-absorbed latent attention over a paged latent cache [num_pages, page_size, r_kv + d_r]: the
+    contiguous latent cache the block table describes, then latent_absorbed()."""
+    pages = _f64(latent_pages)
+    bt = _i32(block_table)
+    Lmax = bt.shape[1] * pages.shape[1]
+    latent = paged_to_contiguous(pages[:, None], bt, Lmax)[:, 0]
+    return latent_absorbed(q_c, q_r, w_uk, w_uv, latent, cache_lens, causal, scale, rows_b=rows_b,
+                           n_threads=n_threads)
+
+
 def gqa_probs(q, k, cache_lens, causal: bool, scale: float, b: int, i: int, t: int, h_kv: int):
     """Softmax probabilities of one query row of the GQA definition (visible keys only)."""
     q, k, lens = _f64(q), _f64(k), _i32(cache_lens)

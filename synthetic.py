@@ -118,6 +118,20 @@ def gqa_paged_inputs(seed, B, h_q, h_kv, d, s_q, L_lo, L_hi, page_size, Lmax=Non
     return inp
 
 
+def latent_paged_inputs(seed, B, h_q, g_groups, d_h, r_kv, d_r, s_q, L_lo, L_hi, page_size, Lmax=None,
+                        dtype=torch.bfloat16, device="cpu", spare_pages=3):
+    """GQLA latent inputs (as latent_inputs) with the latent cache moved into a shuffled page pool
+    [num_pages, page_size, r_kv + d_r] and a block table; the capacity is rounded up to whole pages."""
+    Lmax = L_hi if Lmax is None else Lmax
+    Lmax = -(-Lmax // page_size) * page_size
+    inp = latent_inputs(seed, B, h_q, g_groups, d_h, r_kv, d_r, s_q, L_lo, L_hi, Lmax=Lmax, dtype=dtype,
+                        device=device)
+    g = _gen(seed + 7919, device)
+    (pool,), table = to_pages([inp["latent"][:, None]], inp["cache_lens"], page_size, g, spare_pages)
+    inp.update(latent_pages=pool[:, 0].contiguous(), block_table=table, page_size=page_size)
+    return inp
+
+
 def latent_inputs(seed, B, h_q, g_groups, d_h, r_kv, d_r, s_q, L_lo, L_hi, Lmax=None, dtype=torch.bfloat16,
                   device="cpu"):
     """GQLA latent decode inputs: c^KV, k^R, q^C, q^R ~ N(0,1); W^UK, W^UV ~ N(0, 1/r_kv)."""
@@ -175,6 +189,9 @@ WORKLOADS = {
                                  L_lo=4096, L_hi=4096, causal=True),
     "latent_decode_4k_sq2": dict(kind="latent", seed=4, B=64, h_q=128, g=8, d_h=128, r_kv=512, d_r=64, s_q=2,
                                  L_lo=4096, L_hi=4096, causal=True),
+    # the s_q = 1 layer over a paged latent cache (64-token pages, shuffled pool, block table)
+    "latent_decode_4k_sq1_paged": dict(kind="latent_paged", seed=4, B=64, h_q=128, g=8, d_h=128, r_kv=512, d_r=64,
+                                       s_q=1, L_lo=4096, L_hi=4096, causal=True, page_size=64),
     # half the batch: the small case for full ncu captures of the latent kernels (latent cache 151 MB > L2)
     "latent_decode_4k_sq1_b32": dict(kind="latent", seed=4, B=32, h_q=128, g=8, d_h=128, r_kv=512, d_r=64, s_q=1,
                                      L_lo=4096, L_hi=4096, causal=True),
@@ -206,6 +223,9 @@ def make(w: dict, device="cpu", dtype=torch.bfloat16) -> dict:
     if w["kind"] == "gqa_paged":
         return gqa_paged_inputs(w["seed"], w["B"], w["h_q"], w["h_kv"], w["d"], w["s_q"], w["L_lo"], w["L_hi"],
                                 w["page_size"], dtype=dtype, device=device)
+    if w["kind"] == "latent_paged":
+        return latent_paged_inputs(w["seed"], w["B"], w["h_q"], w["g"], w["d_h"], w["r_kv"], w["d_r"], w["s_q"],
+                                   w["L_lo"], w["L_hi"], w["page_size"], dtype=dtype, device=device)
     if w["kind"] == "latent":
         return latent_inputs(w["seed"], w["B"], w["h_q"], w["g"], w["d_h"], w["r_kv"], w["d_r"], w["s_q"],
                              w["L_lo"], w["L_hi"], dtype=dtype, device=device)

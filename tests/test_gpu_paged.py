@@ -66,3 +66,20 @@ def test_paged_out_of_pool_entry_is_replaced_and_reported():
     lka.gqa_attn_paged(d["q"], d["k_pages"], d["v_pages"], bt, d["cache_lens"], scale=inp["scale"])
     assert lka.device_status() == 7  # LKA_ERR_BAD_PAGE
     lka.clear_status()
+
+
+@pytest.mark.parametrize("page_size,s_q", [(16, 1), (64, 2), (128, 1), (256, 2)])
+def test_latent_absorbed_paged(page_size, s_q):
+    inp = synthetic.latent_paged_inputs(400 + page_size + s_q, 2, 128, 8, 128, 512, 64, s_q, s_q, 700, page_size,
+                                        Lmax=768)
+    d = {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    out, lse = lka.latent_absorbed_attn_paged(d["q_c"], d["q_r"], d["w_uk"], d["w_uv"], d["latent_pages"],
+                                              d["block_table"], d["cache_lens"], causal=True, scale=inp["scale"],
+                                              return_lse=True)
+    ref, ref_lse = oracle.latent_absorbed_paged(inp["q_c"], inp["q_r"], inp["w_uk"], inp["w_uv"], inp["latent_pages"],
+                                                inp["block_table"], inp["cache_lens"], True, inp["scale"])
+    assert_close(out, ref, torch.bfloat16, "latent paged out")
+    assert_lse_close(lse, ref_lse, torch.bfloat16, "latent paged lse")
+    cont = lka.latent_absorbed_attn(d["q_c"], d["q_r"], d["w_uk"], d["w_uv"], d["latent"], d["cache_lens"],
+                                    causal=True, scale=inp["scale"])
+    assert torch.equal(out, cont)

@@ -358,3 +358,12 @@ def test_paged_oracle_shuffled_pool_and_shared_prefix():
     ref, _ = oracle.gqa(q, k, v, lens, True, 0.25)
     out, _ = oracle.gqa_paged(q, pool_k, pool_v, table, lens, True, 0.25)
     assert np.array_equal(out, ref)
+
+
+def test_latent_paged_oracle_equals_contiguous():
+    inp = synthetic.latent_paged_inputs(64, 2, 16, 1, 16, 32, 8, 2, 2, 40, 8, dtype=torch.float32)
+    ref, _ = oracle.latent_absorbed(inp["q_c"], inp["q_r"], inp["w_uk"], inp["w_uv"], inp["latent"],
+                                    inp["cache_lens"], True, inp["scale"])
+    out, _ = oracle.latent_absorbed_paged(inp["q_c"], inp["q_r"], inp["w_uk"], inp["w_uv"], inp["latent_pages"],
+                                          inp["block_table"], inp["cache_lens"], True, inp["scale"])
+    assert np.array_equal(out, ref)
