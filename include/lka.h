@@ -179,6 +179,23 @@ LKA_API lka_status_t latent_expand_gqa_attn(const void *q_c, const void *q_r, co
                                     int h_q, int g, int s_q, int d_h, int d_r, int Lmax, int causal, float scale,
                                     lka_dtype_t dtype, void *ws, size_t ws_bytes, void *stream);
 
+/* (c') The same over paged caches  [GQA "GQA compared with related
+ *  techniques" (PagedAttention); GQLA sec. 2 (paged KV caches)].
+ *   kc_pages, vc_pages [num_pages, g, page_size, d_h]   kr_pages [num_pages, page_size, d_r]
+ *   block_table [B, max_pages] int32: token t of sequence b is row t % page_size of
+ *   page block_table[b][t / page_size] in all three pools.  latent_expand_cache with
+ *   B = num_pages and Lmax = page_size converts a paged latent pool into these pools.
+ *  page_size a power of two >= 8; out-of-pool entries a call needs are replaced by
+ *  page 0 and raise LKA_ERR_BAD_PAGE.  Other arguments and results as in (c). */
+LKA_API size_t latent_expand_gqa_attn_paged_workspace_size(int B, int h_q, int g, int s_q, int d_h, int d_r,
+                                                           int page_size, int max_pages);
+LKA_API lka_status_t latent_expand_gqa_attn_paged(const void *q_c, const void *q_r, const void *kc_pages,
+                                          const void *vc_pages, const void *kr_pages, const int32_t *block_table,
+                                          const int32_t *cache_lens, void *out, float *lse, int B, int h_q, int g,
+                                          int s_q, int d_h, int d_r, int page_size, int max_pages, int num_pages,
+                                          int causal, float scale, lka_dtype_t dtype, void *ws, size_t ws_bytes,
+                                          void *stream);
+
 /* ------------------------------------------------------------------------ */
 /* (d) GTA shared-score attention  [GTA, grouped shared attention matrix]   */
 /*  H heads in G groups of H/G; head h uses group gamma = floor(h/(H/G)).    */

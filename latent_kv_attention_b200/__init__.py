@@ -50,6 +50,8 @@ SIGNATURES = {
     "latent_absorbed_attn_paged": (_I, [_P] * 9 + [_I] * 11 + [_F, _I, _P, _Z, _P]),
     "latent_expand_gqa_attn_workspace_size": (_Z, [_I] * 7),
     "latent_expand_gqa_attn": (_I, [_P] * 8 + [_I] * 8 + [_F, _I, _P, _Z, _P]),
+    "latent_expand_gqa_attn_paged_workspace_size": (_Z, [_I] * 8),
+    "latent_expand_gqa_attn_paged": (_I, [_P] * 9 + [_I] * 10 + [_F, _I, _P, _Z, _P]),
     "gta_shared_score_attn_workspace_size": (_Z, [_I] * 7),
     "gta_shared_score_attn": (_I, [_P] * 6 + [_I] * 8 + [_F, _I, _P, _Z, _P]),
     "latent_expand_cache": (_I, [_P] * 3 + [_I] * 6 + [_P] * 3 + [_I, _P]),
@@ -281,6 +283,36 @@ def latent_expand_gqa_attn(q_c, q_r, kc, vc, kr, cache_lens, causal: bool = True
                                     _ptr(lse), B, h_q, g, s_q, d_h, d_r, Lmax, int(bool(causal)), scale,
                                     _dtype_code(q_c), _ptr(ws), ws.numel(), _stream_ptr())
     _check("latent_expand_gqa_attn", rc)
+    return (out, lse) if return_lse else out
+
+
+def latent_expand_gqa_attn_paged(q_c, q_r, kc_pages, vc_pages, kr_pages, block_table, cache_lens, causal: bool = True,
+                                 scale: float | None = None, out=None, return_lse: bool = False):
+    """latent_expand_gqa_attn over paged caches: kc_pages/vc_pages [num_pages, g, page_size, d_h], kr_pages
+    [num_pages, page_size, d_r], block_table int32 [B, max_pages]."""
+    for n, t in (("q_c", q_c), ("q_r", q_r), ("kc_pages", kc_pages), ("vc_pages", vc_pages), ("kr_pages", kr_pages)):
+        _device_tensor(t, n, torch.bfloat16)
+    B, h_q, s_q, d_h = q_c.shape
+    num_pages, g, page_size, _ = kc_pages.shape
+    d_r = kr_pages.shape[-1]
+    _require(vc_pages.shape == kc_pages.shape and kr_pages.shape[:2] == (num_pages, page_size),
+             "kc/vc pages [num_pages, g, page_size, d_h], kr pages [num_pages, page_size, d_r]")
+    _device_tensor(block_table, "block_table", torch.int32)
+    _require(block_table.dim() == 2 and block_table.shape[0] == B, "block_table must be int32 [B, max_pages]")
+    max_pages = block_table.shape[1]
+    _lens_tensor(cache_lens, B, q_c.device)
+    scale = 1.0 / math.sqrt(d_h + d_r) if scale is None else float(scale)
+    out = torch.empty_like(q_c) if out is None else out
+    lse = torch.empty((B, h_q, s_q), dtype=torch.float32, device=q_c.device) if return_lse else None
+    lib = library()
+    nbytes = lib.latent_expand_gqa_attn_paged_workspace_size(B, h_q, g, s_q, d_h, d_r, page_size, max_pages)
+    _require(nbytes > 0, "unsupported expanded shape or page layout")
+    ws = workspaces.get(nbytes, q_c.device)
+    rc = lib.latent_expand_gqa_attn_paged(_ptr(q_c), _ptr(q_r), _ptr(kc_pages), _ptr(vc_pages), _ptr(kr_pages),
+                                          _ptr(block_table), _ptr(cache_lens), _ptr(out), _ptr(lse), B, h_q, g, s_q,
+                                          d_h, d_r, page_size, max_pages, num_pages, int(bool(causal)), scale, 0,
+                                          _ptr(ws), ws.numel(), _stream_ptr())
+    _check("latent_expand_gqa_attn_paged", rc)
     return (out, lse) if return_lse else out
 
 

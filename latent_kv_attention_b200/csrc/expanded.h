@@ -17,6 +17,10 @@ struct ExpParams {
     int B, h_q, g, s_q, Lmax, causal;
     float scale_log2;
     int split_tokens, nsplit;
+    // paged caches (block_table == nullptr: contiguous kc, vc [B, g, Lmax, 128], kr [B, Lmax, 64])
+    const int32_t* block_table;  // device [B][max_pages] page indices, or nullptr
+    int page_size, max_pages, num_pages;
+    int box_rows;                // rows per TMA box: min(page_size, tile)
 };
 
 cudaError_t expanded_attn_launch(const CUtensorMap& qc, const CUtensorMap& qr, const CUtensorMap& kc,

@@ -127,17 +127,41 @@ __global__ void __launch_bounds__(192, 1)
             // their score MMAs complete, value tiles after their P*V MMAs
             int k_issued = 0, v_issued = 0;
             bool ok = true;
+            // rows of token `tok` in the per-group cache (kc, vc) and in the RoPE-key cache (kr): contiguous
+            // [B][g][Lmax] / [B][Lmax] slabs, or a page of the block table ([num_pages][g][page_size] /
+            // [num_pages][page_size]); entries outside the pool are replaced by page 0 (reported when the
+            // attention needs the token)
+            auto rows_of = [&](int tok, int& yg, int& yr) {
+                if (!p.block_table) {
+                    yg = (b * p.g + grp) * p.Lmax + tok;
+                    yr = b * p.Lmax + tok;
+                    return;
+                }
+                int page = 0;
+                const int j = tok / p.page_size;
+                if (j < p.max_pages) {
+                    page = p.block_table[(size_t)b * p.max_pages + j];
+                    if (page < 0 || page >= p.num_pages) {
+                        if (tok < L) atomicOr(p.status, kDevBadPage);
+                        page = 0;
+                    }
+                }
+                yg = (page * p.g + grp) * p.page_size + tok % p.page_size;
+                yr = page * p.page_size + tok % p.page_size;
+            };
             auto issue_k = [&](int i) {
                 const int s = i % NST;
                 if (i >= NST && !mbar_wait(smem_u32(&k_empty[s]), ((i / NST) - 1) & 1, p.status)) return false;
                 const uint32_t fb = smem_u32(&k_full[s]);
                 mbar_arrive_expect_tx(fb, C::KSTAGE);
                 const uint32_t d = smem_u32(smem + C::OFF_KV + s * C::STAGE);
-                const int k0 = kbeg + i * TK;
-                const int yg = (b * p.g + grp) * p.Lmax + k0;
-                tma_load_2d(d, &tm_kc, 0, yg, fb);
-                tma_load_2d(d + C::BOX, &tm_kc, 64, yg, fb);
-                tma_load_2d(d + 2 * C::BOX, &tm_kr, 0, b * p.Lmax + k0, fb);
+                for (int r0 = 0; r0 < TK; r0 += p.box_rows) {  // one box, or one per page piece of the tile
+                    int yg, yr;
+                    rows_of(kbeg + i * TK + r0, yg, yr);
+                    tma_load_2d(d + r0 * 128, &tm_kc, 0, yg, fb);
+                    tma_load_2d(d + C::BOX + r0 * 128, &tm_kc, 64, yg, fb);
+                    tma_load_2d(d + 2 * C::BOX + r0 * 128, &tm_kr, 0, yr, fb);
+                }
                 ++k_issued;
                 return true;
             };
@@ -147,9 +171,12 @@ __global__ void __launch_bounds__(192, 1)
                 const uint32_t fb = smem_u32(&v_full[s]);
                 mbar_arrive_expect_tx(fb, C::VSTAGE);
                 const uint32_t d = smem_u32(smem + C::OFF_KV + s * C::STAGE + C::KSTAGE);
-                const int yg = (b * p.g + grp) * p.Lmax + kbeg + i * TK;
-                tma_load_2d(d, &tm_vc, 0, yg, fb);
-                tma_load_2d(d + C::BOX, &tm_vc, 64, yg, fb);
+                for (int r0 = 0; r0 < TK; r0 += p.box_rows) {
+                    int yg, yr;
+                    rows_of(kbeg + i * TK + r0, yg, yr);
+                    tma_load_2d(d + r0 * 128, &tm_vc, 0, yg, fb);
+                    tma_load_2d(d + C::BOX + r0 * 128, &tm_vc, 64, yg, fb);
+                }
                 ++v_issued;
                 return true;
             };
@@ -402,11 +429,11 @@ struct ExpPlan {
     int split_tokens, nsplit;
     size_t off_lse, off_o, ws_bytes;
 };
-lka_status_t exp_plan(int B, int h_q, int g, int s_q, int d_h, int d_r, int Lmax, ExpPlan* pl) {
+lka_status_t exp_plan(int B, int h_q, int g, int s_q, int d_h, int d_r, int Lmax, ExpPlan* pl, bool paged = false) {
     if (B < 0 || h_q < 1 || g < 1 || s_q < 1 || d_h < 1 || d_r < 0 || Lmax < 1) return LKA_ERR_INVALID_ARG;
     if (h_q % g) return LKA_ERR_INVALID_ARG;
     if (h_q / g != 16 || d_h != 128 || d_r != 64 || s_q > 2) return LKA_ERR_UNSUPPORTED;
-    if ((long long)B * g * Lmax >= (1ll << 31) || B > 65535 || g > 65535) return LKA_ERR_UNSUPPORTED;
+    if ((!paged && (long long)B * g * Lmax >= (1ll << 31)) || B > 65535 || g > 65535) return LKA_ERR_UNSUPPORTED;
     int st = split_tokens_knob();
     if (st <= 0) {
         const long long units = (long long)(B > 0 ? B : 1) * g;
@@ -438,13 +465,21 @@ size_t latent_expand_gqa_attn_workspace_size(int B, int h_q, int g, int s_q, int
     return exp_plan(B, h_q, g, s_q, d_h, d_r, Lmax, &pl) == LKA_OK ? pl.ws_bytes : 0;
 }
 
-lka_status_t latent_expand_gqa_attn(const void* q_c, const void* q_r, const void* kc, const void* vc, const void* kr,
-                                    const int32_t* cache_lens, void* out, float* lse, int B, int h_q, int g, int s_q,
-                                    int d_h, int d_r, int Lmax, int causal, float scale, lka_dtype_t dtype, void* ws,
-                                    size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+struct ExpPages {
+    const int32_t* block_table;
+    int page_size, max_pages, num_pages;
+};
+
+static lka_status_t expanded_run(const void* q_c, const void* q_r, const void* kc, const void* vc, const void* kr,
+                                 const int32_t* cache_lens, void* out, float* lse, int B, int h_q, int g, int s_q,
+                                 int d_h, int d_r, int Lmax, int causal, float scale, lka_dtype_t dtype, void* ws,
+                                 size_t ws_bytes, void* stream, const ExpPages* pg) {
     if (dtype != LKA_BF16) return LKA_ERR_UNSUPPORTED;
     ExpPlan pl;
-    lka_status_t s = exp_plan(B, h_q, g, s_q, d_h, d_r, Lmax, &pl);
+    lka_status_t s = exp_plan(B, h_q, g, s_q, d_h, d_r, Lmax, &pl, pg != nullptr);
     if (s != LKA_OK) return s;
     if (B == 0) return LKA_OK;
     const void* ptrs[] = {q_c, q_r, kc, vc, kr, cache_lens, out};
@@ -456,11 +491,15 @@ lka_status_t latent_expand_gqa_attn(const void* q_c, const void* q_r, const void
     const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const int NR = 16 * s_q;
     CUtensorMap t_qc, t_qr, t_kc, t_kr, t_vc;
+    // cache rows: per sequence (contiguous) or per page (paged); boxes are a whole 128-token tile or a page piece
+    const uint64_t seqs = pg ? (uint64_t)pg->num_pages : (uint64_t)B;
+    const int rows_per = pg ? pg->page_size : Lmax;
+    const uint32_t box_rows = pg && pg->page_size < 128 ? (uint32_t)pg->page_size : 128u;
     if (!make_tmap_2d(&t_qc, BF, q_c, d_h, (uint64_t)B * h_q * s_q, (uint64_t)d_h * 2, 64, NR) ||
         !make_tmap_2d(&t_qr, BF, q_r, d_r, (uint64_t)B * h_q * s_q, (uint64_t)d_r * 2, 64, NR) ||
-        !make_tmap_2d(&t_kc, BF, kc, d_h, (uint64_t)B * g * Lmax, (uint64_t)d_h * 2, 64, 128) ||
-        !make_tmap_2d(&t_kr, BF, kr, d_r, (uint64_t)B * Lmax, (uint64_t)d_r * 2, 64, 128) ||
-        !make_tmap_2d(&t_vc, BF, vc, d_h, (uint64_t)B * g * Lmax, (uint64_t)d_h * 2, 64, 128))
+        !make_tmap_2d(&t_kc, BF, kc, d_h, seqs * g * rows_per, (uint64_t)d_h * 2, 64, box_rows) ||
+        !make_tmap_2d(&t_kr, BF, kr, d_r, seqs * rows_per, (uint64_t)d_r * 2, 64, box_rows) ||
+        !make_tmap_2d(&t_vc, BF, vc, d_h, seqs * g * rows_per, (uint64_t)d_h * 2, 64, box_rows))
         return LKA_ERR_CUDA;
     uint8_t* w = static_cast<uint8_t*>(ws);
     ExpParams p{};
@@ -479,6 +518,11 @@ lka_status_t latent_expand_gqa_attn(const void* q_c, const void* q_r, const void
     p.scale_log2 = scale * 1.4426950408889634f;
     p.split_tokens = pl.split_tokens;
     p.nsplit = pl.nsplit;
+    p.block_table = pg ? pg->block_table : nullptr;
+    p.page_size = pg ? pg->page_size : 0;
+    p.max_pages = pg ? pg->max_pages : 0;
+    p.num_pages = pg ? pg->num_pages : 0;
+    p.box_rows = (int)box_rows;
     cudaStream_t st = (cudaStream_t)stream;
     if (expanded_attn_launch(t_qc, t_qr, t_kc, t_kr, t_vc, p, st) != cudaSuccess) return LKA_ERR_CUDA;
     if (pl.nsplit > 1) {
@@ -500,6 +544,44 @@ lka_status_t latent_expand_gqa_attn(const void* q_c, const void* q_r, const void
         if (gqa_combine_launch(gp, 2, d_h, st) != cudaSuccess) return LKA_ERR_CUDA;
     }
     return LKA_OK;
+}
+
+
+}  // namespace
+
+extern "C" {
+
+lka_status_t latent_expand_gqa_attn(const void* q_c, const void* q_r, const void* kc, const void* vc, const void* kr,
+                                    const int32_t* cache_lens, void* out, float* lse, int B, int h_q, int g, int s_q,
+                                    int d_h, int d_r, int Lmax, int causal, float scale, lka_dtype_t dtype, void* ws,
+                                    size_t ws_bytes, void* stream) {
+    return expanded_run(q_c, q_r, kc, vc, kr, cache_lens, out, lse, B, h_q, g, s_q, d_h, d_r, Lmax, causal, scale,
+                        dtype, ws, ws_bytes, stream, nullptr);
+}
+
+size_t latent_expand_gqa_attn_paged_workspace_size(int B, int h_q, int g, int s_q, int d_h, int d_r, int page_size,
+                                                   int max_pages) {
+    if (page_size < 8 || (page_size & (page_size - 1)) || max_pages < 1 ||
+        (long long)page_size * max_pages >= (1ll << 31))
+        return 0;
+    ExpPlan pl;
+    return exp_plan(B, h_q, g, s_q, d_h, d_r, page_size * max_pages, &pl, true) == LKA_OK ? pl.ws_bytes : 0;
+}
+
+lka_status_t latent_expand_gqa_attn_paged(const void* q_c, const void* q_r, const void* kc_pages,
+                                          const void* vc_pages, const void* kr_pages, const int32_t* block_table,
+                                          const int32_t* cache_lens, void* out, float* lse, int B, int h_q, int g,
+                                          int s_q, int d_h, int d_r, int page_size, int max_pages, int num_pages,
+                                          int causal, float scale, lka_dtype_t dtype, void* ws, size_t ws_bytes,
+                                          void* stream) {
+    if (page_size < 8 || (page_size & (page_size - 1)) || max_pages < 1 || num_pages < 1 || g < 1)
+        return LKA_ERR_INVALID_ARG;
+    if ((long long)page_size * max_pages >= (1ll << 31) || (long long)num_pages * g * page_size >= (1ll << 31))
+        return LKA_ERR_UNSUPPORTED;
+    if (B > 0 && (!block_table || (reinterpret_cast<uintptr_t>(block_table) & 3u))) return LKA_ERR_INVALID_ARG;
+    const ExpPages pg{block_table, page_size, max_pages, num_pages};
+    return expanded_run(q_c, q_r, kc_pages, vc_pages, kr_pages, cache_lens, out, lse, B, h_q, g, s_q, d_h, d_r,
+                        page_size * max_pages, causal, scale, dtype, ws, ws_bytes, stream, &pg);
 }
 
 }  // extern "C"

@@ -81,8 +81,8 @@ def gqa_inputs(seed, B, h_q, h_kv, d, s_q, L_lo, L_hi, Lmax=None, dtype=torch.bf
 
 
 def to_pages(caches, lens, page_size, gen, spare_pages=0):
-    """Scatters contiguous caches [B, h_kv, Lmax, d] (e.g. K and V) into shuffled page pools [num_pages, h_kv,
-    page_size, d] sharing one block table [B, Lmax / page_size] (int32): the pages a sequence uses
+    """Scatters contiguous caches [B, heads, Lmax, width] (e.g. K and V) into shuffled page pools [num_pages, heads,
+    page_size, width] sharing one block table [B, Lmax / page_size] (int32): the pages a sequence uses
     (ceil(len / page_size)) go to slots of a random permutation of the pool; its unused table entries are -1 and
     unused pool slots hold random values.  Layout only: no attention arithmetic."""
     B, h_kv, Lmax, d = caches[0].shape
@@ -91,8 +91,8 @@ def to_pages(caches, lens, page_size, gen, spare_pages=0):
     num_pages = B * max_pages + spare_pages
     dev = caches[0].device
     perm = torch.randperm(num_pages, generator=gen, device=dev).tolist()
-    pools = [torch.randn((num_pages, h_kv, page_size, d), generator=gen, device=dev, dtype=torch.float32).to(c.dtype)
-             for c in caches]
+    pools = [torch.randn((num_pages, c.shape[1], page_size, c.shape[3]), generator=gen, device=dev,
+                         dtype=torch.float32).to(c.dtype) for c in caches]
     table = torch.full((B, max_pages), -1, dtype=torch.int32)
     lens_l = lens.tolist()
     for b in range(B):
@@ -160,6 +160,21 @@ def expanded_inputs(seed, B, h_q, g_groups, d_h, d_r, s_q, L_lo, L_hi, Lmax=None
     vc = _randn((B, g_groups, Lmax, d_h), g, dtype, device)
     kr = _randn((B, Lmax, d_r), g, dtype, device)
     return dict(q_c=q_c, q_r=q_r, kc=kc, vc=vc, kr=kr, cache_lens=lens, scale=1.0 / math.sqrt(d_h + d_r))
+
+
+def expanded_paged_inputs(seed, B, h_q, g_groups, d_h, d_r, s_q, L_lo, L_hi, page_size, Lmax=None,
+                          dtype=torch.bfloat16, device="cpu", spare_pages=3):
+    """Expanded-path inputs (as expanded_inputs) with kc, vc and kr moved into shuffled page pools sharing one
+    block table; the capacity is rounded up to whole pages."""
+    Lmax = L_hi if Lmax is None else Lmax
+    Lmax = -(-Lmax // page_size) * page_size
+    inp = expanded_inputs(seed, B, h_q, g_groups, d_h, d_r, s_q, L_lo, L_hi, Lmax=Lmax, dtype=dtype, device=device)
+    g = _gen(seed + 7919, device)
+    (kc_p, vc_p, kr_p), table = to_pages([inp["kc"], inp["vc"], inp["kr"][:, None]], inp["cache_lens"], page_size, g,
+                                         spare_pages)
+    inp.update(kc_pages=kc_p, vc_pages=vc_p, kr_pages=kr_p[:, 0].contiguous(), block_table=table,
+               page_size=page_size)
+    return inp
 
 
 def gta_inputs(seed, B, G, H, d_qk, d_v, s_q, L_lo, L_hi, Lmax=None, dtype=torch.bfloat16, device="cpu"):

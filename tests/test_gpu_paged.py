@@ -83,3 +83,21 @@ def test_latent_absorbed_paged(page_size, s_q):
     cont = lka.latent_absorbed_attn(d["q_c"], d["q_r"], d["w_uk"], d["w_uv"], d["latent"], d["cache_lens"],
                                     causal=True, scale=inp["scale"])
     assert torch.equal(out, cont)
+
+
+@pytest.mark.parametrize("page_size,s_q", [(16, 2), (64, 1), (128, 2), (256, 1)])
+def test_expanded_paged(page_size, s_q):
+    from test_gpu_expanded import oracle_expanded
+
+    inp = synthetic.expanded_paged_inputs(500 + page_size + s_q, 3, 128, 8, 128, 64, s_q, s_q, 600, page_size,
+                                          Lmax=640)
+    d = {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    out, lse = lka.latent_expand_gqa_attn_paged(d["q_c"], d["q_r"], d["kc_pages"], d["vc_pages"], d["kr_pages"],
+                                                d["block_table"], d["cache_lens"], causal=True, scale=inp["scale"],
+                                                return_lse=True)
+    ref, ref_lse = oracle_expanded(inp, True)
+    assert_close(out, ref, torch.bfloat16, "expanded paged out")
+    assert_lse_close(lse, ref_lse, torch.bfloat16, "expanded paged lse")
+    cont = lka.latent_expand_gqa_attn(d["q_c"], d["q_r"], d["kc"], d["vc"], d["kr"], d["cache_lens"], causal=True,
+                                      scale=inp["scale"])
+    assert torch.equal(out, cont)
