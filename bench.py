@@ -15,8 +15,8 @@ Unless --no-extras is given, the line also carries `other_paths`: the same
 measurement (step time, GB/s, TFLOP/s, tokens/s, roofline of the main kernel,
 end-to-end time) for the GQA layer over a paged cache (64-token pages), the
 GQLA latent decode layer on the MQA-absorbed path (s_q = 1 and 2; s_q = 1 also
-over a paged latent cache), on the per-group GQA path (s_q = 2), and for the
-GTA causal prefill.
+over a paged latent cache, and top-2048 sparse over a 16K cache), on the
+per-group GQA path (s_q = 2), and for the GTA causal prefill.
 
 Prints ONE JSON line (rank 0).  `value` is the algorithmic HBM traffic of the
 step (every cache byte once, q read once, out written once) divided by the
@@ -343,6 +343,45 @@ class LatentAbsorbedPaged(LatentAbsorbed):
         return c
 
 
+class LatentSparse(LatentAbsorbed):
+    """latent_absorbed_attn_sparse: every query attends to 2048 selected tokens of its 16K-token latent cache
+    (gather of the selected rows into the workspace, then the dense latent kernels over them)."""
+
+    def setup_costs(self):
+        w = self.w
+        sel = [w["topk"]] * w["B"]  # every list holds topk visible positions
+        self.bytes = costs.latent_bytes(sel, w["h_q"], w["g"], w["d_h"], w["r_kv"], w["d_r"], w["s_q"])
+        self.core_flops = costs.latent_core_flops(sel, w["h_q"], w["r_kv"], w["d_r"], w["s_q"], False)
+        self.flops = self.core_flops + costs.latent_proj_flops(w["B"], w["h_q"], w["d_h"], w["r_kv"], w["s_q"])
+        self.tokens = w["B"] * w["s_q"]
+        self.sel_lens = sel
+
+    def kernel_work(self, pk):
+        cache = sum(self.sel_lens) * (self.w["r_kv"] + self.w["d_r"]) * 2
+        t_mem = cache / (pk["hbm_gbs"] * 1e9)
+        t_tc = self.core_flops / (pk["bf16_tflops"] * 1e12)
+        return ("tensor", self.core_flops) if t_tc > t_mem else ("hbm", cache)
+
+    def setup_device(self):
+        w, i = self.w, self.inp
+        self.out = torch.empty_like(i["q_c"])
+        self.launches = 8  # select, gather, lens, absorb GEMM, attention, merge, up-projection, finish (+ status fold)
+        self.h2d_pairs = [(i["q_c"], _pinned(i["q_c"])), (i["q_r"], _pinned(i["q_r"])),
+                          (i["indices"], _pinned(i["indices"])), (i["cache_lens"], _pinned(i["cache_lens"]))]
+        self.out_host = torch.empty_like(self.out, device="cpu").pin_memory()
+
+    def step(self):
+        i = self.inp
+        self.lka.latent_absorbed_attn_sparse(i["q_c"], i["q_r"], i["w_uk"], i["w_uv"], i["latent"], i["indices"],
+                                             i["cache_lens"], scale=i["scale"], out=self.out)
+
+    def config(self):
+        c = super().config()
+        c.update(path="MQA-absorbed, top-k sparse (indices given)", topk=self.w["topk"],
+                 l2="selected rows 151 MB > L2; L2 flushed between timed steps")
+        return c
+
+
 class LatentExpanded(LatentAbsorbed):
     """latent_expand_gqa_attn over the per-group expanded cache (made once, outside the timed steps)."""
 
@@ -444,6 +483,7 @@ WORKLOAD_CLASSES = {
     "latent_decode_4k_sq1": LatentAbsorbed,
     "latent_decode_4k_sq2": LatentAbsorbed,
     "latent_decode_4k_sq1_paged": LatentAbsorbedPaged,
+    "latent_sparse_16k_top2048": LatentSparse,
     "latent_expanded_4k_sq1": LatentExpanded,
     "latent_expanded_4k_sq2": LatentExpanded,
     "gta_prefill_4k": GtaPrefill,
@@ -453,7 +493,7 @@ WORKLOAD_CLASSES = {
     "gta_prefill_4k_b2": GtaPrefill,
 }
 EXTRAS = ["gqa_decode_llama8b_paged", "latent_decode_4k_sq1", "latent_decode_4k_sq1_paged", "latent_decode_4k_sq2",
-          "latent_expanded_4k_sq2", "gta_prefill_4k"]
+          "latent_sparse_16k_top2048", "latent_expanded_4k_sq2", "gta_prefill_4k"]
 
 
 def oracle_sample(wl, target_s: float):

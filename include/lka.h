@@ -196,6 +196,33 @@ LKA_API lka_status_t latent_expand_gqa_attn_paged(const void *q_c, const void *q
                                           int causal, float scale, lka_dtype_t dtype, void *ws, size_t ws_bytes,
                                           void *stream);
 
+/* (c'') Top-k sparse attention of both GQLA paths, given the selection
+ *  [GQLA sec. 1 "TransGQLA and sparse GQLA", sec. 2 "Sparse and long-context
+ *  attention": a token-dependent top-k selection of past keys/values; sparse
+ *  GQLA keeps both decode paths].  The indexer that picks the tokens is the
+ *  caller's.  indices [B, s_q, topk] int32 (device): for query token t of
+ *  sequence b, the cache positions it attends to; entry j counts when
+ *  0 <= j <= L_b - s_q + t, other entries (-1 for padding) are skipped, and
+ *  each entry that counts is one key of the softmax (lists should not repeat
+ *  a position).  A query whose list has no entry that counts gets out = 0 and
+ *  lse = -inf.  s_q <= 2; other arguments, layouts and shape limits as in (b)
+ *  (latent cache) and (c) (expanded caches).  The selected rows are gathered
+ *  into the workspace before the dense kernels run over them. */
+LKA_API size_t latent_absorbed_attn_sparse_workspace_size(int B, int h_q, int g, int s_q, int d_h, int r_kv, int d_r,
+                                                          int topk);
+LKA_API lka_status_t latent_absorbed_attn_sparse(const void *q_c, const void *q_r, const void *w_uk,
+                                         const void *w_uv, const void *latent, const int32_t *indices,
+                                         const int32_t *cache_lens, void *out, float *lse, int B, int h_q, int g,
+                                         int s_q, int d_h, int r_kv, int d_r, int Lmax, int topk, float scale,
+                                         lka_dtype_t dtype, void *ws, size_t ws_bytes, void *stream);
+LKA_API size_t latent_expand_gqa_attn_sparse_workspace_size(int B, int h_q, int g, int s_q, int d_h, int d_r,
+                                                            int topk);
+LKA_API lka_status_t latent_expand_gqa_attn_sparse(const void *q_c, const void *q_r, const void *kc,
+                                           const void *vc, const void *kr, const int32_t *indices,
+                                           const int32_t *cache_lens, void *out, float *lse, int B, int h_q, int g,
+                                           int s_q, int d_h, int d_r, int Lmax, int topk, float scale,
+                                           lka_dtype_t dtype, void *ws, size_t ws_bytes, void *stream);
+
 /* ------------------------------------------------------------------------ */
 /* (d) GTA shared-score attention  [GTA, grouped shared attention matrix]   */
 /*  H heads in G groups of H/G; head h uses group gamma = floor(h/(H/G)).    */

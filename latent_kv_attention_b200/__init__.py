@@ -51,6 +51,10 @@ SIGNATURES = {
     "latent_expand_gqa_attn_workspace_size": (_Z, [_I] * 7),
     "latent_expand_gqa_attn": (_I, [_P] * 8 + [_I] * 8 + [_F, _I, _P, _Z, _P]),
     "latent_expand_gqa_attn_paged_workspace_size": (_Z, [_I] * 8),
+    "latent_absorbed_attn_sparse_workspace_size": (_Z, [_I] * 8),
+    "latent_absorbed_attn_sparse": (_I, [_P] * 9 + [_I] * 9 + [_F, _I, _P, _Z, _P]),
+    "latent_expand_gqa_attn_sparse_workspace_size": (_Z, [_I] * 7),
+    "latent_expand_gqa_attn_sparse": (_I, [_P] * 9 + [_I] * 8 + [_F, _I, _P, _Z, _P]),
     "latent_expand_gqa_attn_paged": (_I, [_P] * 9 + [_I] * 10 + [_F, _I, _P, _Z, _P]),
     "gta_shared_score_attn_workspace_size": (_Z, [_I] * 7),
     "gta_shared_score_attn": (_I, [_P] * 6 + [_I] * 8 + [_F, _I, _P, _Z, _P]),
@@ -313,6 +317,61 @@ def latent_expand_gqa_attn_paged(q_c, q_r, kc_pages, vc_pages, kr_pages, block_t
                                           d_h, d_r, page_size, max_pages, num_pages, int(bool(causal)), scale, 0,
                                           _ptr(ws), ws.numel(), _stream_ptr())
     _check("latent_expand_gqa_attn_paged", rc)
+    return (out, lse) if return_lse else out
+
+
+def latent_absorbed_attn_sparse(q_c, q_r, w_uk, w_uv, latent, indices, cache_lens, scale: float | None = None,
+                                out=None, return_lse: bool = False):
+    """Top-k sparse MQA-absorbed latent attention: indices int32 [B, s_q, topk] are the cache positions each query
+    token attends to (entries outside [0, L_b - s_q + t] are skipped)."""
+    for n, t in (("q_c", q_c), ("q_r", q_r), ("w_uk", w_uk), ("w_uv", w_uv), ("latent", latent)):
+        _device_tensor(t, n, torch.bfloat16)
+    B, h_q, s_q, d_h = q_c.shape
+    d_r = q_r.shape[-1]
+    g, _, r_kv = w_uk.shape
+    Lmax = latent.shape[1]
+    _device_tensor(indices, "indices", torch.int32)
+    _require(indices.dim() == 3 and indices.shape[:2] == (B, s_q), "indices must be int32 [B, s_q, topk]")
+    topk = indices.shape[2]
+    _lens_tensor(cache_lens, B, q_c.device)
+    scale = 1.0 / math.sqrt(d_h + d_r) if scale is None else float(scale)
+    out = torch.empty_like(q_c) if out is None else out
+    lse = torch.empty((B, h_q, s_q), dtype=torch.float32, device=q_c.device) if return_lse else None
+    lib = library()
+    nbytes = lib.latent_absorbed_attn_sparse_workspace_size(B, h_q, g, s_q, d_h, r_kv, d_r, topk)
+    _require(nbytes > 0, "unsupported sparse latent shape")
+    ws = workspaces.get(nbytes, q_c.device)
+    rc = lib.latent_absorbed_attn_sparse(_ptr(q_c), _ptr(q_r), _ptr(w_uk), _ptr(w_uv), _ptr(latent), _ptr(indices),
+                                         _ptr(cache_lens), _ptr(out), _ptr(lse), B, h_q, g, s_q, d_h, r_kv, d_r, Lmax,
+                                         topk, scale, 0, _ptr(ws), ws.numel(), _stream_ptr())
+    _check("latent_absorbed_attn_sparse", rc)
+    return (out, lse) if return_lse else out
+
+
+def latent_expand_gqa_attn_sparse(q_c, q_r, kc, vc, kr, indices, cache_lens, scale: float | None = None, out=None,
+                                  return_lse: bool = False):
+    """Top-k sparse attention on the per-group GQA path: indices int32 [B, s_q, topk] as in
+    latent_absorbed_attn_sparse; kc, vc [B, g, Lmax, d_h], kr [B, Lmax, d_r]."""
+    for n, t in (("q_c", q_c), ("q_r", q_r), ("kc", kc), ("vc", vc), ("kr", kr)):
+        _device_tensor(t, n, torch.bfloat16)
+    B, h_q, s_q, d_h = q_c.shape
+    _, g, Lmax, _ = kc.shape
+    d_r = kr.shape[-1]
+    _device_tensor(indices, "indices", torch.int32)
+    _require(indices.dim() == 3 and indices.shape[:2] == (B, s_q), "indices must be int32 [B, s_q, topk]")
+    topk = indices.shape[2]
+    _lens_tensor(cache_lens, B, q_c.device)
+    scale = 1.0 / math.sqrt(d_h + d_r) if scale is None else float(scale)
+    out = torch.empty_like(q_c) if out is None else out
+    lse = torch.empty((B, h_q, s_q), dtype=torch.float32, device=q_c.device) if return_lse else None
+    lib = library()
+    nbytes = lib.latent_expand_gqa_attn_sparse_workspace_size(B, h_q, g, s_q, d_h, d_r, topk)
+    _require(nbytes > 0, "unsupported sparse expanded shape")
+    ws = workspaces.get(nbytes, q_c.device)
+    rc = lib.latent_expand_gqa_attn_sparse(_ptr(q_c), _ptr(q_r), _ptr(kc), _ptr(vc), _ptr(kr), _ptr(indices),
+                                           _ptr(cache_lens), _ptr(out), _ptr(lse), B, h_q, g, s_q, d_h, d_r, Lmax,
+                                           topk, scale, 0, _ptr(ws), ws.numel(), _stream_ptr())
+    _check("latent_expand_gqa_attn_sparse", rc)
     return (out, lse) if return_lse else out
 
 

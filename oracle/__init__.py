@@ -168,6 +168,70 @@ def latent_absorbed_paged(q_c, q_r, w_uk, w_uv, latent_pages, block_table, cache
                            n_threads=n_threads)
 
 
+def sparse_selection(indices, cache_lens, s_q: int):
+    """The keys each query token attends to under top-k sparse attention ("GQLA ..." sections 1 and 2: a
+    token-dependent top-k selection of past keys/values): for query t of sequence b, the entries j of
+    indices[b, t] with 0 <= j <= L_b - s_q + t, in list order.  Returns a list (over b) of lists (over t)."""
+    idx = _i32(indices)
+    lens = _i32(cache_lens)
+    out = []
+    for b in range(idx.shape[0]):
+        row = []
+        for t in range(s_q):
+            last = int(lens[b]) - s_q + t
+            row.append([int(j) for j in idx[b, t] if 0 <= j <= last])
+        out.append(row)
+    return out
+
+
+def _sparse_apply(dense, q_parts, sel, cache_rows, out_shape, lse_shape):
+    """Runs `dense` (a non-causal single-query attention of this module) per (sequence, query token) over the
+    selected cache rows; an empty selection gives out = 0, lse = -inf."""
+    out = np.zeros(out_shape)
+    lse = np.full(lse_shape, -np.inf)
+    B, s_q = len(sel), len(sel[0])
+    for b in range(B):
+        for t in range(s_q):
+            keys = sel[b][t]
+            if not keys:
+                continue
+            o, l = dense([qp[b:b + 1, :, t:t + 1] for qp in q_parts], [c(b, keys) for c in cache_rows],
+                         np.array([len(keys)], dtype=np.int32))
+            out[b, :, t] = o[0, :, 0]
+            lse[b, :, t] = l[0, :, 0]
+    return out, lse
+
+
+def latent_absorbed_sparse(q_c, q_r, w_uk, w_uv, latent, indices, cache_lens, scale: float):
+    """Top-k sparse attention of the MQA-absorbed latent path: for each query token, latent_absorbed() over the
+    selected latent rows only (sparse_selection)."""
+    q_c, q_r, lat = _f64(q_c), _f64(q_r), _f64(latent)
+    B, h_q, s_q, d_h = q_c.shape
+    sel = sparse_selection(indices, cache_lens, s_q)
+    dense = lambda qs, cs, lens: latent_absorbed(qs[0], qs[1], w_uk, w_uv, cs[0], lens, False, scale)  # noqa: E731
+    return _sparse_apply(dense, [q_c, q_r], sel, [lambda b, keys: lat[b:b + 1, keys]], (B, h_q, s_q, d_h),
+                         (B, h_q, s_q))
+
+
+def expanded_sparse(q_c, q_r, kc, vc, kr, indices, cache_lens, scale: float):
+    """Top-k sparse attention of the per-group GQA path: GQA with key [kc[g] ; kr] and value vc[g] over the
+    selected tokens only (sparse_selection)."""
+    q_c, q_r, kc, vc, kr = _f64(q_c), _f64(q_r), _f64(kc), _f64(vc), _f64(kr)
+    B, h_q, s_q, d_h = q_c.shape
+    g = kc.shape[1]
+    sel = sparse_selection(indices, cache_lens, s_q)
+
+    def dense(qs, cs, lens):
+        key = np.concatenate([cs[0], np.broadcast_to(cs[2][:, None], cs[0].shape[:3] + (cs[2].shape[-1],))], -1)
+        val = np.concatenate([cs[1], np.zeros(cs[1].shape[:3] + (cs[2].shape[-1],))], -1)
+        o, l = gqa(np.concatenate([qs[0], qs[1]], -1), key, val, lens, False, scale)
+        return o[..., :d_h], l
+
+    rows = [lambda b, keys: kc[b:b + 1][:, :, keys], lambda b, keys: vc[b:b + 1][:, :, keys],
+            lambda b, keys: kr[b:b + 1, keys]]
+    return _sparse_apply(dense, [q_c, q_r], sel, rows, (B, h_q, s_q, d_h), (B, h_q, s_q))
+
+
 def gqa_probs(q, k, cache_lens, causal: bool, scale: float, b: int, i: int, t: int, h_kv: int):
     """Softmax probabilities of one query row of the GQA definition (visible keys only)."""
     q, k, lens = _f64(q), _f64(k), _i32(cache_lens)

@@ -177,6 +177,28 @@ def expanded_paged_inputs(seed, B, h_q, g_groups, d_h, d_r, s_q, L_lo, L_hi, pag
     return inp
 
 
+def sparse_indices(seed, cache_lens, s_q, topk, device="cpu", junk=0.0):
+    """Top-k selections for sparse attention: int32 [B, s_q, topk]; for query t of sequence b, distinct positions
+    drawn uniformly from the keys it may see ([0, L_b - s_q + t]), in random order, padded with -1 when fewer
+    are visible.  A fraction `junk` of the entries is replaced by positions the query may not see (beyond its
+    causal limit) or -1, which the attention must skip."""
+    g = _gen(seed, "cpu")
+    lens = cache_lens.cpu().tolist()
+    B = len(lens)
+    out = torch.full((B, s_q, topk), -1, dtype=torch.int32)
+    for b in range(B):
+        for t in range(s_q):
+            vis = int(lens[b]) - s_q + t + 1
+            n = min(topk, vis)
+            out[b, t, :n] = torch.randperm(vis, generator=g)[:n].to(torch.int32)
+            if junk > 0:
+                bad = torch.rand(topk, generator=g) < junk
+                beyond = torch.randint(vis, vis + 50, (topk,), generator=g, dtype=torch.int32)
+                out[b, t] = torch.where(bad, torch.where(torch.rand(topk, generator=g) < 0.5, beyond,
+                                                         torch.full_like(beyond, -1)), out[b, t])
+    return out.to(device)
+
+
 def gta_inputs(seed, B, G, H, d_qk, d_v, s_q, L_lo, L_hi, Lmax=None, dtype=torch.bfloat16, device="cpu"):
     """GTA shared-score inputs, all N(0,1). For prefill pass s_q == L_lo == L_hi."""
     Lmax = L_hi if Lmax is None else Lmax
@@ -207,6 +229,9 @@ WORKLOADS = {
     # the s_q = 1 layer over a paged latent cache (64-token pages, shuffled pool, block table)
     "latent_decode_4k_sq1_paged": dict(kind="latent_paged", seed=4, B=64, h_q=128, g=8, d_h=128, r_kv=512, d_r=64,
                                        s_q=1, L_lo=4096, L_hi=4096, causal=True, page_size=64),
+    # top-k sparse decode: 2048 of the 16K cached tokens per query, selected uniformly at random
+    "latent_sparse_16k_top2048": dict(kind="latent_sparse", seed=8, B=64, h_q=128, g=8, d_h=128, r_kv=512, d_r=64,
+                                      s_q=1, L_lo=16384, L_hi=16384, causal=True, topk=2048),
     # half the batch: the small case for full ncu captures of the latent kernels (latent cache 151 MB > L2)
     "latent_decode_4k_sq1_b32": dict(kind="latent", seed=4, B=32, h_q=128, g=8, d_h=128, r_kv=512, d_r=64, s_q=1,
                                      L_lo=4096, L_hi=4096, causal=True),
@@ -241,6 +266,11 @@ def make(w: dict, device="cpu", dtype=torch.bfloat16) -> dict:
     if w["kind"] == "latent_paged":
         return latent_paged_inputs(w["seed"], w["B"], w["h_q"], w["g"], w["d_h"], w["r_kv"], w["d_r"], w["s_q"],
                                    w["L_lo"], w["L_hi"], w["page_size"], dtype=dtype, device=device)
+    if w["kind"] == "latent_sparse":
+        inp = latent_inputs(w["seed"], w["B"], w["h_q"], w["g"], w["d_h"], w["r_kv"], w["d_r"], w["s_q"],
+                            w["L_lo"], w["L_hi"], dtype=dtype, device=device)
+        inp["indices"] = sparse_indices(w["seed"] + 1, inp["cache_lens"], w["s_q"], w["topk"], device=device)
+        return inp
     if w["kind"] == "latent":
         return latent_inputs(w["seed"], w["B"], w["h_q"], w["g"], w["d_h"], w["r_kv"], w["d_r"], w["s_q"],
                              w["L_lo"], w["L_hi"], dtype=dtype, device=device)

@@ -367,3 +367,39 @@ def test_latent_paged_oracle_equals_contiguous():
     out, _ = oracle.latent_absorbed_paged(inp["q_c"], inp["q_r"], inp["w_uk"], inp["w_uv"], inp["latent_pages"],
                                           inp["block_table"], inp["cache_lens"], True, inp["scale"])
     assert np.array_equal(out, ref)
+
+
+# ------------------------------------------------------------------ top-k sparse attention ------------------
+def test_sparse_oracle_full_selection_equals_dense_causal():
+    """Selecting every key a query may see (in a shuffled order) is the dense causal attention ("GQLA ..."
+    sections 1-2: sparse GQLA attends over a top-k subset of past keys)."""
+    inp = synthetic.latent_inputs(71, 2, 16, 1, 16, 32, 8, 2, 5, 30, dtype=torch.float32)
+    idx = synthetic.sparse_indices(72, inp["cache_lens"], 2, 40)  # topk >= every visible count
+    ref, ref_lse = oracle.latent_absorbed(inp["q_c"], inp["q_r"], inp["w_uk"], inp["w_uv"], inp["latent"],
+                                          inp["cache_lens"], True, inp["scale"])
+    out, lse = oracle.latent_absorbed_sparse(inp["q_c"], inp["q_r"], inp["w_uk"], inp["w_uv"], inp["latent"], idx,
+                                             inp["cache_lens"], inp["scale"])
+    assert np.allclose(out, ref, atol=1e-12, rtol=1e-12) and np.allclose(lse, ref_lse, atol=1e-12, rtol=1e-12)
+
+
+def test_sparse_oracle_subset_equals_dense_over_the_subset_and_skips_junk():
+    inp = synthetic.expanded_inputs(73, 2, 32, 2, 16, 8, 1, 10, 30, dtype=torch.float32)
+    idx = synthetic.sparse_indices(74, inp["cache_lens"], 1, 6, junk=0.3)
+    out, lse = oracle.expanded_sparse(inp["q_c"], inp["q_r"], inp["kc"], inp["vc"], inp["kr"], idx,
+                                      inp["cache_lens"], 0.3)
+    for b in range(2):
+        keys = [int(j) for j in idx[b, 0] if 0 <= j < int(inp["cache_lens"][b])]
+        kc, vc, kr = inp["kc"][b:b + 1, :, keys], inp["vc"][b:b + 1, :, keys], inp["kr"][b:b + 1, keys]
+        key = torch.cat([kc, kr[:, None].expand(-1, kc.shape[1], -1, -1)], -1)
+        val = torch.cat([vc, torch.zeros_like(key[..., vc.shape[-1]:])], -1)
+        q = torch.cat([inp["q_c"][b:b + 1], inp["q_r"][b:b + 1]], -1)
+        ref, ref_lse = oracle.gqa(q, key, val, torch.tensor([len(keys)], dtype=torch.int32), False, 0.3)
+        assert np.allclose(out[b], ref[0, ..., :16], atol=1e-13) and np.allclose(lse[b], ref_lse[0], atol=1e-13)
+
+
+def test_sparse_oracle_empty_selection():
+    inp = synthetic.latent_inputs(75, 1, 16, 1, 16, 32, 8, 1, 9, 9, dtype=torch.float32)
+    idx = torch.full((1, 1, 4), -1, dtype=torch.int32)
+    out, lse = oracle.latent_absorbed_sparse(inp["q_c"], inp["q_r"], inp["w_uk"], inp["w_uv"], inp["latent"], idx,
+                                             inp["cache_lens"], inp["scale"])
+    assert np.all(out == 0) and np.all(np.isneginf(lse))
