@@ -13,7 +13,8 @@ flushed between timed steps anyway.
 
 Unless --no-extras is given, the line also carries `other_paths`: the same
 measurement (step time, GB/s, TFLOP/s, tokens/s, roofline of the main kernel,
-end-to-end time) for the GQA layer over a paged cache (64-token pages), the
+end-to-end time) for the GQA layer over a paged cache (64-token pages) and
+over an e4m3 cache, the
 GQLA latent decode layer on the MQA-absorbed path (s_q = 1 and 2; s_q = 1 also
 over a paged latent cache, and top-2048 sparse over a 16K cache), on the
 per-group GQA path (s_q = 2), and for the GTA causal prefill.
@@ -263,6 +264,34 @@ class GqaDecodePaged(GqaDecode):
         return c
 
 
+class GqaDecodeFp8(GqaDecode):
+    """gqa_attn_fp8kv over the same decode batch with the K/V cache in e4m3 (one scale per KV head)."""
+
+    def setup_costs(self):
+        w = self.w
+        self.bytes = costs.gqa_bytes(self.lens, w["h_q"], w["h_kv"], w["d"], w["s_q"], kv_elem=1)
+        self.flops = costs.gqa_flops(self.lens, w["h_q"], w["d"], w["s_q"], w["causal"])
+        self.tokens = w["B"] * w["s_q"]
+
+    def setup_device(self):
+        w, i = self.w, self.inp
+        self.out = torch.empty_like(i["q"])
+        ws = self.lka.library().gqa_attn_fp8kv_workspace_size(w["B"], w["h_q"], w["h_kv"], w["s_q"], w["d"], w["L_hi"])
+        self.launches = 2 if ws > 256 else 1
+        self.h2d_pairs = [(i["q"], _pinned(i["q"])), (i["cache_lens"], _pinned(i["cache_lens"]))]
+        self.out_host = torch.empty_like(self.out, device="cpu").pin_memory()
+
+    def step(self):
+        i = self.inp
+        self.lka.gqa_attn_fp8kv(i["q"], i["k"], i["v"], i["k_scale"], i["v_scale"], i["cache_lens"],
+                                causal=self.w["causal"], scale=i["scale"], out=self.out)
+
+    def config(self):
+        c = super().config()
+        c["cache_dtype"] = "e4m3 (per-KV-head scales)"
+        return c
+
+
 class LatentAbsorbed(Workload):
     """latent_absorbed_attn over the GQLA/MLA decode batch: absorb GEMM, latent attention, up-projection."""
 
@@ -480,6 +509,7 @@ WORKLOAD_CLASSES = {
     "gqa_decode_llama8b": GqaDecode,
     "gqa_decode_llama8b_b16": GqaDecode,
     "gqa_decode_llama8b_paged": GqaDecodePaged,
+    "gqa_decode_llama8b_fp8": GqaDecodeFp8,
     "latent_decode_4k_sq1": LatentAbsorbed,
     "latent_decode_4k_sq2": LatentAbsorbed,
     "latent_decode_4k_sq1_paged": LatentAbsorbedPaged,
@@ -492,7 +522,7 @@ WORKLOAD_CLASSES = {
     "latent_expanded_4k_sq2_b16": LatentExpanded,
     "gta_prefill_4k_b2": GtaPrefill,
 }
-EXTRAS = ["gqa_decode_llama8b_paged", "latent_decode_4k_sq1", "latent_decode_4k_sq1_paged", "latent_decode_4k_sq2",
+EXTRAS = ["gqa_decode_llama8b_paged", "gqa_decode_llama8b_fp8", "latent_decode_4k_sq1", "latent_decode_4k_sq1_paged", "latent_decode_4k_sq2",
           "latent_sparse_16k_top2048", "latent_expanded_4k_sq2", "gta_prefill_4k"]
 
 

@@ -106,6 +106,22 @@ LKA_API lka_status_t gqa_attn_paged(const void *q, const void *k_pages, const vo
                             int h_q, int h_kv, int s_q, int d_h, int page_size, int max_pages, int num_pages,
                             int causal, float scale, lka_dtype_t dtype, void *ws, size_t ws_bytes, void *stream);
 
+/* (a'') GQA attention over an FP8 (e4m3) KV cache  [GQLA sec. 2: quantised KV
+ *  storage is a complementary system technique that lowers the bytes per
+ *  cached token].  Same computation and layouts as gqa_attn with K and V held
+ *  as e4m3 bytes and one fp32 dequantisation scale per KV head:
+ *    K[b,h,t,:] = k_scale[h] * k[b,h,t,:],  V[b,h,t,:] = v_scale[h] * v[b,h,t,:]
+ *   q, out [B,h_q,s_q,d_h] bf16;  k, v [B,h_kv,Lmax,d_h] e4m3 (one byte each);
+ *   k_scale, v_scale [h_kv] fp32 (device);  lse as in gqa_attn.
+ *  d_h in {128, 256}.  The e4m3 values are widened exactly; the scales are
+ *  applied in fp32 (the key scale with the softmax scale to the query, the
+ *  value scale to the output). */
+LKA_API size_t gqa_attn_fp8kv_workspace_size(int B, int h_q, int h_kv, int s_q, int d_h, int Lmax);
+LKA_API lka_status_t gqa_attn_fp8kv(const void *q, const void *k, const void *v, const float *k_scale,
+                            const float *v_scale, const int32_t *cache_lens, void *out, float *lse, int B, int h_q,
+                            int h_kv, int s_q, int d_h, int Lmax, int causal, float scale, void *ws, size_t ws_bytes,
+                            void *stream);
+
 /* gqa_attn for callers that cannot allocate device memory.  No counterpart in
  * the papers: it exists for callers that are handed only their input and
  * output buffers (a plugin or custom operator inside another runtime) or run

@@ -42,6 +42,8 @@ SIGNATURES = {
     "gqa_attn_workspace_size": (_Z, [_I] * 6),
     "gqa_attn": (_I, [_P] * 6 + [_I] * 7 + [_F, _I, _P, _Z, _P]),
     "gqa_attn_noalloc": (_I, [_P] * 6 + [_I] * 7 + [_F, _I, _P]),
+    "gqa_attn_fp8kv_workspace_size": (_Z, [_I] * 6),
+    "gqa_attn_fp8kv": (_I, [_P] * 8 + [_I] * 7 + [_F, _P, _Z, _P]),
     "gqa_attn_paged_workspace_size": (_Z, [_I] * 7),
     "gqa_attn_paged": (_I, [_P] * 7 + [_I] * 9 + [_F, _I, _P, _Z, _P]),
     "latent_absorbed_attn_workspace_size": (_Z, [_I] * 8),
@@ -177,6 +179,35 @@ def gqa_attn(q, k, v, cache_lens, causal: bool = True, scale: float | None = Non
     rc = lib.gqa_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(cache_lens), _ptr(out), _ptr(lse), B, h_q, h_kv, s_q, d, Lmax,
                       int(bool(causal)), scale, _dtype_code(q), _ptr(ws), ws.numel(), _stream_ptr())
     _check("gqa_attn", rc)
+    return (out, lse) if return_lse else out
+
+
+def gqa_attn_fp8kv(q, k, v, k_scale, v_scale, cache_lens, causal: bool = True, scale: float | None = None, out=None,
+                   return_lse: bool = False):
+    """GQA attention over an e4m3 KV cache: q [B,h_q,s_q,d] bf16; k, v [B,h_kv,Lmax,d] torch.float8_e4m3fn;
+    k_scale, v_scale fp32 [h_kv] (K = k_scale[h] * k, V = v_scale[h] * v); cache_lens int32 [B]."""
+    _device_tensor(q, "q", torch.bfloat16)
+    for n, t in (("k", k), ("v", v)):
+        _device_tensor(t, n, torch.float8_e4m3fn)
+    for n, t in (("k_scale", k_scale), ("v_scale", v_scale)):
+        _device_tensor(t, n, torch.float32)
+    _require(q.dim() == 4 and k.dim() == 4 and v.shape == k.shape, "q [B,h_q,s_q,d], k/v [B,h_kv,Lmax,d]")
+    B, h_q, s_q, d = q.shape
+    _, h_kv, Lmax, dk = k.shape
+    _require(dk == d and k.shape[0] == B and k_scale.numel() == h_kv and v_scale.numel() == h_kv,
+             "q, k/v and the scales disagree on B, d or h_kv")
+    _lens_tensor(cache_lens, B, q.device)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    out = torch.empty_like(q) if out is None else out
+    _device_tensor(out, "out", torch.bfloat16)
+    lse = torch.empty((B, h_q, s_q), dtype=torch.float32, device=q.device) if return_lse else None
+    lib = library()
+    nbytes = lib.gqa_attn_fp8kv_workspace_size(B, h_q, h_kv, s_q, d, Lmax)
+    ws = workspaces.get(nbytes, q.device)
+    rc = lib.gqa_attn_fp8kv(_ptr(q), _ptr(k), _ptr(v), _ptr(k_scale), _ptr(v_scale), _ptr(cache_lens), _ptr(out),
+                            _ptr(lse), B, h_q, h_kv, s_q, d, Lmax, int(bool(causal)), scale, _ptr(ws), ws.numel(),
+                            _stream_ptr())
+    _check("gqa_attn_fp8kv", rc)
     return (out, lse) if return_lse else out
 
 

@@ -40,8 +40,10 @@ def _visible(L: int, s_q: int, causal: bool) -> int:
     return sum(L - s_q + t + 1 for t in range(s_q))
 
 
-def gqa_bytes(lens: Sequence[int], h_q: int, h_kv: int, d: int, s_q: int, elem: int = 2) -> int:
-    kv = sum(int(L) for L in lens) * h_kv * 2 * d * elem
+def gqa_bytes(lens: Sequence[int], h_q: int, h_kv: int, d: int, s_q: int, elem: int = 2, kv_elem: int | None = None) -> int:
+    """Cache bytes read once (kv_elem bytes per value, default elem) plus q read and out written (elem bytes)."""
+    kv_elem = elem if kv_elem is None else kv_elem
+    kv = sum(int(L) for L in lens) * h_kv * 2 * d * kv_elem
     qo = len(lens) * h_q * s_q * d * elem * 2
     return kv + qo
 

@@ -63,17 +63,19 @@ static int pick_rb(int rows, int d, int dtype_bytes) {
 }
 
 static lka_status_t gqa_plan(int B, int h_q, int h_kv, int s_q, int d_h, int Lmax, int dtype_bytes, GqaPlan* pl,
-                             bool paged = false) {
+                             bool paged = false, bool fp8kv = false) {
     if (B < 0 || h_q < 1 || h_kv < 1 || s_q < 1 || Lmax < 1 || d_h < 1) return LKA_ERR_INVALID_ARG;
     if (h_q % h_kv) return LKA_ERR_INVALID_ARG;
-    const bool d_ok = dtype_bytes == 2 ? (d_h == 64 || d_h == 128 || d_h == 256) : (d_h == 64 || d_h == 128);
+    const bool d_ok = fp8kv ? (d_h == 128 || d_h == 256)
+                            : dtype_bytes == 2 ? (d_h == 64 || d_h == 128 || d_h == 256) : (d_h == 64 || d_h == 128);
     if (!d_ok) return LKA_ERR_UNSUPPORTED;
     if (!paged && (long long)B * h_kv * Lmax >= (1ll << 31)) return LKA_ERR_UNSUPPORTED;
     const int R = (h_q / h_kv) * s_q;
     pl->rb = pick_rb(R, d_h, dtype_bytes);
+    if (fp8kv && pl->rb > 4) pl->rb = 4;
     pl->n_rb = cdiv(R, pl->rb);
     if ((long long)h_kv * pl->n_rb > 65535 || B > 65535) return LKA_ERR_UNSUPPORTED;
-    pl->tile = gqa_tile_tokens(dtype_bytes, d_h, pl->rb);
+    pl->tile = fp8kv ? gqa_fp8_tile_tokens(d_h, pl->rb) : gqa_tile_tokens(dtype_bytes, d_h, pl->rb);
     if (pl->tile <= 0) return LKA_ERR_UNSUPPORTED;
     int st = split_tokens_knob();
     if (st <= 0) {
@@ -197,11 +199,15 @@ struct PagedDesc {
 // Shared by gqa_attn (pg == nullptr: contiguous cache [B, h_kv, Lmax, d]) and gqa_attn_paged.
 static lka_status_t gqa_run(const void* q, const void* k, const void* v, const int32_t* cache_lens, void* out,
                             float* lse, int B, int h_q, int h_kv, int s_q, int d_h, int Lmax, int causal, float scale,
-                            lka_dtype_t dtype, void* ws, size_t ws_bytes, void* stream, const PagedDesc* pg) {
+                            lka_dtype_t dtype, void* ws, size_t ws_bytes, void* stream, const PagedDesc* pg,
+                            const float* k_scale = nullptr, const float* v_scale = nullptr) {
     if (dtype != LKA_BF16 && dtype != LKA_FP32) return LKA_ERR_UNSUPPORTED;
+    const bool fp8kv = k_scale != nullptr;  // e4m3 cache with per-KV-head scales (bf16 q / out)
+    if (fp8kv && dtype != LKA_BF16) return LKA_ERR_UNSUPPORTED;
     const int eb = dtype == LKA_BF16 ? 2 : 4;
+    const int kvb = fp8kv ? 1 : eb;  // bytes of one cache element
     GqaPlan pl;
-    lka_status_t s = gqa_plan(B, h_q, h_kv, s_q, d_h, Lmax, eb, &pl, pg != nullptr);
+    lka_status_t s = gqa_plan(B, h_q, h_kv, s_q, d_h, Lmax, eb, &pl, pg != nullptr, fp8kv);
     if (s != LKA_OK) return s;
     if (B == 0) return LKA_OK;
     if (!q || !k || !v || !cache_lens || !out) return LKA_ERR_INVALID_ARG;
@@ -211,7 +217,8 @@ static lka_status_t gqa_run(const void* q, const void* k, const void* v, const i
     if (!ws || ws_bytes < pl.ws_bytes) return LKA_ERR_WORKSPACE;
     if (!aligned16(ws)) return LKA_ERR_INVALID_ARG;
 
-    const CUtensorMapDataType tdt = eb == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    const CUtensorMapDataType tdt = fp8kv ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                    : eb == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     uint64_t rows = (uint64_t)B * h_kv * Lmax;
     uint32_t box_rows = (uint32_t)pl.tile;
     if (pg) {
@@ -219,8 +226,8 @@ static lka_status_t gqa_run(const void* q, const void* k, const void* v, const i
         box_rows = (uint32_t)(pg->page_size < pl.tile ? pg->page_size : pl.tile);
     }
     CUtensorMap tk, tv;
-    if (!make_tmap_2d(&tk, tdt, k, d_h, rows, (uint64_t)d_h * eb, 128 / eb, box_rows) ||
-        !make_tmap_2d(&tv, tdt, v, d_h, rows, (uint64_t)d_h * eb, 128 / eb, box_rows))
+    if (!make_tmap_2d(&tk, tdt, k, d_h, rows, (uint64_t)d_h * kvb, 128 / kvb, box_rows) ||
+        !make_tmap_2d(&tv, tdt, v, d_h, rows, (uint64_t)d_h * kvb, 128 / kvb, box_rows))
         return LKA_ERR_CUDA;
 
     GqaParams p;
@@ -248,6 +255,9 @@ static lka_status_t gqa_run(const void* q, const void* k, const void* v, const i
     p.max_pages = pg ? pg->max_pages : 0;
     p.num_pages = pg ? pg->num_pages : 0;
     p.box_rows = (int)box_rows;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    if (fp8kv) return launch_status(gqa_fp8_decode_launch(tk, tv, p, d_h, pl.rb, pl.nsplit, (cudaStream_t)stream));
     return launch_status(gqa_decode_launch(tk, tv, p, eb, d_h, pl.rb, pl.nsplit, (cudaStream_t)stream));
 }
 
@@ -270,6 +280,25 @@ lka_status_t gqa_attn(const void* q, const void* k, const void* v, const int32_t
                       lka_dtype_t dtype, void* ws, size_t ws_bytes, void* stream) {
     return gqa_run(q, k, v, cache_lens, out, lse, B, h_q, h_kv, s_q, d_h, Lmax, causal, scale, dtype, ws, ws_bytes,
                    stream, nullptr);
+}
+
+size_t gqa_attn_fp8kv_workspace_size(int B, int h_q, int h_kv, int s_q, int d_h, int Lmax) {
+    GqaPlan pl;
+    return gqa_plan(B, h_q, h_kv, s_q, d_h, Lmax, 2, &pl, false, true) == LKA_OK ? pl.ws_bytes : 0;
+}
+
+lka_status_t gqa_attn_fp8kv(const void* q, const void* k, const void* v, const float* k_scale, const float* v_scale,
+                            const int32_t* cache_lens, void* out, float* lse, int B, int h_q, int h_kv, int s_q,
+                            int d_h, int Lmax, int causal, float scale, void* ws, size_t ws_bytes, void* stream) {
+    if (B > 0 && (!k_scale || !v_scale || (reinterpret_cast<uintptr_t>(k_scale) & 3u) ||
+                  (reinterpret_cast<uintptr_t>(v_scale) & 3u)))
+        return LKA_ERR_INVALID_ARG;
+    if (B == 0) {
+        GqaPlan pl;
+        return gqa_plan(B, h_q, h_kv, s_q, d_h, Lmax, 2, &pl, false, true);
+    }
+    return gqa_run(q, k, v, cache_lens, out, lse, B, h_q, h_kv, s_q, d_h, Lmax, causal, scale, LKA_BF16, ws, ws_bytes,
+                   stream, nullptr, k_scale, v_scale);
 }
 
 size_t gqa_attn_paged_workspace_size(int B, int h_q, int h_kv, int s_q, int d_h, int page_size, int max_pages) {

@@ -25,6 +25,9 @@
 // sequence needs a single split writes the final output directly; otherwise it
 // writes an fp32 partial (normalised O and log2-domain lse) that
 // gqa_combine_kernel merges.
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
 #include "common.cuh"
 #include "gqa_decode.h"
 #include "host_util.h"
@@ -44,9 +47,16 @@
 
 namespace lka {
 
-template <typename T, int D, int RB>
+// One byte of an e4m3 (fp8) cache value.
+struct e4m3 {
+    uint8_t bits;
+};
+
+// Geometry of an instance: KV is the element type of the K/V cache (bf16, fp32 or e4m3), D the head dim,
+// RB the query rows per CTA.
+template <typename KV, int D, int RB>
 struct GqaCfg {
-    static constexpr int E = sizeof(T);
+    static constexpr int E = sizeof(KV);
     static constexpr int EPC = 16 / E;           // elements per 16-byte chunk
     static constexpr int CPR = D * E / 16;       // chunks per row
     static constexpr int NSEG = D * E / 128;     // 128-byte swizzle segments per row
@@ -67,7 +77,8 @@ struct GqaCfg {
     static constexpr int MAT_BYTES = T_TILE * D * E;
     static constexpr int STAGE_BYTES = 2 * MAT_BYTES;
     static constexpr int NSTAGE0 = (LKA_GQA_STAGE_KB * 1024) / STAGE_BYTES;
-    static constexpr int NSTAGE = NSTAGE0 < 2 ? 2 : (NSTAGE0 > 4 ? 4 : NSTAGE0);
+    static constexpr int NSTAGE_CAP = E == 1 ? 6 : 4;  // the 1-byte cache has half-size stages: keep more
+    static constexpr int NSTAGE = NSTAGE0 < 2 ? 2 : (NSTAGE0 > NSTAGE_CAP ? NSTAGE_CAP : NSTAGE0);
     static constexpr int P_BYTES = 4 * TW * RB * 8 + 4 * RB * 4;  // probabilities (stored as pairs) + rescale
     static constexpr int MERGE_BYTES = 4 * RB * D * 4 + 2 * 4 * RB * 4;
     static constexpr int SMEM = 1024 /*align slack*/ + NSTAGE * STAGE_BYTES + P_BYTES + 256 /*barriers*/;
@@ -136,6 +147,40 @@ __device__ __forceinline__ void load_chunk<float>(const uint8_t* p, float* f) {
     f[3] = w.w;
 }
 
+// Two e4m3 values (the low 16 bits of w) as fp32, exactly (e4m3 -> f16 is exact, f16 -> f32 too).
+__device__ __forceinline__ float2 e4m3x2_to_f32x2(uint32_t w) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w & 0xffffu), __NV_E4M3);
+    return __half22float2(*reinterpret_cast<const __half2*>(&h));
+}
+template <>
+__device__ __forceinline__ void load_chunk<e4m3>(const uint8_t* p, float* f) {
+    const uint4 w = *reinterpret_cast<const uint4*>(p);
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 a = e4m3x2_to_f32x2(ws[i]), b = e4m3x2_to_f32x2(ws[i] >> 16);
+        f[4 * i] = a.x;
+        f[4 * i + 1] = a.y;
+        f[4 * i + 2] = b.x;
+        f[4 * i + 3] = b.y;
+    }
+}
+template <>
+__device__ __forceinline__ void load_v_slice<e4m3, 4>(const uint8_t* p, float* v) {
+    const uint32_t w = *reinterpret_cast<const uint32_t*>(p);
+    const float2 a = e4m3x2_to_f32x2(w), b = e4m3x2_to_f32x2(w >> 16);
+    v[0] = a.x;
+    v[1] = a.y;
+    v[2] = b.x;
+    v[3] = b.y;
+}
+template <>
+__device__ __forceinline__ void load_v_slice<e4m3, 8>(const uint8_t* p, float* v) {
+    const uint2 w = *reinterpret_cast<const uint2*>(p);
+    load_v_slice<e4m3, 4>(reinterpret_cast<const uint8_t*>(&w.x), v);
+    load_v_slice<e4m3, 4>(reinterpret_cast<const uint8_t*>(&w.y), v + 4);
+}
+
 // (segment, chunk) of the c-th chunk owned by lane li of a token's LPT lanes.
 // Chosen so that every 8-lane shared-memory phase of a 16-byte load touches 8
 // distinct bank groups under the 128-byte swizzle.
@@ -169,11 +214,11 @@ __device__ __forceinline__ int paged_row(const GqaParams& p, int b, int kvh, int
     return (page * p.h_kv + kvh) * p.page_size + tok % p.page_size;
 }
 
-template <typename T, int D, int RB>
-__global__ void __launch_bounds__(160, GqaCfg<T, D, RB>::MINB)
+template <typename T, int D, int RB, typename KV>
+__global__ void __launch_bounds__(160, GqaCfg<KV, D, RB>::MINB)
     gqa_decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const GqaParams p) {
-    using C = GqaCfg<T, D, RB>;
+    using C = GqaCfg<KV, D, RB>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
     uint8_t* stages = smem;
@@ -279,6 +324,8 @@ __global__ void __launch_bounds__(160, GqaCfg<T, D, RB>::MINB)
     // query slice of this lane, pre-scaled into the log2 domain
     // the two halves of each pair multiply consecutive key elements (packed fp32x2 FMAs)
     float qreg[RB][C::CPL * C::EPC];
+    // the softmax scale in the log2 domain, and the dequantisation scale of a quantised key cache
+    const float q_mul = p.scale_log2 * (p.k_scale ? p.k_scale[kvh] : 1.f);
     {
         const T* qbase = reinterpret_cast<const T*>(p.q) +
                          ((size_t)(b * p.h_q + kvh * p.ratio) * p.s_q) * D;  // first row of the group
@@ -292,8 +339,7 @@ __global__ void __launch_bounds__(160, GqaCfg<T, D, RB>::MINB)
                 const int e0 = seg * C::SEG_ELEMS + chunk * C::EPC;
 #pragma unroll
                 for (int e = 0; e < C::EPC; ++e)
-                    qreg[r][c * C::EPC + e] =
-                        ok ? to_f32<T>(qbase[(size_t)(row0 + r) * D + e0 + e]) * p.scale_log2 : 0.f;
+                    qreg[r][c * C::EPC + e] = ok ? to_f32<T>(qbase[(size_t)(row0 + r) * D + e0 + e]) * q_mul : 0.f;
             }
         }
     }
@@ -356,7 +402,7 @@ __global__ void __launch_bounds__(160, GqaCfg<T, D, RB>::MINB)
 #pragma unroll
             for (int c = 0; c < C::CPL; ++c) {
                 float kf[C::EPC];
-                load_chunk<T>(kt + koff[ps % NCLS][c] + (ps / NCLS) * NCLS * C::P * 128, kf);
+                load_chunk<KV>(kt + koff[ps % NCLS][c] + (ps / NCLS) * NCLS * C::P * 128, kf);
 #pragma unroll
                 for (int r = 0; r < RB; ++r)
 #pragma unroll
@@ -448,7 +494,7 @@ __global__ void __launch_bounds__(160, GqaCfg<T, D, RB>::MINB)
 #pragma unroll
                 for (int jj = 0; jj < C::TW; ++jj) {
                     float vf[C::DPLV];
-                    load_v_slice<T, C::DPLV>(vt + voff[jj & 7] + (jj & ~7) * 128, vf);
+                    load_v_slice<KV, C::DPLV>(vt + voff[jj & 7] + (jj & ~7) * 128, vf);
                     float2 pj[RB];
                     if constexpr (RB % 2 == 0) {
                         const float4* pr4 = reinterpret_cast<const float4*>(pw + jj * RB);
@@ -473,7 +519,7 @@ __global__ void __launch_bounds__(160, GqaCfg<T, D, RB>::MINB)
                 for (int jj = 0; jj < nvalid; ++jj) {
                     const int jt = warp * C::TW + jj;
                     float vf[C::DPLV];
-                    load_v_slice<T, C::DPLV>(vt + swz_off<C::T_TILE>(v_seg, jt, v_chunk) + v_in, vf);
+                    load_v_slice<KV, C::DPLV>(vt + swz_off<C::T_TILE>(v_seg, jt, v_chunk) + v_in, vf);
                     const float2* pr = pw + jj * RB;
 #pragma unroll
                     for (int r = 0; r < RB; ++r) {
@@ -512,6 +558,7 @@ __global__ void __launch_bounds__(160, GqaCfg<T, D, RB>::MINB)
     }
     named_barrier(1, 128);
 
+    const float v_mul = p.v_scale ? p.v_scale[kvh] : 1.f;  // dequantisation scale of a quantised value cache
     for (int idx = threadIdx.x; idx < rows_here * D; idx += 128) {
         const int r = idx / D, d = idx % D;
         const int gr = row0 + r;
@@ -531,7 +578,7 @@ __global__ void __launch_bounds__(160, GqaCfg<T, D, RB>::MINB)
             lsum += f * lm[w * RB + r];
             acc += f * om[(w * RB + r) * D + d];
         }
-        const float ov = acc / lsum;
+        const float ov = acc / lsum * v_mul;
         const float lse2 = M + log2f(lsum);
         if (nsp == 1) {
             reinterpret_cast<T*>(p.out)[orow * D + d] = from_f32<T>(ov);
@@ -583,11 +630,11 @@ __global__ void __launch_bounds__(128) gqa_combine_kernel(const GqaParams p) {
 }
 
 // ---- host-side dispatch -------------------------------------------------------
-template <typename T, int D, int RB>
+template <typename T, int D, int RB, typename KV = T>
 static cudaError_t launch_one(const CUtensorMap& tk, const CUtensorMap& tv, const GqaParams& p, int nsplit,
                               cudaStream_t st) {
-    using C = GqaCfg<T, D, RB>;
-    auto kern = gqa_decode_kernel<T, D, RB>;
+    using C = GqaCfg<KV, D, RB>;
+    auto kern = gqa_decode_kernel<T, D, RB, KV>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     dim3 grid(nsplit, p.h_kv * p.n_rb, p.B);
@@ -648,6 +695,25 @@ cudaError_t gqa_decode_launch(const CUtensorMap& tk, const CUtensorMap& tv, cons
     LKA_LAUNCH_CASE(float, 64, 8) LKA_LAUNCH_CASE(float, 64, 16)
     LKA_LAUNCH_CASE(float, 128, 1) LKA_LAUNCH_CASE(float, 128, 2) LKA_LAUNCH_CASE(float, 128, 4)
     LKA_LAUNCH_CASE(float, 128, 8) LKA_LAUNCH_CASE(float, 128, 16)
+#undef LKA_LAUNCH_CASE
+    return cudaErrorInvalidValue;
+}
+
+int gqa_fp8_tile_tokens(int d, int rb) {
+#define LKA_TILE_CASE(DD, R) \
+    if (d == DD && rb == R) return GqaCfg<e4m3, DD, R>::T_TILE;
+    LKA_TILE_CASE(128, 1) LKA_TILE_CASE(128, 2) LKA_TILE_CASE(128, 4)
+    LKA_TILE_CASE(256, 1) LKA_TILE_CASE(256, 2) LKA_TILE_CASE(256, 4)
+#undef LKA_TILE_CASE
+    return 0;
+}
+
+cudaError_t gqa_fp8_decode_launch(const CUtensorMap& tk, const CUtensorMap& tv, const GqaParams& p, int d, int rb,
+                                  int nsplit, cudaStream_t st) {
+#define LKA_LAUNCH_CASE(DD, R) \
+    if (d == DD && rb == R) return launch_one<__nv_bfloat16, DD, R, e4m3>(tk, tv, p, nsplit, st);
+    LKA_LAUNCH_CASE(128, 1) LKA_LAUNCH_CASE(128, 2) LKA_LAUNCH_CASE(128, 4)
+    LKA_LAUNCH_CASE(256, 1) LKA_LAUNCH_CASE(256, 2) LKA_LAUNCH_CASE(256, 4)
 #undef LKA_LAUNCH_CASE
     return cudaErrorInvalidValue;
 }

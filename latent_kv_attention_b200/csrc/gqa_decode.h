@@ -24,8 +24,16 @@ struct GqaParams {
     const int32_t* block_table;  // device [B][max_pages] page indices, or nullptr
     int page_size, max_pages, num_pages;
     int box_rows;           // rows per TMA box: min(page_size, tile)
+    // quantised (e4m3) cache: per-KV-head dequantisation scales, device [h_kv] (nullptr otherwise)
+    const float* k_scale;
+    const float* v_scale;
 };
 
+// The e4m3-cache instances (bf16 q/out, d in {128, 256}, rb <= 4: a 16-byte chunk holds 16 values, so more rows
+// per CTA would not fit the query slice in registers).
+int gqa_fp8_tile_tokens(int d, int rb);
+cudaError_t gqa_fp8_decode_launch(const CUtensorMap& tk, const CUtensorMap& tv, const GqaParams& p, int d, int rb,
+                                  int nsplit, cudaStream_t st);
 // Merge of split partials for rows [B*h_q*s_q] of D values (rows needing one split are skipped).
 cudaError_t gqa_combine_launch(const GqaParams& p, int dtype_bytes, int d, cudaStream_t st);
 // Tokens per TMA tile of the kernel instance (0 if the instance does not exist).

@@ -19,6 +19,7 @@ import subprocess
 import threading
 
 import numpy as np
+import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.c")
@@ -230,6 +231,18 @@ def expanded_sparse(q_c, q_r, kc, vc, kr, indices, cache_lens, scale: float):
     rows = [lambda b, keys: kc[b:b + 1][:, :, keys], lambda b, keys: vc[b:b + 1][:, :, keys],
             lambda b, keys: kr[b:b + 1, keys]]
     return _sparse_apply(dense, [q_c, q_r], sel, rows, (B, h_q, s_q, d_h), (B, h_q, s_q))
+
+
+def dequantize_e4m3(x, head_scale):
+    """An e4m3 cache [B, h_kv, L, d] (torch.float8_e4m3fn) widened exactly and multiplied by its per-KV-head
+    scale [h_kv], in float64."""
+    return _f64(x.to(torch.float32)) * _f64(head_scale)[None, :, None, None]
+
+
+def gqa_fp8kv(q, k, v, k_scale, v_scale, cache_lens, causal: bool, scale: float, rows_b=None, n_threads: int = 0):
+    """GQA attention over an e4m3 KV cache with per-KV-head scales: the dequantised cache, then gqa()."""
+    return gqa(q, dequantize_e4m3(k, k_scale), dequantize_e4m3(v, v_scale), cache_lens, causal, scale,
+               rows_b=rows_b, n_threads=n_threads)
 
 
 def gqa_probs(q, k, cache_lens, causal: bool, scale: float, b: int, i: int, t: int, h_kv: int):

@@ -80,6 +80,23 @@ def gqa_inputs(seed, B, h_q, h_kv, d, s_q, L_lo, L_hi, Lmax=None, dtype=torch.bf
     return dict(q=q, k=k, v=v, cache_lens=lens, scale=1.0 / math.sqrt(d))
 
 
+def gqa_fp8_inputs(seed, B, h_q, h_kv, d, s_q, L_lo, L_hi, Lmax=None, device="cpu"):
+    """GQA inputs with an e4m3 K/V cache: q bf16 N(0,1); K, V drawn N(0,1) in fp32 and stored as e4m3 with one
+    scale per KV head (the head's max |value| / 448, so the largest value maps to e4m3's largest); the scales are
+    returned alongside (K = k_scale[h] * k)."""
+    Lmax = L_hi if Lmax is None else Lmax
+    g = _gen(seed, device)
+    lens = _lens(g, B, L_lo, L_hi, device)
+    q = _randn((B, h_q, s_q, d), g, torch.bfloat16, device)
+    out = dict(q=q, cache_lens=lens, scale=1.0 / math.sqrt(d))
+    for name in ("k", "v"):
+        x = torch.randn((B, h_kv, Lmax, d), generator=g, device=device, dtype=torch.float32)
+        sc = x.abs().amax(dim=(0, 2, 3)).clamp_min(1e-12) / 448.0
+        out[name] = (x / sc[None, :, None, None]).to(torch.float8_e4m3fn)
+        out[name + "_scale"] = sc.contiguous()
+    return out
+
+
 def to_pages(caches, lens, page_size, gen, spare_pages=0):
     """Scatters contiguous caches [B, heads, Lmax, width] (e.g. K and V) into shuffled page pools [num_pages, heads,
     page_size, width] sharing one block table [B, Lmax / page_size] (int32): the pages a sequence uses
@@ -217,6 +234,9 @@ WORKLOADS = {
     # the same layer with a quarter of the batch: the small case for full ncu captures (K/V still > L2)
     "gqa_decode_llama8b_b16": dict(kind="gqa", seed=2, B=16, h_q=32, h_kv=8, d=128, s_q=1, L_lo=1024, L_hi=8192,
                                    causal=True),
+    # the same layer with an e4m3 cache (one scale per KV head)
+    "gqa_decode_llama8b_fp8": dict(kind="gqa_fp8", seed=2, B=64, h_q=32, h_kv=8, d=128, s_q=1, L_lo=1024,
+                                   L_hi=8192, causal=True),
     # the same layer over a paged cache: 64-token pages in a shuffled pool, addressed through a block table
     "gqa_decode_llama8b_paged": dict(kind="gqa_paged", seed=2, B=64, h_q=32, h_kv=8, d=128, s_q=1, L_lo=1024,
                                      L_hi=8192, causal=True, page_size=64),
@@ -260,6 +280,9 @@ def make(w: dict, device="cpu", dtype=torch.bfloat16) -> dict:
     if w["kind"] == "gqa":
         return gqa_inputs(w["seed"], w["B"], w["h_q"], w["h_kv"], w["d"], w["s_q"], w["L_lo"], w["L_hi"],
                           dtype=dtype, device=device)
+    if w["kind"] == "gqa_fp8":
+        return gqa_fp8_inputs(w["seed"], w["B"], w["h_q"], w["h_kv"], w["d"], w["s_q"], w["L_lo"], w["L_hi"],
+                              device=device)
     if w["kind"] == "gqa_paged":
         return gqa_paged_inputs(w["seed"], w["B"], w["h_q"], w["h_kv"], w["d"], w["s_q"], w["L_lo"], w["L_hi"],
                                 w["page_size"], dtype=dtype, device=device)

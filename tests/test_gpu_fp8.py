@@ -1,0 +1,54 @@
+"""GPU parity of gqa_attn_fp8kv (GQA over an e4m3 KV cache) against the fp64 oracle (marked gpu)."""
+import pytest
+import torch
+
+import latent_kv_attention_b200 as lka
+import oracle
+import synthetic
+from parity import assert_close, assert_lse_close
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(autouse=True)
+def _clean_status():
+    lka.clear_status()
+    yield
+    assert lka.device_status() == 0, lka.status_string(lka.device_status())
+
+
+CASES = [
+    # (B, h_q, h_kv, d, s_q, L_lo, L_hi, Lmax, causal)
+    (3, 32, 8, 128, 1, 1, 900, 1024, True),    # Llama-3.1-8B heads, ragged, L=1 possible
+    (2, 8, 2, 128, 1, 100, 700, 768, False),   # 4 heads per group, no mask
+    (2, 32, 8, 128, 2, 2, 600, 640, True),     # MTP: 8 rows per group in two row blocks
+    (2, 8, 8, 128, 1, 60, 130, 130, True),     # MHA
+    (2, 16, 2, 256, 1, 50, 400, 512, True),    # d=256, 8 heads per group
+    (1, 16, 1, 128, 3, 3, 70, 80, True),       # MQA, s_q=3
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[f"B{c[0]}h{c[1]}kv{c[2]}d{c[3]}sq{c[4]}" for c in CASES])
+def test_fp8kv(case):
+    B, h_q, h_kv, d, s_q, lo, hi, Lmax, causal = case
+    inp = synthetic.gqa_fp8_inputs(700 + B * h_q + d + s_q, B, h_q, h_kv, d, s_q, lo, hi, Lmax=Lmax)
+    dd = {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    out, lse = lka.gqa_attn_fp8kv(dd["q"], dd["k"], dd["v"], dd["k_scale"], dd["v_scale"], dd["cache_lens"],
+                                  causal=causal, scale=inp["scale"], return_lse=True)
+    ref, ref_lse = oracle.gqa_fp8kv(inp["q"], inp["k"], inp["v"], inp["k_scale"], inp["v_scale"], inp["cache_lens"],
+                                    causal, inp["scale"])
+    assert_close(out, ref, torch.bfloat16, "fp8kv out")
+    assert_lse_close(lse, ref_lse, torch.bfloat16, "fp8kv lse")
+
+
+def test_fp8kv_matches_bf16_path_on_the_dequantised_cache():
+    """The same attention through gqa_attn on the dequantised cache (rounded to bf16) agrees within bf16 noise."""
+    inp = synthetic.gqa_fp8_inputs(790, 4, 32, 8, 128, 1, 500, 2000, Lmax=2048)
+    dd = {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    a = lka.gqa_attn_fp8kv(dd["q"], dd["k"], dd["v"], dd["k_scale"], dd["v_scale"], dd["cache_lens"],
+                           scale=inp["scale"])
+    k16 = (dd["k"].float() * dd["k_scale"][None, :, None, None]).to(torch.bfloat16)
+    v16 = (dd["v"].float() * dd["v_scale"][None, :, None, None]).to(torch.bfloat16)
+    b = lka.gqa_attn(dd["q"], k16, v16, dd["cache_lens"], scale=inp["scale"])
+    assert (a.float() - b.float()).abs().max().item() <= 2e-2

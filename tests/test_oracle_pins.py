@@ -403,3 +403,20 @@ def test_sparse_oracle_empty_selection():
     out, lse = oracle.latent_absorbed_sparse(inp["q_c"], inp["q_r"], inp["w_uk"], inp["w_uv"], inp["latent"], idx,
                                              inp["cache_lens"], inp["scale"])
     assert np.all(out == 0) and np.all(np.isneginf(lse))
+
+
+# ------------------------------------------------------------------ FP8 (e4m3) KV cache ----------------------
+def test_e4m3_decoding_and_fp8_oracle():
+    """The e4m3 widening the fp8 oracle uses (torch's float8_e4m3fn: 1 sign, 4 exponent bits with bias 7,
+    3 mantissa bits, no infinities) on codes whose values the format fixes, and the per-KV-head scaling."""
+    codes = torch.tensor([0x38, 0x40, 0x01, 0x08, 0x7E, 0xB8, 0x00, 0x3C], dtype=torch.uint8)
+    vals = codes.view(torch.float8_e4m3fn).to(torch.float64).tolist()
+    assert vals == [1.0, 2.0, 2.0 ** -9, 2.0 ** -6, 448.0, -1.0, 0.0, 1.5]
+    inp = synthetic.gqa_fp8_inputs(81, 2, 8, 2, 128, 1, 5, 40)
+    k = inp["k"].to(torch.float64) * inp["k_scale"].double()[None, :, None, None]
+    v = inp["v"].to(torch.float64) * inp["v_scale"].double()[None, :, None, None]
+    assert inp["k_scale"][0] != inp["k_scale"][1]
+    ref, ref_lse = oracle.gqa(inp["q"], k, v, inp["cache_lens"], True, inp["scale"])
+    out, lse = oracle.gqa_fp8kv(inp["q"], inp["k"], inp["v"], inp["k_scale"], inp["v_scale"], inp["cache_lens"], True,
+                                inp["scale"])
+    assert np.array_equal(out, ref) and np.array_equal(lse, ref_lse)
