@@ -503,6 +503,45 @@ class GtaPrefill(Workload):
         return fn, nbytes, oracle.threads_used(0, n * w["H"]), f"first {n} of {w['B']} sequences"
 
 
+class GtaChunkedPrefillPaged(GtaPrefill):
+    """gta_shared_score_attn_paged: a 1024-token prefill chunk per sequence against 4096 cached tokens held in
+    64-token pages of a shuffled pool (bottom-right causal)."""
+
+    def setup_device(self):
+        super().setup_device()
+        for k in ("k_g", "v"):  # the contiguous copies are not used by the paged step
+            self.inp.pop(k, None)
+        torch.cuda.empty_cache()
+        i = self.inp
+        self.h2d_pairs = [(i[k], _pinned(i[k])) for k in ("q_g", "k_pages", "v_pages", "block_table", "cache_lens")]
+
+    def step(self):
+        i = self.inp
+        self.lka.gta_shared_score_attn_paged(i["q_g"], i["k_pages"], i["v_pages"], i["block_table"], i["cache_lens"],
+                                             causal=self.w["causal"], scale=i["scale"], out=self.out)
+
+    def config(self):
+        c = super().config()
+        c["page_size"] = self.w["page_size"]
+        c["cache_layout"] = "paged (shuffled page pool + block table)"
+        c["l2"] = "inputs ~105 MB; L2 flushed between timed steps"
+        return c
+
+    def oracle_run(self, n):
+        import oracle
+
+        i = self.inp
+        w = self.w
+        sub = {k: i[k][:n].cpu() for k in ("q_g", "block_table", "cache_lens")}
+        kp, vp = i["k_pages"].cpu(), i["v_pages"].cpu()
+        fn = lambda: oracle.gta_paged(sub["q_g"], kp, vp, sub["block_table"], sub["cache_lens"], w["causal"],  # noqa: E731
+                                      i["scale"])
+        lens = sub["cache_lens"].tolist()
+        nbytes = costs.gta_bytes(lens, w["G"], w["H"], w["d_qk"], w["d_v"], w["s_q"])
+        self.oracle_flops = costs.gta_flops(lens, w["G"], w["H"], w["d_qk"], w["d_v"], w["s_q"], w["causal"])
+        return fn, nbytes, oracle.threads_used(0, n * w["H"]), f"first {n} of {w['B']} sequences"
+
+
 GqaDecode.kernel_work = lambda self, pk: ("hbm", self.bytes)
 
 WORKLOAD_CLASSES = {
@@ -517,13 +556,15 @@ WORKLOAD_CLASSES = {
     "latent_expanded_4k_sq1": LatentExpanded,
     "latent_expanded_4k_sq2": LatentExpanded,
     "gta_prefill_4k": GtaPrefill,
+    "gta_chunked_prefill_4k_paged": GtaChunkedPrefillPaged,
     # smaller cases for full ncu captures
     "latent_decode_4k_sq1_b32": LatentAbsorbed,
     "latent_expanded_4k_sq2_b16": LatentExpanded,
     "gta_prefill_4k_b2": GtaPrefill,
 }
 EXTRAS = ["gqa_decode_llama8b_paged", "gqa_decode_llama8b_fp8", "latent_decode_4k_sq1", "latent_decode_4k_sq1_paged", "latent_decode_4k_sq2",
-          "latent_sparse_16k_top2048", "latent_expanded_4k_sq2", "gta_prefill_4k"]
+          "latent_sparse_16k_top2048", "latent_expanded_4k_sq2", "gta_prefill_4k",
+          "gta_chunked_prefill_4k_paged"]
 
 
 def oracle_sample(wl, target_s: float):

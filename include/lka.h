@@ -254,6 +254,24 @@ LKA_API lka_status_t gta_shared_score_attn(const void *q_g, const void *k_g, con
                                    int Lmax, int causal, float scale, lka_dtype_t dtype, void *ws, size_t ws_bytes,
                                    void *stream);
 
+/* (d') The same over paged caches (chunked prefill against a paged cache)
+ *  [GQA "GQA compared with related techniques" (PagedAttention); GQLA sec. 2
+ *  (paged KV caches)].
+ *   k_pages [num_pages, G, page_size, d_qk]   v_pages [num_pages, H, page_size, d_v]
+ *   block_table [B, max_pages] int32 (device): token t of sequence b is row
+ *   t % page_size of page block_table[b][t / page_size] in both pools.
+ *  page_size a power of two >= 8; capacity max_pages * page_size per sequence
+ *  (cache_lens entries above it are clamped, raising LKA_ERR_BAD_LENGTH); table
+ *  entries a call needs that are outside [0, num_pages) are replaced by page 0
+ *  and raise LKA_ERR_BAD_PAGE.  Other arguments and results as in (d). */
+LKA_API size_t gta_shared_score_attn_paged_workspace_size(int B, int G, int H, int s_q, int d_qk, int d_v,
+                                                          int page_size, int max_pages);
+LKA_API lka_status_t gta_shared_score_attn_paged(const void *q_g, const void *k_pages, const void *v_pages,
+                                         const int32_t *block_table, const int32_t *cache_lens, void *out,
+                                         float *lse, int B, int G, int H, int s_q, int d_qk, int d_v, int page_size,
+                                         int max_pages, int num_pages, int causal, float scale, lka_dtype_t dtype,
+                                         void *ws, size_t ws_bytes, void *stream);
+
 /* ------------------------------------------------------------------------ */
 /* One-time cache conversion latent -> per-group expanded cache             */
 /* [GQLA sec. 3.1: switching paths needs a one-time compression/expansion   */

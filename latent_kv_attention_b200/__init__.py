@@ -14,6 +14,7 @@ Entry points (same names as the C ABI):
   latent_absorbed_attn     GQLA MQA-absorbed latent path (GQLA paper, sec. 3.1, Figure 2(b))
   latent_expand_gqa_attn   GQLA per-group GQA path       (GQLA paper, sec. 3.1, Figure 2(a))
   gta_shared_score_attn    GTA shared score per group    (GTA article, grouped shared attention matrix)
+  gta_shared_score_attn_paged  the same over paged K/V pools (chunked prefill against a paged cache)
   latent_expand_cache      one-time latent -> expanded cache conversion (GQLA paper, sec. 3.1)
 """
 from __future__ import annotations
@@ -60,6 +61,8 @@ SIGNATURES = {
     "latent_expand_gqa_attn_paged": (_I, [_P] * 9 + [_I] * 10 + [_F, _I, _P, _Z, _P]),
     "gta_shared_score_attn_workspace_size": (_Z, [_I] * 7),
     "gta_shared_score_attn": (_I, [_P] * 6 + [_I] * 8 + [_F, _I, _P, _Z, _P]),
+    "gta_shared_score_attn_paged_workspace_size": (_Z, [_I] * 8),
+    "gta_shared_score_attn_paged": (_I, [_P] * 7 + [_I] * 10 + [_F, _I, _P, _Z, _P]),
     "latent_expand_cache": (_I, [_P] * 3 + [_I] * 6 + [_P] * 3 + [_I, _P]),
     "lka_device_status": (_I, [_P, _P]),
     "lka_clear_status": (_I, [_P, _P]),
@@ -427,6 +430,38 @@ def gta_shared_score_attn(q_g, k_g, v, cache_lens, causal: bool = True, scale: f
                                    s_q, d_qk, d_v, Lmax, int(bool(causal)), scale, _dtype_code(q_g), _ptr(ws),
                                    ws.numel(), _stream_ptr())
     _check("gta_shared_score_attn", rc)
+    return (out, lse) if return_lse else out
+
+
+def gta_shared_score_attn_paged(q_g, k_pages, v_pages, block_table, cache_lens, causal: bool = True,
+                                scale: float | None = None, out=None, return_lse: bool = False):
+    """GTA shared-score attention over paged caches. q_g [B,G,s_q,d_qk]; k_pages [num_pages,G,page_size,d_qk];
+    v_pages [num_pages,H,page_size,d_v]; block_table int32 [B,max_pages] (token t of sequence b: row
+    t % page_size of page block_table[b, t // page_size] in both pools). Returns out [B,H,s_q,d_v]."""
+    for n, t in (("q_g", q_g), ("k_pages", k_pages), ("v_pages", v_pages)):
+        _device_tensor(t, n, q_g.dtype)
+    _require(q_g.dim() == 4 and k_pages.dim() == 4 and v_pages.dim() == 4,
+             "q_g [B,G,s_q,d_qk], k_pages [num_pages,G,page_size,d_qk], v_pages [num_pages,H,page_size,d_v]")
+    B, G, s_q, d_qk = q_g.shape
+    num_pages, H, page_size, d_v = v_pages.shape
+    _require(k_pages.shape == (num_pages, G, page_size, d_qk), "k_pages must be [num_pages,G,page_size,d_qk]")
+    _device_tensor(block_table, "block_table", torch.int32)
+    _require(block_table.dim() == 2 and block_table.shape[0] == B and block_table.device == q_g.device,
+             "block_table must be int32 [B, max_pages] on q_g's device")
+    max_pages = block_table.shape[1]
+    _lens_tensor(cache_lens, B, q_g.device)
+    scale = 1.0 / math.sqrt(d_qk) if scale is None else float(scale)
+    out = torch.empty((B, H, s_q, d_v), dtype=q_g.dtype, device=q_g.device) if out is None else out
+    lse = torch.empty((B, G, s_q), dtype=torch.float32, device=q_g.device) if return_lse else None
+    lib = library()
+    nbytes = lib.gta_shared_score_attn_paged_workspace_size(B, G, H, s_q, d_qk, d_v, page_size, max_pages)
+    _require(nbytes > 0, "page_size must be a power of two >= 8")
+    ws = workspaces.get(nbytes, q_g.device)
+    rc = lib.gta_shared_score_attn_paged(_ptr(q_g), _ptr(k_pages), _ptr(v_pages), _ptr(block_table),
+                                         _ptr(cache_lens), _ptr(out), _ptr(lse), B, G, H, s_q, d_qk, d_v, page_size,
+                                         max_pages, num_pages, int(bool(causal)), scale, _dtype_code(q_g), _ptr(ws),
+                                         ws.numel(), _stream_ptr())
+    _check("gta_shared_score_attn_paged", rc)
     return (out, lse) if return_lse else out
 
 

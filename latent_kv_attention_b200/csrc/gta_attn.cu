@@ -37,6 +37,10 @@ struct GtaParams {
     uint32_t* status;
     int B, G, H, s_q, Lmax, causal;
     float scale_log2;
+    // paged caches (block_table == nullptr: contiguous [B][heads][Lmax] slabs)
+    const int32_t* block_table;  // [B, max_pages]
+    int page_size, max_pages, num_pages;
+    int box_rows;                // rows per TMA box: min(128, page_size), or 128 when contiguous
 };
 
 namespace gta {
@@ -128,12 +132,30 @@ __global__ void __launch_bounds__(gta::NTHREADS, 1)
             tma_load_2d(smem_u32(smem + OFF_Q), &tm_q, 0, (b * p.G + grp) * p.s_q + q0, qb);
             int k_issued = 0, v_issued = 0;
             bool ok = true;
+            // row of token `tok` of head `head` (of `heads`) of this sequence: contiguous [B][heads][Lmax], or
+            // row tok % page_size of that head's block in page block_table[b][tok / page_size]; an entry outside
+            // the pool is replaced by page 0, which is reported when the tile's queries need the token
+            auto cache_row = [&](int tok, int heads, int head) -> int {
+                if (!p.block_table) return (b * heads + head) * p.Lmax + tok;
+                int page = 0;
+                const int jp = tok / p.page_size;
+                if (jp < p.max_pages) {
+                    page = p.block_table[(size_t)b * p.max_pages + jp];
+                    if (page < 0 || page >= p.num_pages) {
+                        if (tok < key_end) atomicOr(p.status, kDevBadPage);
+                        page = 0;
+                    }
+                }
+                return (page * heads + head) * p.page_size + tok % p.page_size;
+            };
             auto issue_k = [&](int i) {
                 const int s = i % NSK;
                 if (i >= NSK && !mbar_wait(smem_u32(&k_empty[s]), ((i / NSK) - 1) & 1, p.status)) return false;
                 const uint32_t fb = smem_u32(&k_full[s]);
                 mbar_arrive_expect_tx(fb, BOX);
-                tma_load_2d(smem_u32(smem + OFF_K + s * BOX), &tm_k, 0, (b * p.G + grp) * p.Lmax + i * TK, fb);
+                for (int r0 = 0; r0 < TK; r0 += p.box_rows)  // one box, or one per page piece of the tile
+                    tma_load_2d(smem_u32(smem + OFF_K + s * BOX) + r0 * 128, &tm_k, 0, cache_row(i * TK + r0, p.G, grp),
+                                fb);
                 ++k_issued;
                 return true;
             };
@@ -144,7 +166,8 @@ __global__ void __launch_bounds__(gta::NTHREADS, 1)
                 mbar_arrive_expect_tx(fb, HPG * BOX);
                 const uint32_t d = smem_u32(smem + OFF_V + s * VSTAGE);
                 for (int hh = 0; hh < HPG; ++hh)
-                    tma_load_2d(d + hh * BOX, &tm_v, 0, (b * p.H + grp * HPG + hh) * p.Lmax + i * TK, fb);
+                    for (int r0 = 0; r0 < TK; r0 += p.box_rows)
+                        tma_load_2d(d + hh * BOX + r0 * 128, &tm_v, 0, cache_row(i * TK + r0, p.H, grp * HPG + hh), fb);
                 ++v_issued;
                 return true;
             };
@@ -360,26 +383,42 @@ size_t gta_shared_score_attn_workspace_size(int B, int G, int H, int s_q, int d_
     return kWsHeaderBytes;  // status word only: one CTA covers the whole key range of its query tile
 }
 
-lka_status_t gta_shared_score_attn(const void* q_g, const void* k_g, const void* v, const int32_t* cache_lens,
-                                   void* out, float* lse, int B, int G, int H, int s_q, int d_qk, int d_v, int Lmax,
-                                   int causal, float scale, lka_dtype_t dtype, void* ws, size_t ws_bytes,
-                                   void* stream) {
+}  // extern "C"
+
+namespace {
+
+struct GtaPages {
+    const int32_t* block_table;
+    int page_size, max_pages, num_pages;
+};
+
+// Validates the arguments and launches the kernel.  Contiguous caches: pg == nullptr, k_g [B,G,Lmax,64],
+// v [B,H,Lmax,64].  Paged: k_g [num_pages,G,page_size,64], v [num_pages,H,page_size,64], and Lmax is the
+// capacity max_pages * page_size.
+lka_status_t gta_run(const void* q_g, const void* k_g, const void* v, const int32_t* cache_lens, void* out,
+                     float* lse, int B, int G, int H, int s_q, int d_qk, int d_v, int Lmax, int causal, float scale,
+                     lka_dtype_t dtype, void* ws, size_t ws_bytes, void* stream, const GtaPages* pg) {
     if (B < 0 || G < 1 || H < 1 || s_q < 1 || Lmax < 1 || d_qk < 1 || d_v < 1) return LKA_ERR_INVALID_ARG;
     if (H % G) return LKA_ERR_INVALID_ARG;
     if (dtype != LKA_BF16 || d_qk != 64 || d_v != 64 || H / G > 4) return LKA_ERR_UNSUPPORTED;
     if ((long long)B * H * Lmax >= (1ll << 31) || (long long)B * G * s_q >= (1ll << 31) || B > 65535 || G > 65535)
         return LKA_ERR_UNSUPPORTED;
+    if (pg && (long long)pg->num_pages * H * pg->page_size >= (1ll << 31)) return LKA_ERR_UNSUPPORTED;
     if (B == 0) return LKA_OK;
     const void* ptrs[] = {q_g, k_g, v, cache_lens, out};
     for (const void* ptr : ptrs)
         if (!ptr || !aligned16(ptr)) return LKA_ERR_INVALID_ARG;
+    if (pg && !pg->block_table) return LKA_ERR_INVALID_ARG;
     if (!isfinite(scale)) return LKA_ERR_INVALID_ARG;
     if (!ws || ws_bytes < kWsHeaderBytes) return LKA_ERR_WORKSPACE;
     const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const int box_rows = pg ? std::min(gta::TK, pg->page_size) : gta::TK;
+    const uint64_t k_rows = pg ? (uint64_t)pg->num_pages * G * pg->page_size : (uint64_t)B * G * Lmax;
+    const uint64_t v_rows = pg ? (uint64_t)pg->num_pages * H * pg->page_size : (uint64_t)B * H * Lmax;
     CUtensorMap tq, tk, tv;
     if (!make_tmap_2d(&tq, BF, q_g, 64, (uint64_t)B * G * s_q, 128, 64, 128) ||
-        !make_tmap_2d(&tk, BF, k_g, 64, (uint64_t)B * G * Lmax, 128, 64, 128) ||
-        !make_tmap_2d(&tv, BF, v, 64, (uint64_t)B * H * Lmax, 128, 64, 128))
+        !make_tmap_2d(&tk, BF, k_g, 64, k_rows, 128, 64, box_rows) ||
+        !make_tmap_2d(&tv, BF, v, 64, v_rows, 128, 64, box_rows))
         return LKA_ERR_CUDA;
     GtaParams p{};
     p.lens = cache_lens;
@@ -393,6 +432,13 @@ lka_status_t gta_shared_score_attn(const void* q_g, const void* k_g, const void*
     p.Lmax = Lmax;
     p.causal = causal ? 1 : 0;
     p.scale_log2 = scale * 1.4426950408889634f;
+    p.box_rows = box_rows;
+    if (pg) {
+        p.block_table = pg->block_table;
+        p.page_size = pg->page_size;
+        p.max_pages = pg->max_pages;
+        p.num_pages = pg->num_pages;
+    }
     cudaStream_t st = (cudaStream_t)stream;
     if (cudaFuncSetAttribute(gta_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gta::SMEM) != cudaSuccess)
         return LKA_ERR_CUDA;
@@ -401,6 +447,40 @@ lka_status_t gta_shared_score_attn(const void* q_g, const void* k_g, const void*
     gta_attn_kernel<<<grid, gta::NTHREADS, gta::SMEM, st>>>(tq, tk, tv, p);
     timer.stop();
     return cudaPeekAtLastError() == cudaSuccess ? LKA_OK : LKA_ERR_CUDA;
+}
+
+bool gta_pages_ok(int page_size, int max_pages, int num_pages) {
+    return page_size >= 8 && (page_size & (page_size - 1)) == 0 && max_pages >= 1 && num_pages >= 1 &&
+           (long long)max_pages * page_size < (1ll << 31);
+}
+
+}  // namespace
+
+extern "C" {
+
+lka_status_t gta_shared_score_attn(const void* q_g, const void* k_g, const void* v, const int32_t* cache_lens,
+                                   void* out, float* lse, int B, int G, int H, int s_q, int d_qk, int d_v, int Lmax,
+                                   int causal, float scale, lka_dtype_t dtype, void* ws, size_t ws_bytes,
+                                   void* stream) {
+    return gta_run(q_g, k_g, v, cache_lens, out, lse, B, G, H, s_q, d_qk, d_v, Lmax, causal, scale, dtype, ws,
+                   ws_bytes, stream, nullptr);
+}
+
+size_t gta_shared_score_attn_paged_workspace_size(int B, int G, int H, int s_q, int d_qk, int d_v, int page_size,
+                                                  int max_pages) {
+    if (!gta_pages_ok(page_size, max_pages, 1)) return 0;
+    return gta_shared_score_attn_workspace_size(B, G, H, s_q, d_qk, d_v, page_size * max_pages);
+}
+
+lka_status_t gta_shared_score_attn_paged(const void* q_g, const void* k_pages, const void* v_pages,
+                                         const int32_t* block_table, const int32_t* cache_lens, void* out,
+                                         float* lse, int B, int G, int H, int s_q, int d_qk, int d_v, int page_size,
+                                         int max_pages, int num_pages, int causal, float scale, lka_dtype_t dtype,
+                                         void* ws, size_t ws_bytes, void* stream) {
+    if (!gta_pages_ok(page_size, max_pages, num_pages)) return LKA_ERR_INVALID_ARG;
+    const GtaPages pg{block_table, page_size, max_pages, num_pages};
+    return gta_run(q_g, k_pages, v_pages, cache_lens, out, lse, B, G, H, s_q, d_qk, d_v, page_size * max_pages,
+                   causal, scale, dtype, ws, ws_bytes, stream, &pg);
 }
 
 }  // extern "C"

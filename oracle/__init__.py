@@ -157,6 +157,17 @@ def gqa_paged(q, k_pages, v_pages, block_table, cache_lens, causal: bool, scale:
     return gqa(q, k, v, cache_lens, causal, scale, rows_b=rows_b, n_threads=n_threads)
 
 
+def gta_paged(q_g, k_pages, v_pages, block_table, cache_lens, causal: bool, scale: float, n_threads: int = 0):
+    """GTA shared-score attention over paged caches (k_pages [num_pages, G, page_size, d_qk], v_pages [num_pages,
+    H, page_size, d_v], one block table): the contiguous caches the block table describes, then gta()."""
+    bt = _i32(block_table)
+    ps = int(np.asarray(k_pages.shape)[2])
+    Lmax = bt.shape[1] * ps
+    k_g = paged_to_contiguous(k_pages, bt, Lmax)
+    v = paged_to_contiguous(v_pages, bt, Lmax)
+    return gta(q_g, k_g, v, cache_lens, causal, scale, n_threads=n_threads)
+
+
 def latent_absorbed_paged(q_c, q_r, w_uk, w_uv, latent_pages, block_table, cache_lens, causal: bool, scale: float,
                           rows_b=None, n_threads: int = 0):
     """The MQA-absorbed latent attention over a paged latent cache [num_pages, page_size, r_kv + d_r]: the

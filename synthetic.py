@@ -135,6 +135,19 @@ def gqa_paged_inputs(seed, B, h_q, h_kv, d, s_q, L_lo, L_hi, page_size, Lmax=Non
     return inp
 
 
+def gta_paged_inputs(seed, B, G, H, d_qk, d_v, s_q, L_lo, L_hi, page_size, Lmax=None, dtype=torch.bfloat16,
+                     device="cpu", spare_pages=3):
+    """GTA inputs (as gta_inputs) with k_g and v moved into shuffled page pools sharing one block table; the
+    capacity is rounded up to whole pages."""
+    Lmax = L_hi if Lmax is None else Lmax
+    Lmax = -(-Lmax // page_size) * page_size
+    inp = gta_inputs(seed, B, G, H, d_qk, d_v, s_q, L_lo, L_hi, Lmax=Lmax, dtype=dtype, device=device)
+    g = _gen(seed + 7919, device)
+    (k_pages, v_pages), table = to_pages([inp["k_g"], inp["v"]], inp["cache_lens"], page_size, g, spare_pages)
+    inp.update(k_pages=k_pages, v_pages=v_pages, block_table=table, page_size=page_size)
+    return inp
+
+
 def latent_paged_inputs(seed, B, h_q, g_groups, d_h, r_kv, d_r, s_q, L_lo, L_hi, page_size, Lmax=None,
                         dtype=torch.bfloat16, device="cpu", spare_pages=3):
     """GQLA latent inputs (as latent_inputs) with the latent cache moved into a shuffled page pool
@@ -257,6 +270,10 @@ WORKLOADS = {
                                      L_lo=4096, L_hi=4096, causal=True),
     "latent_expanded_4k_sq2_b16": dict(kind="latent", seed=4, B=16, h_q=128, g=8, d_h=128, r_kv=512, d_r=64, s_q=2,
                                        L_lo=4096, L_hi=4096, causal=True),
+    # chunked prefill against a paged cache: the last 1024 tokens of each 4096-token sequence as queries, the
+    # keys/values in 64-token pages of a shuffled pool
+    "gta_chunked_prefill_4k_paged": dict(kind="gta_paged", seed=3, B=8, G=3, H=12, d_qk=64, d_v=64, s_q=1024,
+                                         L_lo=4096, L_hi=4096, causal=True, page_size=64),
     "gta_prefill_4k_b2": dict(kind="gta", seed=3, B=2, G=3, H=12, d_qk=64, d_v=64, s_q=4096, L_lo=4096, L_hi=4096,
                               causal=True),
     # the same latent inputs, run through the per-group GQA path after the one-time cache expansion
@@ -297,6 +314,9 @@ def make(w: dict, device="cpu", dtype=torch.bfloat16) -> dict:
     if w["kind"] == "latent":
         return latent_inputs(w["seed"], w["B"], w["h_q"], w["g"], w["d_h"], w["r_kv"], w["d_r"], w["s_q"],
                              w["L_lo"], w["L_hi"], dtype=dtype, device=device)
+    if w["kind"] == "gta_paged":
+        return gta_paged_inputs(w["seed"], w["B"], w["G"], w["H"], w["d_qk"], w["d_v"], w["s_q"], w["L_lo"],
+                                w["L_hi"], w["page_size"], dtype=dtype, device=device)
     if w["kind"] == "gta":
         return gta_inputs(w["seed"], w["B"], w["G"], w["H"], w["d_qk"], w["d_v"], w["s_q"], w["L_lo"], w["L_hi"],
                           dtype=dtype, device=device)

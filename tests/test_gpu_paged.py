@@ -1,4 +1,4 @@
-"""GPU parity of gqa_attn_paged (GQA over a paged KV cache) against the fp64 oracle (marked gpu)."""
+"""GPU parity of the paged-cache entry points (GQA, both GQLA paths, GTA) against the fp64 oracle (marked gpu)."""
 import pytest
 import torch
 
@@ -101,3 +101,30 @@ def test_expanded_paged(page_size, s_q):
     cont = lka.latent_expand_gqa_attn(d["q_c"], d["q_r"], d["kc"], d["vc"], d["kr"], d["cache_lens"], causal=True,
                                       scale=inp["scale"])
     assert torch.equal(out, cont)
+
+
+@pytest.mark.parametrize("page_size,s_q", [(16, 200), (64, 1), (128, 130), (256, 5)])
+def test_gta_paged(page_size, s_q):
+    """Chunked GTA prefill against a paged cache: s_q new queries over a ragged cached prefix (bottom-right
+    causal), two query tiles at s_q = 200, ragged last page and last key tile."""
+    inp = synthetic.gta_paged_inputs(600 + page_size + s_q, 3, 3, 12, 64, 64, s_q, s_q + 17, 470, page_size,
+                                     Lmax=512)
+    d = {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    out, lse = lka.gta_shared_score_attn_paged(d["q_g"], d["k_pages"], d["v_pages"], d["block_table"],
+                                               d["cache_lens"], causal=True, scale=inp["scale"], return_lse=True)
+    ref, ref_lse = oracle.gta_paged(inp["q_g"], inp["k_pages"], inp["v_pages"], inp["block_table"], inp["cache_lens"],
+                                    True, inp["scale"])
+    assert_close(out, ref, torch.bfloat16, "gta paged out")
+    assert_lse_close(lse, ref_lse, torch.bfloat16, "gta paged lse")
+    cont = lka.gta_shared_score_attn(d["q_g"], d["k_g"], d["v"], d["cache_lens"], causal=True, scale=inp["scale"])
+    assert torch.equal(out, cont)
+
+
+def test_gta_paged_out_of_pool_entry_is_replaced_and_reported():
+    inp = synthetic.gta_paged_inputs(650, 2, 2, 4, 64, 64, 4, 100, 120, 32, Lmax=128)
+    d = {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    bt = d["block_table"].clone()
+    bt[0, 1] = -3  # a page the first sequence needs, outside the pool
+    lka.gta_shared_score_attn_paged(d["q_g"], d["k_pages"], d["v_pages"], bt, d["cache_lens"], scale=inp["scale"])
+    assert lka.device_status() == 7  # LKA_ERR_BAD_PAGE
+    lka.clear_status()

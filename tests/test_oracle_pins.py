@@ -369,6 +369,16 @@ def test_latent_paged_oracle_equals_contiguous():
     assert np.array_equal(out, ref)
 
 
+def test_gta_paged_oracle_equals_contiguous():
+    """GTA over shuffled K/V page pools with one block table equals GTA over the contiguous caches."""
+    inp = synthetic.gta_paged_inputs(65, 2, 2, 6, 16, 8, 3, 5, 37, 8, dtype=torch.float32)
+    ref, ref_lse = oracle.gta(inp["q_g"], inp["k_g"], inp["v"], inp["cache_lens"], True, inp["scale"])
+    out, lse = oracle.gta_paged(inp["q_g"], inp["k_pages"], inp["v_pages"], inp["block_table"], inp["cache_lens"],
+                                True, inp["scale"])
+    assert np.array_equal(out, ref) and np.array_equal(lse, ref_lse)
+    assert (inp["block_table"] >= 0).sum() < inp["k_pages"].shape[0]  # spare pages: the pool is not the table
+
+
 # ------------------------------------------------------------------ top-k sparse attention ------------------
 def test_sparse_oracle_full_selection_equals_dense_causal():
     """Selecting every key a query may see (in a shuffled order) is the dense causal attention ("GQLA ..."
