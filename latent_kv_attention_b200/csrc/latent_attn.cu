@@ -26,19 +26,21 @@
 // query slice lives in tensor memory (the A operand of the score MMA), which
 // leaves shared memory to a 4-stage TMA ring, one exchange buffer and an
 // outbox: a partial is written to the outbox and sent with one bulk copy per
-// warp (the copy engine moves it; the warp does not wait for the transfer).
-// The softmax warps fetch and send the partial of tile i+1 before they work on
-// tile i, and the score MMA runs two tiles ahead of P*V, so the exchange is
-// off the per-tile critical path.
+// block (the copy engine moves it; the warp does not wait for the transfer).
+// Sender warps load each partial from tensor memory as soon as it is computed
+// and send it; the softmax warps load their own copy of tile i+1 before they
+// work on tile i, and the score MMA runs two tiles ahead of P*V, so the
+// exchange overlaps the softmax of the previous tile.
 //
 // Per CTA: warp 8 streams 64-token tiles of the latent through the ring; warp 9
 // issues the MMAs (S = Q K^T into the TMEM score tile, O += P V with P read
-// from TMEM); warps 0-7 write the query slice to TMEM once, then per tile
-// exchange, mask and run the online softmax, two warps per group of 32 head
-// rows (warps w and w + 4 take the two 32-token halves of the tile and swap
-// their row maxima through two spare TMEM columns), with lazy rescaling (the
-// running maximum is only moved when it grows by more than 2^8, which leaves
-// the final O / l exact); P is written back to TMEM as bf16.
+// from TMEM); warps 10-13 (one per TMEM lane quarter) send the score partials;
+// warps 0-7 write the query slice to TMEM once, then per tile add the peer's
+// partial to their own, mask and run the online softmax, two warps per group
+// of 32 head rows (warps w and w + 4 take the two 32-token halves of the tile
+// and swap their row maxima through two spare TMEM columns), with lazy
+// rescaling (the running maximum is only moved when it grows by more than 2^8,
+// which leaves the final O / l exact); P is written back to TMEM as bf16.
 #include "common.cuh"
 #include "host_util.h"
 #include "latent.h"
@@ -55,8 +57,9 @@ constexpr int KSTEPS = 18;      // K = 16 steps of this rank's 288 score values
 constexpr int BOX = NT * 128;   // one 64-value box of NT tokens
 constexpr int STAGE = NKB * BOX;
 constexpr int NSW = 8;          // softmax warps: 4 lane quarters x 2 column halves
+constexpr int NXW = 4;          // sender warps: one per lane quarter
 constexpr int CW = NT / 2;      // score columns per softmax warp
-constexpr int NTHREADS = 32 * (NSW + 2);
+constexpr int NTHREADS = 32 * (NSW + 2 + NXW);
 constexpr int XROW = CW * 4;    // bytes of one row of one half of an exchanged partial
 constexpr int XBUF = 2 * 128 * XROW;  // [half][head row][CW] fp32; each warp's block is contiguous
 constexpr int OFF_KV = 0;
@@ -120,7 +123,8 @@ __device__ __forceinline__ void remote_arrive(uint32_t rbar) {
 // peer's "buffer free" arrival (release at cluster scope) is only ever followed by new remote
 // stores, never by reads of data the peer produced.
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(lat::NTHREADS, 1)
+// 14 warps: an SM sub-partition holds up to 4 of them, so at most 16384 / (4 * 32) = 128 registers each
+__global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
     latent_attn_kernel(const __grid_constant__ CUtensorMap tm_lat, const LatentParams p) {
     using namespace lat;
     extern __shared__ uint8_t smem_raw[];
@@ -130,7 +134,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(lat::NTHREADS, 1)
     uint64_t* kv_full = bars + 1;
     uint64_t* kv_empty = kv_full + NST;
     uint64_t* s_ready = kv_empty + NST;   // QK(j) done
-    uint64_t* s_free = s_ready + 1;       // S(j) loaded by all softmax warps
+    uint64_t* s_free = s_ready + 1;       // S(j) loaded by all softmax and sender warps
     uint64_t* p_ready = s_free + 1;       // P(j) written by all softmax warps
     uint64_t* o_ready = p_ready + 1;      // PV(j) done
     uint64_t* xfull = o_ready + 1;        // [NSW] the peer's partial of warp w's block arrived
@@ -161,7 +165,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(lat::NTHREADS, 1)
             mbar_init(smem_u32(&kv_empty[s]), 1);
         }
         mbar_init(smem_u32(s_ready), 1);
-        mbar_init(smem_u32(s_free), NSW);
+        mbar_init(smem_u32(s_free), NSW + NXW);
         mbar_init(smem_u32(p_ready), NSW);
         mbar_init(smem_u32(o_ready), 1);
         for (int i = 0; i < NSW; ++i) {
@@ -234,8 +238,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(lat::NTHREADS, 1)
         }
     } else if (n_tiles > 0 && warp == NSW + 1) {
         // ------------------------------- MMA issuer -------------------------------
-        // Per step j: QK(j) once the softmax warps have loaded S(j-1), then PV(j-2) once P(j-2)
-        // is in tensor memory.  The softmax warps load S(j-1) before they compute P(j-2), so
+        // Per step j: QK(j) once the softmax and sender warps have loaded S(j-1), then PV(j-2) once
+        // P(j-2) is in tensor memory.  The softmax warps load S(j-1) before they compute P(j-2), so
         // QK(j) runs while tile j-2 is being finished.
         constexpr uint32_t idesc_qk = idesc_bf16_f32(128, NT, false, false);
         constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
@@ -289,8 +293,63 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(lat::NTHREADS, 1)
                 __syncwarp();
             }
         }
+    } else if (n_tiles > 0 && warp >= NSW + 2) {
+        // ------------------------------- sender warps -------------------------------
+        // Sender warp q (= warp % 4) owns TMEM lane quarter q (head rows 32q .. +31): per tile it loads
+        // this rank's partial scores of all NT columns from tensor memory, writes them to the outbox and
+        // sends the two 32-column blocks of the quarter to the peer's exchange buffer once the peer's
+        // softmax warps have consumed the previous tile there.  The softmax warps only wait for what
+        // the peer sent; the sending (outbox store, proxy fence, waits, copies) is off their path.
+        const int qx = warp & 3;
+        const uint32_t lane_base = (uint32_t)(qx * 32) << 16;
+        const int sw = lane & 7;
+        int xblk[2];
+        uint32_t xrem[2], xfull_rem[2];
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            xblk[hf] = hf * 128 * XROW + qx * 32 * XROW;  // the block of softmax warp 4 hf + q
+            xrem[hf] = mapa_peer(smem_u32(smem + OFF_X + xblk[hf]), peer);
+            xfull_rem[hf] = mapa_peer(smem_u32(&xfull[hf * 4 + qx]), peer);
+        }
+        uint32_t own[NT];
+        bool ok = true;
+        for (int j = 0; ok && j < n_tiles; ++j) {
+            ok = mbar_wait(smem_u32(s_ready), j & 1, p.status);
+            tc_fence_after();
+#pragma unroll
+            for (int c0 = 0; c0 < NT; c0 += 16) tmem_ld16(tmem + lane_base + T_S + c0, own + c0);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(s_free));
+            if (lane == 0) bulk_wait_read();  // the previous copies have read the outbox
+            __syncwarp();
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                uint8_t* orow = smem + OFF_OUT + xblk[hf] + lane * XROW;
+#pragma unroll
+                for (int c = 0; c < CW / 4; ++c)
+                    *reinterpret_cast<uint4*>(orow + ((c ^ sw) << 4)) =
+                        make_uint4(own[hf * CW + 4 * c], own[hf * CW + 4 * c + 1], own[hf * CW + 4 * c + 2],
+                                   own[hf * CW + 4 * c + 3]);
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the copy engine
+            __syncwarp();
+            if (lane == 0) {
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    // the peer's block is free once its softmax warp has consumed partial j-1
+                    if (ok && j >= 1) ok = mbar_wait(smem_u32(&xempty[hf * 4 + qx]), (j - 1) & 1, p.status);
+                    if (ok) bulk_copy_to_peer(xrem[hf], smem_u32(smem + OFF_OUT + xblk[hf]), 32 * XROW, xfull_rem[hf]);
+                }
+                bulk_commit();
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+        }
+        if (lane == 0) bulk_wait_all();
+        if (!ok) s_abort = 1;
     } else if (warp < NSW) {
-        // ------------------------- softmax / exchange warps -------------------------
+        // -------------------------------- softmax warps --------------------------------
         // Warp w owns head rows 32(w%4) .. +31 (its TMEM lane quarter) and score columns
         // [32(w/4), +32) of every tile, with its own exchange barriers; the two warps of a lane
         // quarter meet once per tile to combine their row maxima.
@@ -299,11 +358,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(lat::NTHREADS, 1)
         const uint32_t lane_base = (uint32_t)(qw * 32) << 16;
         const int col0 = half * CW;
         const int blk = half * 128 * XROW + qw * 32 * XROW;  // this warp's block in the exchange buffer
-        // the peer's exchange block and barriers of this warp
-        const uint32_t xrem = mapa_peer(smem_u32(smem + OFF_X + blk), peer);
-        const uint32_t xfull_rem = mapa_peer(smem_u32(&xfull[warp]), peer);
+        // the peer's "buffer free" barrier of this warp's block
         const uint32_t xempty_rem = mapa_peer(smem_u32(&xempty[warp]), peer);
-        uint8_t* outrow = smem + OFF_OUT + blk + lane * XROW;
         const int sw = lane & 7;
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
@@ -333,8 +389,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(lat::NTHREADS, 1)
             if (lane == 0) mbar_arrive(smem_u32(q_full));
         }
         uint32_t cur[CW];
-        // this warp's block of the partial of tile j: registers, release the TMEM tile, send it
-        auto fetch_and_send = [&](int j) {
+        // this warp's block of this rank's partial of tile j into registers (the sender warps send it)
+        auto fetch = [&](int j) {
             if (ok) ok = mbar_wait(smem_u32(s_ready), j & 1, p.status);
             tc_fence_after();
             tmem_ld16(tmem + lane_base + T_S + col0, cur);
@@ -343,22 +399,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(lat::NTHREADS, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(s_free));
-            // the outbox block of this warp is free once the previous bulk copy has read it
-            if (lane == 0) bulk_wait_read();
-            __syncwarp();
-#pragma unroll
-            for (int c = 0; c < CW / 4; ++c)
-                *reinterpret_cast<uint4*>(outrow + ((c ^ sw) << 4)) =
-                    make_uint4(cur[4 * c], cur[4 * c + 1], cur[4 * c + 2], cur[4 * c + 3]);
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the copy engine
-            __syncwarp();
-            if (lane == 0) {
-                // the peer's buffer is free once it has consumed partial j-1
-                if (ok && j >= 1) ok = mbar_wait(smem_u32(&xempty[warp]), (j - 1) & 1, p.status);
-                if (ok) bulk_copy_to_peer(xrem, smem_u32(smem + OFF_OUT + blk), 32 * XROW, xfull_rem);
-                bulk_commit();
-            }
-            ok = __shfl_sync(0xffffffffu, ok, 0);
         };
         // combine a per-row value with the partner warp's through TMEM column T_R + col (+ 1 for
         // the partner's); both warps of the lane quarter call it with the same col
@@ -372,7 +412,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(lat::NTHREADS, 1)
             tmem_ld_wait();
             return __uint_as_float(o);
         };
-        if (n_tiles > 0) fetch_and_send(0);
+        if (n_tiles > 0) fetch(0);
         for (int i = 0; i < n_tiles; ++i) {
             // ---- the peer's partial of this block, added to this rank's ----
             if (ok) ok = mbar_wait(smem_u32(&xfull[warp]), i & 1, p.status);
@@ -395,8 +435,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(lat::NTHREADS, 1)
                 mbar_arrive_expect_tx(smem_u32(&xfull[warp]), XBUF / NSW);  // reopen for tile i + 1 ...
                 remote_arrive(xempty_rem);                                   // ... and tell the peer
             }
-            // ---- tile i+1 goes out before tile i is finished ----
-            if (i + 1 < n_tiles) fetch_and_send(i + 1);
+            // ---- this rank's partial of tile i+1 (the score MMA may move on to tile i+2) ----
+            if (i + 1 < n_tiles) fetch(i + 1);
             // ---- mask, online softmax ----
             const int k0 = kbeg + i * NT + col0;
             const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
@@ -458,7 +498,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(lat::NTHREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(p_ready));
         }
-        if (lane == 0) bulk_wait_all();
         if (!ok) s_abort = 1;
         // ---- epilogue: the full row sum, then normalise this warp's 128 output columns ----
         l += swap_with_partner(l, 4u);
