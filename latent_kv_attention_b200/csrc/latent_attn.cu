@@ -66,6 +66,12 @@ constexpr int OFF_KV = 0;
 constexpr int OFF_X = OFF_KV + NST * STAGE;
 constexpr int OFF_OUT = OFF_X + XBUF;  // this CTA's partial on its way to the peer
 constexpr int OFF_BAR = OFF_OUT + XBUF;
+// The query slice is staged once through shared memory that is idle at the start: the last ring
+// stage, the exchange buffer and the first part of the outbox (five 128-row x 64-value boxes).
+constexpr int NQB = 5;
+constexpr int QBOX = 128 * 128;
+constexpr int OFF_QST = OFF_KV + (NST - 1) * STAGE;
+static_assert(OFF_QST % 1024 == 0 && OFF_QST + NQB * QBOX <= OFF_BAR, "query staging area");
 constexpr int SMEM = 1024 + OFF_BAR + 512;
 static_assert(SMEM <= 232448, "shared memory budget");
 // tensor memory columns
@@ -125,13 +131,15 @@ __device__ __forceinline__ void remote_arrive(uint32_t rbar) {
 
 // 14 warps: an SM sub-partition holds up to 4 of them, so at most 16384 / (4 * 32) = 128 registers each
 __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
-    latent_attn_kernel(const __grid_constant__ CUtensorMap tm_lat, const LatentParams p) {
+    latent_attn_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant__ CUtensorMap tm_qt,
+                       const __grid_constant__ CUtensorMap tm_qr, const LatentParams p) {
     using namespace lat;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
     uint64_t* q_full = bars + 0;          // the query slice is in tensor memory (all softmax warps arrived)
-    uint64_t* kv_full = bars + 1;
+    uint64_t* q_loaded = bars + 1;        // the query slice is in shared memory
+    uint64_t* kv_full = bars + 2;
     uint64_t* kv_empty = kv_full + NST;
     uint64_t* s_ready = kv_empty + NST;   // QK(j) done
     uint64_t* s_free = s_ready + 1;       // S(j) loaded by all softmax and sender warps
@@ -160,6 +168,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
     if (threadIdx.x == 0) {
         s_abort = 0;
         mbar_init(smem_u32(q_full), NSW);
+        mbar_init(smem_u32(q_loaded), 1);
         for (int s = 0; s < NST; ++s) {
             mbar_init(smem_u32(&kv_full[s]), 1);
             mbar_init(smem_u32(&kv_empty[s]), 1);
@@ -189,6 +198,17 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
         // ------------------------------- TMA producer -------------------------------
         if (lane == 0) {
             prefetch_tensormap(&tm_lat);
+            // this rank's 288 values of the 128 query rows [q~ ; q^R] of (b, t): rank 0 q~[0:320) (the
+            // last 32 unused), rank 1 q~[288:544) (the last 32 past the row: zero fill) and q^R[0:64)
+            {
+                const uint32_t qb = smem_u32(q_loaded);
+                mbar_arrive_expect_tx(qb, NQB * QBOX);
+                const int qrow = (b * p.s_q + t) * 128;
+                const uint32_t qdst = smem_u32(smem + OFF_QST);
+                for (int k = 0; k < (rank ? NQB - 1 : NQB); ++k)
+                    tma_load_2d(qdst + k * QBOX, &tm_qt, (int)rank * 288 + k * 64, qrow, qb);
+                if (rank) tma_load_3d(qdst + (NQB - 1) * QBOX, &tm_qr, 0, t, b * 128, qb);
+            }
             // tiles PF ahead of the one being loaded are prefetched into L2, so that the ring (whose
             // stages stay busy until P*V) is refilled from L2 rather than from DRAM
             // row of token `tok` of this sequence in the cache: contiguous [B][Lmax] slabs, or a page of the
@@ -222,6 +242,11 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
                     break;
                 }
                 if (*(volatile int*)&s_abort) break;
+                // the last stage holds part of the staged query until it is in tensor memory
+                if (i == NST - 1 && !mbar_wait(smem_u32(q_full), 0, p.status)) {
+                    s_abort = 1;
+                    break;
+                }
                 const uint32_t fb = smem_u32(&kv_full[s]);
                 mbar_arrive_expect_tx(fb, NKB * BOX);
                 const uint32_t dst = smem_u32(smem + OFF_KV + s * STAGE);
@@ -312,7 +337,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
             xfull_rem[hf] = mapa_peer(smem_u32(&xfull[hf * 4 + qx]), peer);
         }
         uint32_t own[NT];
-        bool ok = true;
+        bool ok = mbar_wait(smem_u32(q_full), 0, p.status);  // the outbox holds part of the staged query
         for (int j = 0; ok && j < n_tiles; ++j) {
             ok = mbar_wait(smem_u32(s_ready), j & 1, p.status);
             tc_fence_after();
@@ -338,8 +363,9 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
             if (lane == 0) {
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
-                    // the peer's block is free once its softmax warp has consumed partial j-1
-                    if (ok && j >= 1) ok = mbar_wait(smem_u32(&xempty[hf * 4 + qx]), (j - 1) & 1, p.status);
+                    // the peer's block is free once its softmax warps are done with the staged query
+                    // (phase 0) and its softmax warp has consumed partial j-1 (phase j)
+                    if (ok) ok = mbar_wait(smem_u32(&xempty[hf * 4 + qx]), j & 1, p.status);
                     if (ok) bulk_copy_to_peer(xrem[hf], smem_u32(smem + OFF_OUT + xblk[hf]), 32 * XROW, xfull_rem[hf]);
                 }
                 bulk_commit();
@@ -364,18 +390,19 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
         if (n_tiles > 0) {
-            // this rank's 288 values of the query row [q~_h ; q^R_h] -> tensor memory (A operand of the
-            // score MMA, K-major: column c holds values 2c and 2c+1): rank 0 q~[0:288), rank 1
-            // q~[288:512) followed by q^R.  Nine 16-column chunks: the first warp of the lane
-            // quarter writes chunks 0-4, the second 5-8.
-            const uint4* qt = reinterpret_cast<const uint4*>(p.q_t + ((size_t)(b * p.s_q + t) * p.h_q + h) * 512);
-            const uint4* qr = reinterpret_cast<const uint4*>(p.q_r + (((size_t)b * p.h_q + h) * p.s_q + t) * 64);
+            // this rank's 288 values of query row h, staged in shared memory -> tensor memory (A operand
+            // of the score MMA, K-major: column c holds values 2c and 2c+1).  Nine 16-column chunks of
+            // 32 values: the first warp of the lane quarter writes chunks 0-4, the second 5-8.
+            if (ok) ok = mbar_wait(smem_u32(q_loaded), 0, p.status);
             for (int c0 = half * 5; c0 < (half ? KSTEPS / 2 : 5); ++c0) {
+                const int v0 = c0 * 32;  // first value of the chunk within this rank's slice
+                const bool rope = rank == 1 && v0 >= 224;
+                const int box = rope ? NQB - 1 : v0 / 64, u0 = rope ? (v0 - 224) / 8 : (v0 % 64) / 8;
+                const uint8_t* row = smem + OFF_QST + box * QBOX + h * 128;
                 uint32_t w[16];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const int d = (int)rank * 288 + (c0 * 4 + q) * 8;  // first of these 8 values
-                    const uint4 v = d < 512 ? qt[d / 8] : qr[(d - 512) / 8];
+                    const uint4 v = *reinterpret_cast<const uint4*>(row + (((u0 + q) ^ (h & 7)) << 4));
                     w[4 * q] = v.x;
                     w[4 * q + 1] = v.y;
                     w[4 * q + 2] = v.z;
@@ -387,6 +414,10 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(q_full));
+            // the staging area overlaps the exchange buffer: once every softmax warp of this CTA is done
+            // with it, the peer may send its first partial (phase 0 of the buffer-free barrier)
+            if (ok) ok = mbar_wait(smem_u32(q_full), 0, p.status);
+            if (lane == 0) remote_arrive(xempty_rem);
         }
         uint32_t cur[CW];
         // this warp's block of this rank's partial of tile j into registers (the sender warps send it)
@@ -511,24 +542,31 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
             __nv_bfloat16* orow =
                 p.o_lat + ((size_t)grp * p.B * HPG * p.s_q + (size_t)(b * HPG + hh) * p.s_q + t) * 512 + rank * 256;
             float* prt = p.nsplit > 1 ? p.part_o + (prow * p.nsplit + split) * 512 + rank * 256 : nullptr;
-            for (int c0 = half * 128; c0 < half * 128 + 128; c0 += 16) {
-                uint32_t o[16];
-                tmem_ld16(tmem + lane_base + T_O + c0, o);
+            for (int c1 = half * 128; c1 < half * 128 + 128; c1 += 32) {
+                uint32_t o2[32];  // two 16-column loads per wait
+                tmem_ld16(tmem + lane_base + T_O + c1, o2);
+                tmem_ld16(tmem + lane_base + T_O + c1 + 16, o2 + 16);
                 tmem_ld_wait();
-                if (prt) {
-                    float4* d = reinterpret_cast<float4*>(prt + c0);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        d[q] = make_float4(__uint_as_float(o[4 * q]) * inv_l, __uint_as_float(o[4 * q + 1]) * inv_l,
-                                           __uint_as_float(o[4 * q + 2]) * inv_l, __uint_as_float(o[4 * q + 3]) * inv_l);
-                } else {
-                    uint32_t pkk[8];
+                for (int u = 0; u < 2; ++u) {
+                    const int c0 = c1 + 16 * u;
+                    const uint32_t* o = o2 + 16 * u;
+                    if (prt) {
+                        float4* d = reinterpret_cast<float4*>(prt + c0);
 #pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        pkk[q] = pack_bf16x2(__uint_as_float(o[2 * q]) * inv_l, __uint_as_float(o[2 * q + 1]) * inv_l);
-                    uint4* d = reinterpret_cast<uint4*>(orow + c0);
-                    d[0] = make_uint4(pkk[0], pkk[1], pkk[2], pkk[3]);
-                    d[1] = make_uint4(pkk[4], pkk[5], pkk[6], pkk[7]);
+                        for (int q = 0; q < 4; ++q)
+                            d[q] = make_float4(__uint_as_float(o[4 * q]) * inv_l, __uint_as_float(o[4 * q + 1]) * inv_l,
+                                               __uint_as_float(o[4 * q + 2]) * inv_l,
+                                               __uint_as_float(o[4 * q + 3]) * inv_l);
+                    } else {
+                        uint32_t pkk[8];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            pkk[q] = pack_bf16x2(__uint_as_float(o[2 * q]) * inv_l, __uint_as_float(o[2 * q + 1]) * inv_l);
+                        uint4* d = reinterpret_cast<uint4*>(orow + c0);
+                        d[0] = make_uint4(pkk[0], pkk[1], pkk[2], pkk[3]);
+                        d[1] = make_uint4(pkk[4], pkk[5], pkk[6], pkk[7]);
+                    }
                 }
             }
             if (rank == 0 && half == 0) {
@@ -600,12 +638,23 @@ __global__ void __launch_bounds__(128) latent_combine_kernel(const LatentParams 
 int latent_tile_tokens() { return lat::NT; }
 
 cudaError_t latent_attn_launch(const CUtensorMap& tm_lat, const LatentParams& p, cudaStream_t st) {
+    // the query slices: q~ [B*s_q*h_q][512] and q^R [B][h_q][s_q][64], 128 rows of 64 values per box
+    CUtensorMap tm_qt, tm_qr;
+    const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    if (!make_tmap_2d(&tm_qt, BF, p.q_t, 512, (uint64_t)p.B * p.s_q * p.h_q, 1024, 64, 128))
+        return cudaErrorInvalidValue;
+    {
+        const uint64_t dims[3] = {64, (uint64_t)p.s_q, (uint64_t)p.B * p.h_q};
+        const uint64_t strides[2] = {128, (uint64_t)p.s_q * 128};
+        const uint32_t box[3] = {64, 1, 128};
+        if (!make_tmap_nd(&tm_qr, BF, p.q_r, 3, dims, strides, box)) return cudaErrorInvalidValue;
+    }
     cudaError_t e = cudaFuncSetAttribute(latent_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, lat::SMEM);
     if (e != cudaSuccess) return e;
     dim3 grid(2 * p.s_q * p.nsplit, p.B);
     {
         TimedLaunch timer(st);
-        latent_attn_kernel<<<grid, lat::NTHREADS, lat::SMEM, st>>>(tm_lat, p);
+        latent_attn_kernel<<<grid, lat::NTHREADS, lat::SMEM, st>>>(tm_lat, tm_qt, tm_qr, p);
         timer.stop();
     }
     e = cudaPeekAtLastError();
