@@ -351,6 +351,47 @@ class LatentAbsorbed(Workload):
         return fn, nbytes, oracle.threads_used(0, n * w["h_q"]), f"first {n} of {w['B']} sequences"
 
 
+class LatentAbsorbedFp8(LatentAbsorbed):
+    """latent_absorbed_attn_fp8kv over the same decode batch with the latent cache in e4m3 (one scale for the
+    latent part, one for the RoPE key)."""
+
+    def setup_costs(self):
+        super().setup_costs()
+        w = self.w
+        self.bytes = costs.latent_bytes(self.lens, w["h_q"], w["g"], w["d_h"], w["r_kv"], w["d_r"], w["s_q"],
+                                        cache_elem=1)
+
+    def kernel_work(self, pk):
+        cache = sum(self.lens) * (self.w["r_kv"] + self.w["d_r"])
+        t_mem = cache / (pk["hbm_gbs"] * 1e9)
+        t_tc = self.core_flops / (pk["bf16_tflops"] * 1e12)  # f16 tensor-core rate = bf16 rate
+        return ("tensor", self.core_flops) if t_tc > t_mem else ("hbm", cache)
+
+    def step(self):
+        i = self.inp
+        self.lka.latent_absorbed_attn_fp8kv(i["q_c"], i["q_r"], i["w_uk"], i["w_uv"], i["latent8"], i["kv_scale"],
+                                            i["cache_lens"], causal=self.w["causal"], scale=i["scale"], out=self.out)
+
+    def config(self):
+        c = super().config()
+        c["cache_dtype"] = "e4m3 (per-part scales)"
+        return c
+
+    def oracle_run(self, n):
+        import oracle
+
+        i = self.inp
+        sub = {k: (v[:n].cpu() if k in ("q_c", "q_r", "latent8") else v) for k, v in i.items()}
+        lens = i["cache_lens"][:n].cpu()
+        w_uk, w_uv, sc = i["w_uk"].cpu(), i["w_uv"].cpu(), i["kv_scale"].cpu()
+        w = self.w
+        fn = lambda: oracle.latent_absorbed_fp8kv(sub["q_c"], sub["q_r"], w_uk, w_uv, sub["latent8"], sc,  # noqa: E731
+                                                  lens, w["causal"], i["scale"])
+        nbytes = costs.latent_bytes(lens.tolist(), w["h_q"], w["g"], w["d_h"], w["r_kv"], w["d_r"], w["s_q"],
+                                    cache_elem=1)
+        return fn, nbytes, oracle.threads_used(0, n * w["h_q"]), f"first {n} of {w['B']} sequences"
+
+
 class LatentAbsorbedPaged(LatentAbsorbed):
     """latent_absorbed_attn_paged over the s_q = 1 batch with the latent cache in 64-token pages of a shuffled pool."""
 
@@ -552,6 +593,7 @@ WORKLOAD_CLASSES = {
     "latent_decode_4k_sq1": LatentAbsorbed,
     "latent_decode_4k_sq2": LatentAbsorbed,
     "latent_decode_4k_sq1_paged": LatentAbsorbedPaged,
+    "latent_decode_4k_sq1_fp8": LatentAbsorbedFp8,
     "latent_sparse_16k_top2048": LatentSparse,
     "latent_expanded_4k_sq1": LatentExpanded,
     "latent_expanded_4k_sq2": LatentExpanded,
@@ -562,7 +604,8 @@ WORKLOAD_CLASSES = {
     "latent_expanded_4k_sq2_b16": LatentExpanded,
     "gta_prefill_4k_b2": GtaPrefill,
 }
-EXTRAS = ["gqa_decode_llama8b_paged", "gqa_decode_llama8b_fp8", "latent_decode_4k_sq1", "latent_decode_4k_sq1_paged", "latent_decode_4k_sq2",
+EXTRAS = ["gqa_decode_llama8b_paged", "gqa_decode_llama8b_fp8", "latent_decode_4k_sq1", "latent_decode_4k_sq1_paged",
+          "latent_decode_4k_sq1_fp8", "latent_decode_4k_sq2",
           "latent_sparse_16k_top2048", "latent_expanded_4k_sq2", "gta_prefill_4k",
           "gta_chunked_prefill_4k_paged"]
 

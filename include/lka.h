@@ -180,6 +180,25 @@ LKA_API lka_status_t latent_absorbed_attn_paged(const void *q_c, const void *q_r
                                         int num_pages, int causal, float scale, lka_dtype_t dtype, void *ws,
                                         size_t ws_bytes, void *stream);
 
+/* (b'') The same over an FP8 (e4m3) latent cache  [GQLA sec. 2: quantised KV
+ *  storage is a complementary system technique that lowers the bytes per
+ *  cached token].  latent [B, Lmax, r_kv + d_r] holds e4m3 bytes (576 per token,
+ *  half the bf16 cache) with two fp32 dequantisation scales (device [2]):
+ *    c^KV[b,t,:] = kv_scale[0] * latent[b,t,0:r_kv]
+ *    k^R[b,t,:]  = kv_scale[1] * latent[b,t,r_kv:r_kv+d_r]
+ *  q_c, q_r, w_uk, w_uv, out stay bf16; other arguments, results and shape
+ *  limits as in (b); contiguous cache only.  The e4m3 values are widened
+ *  exactly (to f16) in shared memory; the scales are applied in fp32 to the
+ *  query and to the latent-space output (the query and P enter the tensor
+ *  cores as f16). */
+LKA_API size_t latent_absorbed_attn_fp8kv_workspace_size(int B, int h_q, int g, int s_q, int d_h, int r_kv, int d_r,
+                                                         int Lmax);
+LKA_API lka_status_t latent_absorbed_attn_fp8kv(const void *q_c, const void *q_r, const void *w_uk,
+                                        const void *w_uv, const void *latent, const float *kv_scale,
+                                        const int32_t *cache_lens, void *out, float *lse, int B, int h_q, int g,
+                                        int s_q, int d_h, int r_kv, int d_r, int Lmax, int causal, float scale,
+                                        void *ws, size_t ws_bytes, void *stream);
+
 /* ------------------------------------------------------------------------ */
 /* (c) GQLA GQA path over the per-group expanded cache  [GQLA sec. 1,       */
 /*     sec. 3.1, Figure 2(a)]                                               */

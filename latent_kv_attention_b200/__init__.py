@@ -11,8 +11,11 @@ raised.
 Entry points (same names as the C ABI):
   gqa_attn                 GQA decode / prefill          ("Grouped Query Attention (GQA)" glossary page)
   gqa_attn_paged           the same over a paged KV cache (glossary page: PagedAttention comparison)
+  gqa_attn_fp8kv           the same over an e4m3 KV cache with per-KV-head scales (GQLA paper, sec. 2)
   latent_absorbed_attn     GQLA MQA-absorbed latent path (GQLA paper, sec. 3.1, Figure 2(b))
+  latent_absorbed_attn_paged / _fp8kv / _sparse   ... over a paged, an e4m3, or a top-k selected latent cache
   latent_expand_gqa_attn   GQLA per-group GQA path       (GQLA paper, sec. 3.1, Figure 2(a))
+  latent_expand_gqa_attn_paged / _sparse           ... over paged or top-k selected expanded caches
   gta_shared_score_attn    GTA shared score per group    (GTA article, grouped shared attention matrix)
   gta_shared_score_attn_paged  the same over paged K/V pools (chunked prefill against a paged cache)
   latent_expand_cache      one-time latent -> expanded cache conversion (GQLA paper, sec. 3.1)
@@ -49,6 +52,8 @@ SIGNATURES = {
     "gqa_attn_paged": (_I, [_P] * 7 + [_I] * 9 + [_F, _I, _P, _Z, _P]),
     "latent_absorbed_attn_workspace_size": (_Z, [_I] * 8),
     "latent_absorbed_attn": (_I, [_P] * 8 + [_I] * 9 + [_F, _I, _P, _Z, _P]),
+    "latent_absorbed_attn_fp8kv_workspace_size": (_Z, [_I] * 8),
+    "latent_absorbed_attn_fp8kv": (_I, [_P] * 9 + [_I] * 9 + [_F, _P, _Z, _P]),
     "latent_absorbed_attn_paged_workspace_size": (_Z, [_I] * 9),
     "latent_absorbed_attn_paged": (_I, [_P] * 9 + [_I] * 11 + [_F, _I, _P, _Z, _P]),
     "latent_expand_gqa_attn_workspace_size": (_Z, [_I] * 7),
@@ -268,6 +273,36 @@ def latent_absorbed_attn(q_c, q_r, w_uk, w_uv, latent, cache_lens, causal: bool 
                                   _ptr(out), _ptr(lse), B, h_q, g, s_q, d_h, r_kv, d_r, Lmax, int(bool(causal)),
                                   scale, _dtype_code(q_c), _ptr(ws), ws.numel(), _stream_ptr())
     _check("latent_absorbed_attn", rc)
+    return (out, lse) if return_lse else out
+
+
+def latent_absorbed_attn_fp8kv(q_c, q_r, w_uk, w_uv, latent, kv_scale, cache_lens, causal: bool = True,
+                               scale: float | None = None, out=None, return_lse: bool = False):
+    """GQLA MQA-absorbed path over an e4m3 latent cache: latent [B,Lmax,r_kv+d_r] torch.float8_e4m3fn with
+    kv_scale fp32 [2] (c^KV = kv_scale[0] * latent[..., :r_kv], k^R = kv_scale[1] * latent[..., r_kv:]);
+    q_c, q_r, w_uk, w_uv bf16 as in latent_absorbed_attn. Returns out [B,h_q,s_q,d_h] bf16."""
+    for n, t in (("q_c", q_c), ("q_r", q_r), ("w_uk", w_uk), ("w_uv", w_uv)):
+        _device_tensor(t, n, torch.bfloat16)
+    _device_tensor(latent, "latent", torch.float8_e4m3fn)
+    _device_tensor(kv_scale, "kv_scale", torch.float32)
+    _require(kv_scale.numel() == 2, "kv_scale must hold 2 values (latent part, RoPE key)")
+    B, h_q, s_q, d_h = q_c.shape
+    d_r = q_r.shape[-1]
+    g, _, r_kv = w_uk.shape
+    Lmax = latent.shape[1]
+    _require(q_r.shape[:3] == (B, h_q, s_q) and w_uv.shape == w_uk.shape and w_uk.shape[1] == d_h, "shape mismatch")
+    _require(latent.shape == (B, Lmax, r_kv + d_r), "latent must be [B,Lmax,r_kv+d_r]")
+    _lens_tensor(cache_lens, B, q_c.device)
+    scale = 1.0 / math.sqrt(d_h + d_r) if scale is None else float(scale)
+    out = torch.empty_like(q_c) if out is None else out
+    lse = torch.empty((B, h_q, s_q), dtype=torch.float32, device=q_c.device) if return_lse else None
+    lib = library()
+    nbytes = lib.latent_absorbed_attn_fp8kv_workspace_size(B, h_q, g, s_q, d_h, r_kv, d_r, Lmax)
+    ws = workspaces.get(nbytes, q_c.device)
+    rc = lib.latent_absorbed_attn_fp8kv(_ptr(q_c), _ptr(q_r), _ptr(w_uk), _ptr(w_uv), _ptr(latent), _ptr(kv_scale),
+                                        _ptr(cache_lens), _ptr(out), _ptr(lse), B, h_q, g, s_q, d_h, r_kv, d_r, Lmax,
+                                        int(bool(causal)), scale, _ptr(ws), ws.numel(), _stream_ptr())
+    _check("latent_absorbed_attn_fp8kv", rc)
     return (out, lse) if return_lse else out
 
 

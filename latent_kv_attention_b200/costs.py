@@ -53,8 +53,9 @@ def gqa_flops(lens: Sequence[int], h_q: int, d: int, s_q: int, causal: bool) -> 
 
 
 def latent_bytes(lens: Sequence[int], h_q: int, g: int, d_h: int, r_kv: int, d_r: int, s_q: int,
-                 elem: int = 2) -> int:
-    cache = sum(int(L) for L in lens) * (r_kv + d_r) * elem
+                 elem: int = 2, cache_elem: int | None = None) -> int:
+    """Latent cache read once (cache_elem bytes per value, default elem), both weights, q read, out written."""
+    cache = sum(int(L) for L in lens) * (r_kv + d_r) * (elem if cache_elem is None else cache_elem)
     weights = 2 * g * d_h * r_kv * elem
     q = len(lens) * h_q * s_q * (d_h + d_r) * elem
     out = len(lens) * h_q * s_q * d_h * elem

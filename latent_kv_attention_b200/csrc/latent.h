@@ -38,6 +38,9 @@ struct LatentParams {
     const int32_t* block_table;  // device [B][max_pages] page indices, or nullptr
     int page_size, max_pages, num_pages;
     int box_rows;                // rows per TMA box: min(page_size, tile)
+    // FP8 (e4m3) latent cache: dequantisation scales of the latent part and of the RoPE key (device [2]), or
+    // nullptr for a bf16 cache
+    const float* kv_scale;
 };
 
 cudaError_t latent_attn_launch(const CUtensorMap& tm_lat, const LatentParams& p, cudaStream_t st);

@@ -92,8 +92,12 @@ struct LatentPages {
 static lka_status_t latent_run(const void* q_c, const void* q_r, const void* w_uk, const void* w_uv,
                                const void* latent, const int32_t* cache_lens, void* out, float* lse, int B, int h_q,
                                int g, int s_q, int d_h, int r_kv, int d_r, int Lmax, int causal, float scale,
-                               lka_dtype_t dtype, void* ws, size_t ws_bytes, void* stream, const LatentPages* pg) {
+                               lka_dtype_t dtype, void* ws, size_t ws_bytes, void* stream, const LatentPages* pg,
+                               const float* kv_scale = nullptr) {
+    // kv_scale != nullptr: the latent cache holds e4m3 bytes (query and output stay bf16)
     if (dtype != LKA_BF16) return LKA_ERR_UNSUPPORTED;
+    if (kv_scale && pg) return LKA_ERR_UNSUPPORTED;  // an FP8 cache is contiguous
+    if (kv_scale && ((uintptr_t)kv_scale & 3)) return LKA_ERR_INVALID_ARG;
     LatentPlan pl;
     lka_status_t s = latent_plan(B, h_q, g, s_q, d_h, r_kv, d_r, Lmax, &pl, pg != nullptr);
     if (s != LKA_OK) return s;
@@ -139,8 +143,14 @@ static lka_status_t latent_run(const void* q_c, const void* q_r, const void* w_u
     CUtensorMap tm_lat;
     const uint64_t lat_rows = pg ? (uint64_t)pg->num_pages * pg->page_size : (uint64_t)B * Lmax;
     const int box_rows = pg && pg->page_size < latent_tile_tokens() ? pg->page_size : latent_tile_tokens();
-    if (!make_tmap_2d(&tm_lat, BF, latent, r_kv + d_r, lat_rows, (uint64_t)(r_kv + d_r) * 2, 64, box_rows))
+    if (kv_scale) {
+        // e4m3 rows of r_kv + d_r bytes, 64-byte boxes without swizzle (the kernel widens them in shared memory)
+        if (!make_tmap_2d(&tm_lat, CU_TENSOR_MAP_DATA_TYPE_UINT8, latent, r_kv + d_r, lat_rows, (uint64_t)(r_kv + d_r),
+                          64, box_rows, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return LKA_ERR_CUDA;
+    } else if (!make_tmap_2d(&tm_lat, BF, latent, r_kv + d_r, lat_rows, (uint64_t)(r_kv + d_r) * 2, 64, box_rows)) {
         return LKA_ERR_CUDA;
+    }
     LatentParams lp{};
     lp.lens = cache_lens;
     lp.q_t = qt;
@@ -164,6 +174,7 @@ static lka_status_t latent_run(const void* q_c, const void* q_r, const void* w_u
     lp.max_pages = pg ? pg->max_pages : 0;
     lp.num_pages = pg ? pg->num_pages : 0;
     lp.box_rows = box_rows;
+    lp.kv_scale = kv_scale;
     if ((s = st_of(latent_attn_launch(tm_lat, lp, st))) != LKA_OK) return s;
 
     // 3) up-projection out = W^UV_gamma o~
@@ -191,6 +202,20 @@ lka_status_t latent_absorbed_attn(const void* q_c, const void* q_r, const void* 
                                   lka_dtype_t dtype, void* ws, size_t ws_bytes, void* stream) {
     return latent_run(q_c, q_r, w_uk, w_uv, latent, cache_lens, out, lse, B, h_q, g, s_q, d_h, r_kv, d_r, Lmax, causal,
                       scale, dtype, ws, ws_bytes, stream, nullptr);
+}
+
+size_t latent_absorbed_attn_fp8kv_workspace_size(int B, int h_q, int g, int s_q, int d_h, int r_kv, int d_r,
+                                                  int Lmax) {
+    return latent_absorbed_attn_workspace_size(B, h_q, g, s_q, d_h, r_kv, d_r, Lmax);
+}
+
+lka_status_t latent_absorbed_attn_fp8kv(const void* q_c, const void* q_r, const void* w_uk, const void* w_uv,
+                                        const void* latent, const float* kv_scale, const int32_t* cache_lens, void* out,
+                                        float* lse, int B, int h_q, int g, int s_q, int d_h, int r_kv, int d_r,
+                                        int Lmax, int causal, float scale, void* ws, size_t ws_bytes, void* stream) {
+    if (!kv_scale) return LKA_ERR_INVALID_ARG;
+    return latent_run(q_c, q_r, w_uk, w_uv, latent, cache_lens, out, lse, B, h_q, g, s_q, d_h, r_kv, d_r, Lmax, causal,
+                      scale, LKA_BF16, ws, ws_bytes, stream, nullptr, kv_scale);
 }
 
 size_t latent_absorbed_attn_paged_workspace_size(int B, int h_q, int g, int s_q, int d_h, int r_kv, int d_r,

@@ -55,11 +55,14 @@ constexpr int PF = 6;           // L2 prefetch distance in tiles
 constexpr int NKB = 5;          // 64-value boxes per rank and tile
 constexpr int KSTEPS = 18;      // K = 16 steps of this rank's 288 score values
 constexpr int BOX = NT * 128;   // one 64-value box of NT tokens
+constexpr int BOX8 = NT * 64;   // the same box of e4m3 values (FP8 cache), landing in the upper half of a stage
 constexpr int STAGE = NKB * BOX;
 constexpr int NSW = 8;          // softmax warps: 4 lane quarters x 2 column halves
 constexpr int NXW = 4;          // sender warps: one per lane quarter
+constexpr int NCW = 2;          // converter warps (FP8 cache only)
 constexpr int CW = NT / 2;      // score columns per softmax warp
 constexpr int NTHREADS = 32 * (NSW + 2 + NXW);
+constexpr int NTHREADS_F8 = NTHREADS + 32 * NCW;
 constexpr int XROW = CW * 4;    // bytes of one row of one half of an exchanged partial
 constexpr int XBUF = 2 * 128 * XROW;  // [half][head row][CW] fp32; each warp's block is contiguous
 constexpr int OFF_KV = 0;
@@ -129,7 +132,9 @@ __device__ __forceinline__ void remote_arrive(uint32_t rbar) {
 // peer's "buffer free" arrival (release at cluster scope) is only ever followed by new remote
 // stores, never by reads of data the peer produced.
 
-// 14 warps: an SM sub-partition holds up to 4 of them, so at most 16384 / (4 * 32) = 128 registers each
+// 14 warps (16 with an FP8 cache): an SM sub-partition holds up to 4 of them, so at most
+// 16384 / (4 * 32) = 128 registers each
+template <bool F8>
 __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
     latent_attn_kernel(const __grid_constant__ CUtensorMap tm_lat, const __grid_constant__ CUtensorMap tm_qt,
                        const __grid_constant__ CUtensorMap tm_qr, const LatentParams p) {
@@ -147,8 +152,10 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
     uint64_t* o_ready = p_ready + 1;      // PV(j) done
     uint64_t* xfull = o_ready + 1;        // [NSW] the peer's partial of warp w's block arrived
     uint64_t* xempty = xfull + NSW;       // [NSW] the peer has consumed this CTA's partial of warp w's block
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xempty + NSW);
+    uint64_t* conv_full = xempty + NSW;   // [NST] FP8 cache: the stage has been widened to bf16
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(conv_full + NST);
     __shared__ int s_abort;
+    __shared__ int s_conv_bad;  // FP8 cache: a converter thread gave up waiting (read by all converters)
 
     const uint32_t rank = cluster_rank();
     const uint32_t peer = rank ^ 1u;
@@ -167,6 +174,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
 
     if (threadIdx.x == 0) {
         s_abort = 0;
+        s_conv_bad = 0;
         mbar_init(smem_u32(q_full), NSW);
         mbar_init(smem_u32(q_loaded), 1);
         for (int s = 0; s < NST; ++s) {
@@ -181,6 +189,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
             mbar_init(smem_u32(&xfull[i]), 1);
             mbar_init(smem_u32(&xempty[i]), 1);
         }
+        for (int s = 0; s < NST; ++s) mbar_init(smem_u32(&conv_full[s]), NCW);
         fence_barrier_init();
         // the exchange buffer starts open for the peer's partial scores
         for (int i = 0; i < NSW; ++i) mbar_arrive_expect_tx(smem_u32(&xfull[i]), XBUF / NSW);
@@ -230,7 +239,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
             auto prefetch = [&](int i) {
                 for (int r0 = 0; r0 < NT; r0 += p.box_rows) {
                     const int y = cache_row(kbeg + i * NT + r0);
-                    for (int kb = 0; kb < NKB; ++kb) tma_prefetch_2d(&tm_lat, (int)rank * 256 + kb * 64, y);
+                    for (int kb = 0; kb < NKB; ++kb) tma_prefetch_2d(&tm_lat, (int)rank * 256 + kb * 64, y);  // bytes = values for e4m3
                 }
             };
             for (int i = NST; i < min(n_tiles, PF); ++i) prefetch(i);
@@ -248,12 +257,16 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
                     break;
                 }
                 const uint32_t fb = smem_u32(&kv_full[s]);
-                mbar_arrive_expect_tx(fb, NKB * BOX);
-                const uint32_t dst = smem_u32(smem + OFF_KV + s * STAGE);
+                mbar_arrive_expect_tx(fb, NKB * (F8 ? BOX8 : BOX));
+                const uint32_t dst = smem_u32(smem + OFF_KV + s * STAGE) + (F8 ? STAGE / 2 : 0);
                 for (int r0 = 0; r0 < NT; r0 += p.box_rows) {  // one box, or one per page piece of the tile
                     const int y = cache_row(kbeg + i * NT + r0);
-                    for (int kb = 0; kb < NKB; ++kb)
-                        tma_load_2d(dst + kb * BOX + r0 * 128, &tm_lat, (int)rank * 256 + kb * 64, y, fb);
+                    for (int kb = 0; kb < NKB; ++kb) {
+                        if (F8)
+                            tma_load_2d(dst + kb * BOX8 + r0 * 64, &tm_lat, (int)rank * 256 + kb * 64, y, fb);
+                        else
+                            tma_load_2d(dst + kb * BOX + r0 * 128, &tm_lat, (int)rank * 256 + kb * 64, y, fb);
+                    }
                 }
                 if (i + PF < n_tiles) prefetch(i + PF);
                 ++issued;
@@ -266,13 +279,14 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
         // Per step j: QK(j) once the softmax and sender warps have loaded S(j-1), then PV(j-2) once
         // P(j-2) is in tensor memory.  The softmax warps load S(j-1) before they compute P(j-2), so
         // QK(j) runs while tile j-2 is being finished.
-        constexpr uint32_t idesc_qk = idesc_bf16_f32(128, NT, false, false);
-        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
+        // an FP8 cache is widened to f16 (exact), and the query and P are f16 as well
+        constexpr uint32_t idesc_qk = F8 ? idesc_f16_f32(128, NT, false, false) : idesc_bf16_f32(128, NT, false, false);
+        constexpr uint32_t idesc_pv = F8 ? idesc_f16_f32(128, 256, false, true) : idesc_bf16_f32(128, 256, false, true);
         bool ok = mbar_wait(smem_u32(q_full), 0, p.status);
         for (int j = 0; ok && j < n_tiles + 2; ++j) {
             if (j < n_tiles) {
                 const int s = j % NST;
-                if (!mbar_wait(smem_u32(&kv_full[s]), (j / NST) & 1, p.status)) break;
+                if (!mbar_wait(smem_u32(F8 ? &conv_full[s] : &kv_full[s]), (j / NST) & 1, p.status)) break;
                 uint8_t* st = smem + OFF_KV + s * STAGE;
                 const int nvalid = min(NT, kend - (kbeg + j * NT));
                 if (nvalid < NT) {
@@ -318,7 +332,61 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
                 __syncwarp();
             }
         }
-    } else if (n_tiles > 0 && warp >= NSW + 2) {
+    } else if (F8 && n_tiles > 0 && warp >= NSW + 2 + NXW) {
+        // ------------------------------ converter warps ------------------------------
+        // FP8 cache: a tile lands as e4m3 in the upper half of its stage (five boxes of NT rows x 64
+        // bytes); the two converter warps widen it in place to the five f16 boxes (NT rows x 128 bytes,
+        // 128-byte swizzle) the MMAs read.  e4m3 -> f16 is exact: every e4m3 value is an f16 value.  Box k
+        // of the result overlaps only source boxes below k, or (k = 4) its own source: each source box is
+        // read into registers and all 64 threads meet at a barrier before its result is written.
+        // A thread that gives up waiting for a tile sets s_conv_bad before the first barrier of the tile, and all
+        // 64 threads leave together after it, so that no barrier is left with a missing thread.
+        const int ct = threadIdx.x - 32 * (NSW + 2 + NXW);  // 0 .. 63
+        bool bad = false;
+        for (int j = 0; !bad && j < n_tiles; ++j) {
+            const int s = j % NST;
+            if (!mbar_wait(smem_u32(&kv_full[s]), (j / NST) & 1, p.status)) s_conv_bad = 1;
+            uint8_t* st = smem + OFF_KV + s * STAGE;
+            const uint8_t* src = st + STAGE / 2;
+#pragma unroll 1
+            for (int k = 0; k < NKB; ++k) {
+                constexpr int PER = BOX8 / 16 / 64;  // 16-byte source chunks per thread and box
+                uint4 v[PER];
+#pragma unroll
+                for (int u = 0; u < PER; ++u) v[u] = *reinterpret_cast<const uint4*>(src + k * BOX8 + (ct + 64 * u) * 16);
+                named_barrier(5, 64);
+                if (k == 0 && *(volatile int*)&s_conv_bad) {
+                    bad = true;
+                    break;
+                }
+#pragma unroll
+                for (int u = 0; u < PER; ++u) {
+                    const int c = ct + 64 * u;        // chunk of the source box: 4 per 64-byte row
+                    const int r = c >> 2, q = c & 3;  // token row, group of 16 values in the row
+                    const uint32_t ws[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+                    uint32_t w[8];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const __half2_raw lo =
+                            __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(ws[i] & 0xffffu), __NV_E4M3);
+                        const __half2_raw hi =
+                            __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(ws[i] >> 16), __NV_E4M3);
+                        w[2 * i] = (uint32_t)lo.x | ((uint32_t)lo.y << 16);
+                        w[2 * i + 1] = (uint32_t)hi.x | ((uint32_t)hi.y << 16);
+                    }
+                    uint8_t* drow = st + k * BOX + r * 128;
+                    *reinterpret_cast<uint4*>(drow + (((2 * q) ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+                    *reinterpret_cast<uint4*>(drow + (((2 * q + 1) ^ (r & 7)) << 4)) =
+                        make_uint4(w[4], w[5], w[6], w[7]);
+                }
+            }
+            if (bad) break;
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the tensor cores
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&conv_full[s]));
+        }
+        if (bad) s_abort = 1;
+    } else if (n_tiles > 0 && warp >= NSW + 2 && warp < NSW + 2 + NXW) {
         // ------------------------------- sender warps -------------------------------
         // Sender warp q (= warp % 4) owns TMEM lane quarter q (head rows 32q .. +31): per tile it loads
         // this rank's partial scores of all NT columns from tensor memory, writes them to the outbox and
@@ -407,6 +475,16 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
                     w[4 * q + 1] = v.y;
                     w[4 * q + 2] = v.z;
                     w[4 * q + 3] = v.w;
+                }
+                if (F8) {
+                    // FP8 cache: the dequantisation scale of the latent part (or of the RoPE key) goes into
+                    // the query, which becomes f16 like the widened cache
+                    const float qs = p.kv_scale[rope ? 1 : 0];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+                        w[e] = pack_f16x2(f.x * qs, f.y * qs);
+                    }
                 }
                 tmem_st16(tmem + lane_base + T_Q + c0 * 16, w);
             }
@@ -504,7 +582,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
                 const float2 v = __fadd2_rn(make_float2(s[j], s[j + 1]), nm2);
                 s[j] = fast_exp2(v.x);
                 s[j + 1] = fast_exp2(v.y);
-                pk[j / 2] = pack_bf16x2(s[j], s[j + 1]);
+                pk[j / 2] = F8 ? pack_f16x2(s[j], s[j + 1]) : pack_bf16x2(s[j], s[j + 1]);
             }
             const float rs = tree_sum<CW>(s);
             l = (resc ? l * alpha : l) + rs;  // this warp's share of the row sum
@@ -535,7 +613,8 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
         const int last = n_tiles - 1;
         if (ok && n_tiles > 0 && mbar_wait(smem_u32(o_ready), last & 1, p.status)) {
             tc_fence_after();
-            const float inv_l = l > 0.f ? 1.f / l : 0.f;
+            // (FP8 cache: times the latent part's dequantisation scale, the value being the latent itself)
+            const float inv_l = (l > 0.f ? 1.f / l : 0.f) * (F8 ? p.kv_scale[0] : 1.f);
             const int HPG = p.h_q / p.g;
             const int grp = h / HPG, hh = h % HPG;
             const size_t prow = ((size_t)(b * p.s_q + t) * p.h_q + h);
@@ -638,6 +717,7 @@ __global__ void __launch_bounds__(128) latent_combine_kernel(const LatentParams 
 int latent_tile_tokens() { return lat::NT; }
 
 cudaError_t latent_attn_launch(const CUtensorMap& tm_lat, const LatentParams& p, cudaStream_t st) {
+    const bool f8 = p.kv_scale != nullptr;
     // the query slices: q~ [B*s_q*h_q][512] and q^R [B][h_q][s_q][64], 128 rows of 64 values per box
     CUtensorMap tm_qt, tm_qr;
     const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -649,12 +729,18 @@ cudaError_t latent_attn_launch(const CUtensorMap& tm_lat, const LatentParams& p,
         const uint32_t box[3] = {64, 1, 128};
         if (!make_tmap_nd(&tm_qr, BF, p.q_r, 3, dims, strides, box)) return cudaErrorInvalidValue;
     }
-    cudaError_t e = cudaFuncSetAttribute(latent_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, lat::SMEM);
+    cudaError_t e = f8 ? cudaFuncSetAttribute(latent_attn_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              lat::SMEM)
+                       : cudaFuncSetAttribute(latent_attn_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              lat::SMEM);
     if (e != cudaSuccess) return e;
     dim3 grid(2 * p.s_q * p.nsplit, p.B);
     {
         TimedLaunch timer(st);
-        latent_attn_kernel<<<grid, lat::NTHREADS, lat::SMEM, st>>>(tm_lat, tm_qt, tm_qr, p);
+        if (f8)
+            latent_attn_kernel<true><<<grid, lat::NTHREADS_F8, lat::SMEM, st>>>(tm_lat, tm_qt, tm_qr, p);
+        else
+            latent_attn_kernel<false><<<grid, lat::NTHREADS, lat::SMEM, st>>>(tm_lat, tm_qt, tm_qr, p);
         timer.stop();
     }
     e = cudaPeekAtLastError();

@@ -81,6 +81,16 @@ def _i32(x) -> np.ndarray:
     return np.ascontiguousarray(np.asarray(x, dtype=np.int32))
 
 
+def _u8(x) -> np.ndarray:
+    """The raw bytes of a tensor or array of 8-bit codes (a torch float8 tensor is viewed as uint8)."""
+    if hasattr(x, "detach"):
+        x = x.detach().to("cpu")
+        if x.dtype != torch.uint8:
+            x = x.view(torch.uint8)
+        x = x.numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.uint8))
+
+
 def _dp(a: np.ndarray):
     return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
 
@@ -244,10 +254,34 @@ def expanded_sparse(q_c, q_r, kc, vc, kr, indices, cache_lens, scale: float):
     return _sparse_apply(dense, [q_c, q_r], sel, rows, (B, h_q, s_q, d_h), (B, h_q, s_q))
 
 
+def decode_e4m3(x):
+    """The values of e4m3 codes (OCP 8-bit floating point E4M3, as torch.float8_e4m3fn or uint8), in float64, from
+    the format's bit fields: sign bit 7, exponent bits 6-3 with bias 7, mantissa bits 2-0; exponent 0 encodes the
+    subnormals m * 2^-9; S.1111.111 is NaN; there are no infinities (S.1111.000-110 are 256 .. 448)."""
+    u = _u8(x).astype(np.int64)
+    sign = np.where(u & 0x80, -1.0, 1.0)
+    e, m = (u >> 3) & 0xF, u & 0x7
+    mag = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    mag = np.where((e == 15) & (m == 7), np.nan, mag)
+    return sign * mag
+
+
 def dequantize_e4m3(x, head_scale):
-    """An e4m3 cache [B, h_kv, L, d] (torch.float8_e4m3fn) widened exactly and multiplied by its per-KV-head
-    scale [h_kv], in float64."""
-    return _f64(x.to(torch.float32)) * _f64(head_scale)[None, :, None, None]
+    """An e4m3 cache [B, h_kv, L, d] widened exactly (decode_e4m3) and multiplied by its per-KV-head scale [h_kv],
+    in float64."""
+    return decode_e4m3(x) * _f64(head_scale)[None, :, None, None]
+
+
+def latent_absorbed_fp8kv(q_c, q_r, w_uk, w_uv, latent8, kv_scale, cache_lens, causal: bool, scale: float,
+                          rows_b=None, n_threads: int = 0):
+    """The MQA-absorbed latent attention over an e4m3 latent cache [B, L, r_kv + d_r] with one scale for the
+    latent part and one for the RoPE key (kv_scale [2]): the dequantised cache, then latent_absorbed()."""
+    r_kv = int(np.asarray(w_uk.shape)[2])
+    sc = _f64(kv_scale)
+    lat = decode_e4m3(latent8)
+    lat[..., :r_kv] *= sc[0]
+    lat[..., r_kv:] *= sc[1]
+    return latent_absorbed(q_c, q_r, w_uk, w_uv, lat, cache_lens, causal, scale, rows_b=rows_b, n_threads=n_threads)
 
 
 def gqa_fp8kv(q, k, v, k_scale, v_scale, cache_lens, causal: bool, scale: float, rows_b=None, n_threads: int = 0):

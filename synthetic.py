@@ -97,6 +97,21 @@ def gqa_fp8_inputs(seed, B, h_q, h_kv, d, s_q, L_lo, L_hi, Lmax=None, device="cp
     return out
 
 
+def latent_fp8_inputs(seed, B, h_q, g_groups, d_h, r_kv, d_r, s_q, L_lo, L_hi, Lmax=None, device="cpu"):
+    """GQLA latent inputs (as latent_inputs, bf16 queries and weights) with the latent cache drawn N(0,1) in fp32 and
+    stored as e4m3 with one scale for the latent part and one for the RoPE key (each part's max |value| / 448);
+    kv_scale = [scale of c^KV, scale of k^R] (c^KV = kv_scale[0] * latent8[..., :r_kv])."""
+    inp = latent_inputs(seed, B, h_q, g_groups, d_h, r_kv, d_r, s_q, L_lo, L_hi, Lmax=Lmax, device=device)
+    g = _gen(seed + 104729, device)
+    x = torch.randn(inp["latent"].shape, generator=g, device=device, dtype=torch.float32)
+    sc = torch.stack([x[..., :r_kv].abs().amax(), x[..., r_kv:].abs().amax()]).clamp_min(1e-12) / 448.0
+    widths = torch.cat([sc[0].expand(r_kv), sc[1].expand(d_r)])
+    inp["latent8"] = (x / widths).to(torch.float8_e4m3fn)
+    inp["kv_scale"] = sc.contiguous()
+    del inp["latent"]
+    return inp
+
+
 def to_pages(caches, lens, page_size, gen, spare_pages=0):
     """Scatters contiguous caches [B, heads, Lmax, width] (e.g. K and V) into shuffled page pools [num_pages, heads,
     page_size, width] sharing one block table [B, Lmax / page_size] (int32): the pages a sequence uses
@@ -262,6 +277,9 @@ WORKLOADS = {
     # the s_q = 1 layer over a paged latent cache (64-token pages, shuffled pool, block table)
     "latent_decode_4k_sq1_paged": dict(kind="latent_paged", seed=4, B=64, h_q=128, g=8, d_h=128, r_kv=512, d_r=64,
                                        s_q=1, L_lo=4096, L_hi=4096, causal=True, page_size=64),
+    # the same layer with the latent cache in e4m3 (one scale for c^KV, one for k^R)
+    "latent_decode_4k_sq1_fp8": dict(kind="latent_fp8", seed=4, B=64, h_q=128, g=8, d_h=128, r_kv=512, d_r=64,
+                                     s_q=1, L_lo=4096, L_hi=4096, causal=True),
     # top-k sparse decode: 2048 of the 16K cached tokens per query, selected uniformly at random
     "latent_sparse_16k_top2048": dict(kind="latent_sparse", seed=8, B=64, h_q=128, g=8, d_h=128, r_kv=512, d_r=64,
                                       s_q=1, L_lo=16384, L_hi=16384, causal=True, topk=2048),
@@ -306,6 +324,9 @@ def make(w: dict, device="cpu", dtype=torch.bfloat16) -> dict:
     if w["kind"] == "latent_paged":
         return latent_paged_inputs(w["seed"], w["B"], w["h_q"], w["g"], w["d_h"], w["r_kv"], w["d_r"], w["s_q"],
                                    w["L_lo"], w["L_hi"], w["page_size"], dtype=dtype, device=device)
+    if w["kind"] == "latent_fp8":
+        return latent_fp8_inputs(w["seed"], w["B"], w["h_q"], w["g"], w["d_h"], w["r_kv"], w["d_r"], w["s_q"],
+                                 w["L_lo"], w["L_hi"], device=device)
     if w["kind"] == "latent_sparse":
         inp = latent_inputs(w["seed"], w["B"], w["h_q"], w["g"], w["d_h"], w["r_kv"], w["d_r"], w["s_q"],
                             w["L_lo"], w["L_hi"], dtype=dtype, device=device)

@@ -1,4 +1,5 @@
-"""GPU parity of gqa_attn_fp8kv (GQA over an e4m3 KV cache) against the fp64 oracle (marked gpu)."""
+"""GPU parity of the e4m3-cache entry points (gqa_attn_fp8kv, latent_absorbed_attn_fp8kv) against the fp64 oracle
+(marked gpu)."""
 import pytest
 import torch
 
@@ -52,3 +53,62 @@ def test_fp8kv_matches_bf16_path_on_the_dequantised_cache():
     v16 = (dd["v"].float() * dd["v_scale"][None, :, None, None]).to(torch.bfloat16)
     b = lka.gqa_attn(dd["q"], k16, v16, dd["cache_lens"], scale=inp["scale"])
     assert (a.float() - b.float()).abs().max().item() <= 2e-2
+
+
+# ------------------------------------------------------------------ FP8 latent cache (MQA-absorbed path) -----
+LATENT_CASES = [
+    # (B, s_q, L_lo, L_hi, Lmax, causal)
+    (2, 1, 1, 700, 768, True),      # ragged, L = 1 possible, several tiles and a ragged tail
+    (3, 2, 2, 500, 520, True),      # MTP, bottom-right causal
+    (2, 1, 60, 130, 130, False),    # no mask
+]
+
+
+@pytest.mark.parametrize("case", LATENT_CASES, ids=[f"B{c[0]}sq{c[1]}L{c[3]}" for c in LATENT_CASES])
+def test_latent_fp8kv(case):
+    B, s_q, lo, hi, Lmax, causal = case
+    inp = synthetic.latent_fp8_inputs(810 + B * 7 + s_q, B, 128, 8, 128, 512, 64, s_q, lo, hi, Lmax=Lmax)
+    dd = {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    out, lse = lka.latent_absorbed_attn_fp8kv(dd["q_c"], dd["q_r"], dd["w_uk"], dd["w_uv"], dd["latent8"],
+                                              dd["kv_scale"], dd["cache_lens"], causal=causal, scale=inp["scale"],
+                                              return_lse=True)
+    ref, ref_lse = oracle.latent_absorbed_fp8kv(inp["q_c"], inp["q_r"], inp["w_uk"], inp["w_uv"], inp["latent8"],
+                                                inp["kv_scale"], inp["cache_lens"], causal, inp["scale"])
+    assert_close(out, ref, torch.bfloat16, "latent fp8kv out")
+    assert_lse_close(lse, ref_lse, torch.bfloat16, "latent fp8kv lse")
+
+
+def test_latent_fp8kv_forced_splits_and_bf16_agreement():
+    """Key splits (merged partials) give the same result within tolerance, and the bf16 path over the dequantised
+    cache (rounded to bf16, exact for these values) agrees within bf16 noise."""
+    inp = synthetic.latent_fp8_inputs(850, 2, 128, 8, 128, 512, 64, 1, 300, 900, Lmax=960)
+    dd = {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    a = lka.latent_absorbed_attn_fp8kv(dd["q_c"], dd["q_r"], dd["w_uk"], dd["w_uv"], dd["latent8"], dd["kv_scale"],
+                                       dd["cache_lens"], scale=inp["scale"])
+    prev = lka.set_split_tokens(128)
+    try:
+        b = lka.latent_absorbed_attn_fp8kv(dd["q_c"], dd["q_r"], dd["w_uk"], dd["w_uv"], dd["latent8"],
+                                           dd["kv_scale"], dd["cache_lens"], scale=inp["scale"])
+    finally:
+        lka.set_split_tokens(prev)
+    ref, _ = oracle.latent_absorbed_fp8kv(inp["q_c"], inp["q_r"], inp["w_uk"], inp["w_uv"], inp["latent8"],
+                                          inp["kv_scale"], inp["cache_lens"], True, inp["scale"])
+    assert_close(b, ref, torch.bfloat16, "latent fp8kv split")
+    lat = dd["latent8"].to(torch.float32)
+    lat[..., :512] *= dd["kv_scale"][0]
+    lat[..., 512:] *= dd["kv_scale"][1]
+    c = lka.latent_absorbed_attn(dd["q_c"], dd["q_r"], dd["w_uk"], dd["w_uv"], lat.to(torch.bfloat16),
+                                 dd["cache_lens"], scale=inp["scale"])
+    assert (a.float() - c.float()).abs().max().item() <= 2e-2
+    assert (a.float() - b.float()).abs().max().item() <= 2e-2
+
+
+def test_latent_fp8kv_rejects_bad_arguments():
+    inp = synthetic.latent_fp8_inputs(860, 1, 128, 8, 128, 512, 64, 1, 10, 20)
+    dd = {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    with pytest.raises(Exception):
+        lka.latent_absorbed_attn_fp8kv(dd["q_c"], dd["q_r"], dd["w_uk"], dd["w_uv"], dd["latent8"],
+                                       dd["kv_scale"][:1], dd["cache_lens"])
+    with pytest.raises(Exception):  # a bf16 cache is not an e4m3 cache
+        lka.latent_absorbed_attn_fp8kv(dd["q_c"], dd["q_r"], dd["w_uk"], dd["w_uv"],
+                                       dd["latent8"].to(torch.bfloat16), dd["kv_scale"], dd["cache_lens"])

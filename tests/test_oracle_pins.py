@@ -379,6 +379,22 @@ def test_gta_paged_oracle_equals_contiguous():
     assert (inp["block_table"] >= 0).sum() < inp["k_pages"].shape[0]  # spare pages: the pool is not the table
 
 
+def test_latent_fp8_oracle_is_latent_over_the_dequantised_cache():
+    """The fp8 latent oracle equals the latent definition over the cache widened by torch's float8_e4m3fn cast
+    and scaled, the latent part and the RoPE key each by its own scale (two different scales)."""
+    inp = synthetic.latent_fp8_inputs(66, 2, 16, 1, 16, 32, 8, 2, 5, 30)
+    r_kv = 32
+    lat = inp["latent8"].to(torch.float64)
+    lat[..., :r_kv] *= float(inp["kv_scale"][0])
+    lat[..., r_kv:] *= float(inp["kv_scale"][1])
+    assert float(inp["kv_scale"][0]) != float(inp["kv_scale"][1])
+    ref, ref_lse = oracle.latent_absorbed(inp["q_c"], inp["q_r"], inp["w_uk"], inp["w_uv"], lat, inp["cache_lens"],
+                                          True, inp["scale"])
+    out, lse = oracle.latent_absorbed_fp8kv(inp["q_c"], inp["q_r"], inp["w_uk"], inp["w_uv"], inp["latent8"],
+                                            inp["kv_scale"], inp["cache_lens"], True, inp["scale"])
+    assert np.array_equal(out, ref) and np.array_equal(lse, ref_lse)
+
+
 # ------------------------------------------------------------------ top-k sparse attention ------------------
 def test_sparse_oracle_full_selection_equals_dense_causal():
     """Selecting every key a query may see (in a shuffled order) is the dense causal attention ("GQLA ..."
@@ -417,11 +433,19 @@ def test_sparse_oracle_empty_selection():
 
 # ------------------------------------------------------------------ FP8 (e4m3) KV cache ----------------------
 def test_e4m3_decoding_and_fp8_oracle():
-    """The e4m3 widening the fp8 oracle uses (torch's float8_e4m3fn: 1 sign, 4 exponent bits with bias 7,
-    3 mantissa bits, no infinities) on codes whose values the format fixes, and the per-KV-head scaling."""
-    codes = torch.tensor([0x38, 0x40, 0x01, 0x08, 0x7E, 0xB8, 0x00, 0x3C], dtype=torch.uint8)
-    vals = codes.view(torch.float8_e4m3fn).to(torch.float64).tolist()
-    assert vals == [1.0, 2.0, 2.0 ** -9, 2.0 ** -6, 448.0, -1.0, 0.0, 1.5]
+    """The oracle's e4m3 decode (bit fields: 1 sign, 4 exponent bits with bias 7, 3 mantissa bits, subnormals,
+    NaN, no infinities) on codes whose values the format fixes, on all 256 codes against torch's float8_e4m3fn
+    cast (a second, independent decoder), and the per-KV-head scaling of the fp8 GQA oracle."""
+    codes = torch.tensor([0x38, 0x40, 0x01, 0x08, 0x7E, 0xB8, 0x00, 0x3C, 0x07, 0x77, 0x80], dtype=torch.uint8)
+    vals = oracle.decode_e4m3(codes).tolist()
+    assert vals == [1.0, 2.0, 2.0 ** -9, 2.0 ** -6, 448.0, -1.0, 0.0, 1.5, 7 * 2.0 ** -9, 240.0, -0.0]
+    assert math.copysign(1.0, vals[-1]) == -1.0
+    allc = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    mine = oracle.decode_e4m3(allc)
+    lib = allc.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(mine), np.isnan(lib)) and np.isnan(mine).sum() == 2  # 0x7F and 0xFF
+    ok = ~np.isnan(mine)
+    assert np.array_equal(mine[ok], lib[ok])
     inp = synthetic.gqa_fp8_inputs(81, 2, 8, 2, 128, 1, 5, 40)
     k = inp["k"].to(torch.float64) * inp["k_scale"].double()[None, :, None, None]
     v = inp["v"].to(torch.float64) * inp["v_scale"].double()[None, :, None, None]
