@@ -41,12 +41,29 @@
 // and swap their row maxima through two spare TMEM columns), with lazy
 // rescaling (the running maximum is only moved when it grows by more than 2^8,
 // which leaves the final O / l exact); P is written back to TMEM as bf16.
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
 #include "common.cuh"
 #include "host_util.h"
 #include "latent.h"
 #include "tc.cuh"
 
 namespace lka {
+
+// f16 operands (FP8 cache: the widened cache, the query and P): instruction descriptor of kind::f16 with
+// A = B = f16 (format 0), D = fp32, dense, and the f16 pair packing
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool a_mn, bool b_mn) {
+    return (1u << 4)                      // D format fp32
+           | ((a_mn ? 1u : 0u) << 15)     // A major
+           | ((b_mn ? 1u : 0u) << 16)     // B major
+           | ((uint32_t)(N >> 3) << 17)   // N / 8
+           | ((uint32_t)(M >> 4) << 24);  // M / 16
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    __half2 v = __floats2half2_rn(lo, hi);  // .x = lo (low 16 bits), .y = hi
+    return *reinterpret_cast<uint32_t*>(&v);
+}
 
 namespace lat {
 constexpr int NT = 64;          // tokens per tile (the N of the score MMA)

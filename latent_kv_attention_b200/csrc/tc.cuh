@@ -62,15 +62,6 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn, b
            | ((uint32_t)(M >> 4) << 24);  // M / 16
 }
 
-// The same with A = B = f16.
-__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool a_mn, bool b_mn) {
-    return (1u << 4)                      // D format fp32 (A and B format 0: f16)
-           | ((a_mn ? 1u : 0u) << 15)
-           | ((b_mn ? 1u : 0u) << 16)
-           | ((uint32_t)(N >> 3) << 17)
-           | ((uint32_t)(M >> 4) << 24);
-}
-
 // ---- MMA issue (one thread) -----------------------------------------------------------
 // D[tmem] = A[smem] * B[smem]^T (+ D if accumulate)
 __device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
@@ -133,10 +124,6 @@ __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (low 16 bits), .y = hi
-    return *reinterpret_cast<uint32_t*>(&v);
-}
-__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
-    __half2 v = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
