@@ -48,12 +48,38 @@ struct ExpCfg {
     static constexpr int SMEM = 1024 + OFF_BAR + 256;
     static constexpr uint32_t T_S = 0;             // 2 x NR columns
     static constexpr uint32_t T_O = 2 * NR;        // NR columns
-    static constexpr int K_ITEMS = NR * 16 / 128;  // (row, 8-token chunk) items per softmax thread
+    static constexpr int NSW = 8;                  // softmax warps: 4 TMEM lane quarters x 2 column halves
+    static constexpr int HALF = NR / 2;            // score / output columns per softmax warp
+    static constexpr int K_ITEMS = NR * 16 / (32 * NSW);  // (row, 8-token chunk) items per softmax thread
+    static constexpr int NTHREADS = 32 * (NSW + 2);
     static_assert(Q_BYTES <= OFF_KV, "Q region");
 };
 
+// 8 consecutive columns of this warp's 32 TMEM lanes
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* r) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+}
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t* r) {
+    static_assert(N == 8 || N == 16, "8 or 16 columns");
+    if constexpr (N == 8)
+        tmem_ld8(taddr, r);
+    else
+        tmem_ld16(taddr, r);
+}
+template <int N>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t* r) {
+    static_assert(N == 8 || N == 16, "8 or 16 columns");
+    if constexpr (N == 8)
+        tmem_st8(taddr, r);
+    else
+        tmem_st16(taddr, r);
+}
+
 template <int NR>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(ExpCfg<NR>::NTHREADS, 1)
     expanded_attn_kernel(const __grid_constant__ CUtensorMap tm_qc, const __grid_constant__ CUtensorMap tm_qr,
                          const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_kr,
                          const __grid_constant__ CUtensorMap tm_vc, const ExpParams p) {
@@ -76,6 +102,7 @@ __global__ void __launch_bounds__(192, 1)
     float* l_buf = alpha_buf + NR;
     float* m_buf = l_buf + NR;
     __shared__ int s_abort;
+    __shared__ int s_resc[2];  // [tile & 1] some row of the tile moved its reference maximum
 
     const int split = blockIdx.x, grp = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -89,6 +116,7 @@ __global__ void __launch_bounds__(192, 1)
 
     if (threadIdx.x == 0) {
         s_abort = 0;
+        s_resc[0] = s_resc[1] = 0;
         mbar_init(smem_u32(q_full), 1);
         for (int s = 0; s < NST; ++s) {
             mbar_init(smem_u32(&k_full[s]), 1);
@@ -98,13 +126,13 @@ __global__ void __launch_bounds__(192, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(smem_u32(&s_ready[i]), 1);
-            mbar_init(smem_u32(&s_free[i]), 4);
-            mbar_init(smem_u32(&p_ready[i]), 4);
+            mbar_init(smem_u32(&s_free[i]), C::NSW);
+            mbar_init(smem_u32(&p_ready[i]), C::NSW);
             mbar_init(smem_u32(&o_ready[i]), 1);
         }
         fence_barrier_init();
     }
-    if (warp == 5) {
+    if (warp == C::NSW + 1) {
         tmem_alloc(tmem_slot, 128);
         tmem_relinquish();
     }
@@ -113,7 +141,7 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 4) {
+    if (warp == C::NSW) {
         // --------------------------------- producer ---------------------------------
         if (lane == 0) {
             const uint32_t qb = smem_u32(q_full);
@@ -193,7 +221,7 @@ __global__ void __launch_bounds__(192, 1)
                 mbar_wait(smem_u32(&v_full[i % NST]), (i / NST) & 1, p.status);
             mbar_wait(qb, 0, p.status);
         }
-    } else if (warp == 5) {
+    } else if (warp == C::NSW + 1) {
         // -------------------------------- MMA issuer --------------------------------
         // per step j: QK(j) (needs S(j-2) loaded by the softmax warps) and PV(j-1)
         constexpr uint32_t idesc_qk = idesc_bf16_f32(128, NR, false, false);
@@ -265,9 +293,13 @@ __global__ void __launch_bounds__(192, 1)
             }
         }
     } else {
-        // ----------------------------- softmax warps (0-3) -----------------------------
-        const int tid = threadIdx.x;  // token lane of S^T, value dim of O^T
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        // ----------------------------- softmax warps (0-7) -----------------------------
+        // Warp w reads TMEM lane quarter w % 4 (tokens of S^T, value dims of O^T) and the column half w / 4
+        // (query rows); after the transpose through shared memory the (row, 8-token chunk) items are
+        // spread over all 256 threads.
+        const int tid = (warp & 3) * 32 + lane;  // token lane of S^T, value dim of O^T
+        const int half = warp >> 2;
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         float m_ref[C::K_ITEMS], lsum[C::K_ITEMS];
 #pragma unroll
         for (int k = 0; k < C::K_ITEMS; ++k) {
@@ -282,24 +314,26 @@ __global__ void __launch_bounds__(192, 1)
             tc_fence_after();
             float* sc = reinterpret_cast<float*>(smem + C::OFF_SC + x * C::SC_BYTES);
             {
-                uint32_t v[NR];
-#pragma unroll
-                for (int c0 = 0; c0 < NR; c0 += 16) tmem_ld16(tmem + lane_base + C::T_S + x * NR + c0, v + c0);
+                uint32_t v[C::HALF];
+                tmem_ld_cols<C::HALF>(tmem + lane_base + C::T_S + x * NR + half * C::HALF, v);
                 tmem_ld_wait();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&s_free[x]));  // the score buffer may be rewritten
 #pragma unroll
-                for (int r = 0; r < NR; ++r) sc[r * TK + tid] = __uint_as_float(v[r]);
+                for (int r = 0; r < C::HALF; ++r) sc[(half * C::HALF + r) * TK + tid] = __uint_as_float(v[r]);
             }
             // P^T buffer x was last read by PV(i-2)
             if (ok && i >= 2) ok = mbar_wait(smem_u32(&o_ready[x]), ((i >> 1) - 1) & 1, p.status);
-            named_barrier(1, 128);
+            // the rescale flag of this buffer was last read in tile i-2, before every thread passed the
+            // barriers of tile i-1
+            if (threadIdx.x == 0) s_resc[x] = 0;
+            named_barrier(1, 32 * C::NSW);
             uint8_t* pt = smem + C::OFF_PT + x * C::PT_BYTES;
             const int k0 = kbeg + i * TK;
 #pragma unroll
             for (int k = 0; k < C::K_ITEMS; ++k) {
-                const int r = 8 * k + 2 * warp + lane / 16;  // query row: hh * s_q + t
+                const int r = 2 * C::NSW * k + 2 * warp + lane / 16;  // query row: hh * s_q + t (16 lanes per row)
                 const int t = r % p.s_q;
                 const int rend = min(p.causal ? L - p.s_q + t + 1 : L, kbeg + p.split_tokens);
                 const float4 a = *reinterpret_cast<const float4*>(sc + r * TK + 8 * c8);
@@ -307,49 +341,48 @@ __global__ void __launch_bounds__(192, 1)
                 float s[8] = {a.x, a.y, a.z, a.w, bq.x, bq.y, bq.z, bq.w};
 #pragma unroll
                 for (int e = 0; e < 8; ++e) s[e] = (k0 + 8 * c8 + e < rend) ? s[e] * p.scale_log2 : -INFINITY;
+                // lazy rescaling: the reference maximum of a row only moves when one of its scores exceeds it
+                // by more than 2^8, so the row maximum is only reduced over the 16 lanes of the row then (the
+                // warp's two rows together); the row sums stay per lane until the end
                 float mx = tree_max<8>(s);
-#pragma unroll
-                for (int m = 8; m >= 1; m /= 2) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
-                const float m_new = fmaxf(m_ref[k], mx);
                 float alpha = 1.f, m_use = m_ref[k];
-                if (m_ref[k] == -INFINITY) {
-                    m_use = m_new;
-                } else if (m_new > m_ref[k] + 8.0f) {
-                    alpha = fast_exp2(m_ref[k] - m_new);
-                    m_use = m_new;
+                if (__any_sync(0xffffffffu, !(mx <= m_ref[k] + 8.0f))) {
+#pragma unroll
+                    for (int m = 8; m >= 1; m /= 2) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
+                    const float m_new = fmaxf(m_ref[k], mx);
+                    if (m_ref[k] == -INFINITY) {
+                        m_use = m_new;
+                    } else if (m_new > m_ref[k] + 8.0f) {
+                        alpha = fast_exp2(m_ref[k] - m_new);
+                        m_use = m_new;
+                    }
                 }
                 float pv[8];
                 const float m_sub = m_use == -INFINITY ? 0.f : m_use;  // all scores -inf: p = 0
 #pragma unroll
                 for (int e = 0; e < 8; ++e) pv[e] = fast_exp2(s[e] - m_sub);
-                float rs = tree_sum<8>(pv);
-#pragma unroll
-                for (int m = 8; m >= 1; m /= 2) rs += __shfl_xor_sync(0xffffffffu, rs, m);
-                lsum[k] = lsum[k] * alpha + rs;
+                lsum[k] = lsum[k] * alpha + tree_sum<8>(pv);  // this lane's share of the row sum
                 m_ref[k] = m_use;
                 const int kb2 = c8 / 8, cc = c8 % 8;
                 *reinterpret_cast<uint4*>(pt + kb2 * NR * 128 + r * 128 + ((cc ^ (r & 7)) << 4)) =
                     make_uint4(pack_bf16x2(pv[0], pv[1]), pack_bf16x2(pv[2], pv[3]), pack_bf16x2(pv[4], pv[5]),
                                pack_bf16x2(pv[6], pv[7]));
                 if (c8 == 0) alpha_buf[r] = alpha;
+                if (alpha != 1.f) s_resc[x] = 1;
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            named_barrier(1, 128);  // alpha_buf complete
-            bool any = false;
-#pragma unroll
-            for (int r = 0; r < NR; ++r) any |= alpha_buf[r] != 1.f;
-            if (any) {
+            named_barrier(1, 32 * C::NSW);  // alpha_buf and the rescale flag complete
+            if (*(volatile int*)&s_resc[x]) {
                 // O^T may only be rescaled once PV(i-1) has been accumulated into it
                 if (ok && i >= 1) ok = mbar_wait(smem_u32(&o_ready[(i - 1) & 1]), ((i - 1) >> 1) & 1, p.status);
                 tc_fence_after();
-                uint32_t o[NR];
-#pragma unroll
-                for (int c0 = 0; c0 < NR; c0 += 16) tmem_ld16(tmem + lane_base + C::T_O + c0, o + c0);
+                uint32_t o[C::HALF];
+                tmem_ld_cols<C::HALF>(tmem + lane_base + C::T_O + half * C::HALF, o);
                 tmem_ld_wait();
 #pragma unroll
-                for (int r = 0; r < NR; ++r) o[r] = __float_as_uint(__uint_as_float(o[r]) * alpha_buf[r]);
-#pragma unroll
-                for (int c0 = 0; c0 < NR; c0 += 16) tmem_st16(tmem + lane_base + C::T_O + c0, o + c0);
+                for (int r = 0; r < C::HALF; ++r)
+                    o[r] = __float_as_uint(__uint_as_float(o[r]) * alpha_buf[half * C::HALF + r]);
+                tmem_st_cols<C::HALF>(tmem + lane_base + C::T_O + half * C::HALF, o);
                 tmem_st_wait();
             }
             tc_fence_before();
@@ -360,30 +393,32 @@ __global__ void __launch_bounds__(192, 1)
         if (ok) ok = mbar_wait(smem_u32(&o_ready[(n_tiles - 1) & 1]), ((n_tiles - 1) >> 1) & 1, p.status);
 #pragma unroll
         for (int k = 0; k < C::K_ITEMS; ++k) {
-            const int r = 8 * k + 2 * warp + lane / 16;
+            const int r = 2 * C::NSW * k + 2 * warp + lane / 16;
+#pragma unroll
+            for (int m = 8; m >= 1; m /= 2) lsum[k] += __shfl_xor_sync(0xffffffffu, lsum[k], m);  // the row sum
             if (c8 == 0) {
                 l_buf[r] = lsum[k];
                 m_buf[r] = m_ref[k];
             }
         }
-        named_barrier(1, 128);
+        named_barrier(1, 32 * C::NSW);
         if (!ok) {
             s_abort = 1;
         } else {
             tc_fence_after();
-            uint32_t o[NR];
-#pragma unroll
-            for (int c0 = 0; c0 < NR; c0 += 16) tmem_ld16(tmem + lane_base + C::T_O + c0, o + c0);
+            uint32_t o[C::HALF];
+            tmem_ld_cols<C::HALF>(tmem + lane_base + C::T_O + half * C::HALF, o);
             tmem_ld_wait();
 #pragma unroll
-            for (int r = 0; r < NR; ++r) {
+            for (int rr = 0; rr < C::HALF; ++rr) {
+                const int r = half * C::HALF + rr;
                 const int hh = r / p.s_q, t = r % p.s_q;
                 const int n_t = p.causal ? L - p.s_q + t + 1 : L;
                 if (kbeg >= n_t) continue;  // no keys of this row in this split
                 const int nsp = cdiv(n_t, p.split_tokens);
                 const size_t orow = ((size_t)b * p.h_q + grp * HPG + hh) * p.s_q + t;
                 const float l = l_buf[r];
-                const float ov = __uint_as_float(o[r]) / l;
+                const float ov = __uint_as_float(o[rr]) / l;
                 const float lse2 = m_buf[r] + log2f(l);
                 if (nsp == 1) {
                     p.out[orow * 128 + tid] = __float2bfloat16_rn(ov);
@@ -397,7 +432,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) tmem_dealloc(tmem, 128);
+    if (warp == C::NSW + 1) tmem_dealloc(tmem, 128);
 }
 
 cudaError_t expanded_attn_launch(const CUtensorMap& qc, const CUtensorMap& qr, const CUtensorMap& kc,
@@ -409,12 +444,12 @@ cudaError_t expanded_attn_launch(const CUtensorMap& qc, const CUtensorMap& qr, c
         e = cudaFuncSetAttribute(expanded_attn_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  ExpCfg<16>::SMEM);
         if (e != cudaSuccess) return e;
-        expanded_attn_kernel<16><<<grid, 192, ExpCfg<16>::SMEM, st>>>(qc, qr, kc, kr, vc, p);
+        expanded_attn_kernel<16><<<grid, ExpCfg<16>::NTHREADS, ExpCfg<16>::SMEM, st>>>(qc, qr, kc, kr, vc, p);
     } else {
         e = cudaFuncSetAttribute(expanded_attn_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  ExpCfg<32>::SMEM);
         if (e != cudaSuccess) return e;
-        expanded_attn_kernel<32><<<grid, 192, ExpCfg<32>::SMEM, st>>>(qc, qr, kc, kr, vc, p);
+        expanded_attn_kernel<32><<<grid, ExpCfg<32>::NTHREADS, ExpCfg<32>::SMEM, st>>>(qc, qr, kc, kr, vc, p);
     }
     timer.stop();
     return cudaPeekAtLastError();
