@@ -516,7 +516,9 @@ class GtaPrefill(Workload):
         i = self.inp
         w = self.w
         self.out = torch.empty((w["B"], w["H"], w["s_q"], w["d_v"]), dtype=torch.bfloat16, device=self.device)
-        self.launches = 1
+        ws = self.lka.library().gta_shared_score_attn_workspace_size(w["B"], w["G"], w["H"], w["s_q"], w["d_qk"],
+                                                                     w["d_v"], w["L_hi"])
+        self.launches = 2 if ws > 256 else 1  # attention (+ merge of key splits)
         self.h2d_pairs = [(i[k], _pinned(i[k])) for k in ("q_g", "k_g", "v", "cache_lens")]
         self.out_host = torch.empty_like(self.out, device="cpu").pin_memory()
 

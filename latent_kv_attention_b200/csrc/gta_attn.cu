@@ -41,6 +41,11 @@ struct GtaParams {
     const int32_t* block_table;  // [B, max_pages]
     int page_size, max_pages, num_pages;
     int box_rows;                // rows per TMA box: min(128, page_size), or 128 when contiguous
+    // key splits (nsplit > 1): split k covers keys [k * split_tokens, (k + 1) * split_tokens); a row whose keys
+    // need more than one split writes normalised fp32 partials that gta_combine_kernel merges
+    int split_tokens, nsplit;
+    float* part_o;    // [B * H * s_q][nsplit][64]
+    float* part_lse;  // [B * G * s_q][nsplit] log2 domain (one per group: the score matrix is the group's)
 };
 
 namespace gta {
@@ -84,7 +89,8 @@ __global__ void __launch_bounds__(gta::NTHREADS, 1)
     __shared__ int s_abort;
 
     const int n_qt = cdiv(p.s_q, TQ);
-    const int qt = n_qt - 1 - (int)blockIdx.x;  // longest tiles first
+    const int qt = n_qt - 1 - (int)blockIdx.x / p.nsplit;  // longest tiles first
+    const int split = (int)blockIdx.x % p.nsplit;
     const int grp = blockIdx.y, b = blockIdx.z;
     const int HPG = p.H / p.G;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -92,8 +98,11 @@ __global__ void __launch_bounds__(gta::NTHREADS, 1)
                             threadIdx.x == 0 && blockIdx.x == 0 && grp == 0);
     const int q0 = qt * TQ;
     const int q_last = min(q0 + TQ, p.s_q) - 1;
-    const int key_end = p.causal ? (L - p.s_q + q_last + 1) : L;  // keys any row of the tile may see
-    const int n_tiles = cdiv(key_end, TK);
+    const int key_all = p.causal ? (L - p.s_q + q_last + 1) : L;  // keys any row of the tile may see
+    const int kbeg = split * p.split_tokens;
+    const int key_end = min(key_all, kbeg + p.split_tokens);      // this split's share of them
+    if (key_end <= kbeg) return;                                   // no key of this split is visible
+    const int n_tiles = cdiv(key_end - kbeg, TK);
 
     if (threadIdx.x == 0) {
         s_abort = 0;
@@ -154,8 +163,8 @@ __global__ void __launch_bounds__(gta::NTHREADS, 1)
                 const uint32_t fb = smem_u32(&k_full[s]);
                 mbar_arrive_expect_tx(fb, BOX);
                 for (int r0 = 0; r0 < TK; r0 += p.box_rows)  // one box, or one per page piece of the tile
-                    tma_load_2d(smem_u32(smem + OFF_K + s * BOX) + r0 * 128, &tm_k, 0, cache_row(i * TK + r0, p.G, grp),
-                                fb);
+                    tma_load_2d(smem_u32(smem + OFF_K + s * BOX) + r0 * 128, &tm_k, 0,
+                                cache_row(kbeg + i * TK + r0, p.G, grp), fb);
                 ++k_issued;
                 return true;
             };
@@ -167,7 +176,8 @@ __global__ void __launch_bounds__(gta::NTHREADS, 1)
                 const uint32_t d = smem_u32(smem + OFF_V + s * VSTAGE);
                 for (int hh = 0; hh < HPG; ++hh)
                     for (int r0 = 0; r0 < TK; r0 += p.box_rows)
-                        tma_load_2d(d + hh * BOX + r0 * 128, &tm_v, 0, cache_row(i * TK + r0, p.H, grp * HPG + hh), fb);
+                        tma_load_2d(d + hh * BOX + r0 * 128, &tm_v, 0, cache_row(kbeg + i * TK + r0, p.H, grp * HPG + hh),
+                                    fb);
                 ++v_issued;
                 return true;
             };
@@ -192,7 +202,7 @@ __global__ void __launch_bounds__(gta::NTHREADS, 1)
         bool ok = mbar_wait(smem_u32(q_full), 0, p.status);
         // zero the rows of a tile past the cache length (they may hold anything, even NaN)
         auto zero_tail = [&](uint8_t* base, int nbox, int j) {
-            const int nvalid = min(TK, L - j * TK);
+            const int nvalid = min(TK, L - (kbeg + j * TK));
             if (nvalid >= TK) return;
             const int rows = TK - nvalid;
             for (int idx = lane; idx < nbox * rows * 8; idx += 32) {
@@ -267,9 +277,9 @@ __global__ void __launch_bounds__(gta::NTHREADS, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(s_free));  // the next score tile may be written
-            const int k0 = j * TK + col0;
+            const int k0 = kbeg + j * TK + col0;
             float* sf = reinterpret_cast<float*>(sr);
-            if (j * TK + TK <= vis_end) {
+            if (kbeg + j * TK + TK <= vis_end) {
                 const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
 #pragma unroll
                 for (int c = 0; c < CW; c += 2) {
@@ -344,12 +354,24 @@ __global__ void __launch_bounds__(gta::NTHREADS, 1)
         } else {
             tc_fence_after();
             const float inv_l = l > 0.f ? 1.f / l : 0.f;
+            // only a split that holds keys of the row writes for it: its normalised partial when the row's keys
+            // span several splits, else the result
+            const int nsp_row = row_ok ? cdiv(vis_end, p.split_tokens) : 0;
+            const bool mine = row_ok && kbeg < vis_end;
+            const bool partial = mine && nsp_row > 1;
             for (int c0 = half * 16; c0 < 64 * HPG; c0 += 32) {
                 const int hh = c0 / 64;
                 uint32_t o[16];
                 tmem_ld16(tmem + lane_base + T_O + c0, o);
                 tmem_ld_wait();
-                if (row_ok) {
+                if (partial) {
+                    float4* d = reinterpret_cast<float4*>(
+                        p.part_o + ((((size_t)b * p.H + grp * HPG + hh) * p.s_q + q) * p.nsplit + split) * 64 + (c0 % 64));
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        d[e] = make_float4(__uint_as_float(o[4 * e]) * inv_l, __uint_as_float(o[4 * e + 1]) * inv_l,
+                                           __uint_as_float(o[4 * e + 2]) * inv_l, __uint_as_float(o[4 * e + 3]) * inv_l);
+                } else if (mine) {
                     uint32_t pkk[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
@@ -360,7 +382,9 @@ __global__ void __launch_bounds__(gta::NTHREADS, 1)
                     d[1] = make_uint4(pkk[4], pkk[5], pkk[6], pkk[7]);
                 }
             }
-            if (row_ok && p.lse && half == 0)
+            if (partial && half == 0)
+                p.part_lse[(((size_t)b * p.G + grp) * p.s_q + q) * p.nsplit + split] = m_ref + log2f(l);
+            else if (mine && p.lse && half == 0)
                 p.lse[((size_t)b * p.G + grp) * p.s_q + q] =
                     (l > 0.f ? m_ref + log2f(l) : -INFINITY) * 0.69314718055994530942f;
         }
@@ -370,20 +394,94 @@ __global__ void __launch_bounds__(gta::NTHREADS, 1)
     if (warp == NSW + 1) tmem_dealloc(tmem, 512);
 }
 
+// Merge of the key splits of the rows that needed several: 16 threads per (sequence, head, query) row, each
+// with 4 of its 64 values (float4 loads, many rows in flight), weights 2^(lse_i - max lse) from the group's
+// log2-domain lse of each split; writes the bf16 output and, for the first head of the group, the group's
+// natural-log lse.
+__global__ void __launch_bounds__(256) gta_combine_kernel(const GtaParams p) {
+    const size_t row = (size_t)blockIdx.x * 16 + threadIdx.x / 16;  // ((b * H + h) * s_q + q)
+    const int d4 = threadIdx.x % 16;                                 // values 4 d4 .. 4 d4 + 3
+    const size_t nrows = (size_t)p.B * p.H * p.s_q;
+    if (row >= nrows) return;
+    const int q = (int)(row % p.s_q);
+    const int h = (int)((row / p.s_q) % p.H);
+    const int b = (int)(row / ((size_t)p.H * p.s_q));
+    const int HPG = p.H / p.G, grp = h / HPG;
+    const int L = clamp_len(p.lens, b, p.Lmax, p.s_q, p.causal, p.status, false);
+    const int n_t = p.causal ? L - p.s_q + q + 1 : L;
+    const int nsp = cdiv(n_t, p.split_tokens);
+    if (nsp <= 1) return;  // written by the attention kernel
+    const float* pl = p.part_lse + (((size_t)b * p.G + grp) * p.s_q + q) * p.nsplit;
+    float M = -INFINITY;
+    for (int i = 0; i < nsp; ++i) M = fmaxf(M, pl[i]);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float wsum = 0.f;
+    const float4* po = reinterpret_cast<const float4*>(p.part_o + row * p.nsplit * 64) + d4;
+    for (int i = 0; i < nsp; ++i) {
+        const float w = exp2f(pl[i] - M);
+        const float4 v = po[(size_t)i * 16];
+        wsum += w;
+        acc = make_float4(fmaf(w, v.x, acc.x), fmaf(w, v.y, acc.y), fmaf(w, v.z, acc.z), fmaf(w, v.w, acc.w));
+    }
+    const float inv = 1.f / wsum;
+    uint2 o;
+    o.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+    o.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+    reinterpret_cast<uint2*>(p.out + row * 64)[d4] = o;
+    if (p.lse && d4 == 0 && h % HPG == 0)
+        p.lse[((size_t)b * p.G + grp) * p.s_q + q] = (M + log2f(wsum)) * 0.69314718055994530942f;
+}
+
 }  // namespace lka
 
 using namespace lka;
 
 extern "C" {
 
-size_t gta_shared_score_attn_workspace_size(int B, int G, int H, int s_q, int d_qk, int d_v, int Lmax) {
+}  // extern "C"
+
+namespace {
+
+// Key splits: one CTA per (query tile, group, sequence) and key split.  When the query tiles alone give less
+// than about two waves of CTAs (a prefill chunk over a long cached prefix), the keys are split so that they
+// do; the split size stays >= 512 keys.  The split partials (normalised O per head, lse per group) live in
+// the workspace after the status header.
+struct GtaPlan {
+    int split_tokens, nsplit;
+    size_t off_lse, off_o, ws_bytes;
+};
+
+void gta_plan(int B, int G, int H, int s_q, int Lmax, GtaPlan* pl) {
+    int st = split_tokens_knob();
+    if (st <= 0) {
+        const long long units = (long long)cdiv(s_q, gta::TQ) * G * (B > 0 ? B : 1);
+        const long long target = 2LL * sm_count();
+        const long long nsp = units >= target ? 1 : (target + units - 1) / units;
+        st = (int)((Lmax + nsp - 1) / nsp);
+        if (st < 512) st = 512;
+    }
+    st = cdiv(st, gta::TK) * gta::TK;
+    pl->split_tokens = st;
+    pl->nsplit = cdiv(Lmax, st);
+    WsCarve c;
+    pl->off_lse = pl->off_o = 0;
+    if (pl->nsplit > 1) {
+        pl->off_lse = c.take((size_t)B * G * s_q * pl->nsplit * sizeof(float));
+        pl->off_o = c.take((size_t)B * H * s_q * pl->nsplit * 64 * sizeof(float));
+    }
+    pl->ws_bytes = c.off;
+}
+
+}  // namespace
+
+extern "C" size_t gta_shared_score_attn_workspace_size(int B, int G, int H, int s_q, int d_qk, int d_v, int Lmax) {
     if (B < 0 || G < 1 || H < 1 || s_q < 1 || Lmax < 1 || H % G) return 0;
     (void)d_qk;
     (void)d_v;
-    return kWsHeaderBytes;  // status word only: one CTA covers the whole key range of its query tile
+    GtaPlan pl;
+    gta_plan(B, G, H, s_q, Lmax, &pl);
+    return pl.ws_bytes;
 }
-
-}  // extern "C"
 
 namespace {
 
@@ -410,7 +508,10 @@ lka_status_t gta_run(const void* q_g, const void* k_g, const void* v, const int3
         if (!ptr || !aligned16(ptr)) return LKA_ERR_INVALID_ARG;
     if (pg && !pg->block_table) return LKA_ERR_INVALID_ARG;
     if (!isfinite(scale)) return LKA_ERR_INVALID_ARG;
-    if (!ws || ws_bytes < kWsHeaderBytes) return LKA_ERR_WORKSPACE;
+    GtaPlan pl;
+    gta_plan(B, G, H, s_q, Lmax, &pl);
+    if (!ws || ws_bytes < pl.ws_bytes) return LKA_ERR_WORKSPACE;
+    if (!aligned16(ws)) return LKA_ERR_INVALID_ARG;
     const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const int box_rows = pg ? std::min(gta::TK, pg->page_size) : gta::TK;
     const uint64_t k_rows = pg ? (uint64_t)pg->num_pages * G * pg->page_size : (uint64_t)B * G * Lmax;
@@ -433,6 +534,10 @@ lka_status_t gta_run(const void* q_g, const void* k_g, const void* v, const int3
     p.causal = causal ? 1 : 0;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.box_rows = box_rows;
+    p.split_tokens = pl.split_tokens;
+    p.nsplit = pl.nsplit;
+    p.part_lse = pl.nsplit > 1 ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + pl.off_lse) : nullptr;
+    p.part_o = pl.nsplit > 1 ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + pl.off_o) : nullptr;
     if (pg) {
         p.block_table = pg->block_table;
         p.page_size = pg->page_size;
@@ -442,10 +547,18 @@ lka_status_t gta_run(const void* q_g, const void* k_g, const void* v, const int3
     cudaStream_t st = (cudaStream_t)stream;
     if (cudaFuncSetAttribute(gta_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gta::SMEM) != cudaSuccess)
         return LKA_ERR_CUDA;
-    dim3 grid(cdiv(s_q, gta::TQ), G, B);
-    TimedLaunch timer(st);
-    gta_attn_kernel<<<grid, gta::NTHREADS, gta::SMEM, st>>>(tq, tk, tv, p);
-    timer.stop();
+    if ((long long)cdiv(s_q, gta::TQ) * pl.nsplit >= (1ll << 31)) return LKA_ERR_UNSUPPORTED;
+    dim3 grid(cdiv(s_q, gta::TQ) * pl.nsplit, G, B);
+    {
+        TimedLaunch timer(st);
+        gta_attn_kernel<<<grid, gta::NTHREADS, gta::SMEM, st>>>(tq, tk, tv, p);
+        timer.stop();
+    }
+    if (cudaPeekAtLastError() != cudaSuccess) return LKA_ERR_CUDA;
+    if (pl.nsplit > 1) {
+        const size_t rows = (size_t)B * H * s_q;
+        gta_combine_kernel<<<(unsigned)((rows + 15) / 16), 256, 0, st>>>(p);
+    }
     return cudaPeekAtLastError() == cudaSuccess ? LKA_OK : LKA_ERR_CUDA;
 }
 

@@ -74,3 +74,23 @@ def test_gta_full_size_sampled():
     sub = {k: (v[rows].cpu() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
     ref, _ = oracle.gta(sub["q_g"], sub["k_g"], sub["v"], sub["cache_lens"], True, inp["scale"])
     assert_close(out[rows], ref, torch.bfloat16, "gta full-size sample")
+
+
+@pytest.mark.parametrize("split", [128, 384])
+def test_gta_forced_key_splits(split):
+    """Key splits (partials merged by the GTA merge kernel) on a chunked prefill: 200 queries over up to 700 cached
+    keys, ragged lengths; the result stays within tolerance of the definition."""
+    inp = synthetic.gta_inputs(65, 3, 3, 12, 64, 64, 200, 217, 700, Lmax=704)
+    prev = lka.set_split_tokens(split)
+    try:
+        run(inp, True)
+    finally:
+        lka.set_split_tokens(prev)
+
+
+def test_gta_automatic_key_split_chunked_prefill():
+    """A small grid (one query tile per group and sequence) is split along the keys automatically."""
+    inp = synthetic.gta_inputs(66, 2, 3, 12, 64, 64, 100, 1500, 3000, Lmax=3072)
+    run(inp, True)
+    nb = lka.library().gta_shared_score_attn_workspace_size(2, 3, 12, 100, 64, 64, 3072)
+    assert nb > 256  # split partials in the workspace
