@@ -681,10 +681,7 @@ def measure(wl, steps, warmup, pk, device, world, soak_s=1.0, clocks=None):
         e_end.record()
         e_end.synchronize()
         e2e_total += e_start.elapsed_time(e_end)
-    t = torch.tensor([step_ms, e2e_total / steps, kern_ms / max(1, n_timed)], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    step_ms, e2e_ms, kern_ms = t.tolist()
+    step_ms, e2e_ms, kern_ms = max_over_ranks([step_ms, e2e_total / steps, kern_ms / max(1, n_timed)], world, device)
     bound, work = wl.kernel_work(pk)
     if bound == "hbm":
         peak, unit, achieved = pk["hbm_gbs"], "GB/s", work / (kern_ms * 1e-3) / 1e9
@@ -699,6 +696,15 @@ def measure(wl, steps, warmup, pk, device, world, soak_s=1.0, clocks=None):
             "peak_source": f"{pk['source']} (MEASURED_PEAKS.json {peak_src})" if pk["source"] == "measured"
             else "fallback"}
     return dict(step_ms=step_ms, e2e_ms=e2e_ms, roofline=roof, clocks=clk)
+
+
+def max_over_ranks(values, world, device):
+    """Element-wise maximum of per-rank timings over all ranks (the slowest rank sets the job's time)."""
+    if world <= 1:
+        return list(values)
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
 
 
 def summary(wl, m, world):
