@@ -617,11 +617,26 @@ __global__ void __launch_bounds__(128) gqa_combine_kernel(const GqaParams p) {
     for (int d = 0; d < DPL; ++d) acc[d] = 0.f;
     float wsum = 0.f;
     const float* po = p.part_o + row * p.nsplit_max * D;
-    for (int i = 0; i < nsp; ++i) {
-        const float w = exp2f(pl[i] - M);
-        wsum += w;
+    // lane i holds the weight of split i (of each group of 32); 8 splits' values are loaded together
+    for (int i32 = 0; i32 < nsp; i32 += 32) {
+        const float w_lane = i32 + lane < nsp ? exp2f(pl[i32 + lane] - M) : 0.f;
+        const int n = min(32, nsp - i32);
+        for (int u0 = 0; u0 < n; u0 += 8) {
+            float v[8][DPL];
 #pragma unroll
-        for (int d = 0; d < DPL; ++d) acc[d] = fmaf(w, po[(size_t)i * D + d * 32 + lane], acc[d]);
+            for (int u = 0; u < 8; ++u)
+#pragma unroll
+                for (int d = 0; d < DPL; ++d)
+                    v[u][d] = u0 + u < n ? po[(size_t)(i32 + u0 + u) * D + d * 32 + lane] : 0.f;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const float ws = __shfl_sync(0xffffffffu, w_lane, (u0 + u) & 31);
+                const float w = u0 + u < n ? ws : 0.f;
+                wsum += w;
+#pragma unroll
+                for (int d = 0; d < DPL; ++d) acc[d] = fmaf(w, v[u][d], acc[d]);
+            }
+        }
     }
     T* out = reinterpret_cast<T*>(p.out) + row * D;
 #pragma unroll
