@@ -60,7 +60,7 @@ extern "C" {
 typedef enum {
     LKA_OK = 0,
     LKA_ERR_INVALID_ARG = 1,  /* a host-visible argument is out of range or a pointer is NULL/misaligned */
-    LKA_ERR_UNSUPPORTED = 2,  /* valid arguments this build has no kernel for (dtype, head dim, ...) */
+    LKA_ERR_UNSUPPORTED = 2,  /* valid arguments the library has no kernel for (dtype, head dim, ...) */
     LKA_ERR_WORKSPACE = 3,    /* ws is NULL or ws_bytes is below the *_workspace_size value */
     LKA_ERR_CUDA = 4,         /* a CUDA call or kernel launch failed */
     LKA_ERR_TIMEOUT = 5,      /* device status: a bounded in-kernel wait ran out (the kernel exited early) */

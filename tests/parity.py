@@ -1,6 +1,6 @@
 """Comparison helpers for the GPU-vs-oracle parity tests.
 
-Tolerances (fixed by the benchmark spec of the target):
+Tolerances (the library's accuracy target):
   fp32 inputs:  max |gpu - oracle| <= 1e-5
   bf16 inputs:  max |gpu - oracle| <= 2e-2 and ||gpu - oracle||_2 / ||oracle||_2 <= 5e-3
 with fp32 accumulation on the GPU and fp64 in the oracle, on identical inputs
