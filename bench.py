@@ -1,7 +1,7 @@
 #!/usr/bin/env python
 """Benchmark of the grouped / latent-KV attention hot path on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lka|reference] [--workload NAME]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lka|reference] [--workload NAME] [--sweep]
 
 Default workload: one GQA decode attention layer shaped like Llama-3.1-8B
 (32 query heads, 8 KV heads, d_h = 128, bf16 KV cache, batch 64, s_q = 1,
@@ -23,6 +23,10 @@ Prints ONE JSON line (rank 0).  `value` is the algorithmic HBM traffic of the
 step (every cache byte once, q read once, out written once) divided by the
 device time of a step, summed over ranks (weak scaling: every rank runs its own
 replica of the workload; there is no collective on the data path).
+
+--sweep measures the long-context decode sweep instead (batch 64, s_q 1,
+every cache 1K, 2K, ... 64K tokens, GQA layout and latent layout on the
+MQA-absorbed path) and prints one JSON line with an entry per point.
 
 --impl reference times the fp64 CPU oracle on the host cores instead (rank 0
 only), on the same workload, metric and unit; each step is a bounded sample.
@@ -228,7 +232,9 @@ class GqaDecode(Workload):
     def config(self):
         w = self.w
         return {"workload": self.name, "B": w["B"], "h_q": w["h_q"], "h_kv": w["h_kv"], "d_h": w["d"],
-                "s_q": w["s_q"], "cache_lens": f"uniform [{w['L_lo']}, {w['L_hi']}]", "causal": w["causal"],
+                "s_q": w["s_q"],
+                "cache_lens": w["L_hi"] if w["L_lo"] == w["L_hi"] else f"uniform [{w['L_lo']}, {w['L_hi']}]",
+                "causal": w["causal"],
                 "l2": "K/V cache larger than L2; L2 flushed between timed steps", "parallelism": "replicas"}
 
     def oracle_run(self, n):
@@ -606,6 +612,8 @@ WORKLOAD_CLASSES = {
     "latent_expanded_4k_sq2_b16": LatentExpanded,
     "gta_prefill_4k_b2": GtaPrefill,
 }
+# the long-context sweep (batch 64, s_q 1, cache length 1K ... 64K) over the GQA and the latent layout
+WORKLOAD_CLASSES.update({name: (GqaDecode if name.startswith("gqa") else LatentAbsorbed) for name in synthetic.SWEEP})
 EXTRAS = ["gqa_decode_llama8b_paged", "gqa_decode_llama8b_fp8", "latent_decode_4k_sq1", "latent_decode_4k_sq1_paged",
           "latent_decode_4k_sq1_fp8", "latent_decode_4k_sq2",
           "latent_sparse_16k_top2048", "latent_expanded_4k_sq2", "gta_prefill_4k",
@@ -757,6 +765,31 @@ def run_lka(args, rank, world, device):
     return line
 
 
+def run_sweep(args, rank, world, device):
+    """The long-context decode sweep: every point of synthetic.SWEEP measured like the main workload (device
+    time per step with L2 flushed between steps, the main kernel's roofline, end to end through host buffers);
+    one JSON line with one entry per point, clocks sampled over the whole sweep."""
+    pk = peaks()
+    clocks = ClockSampler(device.index if device.index is not None else 0)
+    clocks.start()
+    clocks.wait_first_sample()
+    points = {}
+    for name in synthetic.SWEEP:
+        wl = WORKLOAD_CLASSES[name](name, device)
+        m = measure(wl, min(args.steps, 10), args.warmup, pk, device, world, soak_s=0.2)
+        points[name] = summary(wl, m, world)
+        points[name]["gpu_launches"] = wl.launches * min(args.steps, 10)
+        del wl
+        torch.cuda.empty_cache()
+    clk = clocks.stop()
+    if rank != 0:
+        return None
+    return {"metric": METRIC, "mode": "long-context sweep (batch 64, s_q 1, cache length 1K-64K)",
+            "unit": "GB/s", "n_gpus": world, "steps": min(args.steps, 10), "warmup": args.warmup,
+            "higher_is_better": True, "scaling": "weak", "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) inputs, see synthetic.py)", "clocks": clk, "points": points}
+
+
 def run_reference(args, rank, world, device):
     """The oracle as it stands, on the host cores, same workload/metric/unit; rank 0 only."""
     if rank != 0:
@@ -793,6 +826,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="measure only --workload, not the other paths")
+    ap.add_argument("--sweep", action="store_true",
+                    help="measure the long-context sweep (GQA and latent layouts, cache length 1K-64K) instead")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -808,7 +843,10 @@ def main():
         backend = "nccl" if device.type == "cuda" else "gloo"
         torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
     try:
-        line = (run_lka if args.impl == "lka" else run_reference)(args, rank, world, device)
+        if args.impl == "reference":
+            line = run_reference(args, rank, world, device)
+        else:
+            line = (run_sweep if args.sweep else run_lka)(args, rank, world, device)
         if line is not None:
             print(json.dumps(line), flush=True)
     finally:

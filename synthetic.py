@@ -310,6 +310,13 @@ def sweep_workload(kind: str, L: int) -> dict:
                 causal=True)
 
 
+# The long-context decode sweep: batch 64, s_q 1, cache length 1K ... 64K tokens for every sequence, over the
+# GQA layout (32 query / 8 KV heads, d_h 128) and the latent layout (128 heads, 512 + 64 latent values).
+SWEEP_LENGTHS = (1024, 2048, 4096, 8192, 16384, 32768, 65536)
+SWEEP = {f"{kind}_sweep_{L // 1024}k": sweep_workload(kind, L) for kind in ("gqa", "latent") for L in SWEEP_LENGTHS}
+WORKLOADS.update(SWEEP)
+
+
 def make(w: dict, device="cpu", dtype=torch.bfloat16) -> dict:
     """Materialise a workload description from WORKLOADS / sweep_workload."""
     if w["kind"] == "gqa":

@@ -51,3 +51,20 @@ def test_counters_match_per_token_forms():
     assert costs.gqa_flops([4], 8, 64, 4, True) == (1 + 2 + 3 + 4) * 8 * 4 * 64
     assert costs.gta_flops([3], 3, 12, 64, 64, 3, True) == 6 * (3 * 128 + 12 * 128)
     assert costs.gqa_bytes([10], 32, 8, 128, 1) == 10 * 8 * 256 * 2 + 32 * 128 * 2 * 2
+
+
+def test_long_context_sweep_points():
+    # batch 64, s_q 1, equal cache lengths 1K ... 64K: GQA (32 / 8 heads, d_h 128) reads 64 * L * 4096 cache
+    # bytes, the latent layout 64 * L * 1152 bytes and does 64 * L * 128 * (2 * 576 + 2 * 512) FLOPs
+    import synthetic
+
+    assert synthetic.SWEEP_LENGTHS == tuple(1024 * 2 ** i for i in range(7))
+    for L in synthetic.SWEEP_LENGTHS:
+        g = synthetic.SWEEP[f"gqa_sweep_{L // 1024}k"]
+        lat = synthetic.SWEEP[f"latent_sweep_{L // 1024}k"]
+        assert (g["B"], g["h_q"], g["h_kv"], g["d"], g["s_q"], g["L_lo"], g["L_hi"]) == (64, 32, 8, 128, 1, L, L)
+        assert (lat["B"], lat["h_q"], lat["r_kv"], lat["d_r"], lat["s_q"], lat["L_hi"]) == (64, 128, 512, 64, 1, L)
+        lens = [L] * 64
+        assert costs.gqa_bytes(lens, 32, 8, 128, 1) == 64 * L * 4096 + 64 * 32 * 128 * 2 * 2
+        assert costs.latent_core_flops(lens, 128, 512, 64, 1, True) == 64 * L * 278528
+    assert costs.gqa_bytes([65536] * 64, 32, 8, 128, 1) / 1e9 == pytest.approx(17.18, abs=0.01)
