@@ -75,17 +75,28 @@ static lka_status_t gqa_plan(int B, int h_q, int h_kv, int s_q, int d_h, int Lma
     if (fp8kv && pl->rb > 4) pl->rb = 4;
     pl->n_rb = cdiv(R, pl->rb);
     if ((long long)h_kv * pl->n_rb > 65535 || B > 65535) return LKA_ERR_UNSUPPORTED;
-    pl->tile = fp8kv ? gqa_fp8_tile_tokens(d_h, pl->rb) : gqa_tile_tokens(dtype_bytes, d_h, pl->rb);
+    int per_sm = 1;  // resident CTAs per SM of the kernel instance
+    pl->tile = fp8kv ? gqa_fp8_tile_tokens(d_h, pl->rb, &per_sm) : gqa_tile_tokens(dtype_bytes, d_h, pl->rb, &per_sm);
     if (pl->tile <= 0) return LKA_ERR_UNSUPPORTED;
     int st = split_tokens_knob();
     if (st <= 0) {
-        // aim at ~12 waves of 2 resident CTAs per SM over the worst-case (Lmax) work
+        // One CTA per (sequence, KV head, row block, key split).  Pick the split count n that minimises
+        // waves x (tiles per split + a fixed cost per CTA of about two tiles: filling the TMA ring at the
+        // start, merging the warps and writing at the end), for the worst case of every sequence at Lmax:
+        // ceil(units * n / slots) * (ceil(Lmax_tiles / n) + 2).  Ties go to fewer splits.
         const long long units = (long long)(B > 0 ? B : 1) * h_kv * pl->n_rb;
-        const long long target = (long long)sm_count() * 2 * 12;
-        long long nsp = (target + units - 1) / units;
-        if (nsp < 1) nsp = 1;
-        st = (int)((Lmax + nsp - 1) / nsp);
-        if (st < 4 * pl->tile) st = 4 * pl->tile;
+        const long long slots = (long long)sm_count() * per_sm;
+        const int lt = cdiv(Lmax, pl->tile);
+        int best = 1;
+        long long best_cost = -1;
+        for (int n = 1; n <= lt && n <= 256; ++n) {
+            const long long cost = ((units * n + slots - 1) / slots) * (cdiv(lt, n) + 2);
+            if (best_cost < 0 || cost < best_cost) {
+                best_cost = cost;
+                best = n;
+            }
+        }
+        st = cdiv(lt, best) * pl->tile;
     }
     st = cdiv(st, pl->tile) * pl->tile;
     pl->split_tokens = st;

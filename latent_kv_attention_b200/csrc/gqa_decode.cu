@@ -678,9 +678,12 @@ cudaError_t gqa_combine_launch(const GqaParams& p, int dtype_bytes, int d, cudaS
     return cudaPeekAtLastError();
 }
 
-int gqa_tile_tokens(int dtype_bytes, int d, int rb) {
-#define LKA_TILE_CASE(T, DD, R) \
-    if (dtype_bytes == (int)sizeof(T) && d == DD && rb == R) return GqaCfg<T, DD, R>::T_TILE;
+int gqa_tile_tokens(int dtype_bytes, int d, int rb, int* ctas_per_sm) {
+#define LKA_TILE_CASE(T, DD, R)                                  \
+    if (dtype_bytes == (int)sizeof(T) && d == DD && rb == R) {   \
+        if (ctas_per_sm) *ctas_per_sm = GqaCfg<T, DD, R>::MINB; \
+        return GqaCfg<T, DD, R>::T_TILE;                         \
+    }
     LKA_TILE_CASE(__nv_bfloat16, 64, 1) LKA_TILE_CASE(__nv_bfloat16, 64, 2) LKA_TILE_CASE(__nv_bfloat16, 64, 4)
     LKA_TILE_CASE(__nv_bfloat16, 64, 8)
     LKA_TILE_CASE(__nv_bfloat16, 128, 1) LKA_TILE_CASE(__nv_bfloat16, 128, 2) LKA_TILE_CASE(__nv_bfloat16, 128, 4)
@@ -714,9 +717,12 @@ cudaError_t gqa_decode_launch(const CUtensorMap& tk, const CUtensorMap& tv, cons
     return cudaErrorInvalidValue;
 }
 
-int gqa_fp8_tile_tokens(int d, int rb) {
-#define LKA_TILE_CASE(DD, R) \
-    if (d == DD && rb == R) return GqaCfg<e4m3, DD, R>::T_TILE;
+int gqa_fp8_tile_tokens(int d, int rb, int* ctas_per_sm) {
+#define LKA_TILE_CASE(DD, R)                                       \
+    if (d == DD && rb == R) {                                      \
+        if (ctas_per_sm) *ctas_per_sm = GqaCfg<e4m3, DD, R>::MINB; \
+        return GqaCfg<e4m3, DD, R>::T_TILE;                        \
+    }
     LKA_TILE_CASE(128, 1) LKA_TILE_CASE(128, 2) LKA_TILE_CASE(128, 4)
     LKA_TILE_CASE(256, 1) LKA_TILE_CASE(256, 2) LKA_TILE_CASE(256, 4)
 #undef LKA_TILE_CASE

@@ -31,13 +31,13 @@ struct GqaParams {
 
 // The e4m3-cache instances (bf16 q/out, d in {128, 256}, rb <= 4: a 16-byte chunk holds 16 values, so more rows
 // per CTA would not fit the query slice in registers).
-int gqa_fp8_tile_tokens(int d, int rb);
+int gqa_fp8_tile_tokens(int d, int rb, int* ctas_per_sm);
 cudaError_t gqa_fp8_decode_launch(const CUtensorMap& tk, const CUtensorMap& tv, const GqaParams& p, int d, int rb,
                                   int nsplit, cudaStream_t st);
 // Merge of split partials for rows [B*h_q*s_q] of D values (rows needing one split are skipped).
 cudaError_t gqa_combine_launch(const GqaParams& p, int dtype_bytes, int d, cudaStream_t st);
-// Tokens per TMA tile of the kernel instance (0 if the instance does not exist).
-int gqa_tile_tokens(int dtype_bytes, int d, int rb);
+// Tokens per TMA tile of the kernel instance (0 if the instance does not exist) and its resident CTAs per SM.
+int gqa_tile_tokens(int dtype_bytes, int d, int rb, int* ctas_per_sm);
 // Launches the decode kernel (grid nsplit x h_kv*n_rb x B) and, when nsplit > 1, the merge.
 cudaError_t gqa_decode_launch(const CUtensorMap& tk, const CUtensorMap& tv, const GqaParams& p, int dtype_bytes,
                               int d, int rb, int nsplit, cudaStream_t st);
