@@ -82,16 +82,20 @@ static lka_status_t gqa_plan(int B, int h_q, int h_kv, int s_q, int d_h, int Lma
     if (st <= 0) {
         // One CTA per (sequence, KV head, row block, key split).  Pick the split count n that minimises
         // waves x (tiles per split + a fixed cost per CTA of about two tiles: filling the TMA ring at the
-        // start, merging the warps and writing at the end), for the worst case of every sequence at Lmax:
-        // ceil(units * n / slots) * (ceil(Lmax_tiles / n) + 2).  Ties go to fewer splits.
-        const long long units = (long long)(B > 0 ? B : 1) * h_kv * pl->n_rb;
-        const long long slots = (long long)sm_count() * per_sm;
+        // start, merging the warps and writing at the end), sizing splits for every sequence at Lmax.
+        // With w = units * n / slots, the waves are max(ceil(w), w + 1/4): whole waves when the lengths
+        // are equal, and some tail beyond the average when they differ (CTAs of short sequences end early
+        // and the longest splits run last), which a plan of one long wave cannot absorb.  Ties go to fewer
+        // splits.
+        const double units = (double)(B > 0 ? B : 1) * h_kv * pl->n_rb;
+        const double slots = (double)sm_count() * per_sm;
         const int lt = cdiv(Lmax, pl->tile);
         int best = 1;
-        long long best_cost = -1;
+        double best_cost = -1.0;
         for (int n = 1; n <= lt && n <= 256; ++n) {
-            const long long cost = ((units * n + slots - 1) / slots) * (cdiv(lt, n) + 2);
-            if (best_cost < 0 || cost < best_cost) {
+            const double w = units * n / slots;
+            const double cost = fmax(ceil(w - 1e-9), w + 0.25) * (cdiv(lt, n) + 2);
+            if (best_cost < 0.0 || cost < best_cost - 1e-9) {
                 best_cost = cost;
                 best = n;
             }
