@@ -18,8 +18,11 @@
 // rank 1: [256, 576), i.e. its 256 value columns plus the rest of its score
 // range; the 64 values [256, 320) are read by both ranks, the second read
 // coming from L2).  The two score partials are exchanged through distributed
-// shared memory (st.async with mbarrier transaction counts) and summed
-// identically on both sides, so both run the same online softmax.
+// shared memory, each rank sending its partial rounded to fp16 (half the
+// shared-memory and DSMEM bytes of fp32): a rank adds the peer's rounded
+// partial to its own fp32 one, so the two ranks' scores differ by that rounding
+// (at most 2^-11 of the peer's partial) and each normalises its half of the
+// output with its own row sums.
 //
 // Each tcgen05.mma with M = 128 and K = 16 takes about the same time whatever
 // its N (up to 256), so the tiles are as wide as memory allows: 64 tokens.  The
@@ -80,12 +83,13 @@ constexpr int NCW = 2;          // converter warps (FP8 cache only)
 constexpr int CW = NT / 2;      // score columns per softmax warp
 constexpr int NTHREADS = 32 * (NSW + 2 + NXW);
 constexpr int NTHREADS_F8 = NTHREADS + 32 * NCW;
-constexpr int XROW = CW * 4;    // bytes of one row of one half of an exchanged partial
-constexpr int XBUF = 2 * 128 * XROW;  // [half][head row][CW] fp32; each warp's block is contiguous
+constexpr int XROW = CW * 2;    // bytes of one row of one half of an exchanged partial (fp16)
+constexpr int XBUF = 2 * 128 * XROW;  // [half][head row][CW] fp16; each warp's block is contiguous
+constexpr int XSPACE = 2 * XBUF;      // room reserved for each of the exchange buffer and the outbox
 constexpr int OFF_KV = 0;
 constexpr int OFF_X = OFF_KV + NST * STAGE;
-constexpr int OFF_OUT = OFF_X + XBUF;  // this CTA's partial on its way to the peer
-constexpr int OFF_BAR = OFF_OUT + XBUF;
+constexpr int OFF_OUT = OFF_X + XSPACE;  // this CTA's partial on its way to the peer
+constexpr int OFF_BAR = OFF_OUT + XSPACE;
 // The query slice is staged once through shared memory that is idle at the start: the last ring
 // stage, the exchange buffer and the first part of the outbox (five 128-row x 64-value boxes).
 constexpr int NQB = 5;
@@ -412,7 +416,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
         // the peer sent; the sending (outbox store, proxy fence, waits, copies) is off their path.
         const int qx = warp & 3;
         const uint32_t lane_base = (uint32_t)(qx * 32) << 16;
-        const int sw = lane & 7;
+        const int sw = (lane >> 1) & 3;  // 16-byte chunk swizzle of a 64-byte row: 8 lanes hit 8 bank groups
         int xblk[2];
         uint32_t xrem[2], xfull_rem[2];
 #pragma unroll
@@ -438,10 +442,14 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
             for (int hf = 0; hf < 2; ++hf) {
                 uint8_t* orow = smem + OFF_OUT + xblk[hf] + lane * XROW;
 #pragma unroll
-                for (int c = 0; c < CW / 4; ++c)
-                    *reinterpret_cast<uint4*>(orow + ((c ^ sw) << 4)) =
-                        make_uint4(own[hf * CW + 4 * c], own[hf * CW + 4 * c + 1], own[hf * CW + 4 * c + 2],
-                                   own[hf * CW + 4 * c + 3]);
+                for (int c = 0; c < CW / 8; ++c) {
+                    const uint32_t* o8 = own + hf * CW + 8 * c;
+                    *reinterpret_cast<uint4*>(orow + ((c ^ sw) << 4)) = make_uint4(
+                        pack_f16x2(__uint_as_float(o8[0]), __uint_as_float(o8[1])),
+                        pack_f16x2(__uint_as_float(o8[2]), __uint_as_float(o8[3])),
+                        pack_f16x2(__uint_as_float(o8[4]), __uint_as_float(o8[5])),
+                        pack_f16x2(__uint_as_float(o8[6]), __uint_as_float(o8[7])));
+                }
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the copy engine
             __syncwarp();
@@ -471,7 +479,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
         const int blk = half * 128 * XROW + qw * 32 * XROW;  // this warp's block in the exchange buffer
         // the peer's "buffer free" barrier of this warp's block
         const uint32_t xempty_rem = mapa_peer(smem_u32(&xempty[warp]), peer);
-        const int sw = lane & 7;
+        const int sw = (lane >> 1) & 3;  // the sender's chunk swizzle
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
         if (n_tiles > 0) {
@@ -545,16 +553,17 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
             float s[CW];
             const uint8_t* xr = smem + OFF_X + blk + lane * XROW;
 #pragma unroll
-            for (int c = 0; c < CW / 4; ++c) {
-                const float4 v = *reinterpret_cast<const float4*>(xr + ((c ^ sw) << 4));
-                const float2 a = __fadd2_rn(make_float2(__uint_as_float(cur[4 * c]), __uint_as_float(cur[4 * c + 1])),
-                                            make_float2(v.x, v.y));
-                const float2 bb = __fadd2_rn(
-                    make_float2(__uint_as_float(cur[4 * c + 2]), __uint_as_float(cur[4 * c + 3])), make_float2(v.z, v.w));
-                s[4 * c] = a.x;
-                s[4 * c + 1] = a.y;
-                s[4 * c + 2] = bb.x;
-                s[4 * c + 3] = bb.y;
+            for (int c = 0; c < CW / 8; ++c) {
+                const uint4 v = *reinterpret_cast<const uint4*>(xr + ((c ^ sw) << 4));
+                const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float2 pf = __half22float2(*reinterpret_cast<const __half2*>(&vw[k]));
+                    const float2 a = __fadd2_rn(
+                        make_float2(__uint_as_float(cur[8 * c + 2 * k]), __uint_as_float(cur[8 * c + 2 * k + 1])), pf);
+                    s[8 * c + 2 * k] = a.x;
+                    s[8 * c + 2 * k + 1] = a.y;
+                }
             }
             __syncwarp();
             if (lane == 0 && i + 1 < n_tiles) {
