@@ -22,7 +22,10 @@
 // shared-memory and DSMEM bytes of fp32): a rank adds the peer's rounded
 // partial to its own fp32 one, so the two ranks' scores differ by that rounding
 // (at most 2^-11 of the peer's partial) and each normalises its half of the
-// output with its own row sums.
+// output with its own row sums.  The rounding is absolute in the score, so it
+// grows with the partial's magnitude (a partial logit of 20 after scaling moves
+// by at most 0.01), and a partial beyond the fp16 range (65504 before scaling)
+// overflows: the exchange assumes query and latent values of ordinary size.
 //
 // Each tcgen05.mma with M = 128 and K = 16 takes about the same time whatever
 // its N (up to 256), so the tiles are as wide as memory allows: 64 tokens.  The
