@@ -82,3 +82,17 @@ def test_expand_cache_matches_oracle():
     assert_close(kc, rkc, torch.bfloat16, "kc")
     assert_close(vc, rvc, torch.bfloat16, "vc")
     assert np.array_equal(kr.cpu().double().numpy(), rkr)  # a copy: exact
+
+
+@pytest.mark.parametrize("mul", [2, 4])
+def test_absorbed_peaked_scores(mul):
+    """Queries scaled up (by a power of two, exactly) make the softmax peakier and the score partials that the
+    two CTAs of a cluster exchange larger; the result stays within the bf16 tolerance up to 4x the workload's
+    query magnitude (beyond that the bf16 rounding of P, not the exchange, exceeds the max-abs bound)."""
+    inp = synthetic.latent_inputs(47, 2, 128, 8, 128, 512, 64, 2, 500, 900, Lmax=900)
+    q_c, q_r = inp["q_c"] * mul, inp["q_r"] * mul
+    out = lka.latent_absorbed_attn(q_c.to(DEV), q_r.to(DEV), inp["w_uk"].to(DEV), inp["w_uv"].to(DEV),
+                                   inp["latent"].to(DEV), inp["cache_lens"].to(DEV), causal=True, scale=inp["scale"])
+    ref, _ = oracle.latent_absorbed(q_c, q_r, inp["w_uk"], inp["w_uv"], inp["latent"], inp["cache_lens"], True,
+                                    inp["scale"])
+    assert_close(out, ref, torch.bfloat16, f"latent, queries x{mul}")
