@@ -3,7 +3,9 @@
 Each case edits one plausible mistake into a copy of oracle.c (a wrong group
 index, an off-by-one causal bound, a dropped scale or RoPE term, a transposed
 weight, the wrong up-projection, a missing log, another head's values, a
-missing normalisation), compiles it into a temporary library and runs one of
+missing normalisation of the merge or of the probabilities, a cache expansion
+that copies the wrong RoPE key or uses the key weight for the value), compiles
+it into a temporary library and runs one of
 the pins of test_oracle_pins.py against it: the pin must fail.  This shows the
 pins can tell the definition from its likely corruptions.
 """
@@ -54,6 +56,18 @@ MUTATIONS = {
         "        out[d] = a / z;",
         "        out[d] = a;",
         lambda: pins.test_merge_of_disjoint_partials_equals_full_attention()),
+    "probs_unnormalised": (
+        "    for (int j = 0; j < n; ++j) p[j] = exp(p[j] - m) / z;",
+        "    for (int j = 0; j < n; ++j) p[j] = exp(p[j] - m);",
+        lambda: pins.test_probabilities_sum_to_one_and_reproduce_output()),
+    "expand_cache_rope_from_latent": (
+        "c->kr[((long)b * c->Lmax + j) * c->d_r + e] = cj[c->r_kv + e];",
+        "c->kr[((long)b * c->Lmax + j) * c->d_r + e] = cj[e];",
+        lambda: pins.test_expand_cache_then_gqa_equals_latent()),
+    "expand_cache_value_weight": (
+        "                av += Wv[(long)e * c->r_kv + r] * cj[r];\n            }\n            ko[e] = ak;",
+        "                av += Wk[(long)e * c->r_kv + r] * cj[r];\n            }\n            ko[e] = ak;",
+        lambda: pins.test_expand_cache_then_gqa_equals_latent()),
 }
 
 
