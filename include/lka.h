@@ -82,6 +82,11 @@ typedef enum { LKA_BF16 = 0, LKA_FP32 = 1 } lka_dtype_t;
 /*  log-sum-exp; the split partials live in ws.                              */
 /* ------------------------------------------------------------------------ */
 LKA_API size_t gqa_attn_workspace_size(int B, int h_q, int h_kv, int s_q, int d_h, int Lmax);
+/* Key splits per sequence that gqa_attn plans for these sizes and dtype (the grid is splits x h_kv x row
+ * blocks x B CTAs; a sequence shorter than Lmax uses only the splits its keys reach), or 0 for arguments
+ * gqa_attn rejects.  The plan depends only on the sizes, the dtype, the device's SM count and the split
+ * knob (lka_set_split_tokens); host-only, no device work. */
+LKA_API int gqa_attn_split_count(int B, int h_q, int h_kv, int s_q, int d_h, int Lmax, lka_dtype_t dtype);
 LKA_API lka_status_t gqa_attn(const void *q, const void *k, const void *v, const int32_t *cache_lens, void *out,
                       float *lse, int B, int h_q, int h_kv, int s_q, int d_h, int Lmax, int causal, float scale,
                       lka_dtype_t dtype, void *ws, size_t ws_bytes, void *stream);

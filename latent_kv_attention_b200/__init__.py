@@ -44,6 +44,7 @@ _P, _Z, _I, _F = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_float
 _FP = ctypes.POINTER(ctypes.c_float)
 SIGNATURES = {
     "gqa_attn_workspace_size": (_Z, [_I] * 6),
+    "gqa_attn_split_count": (_I, [_I] * 7),
     "gqa_attn": (_I, [_P] * 6 + [_I] * 7 + [_F, _I, _P, _Z, _P]),
     "gqa_attn_noalloc": (_I, [_P] * 6 + [_I] * 7 + [_F, _I, _P]),
     "gqa_attn_fp8kv_workspace_size": (_Z, [_I] * 6),
@@ -527,6 +528,11 @@ def clear_status(device=None):
     device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     ws = workspaces.get(256, device)
     _check("lka_clear_status", library().lka_clear_status(_ptr(ws), _stream_ptr()))
+
+
+def gqa_split_count(B: int, h_q: int, h_kv: int, s_q: int, d: int, Lmax: int, dtype=torch.bfloat16) -> int:
+    """Key splits per sequence that gqa_attn plans for these sizes (0 if it would reject them); host-only."""
+    return int(library().gqa_attn_split_count(B, h_q, h_kv, s_q, d, Lmax, _DT[dtype]))
 
 
 def set_split_tokens(tokens: int) -> int:

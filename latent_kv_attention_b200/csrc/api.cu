@@ -203,6 +203,12 @@ size_t gqa_attn_workspace_size(int B, int h_q, int h_kv, int s_q, int d_h, int L
     return gqa_ws_size(B, h_q, h_kv, s_q, d_h, Lmax, false);
 }
 
+int gqa_attn_split_count(int B, int h_q, int h_kv, int s_q, int d_h, int Lmax, lka_dtype_t dtype) {
+    if (dtype != LKA_BF16 && dtype != LKA_FP32) return 0;
+    GqaPlan pl;
+    return gqa_plan(B, h_q, h_kv, s_q, d_h, Lmax, dtype == LKA_BF16 ? 2 : 4, &pl) == LKA_OK ? pl.nsplit : 0;
+}
+
 }  // extern "C"
 
 namespace lka {

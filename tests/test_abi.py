@@ -81,3 +81,21 @@ def test_workspace_sizes(lib):
 def test_split_knob_roundtrip(lib):
     prev = lka.set_split_tokens(512)
     assert lka.set_split_tokens(prev) == 512
+
+
+def test_gqa_split_plan(lib):
+    """The GQA split count chosen by the wave-cost rule (host logic; 148 SMs, two resident CTAs per SM for the
+    d_h 128 bf16 kernel): the smallest max(ceil(w), w + 1/4) * (tiles per split + 2) with w = CTAs / 296."""
+    prev = lka.set_split_tokens(0)
+    try:
+        assert lka.gqa_split_count(64, 32, 8, 1, 128, 8192) == 4    # Llama-3.1-8B decode layer, 2048-key splits
+        assert lka.gqa_split_count(16, 32, 8, 1, 128, 8192) == 4    # not one long wave of 256 CTAs
+        assert lka.gqa_split_count(64, 32, 8, 1, 128, 1024) == 1    # 512 CTAs of 16 tiles
+        assert lka.gqa_split_count(64, 32, 8, 1, 128, 4096) == 4
+        assert lka.gqa_split_count(64, 32, 8, 1, 128, 65536) == 8
+        assert lka.gqa_split_count(1, 8, 2, 1, 64, 17) == 1
+        assert lka.gqa_split_count(1, 6, 4, 1, 64, 17) == 0         # invalid grouping
+        lka.set_split_tokens(512)
+        assert lka.gqa_split_count(64, 32, 8, 1, 128, 8192) == 16   # the knob: splits of at most 512 keys
+    finally:
+        lka.set_split_tokens(prev)
