@@ -125,13 +125,6 @@ __device__ __forceinline__ uint32_t mapa_peer(uint32_t saddr, uint32_t peer) {
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-__device__ __forceinline__ void st_async_v4(uint32_t raddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
-                                            uint32_t rbar) {
-    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
-                     raddr),
-                 "r"(a), "r"(b), "r"(c), "r"(d), "r"(rbar)
-                 : "memory");
-}
 // Bulk copy of `bytes` from this CTA's shared memory to the peer's (cluster address `dst`),
 // completing `bytes` of the transaction count of the peer's barrier `rbar`.
 __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t rbar) {
