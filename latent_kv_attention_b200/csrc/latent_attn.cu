@@ -145,9 +145,9 @@ __device__ __forceinline__ void remote_arrive(uint32_t rbar) {
     asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(rbar) : "memory");
 }
 // Waits on the exchange barriers use the default (CTA-scope) acquire: the peer's partial scores
-// arrive through st.async, whose bytes complete the local barrier's transaction count, and the
+// arrive through bulk copies, whose bytes complete the local barrier's transaction count, and the
 // peer's "buffer free" arrival (release at cluster scope) is only ever followed by new remote
-// stores, never by reads of data the peer produced.
+// copies, never by reads of data the peer produced.
 
 // 14 warps (16 with an FP8 cache): an SM sub-partition holds up to 4 of them, so at most
 // 16384 / (4 * 32) = 128 registers each
