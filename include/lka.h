@@ -65,7 +65,9 @@ typedef enum {
     LKA_ERR_CUDA = 4,         /* a CUDA call or kernel launch failed */
     LKA_ERR_TIMEOUT = 5,      /* device status: a bounded in-kernel wait ran out (the kernel exited early) */
     LKA_ERR_BAD_LENGTH = 6,   /* device status: a cache_lens entry was outside its range and was clamped */
-    LKA_ERR_BAD_PAGE = 7      /* device status: a block-table entry a call needed was outside the page pool */
+    LKA_ERR_BAD_PAGE = 7,     /* device status: a block-table entry a call needed was outside the page pool */
+    LKA_ERR_RANGE = 8         /* device status: an intermediate value left the range of its internal format and
+                                 was saturated (the output is finite but not accurate); see (b) */
 } lka_status_t;
 
 typedef enum { LKA_BF16 = 0, LKA_FP32 = 1 } lka_dtype_t;
@@ -136,15 +138,21 @@ LKA_API lka_status_t gqa_attn_fp8kv(const void *q, const void *k, const void *v,
  * array inside the library (held by every GPU that loads the library until
  * the process exits).  This call allocates nothing.  Its first call on a
  * device looks up that array's device address (cudaGetSymbolAddress), so make
- * the first call on each device before any stream capture.  Returns
- * LKA_ERR_WORKSPACE when the workspace gqa_attn_workspace_size reports for the
- * sizes exceeds 16 MiB.  All calls share the one array: calls that overlap on
- * the GPU (other streams, other host threads) race and must be serialised by
- * the caller.  Device-side status flags (LKA_ERR_TIMEOUT, LKA_ERR_BAD_LENGTH)
- * are not reported by this variant. */
+ * the first call on each device before any stream capture; the address is
+ * cached per device ordinal, so do not use this variant on a device after
+ * cudaDeviceReset.  Returns LKA_ERR_WORKSPACE, enqueuing nothing, when the
+ * split plan of the call's sizes and dtype needs more than 16 MiB.  All calls
+ * share the one array: calls that overlap on the GPU (other streams, other
+ * host threads) race and must be serialised by the caller.  Device-side
+ * status flags (LKA_ERR_TIMEOUT, LKA_ERR_BAD_LENGTH) accumulate in the
+ * array's status word; read them with gqa_attn_noalloc_status. */
 LKA_API lka_status_t gqa_attn_noalloc(const void *q, const void *k, const void *v, const int32_t *cache_lens,
                               void *out, float *lse, int B, int h_q, int h_kv, int s_q, int d_h, int Lmax,
                               int causal, float scale, lka_dtype_t dtype, void *stream);
+/* The device status of the no-allocation variant on the current device: synchronises `stream`, reads the
+ * status word of the library's scratch array (flags raised by gqa_attn_noalloc calls since the last read,
+ * returned like lka_device_status), then enqueues its reset on `stream`.  Allocates nothing. */
+LKA_API lka_status_t gqa_attn_noalloc_status(void *stream);
 
 /* ------------------------------------------------------------------------ */
 /* (b) GQLA MQA-absorbed latent attention  [GQLA sec. 1, sec. 3.1 eq. (1),  */
@@ -161,6 +169,10 @@ LKA_API lka_status_t gqa_attn_noalloc(const void *q, const void *k, const void *
 /*   q_c [B,h_q,s_q,d_h]  q_r [B,h_q,s_q,d_r]  w_uk, w_uv [g,d_h,r_kv]       */
 /*   latent [B,Lmax,r_kv+d_r]  out [B,h_q,s_q,d_h]  lse [B,h_q,s_q] or NULL  */
 /*  Supported: bf16, r_kv = 512, d_r = 64, d_h = 128, h_q = 128, s_q <= 2.   */
+/*  The score contraction is split over two CTAs whose partial scores are    */
+/*  exchanged as fp16 after multiplication by scale*log2(e); a scaled        */
+/*  partial beyond the fp16 range (|x| > 65504) is saturated and raises      */
+/*  LKA_ERR_RANGE in the workspace status (finite, inaccurate output).       */
 /* ------------------------------------------------------------------------ */
 LKA_API size_t latent_absorbed_attn_workspace_size(int B, int h_q, int g, int s_q, int d_h, int r_kv, int d_r, int Lmax);
 LKA_API lka_status_t latent_absorbed_attn(const void *q_c, const void *q_r, const void *w_uk, const void *w_uv,
@@ -310,20 +322,22 @@ LKA_API lka_status_t latent_expand_cache(const void *latent, const void *w_uk, c
 /* ------------------------------------------------------------------------ */
 /* Helpers                                                                  */
 /* ------------------------------------------------------------------------ */
-/* Synchronises `stream`, then returns the sticky status word of workspace ws:
- * LKA_OK, LKA_ERR_TIMEOUT (takes precedence), LKA_ERR_BAD_LENGTH or LKA_ERR_BAD_PAGE. */
+/* Synchronises `stream`, then returns the sticky status word of workspace ws: LKA_OK, or the first raised
+ * flag in the order LKA_ERR_TIMEOUT, LKA_ERR_BAD_LENGTH, LKA_ERR_BAD_PAGE, LKA_ERR_RANGE. */
 LKA_API lka_status_t lka_device_status(const void *ws, void *stream);
 /* Enqueues a reset of the workspace status word to LKA_OK on `stream`. */
 LKA_API lka_status_t lka_clear_status(void *ws, void *stream);
 /* Human-readable name of a status code (static string, never NULL). */
 LKA_API const char *lka_status_string(lka_status_t status);
-/* Process-wide split size (KV tokens per CTA) for the split-KV kernels; 0 restores the automatic choice.
- * A tuning and test knob: results do not depend on it beyond rounding.  Returns the previous value. */
+/* Split size (KV tokens per CTA) for the split-KV kernels of the calls made FROM THE CALLING HOST THREAD;
+ * 0 restores the automatic choice.  A tuning and test knob: results do not depend on it beyond rounding,
+ * and calls made from other threads keep their own setting (default 0).  Returns the thread's previous value. */
 LKA_API int lka_set_split_tokens(int tokens);
-/* Timing hook for benchmarks: lka_kernel_timing(1) discards earlier records and starts recording a pair of
- * CUDA events around the main (dominant) kernel of every later entry-point call, on that call's stream;
- * lka_kernel_timing(0) stops recording.  lka_kernel_timing_read waits for the recorded events and returns the
- * number of timed launches and their summed duration in milliseconds. */
+/* Timing hook for benchmarks, per host thread: lka_kernel_timing(1) discards the calling thread's earlier
+ * records and starts recording a pair of CUDA events around the main (dominant) kernel of every later
+ * entry-point call made from that thread, on that call's stream; lka_kernel_timing(0) stops recording.
+ * lka_kernel_timing_read waits for the calling thread's recorded events and returns the number of timed
+ * launches and their summed duration in milliseconds.  Calls from other threads are never timed by it. */
 LKA_API lka_status_t lka_kernel_timing(int enable);
 LKA_API lka_status_t lka_kernel_timing_read(int *launches, double *total_ms);
 /* Self-test of the bounded in-kernel wait: launches one CTA that waits on a barrier nobody arrives at,

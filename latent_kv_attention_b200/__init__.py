@@ -36,7 +36,7 @@ LIB_PATH = os.path.join(_HERE, "liblka.so")
 
 LKA_OK = 0
 STATUS_NAMES = {0: "LKA_OK", 1: "LKA_ERR_INVALID_ARG", 2: "LKA_ERR_UNSUPPORTED", 3: "LKA_ERR_WORKSPACE",
-                4: "LKA_ERR_CUDA", 5: "LKA_ERR_TIMEOUT", 6: "LKA_ERR_BAD_LENGTH", 7: "LKA_ERR_BAD_PAGE"}
+                4: "LKA_ERR_CUDA", 5: "LKA_ERR_TIMEOUT", 6: "LKA_ERR_BAD_LENGTH", 7: "LKA_ERR_BAD_PAGE", 8: "LKA_ERR_RANGE"}
 _DT = {torch.bfloat16: 0, torch.float32: 1}
 
 # Every symbol include/lka.h declares, with its ctypes signature (restype, argtypes).
@@ -47,6 +47,7 @@ SIGNATURES = {
     "gqa_attn_split_count": (_I, [_I] * 7),
     "gqa_attn": (_I, [_P] * 6 + [_I] * 7 + [_F, _I, _P, _Z, _P]),
     "gqa_attn_noalloc": (_I, [_P] * 6 + [_I] * 7 + [_F, _I, _P]),
+    "gqa_attn_noalloc_status": (_I, [_P]),
     "gqa_attn_fp8kv_workspace_size": (_Z, [_I] * 6),
     "gqa_attn_fp8kv": (_I, [_P] * 8 + [_I] * 7 + [_F, _P, _Z, _P]),
     "gqa_attn_paged_workspace_size": (_Z, [_I] * 7),

@@ -15,8 +15,10 @@
 
 namespace lka {
 
-static std::atomic<int> g_split_tokens{0};
-int split_tokens_knob() { return g_split_tokens.load(std::memory_order_relaxed); }
+// Test and benchmark hooks.  Both are per host thread: a setting made on one thread never changes the
+// plan or the launches of calls made on another, so concurrent callers stay independent.
+static thread_local int t_split_tokens = 0;
+int split_tokens_knob() { return t_split_tokens; }
 
 // ---------------------------------------------------------------- kernel timing hook
 struct TimingRegistry {
@@ -26,7 +28,7 @@ struct TimingRegistry {
     std::vector<std::pair<cudaEvent_t, cudaEvent_t>> pending;
 };
 static TimingRegistry& timing_reg() {
-    static TimingRegistry r;
+    static thread_local TimingRegistry r;
     return r;
 }
 bool kernel_timing_on() { return timing_reg().on.load(std::memory_order_relaxed); }
@@ -119,6 +121,14 @@ static lka_status_t gqa_plan(int B, int h_q, int h_kv, int s_q, int d_h, int Lma
 
 static lka_status_t launch_status(cudaError_t e) { return e == cudaSuccess ? LKA_OK : LKA_ERR_CUDA; }
 
+lka_status_t status_from_word(uint32_t st) {
+    if (st & kDevTimeout) return LKA_ERR_TIMEOUT;
+    if (st & kDevBadLength) return LKA_ERR_BAD_LENGTH;
+    if (st & kDevBadPage) return LKA_ERR_BAD_PAGE;
+    if (st & kDevRange) return LKA_ERR_RANGE;
+    return LKA_OK;
+}
+
 // Workspace bytes of a GQA call; the size does not depend on the dtype beyond the supported head dims: plan
 // with bf16, then fp32, and take the larger.
 static size_t gqa_ws_size(int B, int h_q, int h_kv, int s_q, int d_h, int Lmax, bool paged) {
@@ -149,11 +159,16 @@ const char* lka_status_string(lka_status_t s) {
         case LKA_ERR_TIMEOUT: return "LKA_ERR_TIMEOUT";
         case LKA_ERR_BAD_LENGTH: return "LKA_ERR_BAD_LENGTH";
         case LKA_ERR_BAD_PAGE: return "LKA_ERR_BAD_PAGE";
+        case LKA_ERR_RANGE: return "LKA_ERR_RANGE";
     }
     return "LKA_ERR_UNKNOWN";
 }
 
-int lka_set_split_tokens(int tokens) { return g_split_tokens.exchange(tokens < 0 ? 0 : tokens); }
+int lka_set_split_tokens(int tokens) {
+    const int prev = t_split_tokens;
+    t_split_tokens = tokens < 0 ? 0 : tokens;
+    return prev;
+}
 
 lka_status_t lka_kernel_timing(int enable) {
     auto& r = timing_reg();
@@ -188,10 +203,7 @@ lka_status_t lka_device_status(const void* ws, void* stream) {
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return LKA_ERR_CUDA;
     uint32_t st = 0;
     if (cudaMemcpy(&st, ws, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess) return LKA_ERR_CUDA;
-    if (st & kDevTimeout) return LKA_ERR_TIMEOUT;
-    if (st & kDevBadLength) return LKA_ERR_BAD_LENGTH;
-    if (st & kDevBadPage) return LKA_ERR_BAD_PAGE;
-    return LKA_OK;
+    return status_from_word(st);
 }
 
 lka_status_t lka_clear_status(void* ws, void* stream) {

@@ -21,6 +21,7 @@ constexpr size_t kWsHeaderBytes = 256;
 constexpr uint32_t kDevTimeout = 1u;    // a bounded wait ran out
 constexpr uint32_t kDevBadLength = 2u;  // a cache_lens entry was clamped
 constexpr uint32_t kDevBadPage = 4u;    // a block-table entry outside the page pool was replaced
+constexpr uint32_t kDevRange = 8u;      // an intermediate exceeded the range of its internal format (saturated)
 
 // Default limit of a bounded wait (nanoseconds of %globaltimer).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;

@@ -27,7 +27,10 @@ constexpr size_t kNoAllocScratchBytes = 16u << 20;
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 // The array's name is only a host-side stand-in on the host: its device address
-// is looked up once per device, with that device current.
+// is looked up once per device, with that device current, and cached.  The cache
+// is keyed by the device ordinal only: after cudaDeviceReset on a device the
+// library's module is loaded again and the cached address is stale, so this
+// variant must not be used on a device after it has been reset.
 static std::atomic<uint8_t*> g_noalloc_addr[64];
 
 static uint8_t* noalloc_scratch_address() {
@@ -47,19 +50,33 @@ extern "C" lka_status_t gqa_attn_noalloc(const void* q, const void* k, const voi
                                          void* out, float* lse, int B, int h_q, int h_kv, int s_q, int d_h, int Lmax,
                                          int causal, float scale, lka_dtype_t dtype, void* stream) {
     if (dtype != LKA_BF16 && dtype != LKA_FP32) return LKA_ERR_UNSUPPORTED;
-    // the workspace gqa_attn would need for this call must fit in the static scratch
-    const size_t need = gqa_attn_workspace_size(B, h_q, h_kv, s_q, d_h, Lmax);
-    if (need == 0) {
+    if (gqa_attn_workspace_size(B, h_q, h_kv, s_q, d_h, Lmax) == 0) {
         // invalid or unsupported arguments: let gqa_attn report which, without touching the scratch
         return gqa_attn(q, k, v, cache_lens, out, lse, B, h_q, h_kv, s_q, d_h, Lmax, causal, scale, dtype, nullptr,
                         0, stream);
     }
-    if (need > lka::kNoAllocScratchBytes) return LKA_ERR_WORKSPACE;  // larger than the built-in 16 MiB
     uint8_t* ws = lka::noalloc_scratch_address();
     if (!ws) return LKA_ERR_CUDA;
-    // Nothing in the scratch has to start at zero: every split partial the merge reads is written
-    // by the same call first.  The status word at its head only accumulates device-side flags
-    // (timeouts, clamped lengths) that this variant does not report.
+    // gqa_attn checks the scratch size against the split plan of this call's dtype and returns
+    // LKA_ERR_WORKSPACE, before enqueuing anything, when the plan needs more than the array holds.
+    // Nothing in the scratch has to start at zero: every split partial the merge reads is written by the
+    // same call first.  The status word at its head accumulates the device-side flags (timeouts, clamped
+    // lengths) until gqa_attn_noalloc_status reads and clears it.
     return gqa_attn(q, k, v, cache_lens, out, lse, B, h_q, h_kv, s_q, d_h, Lmax, causal, scale, dtype, ws,
                     lka::kNoAllocScratchBytes, stream);
+}
+
+extern "C" lka_status_t gqa_attn_noalloc_status(void* stream) {
+    uint8_t* ws = lka::noalloc_scratch_address();
+    if (!ws) return LKA_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t word = 0;
+    // the flags of every call enqueued before this one on `stream` (and, through the one shared array, of
+    // any other call that has completed), then an enqueued reset for the calls that follow
+    if (cudaStreamSynchronize(st) != cudaSuccess) return LKA_ERR_CUDA;
+    if (cudaMemcpyAsync(&word, ws, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return LKA_ERR_CUDA;
+    if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), st) != cudaSuccess) return LKA_ERR_CUDA;
+    return lka::status_from_word(word);
 }

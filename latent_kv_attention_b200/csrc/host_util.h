@@ -79,11 +79,15 @@ inline int sm_count() {
     return v;
 }
 
-// Process-wide split size knob (0 = automatic).
+// The status code of a workspace status word (the first raised flag in the order timeout, clamped length,
+// bad page, range).
+lka_status_t status_from_word(uint32_t word);
+
+// Split size knob of the calling host thread (0 = automatic).
 int split_tokens_knob();
 
 // Optional timing of the main kernel of each entry point (see
-// lka_kernel_timing): when enabled, a pair of CUDA events is recorded on the
+// lka_kernel_timing): when enabled on the calling thread, a pair of CUDA events is recorded on the
 // launch stream around that kernel.  The events come from a pool that is only
 // created, never device memory.
 bool kernel_timing_on();

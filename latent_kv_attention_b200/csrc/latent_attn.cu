@@ -18,14 +18,16 @@
 // rank 1: [256, 576), i.e. its 256 value columns plus the rest of its score
 // range; the 64 values [256, 320) are read by both ranks, the second read
 // coming from L2).  The two score partials are exchanged through distributed
-// shared memory, each rank sending its partial rounded to fp16 (half the
-// shared-memory and DSMEM bytes of fp32): a rank adds the peer's rounded
-// partial to its own fp32 one, so the two ranks' scores differ by that rounding
-// (at most 2^-11 of the peer's partial) and each normalises its half of the
-// output with its own row sums.  The rounding is absolute in the score, so it
-// grows with the partial's magnitude (a partial logit of 20 after scaling moves
-// by at most 0.01), and a partial beyond the fp16 range (65504 before scaling)
-// overflows: the exchange assumes query and latent values of ordinary size.
+// shared memory, each rank sending its partial multiplied by scale * log2 e
+// and rounded to fp16 (half the shared-memory and DSMEM bytes of fp32): a rank
+// adds the peer's rounded partial to its own fp32 one, so the two ranks' scores
+// differ by that rounding (at most 2^-11 of the peer's scaled partial) and each
+// normalises its half of the output with its own row sums.  The rounding is
+// absolute in the score, so it grows with the partial's magnitude (a scaled
+// partial of 20 moves by at most 0.01).  A scaled partial beyond the fp16
+// range (|x| > 65504, a softmax that is one-hot many times over) is saturated
+// and raises kDevRange in the status word (LKA_ERR_RANGE): the output stays
+// finite but is not accurate.
 //
 // Each tcgen05.mma with M = 128 and K = 16 takes about the same time whatever
 // its N (up to 256), so the tiles are as wide as memory allows: 64 tokens.  The
@@ -110,6 +112,7 @@ constexpr uint32_t T_S = 448;        // NT fp32 score partials
 static_assert(T_Q + KSTEPS * 8 <= T_P && T_P + NT / 2 <= T_R && T_R + 6 <= T_S && T_S + NT <= 512,
               "tensor memory budget");
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 domain
+constexpr float kF16Max = 65504.f;         // largest finite fp16 value
 }  // namespace lat
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -434,19 +437,27 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
             if (lane == 0) mbar_arrive(smem_u32(s_free));
             if (lane == 0) bulk_wait_read();  // the previous copies have read the outbox
             __syncwarp();
+            // the partial goes out already scaled into the log2 domain (scale * log2 e), saturated to the
+            // fp16 range; a partial beyond it (|scaled partial| > 65504) raises kDevRange
+            float amax = 0.f;
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
                 uint8_t* orow = smem + OFF_OUT + xblk[hf] + lane * XROW;
 #pragma unroll
                 for (int c = 0; c < CW / 8; ++c) {
                     const uint32_t* o8 = own + hf * CW + 8 * c;
-                    *reinterpret_cast<uint4*>(orow + ((c ^ sw) << 4)) = make_uint4(
-                        pack_f16x2(__uint_as_float(o8[0]), __uint_as_float(o8[1])),
-                        pack_f16x2(__uint_as_float(o8[2]), __uint_as_float(o8[3])),
-                        pack_f16x2(__uint_as_float(o8[4]), __uint_as_float(o8[5])),
-                        pack_f16x2(__uint_as_float(o8[6]), __uint_as_float(o8[7])));
+                    uint32_t w4[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float y0 = __uint_as_float(o8[2 * e]) * p.scale_log2;
+                        const float y1 = __uint_as_float(o8[2 * e + 1]) * p.scale_log2;
+                        amax = fmaxf(amax, fmaxf(fabsf(y0), fabsf(y1)));
+                        w4[e] = pack_f16x2(fminf(fmaxf(y0, -kF16Max), kF16Max), fminf(fmaxf(y1, -kF16Max), kF16Max));
+                    }
+                    *reinterpret_cast<uint4*>(orow + ((c ^ sw) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
                 }
             }
+            if (__any_sync(0xffffffffu, !(amax <= kF16Max)) && lane == 0) atomicOr(p.status, kDevRange);
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the copy engine
             __syncwarp();
             if (lane == 0) {
@@ -554,9 +565,11 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
                 const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
+                    // own partial scaled into the log2 domain plus the peer's (sent scaled)
                     const float2 pf = __half22float2(*reinterpret_cast<const __half2*>(&vw[k]));
-                    const float2 a = __fadd2_rn(
-                        make_float2(__uint_as_float(cur[8 * c + 2 * k]), __uint_as_float(cur[8 * c + 2 * k + 1])), pf);
+                    const float2 a = __ffma2_rn(
+                        make_float2(__uint_as_float(cur[8 * c + 2 * k]), __uint_as_float(cur[8 * c + 2 * k + 1])),
+                        make_float2(p.scale_log2, p.scale_log2), pf);
                     s[8 * c + 2 * k] = a.x;
                     s[8 * c + 2 * k + 1] = a.y;
                 }
@@ -570,17 +583,9 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
             if (i + 1 < n_tiles) fetch(i + 1);
             // ---- mask, online softmax ----
             const int k0 = kbeg + i * NT + col0;
-            const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
-            if (kbeg + (i + 1) * NT <= kend) {
+            if (kbeg + (i + 1) * NT > kend) {
 #pragma unroll
-                for (int j = 0; j < CW; j += 2) {
-                    const float2 v = __fmul2_rn(make_float2(s[j], s[j + 1]), sc2);
-                    s[j] = v.x;
-                    s[j + 1] = v.y;
-                }
-            } else {
-#pragma unroll
-                for (int j = 0; j < CW; ++j) s[j] = (k0 + j < kend) ? s[j] * p.scale_log2 : -INFINITY;
+                for (int j = 0; j < CW; ++j) s[j] = (k0 + j < kend) ? s[j] : -INFINITY;
             }
             // row maximum of the whole tile: this warp's half and the partner warp's half
             float mx = tree_max<CW>(s);

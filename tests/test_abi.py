@@ -83,6 +83,26 @@ def test_split_knob_roundtrip(lib):
     assert lka.set_split_tokens(prev) == 512
 
 
+def test_split_knob_is_per_thread(lib):
+    """The split knob only changes the plans of calls made from the thread that set it: a caller on another
+    thread keeps the automatic plan (the boundary holds no state shared between concurrent callers)."""
+    import threading
+
+    auto = lka.gqa_split_count(64, 32, 8, 1, 128, 8192)
+    seen = {}
+
+    def other():
+        seen["before"] = lka.gqa_split_count(64, 32, 8, 1, 128, 8192)
+        lka.set_split_tokens(512)
+        seen["set"] = lka.gqa_split_count(64, 32, 8, 1, 128, 8192)
+
+    t = threading.Thread(target=other)
+    t.start()
+    t.join()
+    assert seen == {"before": auto, "set": 16}
+    assert lka.gqa_split_count(64, 32, 8, 1, 128, 8192) == auto  # this thread's plan is untouched
+
+
 def test_gqa_split_plan(lib):
     """The GQA split count chosen by the wave-cost rule (host logic; 148 SMs, two resident CTAs per SM for the
     d_h 128 bf16 kernel): the smallest max(ceil(w), w + 1/4) * (tiles per split + 2) with w = CTAs / 296."""

@@ -96,3 +96,19 @@ def test_absorbed_peaked_scores(mul):
     ref, _ = oracle.latent_absorbed(q_c, q_r, inp["w_uk"], inp["w_uv"], inp["latent"], inp["cache_lens"], True,
                                     inp["scale"])
     assert_close(out, ref, torch.bfloat16, f"latent, queries x{mul}")
+
+
+def test_absorbed_exchange_beyond_fp16_range_is_reported():
+    """The two CTAs of a cluster exchange their partial scores as fp16 after multiplying them by
+    scale * log2(e).  Inputs whose scaled partials exceed the fp16 range (here: queries and latent x64, scale 1)
+    must not turn into NaN silently: the partial is saturated, the output stays finite and the workspace status
+    reports LKA_ERR_RANGE."""
+    inp = synthetic.latent_inputs(48, 2, 128, 8, 128, 512, 64, 1, 200, 300, Lmax=300)
+    q_c, q_r, latent = inp["q_c"] * 64, inp["q_r"] * 64, inp["latent"] * 64
+    out = lka.latent_absorbed_attn(q_c.to(DEV), q_r.to(DEV), inp["w_uk"].to(DEV), inp["w_uv"].to(DEV),
+                                   latent.to(DEV), inp["cache_lens"].to(DEV), causal=True, scale=1.0)
+    assert lka.device_status() == 8, lka.status_string(lka.device_status())  # LKA_ERR_RANGE
+    assert torch.isfinite(out).all()
+    lka.clear_status()
+    # ordinary magnitudes raise nothing
+    absorbed_case(49, 2, 1, 200, 300, 300)

@@ -4,9 +4,10 @@ Callers that cannot allocate device memory (a plugin handed only its input and
 output buffers, or code where the host framework forbids device allocations)
 cannot pass gqa_attn its workspace; gqa_attn_noalloc keeps the split-KV scratch
 in a fixed 16 MiB device array inside the library instead.  Its result must
-match gqa_attn's within the parity tolerance, on consecutive calls that reuse
-the scratch the previous call left behind.  The file name makes pytest collect
-it last.
+match the fp64 oracle within the parity tolerance, and gqa_attn's, on
+consecutive calls that reuse the scratch the previous call left behind; its
+device-side flags are read back through gqa_attn_noalloc_status.  The file
+name makes pytest collect it last.
 """
 import ctypes
 
@@ -14,11 +15,16 @@ import pytest
 import torch
 
 import latent_kv_attention_b200 as lka
+import oracle
 import synthetic
-from parity import assert_close
+from parity import assert_close, assert_lse_close
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
 
 def call_noalloc(q, k, v, lens, out, lse, causal, scale):
@@ -27,22 +33,49 @@ def call_noalloc(q, k, v, lens, out, lse, causal, scale):
     P = lambda t: ctypes.c_void_p(t.data_ptr()) if t is not None else None  # noqa: E731
     dtype = 0 if q.dtype == torch.bfloat16 else 1
     return lka.library().gqa_attn_noalloc(P(q), P(k), P(v), P(lens), P(out), P(lse), B, h_q, h_kv, s_q, d, Lmax,
-                                          int(causal), float(scale), dtype,
-                                          ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+                                          int(causal), float(scale), dtype, _stream())
 
 
-def test_noalloc_matches_gqa_attn_on_two_calls_in_a_row():
+def noalloc_status():
+    return lka.library().gqa_attn_noalloc_status(_stream())
+
+
+def test_noalloc_matches_oracle_and_gqa_attn_on_two_calls_in_a_row():
+    noalloc_status()  # start from a clear status word
     for seed, s_q in ((71, 1), (72, 2)):  # the second call reuses the scratch the first one left behind
-        inp = synthetic.gqa_inputs(seed, 4, 32, 8, 128, s_q, 300, 2000, Lmax=2048, device=DEV)
-        ref, ref_lse = lka.gqa_attn(inp["q"], inp["k"], inp["v"], inp["cache_lens"], causal=True,
-                                    scale=inp["scale"], return_lse=True)
-        out = torch.empty_like(inp["q"])
-        lse = torch.empty(ref_lse.shape, dtype=torch.float32, device=DEV)
-        rc = call_noalloc(inp["q"], inp["k"], inp["v"], inp["cache_lens"], out, lse, True, inp["scale"])
+        inp = synthetic.gqa_inputs(seed, 4, 32, 8, 128, s_q, 300, 2000, Lmax=2048)
+        # the call is split along the keys, so the scratch's partials are written and merged
+        assert lka.gqa_split_count(4, 32, 8, s_q, 128, 2048) > 1
+        q, k, v, lens = (inp[n].to(DEV) for n in ("q", "k", "v", "cache_lens"))
+        out = torch.empty_like(q)
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=DEV)
+        rc = call_noalloc(q, k, v, lens, out, lse, True, inp["scale"])
         assert rc == 0, lka.status_string(rc)
         torch.cuda.synchronize()
-        assert_close(out, ref, torch.bfloat16, f"noalloc call seed {seed}")
-        assert (lse - ref_lse).abs().max().item() <= 1e-4
+        ref, ref_lse = oracle.gqa(inp["q"], inp["k"], inp["v"], inp["cache_lens"], True, inp["scale"])
+        assert_close(out, ref, torch.bfloat16, f"noalloc call seed {seed} vs oracle")
+        assert_lse_close(lse, ref_lse, torch.bfloat16, f"noalloc lse seed {seed} vs oracle")
+        ws_out, ws_lse = lka.gqa_attn(q, k, v, lens, causal=True, scale=inp["scale"], return_lse=True)
+        assert_close(out, ws_out, torch.bfloat16, f"noalloc call seed {seed} vs gqa_attn")
+        assert (lse - ws_lse).abs().max().item() <= 1e-4
+    assert noalloc_status() == 0
+
+
+def test_noalloc_reports_a_clamped_length_through_its_status():
+    noalloc_status()
+    inp = synthetic.gqa_inputs(73, 2, 32, 8, 128, 1, 100, 400, Lmax=512)
+    lens = inp["cache_lens"].clone()
+    lens[1] = 100000  # beyond Lmax: clamped to Lmax on the device and flagged
+    q, k, v = (inp[n].to(DEV) for n in ("q", "k", "v"))
+    out = torch.empty_like(q)
+    rc = call_noalloc(q, k, v, lens.to(DEV), out, None, True, inp["scale"])
+    assert rc == 0  # the device-side clamp cannot be reported by the launch itself
+    assert noalloc_status() == 6  # LKA_ERR_BAD_LENGTH, then cleared
+    assert noalloc_status() == 0
+    # the clamped sequence attends over all Lmax keys
+    lens[1] = 512
+    ref, _ = oracle.gqa(inp["q"], inp["k"], inp["v"], lens, True, inp["scale"])
+    assert_close(out, ref, torch.bfloat16, "noalloc with a clamped length")
 
 
 def test_noalloc_rejects_scratch_beyond_16_mib():
