@@ -762,6 +762,19 @@ def run_lka(args, rank, world, device):
         cb = oracle_sample(wl, args.cpu_seconds)
         line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
         line["cpu_baseline"]["value"] = round(cb["value"], 4)
+    # The MQA-absorbed latent decode (s_q 1 and 2) summarised last, so that a reader keeping only the end of
+    # the line still sees both roofline fractions.
+    lat = {}
+    for name, key in (("latent_decode_4k_sq1", "s_q1"), ("latent_decode_4k_sq2", "s_q2")):
+        x = extras.get(name)
+        if x is None and name == args.workload:
+            x = {"ms_per_step": round(m["step_ms"], 4), "roofline": m["roofline"]}
+        if x is not None:
+            r = x["roofline"]
+            lat[key] = {"frac": r["frac"], "bound": r["bound"], "achieved": r["achieved"], "unit": r["unit"],
+                        "launch_ms": r["launch_ms"], "step_ms": x["ms_per_step"]}
+    if lat:
+        line["latent_absorbed"] = lat
     return line
 
 
