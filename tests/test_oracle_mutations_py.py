@@ -30,6 +30,13 @@ MUTATIONS = {
     # the query token's own key left out of its sparse selection (strict causal bound)
     "sparse_causal_bound": ("if 0 <= j <= last]", "if 0 <= j < last]",
                             pins.test_sparse_oracle_full_selection_equals_dense_causal),
+    # the per-group sparse path with the shared RoPE key's term dropped from the scores
+    "expanded_sparse_rope_dropped": ("o, l = gqa(np.concatenate([qs[0], qs[1]], -1), key, val, lens, False, scale)",
+                                     "o, l = gqa(np.concatenate([qs[0], 0 * qs[1]], -1), key, val, lens, False, scale)",
+                                     pins.test_expanded_sparse_full_selection_equals_latent_definition),
+    # the per-group sparse path attending to the expanded keys as values
+    "expanded_sparse_value_is_key": ("val = np.concatenate([cs[1], np.zeros(", "val = np.concatenate([cs[0], np.zeros(",
+                                     pins.test_expanded_sparse_full_selection_equals_latent_definition),
     # padding entries (-1) not skipped: they index the last cache row
     "sparse_padding_kept": ("if 0 <= j <= last]", "if j <= last]",
                             pins.test_sparse_oracle_subset_equals_dense_over_the_subset_and_skips_junk),

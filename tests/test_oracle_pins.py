@@ -423,6 +423,27 @@ def test_sparse_oracle_subset_equals_dense_over_the_subset_and_skips_junk():
         assert np.allclose(out[b], ref[0, ..., :16], atol=1e-13) and np.allclose(lse[b], ref_lse[0], atol=1e-13)
 
 
+def test_expanded_sparse_full_selection_equals_latent_definition():
+    """GQLA section 3.1: the per-group GQA path over the expanded cache computes the latent attention of eq. (1).
+    A selection listing every position a query may see (in a scrambled order, causal, s_q = 2) makes the sparse
+    composition the dense per-group path, so expanded_sparse over the caches of latent_expand_cache must equal
+    latent_expanded -- eq. (1) evaluated from the latent and the weights, not a restatement of the composition."""
+    s_q = 2
+    inp = synthetic.latent_inputs(76, 2, 32, 2, 16, 32, 8, s_q, 5, 20, dtype=torch.float32)
+    lens = inp["cache_lens"]
+    kc, vc, kr = oracle.latent_expand_cache(inp["latent"], inp["w_uk"], inp["w_uv"])
+    gen = torch.Generator().manual_seed(77)
+    idx = torch.full((2, s_q, int(lens.max())), -1, dtype=torch.int32)
+    for b in range(2):
+        for t in range(s_q):
+            n = int(lens[b]) - s_q + t + 1
+            idx[b, t, :n] = torch.randperm(n, generator=gen).to(torch.int32)
+    out, lse = oracle.expanded_sparse(inp["q_c"], inp["q_r"], kc, vc, kr, idx, lens, inp["scale"])
+    ref, ref_lse = oracle.latent_expanded(inp["q_c"], inp["q_r"], inp["w_uk"], inp["w_uv"], inp["latent"], lens, True,
+                                          inp["scale"])
+    assert np.allclose(out, ref, rtol=1e-11, atol=1e-12) and np.allclose(lse, ref_lse, rtol=1e-12, atol=1e-12)
+
+
 def test_sparse_oracle_empty_selection():
     inp = synthetic.latent_inputs(75, 1, 16, 1, 16, 32, 8, 1, 9, 9, dtype=torch.float32)
     idx = torch.full((1, 1, 4), -1, dtype=torch.int32)
