@@ -298,6 +298,42 @@ class GqaDecodeFp8(GqaDecode):
         return c
 
 
+class GqaPrefill(GqaDecode):
+    """gqa_attn causal prefill of the Llama-3.1-8B layer (4096 queries over their own cache): the tensor-core
+    prefill kernel (128-query x 128-key tiles, tcgen05 MMAs, one CTA per query tile and head)."""
+
+    kernel = "gta_attn_kernel"
+    src = ("latent_kv_attention_b200/csrc/gta_attn.cu", "latent_kv_attention_b200/csrc/tc.cuh",
+           "latent_kv_attention_b200/csrc/common.cuh")
+    bound = "tensor"
+    oracle_n = 1
+
+    def kernel_work(self, pk):
+        return "tensor", self.flops
+
+    def setup_device(self):
+        super().setup_device()
+        self.launches = 1  # 32 query tiles x 32 heads x 2 sequences fill the GPU: no key splits to merge
+
+    def config(self):
+        c = super().config()
+        c["l2"] = "inputs 134 MB (q, k, v); L2 flushed between timed steps"
+        return c
+
+    def oracle_run(self, n):
+        import oracle
+
+        w, i = self.w, self.inp
+        # a bounded sample: the last 256 query positions of the first sequence (each sees 3841 .. 4096 keys)
+        t0 = w["s_q"] - 256
+        q = i["q"][:1, :, t0:].cpu().double()
+        k, v = i["k"][:1].cpu().double(), i["v"][:1].cpu().double()
+        lens = torch.tensor([w["L_hi"]], dtype=torch.int32)
+        fn = lambda: oracle.gqa(q, k, v, lens, True, i["scale"])  # noqa: E731
+        nbytes = costs.gqa_bytes([w["L_hi"]], w["h_q"], w["h_kv"], w["d"], 256)
+        return fn, nbytes, oracle.threads_used(0, w["h_q"]), "last 256 queries of the first sequence"
+
+
 class LatentAbsorbed(Workload):
     """latent_absorbed_attn over the GQLA/MLA decode batch: absorb GEMM, latent attention, up-projection."""
 
@@ -607,6 +643,7 @@ WORKLOAD_CLASSES = {
     "latent_expanded_4k_sq2": LatentExpanded,
     "gta_prefill_4k": GtaPrefill,
     "gta_chunked_prefill_4k_paged": GtaChunkedPrefillPaged,
+    "gqa_prefill_llama8b_4k": GqaPrefill,
     # smaller cases for full ncu captures
     "latent_decode_4k_sq1_b32": LatentAbsorbed,
     "latent_expanded_4k_sq2_b16": LatentExpanded,
@@ -617,7 +654,7 @@ WORKLOAD_CLASSES.update({name: (GqaDecode if name.startswith("gqa") else LatentA
 EXTRAS = ["gqa_decode_llama8b_paged", "gqa_decode_llama8b_fp8", "latent_decode_4k_sq1", "latent_decode_4k_sq1_paged",
           "latent_decode_4k_sq1_fp8", "latent_decode_4k_sq2",
           "latent_sparse_16k_top2048", "latent_expanded_4k_sq2", "gta_prefill_4k",
-          "gta_chunked_prefill_4k_paged"]
+          "gta_chunked_prefill_4k_paged", "gqa_prefill_llama8b_4k"]
 
 
 def oracle_sample(wl, target_s: float):

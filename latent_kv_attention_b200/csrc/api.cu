@@ -129,18 +129,30 @@ lka_status_t status_from_word(uint32_t st) {
     return LKA_OK;
 }
 
+// Whether a GQA call runs the tensor-core prefill (bf16, d = 128, at least kGqaPrefillMinQueries queries).
+static bool gqa_tc_prefill(int dtype_bytes, int d_h, int s_q, bool fp8kv) {
+    return !fp8kv && dtype_bytes == 2 && d_h == 128 && s_q >= kGqaPrefillMinQueries;
+}
+
 // Workspace bytes of a GQA call; the size does not depend on the dtype beyond the supported head dims: plan
-// with bf16, then fp32, and take the larger.
+// with bf16 (the split-KV kernel, or the tensor-core prefill), then fp32, and take the larger.
 static size_t gqa_ws_size(int B, int h_q, int h_kv, int s_q, int d_h, int Lmax, bool paged) {
+    if (B < 0 || h_q < 1 || h_kv < 1 || s_q < 1 || Lmax < 1 || h_q % h_kv) return 0;
+    size_t best = 0;
+    bool any = false;
     GqaPlan pl;
-    if (gqa_plan(B, h_q, h_kv, s_q, d_h, Lmax, 2, &pl, paged) == LKA_OK) {
-        GqaPlan pf;
-        if (gqa_plan(B, h_q, h_kv, s_q, d_h, Lmax, 4, &pf, paged) == LKA_OK && pf.ws_bytes > pl.ws_bytes)
-            return pf.ws_bytes;
-        return pl.ws_bytes;
+    if (gqa_tc_prefill(2, d_h, s_q, false)) {
+        best = gqa_prefill_ws_bytes(B, h_q, s_q, Lmax);
+        any = true;
+    } else if (gqa_plan(B, h_q, h_kv, s_q, d_h, Lmax, 2, &pl, paged) == LKA_OK) {
+        best = pl.ws_bytes;
+        any = true;
     }
-    if (gqa_plan(B, h_q, h_kv, s_q, d_h, Lmax, 4, &pl, paged) == LKA_OK) return pl.ws_bytes;
-    return 0;
+    if (gqa_plan(B, h_q, h_kv, s_q, d_h, Lmax, 4, &pl, paged) == LKA_OK) {
+        best = pl.ws_bytes > best ? pl.ws_bytes : best;
+        any = true;
+    }
+    return any ? best : 0;
 }
 
 }  // namespace lka
@@ -239,6 +251,20 @@ static lka_status_t gqa_run(const void* q, const void* k, const void* v, const i
     if (fp8kv && dtype != LKA_BF16) return LKA_ERR_UNSUPPORTED;
     const int eb = dtype == LKA_BF16 ? 2 : 4;
     const int kvb = fp8kv ? 1 : eb;  // bytes of one cache element
+    if (gqa_tc_prefill(eb, d_h, s_q, fp8kv)) {
+        // prefill: the tensor-core kernel, one CTA per (128-query tile, query head, sequence, key split)
+        if (B < 0 || h_q < 1 || h_kv < 1 || Lmax < 1 || h_q % h_kv) return LKA_ERR_INVALID_ARG;
+        if (!pg && (long long)B * h_kv * Lmax >= (1ll << 31)) return LKA_ERR_UNSUPPORTED;
+        if (B == 0) return LKA_OK;
+        if (!q || !k || !v || !cache_lens || !out) return LKA_ERR_INVALID_ARG;
+        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(cache_lens))
+            return LKA_ERR_INVALID_ARG;
+        if (!isfinite(scale)) return LKA_ERR_INVALID_ARG;
+        if (ws && !aligned16(ws)) return LKA_ERR_INVALID_ARG;
+        return gqa_prefill_tc(q, k, v, cache_lens, out, lse, B, h_q, h_kv, s_q, Lmax, causal, scale, ws, ws_bytes,
+                              (cudaStream_t)stream, pg ? pg->block_table : nullptr, pg ? pg->page_size : 0,
+                              pg ? pg->max_pages : 0, pg ? pg->num_pages : 0);
+    }
     GqaPlan pl;
     lka_status_t s = gqa_plan(B, h_q, h_kv, s_q, d_h, Lmax, eb, &pl, pg != nullptr, fp8kv);
     if (s != LKA_OK) return s;

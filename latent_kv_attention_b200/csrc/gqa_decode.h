@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/lka.h"
+
 namespace lka {
 
 struct GqaParams {
@@ -41,5 +43,16 @@ int gqa_tile_tokens(int dtype_bytes, int d, int rb, int* ctas_per_sm);
 // Launches the decode kernel (grid nsplit x h_kv*n_rb x B) and, when nsplit > 1, the merge.
 cudaError_t gqa_decode_launch(const CUtensorMap& tk, const CUtensorMap& tv, const GqaParams& p, int dtype_bytes,
                               int d, int rb, int nsplit, cudaStream_t st);
+
+// Causal (or full) prefill on the tensor cores for bf16, d = 128 (gta_attn.cu): one CTA per (128-query tile,
+// query head, sequence, key split), keys and values of the head's KV head h / (h_q / h_kv); paged caches when
+// block_table != nullptr (pools [num_pages, h_kv, page_size, 128]).  gqa_prefill_ws_bytes is its workspace.
+size_t gqa_prefill_ws_bytes(int B, int h_q, int s_q, int Lmax);
+lka_status_t gqa_prefill_tc(const void* q, const void* k, const void* v, const int32_t* cache_lens, void* out,
+                            float* lse, int B, int h_q, int h_kv, int s_q, int Lmax, int causal, float scale, void* ws,
+                            size_t ws_bytes, cudaStream_t st, const int32_t* block_table, int page_size, int max_pages,
+                            int num_pages);
+// Query tokens from which gqa_attn (bf16, d = 128) runs the tensor-core prefill instead of the split-KV kernel.
+constexpr int kGqaPrefillMinQueries = 64;
 
 }  // namespace lka

@@ -24,6 +24,13 @@
 // take the two 64-key halves of the tile and combine their row maxima through
 // shared memory), with lazy rescaling (the running maximum only moves when it
 // grows by more than 2^8); P goes to tensor memory.
+//
+// The same pipeline runs the causal prefill of grouped-query attention
+// ("Grouped Query Attention (GQA)" glossary page, "How GQA works"): every query
+// head is then a group of its own, its keys and values are those of its KV head
+// floor(h / (h_q / h_kv)), and the head dimension d = 128 is two 64-column
+// boxes of the query and key tiles and two 64-column blocks of the value tile
+// (the N = 128 of P*V).
 #include "common.cuh"
 #include "host_util.h"
 #include "tc.cuh"
@@ -44,35 +51,50 @@ struct GtaParams {
     // key splits (nsplit > 1): split k covers keys [k * split_tokens, (k + 1) * split_tokens); a row whose keys
     // need more than one split writes normalised fp32 partials that gta_combine_kernel merges
     int split_tokens, nsplit;
-    float* part_o;    // [B * H * s_q][nsplit][64]
+    float* part_o;    // [B * H * s_q][nsplit][64]  (GQA: [B * h_q * s_q][nsplit][d])
     float* part_lse;  // [B * G * s_q][nsplit] log2 domain (one per group: the score matrix is the group's)
+    // GQA mode: G = H = h_q query heads, h_kv KV heads; head h reads KV head h / kv_ratio
+    int h_kv, kv_ratio;
 };
 
 namespace gta {
 constexpr int TQ = 128, TK = 128;
-constexpr int NSK = 4;              // K ring depth: key tiles are released right after S = Q K^T
 constexpr int NSV = 2;              // V ring depth: value tiles live until their P*V MMAs complete
 constexpr int BOX = TK * 128;       // 128 rows x 64 bf16
-constexpr int VSTAGE = 4 * BOX;     // up to 4 heads' value tiles
-constexpr int OFF_Q = 0;
-constexpr int OFF_K = BOX;
-constexpr int OFF_V = OFF_K + NSK * BOX;
 constexpr int NSW = 8;              // softmax warps: 4 lane quarters x 2 key halves
 constexpr int CW = TK / 2;          // score columns per softmax warp
 constexpr int NTHREADS = 32 * (NSW + 2);
-constexpr int OFF_RED = OFF_V + NSV * VSTAGE;  // float [2][NSW][32] row maxima + [NSW][32] row sums
-constexpr int OFF_BAR = OFF_RED + 3 * NSW * 32 * 4;
-constexpr int SMEM = 1024 + OFF_BAR + 256;
 constexpr int K_LEAD = 2;           // key tiles the producer keeps ahead of the value tiles
-constexpr uint32_t T_O = 0;         // 4 heads x 64 fp32 columns
+constexpr uint32_t T_O = 0;         // up to 4 x 64 fp32 columns (GTA: one block per head; GQA: the head's d)
 constexpr uint32_t T_S = 256;       // 128 fp32 columns
 constexpr uint32_t T_P = 384;       // 2 x 64 columns of bf16 pairs (double-buffered P)
+// Shared-memory layout of an instance with NQB 64-column boxes of query / key (d_qk = 64 NQB) and NVB
+// 64-column value blocks per tile (GTA: the group's heads; GQA: the head's d_v = 64 NVB).
+template <int NQB, int NVB>
+struct Cfg {
+    static constexpr int NSK = NQB == 1 ? 4 : 3;  // K ring depth: key tiles are released right after S = Q K^T
+    static constexpr int VSTAGE = NVB * BOX;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = NQB * BOX;
+    static constexpr int OFF_V = OFF_K + NSK * NQB * BOX;
+    static constexpr int OFF_RED = OFF_V + NSV * VSTAGE;  // float [2][NSW][32] row maxima + [NSW][32] row sums
+    static constexpr int OFF_BAR = OFF_RED + 3 * NSW * 32 * 4;
+    static constexpr int SMEM = 1024 + OFF_BAR + 256;
+    static_assert(SMEM <= 232448, "shared memory budget");
+    static_assert(NVB * 64 <= (int)T_S, "output columns");
+};
 }  // namespace gta
 
+// GQA = false: GTA, value blocks = the group's heads (NVB = 4 slots, H / G of them used);
+// GQA = true: one query head per group, K / V of its KV head, value blocks = the NVB column blocks of d.
+template <int NQB, int NVB, bool GQA>
 __global__ void __launch_bounds__(gta::NTHREADS, 1)
     gta_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const GtaParams p) {
     using namespace gta;
+    using CF = Cfg<NQB, NVB>;
+    constexpr int NSK = CF::NSK, VSTAGE = CF::VSTAGE, OFF_Q = CF::OFF_Q, OFF_K = CF::OFF_K, OFF_V = CF::OFF_V;
+    constexpr int OFF_RED = CF::OFF_RED, OFF_BAR = CF::OFF_BAR;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
@@ -93,6 +115,9 @@ __global__ void __launch_bounds__(gta::NTHREADS, 1)
     const int split = (int)blockIdx.x % p.nsplit;
     const int grp = blockIdx.y, b = blockIdx.z;
     const int HPG = p.H / p.G;
+    const int nvb = GQA ? NVB : HPG;                     // value blocks of a tile (64 columns each)
+    const int kv_head = GQA ? grp / p.kv_ratio : grp;    // the head whose keys (and GQA: values) are read
+    const int k_heads = GQA ? p.h_kv : p.G;              // heads of the key (GQA: and value) cache
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int L = clamp_len(p.lens, b, p.Lmax, p.s_q, p.causal, p.status,
                             threadIdx.x == 0 && blockIdx.x == 0 && grp == 0);
@@ -137,8 +162,10 @@ __global__ void __launch_bounds__(gta::NTHREADS, 1)
         // issue order K(0..K_LEAD-1), then per tile i: K(i + K_LEAD), V(i)
         if (lane == 0) {
             const uint32_t qb = smem_u32(q_full);
-            mbar_arrive_expect_tx(qb, BOX);
-            tma_load_2d(smem_u32(smem + OFF_Q), &tm_q, 0, (b * p.G + grp) * p.s_q + q0, qb);
+            mbar_arrive_expect_tx(qb, NQB * BOX);
+#pragma unroll
+            for (int kb = 0; kb < NQB; ++kb)
+                tma_load_2d(smem_u32(smem + OFF_Q + kb * BOX), &tm_q, kb * 64, (b * p.G + grp) * p.s_q + q0, qb);
             int k_issued = 0, v_issued = 0;
             bool ok = true;
             // row of token `tok` of head `head` (of `heads`) of this sequence: contiguous [B][heads][Lmax], or
@@ -161,10 +188,13 @@ __global__ void __launch_bounds__(gta::NTHREADS, 1)
                 const int s = i % NSK;
                 if (i >= NSK && !mbar_wait(smem_u32(&k_empty[s]), ((i / NSK) - 1) & 1, p.status)) return false;
                 const uint32_t fb = smem_u32(&k_full[s]);
-                mbar_arrive_expect_tx(fb, BOX);
-                for (int r0 = 0; r0 < TK; r0 += p.box_rows)  // one box, or one per page piece of the tile
-                    tma_load_2d(smem_u32(smem + OFF_K + s * BOX) + r0 * 128, &tm_k, 0,
-                                cache_row(kbeg + i * TK + r0, p.G, grp), fb);
+                mbar_arrive_expect_tx(fb, NQB * BOX);
+                for (int r0 = 0; r0 < TK; r0 += p.box_rows) {  // one box, or one per page piece of the tile
+                    const int y = cache_row(kbeg + i * TK + r0, k_heads, kv_head);
+#pragma unroll
+                    for (int kb = 0; kb < NQB; ++kb)
+                        tma_load_2d(smem_u32(smem + OFF_K + (s * NQB + kb) * BOX) + r0 * 128, &tm_k, kb * 64, y, fb);
+                }
                 ++k_issued;
                 return true;
             };
@@ -172,12 +202,17 @@ __global__ void __launch_bounds__(gta::NTHREADS, 1)
                 const int s = i % NSV;
                 if (i >= NSV && !mbar_wait(smem_u32(&v_empty[s]), ((i / NSV) - 1) & 1, p.status)) return false;
                 const uint32_t fb = smem_u32(&v_full[s]);
-                mbar_arrive_expect_tx(fb, HPG * BOX);
+                mbar_arrive_expect_tx(fb, nvb * BOX);
                 const uint32_t d = smem_u32(smem + OFF_V + s * VSTAGE);
-                for (int hh = 0; hh < HPG; ++hh)
-                    for (int r0 = 0; r0 < TK; r0 += p.box_rows)
-                        tma_load_2d(d + hh * BOX + r0 * 128, &tm_v, 0, cache_row(kbeg + i * TK + r0, p.H, grp * HPG + hh),
-                                    fb);
+                for (int hh = 0; hh < nvb; ++hh)
+                    for (int r0 = 0; r0 < TK; r0 += p.box_rows) {
+                        if (GQA)  // column block hh of the KV head's value rows
+                            tma_load_2d(d + hh * BOX + r0 * 128, &tm_v, hh * 64,
+                                        cache_row(kbeg + i * TK + r0, k_heads, kv_head), fb);
+                        else      // the value tile of the group's head hh
+                            tma_load_2d(d + hh * BOX + r0 * 128, &tm_v, 0,
+                                        cache_row(kbeg + i * TK + r0, p.H, grp * HPG + hh), fb);
+                    }
                 ++v_issued;
                 return true;
             };
@@ -198,7 +233,7 @@ __global__ void __launch_bounds__(gta::NTHREADS, 1)
     } else if (warp == NSW + 1) {
         // ------------------------------ MMA issuer ------------------------------
         constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
-        const uint32_t idesc_pv = idesc_bf16_f32(128, 64 * HPG, false, true);
+        const uint32_t idesc_pv = idesc_bf16_f32(128, 64 * nvb, false, true);
         bool ok = mbar_wait(smem_u32(q_full), 0, p.status);
         // zero the rows of a tile past the cache length (they may hold anything, even NaN)
         auto zero_tail = [&](uint8_t* base, int nbox, int j) {
@@ -215,16 +250,16 @@ __global__ void __launch_bounds__(gta::NTHREADS, 1)
         auto issue_qk = [&](int j) -> bool {
             const int s = j % NSK;
             if (!mbar_wait(smem_u32(&k_full[s]), (j / NSK) & 1, p.status)) return false;
-            uint8_t* kt = smem + OFF_K + s * BOX;
-            zero_tail(kt, 1, j);
+            uint8_t* kt = smem + OFF_K + s * NQB * BOX;
+            zero_tail(kt, NQB, j);
             if (j >= 1 && !mbar_wait(smem_u32(s_free), (j - 1) & 1, p.status)) return false;
             tc_fence_after();
             if (lane == 0) {
                 const uint32_t qa = smem_u32(smem + OFF_Q), ka = smem_u32(kt);
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    umma_ss(tmem + T_S, smem_desc_sw128(qa + k * 32, 16, 1024), smem_desc_sw128(ka + k * 32, 16, 1024),
-                            idesc_qk, k != 0);
+                for (int k = 0; k < 4 * NQB; ++k)  // K = 16 steps: box k / 4, 32 bytes apart inside it
+                    umma_ss(tmem + T_S, smem_desc_sw128(qa + (k / 4) * BOX + (k % 4) * 32, 16, 1024),
+                            smem_desc_sw128(ka + (k / 4) * BOX + (k % 4) * 32, 16, 1024), idesc_qk, k != 0);
                 umma_commit(smem_u32(s_ready));
                 umma_commit(smem_u32(&k_empty[s]));  // the key tile is free once the scores are computed
             }
@@ -237,7 +272,7 @@ __global__ void __launch_bounds__(gta::NTHREADS, 1)
             const int sv = j % NSV;
             if (!mbar_wait(smem_u32(&v_full[sv]), (j / NSV) & 1, p.status)) break;
             uint8_t* vt = smem + OFF_V + sv * VSTAGE;
-            zero_tail(vt, HPG, j);
+            zero_tail(vt, nvb, j);
             if (!mbar_wait(smem_u32(&p_ready[j & 1]), (j >> 1) & 1, p.status)) break;
             tc_fence_after();
             if (lane == 0) {
@@ -330,7 +365,7 @@ __global__ void __launch_bounds__(gta::NTHREADS, 1)
             for (int c0 = 0; c0 < CW / 2; c0 += 16)
                 tmem_st16(tmem + lane_base + T_P + (j & 1) * 64 + half * (CW / 2) + c0, pk + c0);
             if (any_resc) {
-                for (int c0 = half * 16; c0 < 64 * HPG; c0 += 32) {
+                for (int c0 = half * 16; c0 < 64 * nvb; c0 += 32) {
                     uint32_t o[16];
                     tmem_ld16(tmem + lane_base + T_O + c0, o);
                     tmem_ld_wait();
@@ -359,14 +394,17 @@ __global__ void __launch_bounds__(gta::NTHREADS, 1)
             const int nsp_row = row_ok ? cdiv(vis_end, p.split_tokens) : 0;
             const bool mine = row_ok && kbeg < vis_end;
             const bool partial = mine && nsp_row > 1;
-            for (int c0 = half * 16; c0 < 64 * HPG; c0 += 32) {
-                const int hh = c0 / 64;
+            // output row of the head and its column: GTA head grp * HPG + c0 / 64, 64 values; GQA head grp, 64 nvb
+            constexpr int DOUT = GQA ? 64 * NVB : 64;
+            for (int c0 = half * 16; c0 < 64 * nvb; c0 += 32) {
+                const int head = GQA ? grp : grp * HPG + c0 / 64;
+                const int col = GQA ? c0 : c0 % 64;
                 uint32_t o[16];
                 tmem_ld16(tmem + lane_base + T_O + c0, o);
                 tmem_ld_wait();
                 if (partial) {
                     float4* d = reinterpret_cast<float4*>(
-                        p.part_o + ((((size_t)b * p.H + grp * HPG + hh) * p.s_q + q) * p.nsplit + split) * 64 + (c0 % 64));
+                        p.part_o + ((((size_t)b * p.H + head) * p.s_q + q) * p.nsplit + split) * DOUT + col);
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
                         d[e] = make_float4(__uint_as_float(o[4 * e]) * inv_l, __uint_as_float(o[4 * e + 1]) * inv_l,
@@ -376,8 +414,7 @@ __global__ void __launch_bounds__(gta::NTHREADS, 1)
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
                         pkk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
-                    uint4* d = reinterpret_cast<uint4*>(p.out + (((size_t)b * p.H + grp * HPG + hh) * p.s_q + q) * 64 +
-                                                        (c0 % 64));
+                    uint4* d = reinterpret_cast<uint4*>(p.out + (((size_t)b * p.H + head) * p.s_q + q) * DOUT + col);
                     d[0] = make_uint4(pkk[0], pkk[1], pkk[2], pkk[3]);
                     d[1] = make_uint4(pkk[4], pkk[5], pkk[6], pkk[7]);
                 }
@@ -398,9 +435,11 @@ __global__ void __launch_bounds__(gta::NTHREADS, 1)
 // with 4 of its 64 values (float4 loads, many rows in flight), weights 2^(lse_i - max lse) from the group's
 // log2-domain lse of each split; writes the bf16 output and, for the first head of the group, the group's
 // natural-log lse.
+template <int DOUT>
 __global__ void __launch_bounds__(256) gta_combine_kernel(const GtaParams p) {
-    const size_t row = (size_t)blockIdx.x * 16 + threadIdx.x / 16;  // ((b * H + h) * s_q + q)
-    const int d4 = threadIdx.x % 16;                                 // values 4 d4 .. 4 d4 + 3
+    constexpr int TPR = DOUT / 4;                                             // threads per row
+    const size_t row = (size_t)blockIdx.x * (256 / TPR) + threadIdx.x / TPR;  // ((b * H + h) * s_q + q)
+    const int d4 = threadIdx.x % TPR;                                         // values 4 d4 .. 4 d4 + 3
     const size_t nrows = (size_t)p.B * p.H * p.s_q;
     if (row >= nrows) return;
     const int q = (int)(row % p.s_q);
@@ -416,10 +455,10 @@ __global__ void __launch_bounds__(256) gta_combine_kernel(const GtaParams p) {
     for (int i = 0; i < nsp; ++i) M = fmaxf(M, pl[i]);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float wsum = 0.f;
-    const float4* po = reinterpret_cast<const float4*>(p.part_o + row * p.nsplit * 64) + d4;
+    const float4* po = reinterpret_cast<const float4*>(p.part_o + row * p.nsplit * DOUT) + d4;
     for (int i = 0; i < nsp; ++i) {
         const float w = exp2f(pl[i] - M);
-        const float4 v = po[(size_t)i * 16];
+        const float4 v = po[(size_t)i * TPR];
         wsum += w;
         acc = make_float4(fmaf(w, v.x, acc.x), fmaf(w, v.y, acc.y), fmaf(w, v.z, acc.z), fmaf(w, v.w, acc.w));
     }
@@ -427,7 +466,7 @@ __global__ void __launch_bounds__(256) gta_combine_kernel(const GtaParams p) {
     uint2 o;
     o.x = pack_bf16x2(acc.x * inv, acc.y * inv);
     o.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-    reinterpret_cast<uint2*>(p.out + row * 64)[d4] = o;
+    reinterpret_cast<uint2*>(p.out + row * DOUT)[d4] = o;
     if (p.lse && d4 == 0 && h % HPG == 0)
         p.lse[((size_t)b * p.G + grp) * p.s_q + q] = (M + log2f(wsum)) * 0.69314718055994530942f;
 }
@@ -451,7 +490,7 @@ struct GtaPlan {
     size_t off_lse, off_o, ws_bytes;
 };
 
-void gta_plan(int B, int G, int H, int s_q, int Lmax, GtaPlan* pl) {
+void gta_plan(int B, int G, int H, int s_q, int Lmax, GtaPlan* pl, int dout = 64) {
     int st = split_tokens_knob();
     if (st <= 0) {
         const long long units = (long long)cdiv(s_q, gta::TQ) * G * (B > 0 ? B : 1);
@@ -467,7 +506,7 @@ void gta_plan(int B, int G, int H, int s_q, int Lmax, GtaPlan* pl) {
     pl->off_lse = pl->off_o = 0;
     if (pl->nsplit > 1) {
         pl->off_lse = c.take((size_t)B * G * s_q * pl->nsplit * sizeof(float));
-        pl->off_o = c.take((size_t)B * H * s_q * pl->nsplit * 64 * sizeof(float));
+        pl->off_o = c.take((size_t)B * H * s_q * pl->nsplit * dout * sizeof(float));
     }
     pl->ws_bytes = c.off;
 }
@@ -484,6 +523,32 @@ extern "C" size_t gta_shared_score_attn_workspace_size(int B, int G, int H, int 
 }
 
 namespace {
+
+// Launches the attention kernel instance over grid (query tiles x splits, groups, sequences) and, with key
+// splits, the merge.
+template <int NQB, int NVB, bool GQA>
+lka_status_t gta_launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const GtaParams& p,
+                        cudaStream_t st) {
+    constexpr int SMEM = gta::Cfg<NQB, NVB>::SMEM;
+    auto kern = gta_attn_kernel<NQB, NVB, GQA>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess)
+        return LKA_ERR_CUDA;
+    if ((long long)cdiv(p.s_q, gta::TQ) * p.nsplit >= (1ll << 31)) return LKA_ERR_UNSUPPORTED;
+    dim3 grid(cdiv(p.s_q, gta::TQ) * p.nsplit, p.G, p.B);
+    {
+        TimedLaunch timer(st);
+        kern<<<grid, gta::NTHREADS, SMEM, st>>>(tq, tk, tv, p);
+        timer.stop();
+    }
+    if (cudaPeekAtLastError() != cudaSuccess) return LKA_ERR_CUDA;
+    if (p.nsplit > 1) {
+        constexpr int DOUT = GQA ? 64 * NVB : 64;
+        constexpr int RPB = 256 / (DOUT / 4);  // rows per merge block
+        const size_t rows = (size_t)p.B * p.H * p.s_q;
+        gta_combine_kernel<DOUT><<<(unsigned)((rows + RPB - 1) / RPB), 256, 0, st>>>(p);
+    }
+    return cudaPeekAtLastError() == cudaSuccess ? LKA_OK : LKA_ERR_CUDA;
+}
 
 struct GtaPages {
     const int32_t* block_table;
@@ -544,22 +609,7 @@ lka_status_t gta_run(const void* q_g, const void* k_g, const void* v, const int3
         p.max_pages = pg->max_pages;
         p.num_pages = pg->num_pages;
     }
-    cudaStream_t st = (cudaStream_t)stream;
-    if (cudaFuncSetAttribute(gta_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gta::SMEM) != cudaSuccess)
-        return LKA_ERR_CUDA;
-    if ((long long)cdiv(s_q, gta::TQ) * pl.nsplit >= (1ll << 31)) return LKA_ERR_UNSUPPORTED;
-    dim3 grid(cdiv(s_q, gta::TQ) * pl.nsplit, G, B);
-    {
-        TimedLaunch timer(st);
-        gta_attn_kernel<<<grid, gta::NTHREADS, gta::SMEM, st>>>(tq, tk, tv, p);
-        timer.stop();
-    }
-    if (cudaPeekAtLastError() != cudaSuccess) return LKA_ERR_CUDA;
-    if (pl.nsplit > 1) {
-        const size_t rows = (size_t)B * H * s_q;
-        gta_combine_kernel<<<(unsigned)((rows + 15) / 16), 256, 0, st>>>(p);
-    }
-    return cudaPeekAtLastError() == cudaSuccess ? LKA_OK : LKA_ERR_CUDA;
+    return gta_launch<1, 4, false>(tq, tk, tv, p, (cudaStream_t)stream);
 }
 
 bool gta_pages_ok(int page_size, int max_pages, int num_pages) {
@@ -597,3 +647,59 @@ lka_status_t gta_shared_score_attn_paged(const void* q_g, const void* k_pages, c
 }
 
 }  // extern "C"
+
+namespace lka {
+
+// Causal (or full) prefill of grouped-query attention with d = 128 on the tensor cores (the kernel above in its
+// GQA form): one CTA per (128-query tile, query head, sequence, key split).
+size_t gqa_prefill_ws_bytes(int B, int h_q, int s_q, int Lmax) {
+    GtaPlan pl;
+    gta_plan(B, h_q, h_q, s_q, Lmax, &pl, 128);
+    return pl.ws_bytes;
+}
+
+lka_status_t gqa_prefill_tc(const void* q, const void* k, const void* v, const int32_t* cache_lens, void* out,
+                            float* lse, int B, int h_q, int h_kv, int s_q, int Lmax, int causal, float scale, void* ws,
+                            size_t ws_bytes, cudaStream_t st, const int32_t* block_table, int page_size, int max_pages,
+                            int num_pages) {
+    GtaPlan pl;
+    gta_plan(B, h_q, h_q, s_q, Lmax, &pl, 128);
+    if (!ws || ws_bytes < pl.ws_bytes) return LKA_ERR_WORKSPACE;
+    if ((long long)B * h_q * s_q >= (1ll << 31) || B > 65535 || h_q > 65535) return LKA_ERR_UNSUPPORTED;
+    const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const int box_rows = block_table ? std::min(gta::TK, page_size) : gta::TK;
+    const uint64_t kv_rows = block_table ? (uint64_t)num_pages * h_kv * page_size : (uint64_t)B * h_kv * Lmax;
+    CUtensorMap tq, tk, tv;
+    if (!make_tmap_2d(&tq, BF, q, 128, (uint64_t)B * h_q * s_q, 256, 64, 128) ||
+        !make_tmap_2d(&tk, BF, k, 128, kv_rows, 256, 64, box_rows) ||
+        !make_tmap_2d(&tv, BF, v, 128, kv_rows, 256, 64, box_rows))
+        return LKA_ERR_CUDA;
+    GtaParams p{};
+    p.lens = cache_lens;
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.lse = lse;
+    p.status = static_cast<uint32_t*>(ws);
+    p.B = B;
+    p.G = h_q;
+    p.H = h_q;
+    p.s_q = s_q;
+    p.Lmax = Lmax;
+    p.causal = causal ? 1 : 0;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.box_rows = box_rows;
+    p.split_tokens = pl.split_tokens;
+    p.nsplit = pl.nsplit;
+    p.part_lse = pl.nsplit > 1 ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + pl.off_lse) : nullptr;
+    p.part_o = pl.nsplit > 1 ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + pl.off_o) : nullptr;
+    p.h_kv = h_kv;
+    p.kv_ratio = h_q / h_kv;
+    if (block_table) {
+        p.block_table = block_table;
+        p.page_size = page_size;
+        p.max_pages = max_pages;
+        p.num_pages = num_pages;
+    }
+    return gta_launch<2, 2, true>(tq, tk, tv, p, st);
+}
+
+}  // namespace lka
