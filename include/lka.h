@@ -82,11 +82,15 @@ typedef enum { LKA_BF16 = 0, LKA_FP32 = 1 } lka_dtype_t;
 /*  dtype: LKA_BF16 (d_h in {64, 128, 256}) or LKA_FP32 (d_h in {64, 128}).  */
 /*  Split-KV flash decoding: long caches are split over CTAs and merged by   */
 /*  log-sum-exp; the split partials live in ws.                              */
+/*  Prefill (bf16, d_h = 128, s_q >= 64, any of the paged forms below but    */
+/*  the FP8 cache) runs on the tcgen05 prefill kernel instead: one CTA per   */
+/*  128-query tile, query head, sequence and key split; S = Q K^T and O +=   */
+/*  P V on the tensor cores with the accumulators in tensor memory.          */
 /* ------------------------------------------------------------------------ */
 LKA_API size_t gqa_attn_workspace_size(int B, int h_q, int h_kv, int s_q, int d_h, int Lmax);
-/* Key splits per sequence that gqa_attn plans for these sizes and dtype (the grid is splits x h_kv x row
- * blocks x B CTAs; a sequence shorter than Lmax uses only the splits its keys reach), or 0 for arguments
- * gqa_attn rejects.  The plan depends only on the sizes, the dtype, the device's SM count and the split
+/* Key splits per sequence that gqa_attn plans for these sizes and dtype (decode: the grid is splits x h_kv x
+ * row blocks x B CTAs; prefill: query tiles x splits x h_q x B; a sequence shorter than Lmax uses only the
+ * splits its keys reach), or 0 for arguments gqa_attn rejects.  The plan depends only on the sizes, the dtype, the device's SM count and the split
  * knob (lka_set_split_tokens); host-only, no device work. */
 LKA_API int gqa_attn_split_count(int B, int h_q, int h_kv, int s_q, int d_h, int Lmax, lka_dtype_t dtype);
 LKA_API lka_status_t gqa_attn(const void *q, const void *k, const void *v, const int32_t *cache_lens, void *out,
@@ -223,7 +227,11 @@ LKA_API lka_status_t latent_absorbed_attn_fp8kv(const void *q_c, const void *q_r
 /*  key is stored once and shared by all groups); value: vc[b,gamma,j,:];    */
 /*  query of head i: [q_c ; q_r].  h_q/g query heads per group.              */
 /*   kc, vc [B,g,Lmax,d_h]  kr [B,Lmax,d_r]  other arguments as in (b).      */
-/*  Supported: bf16, d_h = 128, d_r = 64, h_q/g = 16, s_q <= 2.              */
+/*  Supported: bf16, d_h = 128, d_r = 64, and either h_q/g = 16, s_q <= 2    */
+/*  (decode kernel: one CTA per group and key split, the group's 16 heads x  */
+/*  s_q query rows as the MMA rows), or s_q >= 64 with any h_q/g (prefill:   */
+/*  the tcgen05 prefill kernel of (a) with 192-wide keys [kc ; kr], one CTA  */
+/*  per 128-query tile, head, sequence and key split).                       */
 /* ------------------------------------------------------------------------ */
 LKA_API size_t latent_expand_gqa_attn_workspace_size(int B, int h_q, int g, int s_q, int d_h, int d_r, int Lmax);
 LKA_API lka_status_t latent_expand_gqa_attn(const void *q_c, const void *q_r, const void *kc, const void *vc,

@@ -537,7 +537,8 @@ def gqa_split_count(B: int, h_q: int, h_kv: int, s_q: int, d: int, Lmax: int, dt
 
 
 def set_split_tokens(tokens: int) -> int:
-    """Process-wide KV tokens per split of the split-KV kernels (0 = automatic); returns the previous value."""
+    """KV tokens per split of the split-KV kernels for calls made from this thread (0 = automatic); returns the
+    previous value."""
     return int(library().lka_set_split_tokens(int(tokens)))
 
 

@@ -229,6 +229,10 @@ size_t gqa_attn_workspace_size(int B, int h_q, int h_kv, int s_q, int d_h, int L
 
 int gqa_attn_split_count(int B, int h_q, int h_kv, int s_q, int d_h, int Lmax, lka_dtype_t dtype) {
     if (dtype != LKA_BF16 && dtype != LKA_FP32) return 0;
+    if (gqa_tc_prefill(dtype == LKA_BF16 ? 2 : 4, d_h, s_q, false)) {
+        if (B < 0 || h_q < 1 || h_kv < 1 || Lmax < 1 || h_q % h_kv) return 0;
+        return gqa_prefill_nsplit(B, h_q, s_q, Lmax);
+    }
     GqaPlan pl;
     return gqa_plan(B, h_q, h_kv, s_q, d_h, Lmax, dtype == LKA_BF16 ? 2 : 4, &pl) == LKA_OK ? pl.nsplit : 0;
 }

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/lka.h"
+
 namespace lka {
 
 struct ExpParams {
@@ -25,5 +27,14 @@ struct ExpParams {
 
 cudaError_t expanded_attn_launch(const CUtensorMap& qc, const CUtensorMap& qr, const CUtensorMap& kc,
                                  const CUtensorMap& kr, const CUtensorMap& vc, const ExpParams& p, cudaStream_t st);
+
+// Prefill (s_q >= kExpPrefillMinQueries) of the per-group path on the tensor-core prefill kernel (gta_attn.cu):
+// keys [kc[gamma] ; k^R] of d_h + d_r = 192 values, values vc[gamma]; paged pools when block_table != nullptr.
+constexpr int kExpPrefillMinQueries = 64;
+size_t expanded_prefill_ws_bytes(int B, int h_q, int s_q, int Lmax);
+lka_status_t expanded_prefill_tc(const void* q_c, const void* q_r, const void* kc, const void* vc, const void* kr,
+                                 const int32_t* cache_lens, void* out, float* lse, int B, int h_q, int g, int s_q,
+                                 int Lmax, int causal, float scale, void* ws, size_t ws_bytes, cudaStream_t st,
+                                 const int32_t* block_table, int page_size, int max_pages, int num_pages);
 
 }  // namespace lka

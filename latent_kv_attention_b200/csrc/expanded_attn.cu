@@ -495,7 +495,16 @@ lka_status_t exp_plan(int B, int h_q, int g, int s_q, int d_h, int d_r, int Lmax
 
 extern "C" {
 
+// Whether a call of the per-group path runs the tensor-core prefill (d_h = 128, d_h^R = 64, many queries).
+static bool exp_tc_prefill(int d_h, int d_r, int s_q) {
+    return d_h == 128 && d_r == 64 && s_q >= kExpPrefillMinQueries;
+}
+
 size_t latent_expand_gqa_attn_workspace_size(int B, int h_q, int g, int s_q, int d_h, int d_r, int Lmax) {
+    if (exp_tc_prefill(d_h, d_r, s_q)) {
+        if (B < 0 || h_q < 1 || g < 1 || Lmax < 1 || h_q % g) return 0;
+        return expanded_prefill_ws_bytes(B, h_q, s_q, Lmax);
+    }
     ExpPlan pl;
     return exp_plan(B, h_q, g, s_q, d_h, d_r, Lmax, &pl) == LKA_OK ? pl.ws_bytes : 0;
 }
@@ -513,6 +522,20 @@ static lka_status_t expanded_run(const void* q_c, const void* q_r, const void* k
                                  int d_h, int d_r, int Lmax, int causal, float scale, lka_dtype_t dtype, void* ws,
                                  size_t ws_bytes, void* stream, const ExpPages* pg) {
     if (dtype != LKA_BF16) return LKA_ERR_UNSUPPORTED;
+    if (exp_tc_prefill(d_h, d_r, s_q)) {
+        // prefill (GQLA section 1: MHA-like, compute-bound) on the tensor-core prefill kernel
+        if (B < 0 || h_q < 1 || g < 1 || Lmax < 1 || h_q % g) return LKA_ERR_INVALID_ARG;
+        if (!pg && (long long)B * g * Lmax >= (1ll << 31)) return LKA_ERR_UNSUPPORTED;
+        if (B == 0) return LKA_OK;
+        const void* ptrs[] = {q_c, q_r, kc, vc, kr, cache_lens, out};
+        for (const void* ptr : ptrs)
+            if (!ptr || !aligned16(ptr)) return LKA_ERR_INVALID_ARG;
+        if (!isfinite(scale)) return LKA_ERR_INVALID_ARG;
+        if (ws && !aligned16(ws)) return LKA_ERR_INVALID_ARG;
+        return expanded_prefill_tc(q_c, q_r, kc, vc, kr, cache_lens, out, lse, B, h_q, g, s_q, Lmax, causal, scale,
+                                   ws, ws_bytes, (cudaStream_t)stream, pg ? pg->block_table : nullptr,
+                                   pg ? pg->page_size : 0, pg ? pg->max_pages : 0, pg ? pg->num_pages : 0);
+    }
     ExpPlan pl;
     lka_status_t s = exp_plan(B, h_q, g, s_q, d_h, d_r, Lmax, &pl, pg != nullptr);
     if (s != LKA_OK) return s;
@@ -599,6 +622,10 @@ size_t latent_expand_gqa_attn_paged_workspace_size(int B, int h_q, int g, int s_
     if (page_size < 8 || (page_size & (page_size - 1)) || max_pages < 1 ||
         (long long)page_size * max_pages >= (1ll << 31))
         return 0;
+    if (exp_tc_prefill(d_h, d_r, s_q)) {
+        if (B < 0 || h_q < 1 || g < 1 || h_q % g) return 0;
+        return expanded_prefill_ws_bytes(B, h_q, s_q, page_size * max_pages);
+    }
     ExpPlan pl;
     return exp_plan(B, h_q, g, s_q, d_h, d_r, page_size * max_pages, &pl, true) == LKA_OK ? pl.ws_bytes : 0;
 }

@@ -48,6 +48,7 @@ cudaError_t gqa_decode_launch(const CUtensorMap& tk, const CUtensorMap& tv, cons
 // query head, sequence, key split), keys and values of the head's KV head h / (h_q / h_kv); paged caches when
 // block_table != nullptr (pools [num_pages, h_kv, page_size, 128]).  gqa_prefill_ws_bytes is its workspace.
 size_t gqa_prefill_ws_bytes(int B, int h_q, int s_q, int Lmax);
+int gqa_prefill_nsplit(int B, int h_q, int s_q, int Lmax);  // key splits of the prefill plan
 lka_status_t gqa_prefill_tc(const void* q, const void* k, const void* v, const int32_t* cache_lens, void* out,
                             float* lse, int B, int h_q, int h_kv, int s_q, int Lmax, int causal, float scale, void* ws,
                             size_t ws_bytes, cudaStream_t st, const int32_t* block_table, int page_size, int max_pages,

@@ -30,7 +30,10 @@
 // head is then a group of its own, its keys and values are those of its KV head
 // floor(h / (h_q / h_kv)), and the head dimension d = 128 is two 64-column
 // boxes of the query and key tiles and two 64-column blocks of the value tile
-// (the N = 128 of P*V).
+// (the N = 128 of P*V).  The prefill of the GQLA per-group GQA path (GQLA
+// section 1: prefill expands the latent, MHA-like) is the same with a query
+// and key of 192 values: two boxes of q^C / the group's key kc and a third box
+// of q^R / the RoPE key k^R, which all groups share.
 #include "common.cuh"
 #include "host_util.h"
 #include "tc.cuh"
@@ -72,7 +75,8 @@ constexpr uint32_t T_P = 384;       // 2 x 64 columns of bf16 pairs (double-buff
 // 64-column value blocks per tile (GTA: the group's heads; GQA: the head's d_v = 64 NVB).
 template <int NQB, int NVB>
 struct Cfg {
-    static constexpr int NSK = NQB == 1 ? 4 : 3;  // K ring depth: key tiles are released right after S = Q K^T
+    // K ring depth: key tiles are released right after S = Q K^T
+    static constexpr int NSK = NQB == 1 ? 4 : (NQB == 2 ? 3 : 2);
     static constexpr int VSTAGE = NVB * BOX;
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = NQB * BOX;
@@ -87,10 +91,13 @@ struct Cfg {
 
 // GQA = false: GTA, value blocks = the group's heads (NVB = 4 slots, H / G of them used);
 // GQA = true: one query head per group, K / V of its KV head, value blocks = the NVB column blocks of d.
+// NQB = 3 (GQA): the third query box comes from tm_q2 (q^R rows) and the third key box from tm_k2 (the RoPE
+// key, one row per token shared by all heads).
 template <int NQB, int NVB, bool GQA>
 __global__ void __launch_bounds__(gta::NTHREADS, 1)
     gta_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const GtaParams p) {
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q2,
+                    const __grid_constant__ CUtensorMap tm_k2, const GtaParams p) {
     using namespace gta;
     using CF = Cfg<NQB, NVB>;
     constexpr int NSK = CF::NSK, VSTAGE = CF::VSTAGE, OFF_Q = CF::OFF_Q, OFF_K = CF::OFF_K, OFF_V = CF::OFF_V;
@@ -164,8 +171,12 @@ __global__ void __launch_bounds__(gta::NTHREADS, 1)
             const uint32_t qb = smem_u32(q_full);
             mbar_arrive_expect_tx(qb, NQB * BOX);
 #pragma unroll
-            for (int kb = 0; kb < NQB; ++kb)
-                tma_load_2d(smem_u32(smem + OFF_Q + kb * BOX), &tm_q, kb * 64, (b * p.G + grp) * p.s_q + q0, qb);
+            for (int kb = 0; kb < NQB; ++kb) {
+                if (kb < 2)
+                    tma_load_2d(smem_u32(smem + OFF_Q + kb * BOX), &tm_q, kb * 64, (b * p.G + grp) * p.s_q + q0, qb);
+                else
+                    tma_load_2d(smem_u32(smem + OFF_Q + kb * BOX), &tm_q2, 0, (b * p.G + grp) * p.s_q + q0, qb);
+            }
             int k_issued = 0, v_issued = 0;
             bool ok = true;
             // row of token `tok` of head `head` (of `heads`) of this sequence: contiguous [B][heads][Lmax], or
@@ -190,10 +201,16 @@ __global__ void __launch_bounds__(gta::NTHREADS, 1)
                 const uint32_t fb = smem_u32(&k_full[s]);
                 mbar_arrive_expect_tx(fb, NQB * BOX);
                 for (int r0 = 0; r0 < TK; r0 += p.box_rows) {  // one box, or one per page piece of the tile
-                    const int y = cache_row(kbeg + i * TK + r0, k_heads, kv_head);
+                    const int tok = kbeg + i * TK + r0;
+                    const int y = cache_row(tok, k_heads, kv_head);
 #pragma unroll
-                    for (int kb = 0; kb < NQB; ++kb)
-                        tma_load_2d(smem_u32(smem + OFF_K + (s * NQB + kb) * BOX) + r0 * 128, &tm_k, kb * 64, y, fb);
+                    for (int kb = 0; kb < NQB; ++kb) {
+                        const uint32_t dst = smem_u32(smem + OFF_K + (s * NQB + kb) * BOX) + r0 * 128;
+                        if (kb < 2)
+                            tma_load_2d(dst, &tm_k, kb * 64, y, fb);
+                        else  // the shared RoPE key: one row per token ([B, Lmax] or [num_pages, page_size])
+                            tma_load_2d(dst, &tm_k2, 0, cache_row(tok, 1, 0), fb);
+                    }
                 }
                 ++k_issued;
                 return true;
@@ -470,7 +487,6 @@ __global__ void __launch_bounds__(256) gta_combine_kernel(const GtaParams p) {
     if (p.lse && d4 == 0 && h % HPG == 0)
         p.lse[((size_t)b * p.G + grp) * p.s_q + q] = (M + log2f(wsum)) * 0.69314718055994530942f;
 }
-
 }  // namespace lka
 
 using namespace lka;
@@ -527,8 +543,8 @@ namespace {
 // Launches the attention kernel instance over grid (query tiles x splits, groups, sequences) and, with key
 // splits, the merge.
 template <int NQB, int NVB, bool GQA>
-lka_status_t gta_launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const GtaParams& p,
-                        cudaStream_t st) {
+lka_status_t gta_launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq2,
+                        const CUtensorMap& tk2, const GtaParams& p, cudaStream_t st) {
     constexpr int SMEM = gta::Cfg<NQB, NVB>::SMEM;
     auto kern = gta_attn_kernel<NQB, NVB, GQA>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess)
@@ -537,7 +553,7 @@ lka_status_t gta_launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUte
     dim3 grid(cdiv(p.s_q, gta::TQ) * p.nsplit, p.G, p.B);
     {
         TimedLaunch timer(st);
-        kern<<<grid, gta::NTHREADS, SMEM, st>>>(tq, tk, tv, p);
+        kern<<<grid, gta::NTHREADS, SMEM, st>>>(tq, tk, tv, tq2, tk2, p);
         timer.stop();
     }
     if (cudaPeekAtLastError() != cudaSuccess) return LKA_ERR_CUDA;
@@ -609,7 +625,7 @@ lka_status_t gta_run(const void* q_g, const void* k_g, const void* v, const int3
         p.max_pages = pg->max_pages;
         p.num_pages = pg->num_pages;
     }
-    return gta_launch<1, 4, false>(tq, tk, tv, p, (cudaStream_t)stream);
+    return gta_launch<1, 4, false>(tq, tk, tv, tq, tk, p, (cudaStream_t)stream);
 }
 
 bool gta_pages_ok(int page_size, int max_pages, int num_pages) {
@@ -658,6 +674,12 @@ size_t gqa_prefill_ws_bytes(int B, int h_q, int s_q, int Lmax) {
     return pl.ws_bytes;
 }
 
+int gqa_prefill_nsplit(int B, int h_q, int s_q, int Lmax) {
+    GtaPlan pl;
+    gta_plan(B, h_q, h_q, s_q, Lmax, &pl, 128);
+    return pl.nsplit;
+}
+
 lka_status_t gqa_prefill_tc(const void* q, const void* k, const void* v, const int32_t* cache_lens, void* out,
                             float* lse, int B, int h_q, int h_kv, int s_q, int Lmax, int causal, float scale, void* ws,
                             size_t ws_bytes, cudaStream_t st, const int32_t* block_table, int page_size, int max_pages,
@@ -699,7 +721,59 @@ lka_status_t gqa_prefill_tc(const void* q, const void* k, const void* v, const i
         p.max_pages = max_pages;
         p.num_pages = num_pages;
     }
-    return gta_launch<2, 2, true>(tq, tk, tv, p, st);
+    return gta_launch<2, 2, true>(tq, tk, tv, tq, tk, p, st);
+}
+
+// Prefill of the GQLA per-group GQA path (bf16, d_h = 128, d_h^R = 64): keys [kc[gamma] ; k^R] of 192 values,
+// values vc[gamma], h_q / g query heads per group; contiguous caches kc, vc [B, g, Lmax, 128], kr [B, Lmax, 64],
+// or paged pools [num_pages, g, page_size, 128] and [num_pages, page_size, 64] with block_table.
+size_t expanded_prefill_ws_bytes(int B, int h_q, int s_q, int Lmax) { return gqa_prefill_ws_bytes(B, h_q, s_q, Lmax); }
+
+lka_status_t expanded_prefill_tc(const void* q_c, const void* q_r, const void* kc, const void* vc, const void* kr,
+                                 const int32_t* cache_lens, void* out, float* lse, int B, int h_q, int g, int s_q,
+                                 int Lmax, int causal, float scale, void* ws, size_t ws_bytes, cudaStream_t st,
+                                 const int32_t* block_table, int page_size, int max_pages, int num_pages) {
+    GtaPlan pl;
+    gta_plan(B, h_q, h_q, s_q, Lmax, &pl, 128);
+    if (!ws || ws_bytes < pl.ws_bytes) return LKA_ERR_WORKSPACE;
+    if ((long long)B * h_q * s_q >= (1ll << 31) || B > 65535 || h_q > 65535) return LKA_ERR_UNSUPPORTED;
+    const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const int box_rows = block_table ? std::min(gta::TK, page_size) : gta::TK;
+    const uint64_t kv_rows = block_table ? (uint64_t)num_pages * g * page_size : (uint64_t)B * g * Lmax;
+    const uint64_t r_rows = block_table ? (uint64_t)num_pages * page_size : (uint64_t)B * Lmax;
+    const uint64_t q_rows = (uint64_t)B * h_q * s_q;
+    CUtensorMap tq, tq2, tk, tk2, tv;
+    if (!make_tmap_2d(&tq, BF, q_c, 128, q_rows, 256, 64, 128) || !make_tmap_2d(&tq2, BF, q_r, 64, q_rows, 128, 64, 128) ||
+        !make_tmap_2d(&tk, BF, kc, 128, kv_rows, 256, 64, box_rows) ||
+        !make_tmap_2d(&tk2, BF, kr, 64, r_rows, 128, 64, box_rows) ||
+        !make_tmap_2d(&tv, BF, vc, 128, kv_rows, 256, 64, box_rows))
+        return LKA_ERR_CUDA;
+    GtaParams p{};
+    p.lens = cache_lens;
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.lse = lse;
+    p.status = static_cast<uint32_t*>(ws);
+    p.B = B;
+    p.G = h_q;
+    p.H = h_q;
+    p.s_q = s_q;
+    p.Lmax = Lmax;
+    p.causal = causal ? 1 : 0;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.box_rows = box_rows;
+    p.split_tokens = pl.split_tokens;
+    p.nsplit = pl.nsplit;
+    p.part_lse = pl.nsplit > 1 ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + pl.off_lse) : nullptr;
+    p.part_o = pl.nsplit > 1 ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + pl.off_o) : nullptr;
+    p.h_kv = g;
+    p.kv_ratio = h_q / g;
+    if (block_table) {
+        p.block_table = block_table;
+        p.page_size = page_size;
+        p.max_pages = max_pages;
+        p.num_pages = num_pages;
+    }
+    return gta_launch<3, 2, true>(tq, tk, tv, tq2, tk2, p, st);
 }
 
 }  // namespace lka

@@ -103,6 +103,22 @@ def test_split_knob_is_per_thread(lib):
     assert lka.gqa_split_count(64, 32, 8, 1, 128, 8192) == auto  # this thread's plan is untouched
 
 
+def test_gqa_prefill_split_plan(lib):
+    """Prefill shapes (bf16, d 128, s_q >= 64) are planned for the tensor-core prefill kernel: one CTA per
+    128-query tile and query head; the keys are split only while those CTAs number fewer than two per SM
+    (148 SMs), in splits of at least 512 keys (rounded to 128-key tiles)."""
+    prev = lka.set_split_tokens(0)
+    try:
+        assert lka.gqa_split_count(2, 32, 8, 4096, 128, 4096) == 1   # 2048 CTAs already fill the GPU
+        assert lka.gqa_split_count(1, 8, 2, 160, 128, 1024) == 2     # 16 CTAs: 512-key splits
+        assert lka.gqa_split_count(1, 8, 2, 160, 128, 100000) == 19  # ceil(296 / 16) splits of 5376 keys
+        lka.set_split_tokens(128)
+        assert lka.gqa_split_count(1, 8, 2, 160, 128, 1024) == 8
+        assert lka.gqa_split_count(1, 8, 3, 160, 128, 1024) == 0     # h_q not a multiple of h_kv
+    finally:
+        lka.set_split_tokens(prev)
+
+
 def test_gqa_split_plan(lib):
     """The GQA split count chosen by the wave-cost rule (host logic; 148 SMs, two resident CTAs per SM for the
     d_h 128 bf16 kernel): the smallest max(ceil(w), w + 1/4) * (tiles per split + 2) with w = CTAs / 296."""
