@@ -205,9 +205,10 @@ class Workload:
 
 
 class GqaDecode(Workload):
-    """gqa_attn over the Llama-3.1-8B-shaped decode batch: split-KV decode kernel + log-sum-exp merge."""
+    """gqa_attn over the Llama-3.1-8B-shaped decode batch: split-KV decode kernel (the mma.sync instance for bf16
+    caches) + log-sum-exp merge."""
 
-    kernel = "gqa_decode_kernel"
+    kernel = "gqa_decode_mma_kernel"
     src = ("latent_kv_attention_b200/csrc/gqa_decode.cu", "latent_kv_attention_b200/csrc/common.cuh")
 
     def setup_costs(self):
@@ -272,6 +273,8 @@ class GqaDecodePaged(GqaDecode):
 
 class GqaDecodeFp8(GqaDecode):
     """gqa_attn_fp8kv over the same decode batch with the K/V cache in e4m3 (one scale per KV head)."""
+
+    kernel = "gqa_decode_kernel"  # the CUDA-core instance (e4m3 values widened per lane)
 
     def setup_costs(self):
         w = self.w

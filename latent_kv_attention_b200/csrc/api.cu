@@ -56,9 +56,11 @@ struct GqaPlan {
     size_t off_lse, off_o, ws_bytes;
 };
 
-static int pick_rb(int rows, int d, int dtype_bytes) {
-    int cap = 16;
-    if ((dtype_bytes == 2 && d == 64) || d == 256) cap = 8;
+static int pick_rb(int rows, int d, int dtype_bytes, bool fp8kv) {
+    // bf16 caches with d <= 128: the tensor-core instance, whose MMA tile holds 16 query rows
+    if (!fp8kv && dtype_bytes == 2 && d <= 128) return 16;
+    int cap = fp8kv ? 4 : 16;
+    if (d == 256) cap = fp8kv ? 4 : 8;
     int rb = 1;
     while (rb < rows && rb < cap) rb *= 2;
     return rb;
@@ -73,8 +75,7 @@ static lka_status_t gqa_plan(int B, int h_q, int h_kv, int s_q, int d_h, int Lma
     if (!d_ok) return LKA_ERR_UNSUPPORTED;
     if (!paged && (long long)B * h_kv * Lmax >= (1ll << 31)) return LKA_ERR_UNSUPPORTED;
     const int R = (h_q / h_kv) * s_q;
-    pl->rb = pick_rb(R, d_h, dtype_bytes);
-    if (fp8kv && pl->rb > 4) pl->rb = 4;
+    pl->rb = pick_rb(R, d_h, dtype_bytes, fp8kv);
     pl->n_rb = cdiv(R, pl->rb);
     if ((long long)h_kv * pl->n_rb > 65535 || B > 65535) return LKA_ERR_UNSUPPORTED;
     int per_sm = 1;  // resident CTAs per SM of the kernel instance

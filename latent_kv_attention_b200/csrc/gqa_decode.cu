@@ -31,6 +31,7 @@
 #include "common.cuh"
 #include "gqa_decode.h"
 #include "host_util.h"
+#include "tc.cuh"
 
 // Tuning knobs of the build: shared-memory budget of the TMA ring per CTA (KiB) and
 // the number of CTAs per SM the small-row instances are compiled for.
@@ -214,6 +215,94 @@ __device__ __forceinline__ int paged_row(const GqaParams& p, int b, int kvh, int
     return (page * p.h_kv + kvh) * p.page_size + tok % p.page_size;
 }
 
+// The producer warp's lane 0: streams the split's n_tiles KV tiles (K and V of C::T_TILE tokens per stage, as
+// 128-byte swizzled segments of C::SEG_ELEMS values) through the C::NSTAGE ring of full / empty mbarriers, then
+// waits until every copy it issued has landed (a CTA must not exit with copies in flight).
+template <class C>
+__device__ __forceinline__ void gqa_produce(const CUtensorMap* tmK, const CUtensorMap* tmV, const GqaParams& p,
+                                            uint8_t* stages, uint64_t* bars, int* s_abort, int b, int kvh, int L,
+                                            int kbeg, int n_tiles) {
+    prefetch_tensormap(tmK);
+    prefetch_tensormap(tmV);
+    const int ybase = (b * p.h_kv + kvh) * p.Lmax;
+    int issued = 0;
+    for (int it = 0; it < n_tiles; ++it) {
+        const int s = it % C::NSTAGE;
+        if (it >= C::NSTAGE) {
+            if (!mbar_wait(smem_u32(&bars[C::NSTAGE + s]), ((it / C::NSTAGE) - 1) & 1, p.status)) {
+                *s_abort = 1;
+                break;
+            }
+        }
+        if (*(volatile int*)s_abort) break;
+        const uint32_t full = smem_u32(&bars[s]);
+        mbar_arrive_expect_tx(full, C::STAGE_BYTES);
+        const uint32_t kdst = smem_u32(stages + s * C::STAGE_BYTES);
+        const uint32_t vdst = kdst + C::MAT_BYTES;
+        const int tok0 = kbeg + it * C::T_TILE;
+        if (!p.block_table) {
+            const int y = ybase + tok0;
+#pragma unroll
+            for (int sg = 0; sg < C::NSEG; ++sg) {
+                tma_load_2d(kdst + sg * C::T_TILE * 128, tmK, sg * C::SEG_ELEMS, y, full);
+                tma_load_2d(vdst + sg * C::T_TILE * 128, tmV, sg * C::SEG_ELEMS, y, full);
+            }
+        } else {
+            // paged cache: the tile is box_rows-row pieces, each inside one page of the block table
+            for (int r0 = 0; r0 < C::T_TILE; r0 += p.box_rows) {
+                const int tok = tok0 + r0;
+                const int y = paged_row(p, b, kvh, tok, tok < L);
+#pragma unroll
+                for (int sg = 0; sg < C::NSEG; ++sg) {
+                    tma_load_2d(kdst + sg * C::T_TILE * 128 + r0 * 128, tmK, sg * C::SEG_ELEMS, y, full);
+                    tma_load_2d(vdst + sg * C::T_TILE * 128 + r0 * 128, tmV, sg * C::SEG_ELEMS, y, full);
+                }
+            }
+        }
+        ++issued;
+    }
+    for (int it = issued - 1; it >= 0 && it >= issued - C::NSTAGE; --it)
+        mbar_wait(smem_u32(&bars[it % C::NSTAGE]), (it / C::NSTAGE) & 1, p.status);
+}
+
+// Merge of the four consumer warps' states of the block's rows (om [4][RB][D] normalisable outputs, mm / lm
+// [4][RB] log2-domain maxima and row sums, in shared memory) and the write of each row's result: the output (and
+// lse) when the row's keys fit one split, else the split's normalised fp32 partial and lse for the merge kernel.
+template <typename T, int D, int RB>
+__device__ __forceinline__ void gqa_merge_store(const float* om, const float* mm, const float* lm, const GqaParams& p,
+                                                int b, int kvh, int row0, int rows_here, int L, int kbeg, int split,
+                                                float v_mul) {
+    for (int idx = threadIdx.x; idx < rows_here * D; idx += 128) {
+        const int r = idx / D, d = idx % D;
+        const int gr = row0 + r;
+        const int t = gr % p.s_q;
+        const int hq = kvh * p.ratio + gr / p.s_q;
+        const size_t orow = ((size_t)b * p.h_q + hq) * p.s_q + t;
+        const int n_t = p.causal ? (L - p.s_q + t + 1) : L;
+        const int nsp = cdiv(n_t, p.split_tokens);
+        if (kbeg >= n_t) continue;  // this row has no keys in this split
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) M = fmaxf(M, mm[w * RB + r]);
+        float lsum = 0.f, acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const float f = exp2f(mm[w * RB + r] - M);  // warps without keys: exp2(-inf) = 0
+            lsum += f * lm[w * RB + r];
+            acc += f * om[(w * RB + r) * D + d];
+        }
+        const float ov = acc / lsum * v_mul;
+        const float lse2 = M + log2f(lsum);
+        if (nsp == 1) {
+            reinterpret_cast<T*>(p.out)[orow * D + d] = from_f32<T>(ov);
+            if (p.lse && d == 0) p.lse[orow] = lse2 * 0.69314718055994530942f;
+        } else {
+            p.part_o[(orow * p.nsplit_max + split) * D + d] = ov;
+            if (d == 0) p.part_lse[orow * p.nsplit_max + split] = lse2;
+        }
+    }
+}
+
 template <typename T, int D, int RB, typename KV>
 __global__ void __launch_bounds__(160, GqaCfg<KV, D, RB>::MINB)
     gqa_decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -252,7 +341,6 @@ __global__ void __launch_bounds__(160, GqaCfg<KV, D, RB>::MINB)
     if (kbeg >= need) return;  // no row of this block has keys in this split
     const int kend = min(need, kbeg + p.split_tokens);
     const int n_tiles = cdiv(kend - kbeg, C::T_TILE);
-    const int ybase = (b * p.h_kv + kvh) * p.Lmax;
 
     if (threadIdx.x == 0) {
         s_abort = 0;
@@ -266,49 +354,7 @@ __global__ void __launch_bounds__(160, GqaCfg<KV, D, RB>::MINB)
 
     if (warp == 4) {
         // ------------------------------ producer ------------------------------
-        if (lane == 0) {
-            prefetch_tensormap(&tmK);
-            prefetch_tensormap(&tmV);
-            int issued = 0;
-            for (int it = 0; it < n_tiles; ++it) {
-                const int s = it % C::NSTAGE;
-                if (it >= C::NSTAGE) {
-                    if (!mbar_wait(smem_u32(&bars[C::NSTAGE + s]), ((it / C::NSTAGE) - 1) & 1, p.status)) {
-                        s_abort = 1;
-                        break;
-                    }
-                }
-                if (*(volatile int*)&s_abort) break;
-                const uint32_t full = smem_u32(&bars[s]);
-                mbar_arrive_expect_tx(full, C::STAGE_BYTES);
-                const uint32_t kdst = smem_u32(stages + s * C::STAGE_BYTES);
-                const uint32_t vdst = kdst + C::MAT_BYTES;
-                const int tok0 = kbeg + it * C::T_TILE;
-                if (!p.block_table) {
-                    const int y = ybase + tok0;
-#pragma unroll
-                    for (int sg = 0; sg < C::NSEG; ++sg) {
-                        tma_load_2d(kdst + sg * C::T_TILE * 128, &tmK, sg * C::SEG_ELEMS, y, full);
-                        tma_load_2d(vdst + sg * C::T_TILE * 128, &tmV, sg * C::SEG_ELEMS, y, full);
-                    }
-                } else {
-                    // paged cache: the tile is box_rows-row pieces, each inside one page of the block table
-                    for (int r0 = 0; r0 < C::T_TILE; r0 += p.box_rows) {
-                        const int tok = tok0 + r0;
-                        const int y = paged_row(p, b, kvh, tok, tok < L);
-#pragma unroll
-                        for (int sg = 0; sg < C::NSEG; ++sg) {
-                            tma_load_2d(kdst + sg * C::T_TILE * 128 + r0 * 128, &tmK, sg * C::SEG_ELEMS, y, full);
-                            tma_load_2d(vdst + sg * C::T_TILE * 128 + r0 * 128, &tmV, sg * C::SEG_ELEMS, y, full);
-                        }
-                    }
-                }
-                ++issued;
-            }
-            // drain: every issued copy must land before the CTA may exit
-            for (int it = issued - 1; it >= 0 && it >= issued - C::NSTAGE; --it)
-                mbar_wait(smem_u32(&bars[it % C::NSTAGE]), (it / C::NSTAGE) & 1, p.status);
-        }
+        if (lane == 0) gqa_produce<C>(&tmK, &tmV, p, stages, bars, &s_abort, b, kvh, L, kbeg, n_tiles);
         return;
     }
 
@@ -559,35 +605,299 @@ __global__ void __launch_bounds__(160, GqaCfg<KV, D, RB>::MINB)
     named_barrier(1, 128);
 
     const float v_mul = p.v_scale ? p.v_scale[kvh] : 1.f;  // dequantisation scale of a quantised value cache
-    for (int idx = threadIdx.x; idx < rows_here * D; idx += 128) {
-        const int r = idx / D, d = idx % D;
-        const int gr = row0 + r;
-        const int t = gr % p.s_q;
-        const int hq = kvh * p.ratio + gr / p.s_q;
-        const size_t orow = ((size_t)b * p.h_q + hq) * p.s_q + t;
-        const int n_t = p.causal ? (L - p.s_q + t + 1) : L;
-        const int nsp = cdiv(n_t, p.split_tokens);
-        if (kbeg >= n_t) continue;  // this row has no keys in this split
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < 4; ++w) M = fmaxf(M, mm[w * RB + r]);
-        float lsum = 0.f, acc = 0.f;
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            const float f = exp2f(mm[w * RB + r] - M);  // warps without keys: exp2(-inf) = 0
-            lsum += f * lm[w * RB + r];
-            acc += f * om[(w * RB + r) * D + d];
+    gqa_merge_store<T, D, RB>(om, mm, lm, p, b, kvh, row0, rows_here, L, kbeg, split, v_mul);
+}
+
+// ---- tensor-core instance for bf16 caches (d in {64, 128}) ----------------------------------------------------
+// The block's query rows (up to 16: h_q / h_kv heads x s_q tokens; rows past R are zero padding) are the M = 16
+// rows of mma.sync m16n8k16 bf16 MMAs with fp32 accumulators.  Per tile each consumer warp takes 16 tokens: the
+// scores are d/16 k-steps x 2 n-tiles of MMAs whose K operand ldmatrix reads from the swizzled stage; the
+// accumulator layout of the score MMA is the A-operand layout of the P*V MMA, so P goes from the softmax to the
+// d/8 P*V MMAs in registers (as bf16, like every P of the library's tensor-core paths), with V read by the
+// transposing ldmatrix.  At about 4 FLOPs per cache byte the MMAs are not there for throughput: they replace the
+// score / value FMAs, shuffles and conversions of the CUDA-core loop (about 34 warp instructions per token and KV
+// head) with about 7, so that the consumers keep up with the TMA stream at two CTAs per SM.
+template <int D>
+struct GqaMmaCfg {
+    static constexpr int RB = 16;                  // query rows per CTA (the MMA's M)
+    static constexpr int TW = 16;                  // tokens per warp per tile
+    static constexpr int T_TILE = 4 * TW;
+    static constexpr int NSEG = D / 64;            // 128-byte swizzle segments per row
+    static constexpr int SEG_ELEMS = 64;
+    static constexpr int MAT_BYTES = T_TILE * D * 2;
+    static constexpr int STAGE_BYTES = 2 * MAT_BYTES;
+    static constexpr int NSTAGE0 = (LKA_GQA_STAGE_KB * 1024) / STAGE_BYTES;
+    static constexpr int NSTAGE = NSTAGE0 > 8 ? 8 : NSTAGE0;
+    static constexpr int RING = NSTAGE * STAGE_BYTES;
+    static constexpr int MERGE_BYTES = 4 * RB * D * 4 + 2 * 4 * RB * 4;
+    static constexpr int SMEM = 1024 + RING + 256;
+    static constexpr int MINB = 2;
+    static_assert(D == 64 || D == 128, "head dim of the tensor-core instance");
+    static_assert(MERGE_BYTES <= RING && NSTAGE >= 2 && 2 * SMEM <= 225 * 1024, "shared memory");
+};
+
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+                 "{%8, %9}, {%0, %1, %2, %3};"
+                 : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// Four 8x8 b16 matrices from shared memory; lane l gives the address of row l % 8 of matrix l / 8.
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr)
+                 : "memory");
+}
+// The same, each matrix transposed on the way into the registers.
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr)
+                 : "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(160, GqaMmaCfg<D>::MINB)
+    gqa_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                          const GqaParams p) {
+    using C = GqaMmaCfg<D>;
+    constexpr int RB = C::RB, KS = D / 16, NT = D / 8;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
+    uint8_t* stages = smem;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::RING);
+    __shared__ int s_abort;
+
+    const int split = blockIdx.x;
+    const int kvh = blockIdx.y / p.n_rb;
+    const int rb = blockIdx.y % p.n_rb;
+    const int b = blockIdx.z;
+    const int R = p.ratio * p.s_q;  // query rows of this group
+    const int row0 = rb * RB;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+    const int L = clamp_len(p.lens, b, p.Lmax, p.s_q, p.causal, p.status,
+                            threadIdx.x == 0 && split == 0 && kvh == 0 && rb == 0);
+    const int rows_here = R - row0 < RB ? R - row0 : RB;
+    int need = L;  // keys needed by the rows of this block: causal row t sees L - s_q + t + 1
+    if (p.causal) {
+        int tmax = 0;
+        for (int r = 0; r < rows_here; ++r) tmax = max(tmax, (row0 + r) % p.s_q);
+        need = L - p.s_q + tmax + 1;
+    }
+    const int kbeg = split * p.split_tokens;
+    if (kbeg >= need) return;  // no row of this block has keys in this split
+    const int kend = min(need, kbeg + p.split_tokens);
+    const int n_tiles = cdiv(kend - kbeg, C::T_TILE);
+
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        for (int s = 0; s < C::NSTAGE; ++s) {
+            mbar_init(smem_u32(&bars[s]), 1);              // full: producer arrival + tx bytes
+            mbar_init(smem_u32(&bars[C::NSTAGE + s]), 4);  // empty: one arrival per consumer warp
         }
-        const float ov = acc / lsum * v_mul;
-        const float lse2 = M + log2f(lsum);
-        if (nsp == 1) {
-            reinterpret_cast<T*>(p.out)[orow * D + d] = from_f32<T>(ov);
-            if (p.lse && d == 0) p.lse[orow] = lse2 * 0.69314718055994530942f;
-        } else {
-            p.part_o[(orow * p.nsplit_max + split) * D + d] = ov;
-            if (d == 0) p.part_lse[orow * p.nsplit_max + split] = lse2;
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    if (warp == 4) {
+        if (lane == 0) gqa_produce<C>(&tmK, &tmV, p, stages, bars, &s_abort, b, kvh, L, kbeg, n_tiles);
+        return;
+    }
+
+    // -------------------------------- consumers --------------------------------
+    // Fragment coordinates: lane = 4 g + tq holds rows g and g + 8 of the block and, in a score n-tile, the
+    // token columns 2 tq and 2 tq + 1.
+    const int g = lane >> 2, tq = lane & 3;
+    int last[2];  // last visible key of the lane's two rows (-1: a padding row, nothing visible)
+    uint32_t qa[KS][4];  // A fragments of the score MMA: the bf16 queries as given (the scale goes on the fp32 scores)
+    {
+        const __nv_bfloat16* qbase = reinterpret_cast<const __nv_bfloat16*>(p.q) +
+                                     ((size_t)(b * p.h_q + kvh * p.ratio) * p.s_q) * D;  // first row of the group
+        const uint32_t* qrow[2];
+        bool ok[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int gr = row0 + g + 8 * i;
+            ok[i] = gr < R;
+            last[i] = ok[i] ? (p.causal ? L - p.s_q + gr % p.s_q : L - 1) : -1;
+            qrow[i] = reinterpret_cast<const uint32_t*>(qbase + (size_t)(ok[i] ? gr : 0) * D);
+        }
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            qa[ks][0] = ok[0] ? qrow[0][8 * ks + tq] : 0u;
+            qa[ks][1] = ok[1] ? qrow[1][8 * ks + tq] : 0u;
+            qa[ks][2] = ok[0] ? qrow[0][8 * ks + 4 + tq] : 0u;
+            qa[ks][3] = ok[1] ? qrow[1][8 * ks + 4 + tq] : 0u;
         }
     }
+    float o[NT][4];
+#pragma unroll
+    for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+    // keys below mask_from are visible to every row of the block: tiles below it need no mask
+    int mask_from = kend;
+    for (int r = 0; r < rows_here; ++r)
+        mask_from = min(mask_from, p.causal ? L - p.s_q + (row0 + r) % p.s_q + 1 : L);
+
+    // ldmatrix row addresses (byte offsets inside a stage's K or V matrix, 128-byte swizzle: chunk ^ row % 8).
+    // Keys: matrix l / 8 = (token half l / 16, 8-value chunk parity (l / 8) % 2) of the warp's 16 tokens: the
+    // b0 / b1 fragments of n-tiles 0 and 1 for one k-step.  Values (transposed): matrix l / 8 = (chunk parity
+    // l / 16, token half (l / 8) % 2): b0 / b1 of two adjacent 8-column n-tiles of the output.
+    const int r8 = lane & 7;
+    const uint32_t k_row = (uint32_t)(16 * warp + 8 * (lane >> 4) + r8) * 128;
+    const uint32_t v_row = (uint32_t)(16 * warp + 8 * ((lane >> 3) & 1) + r8) * 128;
+    uint32_t k_off[4], v_off[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        k_off[c] = k_row + ((uint32_t)((2 * c + ((lane >> 3) & 1)) ^ r8) << 4);
+        v_off[c] = v_row + ((uint32_t)((2 * c + (lane >> 4)) ^ r8) << 4);
+    }
+
+    bool aborted = false;
+    for (int it = 0; it < n_tiles; ++it) {
+        const int s = it % C::NSTAGE;
+        if (!mbar_wait(smem_u32(&bars[s]), (it / C::NSTAGE) & 1, p.status)) {
+            aborted = true;
+            s_abort = 1;
+            break;
+        }
+        const uint32_t kt = smem_u32(stages + s * C::STAGE_BYTES);
+        const uint32_t vt = kt + C::MAT_BYTES;
+        const int tbase = kbeg + it * C::T_TILE;
+
+        // ---- S = Q K^T for the warp's 16 tokens (two accumulators per n-tile: even / odd k-steps) ----
+        float sc[2][2][4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) sc[nt][h][0] = sc[nt][h][1] = sc[nt][h][2] = sc[nt][h][3] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            uint32_t kb[4];
+            ldsm_x4(kt + (ks >> 2) * C::T_TILE * 128 + k_off[ks & 3], kb);
+            mma_bf16_16816(sc[0][ks & 1], qa[ks], kb[0], kb[1]);
+            mma_bf16_16816(sc[1][ks & 1], qa[ks], kb[2], kb[3]);
+        }
+        // x[nt][e]: row g (e < 2) or g + 8, token tbase + 16 warp + 8 nt + 2 tq + e % 2, in the log2 domain
+        float x[2][4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) x[nt][e] = (sc[nt][0][e] + sc[nt][1][e]) * p.scale_log2;
+        if (tbase + C::T_TILE > mask_from) {
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int tok = tbase + 16 * warp + 8 * nt + 2 * tq + (e & 1);
+                    x[nt][e] = (tok < kend && tok <= last[e >> 1]) ? x[nt][e] : -INFINITY;
+                }
+        }
+        // ---- online softmax of the two rows, lazily rescaled: p is taken against a reference maximum m_run
+        // that only moves when a score exceeds it by more than 2^8 (the final O / l is exact) ----
+        float mx[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            mx[i] = fmaxf(fmaxf(x[0][2 * i], x[0][2 * i + 1]), fmaxf(x[1][2 * i], x[1][2 * i + 1]));
+            mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 1));
+            mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 2));
+        }
+        if (__any_sync(0xffffffffu, mx[0] > m_run[0] + 8.0f || mx[1] > m_run[1] + 8.0f)) {
+            float alpha[2];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const float m_new = fmaxf(m_run[i], mx[i]);
+                alpha[i] = 1.f;
+                if (m_run[i] == -INFINITY) {
+                    m_run[i] = m_new;  // O and l of the row are still zero
+                } else if (m_new > m_run[i] + 8.0f) {
+                    alpha[i] = fast_exp2(m_run[i] - m_new);
+                    m_run[i] = m_new;
+                }
+                l_run[i] *= alpha[i];
+            }
+#pragma unroll
+            for (int j = 0; j < NT; ++j) {
+                o[j][0] *= alpha[0];
+                o[j][1] *= alpha[0];
+                o[j][2] *= alpha[1];
+                o[j][3] *= alpha[1];
+            }
+        }
+        uint32_t pa[4];  // A fragment of the P*V MMA (k = the warp's 16 tokens)
+        {
+            const float ms0 = m_run[0] == -INFINITY ? 0.f : m_run[0];  // no visible key yet: p = 2^-inf = 0
+            const float ms1 = m_run[1] == -INFINITY ? 0.f : m_run[1];
+            float pr[2][4];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                pr[nt][0] = fast_exp2(x[nt][0] - ms0);
+                pr[nt][1] = fast_exp2(x[nt][1] - ms0);
+                pr[nt][2] = fast_exp2(x[nt][2] - ms1);
+                pr[nt][3] = fast_exp2(x[nt][3] - ms1);
+                l_run[0] += pr[nt][0] + pr[nt][1];  // this lane's share; summed over the row's lanes at the end
+                l_run[1] += pr[nt][2] + pr[nt][3];
+            }
+            pa[0] = pack_bf16x2(pr[0][0], pr[0][1]);
+            pa[1] = pack_bf16x2(pr[0][2], pr[0][3]);
+            pa[2] = pack_bf16x2(pr[1][0], pr[1][1]);
+            pa[3] = pack_bf16x2(pr[1][2], pr[1][3]);
+        }
+        // value rows of the warp past the split's keys (the last tile) may hold anything, even NaN, and P = 0
+        // does not cancel that in the MMA: zero them
+        const int nvalid = kend - (tbase + 16 * warp);
+        if (nvalid < 16) {
+            const int first = nvalid < 0 ? 0 : nvalid;
+            uint8_t* vrow = stages + s * C::STAGE_BYTES + C::MAT_BYTES;
+            for (int idx = lane; idx < (16 - first) * C::NSEG * 8; idx += 32) {
+                const int row = 16 * warp + first + idx / (C::NSEG * 8), rem = idx % (C::NSEG * 8);
+                *reinterpret_cast<uint4*>(vrow + (rem / 8) * C::T_TILE * 128 + row * 128 + (rem % 8) * 16) =
+                    make_uint4(0u, 0u, 0u, 0u);
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // before the ring's next copy
+            __syncwarp();
+        }
+        // ---- O += P V ----
+#pragma unroll
+        for (int cc = 0; cc < NT / 2; ++cc) {
+            uint32_t vb[4];
+            ldsm_x4_t(vt + (cc >> 2) * C::T_TILE * 128 + v_off[cc & 3], vb);
+            mma_bf16_16816(o[2 * cc], pa, vb[0], vb[1]);
+            mma_bf16_16816(o[2 * cc + 1], pa, vb[2], vb[3]);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars[C::NSTAGE + s]));
+    }
+
+    // the row sums: this lane's share summed over the four lanes of the row
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        l_run[i] += __shfl_xor_sync(0xffffffffu, l_run[i], 1);
+        l_run[i] += __shfl_xor_sync(0xffffffffu, l_run[i], 2);
+    }
+    // all consumer warps reach here; aborted CTAs stop without writing results
+    named_barrier(1, 128);
+    if (*(volatile int*)&s_abort || aborted) return;
+
+    // ---- merge the four warp states in shared memory (reusing the stage ring) ----
+    float* om = reinterpret_cast<float*>(stages);  // [4][RB][D]
+    float* mm = om + 4 * RB * D;                    // [4][RB]
+    float* lm = mm + 4 * RB;                        // [4][RB]
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+        *reinterpret_cast<float2*>(&om[(warp * RB + g) * D + 8 * j + 2 * tq]) = make_float2(o[j][0], o[j][1]);
+        *reinterpret_cast<float2*>(&om[(warp * RB + g + 8) * D + 8 * j + 2 * tq]) = make_float2(o[j][2], o[j][3]);
+    }
+    if (tq == 0) {
+        mm[warp * RB + g] = m_run[0];
+        mm[warp * RB + g + 8] = m_run[1];
+        lm[warp * RB + g] = l_run[0];
+        lm[warp * RB + g + 8] = l_run[1];
+    }
+    named_barrier(1, 128);
+    gqa_merge_store<__nv_bfloat16, D, RB>(om, mm, lm, p, b, kvh, row0, rows_here, L, kbeg, split, 1.f);
 }
 
 // Merge of split partials: with w_i = 2^(lse_i - max lse),
@@ -666,6 +976,27 @@ static cudaError_t launch_one(const CUtensorMap& tk, const CUtensorMap& tv, cons
     return e;
 }
 
+template <int D>
+static cudaError_t launch_mma(const CUtensorMap& tk, const CUtensorMap& tv, const GqaParams& p, int nsplit,
+                              cudaStream_t st) {
+    using C = GqaMmaCfg<D>;
+    auto kern = gqa_decode_mma_kernel<D>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    dim3 grid(nsplit, p.h_kv * p.n_rb, p.B);
+    TimedLaunch timer(st);
+    kern<<<grid, 160, C::SMEM, st>>>(tk, tv, p);
+    timer.stop();
+    e = cudaPeekAtLastError();
+    if (e != cudaSuccess) return e;
+    const size_t nrows = (size_t)p.B * p.h_q * p.s_q;
+    if (nsplit > 1) {
+        gqa_combine_kernel<__nv_bfloat16, D><<<(unsigned)((nrows + 3) / 4), 128, 0, st>>>(p);
+        e = cudaPeekAtLastError();
+    }
+    return e;
+}
+
 cudaError_t gqa_combine_launch(const GqaParams& p, int dtype_bytes, int d, cudaStream_t st) {
     const size_t nrows = (size_t)p.B * p.h_q * p.s_q;
     const unsigned grid = (unsigned)((nrows + 3) / 4);
@@ -684,10 +1015,10 @@ int gqa_tile_tokens(int dtype_bytes, int d, int rb, int* ctas_per_sm) {
         if (ctas_per_sm) *ctas_per_sm = GqaCfg<T, DD, R>::MINB; \
         return GqaCfg<T, DD, R>::T_TILE;                         \
     }
-    LKA_TILE_CASE(__nv_bfloat16, 64, 1) LKA_TILE_CASE(__nv_bfloat16, 64, 2) LKA_TILE_CASE(__nv_bfloat16, 64, 4)
-    LKA_TILE_CASE(__nv_bfloat16, 64, 8)
-    LKA_TILE_CASE(__nv_bfloat16, 128, 1) LKA_TILE_CASE(__nv_bfloat16, 128, 2) LKA_TILE_CASE(__nv_bfloat16, 128, 4)
-    LKA_TILE_CASE(__nv_bfloat16, 128, 8) LKA_TILE_CASE(__nv_bfloat16, 128, 16)
+    if (dtype_bytes == 2 && (d == 64 || d == 128) && rb == 16) {  // the tensor-core instance
+        if (ctas_per_sm) *ctas_per_sm = d == 64 ? GqaMmaCfg<64>::MINB : GqaMmaCfg<128>::MINB;
+        return d == 64 ? GqaMmaCfg<64>::T_TILE : GqaMmaCfg<128>::T_TILE;
+    }
     LKA_TILE_CASE(__nv_bfloat16, 256, 1) LKA_TILE_CASE(__nv_bfloat16, 256, 2) LKA_TILE_CASE(__nv_bfloat16, 256, 4)
     LKA_TILE_CASE(__nv_bfloat16, 256, 8)
     LKA_TILE_CASE(float, 64, 1) LKA_TILE_CASE(float, 64, 2) LKA_TILE_CASE(float, 64, 4) LKA_TILE_CASE(float, 64, 8)
@@ -702,11 +1033,8 @@ cudaError_t gqa_decode_launch(const CUtensorMap& tk, const CUtensorMap& tv, cons
                               int d, int rb, int nsplit, cudaStream_t st) {
 #define LKA_LAUNCH_CASE(T, DD, R) \
     if (dtype_bytes == (int)sizeof(T) && d == DD && rb == R) return launch_one<T, DD, R>(tk, tv, p, nsplit, st);
-    LKA_LAUNCH_CASE(__nv_bfloat16, 64, 1) LKA_LAUNCH_CASE(__nv_bfloat16, 64, 2)
-    LKA_LAUNCH_CASE(__nv_bfloat16, 64, 4) LKA_LAUNCH_CASE(__nv_bfloat16, 64, 8)
-    LKA_LAUNCH_CASE(__nv_bfloat16, 128, 1) LKA_LAUNCH_CASE(__nv_bfloat16, 128, 2)
-    LKA_LAUNCH_CASE(__nv_bfloat16, 128, 4) LKA_LAUNCH_CASE(__nv_bfloat16, 128, 8)
-    LKA_LAUNCH_CASE(__nv_bfloat16, 128, 16)
+    if (dtype_bytes == 2 && d == 64 && rb == 16) return launch_mma<64>(tk, tv, p, nsplit, st);
+    if (dtype_bytes == 2 && d == 128 && rb == 16) return launch_mma<128>(tk, tv, p, nsplit, st);
     LKA_LAUNCH_CASE(__nv_bfloat16, 256, 1) LKA_LAUNCH_CASE(__nv_bfloat16, 256, 2)
     LKA_LAUNCH_CASE(__nv_bfloat16, 256, 4) LKA_LAUNCH_CASE(__nv_bfloat16, 256, 8)
     LKA_LAUNCH_CASE(float, 64, 1) LKA_LAUNCH_CASE(float, 64, 2) LKA_LAUNCH_CASE(float, 64, 4)
