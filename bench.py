@@ -274,7 +274,7 @@ class GqaDecodePaged(GqaDecode):
 class GqaDecodeFp8(GqaDecode):
     """gqa_attn_fp8kv over the same decode batch with the K/V cache in e4m3 (one scale per KV head)."""
 
-    kernel = "gqa_decode_kernel"  # the CUDA-core instance (e4m3 values widened per lane)
+    kernel = "gqa_decode_mma_kernel"  # the e4m3 tensor-core instance (f16 MMAs)
 
     def setup_costs(self):
         w = self.w

@@ -11,6 +11,8 @@
  *    with the last dimension contiguous, 16-byte aligned.  The library never
  *    allocates device memory and keeps no per-call state: scratch space is the
  *    caller's workspace `ws` (size from the matching *_workspace_size call).
+ *    A workspace must be zero-filled before its first use: its first 256
+ *    bytes hold the sticky status word (see lka_device_status).
  *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is the
  *    legacy default stream).  Calls on one workspace must not overlap.
  *  - cache_lens is a DEVICE int32 array [B]: cache_lens[b] = L_b counts the

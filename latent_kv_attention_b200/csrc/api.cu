@@ -57,8 +57,9 @@ struct GqaPlan {
 };
 
 static int pick_rb(int rows, int d, int dtype_bytes, bool fp8kv) {
-    // bf16 caches with d <= 128: the tensor-core instance, whose MMA tile holds 16 query rows
-    if (!fp8kv && dtype_bytes == 2 && d <= 128) return 16;
+    // bf16 caches with d <= 128 and e4m3 caches with d = 128: the tensor-core instances, whose MMA tile holds
+    // 16 query rows
+    if ((!fp8kv && dtype_bytes == 2 && d <= 128) || (fp8kv && d == 128)) return 16;
     int cap = fp8kv ? 4 : 16;
     if (d == 256) cap = fp8kv ? 4 : 8;
     int rb = 1;

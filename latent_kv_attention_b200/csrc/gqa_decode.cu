@@ -608,39 +608,73 @@ __global__ void __launch_bounds__(160, GqaCfg<KV, D, RB>::MINB)
     gqa_merge_store<T, D, RB>(om, mm, lm, p, b, kvh, row0, rows_here, L, kbeg, split, v_mul);
 }
 
-// ---- tensor-core instance for bf16 caches (d in {64, 128}) ----------------------------------------------------
+// Whether `pred` holds in any of the 128 consumer threads (named barrier 1 with an OR reduction): a value every
+// consumer sees the same.
+__device__ __forceinline__ bool consumers_any(bool pred) {
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 1, 128, p;\n\t"
+                 "selp.u32 %0, 1, 0, q;\n\t}"
+                 : "=r"(r)
+                 : "r"((uint32_t)pred)
+                 : "memory");
+    return r != 0;
+}
+
+// ---- tensor-core instances: bf16 caches (d in {64, 128}) and e4m3 caches (d = 128) -------------------------------
 // The block's query rows (up to 16: h_q / h_kv heads x s_q tokens; rows past R are zero padding) are the M = 16
-// rows of mma.sync m16n8k16 bf16 MMAs with fp32 accumulators.  Per tile each consumer warp takes 16 tokens: the
-// scores are d/16 k-steps x 2 n-tiles of MMAs whose K operand ldmatrix reads from the swizzled stage; the
-// accumulator layout of the score MMA is the A-operand layout of the P*V MMA, so P goes from the softmax to the
-// d/8 P*V MMAs in registers (as bf16, like every P of the library's tensor-core paths), with V read by the
-// transposing ldmatrix.  At about 4 FLOPs per cache byte the MMAs are not there for throughput: they replace the
-// score / value FMAs, shuffles and conversions of the CUDA-core loop (about 34 warp instructions per token and KV
-// head) with about 7, so that the consumers keep up with the TMA stream at two CTAs per SM.
-template <int D>
+// rows of mma.sync m16n8k16 MMAs with fp32 accumulators.  Per tile each consumer warp takes 16 tokens: the scores
+// are d/16 k-steps x 2 n-tiles of MMAs, and the accumulator layout of the score MMA is the A-operand layout of the
+// P*V MMA, so P goes from the softmax to the d/8 P*V MMAs in registers.  At about 4 FLOPs per cache byte the MMAs
+// are not there for throughput: they replace the score / value FMAs, shuffles and conversions of the CUDA-core loop
+// (about 34 warp instructions per token and KV head) with a handful, so that the consumers keep up with the TMA
+// stream at two CTAs per SM.
+//   bf16 cache: bf16 MMAs; ldmatrix reads K (and, transposed, V) straight from the swizzled stage; P is bf16 (as in
+//     every tensor-core path of the library).
+//   e4m3 cache: f16 MMAs (e4m3 -> f16 is exact; q bf16 -> f16 too, for values of ordinary size).  The score
+//     contraction runs over the head dim in a permuted order, the same for q and k, so that each lane reads 16
+//     consecutive key bytes per token with one shared-memory load and widens them in registers: in 64-value
+//     group G, lane tq's k-step 4 G + j covers values 64 G + 16 tq + 4 j + {0, 1} (as k = 2 tq, 2 tq + 1) and
+//     + {2, 3} (as k = 2 tq + 8, 2 tq + 9).  The n-th token column of an n-tile is token pi(n) = n / 2 + 4 (n % 2)
+//     of its 8 (so that the two rows a shared-memory phase reads fall in different bank halves); each warp widens
+//     its 16 value rows once per tile into an f16 scratch tile (in that token order, zero past the split's keys),
+//     which the transposing ldmatrix reads as in the bf16 case.  P is f16; the per-KV-head scales are applied to
+//     the fp32 scores and to the merged output.
+template <int D, bool F8>
 struct GqaMmaCfg {
     static constexpr int RB = 16;                  // query rows per CTA (the MMA's M)
     static constexpr int TW = 16;                  // tokens per warp per tile
     static constexpr int T_TILE = 4 * TW;
-    static constexpr int NSEG = D / 64;            // 128-byte swizzle segments per row
-    static constexpr int SEG_ELEMS = 64;
-    static constexpr int MAT_BYTES = T_TILE * D * 2;
+    static constexpr int E = F8 ? 1 : 2;           // bytes per cache element
+    static constexpr int SEG_ELEMS = 128 / E;      // elements per 128-byte swizzle segment (TMA box width)
+    static constexpr int NSEG = D * E / 128;
+    static constexpr int MAT_BYTES = T_TILE * D * E;
     static constexpr int STAGE_BYTES = 2 * MAT_BYTES;
     static constexpr int NSTAGE0 = (LKA_GQA_STAGE_KB * 1024) / STAGE_BYTES;
-    static constexpr int NSTAGE = NSTAGE0 > 8 ? 8 : NSTAGE0;
+    static constexpr int NSTAGE_CAP = F8 ? 3 : 6;
+    static constexpr int NSTAGE = NSTAGE0 > NSTAGE_CAP ? NSTAGE_CAP : NSTAGE0;
     static constexpr int RING = NSTAGE * STAGE_BYTES;
+    static constexpr int SCR_W = F8 ? TW * D * 2 : 0;  // per-warp f16 value tile (e4m3 cache)
+    static constexpr int OFF_BAR = RING + 4 * SCR_W;
     static constexpr int MERGE_BYTES = 4 * RB * D * 4 + 2 * 4 * RB * 4;
-    static constexpr int SMEM = 1024 + RING + 256;
-    static constexpr int MINB = 2;
-    static_assert(D == 64 || D == 128, "head dim of the tensor-core instance");
-    static_assert(MERGE_BYTES <= RING && NSTAGE >= 2 && 2 * SMEM <= 225 * 1024, "shared memory");
+    static constexpr int SMEM = 1024 + OFF_BAR + 256;
+    // resident CTAs per SM: the e4m3 consumers do more work per byte (the widening), so more of them hide latency
+    static constexpr int MINB = F8 ? 3 : 2;
+    static_assert(F8 ? D == 128 : (D == 64 || D == 128), "head dim of the tensor-core instances");
+    static_assert(MERGE_BYTES <= RING && NSTAGE >= 2 && MINB * (SMEM + 1024) <= 228 * 1024, "shared memory");
 };
 
-__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-                 "{%8, %9}, {%0, %1, %2, %3};"
-                 : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+template <bool F16>
+__device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    if constexpr (F16)
+        asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+                     "{%8, %9}, {%0, %1, %2, %3};"
+                     : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+                     : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    else
+        asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+                     "{%8, %9}, {%0, %1, %2, %3};"
+                     : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+                     : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 // Four 8x8 b16 matrices from shared memory; lane l gives the address of row l % 8 of matrix l / 8.
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
@@ -656,17 +690,37 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
                  : "r"(addr)
                  : "memory");
 }
+// The two e4m3 values of the low (bytes 0, 1) or high (bytes 2, 3) half of w as an f16 pair, exactly; the lower
+// byte becomes the lower half.  One conversion instruction reading the register half in place.
+__device__ __forceinline__ uint32_t e4m3x2_lo_to_f16x2(uint32_t w) {
+    uint32_t r;
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, lo;\n\t}" : "=r"(r) : "r"(w));
+    return r;
+}
+__device__ __forceinline__ uint32_t e4m3x2_hi_to_f16x2(uint32_t w) {
+    uint32_t r;
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, hi;\n\t}" : "=r"(r) : "r"(w));
+    return r;
+}
+__device__ __forceinline__ uint32_t pack_f16x2_rn(float lo, float hi) {
+    const __half2 v = __floats2half2_rn(lo, hi);  // .x = lo (low 16 bits), .y = hi
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+// Physical token (of 8) of token column n of an n-tile in the e4m3 instance, and the inverse.
+__device__ __forceinline__ int f8_tok(int n) { return (n >> 1) + 4 * (n & 1); }
+__device__ __forceinline__ int f8_col(int t) { return 2 * (t & 3) + (t >> 2); }
 
-template <int D>
-__global__ void __launch_bounds__(160, GqaMmaCfg<D>::MINB)
+// (two CTAs per SM whatever the cache type: the 16-row e4m3 form does not fit three in registers)
+template <int D, bool F8>
+__global__ void __launch_bounds__(160, 2)
     gqa_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                           const GqaParams p) {
-    using C = GqaMmaCfg<D>;
+    using C = GqaMmaCfg<D, F8>;
     constexpr int RB = C::RB, KS = D / 16, NT = D / 8;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
     uint8_t* stages = smem;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::RING);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     __shared__ int s_abort;
 
     const int split = blockIdx.x;
@@ -711,7 +765,7 @@ __global__ void __launch_bounds__(160, GqaMmaCfg<D>::MINB)
     // token columns 2 tq and 2 tq + 1.
     const int g = lane >> 2, tq = lane & 3;
     int last[2];  // last visible key of the lane's two rows (-1: a padding row, nothing visible)
-    uint32_t qa[KS][4];  // A fragments of the score MMA: the bf16 queries as given (the scale goes on the fp32 scores)
+    uint32_t qa[KS][4];  // A fragments of the score MMA: the queries as given (the scale goes on the fp32 scores)
     {
         const __nv_bfloat16* qbase = reinterpret_cast<const __nv_bfloat16*>(p.q) +
                                      ((size_t)(b * p.h_q + kvh * p.ratio) * p.s_q) * D;  // first row of the group
@@ -724,36 +778,58 @@ __global__ void __launch_bounds__(160, GqaMmaCfg<D>::MINB)
             last[i] = ok[i] ? (p.causal ? L - p.s_q + gr % p.s_q : L - 1) : -1;
             qrow[i] = reinterpret_cast<const uint32_t*>(qbase + (size_t)(ok[i] ? gr : 0) * D);
         }
+        // bf16 pair u (values 2u, 2u + 1) of row i, as the MMA's operand type
+        auto qpair = [&](int i, int u) -> uint32_t {
+            const uint32_t w = ok[i] ? qrow[i][u] : 0u;
+            if constexpr (F8) {
+                float lo, hi;
+                bf16x2_to_f32(w, lo, hi);
+                return pack_f16x2_rn(lo, hi);
+            } else {
+                return w;
+            }
+        };
 #pragma unroll
         for (int ks = 0; ks < KS; ++ks) {
-            qa[ks][0] = ok[0] ? qrow[0][8 * ks + tq] : 0u;
-            qa[ks][1] = ok[1] ? qrow[1][8 * ks + tq] : 0u;
-            qa[ks][2] = ok[0] ? qrow[0][8 * ks + 4 + tq] : 0u;
-            qa[ks][3] = ok[1] ? qrow[1][8 * ks + 4 + tq] : 0u;
+            // pairs of values: bf16 layout 16 ks + 2 tq (+ 8); e4m3 permuted layout 64 G + 16 tq + 4 j (+ 2)
+            const int u0 = F8 ? 32 * (ks >> 2) + 8 * tq + 2 * (ks & 3) : 8 * ks + tq;
+            const int u1 = F8 ? u0 + 1 : u0 + 4;
+            qa[ks][0] = qpair(0, u0);
+            qa[ks][1] = qpair(1, u0);
+            qa[ks][2] = qpair(0, u1);
+            qa[ks][3] = qpair(1, u1);
         }
     }
     float o[NT][4];
 #pragma unroll
     for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
     float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+    // the softmax scale in the log2 domain, and the dequantisation scale of an e4m3 key cache
+    const float s_mul = F8 ? p.scale_log2 * p.k_scale[kvh] : p.scale_log2;
     // keys below mask_from are visible to every row of the block: tiles below it need no mask
     int mask_from = kend;
     for (int r = 0; r < rows_here; ++r)
         mask_from = min(mask_from, p.causal ? L - p.s_q + (row0 + r) % p.s_q + 1 : L);
+    // token (of the warp's 16) of score element (nt, e) of this lane
+    auto tok_of = [&](int nt, int e) { return 8 * nt + (F8 ? f8_tok(2 * tq + (e & 1)) : 2 * tq + (e & 1)); };
 
-    // ldmatrix row addresses (byte offsets inside a stage's K or V matrix, 128-byte swizzle: chunk ^ row % 8).
-    // Keys: matrix l / 8 = (token half l / 16, 8-value chunk parity (l / 8) % 2) of the warp's 16 tokens: the
-    // b0 / b1 fragments of n-tiles 0 and 1 for one k-step.  Values (transposed): matrix l / 8 = (chunk parity
-    // l / 16, token half (l / 8) % 2): b0 / b1 of two adjacent 8-column n-tiles of the output.
+    // ldmatrix row addresses (byte offsets, 128-byte swizzle: chunk ^ row % 8).  bf16 keys: matrix l / 8 = (token
+    // half l / 16, 8-value chunk parity (l / 8) % 2) of the warp's 16 tokens: the b0 / b1 fragments of n-tiles 0
+    // and 1 for one k-step.  Values (transposed; the stage for bf16, the warp's scratch tile for e4m3): matrix
+    // l / 8 = (chunk parity l / 16, token half (l / 8) % 2): b0 / b1 of two adjacent 8-column output n-tiles.
     const int r8 = lane & 7;
     const uint32_t k_row = (uint32_t)(16 * warp + 8 * (lane >> 4) + r8) * 128;
-    const uint32_t v_row = (uint32_t)(16 * warp + 8 * ((lane >> 3) & 1) + r8) * 128;
+    const uint32_t v_row = (uint32_t)((F8 ? 0 : 16 * warp) + 8 * ((lane >> 3) & 1) + r8) * 128;
+    constexpr int V_SEG = F8 ? C::TW * 128 : C::T_TILE * 128;  // bytes per 64-value segment of a value tile
     uint32_t k_off[4], v_off[4];
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
         k_off[c] = k_row + ((uint32_t)((2 * c + ((lane >> 3) & 1)) ^ r8) << 4);
         v_off[c] = v_row + ((uint32_t)((2 * c + (lane >> 4)) ^ r8) << 4);
     }
+    // e4m3: this lane's key row of n-tile nt (token column g) and value row to widen (token lane / 2, half lane % 2)
+    uint8_t* scr = smem + C::RING + warp * C::SCR_W;
+    const int kf_row0 = 16 * warp + f8_tok(g);
 
     bool aborted = false;
     for (int it = 0; it < n_tiles; ++it) {
@@ -773,25 +849,44 @@ __global__ void __launch_bounds__(160, GqaMmaCfg<D>::MINB)
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
             for (int h = 0; h < 2; ++h) sc[nt][h][0] = sc[nt][h][1] = sc[nt][h][2] = sc[nt][h][3] = 0.f;
+        if constexpr (F8) {
+            const uint8_t* kst = stages + s * C::STAGE_BYTES;
 #pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-            uint32_t kb[4];
-            ldsm_x4(kt + (ks >> 2) * C::T_TILE * 128 + k_off[ks & 3], kb);
-            mma_bf16_16816(sc[0][ks & 1], qa[ks], kb[0], kb[1]);
-            mma_bf16_16816(sc[1][ks & 1], qa[ks], kb[2], kb[3]);
+            for (int nt = 0; nt < 2; ++nt) {
+                const int row = kf_row0 + 8 * nt;
+#pragma unroll
+                for (int G = 0; G < D / 64; ++G) {
+                    const int seg = G >> 1, chunk = 4 * (G & 1) + tq;
+                    const uint4 w = *reinterpret_cast<const uint4*>(kst + seg * C::T_TILE * 128 + row * 128 +
+                                                                    ((chunk ^ (row & 7)) << 4));
+                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        mma_16816<true>(sc[nt][j & 1], qa[4 * G + j], e4m3x2_lo_to_f16x2(ws[j]),
+                                        e4m3x2_hi_to_f16x2(ws[j]));
+                }
+            }
+        } else {
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+                uint32_t kb[4];
+                ldsm_x4(kt + (ks >> 2) * C::T_TILE * 128 + k_off[ks & 3], kb);
+                mma_16816<false>(sc[0][ks & 1], qa[ks], kb[0], kb[1]);
+                mma_16816<false>(sc[1][ks & 1], qa[ks], kb[2], kb[3]);
+            }
         }
-        // x[nt][e]: row g (e < 2) or g + 8, token tbase + 16 warp + 8 nt + 2 tq + e % 2, in the log2 domain
+        // x[nt][e]: row g (e < 2) or g + 8, token tbase + 16 warp + tok_of(nt, e), in the log2 domain
         float x[2][4];
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) x[nt][e] = (sc[nt][0][e] + sc[nt][1][e]) * p.scale_log2;
+            for (int e = 0; e < 4; ++e) x[nt][e] = (sc[nt][0][e] + sc[nt][1][e]) * s_mul;
         if (tbase + C::T_TILE > mask_from) {
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const int tok = tbase + 16 * warp + 8 * nt + 2 * tq + (e & 1);
+                    const int tok = tbase + 16 * warp + tok_of(nt, e);
                     x[nt][e] = (tok < kend && tok <= last[e >> 1]) ? x[nt][e] : -INFINITY;
                 }
         }
@@ -826,7 +921,7 @@ __global__ void __launch_bounds__(160, GqaMmaCfg<D>::MINB)
                 o[j][3] *= alpha[1];
             }
         }
-        uint32_t pa[4];  // A fragment of the P*V MMA (k = the warp's 16 tokens)
+        uint32_t pa[4];  // A fragment of the P*V MMA (k = the warp's 16 tokens in score-column order)
         {
             const float ms0 = m_run[0] == -INFINITY ? 0.f : m_run[0];  // no visible key yet: p = 2^-inf = 0
             const float ms1 = m_run[1] == -INFINITY ? 0.f : m_run[1];
@@ -840,15 +935,50 @@ __global__ void __launch_bounds__(160, GqaMmaCfg<D>::MINB)
                 l_run[0] += pr[nt][0] + pr[nt][1];  // this lane's share; summed over the row's lanes at the end
                 l_run[1] += pr[nt][2] + pr[nt][3];
             }
-            pa[0] = pack_bf16x2(pr[0][0], pr[0][1]);
-            pa[1] = pack_bf16x2(pr[0][2], pr[0][3]);
-            pa[2] = pack_bf16x2(pr[1][0], pr[1][1]);
-            pa[3] = pack_bf16x2(pr[1][2], pr[1][3]);
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                pa[2 * nt] = F8 ? pack_f16x2_rn(pr[nt][0], pr[nt][1]) : pack_bf16x2(pr[nt][0], pr[nt][1]);
+                pa[2 * nt + 1] = F8 ? pack_f16x2_rn(pr[nt][2], pr[nt][3]) : pack_bf16x2(pr[nt][2], pr[nt][3]);
+            }
         }
-        // value rows of the warp past the split's keys (the last tile) may hold anything, even NaN, and P = 0
-        // does not cancel that in the MMA: zero them
-        const int nvalid = kend - (tbase + 16 * warp);
-        if (nvalid < 16) {
+        uint32_t vbase = vt;
+        const int nvalid = kend - (tbase + 16 * warp);  // value rows of the warp that are keys of the split
+        if constexpr (F8) {
+            // widen the warp's 16 value rows into its f16 scratch tile, rows in score-column order; rows past the
+            // split's keys may hold anything (even NaN), which P = 0 would not cancel in the MMA: they become 0
+            const int t = lane >> 1, hf = lane & 1;
+            const int srow = 16 * warp + t;                   // stage row
+            const int lrow = 8 * (t >> 3) + f8_col(t & 7);    // scratch row
+            const bool live = t < nvalid, tail = nvalid < 16;  // (tail: warp-uniform, the last tile only)
+            const uint8_t* vsrc = stages + s * C::STAGE_BYTES + C::MAT_BYTES;
+#pragma unroll
+            for (int i = 0; i < D / 32; ++i) {  // 16 e4m3 values: scratch chunks 2 i, 2 i + 1 of segment hf
+                const int byte = hf * (D / 2) + 16 * i;
+                const int ch = (byte % 128) / 16;
+                uint4 w = *reinterpret_cast<const uint4*>(vsrc + (byte / 128) * C::T_TILE * 128 + srow * 128 +
+                                                          ((ch ^ (srow & 7)) << 4));
+                if (tail && !live) w = make_uint4(0u, 0u, 0u, 0u);
+                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+                uint32_t hv[8];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    hv[2 * q] = e4m3x2_lo_to_f16x2(ws[q]);
+                    hv[2 * q + 1] = e4m3x2_hi_to_f16x2(ws[q]);
+                }
+                const int col = hf * (D / 2) + 16 * i;  // first f16 value of the 16
+                const int sseg = col / 64;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int sch = (col % 64) / 8 + hh;
+                    *reinterpret_cast<uint4*>(scr + sseg * C::TW * 128 + lrow * 128 + ((sch ^ (lrow & 7)) << 4)) =
+                        make_uint4(hv[4 * hh], hv[4 * hh + 1], hv[4 * hh + 2], hv[4 * hh + 3]);
+                }
+            }
+            __syncwarp();
+            vbase = smem_u32(scr);
+        } else if (nvalid < 16) {
+            // value rows of the warp past the split's keys (the last tile) may hold anything, even NaN, and
+            // P = 0 does not cancel that in the MMA: zero them
             const int first = nvalid < 0 ? 0 : nvalid;
             uint8_t* vrow = stages + s * C::STAGE_BYTES + C::MAT_BYTES;
             for (int idx = lane; idx < (16 - first) * C::NSEG * 8; idx += 32) {
@@ -863,9 +993,9 @@ __global__ void __launch_bounds__(160, GqaMmaCfg<D>::MINB)
 #pragma unroll
         for (int cc = 0; cc < NT / 2; ++cc) {
             uint32_t vb[4];
-            ldsm_x4_t(vt + (cc >> 2) * C::T_TILE * 128 + v_off[cc & 3], vb);
-            mma_bf16_16816(o[2 * cc], pa, vb[0], vb[1]);
-            mma_bf16_16816(o[2 * cc + 1], pa, vb[2], vb[3]);
+            ldsm_x4_t(vbase + (cc >> 2) * V_SEG + v_off[cc & 3], vb);
+            mma_16816<F8>(o[2 * cc], pa, vb[0], vb[1]);
+            mma_16816<F8>(o[2 * cc + 1], pa, vb[2], vb[3]);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&bars[C::NSTAGE + s]));
@@ -877,27 +1007,337 @@ __global__ void __launch_bounds__(160, GqaMmaCfg<D>::MINB)
         l_run[i] += __shfl_xor_sync(0xffffffffu, l_run[i], 1);
         l_run[i] += __shfl_xor_sync(0xffffffffu, l_run[i], 2);
     }
-    // all consumer warps reach here; aborted CTAs stop without writing results
-    named_barrier(1, 128);
-    if (*(volatile int*)&s_abort || aborted) return;
-
-    // ---- merge the four warp states in shared memory (reusing the stage ring) ----
-    float* om = reinterpret_cast<float*>(stages);  // [4][RB][D]
-    float* mm = om + 4 * RB * D;                    // [4][RB]
-    float* lm = mm + 4 * RB;                        // [4][RB]
+    // all consumer warps reach here; a CTA that gave up on a wait writes no results
+    if (!consumers_any(aborted || *(volatile int*)&s_abort)) {
+        // ---- merge the four warp states in shared memory (reusing the stage ring) ----
+        float* om = reinterpret_cast<float*>(stages);  // [4][RB][D]
+        float* mm = om + 4 * RB * D;                    // [4][RB]
+        float* lm = mm + 4 * RB;                        // [4][RB]
 #pragma unroll
-    for (int j = 0; j < NT; ++j) {
-        *reinterpret_cast<float2*>(&om[(warp * RB + g) * D + 8 * j + 2 * tq]) = make_float2(o[j][0], o[j][1]);
-        *reinterpret_cast<float2*>(&om[(warp * RB + g + 8) * D + 8 * j + 2 * tq]) = make_float2(o[j][2], o[j][3]);
+        for (int j = 0; j < NT; ++j) {
+            *reinterpret_cast<float2*>(&om[(warp * RB + g) * D + 8 * j + 2 * tq]) = make_float2(o[j][0], o[j][1]);
+            *reinterpret_cast<float2*>(&om[(warp * RB + g + 8) * D + 8 * j + 2 * tq]) =
+                make_float2(o[j][2], o[j][3]);
+        }
+        if (tq == 0) {
+            mm[warp * RB + g] = m_run[0];
+            mm[warp * RB + g + 8] = m_run[1];
+            lm[warp * RB + g] = l_run[0];
+            lm[warp * RB + g + 8] = l_run[1];
+        }
+        named_barrier(1, 128);
+        gqa_merge_store<__nv_bfloat16, D, RB>(om, mm, lm, p, b, kvh, row0, rows_here, L, kbeg, split,
+                                              F8 ? p.v_scale[kvh] : 1.f);
     }
-    if (tq == 0) {
-        mm[warp * RB + g] = m_run[0];
-        mm[warp * RB + g + 8] = m_run[1];
-        lm[warp * RB + g] = l_run[0];
-        lm[warp * RB + g + 8] = l_run[1];
+}
+
+// The swapped form for blocks of at most 8 query rows (the common GQA groups of 4 or 8 heads at s_q = 1): the
+// warp's 16 tokens are the M = 16 rows of the MMAs and the query rows the N = 8 columns, so that a 16-token tile
+// costs d/16 score MMAs (S^T = K Q^T, K read by ldmatrix as the A operand, Q^T held in registers) and d/16 P*V
+// MMAs (O^T = V^T P^T, V^T read by the transposing ldmatrix as the A operand) instead of twice that with 8 of 16
+// rows empty.  The score accumulator holds P^T (tokens x rows); movmatrix transposes its two 8 x 8 halves into the
+// B operand of the P*V MMA.  Everything else (softmax, scales, the e4m3 handling with its permuted head-dim order
+// and token order, the merge) is as in the 16-row form above.
+template <int D, bool F8>
+__global__ void __launch_bounds__(160, GqaMmaCfg<D, F8>::MINB)
+    gqa_decode_mma8_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                           const GqaParams p) {
+    using C = GqaMmaCfg<D, F8>;
+    constexpr int RB = 8, KS = D / 16, MT = D / 16;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
+    uint8_t* stages = smem;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    __shared__ int s_abort;
+
+    const int split = blockIdx.x;
+    const int kvh = blockIdx.y / p.n_rb;
+    const int rb = blockIdx.y % p.n_rb;
+    const int b = blockIdx.z;
+    const int R = p.ratio * p.s_q;  // query rows of this group
+    const int row0 = rb * RB;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+    const int L = clamp_len(p.lens, b, p.Lmax, p.s_q, p.causal, p.status,
+                            threadIdx.x == 0 && split == 0 && kvh == 0 && rb == 0);
+    const int rows_here = R - row0 < RB ? R - row0 : RB;
+    int need = L;  // keys needed by the rows of this block: causal row t sees L - s_q + t + 1
+    if (p.causal) {
+        int tmax = 0;
+        for (int r = 0; r < rows_here; ++r) tmax = max(tmax, (row0 + r) % p.s_q);
+        need = L - p.s_q + tmax + 1;
     }
-    named_barrier(1, 128);
-    gqa_merge_store<__nv_bfloat16, D, RB>(om, mm, lm, p, b, kvh, row0, rows_here, L, kbeg, split, 1.f);
+    const int kbeg = split * p.split_tokens;
+    if (kbeg >= need) return;  // no row of this block has keys in this split
+    const int kend = min(need, kbeg + p.split_tokens);
+    const int n_tiles = cdiv(kend - kbeg, C::T_TILE);
+
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        for (int s = 0; s < C::NSTAGE; ++s) {
+            mbar_init(smem_u32(&bars[s]), 1);              // full: producer arrival + tx bytes
+            mbar_init(smem_u32(&bars[C::NSTAGE + s]), 4);  // empty: one arrival per consumer warp
+        }
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    if (warp == 4) {
+        if (lane == 0) gqa_produce<C>(&tmK, &tmV, p, stages, bars, &s_abort, b, kvh, L, kbeg, n_tiles);
+        return;
+    }
+
+    // -------------------------------- consumers --------------------------------
+    // Fragment coordinates: lane = 4 g + tq.  Score accumulator: tokens (MMA rows) g and g + 8 of the warp's 16,
+    // query rows (MMA columns) 2 tq and 2 tq + 1.  B operand of the score MMA: query row g.
+    const int g = lane >> 2, tq = lane & 3;
+    int last[2];  // last visible key of query rows 2 tq and 2 tq + 1 (-1: a padding row, nothing visible)
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int gr = row0 + 2 * tq + i;
+        last[i] = gr < R ? (p.causal ? L - p.s_q + gr % p.s_q : L - 1) : -1;
+    }
+    uint32_t qb[KS][2];  // B fragments of the score MMA: query row g, as given (the scale goes on the fp32 scores)
+    {
+        const __nv_bfloat16* qbase = reinterpret_cast<const __nv_bfloat16*>(p.q) +
+                                     ((size_t)(b * p.h_q + kvh * p.ratio) * p.s_q) * D;  // first row of the group
+        const bool ok = row0 + g < R;
+        const uint32_t* qrow = reinterpret_cast<const uint32_t*>(qbase + (size_t)(ok ? row0 + g : 0) * D);
+        auto qpair = [&](int u) -> uint32_t {
+            const uint32_t w = ok ? qrow[u] : 0u;
+            if constexpr (F8) {
+                float lo, hi;
+                bf16x2_to_f32(w, lo, hi);
+                return pack_f16x2_rn(lo, hi);
+            } else {
+                return w;
+            }
+        };
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            // pairs of values: bf16 layout 16 ks + 2 tq (+ 8); e4m3 permuted layout 64 G + 16 tq + 4 j (+ 2)
+            const int u0 = F8 ? 32 * (ks >> 2) + 8 * tq + 2 * (ks & 3) : 8 * ks + tq;
+            qb[ks][0] = qpair(u0);
+            qb[ks][1] = qpair(F8 ? u0 + 1 : u0 + 4);
+        }
+    }
+    float o[MT][4];  // O^T: head-dim values 16 mt + g (+ 8), query rows 2 tq, 2 tq + 1
+#pragma unroll
+    for (int j = 0; j < MT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+    const float s_mul = F8 ? p.scale_log2 * p.k_scale[kvh] : p.scale_log2;
+    int mask_from = kend;  // keys below mask_from are visible to every row of the block
+    for (int r = 0; r < rows_here; ++r)
+        mask_from = min(mask_from, p.causal ? L - p.s_q + (row0 + r) % p.s_q + 1 : L);
+    // token (of the warp's 16) of MMA row g + 8 h
+    const int tok_g[2] = {F8 ? f8_tok(g) : g, 8 + (F8 ? f8_tok(g) : g)};
+
+    // ldmatrix row addresses (byte offsets, 128-byte swizzle).  Both operands are A fragments read from token rows:
+    // matrix l / 8 = (token half l / 16, 8-value chunk parity (l / 8) % 2).  bf16 keys: non-transposed, one k-step;
+    // values (transposed; the stage for bf16, the warp's scratch tile for e4m3): one 16-value m-tile of O^T.
+    const int r8 = lane & 7;
+    const uint32_t k_row = (uint32_t)(16 * warp + 8 * (lane >> 4) + r8) * 128;
+    const uint32_t v_row = (uint32_t)((F8 ? 0 : 16 * warp) + 8 * (lane >> 4) + r8) * 128;
+    constexpr int V_SEG = F8 ? C::TW * 128 : C::T_TILE * 128;  // bytes per 64-value segment of a value tile
+    uint32_t k_off[4], v_off[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        k_off[c] = k_row + ((uint32_t)((2 * c + ((lane >> 3) & 1)) ^ r8) << 4);
+        v_off[c] = v_row + ((uint32_t)((2 * c + ((lane >> 3) & 1)) ^ r8) << 4);
+    }
+    uint8_t* scr = smem + C::RING + warp * C::SCR_W;
+
+    bool aborted = false;
+    for (int it = 0; it < n_tiles; ++it) {
+        const int s = it % C::NSTAGE;
+        if (!mbar_wait(smem_u32(&bars[s]), (it / C::NSTAGE) & 1, p.status)) {
+            aborted = true;
+            s_abort = 1;
+            break;
+        }
+        const uint32_t kt = smem_u32(stages + s * C::STAGE_BYTES);
+        const uint32_t vt = kt + C::MAT_BYTES;
+        const int tbase = kbeg + it * C::T_TILE;
+
+        // ---- S^T = K Q^T for the warp's 16 tokens (two accumulators: even / odd k-steps) ----
+        float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        if constexpr (F8) {
+            const uint8_t* kst = stages + s * C::STAGE_BYTES;
+#pragma unroll
+            for (int G = 0; G < D / 64; ++G) {
+                const int seg = G >> 1, chunk = 4 * (G & 1) + tq;
+                uint4 w[2];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int row = 16 * warp + tok_g[h];
+                    w[h] = *reinterpret_cast<const uint4*>(kst + seg * C::T_TILE * 128 + row * 128 +
+                                                           ((chunk ^ (row & 7)) << 4));
+                }
+                const uint32_t w0[4] = {w[0].x, w[0].y, w[0].z, w[0].w}, w1[4] = {w[1].x, w[1].y, w[1].z, w[1].w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t a[4] = {e4m3x2_lo_to_f16x2(w0[j]), e4m3x2_lo_to_f16x2(w1[j]),
+                                           e4m3x2_hi_to_f16x2(w0[j]), e4m3x2_hi_to_f16x2(w1[j])};
+                    mma_16816<true>(sc[j & 1], a, qb[4 * G + j][0], qb[4 * G + j][1]);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+                uint32_t a[4];
+                ldsm_x4(kt + (ks >> 2) * C::T_TILE * 128 + k_off[ks & 3], a);
+                // ldmatrix order (tokens 0-7 lo, tokens 0-7 hi, tokens 8-15 lo, tokens 8-15 hi) -> a0 a2 a1 a3
+                const uint32_t af[4] = {a[0], a[2], a[1], a[3]};
+                mma_16816<false>(sc[ks & 1], af, qb[ks][0], qb[ks][1]);
+            }
+        }
+        // x[e]: token tbase + 16 warp + tok_g[e / 2], query row 2 tq + e % 2, in the log2 domain
+        float x[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[e] = (sc[0][e] + sc[1][e]) * s_mul;
+        if (tbase + C::T_TILE > mask_from) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int tok = tbase + 16 * warp + tok_g[e >> 1];
+                x[e] = (tok < kend && tok <= last[e & 1]) ? x[e] : -INFINITY;
+            }
+        }
+        // ---- online softmax of the two rows (over the 8 lanes that share tq), lazily rescaled ----
+        float mx[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            mx[i] = fmaxf(x[i], x[2 + i]);
+            mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 4));
+            mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 8));
+            mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 16));
+        }
+        if (__any_sync(0xffffffffu, mx[0] > m_run[0] + 8.0f || mx[1] > m_run[1] + 8.0f)) {
+            float alpha[2];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const float m_new = fmaxf(m_run[i], mx[i]);
+                alpha[i] = 1.f;
+                if (m_run[i] == -INFINITY) {
+                    m_run[i] = m_new;  // O and l of the row are still zero
+                } else if (m_new > m_run[i] + 8.0f) {
+                    alpha[i] = fast_exp2(m_run[i] - m_new);
+                    m_run[i] = m_new;
+                }
+                l_run[i] *= alpha[i];
+            }
+#pragma unroll
+            for (int j = 0; j < MT; ++j) {
+                o[j][0] *= alpha[0];
+                o[j][1] *= alpha[1];
+                o[j][2] *= alpha[0];
+                o[j][3] *= alpha[1];
+            }
+        }
+        uint32_t pb[2];  // B fragment of the P*V MMA: query row g, tokens 2 tq, 2 tq + 1 (+ 8)
+        {
+            const float ms0 = m_run[0] == -INFINITY ? 0.f : m_run[0];  // no visible key yet: p = 2^-inf = 0
+            const float ms1 = m_run[1] == -INFINITY ? 0.f : m_run[1];
+            const float p0 = fast_exp2(x[0] - ms0), p1 = fast_exp2(x[1] - ms1);
+            const float p2 = fast_exp2(x[2] - ms0), p3 = fast_exp2(x[3] - ms1);
+            l_run[0] += p0 + p2;  // this lane's share; summed over the row's lanes at the end
+            l_run[1] += p1 + p3;
+            // P^T halves (tokens g / g + 8 x rows 2 tq, 2 tq + 1) transposed into P halves (row g x tokens)
+            const uint32_t t0 = F8 ? pack_f16x2_rn(p0, p1) : pack_bf16x2(p0, p1);
+            const uint32_t t1 = F8 ? pack_f16x2_rn(p2, p3) : pack_bf16x2(p2, p3);
+            asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(pb[0]) : "r"(t0));
+            asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(pb[1]) : "r"(t1));
+        }
+        uint32_t vbase = vt;
+        const int nvalid = kend - (tbase + 16 * warp);  // value rows of the warp that are keys of the split
+        if constexpr (F8) {
+            // widen the warp's 16 value rows into its f16 scratch tile, rows in MMA-row order; rows past the
+            // split's keys may hold anything (even NaN), which P = 0 would not cancel in the MMA: they become 0
+            const int t = lane >> 1, hf = lane & 1;
+            const int srow = 16 * warp + t;                  // stage row
+            const int lrow = 8 * (t >> 3) + f8_col(t & 7);   // scratch row
+            const bool live = t < nvalid, tail = nvalid < 16;  // (tail: warp-uniform, the last tile only)
+            const uint8_t* vsrc = stages + s * C::STAGE_BYTES + C::MAT_BYTES;
+#pragma unroll
+            for (int i = 0; i < D / 32; ++i) {  // 16 e4m3 values: scratch chunks 2 i, 2 i + 1 of segment hf
+                const int byte = hf * (D / 2) + 16 * i;
+                const int ch = (byte % 128) / 16;
+                uint4 w = *reinterpret_cast<const uint4*>(vsrc + (byte / 128) * C::T_TILE * 128 + srow * 128 +
+                                                          ((ch ^ (srow & 7)) << 4));
+                if (tail && !live) w = make_uint4(0u, 0u, 0u, 0u);
+                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+                uint32_t hv[8];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    hv[2 * q] = e4m3x2_lo_to_f16x2(ws[q]);
+                    hv[2 * q + 1] = e4m3x2_hi_to_f16x2(ws[q]);
+                }
+                const int col = hf * (D / 2) + 16 * i;  // first f16 value of the 16
+                const int sseg = col / 64;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int sch = (col % 64) / 8 + hh;
+                    *reinterpret_cast<uint4*>(scr + sseg * C::TW * 128 + lrow * 128 + ((sch ^ (lrow & 7)) << 4)) =
+                        make_uint4(hv[4 * hh], hv[4 * hh + 1], hv[4 * hh + 2], hv[4 * hh + 3]);
+                }
+            }
+            __syncwarp();
+            vbase = smem_u32(scr);
+        } else if (nvalid < 16) {
+            // value rows of the warp past the split's keys (the last tile) may hold anything, even NaN, and
+            // P = 0 does not cancel that in the MMA: zero them
+            const int first = nvalid < 0 ? 0 : nvalid;
+            uint8_t* vrow = stages + s * C::STAGE_BYTES + C::MAT_BYTES;
+            for (int idx = lane; idx < (16 - first) * C::NSEG * 8; idx += 32) {
+                const int row = 16 * warp + first + idx / (C::NSEG * 8), rem = idx % (C::NSEG * 8);
+                *reinterpret_cast<uint4*>(vrow + (rem / 8) * C::T_TILE * 128 + row * 128 + (rem % 8) * 16) =
+                    make_uint4(0u, 0u, 0u, 0u);
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // before the ring's next copy
+            __syncwarp();
+        }
+        // ---- O^T += V^T P^T: one MMA per 16 head-dim values ----
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            uint32_t a[4];
+            ldsm_x4_t(vbase + (mt >> 2) * V_SEG + v_off[mt & 3], a);
+            // ldmatrix order (tokens 0-7 x d lo, tokens 0-7 x d hi, tokens 8-15 x d lo, tokens 8-15 x d hi),
+            // transposed: (d lo, k lo) (d hi, k lo) (d lo, k hi) (d hi, k hi) = a0 a1 a2 a3
+            mma_16816<F8>(o[mt], a, pb[0], pb[1]);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars[C::NSTAGE + s]));
+    }
+
+    // the row sums: this lane's share summed over the eight lanes of the row
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        l_run[i] += __shfl_xor_sync(0xffffffffu, l_run[i], 4);
+        l_run[i] += __shfl_xor_sync(0xffffffffu, l_run[i], 8);
+        l_run[i] += __shfl_xor_sync(0xffffffffu, l_run[i], 16);
+    }
+    // all consumer warps reach here; a CTA that gave up on a wait writes no results
+    if (!consumers_any(aborted || *(volatile int*)&s_abort)) {
+        // ---- merge the four warp states in shared memory (reusing the stage ring) ----
+        float* om = reinterpret_cast<float*>(stages);  // [4][RB][D]
+        float* mm = om + 4 * RB * D;                    // [4][RB]
+        float* lm = mm + 4 * RB;                        // [4][RB]
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            om[(warp * RB + 2 * tq) * D + 16 * mt + g] = o[mt][0];
+            om[(warp * RB + 2 * tq + 1) * D + 16 * mt + g] = o[mt][1];
+            om[(warp * RB + 2 * tq) * D + 16 * mt + g + 8] = o[mt][2];
+            om[(warp * RB + 2 * tq + 1) * D + 16 * mt + g + 8] = o[mt][3];
+        }
+        if (g == 0) {
+            mm[warp * RB + 2 * tq] = m_run[0];
+            mm[warp * RB + 2 * tq + 1] = m_run[1];
+            lm[warp * RB + 2 * tq] = l_run[0];
+            lm[warp * RB + 2 * tq + 1] = l_run[1];
+        }
+        named_barrier(1, 128);
+        gqa_merge_store<__nv_bfloat16, D, RB>(om, mm, lm, p, b, kvh, row0, rows_here, L, kbeg, split,
+                                              F8 ? p.v_scale[kvh] : 1.f);
+    }
 }
 
 // Merge of split partials: with w_i = 2^(lse_i - max lse),
@@ -976,11 +1416,11 @@ static cudaError_t launch_one(const CUtensorMap& tk, const CUtensorMap& tv, cons
     return e;
 }
 
-template <int D>
+template <int D, bool F8>
 static cudaError_t launch_mma(const CUtensorMap& tk, const CUtensorMap& tv, const GqaParams& p, int nsplit,
                               cudaStream_t st) {
-    using C = GqaMmaCfg<D>;
-    auto kern = gqa_decode_mma_kernel<D>;
+    using C = GqaMmaCfg<D, F8>;
+    auto kern = p.n_rb == 1 && p.ratio * p.s_q <= 8 ? gqa_decode_mma8_kernel<D, F8> : gqa_decode_mma_kernel<D, F8>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     dim3 grid(nsplit, p.h_kv * p.n_rb, p.B);
@@ -1016,8 +1456,8 @@ int gqa_tile_tokens(int dtype_bytes, int d, int rb, int* ctas_per_sm) {
         return GqaCfg<T, DD, R>::T_TILE;                         \
     }
     if (dtype_bytes == 2 && (d == 64 || d == 128) && rb == 16) {  // the tensor-core instance
-        if (ctas_per_sm) *ctas_per_sm = d == 64 ? GqaMmaCfg<64>::MINB : GqaMmaCfg<128>::MINB;
-        return d == 64 ? GqaMmaCfg<64>::T_TILE : GqaMmaCfg<128>::T_TILE;
+        if (ctas_per_sm) *ctas_per_sm = d == 64 ? GqaMmaCfg<64, false>::MINB : GqaMmaCfg<128, false>::MINB;
+        return d == 64 ? GqaMmaCfg<64, false>::T_TILE : GqaMmaCfg<128, false>::T_TILE;
     }
     LKA_TILE_CASE(__nv_bfloat16, 256, 1) LKA_TILE_CASE(__nv_bfloat16, 256, 2) LKA_TILE_CASE(__nv_bfloat16, 256, 4)
     LKA_TILE_CASE(__nv_bfloat16, 256, 8)
@@ -1033,8 +1473,8 @@ cudaError_t gqa_decode_launch(const CUtensorMap& tk, const CUtensorMap& tv, cons
                               int d, int rb, int nsplit, cudaStream_t st) {
 #define LKA_LAUNCH_CASE(T, DD, R) \
     if (dtype_bytes == (int)sizeof(T) && d == DD && rb == R) return launch_one<T, DD, R>(tk, tv, p, nsplit, st);
-    if (dtype_bytes == 2 && d == 64 && rb == 16) return launch_mma<64>(tk, tv, p, nsplit, st);
-    if (dtype_bytes == 2 && d == 128 && rb == 16) return launch_mma<128>(tk, tv, p, nsplit, st);
+    if (dtype_bytes == 2 && d == 64 && rb == 16) return launch_mma<64, false>(tk, tv, p, nsplit, st);
+    if (dtype_bytes == 2 && d == 128 && rb == 16) return launch_mma<128, false>(tk, tv, p, nsplit, st);
     LKA_LAUNCH_CASE(__nv_bfloat16, 256, 1) LKA_LAUNCH_CASE(__nv_bfloat16, 256, 2)
     LKA_LAUNCH_CASE(__nv_bfloat16, 256, 4) LKA_LAUNCH_CASE(__nv_bfloat16, 256, 8)
     LKA_LAUNCH_CASE(float, 64, 1) LKA_LAUNCH_CASE(float, 64, 2) LKA_LAUNCH_CASE(float, 64, 4)
@@ -1046,12 +1486,15 @@ cudaError_t gqa_decode_launch(const CUtensorMap& tk, const CUtensorMap& tv, cons
 }
 
 int gqa_fp8_tile_tokens(int d, int rb, int* ctas_per_sm) {
+    if (d == 128 && rb == 16) {  // the tensor-core instance
+        if (ctas_per_sm) *ctas_per_sm = GqaMmaCfg<128, true>::MINB;
+        return GqaMmaCfg<128, true>::T_TILE;
+    }
 #define LKA_TILE_CASE(DD, R)                                       \
     if (d == DD && rb == R) {                                      \
         if (ctas_per_sm) *ctas_per_sm = GqaCfg<e4m3, DD, R>::MINB; \
         return GqaCfg<e4m3, DD, R>::T_TILE;                        \
     }
-    LKA_TILE_CASE(128, 1) LKA_TILE_CASE(128, 2) LKA_TILE_CASE(128, 4)
     LKA_TILE_CASE(256, 1) LKA_TILE_CASE(256, 2) LKA_TILE_CASE(256, 4)
 #undef LKA_TILE_CASE
     return 0;
@@ -1059,9 +1502,9 @@ int gqa_fp8_tile_tokens(int d, int rb, int* ctas_per_sm) {
 
 cudaError_t gqa_fp8_decode_launch(const CUtensorMap& tk, const CUtensorMap& tv, const GqaParams& p, int d, int rb,
                                   int nsplit, cudaStream_t st) {
+    if (d == 128 && rb == 16) return launch_mma<128, true>(tk, tv, p, nsplit, st);
 #define LKA_LAUNCH_CASE(DD, R) \
     if (d == DD && rb == R) return launch_one<__nv_bfloat16, DD, R, e4m3>(tk, tv, p, nsplit, st);
-    LKA_LAUNCH_CASE(128, 1) LKA_LAUNCH_CASE(128, 2) LKA_LAUNCH_CASE(128, 4)
     LKA_LAUNCH_CASE(256, 1) LKA_LAUNCH_CASE(256, 2) LKA_LAUNCH_CASE(256, 4)
 #undef LKA_LAUNCH_CASE
     return cudaErrorInvalidValue;

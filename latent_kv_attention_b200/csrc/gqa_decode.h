@@ -31,8 +31,8 @@ struct GqaParams {
     const float* v_scale;
 };
 
-// The e4m3-cache instances (bf16 q/out, d in {128, 256}, rb <= 4: a 16-byte chunk holds 16 values, so more rows
-// per CTA would not fit the query slice in registers).
+// The e4m3-cache instances (bf16 q/out): d = 128 on the tensor-core instance (rb = 16), d = 256 on the CUDA-core
+// one (rb <= 4: a 16-byte chunk holds 16 values, so more rows per CTA would not fit the query slice in registers).
 int gqa_fp8_tile_tokens(int d, int rb, int* ctas_per_sm);
 cudaError_t gqa_fp8_decode_launch(const CUtensorMap& tk, const CUtensorMap& tv, const GqaParams& p, int d, int rb,
                                   int nsplit, cudaStream_t st);

@@ -59,6 +59,10 @@ CASES = [
     (1, 32, 2, 128, 1, 500, 1000, 1024, True),  # 16 heads per group (two row blocks of 8... or one of 16)
     (2, 4, 4, 128, 37, 37, 90, 96, True),       # prefill-like s_q
     (1, 2, 1, 128, 1, 63, 63, 64, True),        # L < tile
+    (2, 24, 2, 128, 1, 70, 500, 512, True),     # 12 rows: the 16-row tensor-core form with padding rows
+    (1, 64, 2, 128, 1, 200, 400, 400, True),    # 32 rows: two row blocks of 16
+    (2, 8, 2, 128, 3, 3, 300, 320, True),       # 12 rows of 3 query tokens (per-row causal limits)
+    (2, 8, 4, 64, 4, 4, 150, 160, True),        # 8 rows of 4 query tokens: the 8-row form, d = 64
 ]
 
 
@@ -70,6 +74,25 @@ def test_gqa_random(case, dtype):
         pytest.skip("fp32 supports d_h in {64, 128}")
     inp = synthetic.gqa_inputs(100 + len(str(case)), B, h_q, h_kv, d, s_q, lo, hi, Lmax=Lmax, dtype=dtype)
     run_case(inp, causal, dtype)
+
+
+def test_fused_split_merge_is_repeatable():
+    """Repeated calls with different key-split plans on one workspace (rows of one block needing different
+    split counts, s_q = 4 causal) give the oracle's result every time, and the same bits for the same plan:
+    nothing a call leaves in the workspace changes the next one."""
+    inp = synthetic.gqa_inputs(8, 3, 16, 4, 128, 4, 300, 1000, Lmax=1024, dtype=torch.bfloat16)
+    q, k, v, lens = (inp[n].to(DEV) for n in ("q", "k", "v", "cache_lens"))
+    ref, _ = oracle.gqa(inp["q"], inp["k"], inp["v"], inp["cache_lens"], True, inp["scale"])
+    outs = []
+    for split in (128, 64, 128, 0, 128):
+        prev = lka.set_split_tokens(split)
+        try:
+            out = lka.gqa_attn(q, k, v, lens, causal=True, scale=inp["scale"])
+        finally:
+            lka.set_split_tokens(prev)
+        assert_close(out, ref, torch.bfloat16, f"splits of {split}")
+        outs.append(out)
+    assert torch.equal(outs[0], outs[2]) and torch.equal(outs[0], outs[4])
 
 
 @pytest.mark.parametrize("split", [64, 128, 448, 4096])
