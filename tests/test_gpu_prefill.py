@@ -59,6 +59,15 @@ def test_prefill_matches_oracle(case):
     run_case(inp, causal)
 
 
+@pytest.mark.parametrize("scale", [-0.05, 0.0])
+def test_prefill_any_scale(scale):
+    """The prefill kernel applies the scale inside the exponent (raw scores masked, their maximum scaled): a negative
+    scale flips the scores, a zero scale gives the mean of the visible values, both as in the definition."""
+    inp = synthetic.gqa_inputs(95, 1, 8, 2, 128, 130, 130, 260, Lmax=260, dtype=torch.bfloat16)
+    inp["scale"] = scale
+    run_case(inp, True)
+
+
 @pytest.mark.parametrize("split", [128, 256])
 def test_prefill_key_splits(split):
     """Key splits (the merge of normalised partials by their lse) give the same result as one pass."""
