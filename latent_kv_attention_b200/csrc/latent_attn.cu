@@ -88,6 +88,11 @@ constexpr int NCW = 2;          // converter warps (FP8 cache only)
 constexpr int CW = NT / 2;      // score columns per softmax warp
 constexpr int NTHREADS = 32 * (NSW + 2 + NXW);
 constexpr int NTHREADS_F8 = NTHREADS + 32 * NCW;
+// bf16 cache: one more warp, which issues the P*V MMAs, so that the score chain (waiting for key tiles and a
+// free score buffer) and the P*V chain (waiting for P) do not hold each other up in one issuing thread.  (The
+// FP8 instance, with its converter warps, keeps one issuer: 17 warps would not fit 128 registers a thread.)
+constexpr int PV_WARP = NSW + 2 + NXW;
+constexpr int NTHREADS_BF = NTHREADS + 32;
 constexpr int XROW = CW * 2;    // bytes of one row of one half of an exchanged partial (fp16)
 constexpr int XBUF = 2 * 128 * XROW;  // [half][head row][CW] fp16; each warp's block is contiguous
 constexpr int XSPACE = 2 * XBUF;      // room reserved for each of the exchange buffer and the outbox
@@ -303,7 +308,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
         constexpr uint32_t idesc_qk = F8 ? idesc_f16_f32(128, NT, false, false) : idesc_bf16_f32(128, NT, false, false);
         constexpr uint32_t idesc_pv = F8 ? idesc_f16_f32(128, 256, false, true) : idesc_bf16_f32(128, 256, false, true);
         bool ok = mbar_wait(smem_u32(q_full), 0, p.status);
-        for (int j = 0; ok && j < n_tiles + 2; ++j) {
+        for (int j = 0; ok && j < (F8 ? n_tiles + 2 : n_tiles); ++j) {
             if (j < n_tiles) {
                 const int s = j % NST;
                 if (!mbar_wait(smem_u32(F8 ? &conv_full[s] : &kv_full[s]), (j / NST) & 1, p.status)) break;
@@ -336,7 +341,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
                 }
                 __syncwarp();
             }
-            if (j >= 2) {
+            if (F8 && j >= 2) {
                 const int i = j - 2;
                 if (!mbar_wait(smem_u32(p_ready), i & 1, p.status)) break;
                 tc_fence_after();
@@ -351,6 +356,26 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
                 }
                 __syncwarp();
             }
+        }
+    } else if (!F8 && n_tiles > 0 && warp == PV_WARP) {
+        // ----------------------------- P*V MMA issuer (bf16) -----------------------------
+        // O += P(i) V(i) once P(i) is in tensor memory; the stage was zeroed past the last key before the score
+        // MMA of the tile, and its commit to kv_empty releases it (this chain reads it last).  The commits track
+        // this thread's MMAs only.
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
+        for (int i = 0; i < n_tiles; ++i) {
+            if (!mbar_wait(smem_u32(p_ready), i & 1, p.status)) break;
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t va = smem_u32(smem + OFF_KV + (i % NST) * STAGE);
+#pragma unroll
+                for (int kk = 0; kk < NT / 16; ++kk)
+                    umma_ts(tmem + T_O, tmem + T_P + kk * 8, smem_desc_sw128(va + kk * 2048, BOX, 1024), idesc_pv,
+                            (i | kk) != 0);
+                umma_commit(smem_u32(&kv_empty[i % NST]));
+                umma_commit(smem_u32(o_ready));
+            }
+            __syncwarp();
         }
     } else if (F8 && n_tiles > 0 && warp >= NSW + 2 + NXW) {
         // ------------------------------ converter warps ------------------------------
@@ -767,7 +792,7 @@ cudaError_t latent_attn_launch(const CUtensorMap& tm_lat, const LatentParams& p,
         if (f8)
             latent_attn_kernel<true><<<grid, lat::NTHREADS_F8, lat::SMEM, st>>>(tm_lat, tm_qt, tm_qr, p);
         else
-            latent_attn_kernel<false><<<grid, lat::NTHREADS, lat::SMEM, st>>>(tm_lat, tm_qt, tm_qr, p);
+            latent_attn_kernel<false><<<grid, lat::NTHREADS_BF, lat::SMEM, st>>>(tm_lat, tm_qt, tm_qr, p);
         timer.stop();
     }
     e = cudaPeekAtLastError();
