@@ -209,7 +209,8 @@ class GqaDecode(Workload):
     caches) + log-sum-exp merge."""
 
     kernel = "gqa_decode_mma_kernel"
-    src = ("latent_kv_attention_b200/csrc/gqa_decode.cu", "latent_kv_attention_b200/csrc/common.cuh")
+    src = ("latent_kv_attention_b200/csrc/gqa_decode.cu", "latent_kv_attention_b200/csrc/common.cuh",
+           "latent_kv_attention_b200/csrc/tc.cuh")
 
     def setup_costs(self):
         w = self.w
@@ -647,6 +648,7 @@ WORKLOAD_CLASSES = {
     "gta_prefill_4k": GtaPrefill,
     "gta_chunked_prefill_4k_paged": GtaChunkedPrefillPaged,
     "gqa_prefill_llama8b_4k": GqaPrefill,
+    "gqa_prefill_llama8b_2k_b1": GqaPrefill,
     # smaller cases for full ncu captures
     "latent_decode_4k_sq1_b32": LatentAbsorbed,
     "latent_expanded_4k_sq2_b16": LatentExpanded,

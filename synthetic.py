@@ -271,6 +271,9 @@ WORKLOADS = {
     # causal prefill of the same layer: 4096 query tokens per sequence over their own 4096-token cache
     "gqa_prefill_llama8b_4k": dict(kind="gqa", seed=6, B=2, h_q=32, h_kv=8, d=128, s_q=4096, L_lo=4096, L_hi=4096,
                                    causal=True),
+    # a small case of the same layer for profiler captures (the full prefill holds ~300 MB)
+    "gqa_prefill_llama8b_2k_b1": dict(kind="gqa", seed=6, B=1, h_q=32, h_kv=8, d=128, s_q=2048, L_lo=2048, L_hi=2048,
+                                      causal=True),
     "gta_prefill_4k": dict(kind="gta", seed=3, B=8, G=3, H=12, d_qk=64, d_v=64, s_q=4096, L_lo=4096,
                            L_hi=4096, causal=True),
     "latent_decode_4k_sq1": dict(kind="latent", seed=4, B=64, h_q=128, g=8, d_h=128, r_kv=512, d_r=64, s_q=1,
