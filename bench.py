@@ -54,7 +54,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 import synthetic  # noqa: E402
-from latent_kv_attention_b200 import costs  # noqa: E402
+from latent_kv_attention_b200 import costs, sharding  # noqa: E402
 
 METRIC = "decode-attention HBM GB/s (% of peak), TFLOPS (% of roofline), tokens/s"
 FALLBACK_HBM_GBS = 6650.0
@@ -249,6 +249,34 @@ class GqaDecode(Workload):
         fn = lambda: oracle.gqa(sub["q"], sub["k"], sub["v"], lens, w["causal"], self.inp["scale"])  # noqa: E731
         nbytes = costs.gqa_bytes(lens.tolist(), w["h_q"], w["h_kv"], w["d"], w["s_q"])
         return fn, nbytes, oracle.threads_used(0, n * w["h_q"]), f"first {n} of {w['B']} sequences"
+
+
+class GqaDecodeSharded(GqaDecode):
+    """gqa_attn on this rank's slice of the KV heads and their query heads (`--shard heads`): head-axis tensor
+    parallelism with no exchange inside the attention (latent_kv_attention_b200.sharding).  Every rank draws the
+    same seeded layer and keeps its slice; the job's time is the slowest rank's, its bytes the whole layer's."""
+
+    def __init__(self, name, device, rank, world, reference=False):
+        self.rank, self.world = rank, world
+        super().__init__(name, device, reference)
+
+    def setup_costs(self):
+        self.full_w = self.w
+        w = dict(self.w)
+        (q0, q1), (k0, k1) = sharding.gqa_head_slice(w["h_q"], w["h_kv"], self.rank, self.world)
+        i = self.inp
+        i["q"] = i["q"][:, q0:q1].contiguous()
+        i["k"] = i["k"][:, k0:k1].contiguous()
+        i["v"] = i["v"][:, k0:k1].contiguous()
+        w["h_q"], w["h_kv"] = q1 - q0, k1 - k0
+        self.w = w
+        super().setup_costs()
+
+    def config(self):
+        c = super().config()
+        c["h_q"], c["h_kv"] = self.full_w["h_q"], self.full_w["h_kv"]
+        c["parallelism"] = f"heads{self.world} (KV heads split over the ranks, no collective in the call)"
+        return c
 
 
 class GqaDecodePaged(GqaDecode):
@@ -767,11 +795,17 @@ def summary(wl, m, world):
 
 def run_lka(args, rank, world, device):
     pk = peaks()
-    wl = WORKLOAD_CLASSES[args.workload](args.workload, device)
+    sharded = args.shard == "heads"
+    if sharded:
+        if WORKLOAD_CLASSES[args.workload] is not GqaDecode:
+            raise SystemExit("--shard heads applies to the contiguous GQA decode workloads")
+        wl = GqaDecodeSharded(args.workload, device, rank, world)
+    else:
+        wl = WORKLOAD_CLASSES[args.workload](args.workload, device)
     clocks = ClockSampler(device.index if device.index is not None else 0)
     m = measure(wl, args.steps, args.warmup, pk, device, world, clocks=clocks)
     extras = {}
-    if not args.no_extras:
+    if not args.no_extras and not sharded:
         for name in EXTRAS:
             if name == args.workload:
                 continue
@@ -786,7 +820,8 @@ def run_lka(args, rank, world, device):
     gbs = wl.bytes * world / t / 1e9
     line = {
         "metric": METRIC, "value": round(gbs, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(m["step_ms"], 4), "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": round(m["step_ms"], 4), "higher_is_better": True,
+        "scaling": "strong" if sharded else "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) inputs, see synthetic.py)",
         "config": wl.config(),
         "tokens_per_s": round(wl.tokens * world / t, 1),
@@ -881,6 +916,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="measure only --workload, not the other paths")
+    ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
+                    help="N > 1: independent replicas (default, weak scaling) or the layer's KV heads split over the "
+                         "ranks (strong scaling)")
     ap.add_argument("--sweep", action="store_true",
                     help="measure the long-context sweep (GQA and latent layouts, cache length 1K-64K) instead")
     args = ap.parse_args()
