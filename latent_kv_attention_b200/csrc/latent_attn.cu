@@ -31,18 +31,24 @@
 //
 // Each tcgen05.mma with M = 128 and K = 16 takes about the same time whatever
 // its N (up to 256), so the tiles are as wide as memory allows: 64 tokens.  The
-// query slice lives in tensor memory (the A operand of the score MMA), which
-// leaves shared memory to a 4-stage TMA ring, one exchange buffer and an
-// outbox: a partial is written to the outbox and sent with one bulk copy per
-// block (the copy engine moves it; the warp does not wait for the transfer).
+// query slice is the A operand of the score MMA: ten of its eighteen k-steps
+// live in tensor memory (TS-MMAs), the other eight (query values 64-191 of the
+// rank's slice) in two swizzled shared-memory boxes (SS-MMAs), which leaves
+// tensor memory room for two score buffers, so that the score MMA of tile j + 2
+// need not wait until tile j + 1 has left the exchange.  Shared memory holds a
+// 4-stage TMA ring, the two query boxes, one exchange buffer and an outbox: a
+// partial is written to the outbox and sent with one bulk copy per block (the
+// copy engine moves it; the warp does not wait for the transfer).
 // Sender warps load each partial from tensor memory as soon as it is computed
 // and send it; the softmax warps load their own copy of tile i+1 before they
 // work on tile i, and the score MMA runs two tiles ahead of P*V, so the
 // exchange overlaps the softmax of the previous tile.
 //
 // Per CTA: warp 8 streams 64-token tiles of the latent through the ring; warp 9
-// issues the MMAs (S = Q K^T into the TMEM score tile, O += P V with P read
-// from TMEM); warps 10-13 (one per TMEM lane quarter) send the score partials;
+// issues the score MMAs (S = Q K^T into score buffer j % 2) and, with a bf16
+// cache, warp 14 the P*V MMAs (O += P V with P read from TMEM; with an FP8
+// cache warp 9 issues both); warps 10-13 (one per TMEM lane quarter) send the
+// score partials;
 // warps 0-7 write the query slice to TMEM once, then per tile add the peer's
 // partial to their own, mask and run the online softmax, two warps per group
 // of 32 head rows (warps w and w + 4 take the two 32-token halves of the tile
@@ -167,7 +173,7 @@ __device__ __forceinline__ void remote_arrive(uint32_t rbar) {
 // peer's "buffer free" arrival (release at cluster scope) is only ever followed by new remote
 // copies, never by reads of data the peer produced.
 
-// 14 warps (16 with an FP8 cache): an SM sub-partition holds up to 4 of them, so at most
+// 15 warps (16 with an FP8 cache): an SM sub-partition holds up to 4 of them, so at most
 // 16384 / (4 * 32) = 128 registers each
 template <bool F8>
 __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
