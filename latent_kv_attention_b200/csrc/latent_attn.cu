@@ -31,21 +31,17 @@
 //
 // Each tcgen05.mma with M = 128 and K = 16 takes about the same time whatever
 // its N (up to 256), so the tiles are as wide as memory allows: 64 tokens.  The
-// query slice is the A operand of the score MMA: ten of its eighteen k-steps
-// live in tensor memory (TS-MMAs), the other eight (query values 64-191 of the
-// rank's slice) in two swizzled shared-memory boxes (SS-MMAs), which leaves
-// tensor memory room for two score buffers, so that the score MMA of tile j + 2
-// need not wait until tile j + 1 has left the exchange.  Shared memory holds a
-// 4-stage TMA ring, the two query boxes, one exchange buffer and an outbox: a
-// partial is written to the outbox and sent with one bulk copy per block (the
-// copy engine moves it; the warp does not wait for the transfer).
+// query slice lives in tensor memory (the A operand of the score MMA), which
+// leaves shared memory to a 4-stage TMA ring, one exchange buffer and an
+// outbox: a partial is written to the outbox and sent with one bulk copy per
+// block (the copy engine moves it; the warp does not wait for the transfer).
 // Sender warps load each partial from tensor memory as soon as it is computed
 // and send it; the softmax warps load their own copy of tile i+1 before they
 // work on tile i, and the score MMA runs two tiles ahead of P*V, so the
 // exchange overlaps the softmax of the previous tile.
 //
 // Per CTA: warp 8 streams 64-token tiles of the latent through the ring; warp 9
-// issues the score MMAs (S = Q K^T into score buffer j % 2) and, with a bf16
+// issues the score MMAs (S = Q K^T into the TMEM score tile) and, with a bf16
 // cache, warp 14 the P*V MMAs (O += P V with P read from TMEM; with an FP8
 // cache warp 9 issues both); warps 10-13 (one per TMEM lane quarter) send the
 // score partials;
@@ -101,36 +97,26 @@ constexpr int PV_WARP = NSW + 2 + NXW;
 constexpr int NTHREADS_BF = NTHREADS + 32;
 constexpr int XROW = CW * 2;    // bytes of one row of one half of an exchanged partial (fp16)
 constexpr int XBUF = 2 * 128 * XROW;  // [half][head row][CW] fp16; each warp's block is contiguous
+constexpr int XSPACE = 2 * XBUF;      // room reserved for each of the exchange buffer and the outbox
 constexpr int OFF_KV = 0;
 constexpr int OFF_X = OFF_KV + NST * STAGE;
-constexpr int OFF_OUT = OFF_X + XBUF;   // this CTA's partial on its way to the peer
-constexpr int QBOX = 128 * 128;         // 128 query rows x 64 values, 128-byte swizzle
-// Query values 64 .. 191 of this rank's slice (k-steps 4 .. 11 of the score MMA) stay in shared memory for the
-// whole work item, two boxes read by SS-MMAs; the rest live in tensor memory.  (Tensor memory then has room
-// for two score buffers: the score MMA of tile j + 2 need not wait until tile j + 1 has left the exchange.)
-constexpr int OFF_QP = OFF_OUT + XBUF;
-constexpr int OFF_BAR = OFF_QP + 2 * QBOX;
-// The query slice is five 128-row x 64-value boxes: boxes 1 and 2 land in their shared-memory home (OFF_QP);
-// boxes 0, 3 and 4 are staged through shared memory that is idle at the start (the last ring stage and the
-// exchange buffer), in slots 0, 1 and 2, on their way to tensor memory.
+constexpr int OFF_OUT = OFF_X + XSPACE;  // this CTA's partial on its way to the peer
+constexpr int OFF_BAR = OFF_OUT + XSPACE;
+// The query slice is staged once through shared memory that is idle at the start: the last ring
+// stage, the exchange buffer and the first part of the outbox (five 128-row x 64-value boxes).
 constexpr int NQB = 5;
+constexpr int QBOX = 128 * 128;
 constexpr int OFF_QST = OFF_KV + (NST - 1) * STAGE;
-static_assert(OFF_QST % 1024 == 0 && OFF_QST + 3 * QBOX <= OFF_OUT && OFF_QP % 1024 == 0, "query staging area");
-// shared-memory address of query box k (0 .. 4)
-__device__ __forceinline__ uint32_t q_box_addr(uint8_t* smem, int k) {
-    return smem_u32(smem + (k == 1 || k == 2 ? OFF_QP + (k - 1) * QBOX : OFF_QST + (k == 0 ? 0 : k - 2) * QBOX));
-}
+static_assert(OFF_QST % 1024 == 0 && OFF_QST + NQB * QBOX <= OFF_BAR, "query staging area");
 constexpr int SMEM = 1024 + OFF_BAR + 512;
 static_assert(SMEM <= 232448, "shared memory budget");
 // tensor memory columns
 constexpr uint32_t T_O = 0;          // 256 fp32 columns: this rank's half of the output
-constexpr uint32_t T_Q = 256;        // 80 columns: query values 0-63 and 192-287 as bf16 pairs (k-steps 0-3, 12-17)
-constexpr uint32_t T_P = 336;        // NT/2 columns of bf16 pairs
-constexpr uint32_t T_R = 368;        // 6 columns: row maxima (2 tiles x 2 halves) and row sums of the warp pairs
-constexpr uint32_t T_S = 384;        // 2 x NT fp32 score partials (tile j in buffer j % 2)
-// tensor-memory column of k-step ks of the query (k-steps 4 .. 11 are in shared memory)
-__host__ __device__ constexpr uint32_t q_col(int ks) { return T_Q + (uint32_t)(ks < 4 ? ks : ks - 8) * 8; }
-static_assert(T_Q + 10 * 8 <= T_P && T_P + NT / 2 <= T_R && T_R + 6 <= T_S && T_S + 2 * NT <= 512,
+constexpr uint32_t T_Q = 256;        // 144 columns: this rank's 288 query values as bf16 pairs
+constexpr uint32_t T_P = 400;        // NT/2 columns of bf16 pairs
+constexpr uint32_t T_R = 432;        // 6 columns: row maxima (2 tiles x 2 halves) and row sums of the warp pairs
+constexpr uint32_t T_S = 448;        // NT fp32 score partials
+static_assert(T_Q + KSTEPS * 8 <= T_P && T_P + NT / 2 <= T_R && T_R + 6 <= T_S && T_S + NT <= 512,
               "tensor memory budget");
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 domain
 constexpr float kF16Max = 65504.f;         // largest finite fp16 value
@@ -187,9 +173,9 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
     uint64_t* q_loaded = bars + 1;        // the query slice is in shared memory
     uint64_t* kv_full = bars + 2;
     uint64_t* kv_empty = kv_full + NST;
-    uint64_t* s_ready = kv_empty + NST;   // [2] QK(j) done (score buffer j % 2)
-    uint64_t* s_free = s_ready + 2;       // [2] S(j) loaded by all softmax and sender warps
-    uint64_t* p_ready = s_free + 2;       // P(j) written by all softmax warps
+    uint64_t* s_ready = kv_empty + NST;   // QK(j) done
+    uint64_t* s_free = s_ready + 1;       // S(j) loaded by all softmax and sender warps
+    uint64_t* p_ready = s_free + 1;       // P(j) written by all softmax warps
     uint64_t* o_ready = p_ready + 1;      // PV(j) done
     uint64_t* xfull = o_ready + 1;        // [NSW] the peer's partial of warp w's block arrived
     uint64_t* xempty = xfull + NSW;       // [NSW] the peer has consumed this CTA's partial of warp w's block
@@ -222,10 +208,8 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
             mbar_init(smem_u32(&kv_full[s]), 1);
             mbar_init(smem_u32(&kv_empty[s]), 1);
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(smem_u32(&s_ready[i]), 1);
-            mbar_init(smem_u32(&s_free[i]), NSW + NXW);
-        }
+        mbar_init(smem_u32(s_ready), 1);
+        mbar_init(smem_u32(s_free), NSW + NXW);
         mbar_init(smem_u32(p_ready), NSW);
         mbar_init(smem_u32(o_ready), 1);
         for (int i = 0; i < NSW; ++i) {
@@ -256,9 +240,10 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
                 const uint32_t qb = smem_u32(q_loaded);
                 mbar_arrive_expect_tx(qb, NQB * QBOX);
                 const int qrow = (b * p.s_q + t) * 128;
+                const uint32_t qdst = smem_u32(smem + OFF_QST);
                 for (int k = 0; k < (rank ? NQB - 1 : NQB); ++k)
-                    tma_load_2d(q_box_addr(smem, k), &tm_qt, (int)rank * 288 + k * 64, qrow, qb);
-                if (rank) tma_load_3d(q_box_addr(smem, NQB - 1), &tm_qr, 0, t, b * 128, qb);
+                    tma_load_2d(qdst + k * QBOX, &tm_qt, (int)rank * 288 + k * 64, qrow, qb);
+                if (rank) tma_load_3d(qdst + (NQB - 1) * QBOX, &tm_qr, 0, t, b * 128, qb);
             }
             // tiles PF ahead of the one being loaded are prefetched into L2, so that the ring (whose
             // stages stay busy until P*V) is refilled from L2 rather than from DRAM
@@ -343,7 +328,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     __syncwarp();
                 }
-                if (j >= 2 && !mbar_wait(smem_u32(&s_free[j & 1]), ((j >> 1) - 1) & 1, p.status)) break;
+                if (j >= 1 && !mbar_wait(smem_u32(s_free), (j - 1) & 1, p.status)) break;
                 tc_fence_after();
                 if (lane == 0) {
                     const uint32_t kva = smem_u32(st);
@@ -351,15 +336,10 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
                     for (int ks = 0; ks < KSTEPS; ++ks) {
                         // score value 288 rank + 16 ks sits at offset 32 rank + 16 ks of this rank's tile
                         const int off = (int)rank * 32 + ks * 16;
-                        const uint64_t bd = smem_desc_sw128(kva + (off / 64) * BOX + (off % 64) * 2, 16, 1024);
-                        if (ks >= 4 && ks < 12)  // query values 64 .. 191: boxes 1 and 2 in shared memory
-                            umma_ss(tmem + T_S + (j & 1) * NT,
-                                    smem_desc_sw128(q_box_addr(smem, 1 + (ks - 4) / 4) + (ks % 4) * 32, 16, 1024), bd,
-                                    idesc_qk, ks != 0);
-                        else
-                            umma_ts(tmem + T_S + (j & 1) * NT, tmem + q_col(ks), bd, idesc_qk, ks != 0);
+                        umma_ts(tmem + T_S, tmem + T_Q + ks * 8,
+                                smem_desc_sw128(kva + (off / 64) * BOX + (off % 64) * 2, 16, 1024), idesc_qk, ks != 0);
                     }
-                    umma_commit(smem_u32(&s_ready[j & 1]));
+                    umma_commit(smem_u32(s_ready));
                 }
                 __syncwarp();
             }
@@ -474,14 +454,14 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
         uint32_t own[NT];
         bool ok = mbar_wait(smem_u32(q_full), 0, p.status);  // the outbox holds part of the staged query
         for (int j = 0; ok && j < n_tiles; ++j) {
-            ok = mbar_wait(smem_u32(&s_ready[j & 1]), (j >> 1) & 1, p.status);
+            ok = mbar_wait(smem_u32(s_ready), j & 1, p.status);
             tc_fence_after();
 #pragma unroll
-            for (int c0 = 0; c0 < NT; c0 += 16) tmem_ld16(tmem + lane_base + T_S + (j & 1) * NT + c0, own + c0);
+            for (int c0 = 0; c0 < NT; c0 += 16) tmem_ld16(tmem + lane_base + T_S + c0, own + c0);
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&s_free[j & 1]));
+            if (lane == 0) mbar_arrive(smem_u32(s_free));
             if (lane == 0) bulk_wait_read();  // the previous copies have read the outbox
             __syncwarp();
             // the partial goes out already scaled into the log2 domain (scale * log2 e), saturated to the
@@ -537,17 +517,15 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
         if (n_tiles > 0) {
-            // this rank's query values 0-63 and 192-287 of row h, staged in shared memory -> tensor memory (A
-            // operand of the score MMA, K-major: a column holds two consecutive values), five 16-column chunks of
-            // 32 values (chunks 0, 1, 6, 7, 8 of the slice): the first warp of the lane quarter writes chunks 0, 1,
-            // 6, the second 7, 8.  Values 64-191 (chunks 2-5) stay in shared memory (query boxes 1 and 2).
+            // this rank's 288 values of query row h, staged in shared memory -> tensor memory (A operand
+            // of the score MMA, K-major: column c holds values 2c and 2c+1).  Nine 16-column chunks of
+            // 32 values: the first warp of the lane quarter writes chunks 0-4, the second 5-8.
             if (ok) ok = mbar_wait(smem_u32(q_loaded), 0, p.status);
-            for (int n = half * 3; n < (half ? 5 : 3); ++n) {
-                const int c0 = n < 2 ? n : n + 4;
+            for (int c0 = half * 5; c0 < (half ? KSTEPS / 2 : 5); ++c0) {
                 const int v0 = c0 * 32;  // first value of the chunk within this rank's slice
                 const bool rope = rank == 1 && v0 >= 224;
                 const int box = rope ? NQB - 1 : v0 / 64, u0 = rope ? (v0 - 224) / 8 : (v0 % 64) / 8;
-                const uint8_t* row = smem + (q_box_addr(smem, box) - smem_u32(smem)) + h * 128;
+                const uint8_t* row = smem + OFF_QST + box * QBOX + h * 128;
                 uint32_t w[16];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
@@ -567,24 +545,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
                         w[e] = pack_f16x2(f.x * qs, f.y * qs);
                     }
                 }
-                tmem_st16(tmem + lane_base + q_col(2 * c0), w);
-            }
-            if (F8) {
-                // the query boxes that stay in shared memory become f16 too, in place (latent values only: the
-                // latent scale); 2048 16-byte chunks over the 256 softmax threads
-                const float qs = p.kv_scale[0];
-                uint8_t* qp = smem + OFF_QP;
-                for (int c = threadIdx.x; c < 2 * QBOX / 16; c += 32 * NSW) {
-                    uint4 v = *reinterpret_cast<const uint4*>(qp + c * 16);
-                    uint32_t* vw = reinterpret_cast<uint32_t*>(&v);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vw[e]));
-                        vw[e] = pack_f16x2(f.x * qs, f.y * qs);
-                    }
-                    *reinterpret_cast<uint4*>(qp + c * 16) = v;
-                }
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the tensor cores
+                tmem_st16(tmem + lane_base + T_Q + c0 * 16, w);
             }
             tmem_st_wait();
             tc_fence_before();
@@ -598,14 +559,14 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
         uint32_t cur[CW];
         // this warp's block of this rank's partial of tile j into registers (the sender warps send it)
         auto fetch = [&](int j) {
-            if (ok) ok = mbar_wait(smem_u32(&s_ready[j & 1]), (j >> 1) & 1, p.status);
+            if (ok) ok = mbar_wait(smem_u32(s_ready), j & 1, p.status);
             tc_fence_after();
-            tmem_ld16(tmem + lane_base + T_S + (j & 1) * NT + col0, cur);
-            tmem_ld16(tmem + lane_base + T_S + (j & 1) * NT + col0 + 16, cur + 16);
+            tmem_ld16(tmem + lane_base + T_S + col0, cur);
+            tmem_ld16(tmem + lane_base + T_S + col0 + 16, cur + 16);
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&s_free[j & 1]));
+            if (lane == 0) mbar_arrive(smem_u32(s_free));
         };
         // combine a per-row value with the partner warp's through TMEM column T_R + col (+ 1 for
         // the partner's); both warps of the lane quarter call it with the same col
