@@ -215,6 +215,18 @@ __device__ __forceinline__ int paged_row(const GqaParams& p, int b, int kvh, int
     return (page * p.h_kv + kvh) * p.page_size + tok % p.page_size;
 }
 
+// Whether `pred` holds in any of the 128 consumer threads (named barrier 1 with an OR reduction): a value every
+// consumer sees the same.
+__device__ __forceinline__ bool consumers_any(bool pred) {
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 1, 128, p;\n\t"
+                 "selp.u32 %0, 1, 0, q;\n\t}"
+                 : "=r"(r)
+                 : "r"((uint32_t)pred)
+                 : "memory");
+    return r != 0;
+}
+
 // The producer warp's lane 0: streams the split's n_tiles KV tiles (K and V of C::T_TILE tokens per stage, as
 // 128-byte swizzled segments of C::SEG_ELEMS values) through the C::NSTAGE ring of full / empty mbarriers, then
 // waits until every copy it issued has landed (a CTA must not exit with copies in flight).
@@ -585,9 +597,9 @@ __global__ void __launch_bounds__(160, GqaCfg<KV, D, RB>::MINB)
 #pragma unroll
     for (int m = C::LPT; m < 32; m *= 2) l_run += __shfl_xor_sync(0xffffffffu, l_run, m);
 
-    // all consumer warps reach here; aborted CTAs stop without writing results
-    named_barrier(1, 128);
-    if (*(volatile int*)&s_abort || aborted) return;
+    // all consumer warps reach here; aborted CTAs stop without writing results (the decision is the same in
+    // every consumer thread)
+    if (consumers_any(aborted || *(volatile int*)&s_abort)) return;
 
     // ---- merge the four warp states in shared memory (reusing the stage ring) ----
     float* om = reinterpret_cast<float*>(stages);  // [4][RB][D]
@@ -608,17 +620,6 @@ __global__ void __launch_bounds__(160, GqaCfg<KV, D, RB>::MINB)
     gqa_merge_store<T, D, RB>(om, mm, lm, p, b, kvh, row0, rows_here, L, kbeg, split, v_mul);
 }
 
-// Whether `pred` holds in any of the 128 consumer threads (named barrier 1 with an OR reduction): a value every
-// consumer sees the same.
-__device__ __forceinline__ bool consumers_any(bool pred) {
-    uint32_t r;
-    asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 1, 128, p;\n\t"
-                 "selp.u32 %0, 1, 0, q;\n\t}"
-                 : "=r"(r)
-                 : "r"((uint32_t)pred)
-                 : "memory");
-    return r != 0;
-}
 
 // ---- tensor-core instances: bf16 caches (d in {64, 128}) and e4m3 caches (d = 128) -------------------------------
 // The block's query rows (up to 16: h_q / h_kv heads x s_q tokens; rows past R are zero padding) are the M = 16
