@@ -59,6 +59,9 @@ from latent_kv_attention_b200 import costs, sharding  # noqa: E402
 METRIC = "decode-attention HBM GB/s (% of peak), TFLOPS (% of roofline), tokens/s"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+# NVIDIA's B200 datasheet figures, reported beside the measured peaks: HBM3e 8 TB/s, dense bf16 2.25 PFLOP/s
+DATASHEET_HBM_GBS = 8000.0
+DATASHEET_BF16_TFLOPS = 2250.0
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -768,11 +771,13 @@ def measure(wl, steps, warmup, pk, device, world, soak_s=1.0, clocks=None):
         peak, unit, achieved = pk["bf16_tflops"], "TFLOP/s", work / (kern_ms * 1e-3) / 1e12
         peak_src = "bf16_tflops (burst)"
     traffic = recorded_traffic(wl.kernel, wl.name, wl.src)
+    datasheet = DATASHEET_HBM_GBS if unit == "GB/s" else DATASHEET_BF16_TFLOPS
     roof = {"bound": bound, "kernel": wl.kernel, "achieved": round(achieved, 1), "peak": peak, "unit": unit,
             "frac": round(achieved / peak, 4), "traffic": traffic, "algorithmic_work_per_launch": work,
             "launch_ms": round(kern_ms, 4),
             "peak_source": f"{pk['source']} (MEASURED_PEAKS.json {peak_src})" if pk["source"] == "measured"
-            else "fallback"}
+            else "fallback",
+            "datasheet_peak": datasheet, "datasheet_frac": round(achieved / datasheet, 4)}
     return dict(step_ms=step_ms, e2e_ms=e2e_ms, roofline=roof, clocks=clk)
 
 
