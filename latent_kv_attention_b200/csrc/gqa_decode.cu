@@ -227,16 +227,41 @@ __device__ __forceinline__ bool consumers_any(bool pred) {
     return r != 0;
 }
 
-// The producer warp's lane 0: streams the split's n_tiles KV tiles (K and V of C::T_TILE tokens per stage, as
-// 128-byte swizzled segments of C::SEG_ELEMS values) through the C::NSTAGE ring of full / empty mbarriers, then
-// waits until every copy it issued has landed (a CTA must not exit with copies in flight).
+// Issues the copies of one KV tile (K and V of C::T_TILE tokens from token tok0 of sequence b, KV head kvh, as
+// 128-byte swizzled segments of C::SEG_ELEMS values) into kdst / vdst, completing on `full`.
+template <class C>
+__device__ __forceinline__ void gqa_issue_tile(const CUtensorMap* tmK, const CUtensorMap* tmV, const GqaParams& p,
+                                               uint32_t kdst, uint32_t vdst, uint32_t full, int b, int kvh, int L,
+                                               int tok0) {
+    if (!p.block_table) {
+        const int y = (b * p.h_kv + kvh) * p.Lmax + tok0;
+#pragma unroll
+        for (int sg = 0; sg < C::NSEG; ++sg) {
+            tma_load_2d(kdst + sg * C::T_TILE * 128, tmK, sg * C::SEG_ELEMS, y, full);
+            tma_load_2d(vdst + sg * C::T_TILE * 128, tmV, sg * C::SEG_ELEMS, y, full);
+        }
+    } else {
+        // paged cache: the tile is box_rows-row pieces, each inside one page of the block table
+        for (int r0 = 0; r0 < C::T_TILE; r0 += p.box_rows) {
+            const int tok = tok0 + r0;
+            const int y = paged_row(p, b, kvh, tok, tok < L);
+#pragma unroll
+            for (int sg = 0; sg < C::NSEG; ++sg) {
+                tma_load_2d(kdst + sg * C::T_TILE * 128 + r0 * 128, tmK, sg * C::SEG_ELEMS, y, full);
+                tma_load_2d(vdst + sg * C::T_TILE * 128 + r0 * 128, tmV, sg * C::SEG_ELEMS, y, full);
+            }
+        }
+    }
+}
+
+// The producer warp's lane 0: streams the split's n_tiles KV tiles through the C::NSTAGE ring of full / empty
+// mbarriers, then waits until every copy it issued has landed (a CTA must not exit with copies in flight).
 template <class C>
 __device__ __forceinline__ void gqa_produce(const CUtensorMap* tmK, const CUtensorMap* tmV, const GqaParams& p,
                                             uint8_t* stages, uint64_t* bars, int* s_abort, int b, int kvh, int L,
                                             int kbeg, int n_tiles) {
     prefetch_tensormap(tmK);
     prefetch_tensormap(tmV);
-    const int ybase = (b * p.h_kv + kvh) * p.Lmax;
     int issued = 0;
     for (int it = 0; it < n_tiles; ++it) {
         const int s = it % C::NSTAGE;
@@ -250,27 +275,7 @@ __device__ __forceinline__ void gqa_produce(const CUtensorMap* tmK, const CUtens
         const uint32_t full = smem_u32(&bars[s]);
         mbar_arrive_expect_tx(full, C::STAGE_BYTES);
         const uint32_t kdst = smem_u32(stages + s * C::STAGE_BYTES);
-        const uint32_t vdst = kdst + C::MAT_BYTES;
-        const int tok0 = kbeg + it * C::T_TILE;
-        if (!p.block_table) {
-            const int y = ybase + tok0;
-#pragma unroll
-            for (int sg = 0; sg < C::NSEG; ++sg) {
-                tma_load_2d(kdst + sg * C::T_TILE * 128, tmK, sg * C::SEG_ELEMS, y, full);
-                tma_load_2d(vdst + sg * C::T_TILE * 128, tmV, sg * C::SEG_ELEMS, y, full);
-            }
-        } else {
-            // paged cache: the tile is box_rows-row pieces, each inside one page of the block table
-            for (int r0 = 0; r0 < C::T_TILE; r0 += p.box_rows) {
-                const int tok = tok0 + r0;
-                const int y = paged_row(p, b, kvh, tok, tok < L);
-#pragma unroll
-                for (int sg = 0; sg < C::NSEG; ++sg) {
-                    tma_load_2d(kdst + sg * C::T_TILE * 128 + r0 * 128, tmK, sg * C::SEG_ELEMS, y, full);
-                    tma_load_2d(vdst + sg * C::T_TILE * 128 + r0 * 128, tmV, sg * C::SEG_ELEMS, y, full);
-                }
-            }
-        }
+        gqa_issue_tile<C>(tmK, tmV, p, kdst, kdst + C::MAT_BYTES, full, b, kvh, L, kbeg + it * C::T_TILE);
         ++issued;
     }
     for (int it = issued - 1; it >= 0 && it >= issued - C::NSTAGE; --it)
@@ -640,7 +645,7 @@ __global__ void __launch_bounds__(160, GqaCfg<KV, D, RB>::MINB)
 //     its 16 value rows once per tile into an f16 scratch tile (in that token order, zero past the split's keys),
 //     which the transposing ldmatrix reads as in the bf16 case.  P is f16; the per-KV-head scales are applied to
 //     the fp32 scores and to the merged output.
-template <int D, bool F8>
+template <int D, bool F8, bool R8 = false>
 struct GqaMmaCfg {
     static constexpr int RB = 16;                  // query rows per CTA (the MMA's M)
     static constexpr int TW = 16;                  // tokens per warp per tile
@@ -651,10 +656,12 @@ struct GqaMmaCfg {
     static constexpr int MAT_BYTES = T_TILE * D * E;
     static constexpr int STAGE_BYTES = 2 * MAT_BYTES;
     static constexpr int NSTAGE0 = (LKA_GQA_STAGE_KB * 1024) / STAGE_BYTES;
-    static constexpr int NSTAGE_CAP = F8 ? 3 : 6;
+    // R8: the 8-row form, which reads e4m3 values straight from the stage (no scratch tile): room for a fourth
+    // stage beside three CTAs per SM
+    static constexpr int NSTAGE_CAP = F8 ? (R8 ? 4 : 3) : 6;
     static constexpr int NSTAGE = NSTAGE0 > NSTAGE_CAP ? NSTAGE_CAP : NSTAGE0;
     static constexpr int RING = NSTAGE * STAGE_BYTES;
-    static constexpr int SCR_W = F8 ? TW * D * 2 : 0;  // per-warp f16 value tile (e4m3 cache)
+    static constexpr int SCR_W = F8 && !R8 ? TW * D * 2 : 0;  // per-warp f16 value tile (16-row form, e4m3)
     static constexpr int OFF_BAR = RING + 4 * SCR_W;
     static constexpr int MERGE_BYTES = 4 * RB * D * 4 + 2 * 4 * RB * 4;
     static constexpr int SMEM = 1024 + OFF_BAR + 256;
@@ -1039,12 +1046,280 @@ __global__ void __launch_bounds__(160, 2)
 // rows empty.  The score accumulator holds P^T (tokens x rows); movmatrix transposes its two 8 x 8 halves into the
 // B operand of the P*V MMA.  Everything else (softmax, scales, the e4m3 handling with its permuted head-dim order
 // and token order, the merge) is as in the 16-row form above.
+//
+// Per-warp state of the 8-row form over one work item: the query slice as B fragments of the score MMA, the
+// last visible key of the lane's two query rows, the O^T accumulators and the lazily moved maxima with this
+// lane's shares of the row sums.
+template <int D>
+struct Mma8Warp {
+    uint32_t qb[D / 16][2];  // query row g: bf16 pairs as given, or f16 pairs in the permuted e4m3 order
+    int last[2];             // last visible key of query rows 2 tq, 2 tq + 1 (-1: a padding row, nothing visible)
+    float o[D / 16][4];      // O^T: head-dim values 16 mt + g (+ 8), query rows 2 tq, 2 tq + 1
+    float m_run[2], l_run[2];
+};
+
+// Query row g of the block into the B fragments of lane (g, tq) (zeros when ok is false); qrow points at the
+// row's D bf16 values.  The scale goes on the fp32 scores, so the values are taken as given.
 template <int D, bool F8>
-__global__ void __launch_bounds__(160, GqaMmaCfg<D, F8>::MINB)
+__device__ __forceinline__ void mma8_load_q(uint32_t (&qb)[D / 16][2], const uint32_t* qrow, bool ok, int tq) {
+    auto qpair = [&](int u) -> uint32_t {
+        const uint32_t w = ok ? qrow[u] : 0u;
+        if constexpr (F8) {
+            float lo, hi;
+            bf16x2_to_f32(w, lo, hi);
+            return pack_f16x2_rn(lo, hi);
+        } else {
+            return w;
+        }
+    };
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+        // pairs of values: bf16 layout 16 ks + 2 tq (+ 8); e4m3 permuted layout 64 G + 16 tq + 4 j (+ 2)
+        const int u0 = F8 ? 32 * (ks >> 2) + 8 * tq + 2 * (ks & 3) : 8 * ks + tq;
+        qb[ks][0] = qpair(u0);
+        qb[ks][1] = qpair(F8 ? u0 + 1 : u0 + 4);
+    }
+}
+
+// A fresh online-softmax state and the row limits of lane (g, tq) for the block of rows row0 .. row0 + 7 of a
+// group of R query rows (row gr of the group is query position gr mod s_q) over L cache tokens.
+template <int D>
+__device__ __forceinline__ void mma8_reset(Mma8Warp<D>& st, const GqaParams& p, int row0, int R, int L, int tq) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int gr = row0 + 2 * tq + i;
+        st.last[i] = gr < R ? (p.causal ? L - p.s_q + gr % p.s_q : L - 1) : -1;
+        st.m_run[i] = -INFINITY;
+        st.l_run[i] = 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < D / 16; ++j) st.o[j][0] = st.o[j][1] = st.o[j][2] = st.o[j][3] = 0.f;
+}
+
+// One tile of the 8-row form for consumer warp `warp`: the scores of its 16 tokens of the stage (keys at
+// `stage`, values MAT_BYTES after them), the online softmax and O^T += V^T P^T.  tbase: the tile's first key;
+// kend: the split's end; keys below mask_from are visible to every row.  The warp arrives on `empty` after its
+// P*V MMAs, when it no longer reads the stage.
+template <int D, bool F8>
+__device__ __forceinline__ void mma8_tile(Mma8Warp<D>& st, uint8_t* stage, int tbase, int kend, int mask_from,
+                                          float s_mul, const uint32_t (&k_off)[4], const uint32_t (&v_off)[4],
+                                          const int (&tok_g)[2], uint32_t empty, int warp, int lane) {
+    using C = GqaMmaCfg<D, F8, true>;
+    constexpr int KS = D / 16, MT = D / 16;
+    constexpr int V_SEG = C::T_TILE * 128;  // bytes per 64-value segment of a bf16 value tile
+    const int g = lane >> 2, tq = lane & 3;
+    const uint32_t kt = smem_u32(stage);
+    const uint32_t vt = kt + C::MAT_BYTES;
+    // ---- S^T = K Q^T for the warp's 16 tokens (two accumulators: even / odd k-steps) ----
+    float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    if constexpr (F8) {
+#pragma unroll
+        for (int G = 0; G < D / 64; ++G) {
+            const int seg = G >> 1, chunk = 4 * (G & 1) + tq;
+            uint4 w[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int row = 16 * warp + tok_g[h];
+                w[h] = *reinterpret_cast<const uint4*>(stage + seg * C::T_TILE * 128 + row * 128 +
+                                                       ((chunk ^ (row & 7)) << 4));
+            }
+            const uint32_t w0[4] = {w[0].x, w[0].y, w[0].z, w[0].w}, w1[4] = {w[1].x, w[1].y, w[1].z, w[1].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t a[4] = {e4m3x2_lo_to_f16x2(w0[j]), e4m3x2_lo_to_f16x2(w1[j]),
+                                       e4m3x2_hi_to_f16x2(w0[j]), e4m3x2_hi_to_f16x2(w1[j])};
+                mma_16816<true>(sc[j & 1], a, st.qb[4 * G + j][0], st.qb[4 * G + j][1]);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            uint32_t a[4];
+            ldsm_x4(kt + (ks >> 2) * C::T_TILE * 128 + k_off[ks & 3], a);
+            // ldmatrix order (tokens 0-7 lo, tokens 0-7 hi, tokens 8-15 lo, tokens 8-15 hi) -> a0 a2 a1 a3
+            const uint32_t af[4] = {a[0], a[2], a[1], a[3]};
+            mma_16816<false>(sc[ks & 1], af, st.qb[ks][0], st.qb[ks][1]);
+        }
+    }
+    // x[e]: token tbase + 16 warp + tok_g[e / 2], query row 2 tq + e % 2, in the log2 domain
+    float x[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) x[e] = (sc[0][e] + sc[1][e]) * s_mul;
+    if (tbase + C::T_TILE > mask_from) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int tok = tbase + 16 * warp + tok_g[e >> 1];
+            x[e] = (tok < kend && tok <= st.last[e & 1]) ? x[e] : -INFINITY;
+        }
+    }
+    // ---- online softmax of the two rows (over the 8 lanes that share tq), lazily rescaled ----
+    float mx[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        mx[i] = fmaxf(x[i], x[2 + i]);
+        mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 4));
+        mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 8));
+        mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 16));
+    }
+    if (__any_sync(0xffffffffu, mx[0] > st.m_run[0] + 8.0f || mx[1] > st.m_run[1] + 8.0f)) {
+        float alpha[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const float m_new = fmaxf(st.m_run[i], mx[i]);
+            alpha[i] = 1.f;
+            if (st.m_run[i] == -INFINITY) {
+                st.m_run[i] = m_new;  // O and l of the row are still zero
+            } else if (m_new > st.m_run[i] + 8.0f) {
+                alpha[i] = fast_exp2(st.m_run[i] - m_new);
+                st.m_run[i] = m_new;
+            }
+            st.l_run[i] *= alpha[i];
+        }
+#pragma unroll
+        for (int j = 0; j < MT; ++j) {
+            st.o[j][0] *= alpha[0];
+            st.o[j][1] *= alpha[1];
+            st.o[j][2] *= alpha[0];
+            st.o[j][3] *= alpha[1];
+        }
+    }
+    uint32_t pb[2];  // B fragment of the P*V MMA: query row g, tokens 2 tq, 2 tq + 1 (+ 8)
+    {
+        const float ms0 = st.m_run[0] == -INFINITY ? 0.f : st.m_run[0];  // no visible key yet: p = 2^-inf = 0
+        const float ms1 = st.m_run[1] == -INFINITY ? 0.f : st.m_run[1];
+        const float p0 = fast_exp2(x[0] - ms0), p1 = fast_exp2(x[1] - ms1);
+        const float p2 = fast_exp2(x[2] - ms0), p3 = fast_exp2(x[3] - ms1);
+        st.l_run[0] += p0 + p2;  // this lane's share; summed over the row's lanes at the end
+        st.l_run[1] += p1 + p3;
+        // P^T halves (tokens g / g + 8 x rows 2 tq, 2 tq + 1) transposed into P halves (row g x tokens)
+        const uint32_t t0 = F8 ? pack_f16x2_rn(p0, p1) : pack_bf16x2(p0, p1);
+        const uint32_t t1 = F8 ? pack_f16x2_rn(p2, p3) : pack_bf16x2(p2, p3);
+        asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(pb[0]) : "r"(t0));
+        asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(pb[1]) : "r"(t1));
+    }
+    const int nvalid = kend - (tbase + 16 * warp);  // value rows of the warp that are keys of the split
+    if constexpr (F8) {
+        // ---- O^T += V^T P^T straight from the e4m3 stage ----
+        // Lane (g, tq) reads the 16 value bytes of head-dim chunk vch(g) of the warp's tokens tq, tq + 4, 8 + tq and
+        // 12 + tq: the tokens of the MMA's k-indices 2 tq, 2 tq + 1, 2 tq + 8, 2 tq + 9 in the permuted token order.
+        // A byte permute pairs the two tokens of a k-pair value by value and one conversion widens the pair, so
+        // that A-fragment rows g and g + 8 of m-tile mt hold head-dim values 16 vch(g) + 2 mt and + 1.  vch puts
+        // the chunks of lanes g = 2 i and 2 i + 1 in different halves of the swizzled row, so the 8 lanes of a
+        // shared-memory phase read 8 different 16-byte columns.  Rows past the split's keys may hold anything
+        // (even NaN), which P = 0 would not cancel in the MMA: they become 0.
+        const int vch = ((g & 1) << 2) | (g >> 1);
+        const uint8_t* vsrc = stage + C::MAT_BYTES;
+        uint32_t vw[4][4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int t = tq + 4 * j;  // token of the warp's 16
+            const int row = 16 * warp + t;
+            uint4 w = *reinterpret_cast<const uint4*>(vsrc + row * 128 + ((vch ^ (row & 7)) << 4));
+            if (t >= nvalid) w = make_uint4(0u, 0u, 0u, 0u);
+            vw[j][0] = w.x;
+            vw[j][1] = w.y;
+            vw[j][2] = w.z;
+            vw[j][3] = w.w;
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {  // value bytes 4 q .. 4 q + 3 of the chunk: m-tiles 2 q and 2 q + 1
+            const uint32_t lo01 = __byte_perm(vw[0][q], vw[1][q], 0x5140), hi01 = __byte_perm(vw[0][q], vw[1][q], 0x7362);
+            const uint32_t lo23 = __byte_perm(vw[2][q], vw[3][q], 0x5140), hi23 = __byte_perm(vw[2][q], vw[3][q], 0x7362);
+            const uint32_t a0[4] = {e4m3x2_lo_to_f16x2(lo01), e4m3x2_hi_to_f16x2(lo01), e4m3x2_lo_to_f16x2(lo23),
+                                    e4m3x2_hi_to_f16x2(lo23)};
+            mma_16816<true>(st.o[2 * q], a0, pb[0], pb[1]);
+            const uint32_t a1[4] = {e4m3x2_lo_to_f16x2(hi01), e4m3x2_hi_to_f16x2(hi01), e4m3x2_lo_to_f16x2(hi23),
+                                    e4m3x2_hi_to_f16x2(hi23)};
+            mma_16816<true>(st.o[2 * q + 1], a1, pb[0], pb[1]);
+        }
+    } else {
+        if (nvalid < 16) {
+            // value rows of the warp past the split's keys (the last tile) may hold anything, even NaN, and
+            // P = 0 does not cancel that in the MMA: zero them
+            const int first = nvalid < 0 ? 0 : nvalid;
+            uint8_t* vrow = stage + C::MAT_BYTES;
+            for (int idx = lane; idx < (16 - first) * C::NSEG * 8; idx += 32) {
+                const int row = 16 * warp + first + idx / (C::NSEG * 8), rem = idx % (C::NSEG * 8);
+                *reinterpret_cast<uint4*>(vrow + (rem / 8) * C::T_TILE * 128 + row * 128 + (rem % 8) * 16) =
+                    make_uint4(0u, 0u, 0u, 0u);
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // before the ring's next copy
+            __syncwarp();
+        }
+        // ---- O^T += V^T P^T: one MMA per 16 head-dim values ----
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            uint32_t a[4];
+            ldsm_x4_t(vt + (mt >> 2) * V_SEG + v_off[mt & 3], a);
+            // ldmatrix order (tokens 0-7 x d lo, tokens 0-7 x d hi, tokens 8-15 x d lo, tokens 8-15 x d hi),
+            // transposed: (d lo, k lo) (d hi, k lo) (d lo, k hi) (d hi, k hi) = a0 a1 a2 a3
+            mma_16816<false>(st.o[mt], a, pb[0], pb[1]);
+        }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty);
+}
+
+// Sums this lane's row-sum shares over the row's eight lanes and writes the warp's state for the merge:
+// om [4][8][D] (the O^T fragments back in row-major order), mm / lm [4][8].
+template <int D, bool F8>
+__device__ __forceinline__ void mma8_stash(Mma8Warp<D>& st, float* om, float* mm, float* lm, int warp, int lane) {
+    constexpr int RB = 8;
+    const int g = lane >> 2, tq = lane & 3;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        st.l_run[i] += __shfl_xor_sync(0xffffffffu, st.l_run[i], 4);
+        st.l_run[i] += __shfl_xor_sync(0xffffffffu, st.l_run[i], 8);
+        st.l_run[i] += __shfl_xor_sync(0xffffffffu, st.l_run[i], 16);
+    }
+    float* o0 = om + (warp * RB + 2 * tq) * D;  // query row 2 tq (o1: 2 tq + 1)
+    float* o1 = o0 + D;
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) {
+        if constexpr (F8) {  // rows g, g + 8 of m-tile mt: head-dim values d, d + 1 for d = 16 vch(g) + 2 mt
+            const int d = 16 * (((g & 1) << 2) | (g >> 1)) + 2 * mt;
+            *reinterpret_cast<float2*>(o0 + d) = make_float2(st.o[mt][0], st.o[mt][2]);
+            *reinterpret_cast<float2*>(o1 + d) = make_float2(st.o[mt][1], st.o[mt][3]);
+        } else {  // rows g, g + 8 of m-tile mt: head-dim values 16 mt + g, + 8
+            o0[16 * mt + g] = st.o[mt][0];
+            o1[16 * mt + g] = st.o[mt][1];
+            o0[16 * mt + g + 8] = st.o[mt][2];
+            o1[16 * mt + g + 8] = st.o[mt][3];
+        }
+    }
+    if (g == 0) {
+        mm[warp * RB + 2 * tq] = st.m_run[0];
+        mm[warp * RB + 2 * tq + 1] = st.m_run[1];
+        lm[warp * RB + 2 * tq] = st.l_run[0];
+        lm[warp * RB + 2 * tq + 1] = st.l_run[1];
+    }
+}
+
+// ldmatrix row addresses of lane `lane` in warp `warp` for a bf16 stage (byte offsets, 128-byte swizzle), and
+// the token of the warp's 16 held by MMA row g + 8 h.  Both operands are A fragments read from token rows: matrix
+// l / 8 = (token half l / 16, 8-value chunk parity (l / 8) % 2).  Keys: non-transposed, one k-step; values
+// (transposed): one 16-value m-tile of O^T.
+template <bool F8>
+__device__ __forceinline__ void mma8_offsets(uint32_t (&k_off)[4], uint32_t (&v_off)[4], int (&tok_g)[2], int warp,
+                                             int lane) {
+    const int g = lane >> 2, r8 = lane & 7;
+    const uint32_t k_row = (uint32_t)(16 * warp + 8 * (lane >> 4) + r8) * 128;
+    const uint32_t v_row = k_row;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        k_off[c] = k_row + ((uint32_t)((2 * c + ((lane >> 3) & 1)) ^ r8) << 4);
+        v_off[c] = v_row + ((uint32_t)((2 * c + ((lane >> 3) & 1)) ^ r8) << 4);
+    }
+    tok_g[0] = F8 ? f8_tok(g) : g;
+    tok_g[1] = 8 + tok_g[0];
+}
+
+template <int D, bool F8>
+__global__ void __launch_bounds__(160, GqaMmaCfg<D, F8, true>::MINB)
     gqa_decode_mma8_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                            const GqaParams p) {
-    using C = GqaMmaCfg<D, F8>;
-    constexpr int RB = 8, KS = D / 16, MT = D / 16;
+    using C = GqaMmaCfg<D, F8, true>;
+    constexpr int RB = 8;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
     uint8_t* stages = smem;
@@ -1092,61 +1367,22 @@ __global__ void __launch_bounds__(160, GqaMmaCfg<D, F8>::MINB)
     // Fragment coordinates: lane = 4 g + tq.  Score accumulator: tokens (MMA rows) g and g + 8 of the warp's 16,
     // query rows (MMA columns) 2 tq and 2 tq + 1.  B operand of the score MMA: query row g.
     const int g = lane >> 2, tq = lane & 3;
-    int last[2];  // last visible key of query rows 2 tq and 2 tq + 1 (-1: a padding row, nothing visible)
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const int gr = row0 + 2 * tq + i;
-        last[i] = gr < R ? (p.causal ? L - p.s_q + gr % p.s_q : L - 1) : -1;
-    }
-    uint32_t qb[KS][2];  // B fragments of the score MMA: query row g, as given (the scale goes on the fp32 scores)
+    Mma8Warp<D> st;
+    mma8_reset<D>(st, p, row0, R, L, tq);
     {
         const __nv_bfloat16* qbase = reinterpret_cast<const __nv_bfloat16*>(p.q) +
                                      ((size_t)(b * p.h_q + kvh * p.ratio) * p.s_q) * D;  // first row of the group
         const bool ok = row0 + g < R;
-        const uint32_t* qrow = reinterpret_cast<const uint32_t*>(qbase + (size_t)(ok ? row0 + g : 0) * D);
-        auto qpair = [&](int u) -> uint32_t {
-            const uint32_t w = ok ? qrow[u] : 0u;
-            if constexpr (F8) {
-                float lo, hi;
-                bf16x2_to_f32(w, lo, hi);
-                return pack_f16x2_rn(lo, hi);
-            } else {
-                return w;
-            }
-        };
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-            // pairs of values: bf16 layout 16 ks + 2 tq (+ 8); e4m3 permuted layout 64 G + 16 tq + 4 j (+ 2)
-            const int u0 = F8 ? 32 * (ks >> 2) + 8 * tq + 2 * (ks & 3) : 8 * ks + tq;
-            qb[ks][0] = qpair(u0);
-            qb[ks][1] = qpair(F8 ? u0 + 1 : u0 + 4);
-        }
+        mma8_load_q<D, F8>(st.qb, reinterpret_cast<const uint32_t*>(qbase + (size_t)(ok ? row0 + g : 0) * D), ok,
+                           tq);
     }
-    float o[MT][4];  // O^T: head-dim values 16 mt + g (+ 8), query rows 2 tq, 2 tq + 1
-#pragma unroll
-    for (int j = 0; j < MT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
     const float s_mul = F8 ? p.scale_log2 * p.k_scale[kvh] : p.scale_log2;
     int mask_from = kend;  // keys below mask_from are visible to every row of the block
     for (int r = 0; r < rows_here; ++r)
         mask_from = min(mask_from, p.causal ? L - p.s_q + (row0 + r) % p.s_q + 1 : L);
-    // token (of the warp's 16) of MMA row g + 8 h
-    const int tok_g[2] = {F8 ? f8_tok(g) : g, 8 + (F8 ? f8_tok(g) : g)};
-
-    // ldmatrix row addresses (byte offsets, 128-byte swizzle).  Both operands are A fragments read from token rows:
-    // matrix l / 8 = (token half l / 16, 8-value chunk parity (l / 8) % 2).  bf16 keys: non-transposed, one k-step;
-    // values (transposed; the stage for bf16, the warp's scratch tile for e4m3): one 16-value m-tile of O^T.
-    const int r8 = lane & 7;
-    const uint32_t k_row = (uint32_t)(16 * warp + 8 * (lane >> 4) + r8) * 128;
-    const uint32_t v_row = (uint32_t)((F8 ? 0 : 16 * warp) + 8 * (lane >> 4) + r8) * 128;
-    constexpr int V_SEG = F8 ? C::TW * 128 : C::T_TILE * 128;  // bytes per 64-value segment of a value tile
     uint32_t k_off[4], v_off[4];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        k_off[c] = k_row + ((uint32_t)((2 * c + ((lane >> 3) & 1)) ^ r8) << 4);
-        v_off[c] = v_row + ((uint32_t)((2 * c + ((lane >> 3) & 1)) ^ r8) << 4);
-    }
-    uint8_t* scr = smem + C::RING + warp * C::SCR_W;
+    int tok_g[2];
+    mma8_offsets<F8>(k_off, v_off, tok_g, warp, lane);
 
     bool aborted = false;
     for (int it = 0; it < n_tiles; ++it) {
@@ -1156,190 +1392,23 @@ __global__ void __launch_bounds__(160, GqaMmaCfg<D, F8>::MINB)
             s_abort = 1;
             break;
         }
-        const uint32_t kt = smem_u32(stages + s * C::STAGE_BYTES);
-        const uint32_t vt = kt + C::MAT_BYTES;
-        const int tbase = kbeg + it * C::T_TILE;
-
-        // ---- S^T = K Q^T for the warp's 16 tokens (two accumulators: even / odd k-steps) ----
-        float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        if constexpr (F8) {
-            const uint8_t* kst = stages + s * C::STAGE_BYTES;
-#pragma unroll
-            for (int G = 0; G < D / 64; ++G) {
-                const int seg = G >> 1, chunk = 4 * (G & 1) + tq;
-                uint4 w[2];
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int row = 16 * warp + tok_g[h];
-                    w[h] = *reinterpret_cast<const uint4*>(kst + seg * C::T_TILE * 128 + row * 128 +
-                                                           ((chunk ^ (row & 7)) << 4));
-                }
-                const uint32_t w0[4] = {w[0].x, w[0].y, w[0].z, w[0].w}, w1[4] = {w[1].x, w[1].y, w[1].z, w[1].w};
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint32_t a[4] = {e4m3x2_lo_to_f16x2(w0[j]), e4m3x2_lo_to_f16x2(w1[j]),
-                                           e4m3x2_hi_to_f16x2(w0[j]), e4m3x2_hi_to_f16x2(w1[j])};
-                    mma_16816<true>(sc[j & 1], a, qb[4 * G + j][0], qb[4 * G + j][1]);
-                }
-            }
-        } else {
-#pragma unroll
-            for (int ks = 0; ks < KS; ++ks) {
-                uint32_t a[4];
-                ldsm_x4(kt + (ks >> 2) * C::T_TILE * 128 + k_off[ks & 3], a);
-                // ldmatrix order (tokens 0-7 lo, tokens 0-7 hi, tokens 8-15 lo, tokens 8-15 hi) -> a0 a2 a1 a3
-                const uint32_t af[4] = {a[0], a[2], a[1], a[3]};
-                mma_16816<false>(sc[ks & 1], af, qb[ks][0], qb[ks][1]);
-            }
-        }
-        // x[e]: token tbase + 16 warp + tok_g[e / 2], query row 2 tq + e % 2, in the log2 domain
-        float x[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) x[e] = (sc[0][e] + sc[1][e]) * s_mul;
-        if (tbase + C::T_TILE > mask_from) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int tok = tbase + 16 * warp + tok_g[e >> 1];
-                x[e] = (tok < kend && tok <= last[e & 1]) ? x[e] : -INFINITY;
-            }
-        }
-        // ---- online softmax of the two rows (over the 8 lanes that share tq), lazily rescaled ----
-        float mx[2];
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            mx[i] = fmaxf(x[i], x[2 + i]);
-            mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 4));
-            mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 8));
-            mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 16));
-        }
-        if (__any_sync(0xffffffffu, mx[0] > m_run[0] + 8.0f || mx[1] > m_run[1] + 8.0f)) {
-            float alpha[2];
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const float m_new = fmaxf(m_run[i], mx[i]);
-                alpha[i] = 1.f;
-                if (m_run[i] == -INFINITY) {
-                    m_run[i] = m_new;  // O and l of the row are still zero
-                } else if (m_new > m_run[i] + 8.0f) {
-                    alpha[i] = fast_exp2(m_run[i] - m_new);
-                    m_run[i] = m_new;
-                }
-                l_run[i] *= alpha[i];
-            }
-#pragma unroll
-            for (int j = 0; j < MT; ++j) {
-                o[j][0] *= alpha[0];
-                o[j][1] *= alpha[1];
-                o[j][2] *= alpha[0];
-                o[j][3] *= alpha[1];
-            }
-        }
-        uint32_t pb[2];  // B fragment of the P*V MMA: query row g, tokens 2 tq, 2 tq + 1 (+ 8)
-        {
-            const float ms0 = m_run[0] == -INFINITY ? 0.f : m_run[0];  // no visible key yet: p = 2^-inf = 0
-            const float ms1 = m_run[1] == -INFINITY ? 0.f : m_run[1];
-            const float p0 = fast_exp2(x[0] - ms0), p1 = fast_exp2(x[1] - ms1);
-            const float p2 = fast_exp2(x[2] - ms0), p3 = fast_exp2(x[3] - ms1);
-            l_run[0] += p0 + p2;  // this lane's share; summed over the row's lanes at the end
-            l_run[1] += p1 + p3;
-            // P^T halves (tokens g / g + 8 x rows 2 tq, 2 tq + 1) transposed into P halves (row g x tokens)
-            const uint32_t t0 = F8 ? pack_f16x2_rn(p0, p1) : pack_bf16x2(p0, p1);
-            const uint32_t t1 = F8 ? pack_f16x2_rn(p2, p3) : pack_bf16x2(p2, p3);
-            asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(pb[0]) : "r"(t0));
-            asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(pb[1]) : "r"(t1));
-        }
-        uint32_t vbase = vt;
-        const int nvalid = kend - (tbase + 16 * warp);  // value rows of the warp that are keys of the split
-        if constexpr (F8) {
-            // widen the warp's 16 value rows into its f16 scratch tile, rows in MMA-row order; rows past the
-            // split's keys may hold anything (even NaN), which P = 0 would not cancel in the MMA: they become 0
-            const int t = lane >> 1, hf = lane & 1;
-            const int srow = 16 * warp + t;                  // stage row
-            const int lrow = 8 * (t >> 3) + f8_col(t & 7);   // scratch row
-            const bool live = t < nvalid, tail = nvalid < 16;  // (tail: warp-uniform, the last tile only)
-            const uint8_t* vsrc = stages + s * C::STAGE_BYTES + C::MAT_BYTES;
-#pragma unroll
-            for (int i = 0; i < D / 32; ++i) {  // 16 e4m3 values: scratch chunks 2 i, 2 i + 1 of segment hf
-                const int byte = hf * (D / 2) + 16 * i;
-                const int ch = (byte % 128) / 16;
-                uint4 w = *reinterpret_cast<const uint4*>(vsrc + (byte / 128) * C::T_TILE * 128 + srow * 128 +
-                                                          ((ch ^ (srow & 7)) << 4));
-                if (tail && !live) w = make_uint4(0u, 0u, 0u, 0u);
-                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-                uint32_t hv[8];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    hv[2 * q] = e4m3x2_lo_to_f16x2(ws[q]);
-                    hv[2 * q + 1] = e4m3x2_hi_to_f16x2(ws[q]);
-                }
-                const int col = hf * (D / 2) + 16 * i;  // first f16 value of the 16
-                const int sseg = col / 64;
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int sch = (col % 64) / 8 + hh;
-                    *reinterpret_cast<uint4*>(scr + sseg * C::TW * 128 + lrow * 128 + ((sch ^ (lrow & 7)) << 4)) =
-                        make_uint4(hv[4 * hh], hv[4 * hh + 1], hv[4 * hh + 2], hv[4 * hh + 3]);
-                }
-            }
-            __syncwarp();
-            vbase = smem_u32(scr);
-        } else if (nvalid < 16) {
-            // value rows of the warp past the split's keys (the last tile) may hold anything, even NaN, and
-            // P = 0 does not cancel that in the MMA: zero them
-            const int first = nvalid < 0 ? 0 : nvalid;
-            uint8_t* vrow = stages + s * C::STAGE_BYTES + C::MAT_BYTES;
-            for (int idx = lane; idx < (16 - first) * C::NSEG * 8; idx += 32) {
-                const int row = 16 * warp + first + idx / (C::NSEG * 8), rem = idx % (C::NSEG * 8);
-                *reinterpret_cast<uint4*>(vrow + (rem / 8) * C::T_TILE * 128 + row * 128 + (rem % 8) * 16) =
-                    make_uint4(0u, 0u, 0u, 0u);
-            }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // before the ring's next copy
-            __syncwarp();
-        }
-        // ---- O^T += V^T P^T: one MMA per 16 head-dim values ----
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-            uint32_t a[4];
-            ldsm_x4_t(vbase + (mt >> 2) * V_SEG + v_off[mt & 3], a);
-            // ldmatrix order (tokens 0-7 x d lo, tokens 0-7 x d hi, tokens 8-15 x d lo, tokens 8-15 x d hi),
-            // transposed: (d lo, k lo) (d hi, k lo) (d lo, k hi) (d hi, k hi) = a0 a1 a2 a3
-            mma_16816<F8>(o[mt], a, pb[0], pb[1]);
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&bars[C::NSTAGE + s]));
+        mma8_tile<D, F8>(st, stages + s * C::STAGE_BYTES, kbeg + it * C::T_TILE, kend, mask_from, s_mul, k_off,
+                         v_off, tok_g, smem_u32(&bars[C::NSTAGE + s]), warp, lane);
     }
 
-    // the row sums: this lane's share summed over the eight lanes of the row
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        l_run[i] += __shfl_xor_sync(0xffffffffu, l_run[i], 4);
-        l_run[i] += __shfl_xor_sync(0xffffffffu, l_run[i], 8);
-        l_run[i] += __shfl_xor_sync(0xffffffffu, l_run[i], 16);
-    }
     // all consumer warps reach here; a CTA that gave up on a wait writes no results
     if (!consumers_any(aborted || *(volatile int*)&s_abort)) {
         // ---- merge the four warp states in shared memory (reusing the stage ring) ----
         float* om = reinterpret_cast<float*>(stages);  // [4][RB][D]
         float* mm = om + 4 * RB * D;                    // [4][RB]
         float* lm = mm + 4 * RB;                        // [4][RB]
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-            om[(warp * RB + 2 * tq) * D + 16 * mt + g] = o[mt][0];
-            om[(warp * RB + 2 * tq + 1) * D + 16 * mt + g] = o[mt][1];
-            om[(warp * RB + 2 * tq) * D + 16 * mt + g + 8] = o[mt][2];
-            om[(warp * RB + 2 * tq + 1) * D + 16 * mt + g + 8] = o[mt][3];
-        }
-        if (g == 0) {
-            mm[warp * RB + 2 * tq] = m_run[0];
-            mm[warp * RB + 2 * tq + 1] = m_run[1];
-            lm[warp * RB + 2 * tq] = l_run[0];
-            lm[warp * RB + 2 * tq + 1] = l_run[1];
-        }
+        mma8_stash<D, F8>(st, om, mm, lm, warp, lane);
         named_barrier(1, 128);
         gqa_merge_store<__nv_bfloat16, D, RB>(om, mm, lm, p, b, kvh, row0, rows_here, L, kbeg, split,
                                               F8 ? p.v_scale[kvh] : 1.f);
     }
 }
+
 
 // Merge of split partials: with w_i = 2^(lse_i - max lse),
 // O = sum_i w_i O_i / sum_i w_i and lse = max lse + log2(sum_i w_i).
@@ -1421,12 +1490,14 @@ template <int D, bool F8>
 static cudaError_t launch_mma(const CUtensorMap& tk, const CUtensorMap& tv, const GqaParams& p, int nsplit,
                               cudaStream_t st) {
     using C = GqaMmaCfg<D, F8>;
-    auto kern = p.n_rb == 1 && p.ratio * p.s_q <= 8 ? gqa_decode_mma8_kernel<D, F8> : gqa_decode_mma_kernel<D, F8>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    const bool rows8 = p.n_rb == 1 && p.ratio * p.s_q <= 8;
+    auto kern = rows8 ? gqa_decode_mma8_kernel<D, F8> : gqa_decode_mma_kernel<D, F8>;
+    const int smem = rows8 ? GqaMmaCfg<D, F8, true>::SMEM : C::SMEM;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     dim3 grid(nsplit, p.h_kv * p.n_rb, p.B);
     TimedLaunch timer(st);
-    kern<<<grid, 160, C::SMEM, st>>>(tk, tv, p);
+    kern<<<grid, 160, smem, st>>>(tk, tv, p);
     timer.stop();
     e = cudaPeekAtLastError();
     if (e != cudaSuccess) return e;
