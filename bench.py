@@ -211,7 +211,7 @@ class GqaDecode(Workload):
     """gqa_attn over the Llama-3.1-8B-shaped decode batch: split-KV decode kernel (the mma.sync instance for bf16
     caches) + log-sum-exp merge."""
 
-    kernel = "gqa_decode_mma_kernel"
+    kernel = "gqa_decode_mma8_kernel"  # the 8-row tensor-core form (4 query rows per KV head)
     src = ("latent_kv_attention_b200/csrc/gqa_decode.cu", "latent_kv_attention_b200/csrc/common.cuh",
            "latent_kv_attention_b200/csrc/tc.cuh")
 
@@ -306,7 +306,7 @@ class GqaDecodePaged(GqaDecode):
 class GqaDecodeFp8(GqaDecode):
     """gqa_attn_fp8kv over the same decode batch with the K/V cache in e4m3 (one scale per KV head)."""
 
-    kernel = "gqa_decode_mma_kernel"  # the e4m3 tensor-core instance (f16 MMAs)
+    kernel = "gqa_decode_mma8_kernel"  # its e4m3 instance (f16 MMAs)
 
     def setup_costs(self):
         w = self.w
