@@ -641,9 +641,10 @@ __global__ void __launch_bounds__(160, GqaCfg<KV, D, RB>::MINB)
 //     consecutive key bytes per token with one shared-memory load and widens them in registers: in 64-value
 //     group G, lane tq's k-step 4 G + j covers values 64 G + 16 tq + 4 j + {0, 1} (as k = 2 tq, 2 tq + 1) and
 //     + {2, 3} (as k = 2 tq + 8, 2 tq + 9).  The n-th token column of an n-tile is token pi(n) = n / 2 + 4 (n % 2)
-//     of its 8 (so that the two rows a shared-memory phase reads fall in different bank halves); each warp widens
-//     its 16 value rows once per tile into an f16 scratch tile (in that token order, zero past the split's keys),
-//     which the transposing ldmatrix reads as in the bf16 case.  P is f16; the per-KV-head scales are applied to
+//     of its 8 (so that the two rows a shared-memory phase reads fall in different bank halves).  Values go from
+//     the stage to the P*V MMA in registers: each lane reads the 16 value bytes of one head-dim chunk of the four
+//     tokens of its k-pairs, pairs the two tokens of each k-pair byte by byte (prmt) and widens the pair with one
+//     conversion, the output columns following the chunk order.  P is f16; the per-KV-head scales are applied to
 //     the fp32 scores and to the merged output.
 template <int D, bool F8, bool R8 = false>
 struct GqaMmaCfg {
@@ -656,17 +657,15 @@ struct GqaMmaCfg {
     static constexpr int MAT_BYTES = T_TILE * D * E;
     static constexpr int STAGE_BYTES = 2 * MAT_BYTES;
     static constexpr int NSTAGE0 = (LKA_GQA_STAGE_KB * 1024) / STAGE_BYTES;
-    // R8: the 8-row form, which reads e4m3 values straight from the stage (no scratch tile): room for a fourth
-    // stage beside three CTAs per SM
-    static constexpr int NSTAGE_CAP = F8 ? (R8 ? 4 : 3) : 6;
+    // R8: the 8-row form.  Its e4m3 instance runs three CTAs per SM (four stages each); every other instance runs
+    // two (the 16-row e4m3 form does not fit three in registers)
+    static constexpr int NSTAGE_CAP = F8 && R8 ? 4 : 6;
     static constexpr int NSTAGE = NSTAGE0 > NSTAGE_CAP ? NSTAGE_CAP : NSTAGE0;
     static constexpr int RING = NSTAGE * STAGE_BYTES;
-    static constexpr int SCR_W = F8 && !R8 ? TW * D * 2 : 0;  // per-warp f16 value tile (16-row form, e4m3)
-    static constexpr int OFF_BAR = RING + 4 * SCR_W;
+    static constexpr int OFF_BAR = RING;
     static constexpr int MERGE_BYTES = 4 * RB * D * 4 + 2 * 4 * RB * 4;
     static constexpr int SMEM = 1024 + OFF_BAR + 256;
-    // resident CTAs per SM: the e4m3 consumers do more work per byte (the widening), so more of them hide latency
-    static constexpr int MINB = F8 ? 3 : 2;
+    static constexpr int MINB = F8 && R8 ? 3 : 2;
     static_assert(F8 ? D == 128 : (D == 64 || D == 128), "head dim of the tensor-core instances");
     static_assert(MERGE_BYTES <= RING && NSTAGE >= 2 && MINB * (SMEM + 1024) <= 228 * 1024, "shared memory");
 };
@@ -718,9 +717,8 @@ __device__ __forceinline__ uint32_t pack_f16x2_rn(float lo, float hi) {
 __device__ __forceinline__ int f8_tok(int n) { return (n >> 1) + 4 * (n & 1); }
 __device__ __forceinline__ int f8_col(int t) { return 2 * (t & 3) + (t >> 2); }
 
-// (two CTAs per SM whatever the cache type: the 16-row e4m3 form does not fit three in registers)
 template <int D, bool F8>
-__global__ void __launch_bounds__(160, 2)
+__global__ void __launch_bounds__(160, GqaMmaCfg<D, F8>::MINB)
     gqa_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                           const GqaParams p) {
     using C = GqaMmaCfg<D, F8>;
@@ -821,23 +819,25 @@ __global__ void __launch_bounds__(160, 2)
     // token (of the warp's 16) of score element (nt, e) of this lane
     auto tok_of = [&](int nt, int e) { return 8 * nt + (F8 ? f8_tok(2 * tq + (e & 1)) : 2 * tq + (e & 1)); };
 
-    // ldmatrix row addresses (byte offsets, 128-byte swizzle: chunk ^ row % 8).  bf16 keys: matrix l / 8 = (token
-    // half l / 16, 8-value chunk parity (l / 8) % 2) of the warp's 16 tokens: the b0 / b1 fragments of n-tiles 0
-    // and 1 for one k-step.  Values (transposed; the stage for bf16, the warp's scratch tile for e4m3): matrix
-    // l / 8 = (chunk parity l / 16, token half (l / 8) % 2): b0 / b1 of two adjacent 8-column output n-tiles.
+    // ldmatrix row addresses of the bf16 stage (byte offsets, 128-byte swizzle: chunk ^ row % 8).  Keys: matrix
+    // l / 8 = (token half l / 16, 8-value chunk parity (l / 8) % 2) of the warp's 16 tokens: the b0 / b1 fragments
+    // of n-tiles 0 and 1 for one k-step.  Values (transposed): matrix l / 8 = (chunk parity l / 16, token half
+    // (l / 8) % 2): b0 / b1 of two adjacent 8-column output n-tiles.
     const int r8 = lane & 7;
     const uint32_t k_row = (uint32_t)(16 * warp + 8 * (lane >> 4) + r8) * 128;
-    const uint32_t v_row = (uint32_t)((F8 ? 0 : 16 * warp) + 8 * ((lane >> 3) & 1) + r8) * 128;
-    constexpr int V_SEG = F8 ? C::TW * 128 : C::T_TILE * 128;  // bytes per 64-value segment of a value tile
+    const uint32_t v_row = (uint32_t)(16 * warp + 8 * ((lane >> 3) & 1) + r8) * 128;
+    constexpr int V_SEG = C::T_TILE * 128;  // bytes per 64-value segment of a bf16 value tile
     uint32_t k_off[4], v_off[4];
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
         k_off[c] = k_row + ((uint32_t)((2 * c + ((lane >> 3) & 1)) ^ r8) << 4);
         v_off[c] = v_row + ((uint32_t)((2 * c + (lane >> 4)) ^ r8) << 4);
     }
-    // e4m3: this lane's key row of n-tile nt (token column g) and value row to widen (token lane / 2, half lane % 2)
-    uint8_t* scr = smem + C::RING + warp * C::SCR_W;
+    // e4m3: this lane's key row of n-tile nt (token column g), and its head-dim chunk of the values: column n of
+    // output n-tile nt is head-dim value 16 vch(n) + nt, vch putting the chunks of lanes g = 2 i, 2 i + 1 in
+    // different halves of the swizzled row (the 8 lanes of a shared-memory phase read 8 different columns)
     const int kf_row0 = 16 * warp + f8_tok(g);
+    auto vch = [](int n) { return ((n & 1) << 2) | (n >> 1); };
 
     bool aborted = false;
     for (int it = 0; it < n_tiles; ++it) {
@@ -949,61 +949,58 @@ __global__ void __launch_bounds__(160, 2)
                 pa[2 * nt + 1] = F8 ? pack_f16x2_rn(pr[nt][2], pr[nt][3]) : pack_bf16x2(pr[nt][2], pr[nt][3]);
             }
         }
-        uint32_t vbase = vt;
         const int nvalid = kend - (tbase + 16 * warp);  // value rows of the warp that are keys of the split
         if constexpr (F8) {
-            // widen the warp's 16 value rows into its f16 scratch tile, rows in score-column order; rows past the
-            // split's keys may hold anything (even NaN), which P = 0 would not cancel in the MMA: they become 0
-            const int t = lane >> 1, hf = lane & 1;
-            const int srow = 16 * warp + t;                   // stage row
-            const int lrow = 8 * (t >> 3) + f8_col(t & 7);    // scratch row
-            const bool live = t < nvalid, tail = nvalid < 16;  // (tail: warp-uniform, the last tile only)
+            // ---- O += P V straight from the e4m3 stage: lane (g, tq) reads value chunk vch(g) of the warp's
+            // tokens tq, tq + 4, 8 + tq, 12 + tq (k-indices 2 tq, 2 tq + 1, 2 tq + 8, 2 tq + 9 in score-column
+            // order); byte permutes pair the two tokens of each k-pair, one conversion widens a pair into a B
+            // register.  Rows past the split's keys may hold anything (even NaN), which P = 0 would not cancel in
+            // the MMA: they become 0 ----
             const uint8_t* vsrc = stages + s * C::STAGE_BYTES + C::MAT_BYTES;
+            const int ch = vch(g);
+            uint32_t vw[4][4];
 #pragma unroll
-            for (int i = 0; i < D / 32; ++i) {  // 16 e4m3 values: scratch chunks 2 i, 2 i + 1 of segment hf
-                const int byte = hf * (D / 2) + 16 * i;
-                const int ch = (byte % 128) / 16;
-                uint4 w = *reinterpret_cast<const uint4*>(vsrc + (byte / 128) * C::T_TILE * 128 + srow * 128 +
-                                                          ((ch ^ (srow & 7)) << 4));
-                if (tail && !live) w = make_uint4(0u, 0u, 0u, 0u);
-                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-                uint32_t hv[8];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    hv[2 * q] = e4m3x2_lo_to_f16x2(ws[q]);
-                    hv[2 * q + 1] = e4m3x2_hi_to_f16x2(ws[q]);
-                }
-                const int col = hf * (D / 2) + 16 * i;  // first f16 value of the 16
-                const int sseg = col / 64;
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int sch = (col % 64) / 8 + hh;
-                    *reinterpret_cast<uint4*>(scr + sseg * C::TW * 128 + lrow * 128 + ((sch ^ (lrow & 7)) << 4)) =
-                        make_uint4(hv[4 * hh], hv[4 * hh + 1], hv[4 * hh + 2], hv[4 * hh + 3]);
-                }
+            for (int j = 0; j < 4; ++j) {
+                const int t = tq + 4 * j;  // token of the warp's 16
+                const int row = 16 * warp + t;
+                uint4 w = *reinterpret_cast<const uint4*>(vsrc + row * 128 + ((ch ^ (row & 7)) << 4));
+                if (t >= nvalid) w = make_uint4(0u, 0u, 0u, 0u);
+                vw[j][0] = w.x;
+                vw[j][1] = w.y;
+                vw[j][2] = w.z;
+                vw[j][3] = w.w;
             }
-            __syncwarp();
-            vbase = smem_u32(scr);
-        } else if (nvalid < 16) {
-            // value rows of the warp past the split's keys (the last tile) may hold anything, even NaN, and
-            // P = 0 does not cancel that in the MMA: zero them
-            const int first = nvalid < 0 ? 0 : nvalid;
-            uint8_t* vrow = stages + s * C::STAGE_BYTES + C::MAT_BYTES;
-            for (int idx = lane; idx < (16 - first) * C::NSEG * 8; idx += 32) {
-                const int row = 16 * warp + first + idx / (C::NSEG * 8), rem = idx % (C::NSEG * 8);
-                *reinterpret_cast<uint4*>(vrow + (rem / 8) * C::T_TILE * 128 + row * 128 + (rem % 8) * 16) =
-                    make_uint4(0u, 0u, 0u, 0u);
-            }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // before the ring's next copy
-            __syncwarp();
-        }
-        // ---- O += P V ----
 #pragma unroll
-        for (int cc = 0; cc < NT / 2; ++cc) {
-            uint32_t vb[4];
-            ldsm_x4_t(vbase + (cc >> 2) * V_SEG + v_off[cc & 3], vb);
-            mma_16816<F8>(o[2 * cc], pa, vb[0], vb[1]);
-            mma_16816<F8>(o[2 * cc + 1], pa, vb[2], vb[3]);
+            for (int q = 0; q < 4; ++q) {  // value bytes 4 q .. 4 q + 3 of the chunk: n-tiles 4 q .. 4 q + 3
+                const uint32_t lo01 = __byte_perm(vw[0][q], vw[1][q], 0x5140), hi01 = __byte_perm(vw[0][q], vw[1][q], 0x7362);
+                const uint32_t lo23 = __byte_perm(vw[2][q], vw[3][q], 0x5140), hi23 = __byte_perm(vw[2][q], vw[3][q], 0x7362);
+                mma_16816<true>(o[4 * q], pa, e4m3x2_lo_to_f16x2(lo01), e4m3x2_lo_to_f16x2(lo23));
+                mma_16816<true>(o[4 * q + 1], pa, e4m3x2_hi_to_f16x2(lo01), e4m3x2_hi_to_f16x2(lo23));
+                mma_16816<true>(o[4 * q + 2], pa, e4m3x2_lo_to_f16x2(hi01), e4m3x2_lo_to_f16x2(hi23));
+                mma_16816<true>(o[4 * q + 3], pa, e4m3x2_hi_to_f16x2(hi01), e4m3x2_hi_to_f16x2(hi23));
+            }
+        } else {
+            if (nvalid < 16) {
+                // value rows of the warp past the split's keys (the last tile) may hold anything, even NaN, and
+                // P = 0 does not cancel that in the MMA: zero them
+                const int first = nvalid < 0 ? 0 : nvalid;
+                uint8_t* vrow = stages + s * C::STAGE_BYTES + C::MAT_BYTES;
+                for (int idx = lane; idx < (16 - first) * C::NSEG * 8; idx += 32) {
+                    const int row = 16 * warp + first + idx / (C::NSEG * 8), rem = idx % (C::NSEG * 8);
+                    *reinterpret_cast<uint4*>(vrow + (rem / 8) * C::T_TILE * 128 + row * 128 + (rem % 8) * 16) =
+                        make_uint4(0u, 0u, 0u, 0u);
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // before the ring's next copy
+                __syncwarp();
+            }
+            // ---- O += P V ----
+#pragma unroll
+            for (int cc = 0; cc < NT / 2; ++cc) {
+                uint32_t vb[4];
+                ldsm_x4_t(vt + (cc >> 2) * V_SEG + v_off[cc & 3], vb);
+                mma_16816<false>(o[2 * cc], pa, vb[0], vb[1]);
+                mma_16816<false>(o[2 * cc + 1], pa, vb[2], vb[3]);
+            }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&bars[C::NSTAGE + s]));
@@ -1023,9 +1020,17 @@ __global__ void __launch_bounds__(160, 2)
         float* lm = mm + 4 * RB;                        // [4][RB]
 #pragma unroll
         for (int j = 0; j < NT; ++j) {
-            *reinterpret_cast<float2*>(&om[(warp * RB + g) * D + 8 * j + 2 * tq]) = make_float2(o[j][0], o[j][1]);
-            *reinterpret_cast<float2*>(&om[(warp * RB + g + 8) * D + 8 * j + 2 * tq]) =
-                make_float2(o[j][2], o[j][3]);
+            float* r0 = om + (warp * RB + g) * D;  // row g (r0 + D: row g + 8)
+            if constexpr (F8) {  // columns 2 tq, 2 tq + 1 of n-tile j: head-dim values 16 vch(n) + j
+                const int d0 = 16 * vch(2 * tq) + j, d1 = 16 * vch(2 * tq + 1) + j;
+                r0[d0] = o[j][0];
+                r0[d1] = o[j][1];
+                r0[8 * D + d0] = o[j][2];
+                r0[8 * D + d1] = o[j][3];
+            } else {
+                *reinterpret_cast<float2*>(r0 + 8 * j + 2 * tq) = make_float2(o[j][0], o[j][1]);
+                *reinterpret_cast<float2*>(r0 + 8 * D + 8 * j + 2 * tq) = make_float2(o[j][2], o[j][3]);
+            }
         }
         if (tq == 0) {
             mm[warp * RB + g] = m_run[0];
@@ -1559,8 +1564,9 @@ cudaError_t gqa_decode_launch(const CUtensorMap& tk, const CUtensorMap& tv, cons
 
 int gqa_fp8_tile_tokens(int d, int rb, int* ctas_per_sm) {
     if (d == 128 && rb == 16) {  // the tensor-core instance
-        if (ctas_per_sm) *ctas_per_sm = GqaMmaCfg<128, true>::MINB;
-        return GqaMmaCfg<128, true>::T_TILE;
+        // (the plan assumes the 8-row form of the usual GQA groups: three CTAs per SM)
+        if (ctas_per_sm) *ctas_per_sm = GqaMmaCfg<128, true, true>::MINB;
+        return GqaMmaCfg<128, true, true>::T_TILE;
     }
 #define LKA_TILE_CASE(DD, R)                                       \
     if (d == DD && rb == R) {                                      \

@@ -56,11 +56,11 @@ def test_fp8kv_matches_bf16_path_on_the_dequantised_cache():
 
 
 @pytest.mark.parametrize("split_tokens", [64, 192, 0], ids=["one_tile_items", "uneven_items", "auto"])
-@pytest.mark.parametrize("s_q,causal", [(1, True), (2, True), (1, False)])
+@pytest.mark.parametrize("s_q,causal", [(1, True), (2, True), (1, False), (3, False), (4, True)])
 def test_fp8kv_split_sizes_are_repeatable(split_tokens, s_q, causal):
-    """The 8-row e4m3 kernel (at most 8 query rows per KV head) under forced split sizes: one-tile splits, splits
-    that end mid-tile, empty last splits of short sequences; three calls in a row give the same bytes, and the
-    first matches the oracle."""
+    """The e4m3 tensor-core kernels under forced split sizes (s_q <= 2: the 8-row form, 4 or 8 rows per KV head;
+    s_q 3, 4: the 16-row form, 12 or 16 rows): one-tile splits, splits that end mid-tile, empty last splits of
+    short sequences; three calls in a row give the same bytes, and the first matches the oracle."""
     inp = synthetic.gqa_fp8_inputs(811 + s_q + split_tokens, 6, 32, 8, 128, s_q, s_q, 3000, Lmax=3072)
     dd = {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
     prev = lka.set_split_tokens(split_tokens)
