@@ -1047,10 +1047,11 @@ __global__ void __launch_bounds__(160, GqaMmaCfg<D, F8>::MINB)
 // The swapped form for blocks of at most 8 query rows (the common GQA groups of 4 or 8 heads at s_q = 1): the
 // warp's 16 tokens are the M = 16 rows of the MMAs and the query rows the N = 8 columns, so that a 16-token tile
 // costs d/16 score MMAs (S^T = K Q^T, K read by ldmatrix as the A operand, Q^T held in registers) and d/16 P*V
-// MMAs (O^T = V^T P^T, V^T read by the transposing ldmatrix as the A operand) instead of twice that with 8 of 16
-// rows empty.  The score accumulator holds P^T (tokens x rows); movmatrix transposes its two 8 x 8 halves into the
-// B operand of the P*V MMA.  Everything else (softmax, scales, the e4m3 handling with its permuted head-dim order
-// and token order, the merge) is as in the 16-row form above.
+// MMAs (O^T = V^T P^T, V^T the A operand: read by the transposing ldmatrix from a bf16 stage, paired and widened
+// in registers from an e4m3 one) instead of twice that with 8 of 16 rows empty.  The score accumulator holds P^T
+// (tokens x rows); movmatrix transposes its two 8 x 8 halves into the B operand of the P*V MMA.  Everything else
+// (softmax, scales, the e4m3 key handling with its permuted head-dim order and token order, the merge) is as in
+// the 16-row form above.
 //
 // Per-warp state of the 8-row form over one work item: the query slice as B fragments of the score MMA, the
 // last visible key of the lane's two query rows, the O^T accumulators and the lazily moved maxima with this
@@ -1059,7 +1060,8 @@ template <int D>
 struct Mma8Warp {
     uint32_t qb[D / 16][2];  // query row g: bf16 pairs as given, or f16 pairs in the permuted e4m3 order
     int last[2];             // last visible key of query rows 2 tq, 2 tq + 1 (-1: a padding row, nothing visible)
-    float o[D / 16][4];      // O^T: head-dim values 16 mt + g (+ 8), query rows 2 tq, 2 tq + 1
+    float o[D / 16][4];      // O^T rows g, g + 8 of m-tile mt (head-dim values 16 mt + g, + 8 for bf16; 16 vch(g)
+                             // + 2 mt, + 1 for e4m3), query rows 2 tq, 2 tq + 1
     float m_run[2], l_run[2];
 };
 
