@@ -42,6 +42,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -77,11 +78,18 @@ def peaks():
                 source="fallback")
 
 
+def _code_only(text: str) -> str:
+    """C/C++/CUDA source without its comments and blank lines (a comment edit leaves the kernel as it was)."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = (re.sub(r"//.*", "", ln).rstrip() for ln in text.splitlines())
+    return "\n".join(ln for ln in lines if ln)
+
+
 def source_hash(*rel_paths):
     h = hashlib.sha256()
     for r in rel_paths:
-        with open(os.path.join(ROOT, r), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, r), encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 
